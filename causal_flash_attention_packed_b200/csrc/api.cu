@@ -1,0 +1,304 @@
+// C-ABI entry points of fapk (declared in include/fapk.h): argument
+// validation on the host, workspace layout, TMA descriptor creation and the
+// kernel launches.  No entry point allocates device memory or synchronises,
+// except fapk_status.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fapk {
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+// --- driver entry point for tensor-map encoding (no libcuda link needed) ---
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// --- per-device cached attributes ---
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+int g_num_sms[kMaxDevices] = {0};
+
+int device_num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_num_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// --- problem validation ---
+int validate_problem(const fapk_problem_t* P) {
+  if (!P) return FAPK_ERR_INVALID_ARG;
+  if (P->T < 0 || P->n_docs < 0 || P->Hq <= 0 || P->Hkv <= 0) return FAPK_ERR_INVALID_ARG;
+  if (P->d != 64 && P->d != 128) return FAPK_ERR_UNSUPPORTED;
+  if (P->Hq % P->Hkv != 0) return FAPK_ERR_UNSUPPORTED;
+  if (P->prec != FAPK_BF16 && P->prec != FAPK_MXFP8) return FAPK_ERR_UNSUPPORTED;
+  if (P->scale_rule != FAPK_SCALE_RCEIL && P->scale_rule != FAPK_SCALE_OCP) return FAPK_ERR_UNSUPPORTED;
+  if (P->grad_dtype != FAPK_GRAD_F32 && P->grad_dtype != FAPK_GRAD_BF16) return FAPK_ERR_UNSUPPORTED;
+  if (!std::isfinite(P->scale)) return FAPK_ERR_INVALID_ARG;
+  if (P->T > 0) {
+    if (P->n_docs < 1 || P->max_seqlen < 1 || !P->cu_seqlens_dev) return FAPK_ERR_INVALID_ARG;
+    // 64-bit element offsets are used everywhere; keep token and head counts
+    // inside what the TMA coordinates (int32) and grid dimensions allow
+    if ((long long)P->T * P->Hq * P->d > (1LL << 40)) return FAPK_ERR_UNSUPPORTED;
+  }
+  if (P->cu_seqlens_host) {
+    const int32_t* cu = P->cu_seqlens_host;
+    if (cu[0] != 0 || cu[P->n_docs] != P->T) return FAPK_ERR_BAD_SEQLENS;
+    for (int k = 0; k < P->n_docs; ++k) {
+      const int L = cu[k + 1] - cu[k];
+      if (L < 0 || L > P->max_seqlen) return FAPK_ERR_BAD_SEQLENS;
+    }
+  }
+  return FAPK_OK;
+}
+
+uint64_t timeout_ns_of(const fapk_problem_t* P) {
+  const int ms = P->timeout_ms > 0 ? P->timeout_ms : 2000;
+  return (uint64_t)ms * 1000000ull;
+}
+
+// --- workspace layout ---
+struct SchedLayout {
+  size_t level_off, n_items, list, end;
+  int max_levels, max_items;
+};
+
+SchedLayout sched_layout(size_t base, int T, int n_docs, int max_seqlen, int rows) {
+  SchedLayout s;
+  s.max_levels = (max_seqlen + rows - 1) / rows;
+  s.max_items = T / rows + n_docs + 1;
+  s.level_off = align_up(base);
+  s.n_items = align_up(s.level_off + sizeof(int) * (size_t)(s.max_levels + 2));
+  s.list = align_up(s.n_items + sizeof(int));
+  s.end = align_up(s.list + sizeof(int2) * (size_t)s.max_items);
+  return s;
+}
+
+SchedBuf sched_buf(void* ws, const SchedLayout& s) {
+  char* w = static_cast<char*>(ws);
+  SchedBuf b;
+  b.level_off = reinterpret_cast<int*>(w + s.level_off);
+  b.n_items = reinterpret_cast<int*>(w + s.n_items);
+  b.list = reinterpret_cast<int2*>(w + s.list);
+  b.max_levels = s.max_levels;
+  b.max_items = s.max_items;
+  return b;
+}
+
+constexpr int kFwdRows = 256;  // query rows per forward work item (two 128-row tiles)
+constexpr int kBwdRows = 128;  // rows per backward work item
+
+struct FwdLayout {
+  SchedLayout sched;
+  size_t total;
+};
+FwdLayout fwd_layout(const fapk_problem_t* P) {
+  FwdLayout L;
+  L.sched = sched_layout(kAlign, P->T, P->n_docs, P->max_seqlen, kFwdRows);
+  L.total = L.sched.end;
+  return L;
+}
+
+struct BwdLayout {
+  SchedLayout kv, q;
+  size_t delta, total;
+};
+BwdLayout bwd_layout(const fapk_problem_t* P) {
+  BwdLayout L;
+  L.kv = sched_layout(kAlign, P->T, P->n_docs, P->max_seqlen, kBwdRows);
+  L.q = sched_layout(L.kv.end, P->T, P->n_docs, P->max_seqlen, kBwdRows);
+  L.delta = L.q.end;
+  L.total = align_up(L.delta + sizeof(float) * (size_t)P->Hq * (size_t)P->T);
+  return L;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? FAPK_OK : FAPK_ERR_CUDA; }
+
+}  // namespace
+
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace fapk
+
+using namespace fapk;
+
+extern "C" {
+
+size_t fapk_workspace_size(const fapk_problem_t* prob, int which) {
+  if (validate_problem(prob) != FAPK_OK) return 0;
+  if (which == FAPK_FWD) return fwd_layout(prob).total;
+  if (which == FAPK_BWD) return bwd_layout(prob).total;
+  return 0;
+}
+
+size_t fapk_ctx_size(const fapk_problem_t* prob) {
+  if (validate_problem(prob) != FAPK_OK) return 0;
+  return 0;
+}
+
+int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const void* v, void* o,
+                  float* lse, void* ctx, void* ws, size_t ws_bytes, void* stream) {
+  (void)ctx;
+  int rc = validate_problem(P);
+  if (rc != FAPK_OK) return rc;
+  if (P->T == 0) return FAPK_OK;
+  if (!q || !k || !v || !o || !lse || !ws) return FAPK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+    return FAPK_ERR_INVALID_ARG;
+  const FwdLayout L = fwd_layout(P);
+  if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
+  if (P->prec != FAPK_BF16) return FAPK_ERR_UNSUPPORTED;
+  const int sms = device_num_sms();
+  if (sms <= 0) return FAPK_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* status = static_cast<DeviceStatus*>(ws);
+  FwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+  a.cu = P->cu_seqlens_dev;
+  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.d = P->d;
+  a.scale = P->scale;
+  a.sched = sched_buf(ws, L.sched);
+  a.status = status;
+  a.timeout_ns = timeout_ns_of(P);
+  a.flags = P->flags;
+  a.num_sms = sms;
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRows, kSchedQ, a.sched, status, true, st));
+  if (rc != FAPK_OK) return rc;
+  return cuda_status(launch_fwd_bf16(a, st));
+}
+
+int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const void* v, const void* o,
+                  const float* lse, const void* dout, const void* ctx, void* dq, void* dk, void* dv,
+                  void* ws, size_t ws_bytes, void* stream) {
+  (void)ctx;
+  int rc = validate_problem(P);
+  if (rc != FAPK_OK) return rc;
+  if (P->T == 0) return FAPK_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !ws) return FAPK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+    return FAPK_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(P);
+  if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
+  if (P->prec != FAPK_BF16) return FAPK_ERR_UNSUPPORTED;
+  const int sms = device_num_sms();
+  if (sms <= 0) return FAPK_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* status = static_cast<DeviceStatus*>(ws);
+  BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.delta = reinterpret_cast<float*>(static_cast<char*>(ws) + L.delta);
+  a.cu = P->cu_seqlens_dev;
+  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.d = P->d;
+  a.scale = P->scale;
+  a.grad_bf16 = P->grad_dtype == FAPK_GRAD_BF16;
+  a.sched_kv = sched_buf(ws, L.kv);
+  a.sched_q = sched_buf(ws, L.q);
+  a.status = status;
+  a.timeout_ns = timeout_ns_of(P);
+  a.flags = P->flags;
+  a.num_sms = sms;
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedKV, a.sched_kv, status, true, st));
+  if (rc != FAPK_OK) return rc;
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedQ, a.sched_q, status, false, st));
+  if (rc != FAPK_OK) return rc;
+  return cuda_status(launch_bwd_bf16(a, st));
+}
+
+int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const int32_t* cu_seqlens_dev,
+                        const int32_t* cu_seqlens_host, int n_docs, int forms, int scale_rule,
+                        uint8_t* val_tb, uint8_t* scale_tb, uint8_t* val_pt, uint8_t* scale_pt,
+                        void* stream) {
+  if (T < 0 || H <= 0 || n_docs < 0) return FAPK_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FAPK_ERR_UNSUPPORTED;
+  if (scale_rule != FAPK_SCALE_RCEIL && scale_rule != FAPK_SCALE_OCP) return FAPK_ERR_UNSUPPORTED;
+  if ((forms & ~(FAPK_FORM_TB | FAPK_FORM_PT)) != 0 || forms == 0) return FAPK_ERR_INVALID_ARG;
+  if (T == 0) return FAPK_OK;
+  if (H > 65535 || (long long)T / 32 + n_docs > 0x7FFFFFFFLL) return FAPK_ERR_UNSUPPORTED;
+  if (!x_bf16 || !cu_seqlens_dev || n_docs < 1 || !aligned16(x_bf16)) return FAPK_ERR_INVALID_ARG;
+  if ((forms & FAPK_FORM_TB) && (!val_tb || !scale_tb)) return FAPK_ERR_INVALID_ARG;
+  if ((forms & FAPK_FORM_PT) && (!val_pt || !scale_pt)) return FAPK_ERR_INVALID_ARG;
+  if ((val_tb && !aligned16(val_tb)) || (val_pt && !aligned16(val_pt))) return FAPK_ERR_INVALID_ARG;
+  if (cu_seqlens_host) {
+    if (cu_seqlens_host[0] != 0 || cu_seqlens_host[n_docs] != T) return FAPK_ERR_BAD_SEQLENS;
+    for (int k = 0; k < n_docs; ++k)
+      if (cu_seqlens_host[k + 1] < cu_seqlens_host[k]) return FAPK_ERR_BAD_SEQLENS;
+  }
+  return cuda_status(launch_quantize_mxfp8(x_bf16, T, H, d, cu_seqlens_dev, n_docs, forms, scale_rule, val_tb,
+                                           scale_tb, val_pt, scale_pt, static_cast<cudaStream_t>(stream)));
+}
+
+int fapk_status(const void* ws, void* stream) {
+  if (!ws) return FAPK_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FAPK_ERR_CUDA;
+  DeviceStatus s;
+  if (cudaMemcpy(&s, ws, sizeof(s), cudaMemcpyDeviceToHost) != cudaSuccess) return FAPK_ERR_CUDA;
+  return s.code;
+}
+
+const char* fapk_strerror(int status) {
+  switch (status) {
+    case FAPK_OK: return "ok";
+    case FAPK_ERR_INVALID_ARG: return "invalid argument";
+    case FAPK_ERR_UNSUPPORTED: return "unsupported problem (head dim, head grouping or mode)";
+    case FAPK_ERR_BAD_SEQLENS: return "malformed cu_seqlens or a document longer than max_seqlen";
+    case FAPK_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case FAPK_ERR_CUDA: return "CUDA runtime error";
+    case FAPK_ERR_DEVICE_TIMEOUT: return "device watchdog timeout in a pipeline wait";
+    default: return "unknown status";
+  }
+}
+
+uint64_t fapk_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int fapk_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// Internal interfaces between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "fapk.h"
+
+namespace fapk {
+
+struct DeviceStatus;
+
+// Work-list modes of the scheduler (schedule.cu).  An item is (doc, tile)
+// with tile in [0, ceil(L / rows)); items are ordered by a cost level,
+// highest first, so that persistent CTAs take the longest work first (LPT).
+//  kSchedQ:  level = tile               (a later query tile sees more keys)
+//  kSchedKV: level = ntiles - 1 - tile  (an earlier key tile is seen by more
+//                                        queries)
+enum SchedMode : int { kSchedQ = 0, kSchedKV = 1 };
+
+// Scratch of one work list inside the workspace.
+struct SchedBuf {
+  int* level_off;  // [max_levels + 2]
+  int2* list;      // [max_items]
+  int* n_items;    // 1 int
+  int max_levels;
+  int max_items;
+};
+
+cudaError_t launch_schedule(const int32_t* cu, int n_docs, int rows, int mode, const SchedBuf& sb,
+                            DeviceStatus* status, bool clear_status, cudaStream_t stream);
+
+cudaError_t launch_quantize_mxfp8(const void* x, int T, int H, int d, const int32_t* cu, int n_docs,
+                                  int forms, int rule, uint8_t* vtb, uint8_t* stb, uint8_t* vpt,
+                                  uint8_t* spt, cudaStream_t stream);
+
+// Forward, bf16 operands (fwd_bf16.cu).
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  const int32_t* cu;
+  int T, Hq, Hkv, d;
+  float scale;
+  SchedBuf sched;
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+  int flags;
+  int num_sms;
+};
+cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t stream);
+
+// Backward, bf16 operands (bwd_bf16.cu).
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const float* lse;
+  const void* dout;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* delta;  // [Hq][T] fp32 scratch: D_i = dO_i . O_i
+  const int32_t* cu;
+  int T, Hq, Hkv, d;
+  float scale;
+  int grad_bf16;
+  SchedBuf sched_kv;
+  SchedBuf sched_q;
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+  int flags;
+  int num_sms;
+};
+cudaError_t launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream);
+
+// Tensor map of a bf16 [T][H][d] tensor as a 3-D (d, H, T) view with a box of
+// 64 channels x 1 head x 128 tokens and 128-byte swizzle (api.cu).
+bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d);
+
+// Count of kernels launched by this library (api.cu).
+void note_launches(int n);
+
+}  // namespace fapk

@@ -1,0 +1,187 @@
+/*
+ * fapk.h -- C ABI of the causal packed-document flash-attention library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  Exact causal self-attention over packed variable-length
+ * documents, forward and backward:
+ *   S = scale * Q K^T                 ("GPT Kernel Programlama: MatMul, Softmax
+ *                                       ve Attention Hesabi", sec. 3)
+ *   key j is visible to query i iff j <= i and both lie in the same document
+ *                                      (same page, sec. 4; FLAMIA page, sec.
+ *                                       "FLAMIA Mimarisi ve Temel Tasarim
+ *                                       Ilkeleri": packed layouts, no repacking)
+ *   P = softmax over the visible keys (same page, sec. 5), O = P V (sec. 6),
+ * computed tile by tile with an online softmax so that S and P never reach
+ * global memory ("FlashAttention (HU)", secs. "Tiling es blokkos
+ * feldolgozas", "Online Softmax-szamitas", "Muveletek osszevonasa egyetlen
+ * CUDA-kernelbe").  LSE_i = ln sum_j exp(S_ij) (natural log, scale included).
+ * The backward is the analytic derivative: D_i = dO_i . O_i, dP = dO V^T,
+ * dS = P * (dP - D), dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
+ *
+ * Two precisions.  FAPK_BF16: bf16 operands, fp32 accumulation.  FAPK_MXFP8:
+ * the FLAMIA page's MXFP8 path -- E4M3 values with one E8M0 scale per 32
+ * elements along the contraction, token-block scales reused across the
+ * forward and backward orientations, document-local scale blocks, and a leak
+ * guard that quantises per token any token block that crosses the causal
+ * diagonal (FLAMIA page, same section).
+ *
+ * Layouts (all row-major, contiguous, device memory, 16-byte aligned):
+ *   q, o, dout, dq : [T][Hq][d]      k, v, dk, dv : [T][Hkv][d]
+ *   lse            : fp32 [Hq][T]    cu_seqlens   : int32 [n_docs + 1]
+ * with cu[0] = 0, cu non-decreasing, cu[n_docs] = T; document k holds tokens
+ * [cu[k], cu[k+1]); zero-length documents are allowed and produce nothing.
+ * Query head h reads KV head h / (Hq / Hkv).  d must be 64 or 128.
+ *
+ * Ownership and threading.  The caller owns every buffer (inputs, outputs,
+ * workspace, ctx).  The library allocates no device memory and keeps no
+ * global state apart from cached kernel attributes; calls on different
+ * streams with different workspaces may run concurrently.
+ *
+ * Execution and errors.  Every call is asynchronous on the given stream
+ * (a cudaStream_t passed as void*, NULL for the legacy default stream) and
+ * none synchronises, except fapk_status.  A return of FAPK_OK means the work
+ * was launched.  Argument errors are detected on the host before anything is
+ * launched and returned as codes; nothing is thrown across the ABI and nothing
+ * calls exit().  Errors found on the device (a watchdog timeout of a pipeline
+ * wait, a document longer than max_seqlen) are written into a status word
+ * inside the workspace and read back with fapk_status after the stream's work
+ * is done.
+ */
+#ifndef FAPK_H_
+#define FAPK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FAPK_API __attribute__((visibility("default")))
+#else
+#define FAPK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+  FAPK_OK = 0,
+  FAPK_ERR_INVALID_ARG = 1,         /* null pointer, bad size, misaligned buffer */
+  FAPK_ERR_UNSUPPORTED = 2,         /* d not in {64,128}, Hq % Hkv != 0, unknown mode */
+  FAPK_ERR_BAD_SEQLENS = 3,         /* cu_seqlens not 0..T non-decreasing, or a document
+                                       longer than max_seqlen */
+  FAPK_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below fapk_workspace_size() */
+  FAPK_ERR_CUDA = 5,                /* a CUDA runtime call failed (launch, no device) */
+  FAPK_ERR_DEVICE_TIMEOUT = 6       /* a bounded device-side wait gave up */
+} fapk_status_t;
+
+/* Operand precision of the attention path. */
+typedef enum { FAPK_BF16 = 0, FAPK_MXFP8 = 1 } fapk_prec_t;
+
+/* Element type of dq, dk, dv. */
+typedef enum { FAPK_GRAD_F32 = 0, FAPK_GRAD_BF16 = 1 } fapk_grad_dtype_t;
+
+/* E8M0 scale-exponent rule of the MXFP8 quantiser.
+ *  FAPK_SCALE_RCEIL (default): X = ceil(log2(amax / 448)), the smallest
+ *    exponent at which the block maximum fits E4M3 without saturating.
+ *  FAPK_SCALE_OCP: X = floor(log2(amax)) - 8 (OCP Microscaling v1.0);
+ *    block maxima whose mantissa exceeds 1.75 saturate to 448.
+ * Both clamp X to [-127, 127]; an all-zero block takes X = -127.  The scale
+ * byte is X + 127. */
+typedef enum { FAPK_SCALE_RCEIL = 0, FAPK_SCALE_OCP = 1 } fapk_scale_rule_t;
+
+/* Which pass a workspace is sized for. */
+enum { FAPK_FWD = 0, FAPK_BWD = 1 };
+
+/* Forms produced by fapk_quantize_mxfp8 (bit mask). */
+enum { FAPK_FORM_TB = 1, FAPK_FORM_PT = 2 };
+
+/* Debug flags (fapk_problem_t.flags). */
+enum {
+  /* Fault injection for the watchdog test: the forward's load producer drops
+   * one K/V tile copy, so the consumer's bounded wait runs out and the call
+   * reports FAPK_ERR_DEVICE_TIMEOUT through fapk_status.  No fault, trap or
+   * hang is involved. */
+  FAPK_FLAG_INJECT_DROP_LOAD = 1 << 0
+};
+
+/* One attention problem.  All fields are read during the call only. */
+typedef struct {
+  int T;                         /* total packed tokens (>= 0) */
+  int n_docs;                    /* number of documents (>= 1 when T > 0) */
+  int max_seqlen;                /* upper bound of any document length (>= 1 when T > 0) */
+  int Hq, Hkv, d;                /* query heads, KV heads (Hq % Hkv == 0), head dim (64|128) */
+  float scale;                   /* softmax scale, usually 1/sqrt(d) */
+  int prec;                      /* fapk_prec_t */
+  int scale_rule;                /* fapk_scale_rule_t (MXFP8 path) */
+  const int32_t* cu_seqlens_dev; /* device copy of cu_seqlens (required) */
+  const int32_t* cu_seqlens_host;/* host copy; when non-NULL it is validated on the host */
+  int grad_dtype;                /* fapk_grad_dtype_t of dq, dk, dv */
+  int flags;                     /* debug flags, 0 in normal use */
+  int timeout_ms;                /* device watchdog per wait; <= 0 selects 2000 ms */
+} fapk_problem_t;
+
+/* Bytes of workspace the forward (which = FAPK_FWD) or backward
+ * (which = FAPK_BWD) needs for this problem; 0 if the problem is invalid.
+ * The workspace is scratch owned by the caller: device memory, 256-byte
+ * aligned, contents need not be initialised, not shared by concurrent calls. */
+FAPK_API size_t fapk_workspace_size(const fapk_problem_t* prob, int which);
+
+/* Bytes of the saved-operand buffer that the MXFP8 forward fills and the
+ * MXFP8 backward reads (the quantised token-block operands reused across
+ * orientations, FLAMIA page: "token-block scaling").  0 for FAPK_BF16. */
+FAPK_API size_t fapk_ctx_size(const fapk_problem_t* prob);
+
+/* Forward.  Reads q, k, v (bf16); writes o (bf16) and lse (fp32, natural
+ * log).  ctx: device buffer of fapk_ctx_size() bytes (MXFP8) or NULL (BF16).
+ * ws: workspace of at least fapk_workspace_size(prob, FAPK_FWD) bytes. */
+FAPK_API int fapk_attn_fwd(const fapk_problem_t* prob, const void* q, const void* k, const void* v,
+                  void* o, float* lse, void* ctx, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward.  Reads q, k, v, o, lse, dout (bf16 except lse) and, for MXFP8,
+ * the ctx written by the matching forward; writes dq [T][Hq][d] and
+ * dk, dv [T][Hkv][d] in grad_dtype.  dk and dv are summed over the query
+ * heads that share a KV head.  ws: at least fapk_workspace_size(prob,
+ * FAPK_BWD) bytes. */
+FAPK_API int fapk_attn_bwd(const fapk_problem_t* prob, const void* q, const void* k, const void* v,
+                  const void* o, const float* lse, const void* dout, const void* ctx,
+                  void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, void* stream);
+
+/* MXFP8 quantisation of a bf16 tensor x [T][H][d] (FLAMIA page: MXFP8,
+ * token-block scaling, document-local scaling).  E4M3 codes (round to nearest
+ * even, saturating to +-448, a zero result is always code 0x00) and E8M0
+ * scale bytes.
+ *   forms & FAPK_FORM_TB: token-block form.  One scale per 32 tokens x 32
+ *     channels of one head; token blocks are document-local: block m of
+ *     document k covers tokens [s_k + 32m, min(s_k + 32m + 32, e_k)).
+ *     val_tb [T][H][d] codes; scale_tb [T/32 + n_docs][H][d/32] scale bytes,
+ *     block m of document k in slot floor(s_k/32) + k + m (slots holding no
+ *     block are not written).
+ *   forms & FAPK_FORM_PT: per-token form.  One scale per token x 32 channels.
+ *     val_pt [T][H][d]; scale_pt [T][H][d/32].
+ * Pointers of a form not requested may be NULL.  x must be 16-byte aligned;
+ * d is 64 or 128. */
+FAPK_API int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const int32_t* cu_seqlens_dev,
+                        const int32_t* cu_seqlens_host, int n_docs, int forms, int scale_rule,
+                        uint8_t* val_tb, uint8_t* scale_tb, uint8_t* val_pt, uint8_t* scale_pt,
+                        void* stream);
+
+/* Synchronises `stream`, then returns the device status word of the last call
+ * that used workspace `ws` (FAPK_OK, FAPK_ERR_DEVICE_TIMEOUT, or
+ * FAPK_ERR_BAD_SEQLENS), or FAPK_ERR_CUDA if the stream reported an error. */
+FAPK_API int fapk_status(const void* ws, void* stream);
+
+/* Static text for a status code. */
+FAPK_API const char* fapk_strerror(int status);
+
+/* Number of kernels this library has launched in this process (all threads). */
+FAPK_API uint64_t fapk_launch_count(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+FAPK_API int fapk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FAPK_H_ */

@@ -1,0 +1,113 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+declared in include/fapk.h, and rejects bad arguments on the host before
+anything is launched."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from causal_flash_attention_packed_b200 import build, fapk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return fapk.lib()
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "fapk.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fapk_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    syms = _declared_symbols()
+    assert {"fapk_attn_fwd", "fapk_attn_bwd", "fapk_quantize_mxfp8"} <= set(syms)
+    for s in syms:
+        assert hasattr(L, s), s
+
+
+def test_strerror_and_version(L):
+    for code in range(7):
+        assert fapk.strerror(code)
+    assert "unknown" in fapk.strerror(99)
+    assert L.fapk_version() >= 100
+
+
+def _problem(**kw):
+    seq = type("S", (), {})()
+    P = fapk.Problem()
+    P.T, P.n_docs, P.max_seqlen, P.Hq, P.Hkv, P.d = 300, 2, 200, 4, 2, 128
+    P.scale = 0.088
+    P.prec = fapk.BF16
+    P.scale_rule = fapk.SCALE_RCEIL
+    P.cu_seqlens_dev = 0x1000
+    P.cu_seqlens_host = None
+    P.grad_dtype = fapk.GRAD_F32
+    P.flags = 0
+    P.timeout_ms = 0
+    for k, v in kw.items():
+        setattr(P, k, v)
+    return P
+
+
+def test_workspace_size(L):
+    P = _problem()
+    fwd = fapk.workspace_size(P, fapk.FWD)
+    bwd = fapk.workspace_size(P, fapk.BWD)
+    assert fwd > 0 and bwd >= 4 * 300 * 4  # bwd holds D = rowsum(dO*O) in fp32 [Hq][T]
+    assert fwd % 256 == 0 and bwd % 256 == 0
+    assert fapk.workspace_size(_problem(d=96), fapk.FWD) == 0
+    assert fapk.workspace_size(P, 7) == 0
+
+
+def _fwd(L, P, ws_bytes=1 << 20, ptrs=(16, 16, 16, 16, 16), ws=256):
+    return L.fapk_attn_fwd(ctypes.byref(P), *ptrs, None, ws, ws_bytes, None)
+
+
+def test_host_validation_codes(L):
+    """Every error below is detected on the host, before any CUDA call."""
+    assert _fwd(L, _problem(d=96)) == fapk.ERR_UNSUPPORTED
+    assert _fwd(L, _problem(Hq=3, Hkv=2)) == fapk.ERR_UNSUPPORTED
+    assert _fwd(L, _problem(prec=7)) == fapk.ERR_UNSUPPORTED
+    assert _fwd(L, _problem(Hq=0)) == fapk.ERR_INVALID_ARG
+    assert _fwd(L, _problem(T=-1)) == fapk.ERR_INVALID_ARG
+    assert _fwd(L, _problem(max_seqlen=0)) == fapk.ERR_INVALID_ARG
+    assert _fwd(L, _problem(cu_seqlens_dev=None)) == fapk.ERR_INVALID_ARG
+    assert _fwd(L, _problem(), ptrs=(16, None, 16, 16, 16)) == fapk.ERR_INVALID_ARG
+    assert _fwd(L, _problem(), ptrs=(16, 24, 16, 16, 16)) == fapk.ERR_INVALID_ARG  # misaligned
+    assert _fwd(L, _problem(), ws=512 + 8) == fapk.ERR_INVALID_ARG                  # ws alignment
+    assert _fwd(L, _problem(), ws_bytes=16) == fapk.ERR_WORKSPACE_TOO_SMALL
+    assert _fwd(L, _problem(scale=float("nan"))) == fapk.ERR_INVALID_ARG
+    # T = 0 is a no-op
+    assert _fwd(L, _problem(T=0, n_docs=0)) == fapk.OK
+
+
+@pytest.mark.parametrize("cu,maxlen", [
+    ([1, 100, 300], 200),      # does not start at 0
+    ([0, 100, 299], 200),      # does not end at T
+    ([0, 150, 100, 300], 200), # decreasing
+    ([0, 50, 300], 200),       # a document longer than max_seqlen
+])
+def test_bad_seqlens_detected_on_host(L, cu, maxlen):
+    host = np.asarray(cu, dtype=np.int32)
+    P = _problem(n_docs=len(cu) - 1, max_seqlen=maxlen, cu_seqlens_host=host.ctypes.data)
+    assert _fwd(L, P) == fapk.ERR_BAD_SEQLENS
+
+
+def test_quantize_validation(L):
+    q = L.fapk_quantize_mxfp8
+    x = 256
+    assert q(x, 64, 2, 96, 16, None, 1, 3, 0, 256, 256, 256, 256, None) == fapk.ERR_UNSUPPORTED
+    assert q(x, 64, 2, 64, 16, None, 1, 0, 0, 256, 256, 256, 256, None) == fapk.ERR_INVALID_ARG
+    assert q(x, 64, 2, 64, 16, None, 1, 3, 5, 256, 256, 256, 256, None) == fapk.ERR_UNSUPPORTED
+    assert q(x, 64, 2, 64, 16, None, 1, 1, 0, None, 256, None, None, None) == fapk.ERR_INVALID_ARG
+    assert q(x + 8, 64, 2, 64, 16, None, 1, 2, 0, None, None, 256, 256, None) == fapk.ERR_INVALID_ARG
+    cu = np.array([0, 10, 60], np.int32)
+    assert q(x, 64, 2, 64, 16, cu.ctypes.data, 2, 2, 0, None, None, 256, 256, None) == fapk.ERR_BAD_SEQLENS
+    assert q(x, 0, 2, 64, None, None, 0, 3, 0, None, None, None, None, None) == fapk.OK
