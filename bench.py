@@ -1,0 +1,344 @@
+"""Benchmark of causal packed-document attention, forward + backward.
+
+One step = one fwd + bwd pass over the whole workload (every query head, every
+document) through the C ABI.  Default workload: 32768 packed tokens,
+log-normal document lengths (median 2048, sigma 1, clipped to [64, 16384]),
+32 heads, d = 128, 1% of tokens x8 (seed 0).  Metric: causal-aware TFLOP/s
+with the algorithmic FLOP count 14 d Hq sum_k L_k (L_k + 1) / 2 (masked work is
+never counted), and its fraction of the B200 tensor peaks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fapk|reference]
+                  [--config 1..5]
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+path has no cross-GPU exchange), timings are max-reduced over ranks and
+``value`` counts the work of all ranks.  ``--impl reference`` times the fp64
+CPU oracle on a bounded sample of the same workload on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "causal fwd+bwd attention TFLOP/s (bf16, MXFP8 incl. quant) & % of B200 tensor peak"
+DENSE_BF16_TFLOPS = 2250.0   # NVIDIA B200 datasheet, dense
+DENSE_FP8_TFLOPS = 4500.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk["bf16_tflops_sustained"], "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fapk_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def cpu_oracle_sample(w, target_s: float = 15.0):
+    """Time the fp64 oracle (fwd + bwd) on a bounded sample of the workload:
+    query heads 0..h-1 of the first documents whose cost fits about
+    `target_s` seconds on this host's cores.  Returns (TFLOP/s, cores, text)."""
+    import oracle
+    oracle.build()
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    q, k, v, do = w.tensors()
+    cu = w.cu
+    # sample: a prefix of whole documents, KV head 0 and its query heads
+    G = w.Hq // w.Hkv
+    lengths = np.diff(cu.astype(np.int64))
+    # calibrate on the first document
+    n_docs = 1
+    T1 = int(cu[1])
+    sl = slice(0, T1)
+    args = [t[sl, :G].double().numpy() if i != 1 and i != 2 else t[sl, :1].double().numpy()
+            for i, t in enumerate((q, k, v, do))]
+    t0 = time.perf_counter()
+    oracle.attn_bwd(*args, cu[:2], w.scale)
+    dt = time.perf_counter() - t0
+    flops1 = 14.0 * w.d * G * float(lengths[0] * (lengths[0] + 1) // 2)
+    rate = flops1 / max(dt, 1e-9)
+    # grow the prefix while it fits the budget
+    budget = target_s * rate
+    acc = flops1
+    while n_docs < len(lengths):
+        nxt = 14.0 * w.d * G * float(lengths[n_docs] * (lengths[n_docs] + 1) // 2)
+        if acc + nxt > budget:
+            break
+        acc += nxt
+        n_docs += 1
+    Tn = int(cu[n_docs])
+    sl = slice(0, Tn)
+    args = [t[sl, :G].double().numpy() if i not in (1, 2) else t[sl, :1].double().numpy()
+            for i, t in enumerate((q, k, v, do))]
+    t0 = time.perf_counter()
+    oracle.attn_bwd(*args, cu[: n_docs + 1], w.scale)
+    dt = time.perf_counter() - t0
+    tflops = acc / dt / 1e12
+    text = (f"oracle fp64 fwd+bwd on the first {n_docs} document(s) ({Tn} tokens), KV head 0 and its "
+            f"{G} query head(s): {acc:.3g} FLOP in {dt:.1f} s")
+    return tflops, cores, text, dt
+
+
+def run_reference(args, w, world, rank):
+    """--impl reference: the fp64 CPU oracle, as it stands, on a bounded sample."""
+    if rank != 0:
+        return
+    vals = []
+    text = ""
+    cores = len(os.sched_getaffinity(0))
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        pass
+    for _ in range(args.steps):
+        v, cores, text, _ = cpu_oracle_sample(w, target_s=args.ref_seconds)
+        vals.append(v)
+    val = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {**w.describe(), "path": "oracle fp64 (CPU)"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": text},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fapk", choices=["fapk", "reference"])
+    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--ref-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from causal_flash_attention_packed_b200 import workloads as W
+    w = W.config(args.config, args.seed)
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, w, world, rank)
+        return
+
+    world, rank, local = dist_setup()
+    from causal_flash_attention_packed_b200 import fapk
+    fapk.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+
+    q, k, v, do = w.tensors()
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    seq = fapk.Seqlens(w.cu, dev)
+    P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale)
+    ws_f = fapk.workspace(P, fapk.FWD, dev)
+    ws_b = fapk.workspace(P, fapk.BWD, dev)
+    o = torch.empty((w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.Hq, w.T), dtype=torch.float32, device=dev)
+    dq = torch.empty((w.T, w.Hq, w.d), dtype=torch.float32, device=dev)
+    dk = torch.empty((w.T, w.Hkv, w.d), dtype=torch.float32, device=dev)
+    dv = torch.empty((w.T, w.Hkv, w.d), dtype=torch.float32, device=dev)
+    ctx = torch.empty(max(fapk.ctx_size(P), 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fapk.attn_fwd(P, qd, kd, vd, o=o, lse=lse, ctx=ctx, ws=ws_f, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        fapk.attn_bwd(P, qd, kd, vd, o, lse, dod, ctx=ctx, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert fapk.status(ws_f) == 0 and fapk.status(ws_b) == 0
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    launches0 = fapk.launch_count()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.start()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    launches = fapk.launch_count() - launches0
+    st_ok = fapk.status(ws_f) == 0 and fapk.status(ws_b) == 0
+    total_ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    fwd_ms = max_over_ranks(fwd_ms, world, dev)
+    bwd_ms = max_over_ranks(bwd_ms, world, dev)
+    ms_per_step = total_ms / args.steps
+    flops = w.flops()
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the C ABI with host buffers (pinned), copies included
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hdq = torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True)
+        hdk = torch.empty(dk.shape, dtype=dk.dtype, pin_memory=True)
+        hdv = torch.empty(dv.shape, dtype=dv.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdk, hdv))
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for src, dst in ((hq, qd), (hk, kd), (hv, vd), (hdo, dod)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for src, dst in ((o, ho), (dq, hdq), (dk, hdk), (dv, hdv)):
+                dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
+        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    fwd_flops = 4.0 * w.d * w.Hq * w.pairs()
+    bwd_flops = 10.0 * w.d * w.Hq * w.pairs()
+    dom_is_bwd = bwd_ms >= fwd_ms
+    dom_ms = bwd_ms if dom_is_bwd else fwd_ms
+    dom_flops = bwd_flops if dom_is_bwd else fwd_flops
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "attn_bwd call (delta, dK/dV and dQ kernels)" if dom_is_bwd
+                else "attn_fwd call (forward kernel)",
+                "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)",
+                "fwd": {"ms": fwd_ms, "tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12},
+                "bwd": {"ms": bwd_ms, "tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12}}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v_cpu, cores, text, _ = cpu_oracle_sample(w, target_s=15.0)
+        cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": text}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**w.describe(), "path": "bf16", "parallelism": f"replicas x{world}",
+                   "l2": f"inputs {sum(t.numel() * 2 for t in (q, k, v, do)) / 1e9:.2f} GB > 126 MB L2, no flush"},
+        "pct_of_dense_bf16_peak": 100.0 * (value / world) / DENSE_BF16_TFLOPS,
+        "pct_of_measured_bf16_peak": 100.0 * (value / world) / peaks["bf16_tflops"],
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "clocks": clk, "status_ok": st_ok,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -145,6 +145,20 @@ BwdLayout bwd_layout(const fapk_problem_t* P) {
   return L;
 }
 
+// Saved state from the forward to the backward (the caller's ctx buffer):
+//  o_resid: bf16 [T][Hq][d], O_fp32 - bf16(O_fp32), so that the backward's
+//           D_i = dO_i . O_i uses O to about 16 significant bits rather than
+//           the 8 of the bf16 output.
+struct CtxLayout {
+  size_t o_resid, total;
+};
+CtxLayout ctx_layout(const fapk_problem_t* P) {
+  CtxLayout L;
+  L.o_resid = 0;
+  L.total = align_up(sizeof(uint16_t) * (size_t)P->T * P->Hq * P->d);
+  return L;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? FAPK_OK : FAPK_ERR_CUDA; }
 
 }  // namespace
@@ -178,18 +192,17 @@ size_t fapk_workspace_size(const fapk_problem_t* prob, int which) {
 
 size_t fapk_ctx_size(const fapk_problem_t* prob) {
   if (validate_problem(prob) != FAPK_OK) return 0;
-  return 0;
+  return ctx_layout(prob).total;
 }
 
 int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const void* v, void* o,
                   float* lse, void* ctx, void* ws, size_t ws_bytes, void* stream) {
-  (void)ctx;
   int rc = validate_problem(P);
   if (rc != FAPK_OK) return rc;
   if (P->T == 0) return FAPK_OK;
   if (!q || !k || !v || !o || !lse || !ws) return FAPK_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
-      (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+      !aligned16(ctx) || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
     return FAPK_ERR_INVALID_ARG;
   const FwdLayout L = fwd_layout(P);
   if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
@@ -200,6 +213,7 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
   auto* status = static_cast<DeviceStatus*>(ws);
   FwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+  a.o_resid = ctx ? static_cast<char*>(ctx) + ctx_layout(P).o_resid : nullptr;
   a.cu = P->cu_seqlens_dev;
   a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.d = P->d;
   a.scale = P->scale;
@@ -216,13 +230,12 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
 int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const void* v, const void* o,
                   const float* lse, const void* dout, const void* ctx, void* dq, void* dk, void* dv,
                   void* ws, size_t ws_bytes, void* stream) {
-  (void)ctx;
   int rc = validate_problem(P);
   if (rc != FAPK_OK) return rc;
   if (P->T == 0) return FAPK_OK;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !ws) return FAPK_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
-      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(ctx) ||
       (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
     return FAPK_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(P);
@@ -234,6 +247,7 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   auto* status = static_cast<DeviceStatus*>(ws);
   BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
+  a.o_resid = ctx ? static_cast<const char*>(ctx) + ctx_layout(P).o_resid : nullptr;
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.delta = reinterpret_cast<float*>(static_cast<char*>(ws) + L.delta);
   a.cu = P->cu_seqlens_dev;

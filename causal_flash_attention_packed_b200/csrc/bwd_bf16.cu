@@ -1,2 +1,707 @@
+// Backward of causal packed-document attention, bf16 operands, for sm_100a.
+//
+// The analytic derivative of the forward (the pages give none):
+//   D_i   = dO_i . O_i
+//   P_ij  = exp(S_ij - LSE_i)           (recomputed from the saved LSE)
+//   dP_ij = dO_i . V_j,   dS_ij = P_ij (dP_ij - D_i)
+//   dV_j  = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij Q_i,  dQ_i = scale sum_j dS_ij K_j
+// over visible pairs only (j <= i, same document).
+//
+// Three kernels, all deterministic (no atomics, fixed summation order):
+//  1. delta_kernel: D for every (token, head).
+//  2. dkdv kernel: one work item per (document, 128-key tile, KV head).  For
+//     each query head of the group and each query tile at or after the key
+//     tile: S^T = K Q^T and dP^T = V dO^T into TMEM (one thread per key row),
+//     P^T and dS^T written back into TMEM as bf16, then dV += P^T dO and
+//     dK += dS^T Q with A read from TMEM.  dK, dV accumulate in TMEM across
+//     the whole item (query heads of the group included) and are written once.
+//  3. dq kernel: one work item per (document, 128-query tile, query head).
+//     For each key tile at or before it: S = Q K^T, dP = dO V^T, dS in TMEM,
+//     dQ += dS K.
+// Warp roles as in the forward: warp 8 loads (TMA), warp 9 issues tcgen05
+// MMAs, warps 0-7 compute P and dS (warpgroup 0 on columns 0-63, warpgroup 1
+// on columns 64-127 of each 128x128 tile, every thread owning one TMEM lane).
+#include <cuda_bf16.h>
+
 #include "internal.h"
-namespace fapk { cudaError_t launch_bwd_bf16(const BwdArgs&, cudaStream_t) { return cudaErrorNotSupported; } }
+#include "ptx.cuh"
+
+namespace fapk {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct Geo {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kBoxBytes = 128 * 64 * 2;
+  static constexpr int kNumBox = D / 64;
+};
+
+// Bounded wait that ignores the abort flag (teardown: drain what is in flight).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > budget_ns) return;
+  }
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd, int where) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
+}
+
+// 64 TMEM columns of this thread's lane -> registers.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
+
+// K-major operand (rows of 128 bytes, 64 bf16 along K per box): descriptor of
+// the kk-th 16-element K step.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk, int box_bytes) {
+  return sdesc_sw128(tile + (kk >> 2) * box_bytes + (kk & 3) * 32, 16, 1024);
+}
+// MN-major operand (rows = K index, 64 bf16 along MN per 128-byte row, boxes
+// 16 KB apart along MN): descriptor of the kk-th 16-row K step.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk, int box_bytes) {
+  return sdesc_sw128(tile + kk * 2048, box_bytes, 1024);
+}
+
+// Column of the kk-th 16-element K step of a bf16 A operand that the two
+// warpgroups wrote into TMEM: steps 0-3 (elements 0-63) at base + 8 kk,
+// steps 4-7 (elements 64-127) at base + 64 + 8 (kk - 4).
+__device__ __forceinline__ uint32_t split_a_col(uint32_t base, int kk) {
+  return base + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4));
+}
+
+// ---------------------------------------------------------------------------
+// 1. D = rowsum(dO * O), fp32 [Hq][T]
+// ---------------------------------------------------------------------------
+// O is taken as o + o_resid when the forward saved its rounding residual
+// (about 16 significant bits), else as the bf16 o alone.
+template <int D>
+__global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o,
+                                                    const __nv_bfloat16* __restrict__ o_resid,
+                                                    const __nv_bfloat16* __restrict__ dout,
+                                                    float* __restrict__ delta, int T, int Hq) {
+  constexpr int TPR = D / 8;  // threads per (token, head) row
+  const long long row = (long long)blockIdx.x * (256 / TPR) + threadIdx.x / TPR;
+  const int c8 = threadIdx.x % TPR;
+  float acc = 0.f;
+  if (row < (long long)T * Hq) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + row * D) + c8);
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + c8);
+    const uint4 r = o_resid ? __ldg(reinterpret_cast<const uint4*>(o_resid + row * D) + c8) : make_uint4(0, 0, 0, 0);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w}, wr[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc += (__uint_as_float(wa[i] << 16) + __uint_as_float(wr[i] << 16)) * __uint_as_float(wb[i] << 16);
+      acc += (__uint_as_float(wa[i] & 0xFFFF0000u) + __uint_as_float(wr[i] & 0xFFFF0000u)) *
+             __uint_as_float(wb[i] & 0xFFFF0000u);
+    }
+  }
+#pragma unroll
+  for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+  if (row < (long long)T * Hq && c8 == 0) {
+    const long long t = row / Hq, h = row % Hq;
+    delta[h * T + t] = acc;
+  }
+}
+
+struct BwdParams {
+  const int32_t* cu;
+  const int2* list;
+  const int* n_items;
+  const float* lse;
+  const float* delta;
+  void* out0;  // dkdv: dk;  dq: dq
+  void* out1;  // dkdv: dv
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+  int T, Hq, Hkv;
+  float scale;       // softmax scale (dK, dQ factor)
+  float scale_log2;  // scale * log2(e)
+  int grad_bf16;
+};
+
+// Store 32 fp32 values (times `mul`) of one row as fp32 or bf16.
+__device__ __forceinline__ void store_row32(void* base, size_t elem_off, const uint32_t (&t)[32], float mul,
+                                            bool bf16) {
+  if (bf16) {
+    uint32_t ob[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      ob[e] = pack_bf16x2(__uint_as_float(t[2 * e]) * mul, __uint_as_float(t[2 * e + 1]) * mul);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + elem_off);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+  } else {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(base) + elem_off);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      dst[e] = make_float4(__uint_as_float(t[4 * e]) * mul, __uint_as_float(t[4 * e + 1]) * mul,
+                           __uint_as_float(t[4 * e + 2]) * mul, __uint_as_float(t[4 * e + 3]) * mul);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. dK, dV
+// ---------------------------------------------------------------------------
+template <int D>
+struct KvCfg : Geo<D> {
+  static constexpr int kStages = (D == 128) ? 2 : 3;
+  static constexpr int kStageBytes = 2 * Geo<D>::kTileBytes + 1024;  // Q, dO, LSE*log2e[128], D[128]
+  static constexpr int kSmemTiles = 2 * Geo<D>::kTileBytes + kStages * kStageBytes;
+  // TMEM: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D)
+  static constexpr uint32_t kS = 0, kDP = 128, kDV = 256, kDK = 256 + D;
+  // bars: kv_full, kv_empty, st_full[S], st_empty[S], s_full, p_full, acc_full, acc_free, fin
+  static constexpr int kNumBars = 2 + 2 * kStages + 5;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
+};
+
+struct KvItem {
+  int s, e, v, g, k0, nq;  // k0: first key of the tile; nq: query tiles v..nq-1
+};
+
+__device__ __forceinline__ KvItem kv_decode(const BwdParams& p, int w) {
+  KvItem it;
+  const int2 pr = p.list[w / p.Hkv];
+  it.g = w % p.Hkv;
+  it.s = p.cu[pr.x];
+  it.e = p.cu[pr.x + 1];
+  it.v = pr.y;
+  it.k0 = it.s + 128 * it.v;
+  it.nq = (it.e - it.s + 127) / 128;
+  return it;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdParams p) {
+  using C = KvCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + C::kTileBytes;
+  uint8_t* sStage = smem + 2 * C::kTileBytes;  // per stage: Q tile, dO tile, lse2[128], delta[128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* st_full = bars + 2;
+  uint64_t* st_empty = bars + 2 + C::kStages;
+  uint64_t* s_full = bars + 2 + 2 * C::kStages;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* acc_full = s_full + 2;
+  uint64_t* acc_free = s_full + 3;
+  uint64_t* fin = s_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(st_full + i, 32);  // lane 0's expect_tx arrive + 31 lanes after their smem stores
+      mbar_init(st_empty + i, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 256);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_free, 256);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{p.status, abort_flag, p.timeout_ns};
+  const int n_units = (*p.n_items) * p.Hkv;
+  const int G = p.Hq / p.Hkv;
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ loads
+    uint32_t st_it = 0;
+    int unit_i = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      const KvItem it = kv_decode(p, w);
+      if (unit_i > 0 && !warp_wait(kv_empty, (unit_i - 1) & 1, wd, 21)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+        for (int b = 0; b < C::kNumBox; ++b) {
+          tma_load_3d(sK + b * C::kBoxBytes, &tm_k, kv_full, 64 * b, it.g, it.k0);
+          tma_load_3d(sV + b * C::kBoxBytes, &tm_v, kv_full, 64 * b, it.g, it.k0);
+        }
+      }
+      for (int h = it.g * G; h < (it.g + 1) * G && ok; ++h) {
+        for (int m = it.v; m < it.nq; ++m, ++st_it) {
+          const int stage = st_it % C::kStages;
+          const uint32_t use = st_it / C::kStages;
+          if (use > 0 && !warp_wait(st_empty + stage, (use - 1) & 1, wd, 22)) { ok = false; break; }
+          uint8_t* sb = sStage + stage * C::kStageBytes;
+          const int q0 = it.s + 128 * m;
+          float* lse2 = reinterpret_cast<float*>(sb + 2 * C::kTileBytes);
+          float* dl = lse2 + 128;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int i = q0 + lane * 4 + r;
+            const bool in = i < p.T;
+            lse2[lane * 4 + r] = in ? p.lse[(size_t)h * p.T + i] * kLog2e : 0.f;
+            dl[lane * 4 + r] = in ? p.delta[(size_t)h * p.T + i] : 0.f;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(st_full + stage, 2 * C::kTileBytes);
+            for (int b = 0; b < C::kNumBox; ++b) {
+              tma_load_3d(sb + b * C::kBoxBytes, &tm_q, st_full + stage, 64 * b, h, q0);
+              tma_load_3d(sb + C::kTileBytes + b * C::kBoxBytes, &tm_do, st_full + stage, 64 * b, h, q0);
+            }
+          } else {
+            mbar_arrive(st_full + stage);
+          }
+        }
+      }
+    }
+    if (lane == 0) {
+      // teardown: let this thread's copies land before the CTA exits
+      if (unit_i > 0) drain_wait(kv_full, (unit_i - 1) & 1, p.timeout_ns);
+      for (uint32_t i = (st_it > C::kStages ? st_it - C::kStages : 0); i < st_it; ++i)
+        drain_wait(st_full + (i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);  // K-major x K-major
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);     // TMEM A x MN-major B
+      const uint32_t sk = smem_u32(sK), sv = smem_u32(sV), sst = smem_u32(sStage);
+      uint32_t st_it = 0, p_cnt = 0;
+      int unit_i = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+        const KvItem it = kv_decode(p, w);
+        if (!mbar_wait(kv_full, unit_i & 1, wd, 23)) break;
+        if (unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 24)) break;
+        tc_fence_after();
+        bool first = true;
+        for (int h = it.g * G; h < (it.g + 1) * G && ok; ++h) {
+          for (int m = it.v; m < it.nq; ++m, ++st_it) {
+            const int stage = st_it % C::kStages;
+            if (!mbar_wait(st_full + stage, (st_it / C::kStages) & 1, wd, 25)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sq = sst + stage * C::kStageBytes, sdo = sq + C::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              mma_f16_ss(tmem + C::kS, kmajor_desc(sk, kk, C::kBoxBytes), kmajor_desc(sq, kk, C::kBoxBytes),
+                         idesc_s, kk > 0);
+              mma_f16_ss(tmem + C::kDP, kmajor_desc(sv, kk, C::kBoxBytes), kmajor_desc(sdo, kk, C::kBoxBytes),
+                         idesc_s, kk > 0);
+            }
+            tc_commit(s_full);
+            if (!mbar_wait(p_full, p_cnt & 1, wd, 26)) { ok = false; break; }
+            ++p_cnt;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+              mma_f16_ts(tmem + C::kDV, split_a_col(tmem + C::kS, kk), mnmajor_desc(sdo, kk, C::kBoxBytes),
+                         idesc_g, acc);
+              mma_f16_ts(tmem + C::kDK, split_a_col(tmem + C::kDP, kk), mnmajor_desc(sq, kk, C::kBoxBytes),
+                         idesc_g, acc);
+            }
+            first = false;
+            tc_commit(st_empty + stage);
+          }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        tc_commit(kv_empty);
+      }
+      tc_commit(fin);
+      drain_wait(fin, 0, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ P^T, dS^T
+    const int wg = warp >> 2, quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // key row of the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_addr = lane_base + C::kS + 64 * wg;   // S^T columns of this warpgroup
+    const uint32_t dp_addr = lane_base + C::kDP + 64 * wg;
+    uint32_t s_cnt = 0, st_it = 0;
+    int unit_i = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      const KvItem it = kv_decode(p, w);
+      const int j = it.k0 + row;  // key index
+      for (int h = it.g * G; h < (it.g + 1) * G && ok; ++h) {
+        for (int m = it.v; m < it.nq; ++m, ++st_it) {
+          const int stage = st_it % C::kStages;
+          if (!warp_wait(s_full, s_cnt & 1, wd, 27)) { ok = false; break; }
+          ++s_cnt;
+          tc_fence_after();
+          const float* lse2 = reinterpret_cast<const float*>(sStage + stage * C::kStageBytes + 2 * C::kTileBytes);
+          const float* dl = lse2 + 128;
+          uint32_t sr[64], dr[64];
+          tmem_ld64(s_addr, sr);
+          tmem_ld64(dp_addr, dr);
+          const int i0 = it.s + 128 * m + 64 * wg;  // query index of column 0 of this half
+          // visible iff j <= i < e; only the diagonal and the last query tile need the test
+          const bool full = (m > it.v) && (it.s + 128 * m + 128 <= it.e);
+          uint32_t pk[32], dk[32];
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            float pv[2], dv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int cc = c + u;
+              const float l2 = lse2[64 * wg + cc];
+              float pp = fast_exp2(__uint_as_float(sr[cc]) * p.scale_log2 - l2);
+              if (!full) {
+                const int i = i0 + cc;
+                if (i < j || i >= it.e) pp = 0.f;
+              }
+              pv[u] = pp;
+              dv[u] = pp * (__uint_as_float(dr[cc]) - dl[64 * wg + cc]);
+            }
+            pk[c / 2] = pack_bf16x2(pv[0], pv[1]);
+            dk[c / 2] = pack_bf16x2(dv[0], dv[1]);
+          }
+          tmem_st32(s_addr, pk);    // P^T  -> columns [64 wg, 64 wg + 32) of S^T
+          tmem_st32(dp_addr, dk);   // dS^T -> columns [64 wg, 64 wg + 32) of dP^T
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(p_full);
+        }
+      }
+      if (!ok) break;
+      // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK * scale
+      if (!warp_wait(acc_full, unit_i & 1, wd, 28)) break;
+      tc_fence_after();
+      const bool valid = j < it.e;
+      const uint32_t acc_addr = lane_base + (wg ? C::kDK : C::kDV);
+      void* out = wg ? p.out0 : p.out1;
+      const float mul = wg ? p.scale : 1.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t t[32];
+        tmem_ld32(acc_addr + 32 * c, t);
+        tmem_wait_ld(t);
+        if (valid) store_row32(out, ((size_t)j * p.Hkv + it.g) * D + 32 * c, t, mul, p.grad_bf16);
+      }
+      tc_fence_before();
+      mbar_arrive(acc_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// 3. dQ
+// ---------------------------------------------------------------------------
+template <int D>
+struct QCfg : Geo<D> {
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kStageBytes = 2 * Geo<D>::kTileBytes;  // K, V
+  static constexpr int kSmemTiles = 2 * Geo<D>::kTileBytes + kStages * kStageBytes;
+  // TMEM: S [0,128), dP [128,256), dQ [256,256+D)
+  static constexpr uint32_t kS = 0, kDP = 128, kDQ = 256;
+  // bars: q_full, q_empty, st_full[S], st_empty[S], s_full, p_full, acc_full, acc_free, fin
+  static constexpr int kNumBars = 2 + 2 * kStages + 5;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
+};
+
+struct QItem {
+  int s, e, m, h, g, q0;  // key tiles 0..m
+};
+
+__device__ __forceinline__ QItem q_decode(const BwdParams& p, int w) {
+  QItem it;
+  const int2 pr = p.list[w / p.Hq];
+  it.h = w % p.Hq;
+  it.g = it.h / (p.Hq / p.Hkv);
+  it.s = p.cu[pr.x];
+  it.e = p.cu[pr.x + 1];
+  it.m = pr.y;
+  it.q0 = it.s + 128 * it.m;
+  return it;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const BwdParams p) {
+  using C = QCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sDO = smem + C::kTileBytes;
+  uint8_t* sStage = smem + 2 * C::kTileBytes;  // per stage: K tile, V tile
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* st_full = bars + 2;
+  uint64_t* st_empty = bars + 2 + C::kStages;
+  uint64_t* s_full = bars + 2 + 2 * C::kStages;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* acc_full = s_full + 2;
+  uint64_t* acc_free = s_full + 3;
+  uint64_t* fin = s_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(st_full + i, 1);
+      mbar_init(st_empty + i, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 256);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_free, 256);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{p.status, abort_flag, p.timeout_ns};
+  const int n_units = (*p.n_items) * p.Hq;
+
+  if (warp == kLoadWarp) {
+    if (lane == 0) {
+      uint32_t st_it = 0;
+      int unit_i = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+        const QItem it = q_decode(p, w);
+        if (unit_i > 0 && !mbar_wait(q_empty, (unit_i - 1) & 1, wd, 31)) break;
+        mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
+        for (int b = 0; b < C::kNumBox; ++b) {
+          tma_load_3d(sQ + b * C::kBoxBytes, &tm_q, q_full, 64 * b, it.h, it.q0);
+          tma_load_3d(sDO + b * C::kBoxBytes, &tm_do, q_full, 64 * b, it.h, it.q0);
+        }
+        for (int v = 0; v <= it.m; ++v, ++st_it) {
+          const int stage = st_it % C::kStages;
+          const uint32_t use = st_it / C::kStages;
+          if (use > 0 && !mbar_wait(st_empty + stage, (use - 1) & 1, wd, 32)) { ok = false; break; }
+          uint8_t* sb = sStage + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(st_full + stage, 2 * C::kTileBytes);
+          for (int b = 0; b < C::kNumBox; ++b) {
+            tma_load_3d(sb + b * C::kBoxBytes, &tm_k, st_full + stage, 64 * b, it.g, it.s + 128 * v);
+            tma_load_3d(sb + C::kTileBytes + b * C::kBoxBytes, &tm_v, st_full + stage, 64 * b, it.g,
+                        it.s + 128 * v);
+          }
+        }
+      }
+      if (unit_i > 0) drain_wait(q_full, (unit_i - 1) & 1, p.timeout_ns);
+      for (uint32_t i = (st_it > C::kStages ? st_it - C::kStages : 0); i < st_it; ++i)
+        drain_wait(st_full + (i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);
+      const uint32_t sq = smem_u32(sQ), sdo = smem_u32(sDO), sst = smem_u32(sStage);
+      uint32_t st_it = 0, p_cnt = 0;
+      int unit_i = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+        const QItem it = q_decode(p, w);
+        if (!mbar_wait(q_full, unit_i & 1, wd, 33)) break;
+        if (unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 34)) break;
+        tc_fence_after();
+        for (int v = 0; v <= it.m; ++v, ++st_it) {
+          const int stage = st_it % C::kStages;
+          if (!mbar_wait(st_full + stage, (st_it / C::kStages) & 1, wd, 35)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sk = sst + stage * C::kStageBytes, sv = sk + C::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            mma_f16_ss(tmem + C::kS, kmajor_desc(sq, kk, C::kBoxBytes), kmajor_desc(sk, kk, C::kBoxBytes),
+                       idesc_s, kk > 0);
+            mma_f16_ss(tmem + C::kDP, kmajor_desc(sdo, kk, C::kBoxBytes), kmajor_desc(sv, kk, C::kBoxBytes),
+                       idesc_s, kk > 0);
+          }
+          tc_commit(s_full);
+          if (!mbar_wait(p_full, p_cnt & 1, wd, 36)) { ok = false; break; }
+          ++p_cnt;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16_ts(tmem + C::kDQ, split_a_col(tmem + C::kS, kk), mnmajor_desc(sk, kk, C::kBoxBytes), idesc_g,
+                       (v > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(st_empty + stage);
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        tc_commit(q_empty);
+      }
+      tc_commit(fin);
+      drain_wait(fin, 0, p.timeout_ns);
+    }
+  } else {
+    const int wg = warp >> 2, quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // query row of the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_addr = lane_base + C::kS + 64 * wg;
+    const uint32_t dp_addr = lane_base + C::kDP + 64 * wg;
+    uint32_t s_cnt = 0;
+    int unit_i = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      const QItem it = q_decode(p, w);
+      const int i = it.q0 + row;
+      const bool valid = i < it.e;
+      const float l2 = (i < p.T) ? p.lse[(size_t)it.h * p.T + i] * kLog2e : 0.f;
+      const float dl = (i < p.T) ? p.delta[(size_t)it.h * p.T + i] : 0.f;
+      for (int v = 0; v <= it.m; ++v) {
+        if (!warp_wait(s_full, s_cnt & 1, wd, 37)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[64], dr[64];
+        tmem_ld64(s_addr, sr);
+        tmem_ld64(dp_addr, dr);
+        const int j0 = it.s + 128 * v + 64 * wg;  // key index of column 0 of this half
+        const bool diag = v == it.m;
+        uint32_t dk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float dv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int cc = c + u;
+            float pp = fast_exp2(__uint_as_float(sr[cc]) * p.scale_log2 - l2);
+            if (diag && j0 + cc > i) pp = 0.f;
+            dv[u] = pp * (__uint_as_float(dr[cc]) - dl);
+          }
+          dk[c / 2] = pack_bf16x2(dv[0], dv[1]);
+        }
+        tmem_st32(s_addr, dk);  // dS -> columns [64 wg, 64 wg + 32) of S
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      if (!warp_wait(acc_full, unit_i & 1, wd, 38)) break;
+      tc_fence_after();
+      // warpgroup wg writes channels [wg D/2, (wg+1) D/2) of dQ * scale
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t t[32];
+        const int col = wg * (D / 2) + 32 * c;
+        tmem_ld32(lane_base + C::kDQ + col, t);
+        tmem_wait_ld(t);
+        if (valid) store_row32(p.out0, ((size_t)i * p.Hq + it.h) * D + col, t, p.scale, p.grad_bf16);
+      }
+      tc_fence_before();
+      mbar_arrive(acc_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+template <int D>
+cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap_thd(&tq, a.q, a.T, a.Hq, D) || !make_tmap_thd(&tk, a.k, a.T, a.Hkv, D) ||
+      !make_tmap_thd(&tv, a.v, a.T, a.Hkv, D) || !make_tmap_thd(&tdo, a.dout, a.T, a.Hq, D))
+    return cudaErrorInvalidValue;
+  // 1. D
+  {
+    constexpr int rows_per_block = 256 / (D / 8);
+    const long long rows = (long long)a.T * a.Hq;
+    const unsigned grid = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
+    delta_kernel<D><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.o),
+                                               static_cast<const __nv_bfloat16*>(a.o_resid),
+                                               static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.T, a.Hq);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  BwdParams p;
+  p.cu = a.cu;
+  p.lse = a.lse;
+  p.delta = a.delta;
+  p.status = a.status;
+  p.timeout_ns = a.timeout_ns;
+  p.T = a.T;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * kLog2e;
+  p.grad_bf16 = a.grad_bf16;
+  // 2. dK, dV
+  {
+    using C = KvCfg<D>;
+    cudaError_t e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    BwdParams pk = p;
+    pk.list = a.sched_kv.list;
+    pk.n_items = a.sched_kv.n_items;
+    pk.out0 = a.dk;
+    pk.out1 = a.dv;
+    const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
+    const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
+    dkdv_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, pk);
+    note_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // 3. dQ
+  {
+    using C = QCfg<D>;
+    cudaError_t e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    BwdParams pq = p;
+    pq.list = a.sched_q.list;
+    pq.n_items = a.sched_q.n_items;
+    pq.out0 = a.dq;
+    pq.out1 = nullptr;
+    const long long max_units = (long long)a.sched_q.max_items * a.Hq;
+    const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
+    dq_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, pq);
+    note_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream) {
+  return a.d == 128 ? launch_d<128>(a, stream) : launch_d<64>(a, stream);
+}
+
+}  // namespace fapk

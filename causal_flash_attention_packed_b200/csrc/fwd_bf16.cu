@@ -61,6 +61,7 @@ struct Params {
   const int* n_items;
   __nv_bfloat16* o;
   float* lse;
+  __nv_bfloat16* o_resid;
   DeviceStatus* status;
   uint64_t timeout_ns;
   int T, Hq, Hkv;
@@ -374,14 +375,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t t[32];
         tmem_ld32(o_addr + 32 * c, t);
         tmem_wait_ld(t);
-        uint32_t ob[16];
+        uint32_t ob[16], rb[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          ob[e] = pack_bf16x2(__uint_as_float(t[2 * e]) * inv_l, __uint_as_float(t[2 * e + 1]) * inv_l);
+        for (int e = 0; e < 16; ++e) {
+          const float f0 = __uint_as_float(t[2 * e]) * inv_l, f1 = __uint_as_float(t[2 * e + 1]) * inv_l;
+          ob[e] = pack_bf16x2(f0, f1);
+          // residual: what bf16 rounding dropped (exactly representable up to bf16 rounding again)
+          rb[e] = pack_bf16x2(f0 - __uint_as_float(ob[e] << 16), f1 - __uint_as_float(ob[e] & 0xFFFF0000u));
+        }
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+          if (p.o_resid) {
+            uint4* rdst = reinterpret_cast<uint4*>(p.o_resid + ((size_t)q_idx * p.Hq + it.h) * D + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) rdst[e] = make_uint4(rb[4 * e], rb[4 * e + 1], rb[4 * e + 2], rb[4 * e + 3]);
+          }
         }
       }
       tc_fence_before();
@@ -411,6 +421,7 @@ cudaError_t launch_d(const FwdArgs& a, cudaStream_t stream) {
   p.n_items = a.sched.n_items;
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.lse = a.lse;
+  p.o_resid = static_cast<__nv_bfloat16*>(a.o_resid);
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
   p.T = a.T;

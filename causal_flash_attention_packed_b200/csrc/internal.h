@@ -43,6 +43,7 @@ struct FwdArgs {
   const void* v;
   void* o;
   float* lse;
+  void* o_resid;  // optional bf16 [T][Hq][d]: O_fp32 - bf16(O_fp32), for the backward's D
   const int32_t* cu;
   int T, Hq, Hkv, d;
   float scale;
@@ -62,6 +63,7 @@ struct BwdArgs {
   const void* o;
   const float* lse;
   const void* dout;
+  const void* o_resid;  // optional residual of O written by the forward (NULL: D from bf16 O)
   void* dq;
   void* dk;
   void* dv;

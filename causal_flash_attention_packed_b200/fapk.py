@@ -177,12 +177,13 @@ def attn_fwd(P: Problem, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
              o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
              ctx: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
              stream=None) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
-    """fapk_attn_fwd: returns (o [T,Hq,d] bf16, lse [Hq,T] fp32, ctx)."""
+    """fapk_attn_fwd: returns (o [T,Hq,d] bf16, lse [Hq,T] fp32, ctx).  Pass the
+    returned ctx to attn_bwd."""
     if o is None:
         o = torch.empty((P.T, P.Hq, P.d), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((P.Hq, P.T), dtype=torch.float32, device=q.device)
-    if ctx is None and P.prec == MXFP8:
+    if ctx is None:
         ctx = torch.empty(max(ctx_size(P), 256), dtype=torch.uint8, device=q.device)
     if ws is None:
         ws = workspace(P, FWD, q.device)

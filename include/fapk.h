@@ -127,19 +127,25 @@ typedef struct {
  * aligned, contents need not be initialised, not shared by concurrent calls. */
 FAPK_API size_t fapk_workspace_size(const fapk_problem_t* prob, int which);
 
-/* Bytes of the saved-operand buffer that the MXFP8 forward fills and the
- * MXFP8 backward reads (the quantised token-block operands reused across
- * orientations, FLAMIA page: "token-block scaling").  0 for FAPK_BF16. */
+/* Bytes of the saved-state buffer `ctx` that the forward fills and the
+ * backward reads.  It holds the bf16 rounding residual of O (O_fp32 minus its
+ * bf16 rounding, [T][Hq][d] bf16), so that the backward's D_i = dO_i . O_i
+ * sees O to about 16 significant bits; the MXFP8 path adds its quantised
+ * token-block operands, reused across orientations (FLAMIA page: "token-block
+ * scaling"). */
 FAPK_API size_t fapk_ctx_size(const fapk_problem_t* prob);
 
 /* Forward.  Reads q, k, v (bf16); writes o (bf16) and lse (fp32, natural
- * log).  ctx: device buffer of fapk_ctx_size() bytes (MXFP8) or NULL (BF16).
+ * log).  ctx: device buffer of fapk_ctx_size() bytes, 16-byte aligned, filled
+ * for the backward; it may be NULL for FAPK_BF16 (the backward then takes D
+ * from the bf16 o alone, which loses accuracy where dS cancels).
  * ws: workspace of at least fapk_workspace_size(prob, FAPK_FWD) bytes. */
 FAPK_API int fapk_attn_fwd(const fapk_problem_t* prob, const void* q, const void* k, const void* v,
                   void* o, float* lse, void* ctx, void* ws, size_t ws_bytes, void* stream);
 
-/* Backward.  Reads q, k, v, o, lse, dout (bf16 except lse) and, for MXFP8,
- * the ctx written by the matching forward; writes dq [T][Hq][d] and
+/* Backward.  Reads q, k, v, o, lse, dout (bf16 except lse) and the ctx
+ * written by the matching forward (NULL allowed for FAPK_BF16, see
+ * fapk_attn_fwd); writes dq [T][Hq][d] and
  * dk, dv [T][Hkv][d] in grad_dtype.  dk and dv are summed over the query
  * heads that share a KV head.  ws: at least fapk_workspace_size(prob,
  * FAPK_BWD) bytes. */
