@@ -132,30 +132,39 @@ FwdLayout fwd_layout(const fapk_problem_t* P) {
   return L;
 }
 
+// Backward workspace: two work lists, D = rowsum(dO * O) in fp32 and the fp16
+// copies of Q, K and dO that the gradient MMAs read.
 struct BwdLayout {
   SchedLayout kv, q;
-  size_t delta, total;
+  size_t delta, q16, k16, do16, total;
 };
 BwdLayout bwd_layout(const fapk_problem_t* P) {
   BwdLayout L;
+  const size_t nq = (size_t)P->T * P->Hq * P->d, nk = (size_t)P->T * P->Hkv * P->d;
   L.kv = sched_layout(kAlign, P->T, P->n_docs, P->max_seqlen, kBwdRows);
   L.q = sched_layout(L.kv.end, P->T, P->n_docs, P->max_seqlen, kBwdRows);
   L.delta = L.q.end;
-  L.total = align_up(L.delta + sizeof(float) * (size_t)P->Hq * (size_t)P->T);
+  L.q16 = align_up(L.delta + sizeof(float) * (size_t)P->Hq * (size_t)P->T);
+  L.k16 = align_up(L.q16 + 2 * nq);
+  L.do16 = align_up(L.k16 + 2 * nk);
+  L.total = align_up(L.do16 + 2 * nq);
   return L;
 }
 
 // Saved state from the forward to the backward (the caller's ctx buffer):
 //  o_resid: bf16 [T][Hq][d], O_fp32 - bf16(O_fp32), so that the backward's
 //           D_i = dO_i . O_i uses O to about 16 significant bits rather than
-//           the 8 of the bf16 output.
+//           the 8 of the bf16 output;
+//  v16:     fp16 copy of V [T][Hkv][d], the B operand of O += P V (and of the
+//           backward's dP = dO V^T).
 struct CtxLayout {
-  size_t o_resid, total;
+  size_t o_resid, v16, total;
 };
 CtxLayout ctx_layout(const fapk_problem_t* P) {
   CtxLayout L;
   L.o_resid = 0;
-  L.total = align_up(sizeof(uint16_t) * (size_t)P->T * P->Hq * P->d);
+  L.v16 = align_up(sizeof(uint16_t) * (size_t)P->T * P->Hq * P->d);
+  L.total = align_up(L.v16 + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
   return L;
 }
 
@@ -165,14 +174,15 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? FAPK_OK : FAPK_ERR_CU
 
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
-bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d) {
+bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
   const cuuint32_t box[3] = {64, 1, 128};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  return enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -200,7 +210,7 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
   int rc = validate_problem(P);
   if (rc != FAPK_OK) return rc;
   if (P->T == 0) return FAPK_OK;
-  if (!q || !k || !v || !o || !lse || !ws) return FAPK_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !ctx || !ws) return FAPK_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(ctx) || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
     return FAPK_ERR_INVALID_ARG;
@@ -213,7 +223,9 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
   auto* status = static_cast<DeviceStatus*>(ws);
   FwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
-  a.o_resid = ctx ? static_cast<char*>(ctx) + ctx_layout(P).o_resid : nullptr;
+  const CtxLayout CL = ctx_layout(P);
+  a.o_resid = static_cast<char*>(ctx) + CL.o_resid;
+  a.v16 = static_cast<char*>(ctx) + CL.v16;
   a.cu = P->cu_seqlens_dev;
   a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.d = P->d;
   a.scale = P->scale;
@@ -224,6 +236,8 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
   a.num_sms = sms;
   rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRows, kSchedQ, a.sched, status, true, st));
   if (rc != FAPK_OK) return rc;
+  rc = cuda_status(launch_convert_f16(v, a.v16, (long long)P->T * P->Hkv * P->d, status, sms, st));
+  if (rc != FAPK_OK) return rc;
   return cuda_status(launch_fwd_bf16(a, st));
 }
 
@@ -233,7 +247,7 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   int rc = validate_problem(P);
   if (rc != FAPK_OK) return rc;
   if (P->T == 0) return FAPK_OK;
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !ws) return FAPK_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !dout || !ctx || !dq || !dk || !dv || !ws) return FAPK_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(ctx) ||
       (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
@@ -247,7 +261,12 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   auto* status = static_cast<DeviceStatus*>(ws);
   BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
-  a.o_resid = ctx ? static_cast<const char*>(ctx) + ctx_layout(P).o_resid : nullptr;
+  const CtxLayout CL = ctx_layout(P);
+  a.o_resid = static_cast<const char*>(ctx) + CL.o_resid;
+  a.v16 = static_cast<const char*>(ctx) + CL.v16;
+  a.q16 = static_cast<char*>(ws) + L.q16;
+  a.k16 = static_cast<char*>(ws) + L.k16;
+  a.do16 = static_cast<char*>(ws) + L.do16;
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.delta = reinterpret_cast<float*>(static_cast<char*>(ws) + L.delta);
   a.cu = P->cu_seqlens_dev;
@@ -263,6 +282,8 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedKV, a.sched_kv, status, true, st));
   if (rc != FAPK_OK) return rc;
   rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedQ, a.sched_q, status, false, st));
+  if (rc != FAPK_OK) return rc;
+  rc = cuda_status(launch_convert_f16(k, a.k16, (long long)P->T * P->Hkv * P->d, status, sms, st));
   if (rc != FAPK_OK) return rc;
   return cuda_status(launch_bwd_bf16(a, st));
 }
@@ -307,6 +328,7 @@ const char* fapk_strerror(int status) {
     case FAPK_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case FAPK_ERR_CUDA: return "CUDA runtime error";
     case FAPK_ERR_DEVICE_TIMEOUT: return "device watchdog timeout in a pipeline wait";
+    case FAPK_ERR_RANGE: return "a value reached 65504, the fp16 range of the P/dS operand path";
     default: return "unknown status";
   }
 }

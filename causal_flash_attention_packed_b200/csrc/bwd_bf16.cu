@@ -21,6 +21,10 @@
 // Warp roles as in the forward: warp 8 loads (TMA), warp 9 issues tcgen05
 // MMAs, warps 0-7 compute P and dS (warpgroup 0 on columns 0-63, warpgroup 1
 // on columns 64-127 of each 128x128 tile, every thread owning one TMEM lane).
+// Every MMA of the backward runs on fp16 operands: the prepass copies Q, K, dO
+// to fp16 (V comes from the forward's ctx), which is lossless for bf16 values
+// below 65504, and P and dS are packed to fp16 (11 significant bits, where
+// bf16 keeps 8).  |dS| reaching 65504 is reported as kStatusRange.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -83,21 +87,41 @@ __device__ __forceinline__ uint32_t split_a_col(uint32_t base, int kk) {
 // ---------------------------------------------------------------------------
 // 1. D = rowsum(dO * O), fp32 [Hq][T]
 // ---------------------------------------------------------------------------
-// O is taken as o + o_resid when the forward saved its rounding residual
-// (about 16 significant bits), else as the bf16 o alone.
+// O is taken as o + o_resid, the forward's bf16 output plus its rounding
+// residual (about 16 significant bits).
+// The same pass writes the fp16 copies of dO and Q used by the gradient MMAs.
 template <int D>
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o,
                                                     const __nv_bfloat16* __restrict__ o_resid,
                                                     const __nv_bfloat16* __restrict__ dout,
-                                                    float* __restrict__ delta, int T, int Hq) {
+                                                    const __nv_bfloat16* __restrict__ q,
+                                                    uint4* __restrict__ do16, uint4* __restrict__ q16,
+                                                    float* __restrict__ delta, int T, int Hq,
+                                                    DeviceStatus* status) {
   constexpr int TPR = D / 8;  // threads per (token, head) row
   const long long row = (long long)blockIdx.x * (256 / TPR) + threadIdx.x / TPR;
   const int c8 = threadIdx.x % TPR;
   float acc = 0.f;
+  bool in_range = true;
   if (row < (long long)T * Hq) {
     const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + row * D) + c8);
     const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + c8);
-    const uint4 r = o_resid ? __ldg(reinterpret_cast<const uint4*>(o_resid + row * D) + c8) : make_uint4(0, 0, 0, 0);
+    const uint4 qq = __ldg(reinterpret_cast<const uint4*>(q + row * D) + c8);
+    {
+      const uint32_t wb[4] = {b.x, b.y, b.z, b.w}, wq[4] = {qq.x, qq.y, qq.z, qq.w};
+      uint32_t hb[4], hq[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float b0 = __uint_as_float(wb[i] << 16), b1 = __uint_as_float(wb[i] & 0xFFFF0000u);
+        const float q0 = __uint_as_float(wq[i] << 16), q1 = __uint_as_float(wq[i] & 0xFFFF0000u);
+        in_range &= fmaxf(fmaxf(fabsf(b0), fabsf(b1)), fmaxf(fabsf(q0), fabsf(q1))) < kF16Max;
+        hb[i] = pack_f16x2(b0, b1);
+        hq[i] = pack_f16x2(q0, q1);
+      }
+      do16[row * (D / 8) + c8] = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+      q16[row * (D / 8) + c8] = make_uint4(hq[0], hq[1], hq[2], hq[3]);
+    }
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(o_resid + row * D) + c8);
     const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w}, wr[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -112,6 +136,7 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
     const long long t = row / Hq, h = row % Hq;
     delta[h * T + t] = acc;
   }
+  if (!__all_sync(0xFFFFFFFFu, in_range) && (threadIdx.x & 31) == 0) record_error(status, kStatusRange, 41);
 }
 
 struct BwdParams {
@@ -285,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);  // K-major x K-major
-      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);     // TMEM A x MN-major B
+      constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);  // K-major x K-major
+      constexpr uint32_t idesc_g = idesc_f16_f32(128, D, false, true);     // TMEM A x MN-major B
       const uint32_t sk = smem_u32(sK), sv = smem_u32(sV), sst = smem_u32(sStage);
       uint32_t st_it = 0, p_cnt = 0;
       int unit_i = 0;
@@ -361,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // visible iff j <= i < e; only the diagonal and the last query tile need the test
           const bool full = (m > it.v) && (it.s + 128 * m + 128 <= it.e);
           uint32_t pk[32], dk[32];
+          float dmax = 0.f;
 #pragma unroll
           for (int c = 0; c < 64; c += 2) {
             float pv[2], dv[2];
@@ -375,10 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               pv[u] = pp;
               dv[u] = pp * (__uint_as_float(dr[cc]) - dl[64 * wg + cc]);
+              dmax = fmaxf(dmax, fabsf(dv[u]));
             }
-            pk[c / 2] = pack_bf16x2(pv[0], pv[1]);
-            dk[c / 2] = pack_bf16x2(dv[0], dv[1]);
+            pk[c / 2] = pack_f16x2(pv[0], pv[1]);
+            dk[c / 2] = pack_f16x2(dv[0], dv[1]);
           }
+          if (!(dmax < kF16Max)) record_error(p.status, kStatusRange, 42);
           tmem_st32(s_addr, pk);    // P^T  -> columns [64 wg, 64 wg + 32) of S^T
           tmem_st32(dp_addr, dk);   // dS^T -> columns [64 wg, 64 wg + 32) of dP^T
           tmem_wait_st();
@@ -526,8 +554,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_g = idesc_f16_f32(128, D, false, true);
       const uint32_t sq = smem_u32(sQ), sdo = smem_u32(sDO), sst = smem_u32(sStage);
       uint32_t st_it = 0, p_cnt = 0;
       int unit_i = 0;
@@ -579,8 +607,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const QItem it = q_decode(p, w);
       const int i = it.q0 + row;
       const bool valid = i < it.e;
-      const float l2 = (i < p.T) ? p.lse[(size_t)it.h * p.T + i] * kLog2e : 0.f;
-      const float dl = (i < p.T) ? p.delta[(size_t)it.h * p.T + i] : 0.f;
+      // rows past the document end (the tail of the last tile) get P = 0
+      const float l2 = valid ? p.lse[(size_t)it.h * p.T + i] * kLog2e : INFINITY;
+      const float dl = valid ? p.delta[(size_t)it.h * p.T + i] : 0.f;
       for (int v = 0; v <= it.m; ++v) {
         if (!warp_wait(s_full, s_cnt & 1, wd, 37)) { ok = false; break; }
         ++s_cnt;
@@ -591,6 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j0 = it.s + 128 * v + 64 * wg;  // key index of column 0 of this half
         const bool diag = v == it.m;
         uint32_t dk[32];
+        float dmax = 0.f;
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           float dv[2];
@@ -600,9 +630,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             float pp = fast_exp2(__uint_as_float(sr[cc]) * p.scale_log2 - l2);
             if (diag && j0 + cc > i) pp = 0.f;
             dv[u] = pp * (__uint_as_float(dr[cc]) - dl);
+            dmax = fmaxf(dmax, fabsf(dv[u]));
           }
-          dk[c / 2] = pack_bf16x2(dv[0], dv[1]);
+          dk[c / 2] = pack_f16x2(dv[0], dv[1]);
         }
+        if (!(dmax < kF16Max)) record_error(p.status, kStatusRange, 43);
         tmem_st32(s_addr, dk);  // dS -> columns [64 wg, 64 wg + 32) of S
         tmem_wait_st();
         tc_fence_before();
@@ -634,17 +666,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_tmap_thd(&tq, a.q, a.T, a.Hq, D) || !make_tmap_thd(&tk, a.k, a.T, a.Hkv, D) ||
-      !make_tmap_thd(&tv, a.v, a.T, a.Hkv, D) || !make_tmap_thd(&tdo, a.dout, a.T, a.Hq, D))
+  if (!make_tmap_thd(&tq, a.q16, a.T, a.Hq, D, true) || !make_tmap_thd(&tk, a.k16, a.T, a.Hkv, D, true) ||
+      !make_tmap_thd(&tv, a.v16, a.T, a.Hkv, D, true) || !make_tmap_thd(&tdo, a.do16, a.T, a.Hq, D, true))
     return cudaErrorInvalidValue;
   // 1. D
   {
     constexpr int rows_per_block = 256 / (D / 8);
     const long long rows = (long long)a.T * a.Hq;
     const unsigned grid = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
-    delta_kernel<D><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.o),
-                                               static_cast<const __nv_bfloat16*>(a.o_resid),
-                                               static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.T, a.Hq);
+    delta_kernel<D><<<grid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.o_resid),
+        static_cast<const __nv_bfloat16*>(a.dout), static_cast<const __nv_bfloat16*>(a.q),
+        static_cast<uint4*>(a.do16), static_cast<uint4*>(a.q16), a.delta, a.T, a.Hq, a.status);
     note_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -14,10 +14,12 @@
 //    query row (rows past the document end are computed and discarded);
 //  * warp 8 (one lane): TMA loads of Q0/Q1 once per item and of K_j, V_j
 //    into a ring of shared-memory slots (128-byte swizzle);
-//  * warp 9 (one lane): tcgen05 MMAs.  S_i = Q_i K_j^T (both operands
-//    K-major in shared memory) into TMEM; O_i += P_i V_j with P_i read from
-//    TMEM (it overwrites S_i in place as packed bf16) and V_j MN-major in
-//    shared memory;
+//  * warp 9 (one lane): tcgen05 MMAs.  S_i = Q_i K_j^T (bf16, both operands
+//    K-major in shared memory) into TMEM; O_i += P_i V_j in fp16 with P_i read
+//    from TMEM (it overwrites S_i in place as packed fp16) and V_j MN-major in
+//    shared memory (the fp16 copy of V made by the prepass).  fp16 keeps 11
+//    significant bits of P where bf16 keeps 8; the backward's D = dO . O
+//    inherits this accuracy;
 //  * warps 0-3 / 4-7: softmax of query tile 0 / 1, one thread per query row
 //    (one TMEM lane).  The running maximum is kept in log2 units and only
 //    moved when it grows by more than 8 (P <= 2^8 in between), so the O
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idesc_pv = idesc_f16_f32(128, D, false, true);
       const uint32_t sq_addr = smem_u32(sQ), skv_addr = smem_u32(sKV);
       uint32_t kv_it = 0, p_cnt[2] = {0, 0}, o_used[2] = {0, 0};
       int unit_i = 0;
@@ -342,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 64; ++c) {
           const float a = fast_exp2(x[2 * c] - m), b = fast_exp2(x[2 * c + 1] - m);
           rs += a + b;
-          pk[c] = pack_bf16x2(a, b);
+          pk[c] = pack_f16x2(a, b);
         }
         l += rs;
         tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
@@ -411,7 +413,7 @@ cudaError_t launch_d(const FwdArgs& a, cudaStream_t stream) {
   using C = Cfg<D>;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_thd(&tq, a.q, a.T, a.Hq, D) || !make_tmap_thd(&tk, a.k, a.T, a.Hkv, D) ||
-      !make_tmap_thd(&tv, a.v, a.T, a.Hkv, D))
+      !make_tmap_thd(&tv, a.v16, a.T, a.Hkv, D, true))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;

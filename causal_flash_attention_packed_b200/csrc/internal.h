@@ -43,7 +43,8 @@ struct FwdArgs {
   const void* v;
   void* o;
   float* lse;
-  void* o_resid;  // optional bf16 [T][Hq][d]: O_fp32 - bf16(O_fp32), for the backward's D
+  void* o_resid;  // bf16 [T][Hq][d]: O_fp32 - bf16(O_fp32), for the backward's D
+  void* v16;      // fp16 copy of V [T][Hkv][d] (the PV operand), kept for the backward
   const int32_t* cu;
   int T, Hq, Hkv, d;
   float scale;
@@ -63,7 +64,11 @@ struct BwdArgs {
   const void* o;
   const float* lse;
   const void* dout;
-  const void* o_resid;  // optional residual of O written by the forward (NULL: D from bf16 O)
+  const void* o_resid;  // residual of O written by the forward
+  const void* v16;      // fp16 V written by the forward
+  void* q16;            // fp16 copies made by the backward's prepass ([T][Hq][d], [T][Hkv][d], [T][Hq][d])
+  void* k16;
+  void* do16;
   void* dq;
   void* dk;
   void* dv;
@@ -81,9 +86,15 @@ struct BwdArgs {
 };
 cudaError_t launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream);
 
-// Tensor map of a bf16 [T][H][d] tensor as a 3-D (d, H, T) view with a box of
-// 64 channels x 1 head x 128 tokens and 128-byte swizzle (api.cu).
-bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d);
+// Tensor map of a 16-bit [T][H][d] tensor (bf16, or fp16 when `f16`) as a 3-D
+// (d, H, T) view with a box of 64 channels x 1 head x 128 tokens and 128-byte
+// swizzle (api.cu).
+bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16 = false);
+
+// bf16 -> fp16 copy of n elements (n a multiple of 8); magnitudes >= 65504
+// record kStatusRange (convert.cu).
+cudaError_t launch_convert_f16(const void* src, void* dst, long long n, DeviceStatus* status, int num_sms,
+                               cudaStream_t stream);
 
 // Count of kernels launched by this library (api.cu).
 void note_launches(int n);

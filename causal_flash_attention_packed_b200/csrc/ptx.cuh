@@ -13,7 +13,7 @@ namespace fapk {
 // ---------------------------------------------------------------------------
 // Status word in the workspace (device errors) and the CTA abort flag.
 // ---------------------------------------------------------------------------
-enum : int { kStatusOk = 0, kStatusBadSeqlens = 3, kStatusTimeout = 6 };
+enum : int { kStatusOk = 0, kStatusBadSeqlens = 3, kStatusTimeout = 6, kStatusRange = 7 };
 
 struct DeviceStatus {
   int code;       // first error recorded (0 = none)
@@ -177,6 +177,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Same with fp16 A and B (format 0 in both fields).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand tile.
 // [0,14) start address >> 4, [16,30) leading-dimension byte offset >> 4,
 // [32,46) stride-dimension byte offset >> 4, [46,48) version 1 (sm_100),
@@ -255,5 +261,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+
+// Two fp32 -> packed fp16x2 (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Largest finite fp16 magnitude: values at or above it cannot be converted.
+constexpr float kF16Max = 65504.0f;
 
 }  // namespace fapk

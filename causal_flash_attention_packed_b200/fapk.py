@@ -28,6 +28,7 @@ ERR_BAD_SEQLENS = 3
 ERR_WORKSPACE_TOO_SMALL = 4
 ERR_CUDA = 5
 ERR_DEVICE_TIMEOUT = 6
+ERR_RANGE = 7
 
 BF16 = 0
 MXFP8 = 1

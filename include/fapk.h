@@ -72,7 +72,10 @@ typedef enum {
                                        longer than max_seqlen */
   FAPK_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below fapk_workspace_size() */
   FAPK_ERR_CUDA = 5,                /* a CUDA runtime call failed (launch, no device) */
-  FAPK_ERR_DEVICE_TIMEOUT = 6       /* a bounded device-side wait gave up */
+  FAPK_ERR_DEVICE_TIMEOUT = 6,      /* a bounded device-side wait gave up */
+  FAPK_ERR_RANGE = 7                /* an input or a computed gradient operand reached
+                                       65504, the fp16 range of the bf16 path's
+                                       P/dS operands (see fapk_attn_fwd) */
 } fapk_status_t;
 
 /* Operand precision of the attention path. */
@@ -136,16 +139,21 @@ FAPK_API size_t fapk_workspace_size(const fapk_problem_t* prob, int which);
 FAPK_API size_t fapk_ctx_size(const fapk_problem_t* prob);
 
 /* Forward.  Reads q, k, v (bf16); writes o (bf16) and lse (fp32, natural
- * log).  ctx: device buffer of fapk_ctx_size() bytes, 16-byte aligned, filled
- * for the backward; it may be NULL for FAPK_BF16 (the backward then takes D
- * from the bf16 o alone, which loses accuracy where dS cancels).
- * ws: workspace of at least fapk_workspace_size(prob, FAPK_FWD) bytes. */
+ * log).  ctx (required): device buffer of fapk_ctx_size() bytes, 16-byte
+ * aligned, filled for the backward.  ws: workspace of at least
+ * fapk_workspace_size(prob, FAPK_FWD) bytes.
+ * FAPK_BF16 numerics: S = Q K^T on bf16 operands with fp32 accumulation; the
+ * probabilities P (computed in fp32) multiply V as fp16 operands, which keep
+ * 11 significant bits where bf16 keeps 8 (a bf16 value converts to fp16
+ * exactly when its magnitude is below 65504).  Inputs reaching 65504 in
+ * magnitude are reported as FAPK_ERR_RANGE by fapk_status. */
 FAPK_API int fapk_attn_fwd(const fapk_problem_t* prob, const void* q, const void* k, const void* v,
                   void* o, float* lse, void* ctx, void* ws, size_t ws_bytes, void* stream);
 
 /* Backward.  Reads q, k, v, o, lse, dout (bf16 except lse) and the ctx
- * written by the matching forward (NULL allowed for FAPK_BF16, see
- * fapk_attn_fwd); writes dq [T][Hq][d] and
+ * written by the matching forward (required); every MMA of the FAPK_BF16
+ * backward runs on fp16 operands (P and dS with 11 significant bits), and a
+ * |dS| reaching 65504 is reported as FAPK_ERR_RANGE; writes dq [T][Hq][d] and
  * dk, dv [T][Hkv][d] in grad_dtype.  dk and dv are summed over the query
  * heads that share a KV head.  ws: at least fapk_workspace_size(prob,
  * FAPK_BWD) bytes. */

@@ -33,7 +33,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_strerror_and_version(L):
-    for code in range(7):
+    for code in range(8):
         assert fapk.strerror(code)
     assert "unknown" in fapk.strerror(99)
     assert L.fapk_version() >= 100
@@ -61,13 +61,15 @@ def test_workspace_size(L):
     fwd = fapk.workspace_size(P, fapk.FWD)
     bwd = fapk.workspace_size(P, fapk.BWD)
     assert fwd > 0 and bwd >= 4 * 300 * 4  # bwd holds D = rowsum(dO*O) in fp32 [Hq][T]
+    # ctx: O residual (bf16, T*Hq*d) + fp16 V (T*Hkv*d)
+    assert fapk.ctx_size(P) >= 2 * 300 * 128 * (4 + 2)
     assert fwd % 256 == 0 and bwd % 256 == 0
     assert fapk.workspace_size(_problem(d=96), fapk.FWD) == 0
     assert fapk.workspace_size(P, 7) == 0
 
 
-def _fwd(L, P, ws_bytes=1 << 20, ptrs=(16, 16, 16, 16, 16), ws=256):
-    return L.fapk_attn_fwd(ctypes.byref(P), *ptrs, None, ws, ws_bytes, None)
+def _fwd(L, P, ws_bytes=1 << 30, ptrs=(16, 16, 16, 16, 16), ws=256, ctx=4096):
+    return L.fapk_attn_fwd(ctypes.byref(P), *ptrs, ctx, ws, ws_bytes, None)
 
 
 def test_host_validation_codes(L):
@@ -82,6 +84,8 @@ def test_host_validation_codes(L):
     assert _fwd(L, _problem(), ptrs=(16, None, 16, 16, 16)) == fapk.ERR_INVALID_ARG
     assert _fwd(L, _problem(), ptrs=(16, 24, 16, 16, 16)) == fapk.ERR_INVALID_ARG  # misaligned
     assert _fwd(L, _problem(), ws=512 + 8) == fapk.ERR_INVALID_ARG                  # ws alignment
+    assert _fwd(L, _problem(), ctx=None) == fapk.ERR_INVALID_ARG                    # ctx is required
+    assert _fwd(L, _problem(), ctx=4096 + 8) == fapk.ERR_INVALID_ARG                # ctx alignment
     assert _fwd(L, _problem(), ws_bytes=16) == fapk.ERR_WORKSPACE_TOO_SMALL
     assert _fwd(L, _problem(scale=float("nan"))) == fapk.ERR_INVALID_ARG
     # T = 0 is a no-op
