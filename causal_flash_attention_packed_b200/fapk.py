@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
     L.fapk_attn_fwd.restype = i
     L.fapk_attn_bwd.argtypes = [PP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.fapk_attn_bwd.restype = i
+    L.fapk_attn_fwd_noalloc.argtypes = [PP, vp, vp, vp, vp, vp, vp, vp]
+    L.fapk_attn_fwd_noalloc.restype = i
     L.fapk_quantize_mxfp8.argtypes = [vp, i, i, i, vp, vp, i, i, i, vp, vp, vp, vp, vp]
     L.fapk_quantize_mxfp8.restype = i
     L.fapk_status.argtypes = [vp, vp]
@@ -191,6 +193,16 @@ def attn_fwd(P: Problem, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     rc = lib().fapk_attn_fwd(ctypes.byref(P), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                              _ptr(ctx), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "fapk_attn_fwd")
+    return o, lse, ctx
+
+
+def attn_fwd_noalloc(P: Problem, q, k, v, o, lse, ctx, stream=None):
+    """fapk_attn_fwd_noalloc: the forward with the library's fixed scratch array
+    instead of a workspace, for callers that cannot allocate device memory.  The
+    caller passes every buffer (o, lse, ctx)."""
+    rc = lib().fapk_attn_fwd_noalloc(ctypes.byref(P), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                     _ptr(ctx), _stream(stream))
+    _check(rc, "fapk_attn_fwd_noalloc")
     return o, lse, ctx
 
 

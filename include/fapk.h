@@ -180,6 +180,27 @@ FAPK_API int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const 
                         uint8_t* val_tb, uint8_t* scale_tb, uint8_t* val_pt, uint8_t* scale_pt,
                         void* stream);
 
+/* Forward that allocates nothing.  The pages have no counterpart: this entry
+ * point exists for callers that cannot obtain device memory where they run the
+ * forward -- a plugin handed its buffers by a host framework that must not
+ * allocate on its own, code inside a host callback, or a runtime that reserves
+ * all device memory at start-up.  Same arguments and results as
+ * fapk_attn_fwd minus the workspace: inputs, outputs and ctx are still the
+ * caller's, and the forward's scratch (status word and work list) is a 1 MiB
+ * array of device memory inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *  - A problem whose forward workspace (fapk_workspace_size(prob, FAPK_FWD))
+ *    exceeds 1 MiB is rejected with FAPK_ERR_WORKSPACE_TOO_SMALL; at T = 32768
+ *    tokens that size is about 1 KiB plus 8 bytes per document.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current; make that first call before any stream capture.
+ *  - All calls share the array and it keeps the last call's contents; each
+ *    call clears the status word and counters it uses when it starts.  Calls
+ *    whose GPU work overlaps (different streams or host threads) race on it.
+ *  - The device status word of these calls is not readable by the caller. */
+FAPK_API int fapk_attn_fwd_noalloc(const fapk_problem_t* prob, const void* q, const void* k,
+                                   const void* v, void* o, float* lse, void* ctx, void* stream);
+
 /* Synchronises `stream`, then returns the device status word of the last call
  * that used workspace `ws` (FAPK_OK, FAPK_ERR_DEVICE_TIMEOUT, or
  * FAPK_ERR_BAD_SEQLENS), or FAPK_ERR_CUDA if the stream reported an error. */
