@@ -232,15 +232,11 @@ def main():
     ctx = torch.empty(max(fapk.ctx_size(P), 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        fapk.attn_fwd(P, qd, kd, vd, o=o, lse=lse, ctx=ctx, ws=ws_f, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        fapk.attn_bwd(P, qd, kd, vd, o, lse, dod, ctx=ctx, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
+    def step(timers=None):
+        Pf = timers[0].with_events(P) if timers else P
+        Pb = timers[1].with_events(P) if timers else P
+        fapk.attn_fwd(Pf, qd, kd, vd, o=o, lse=lse, ctx=ctx, ws=ws_f, stream=stream)
+        fapk.attn_bwd(Pb, qd, kd, vd, o, lse, dod, ctx=ctx, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -248,7 +244,8 @@ def main():
     assert fapk.status(ws_f) == 0 and fapk.status(ws_b) == 0
 
     clocks = ClockSampler(local) if rank == 0 else None
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # the library records these events between its own kernel launches
+    timers = [(fapk.KernelTimer(4), fapk.KernelTimer(7)) for _ in range(args.steps)]
     launches0 = fapk.launch_count()
     barrier(world)
     torch.cuda.synchronize(dev)
@@ -258,7 +255,7 @@ def main():
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step(timers[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
@@ -266,10 +263,12 @@ def main():
     launches = fapk.launch_count() - launches0
     st_ok = fapk.status(ws_f) == 0 and fapk.status(ws_b) == 0
     total_ms = max_over_ranks(start.elapsed_time(end), world, dev)
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    fwd_ms = max_over_ranks(fwd_ms, world, dev)
-    bwd_ms = max_over_ranks(bwd_ms, world, dev)
+    names = ["schedule_fwd", "convert_v_f16", "fwd_kernel", "schedule_kv", "schedule_q", "convert_k_f16",
+             "delta_kernel", "dkdv_kernel", "dq_kernel"]
+    per = [tf.durations_ms() + tb.durations_ms() for tf, tb in timers]
+    kern_ms = {n: max_over_ranks(statistics.mean(row[i] for row in per), world, dev) for i, n in enumerate(names)}
+    fwd_ms = sum(kern_ms[n] for n in names[:3])
+    bwd_ms = sum(kern_ms[n] for n in names[3:])
     ms_per_step = total_ms / args.steps
     flops = w.flops()
     value = flops * world / (ms_per_step * 1e-3) / 1e12
@@ -308,16 +307,20 @@ def main():
 
     fwd_flops = 4.0 * w.d * w.Hq * w.pairs()
     bwd_flops = 10.0 * w.d * w.Hq * w.pairs()
-    dom_is_bwd = bwd_ms >= fwd_ms
-    dom_ms = bwd_ms if dom_is_bwd else fwd_ms
-    dom_flops = bwd_flops if dom_is_bwd else fwd_flops
-    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    # algorithmic tensor work of each attention kernel (per visible pair and
+    # query head): forward S and PV = 4 d; dK/dV kernel S, dP, dV, dK = 8 d;
+    # dQ kernel S, dP, dQ = 6 d
+    kern_flops = {"fwd_kernel": 4.0, "dkdv_kernel": 8.0, "dq_kernel": 6.0}
+    dom = max(kern_flops, key=lambda n: kern_ms[n])
+    dom_flops = kern_flops[dom] * w.d * w.Hq * w.pairs()
+    achieved = dom_flops / (kern_ms[dom] * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
-                "kernel": "attn_bwd call (delta, dK/dV and dQ kernels)" if dom_is_bwd
-                else "attn_fwd call (forward kernel)",
+                "frac": achieved / peak, "traffic": None, "kernel": dom,
                 "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)",
+                "kernels_ms": kern_ms,
+                "kernels_tflops": {n: kern_flops[n] * w.d * w.Hq * w.pairs() / (kern_ms[n] * 1e-3) / 1e12
+                                   for n in kern_flops},
                 "fwd": {"ms": fwd_ms, "tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12},
                 "bwd": {"ms": bwd_ms, "tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12}}
     cpu = None

@@ -234,11 +234,17 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
   a.timeout_ns = timeout_ns_of(P);
   a.flags = P->flags;
   a.num_sms = sms;
+  const Marks mk{P->timing_events, P->n_timing_events};
+  mk.at(0, st);
   rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRows, kSchedQ, a.sched, status, true, st));
   if (rc != FAPK_OK) return rc;
+  mk.at(1, st);
   rc = cuda_status(launch_convert_f16(v, a.v16, (long long)P->T * P->Hkv * P->d, status, sms, st));
   if (rc != FAPK_OK) return rc;
-  return cuda_status(launch_fwd_bf16(a, st));
+  mk.at(2, st);
+  rc = cuda_status(launch_fwd_bf16(a, st));
+  mk.at(3, st);
+  return rc;
 }
 
 int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const void* v, const void* o,
@@ -279,10 +285,14 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   a.timeout_ns = timeout_ns_of(P);
   a.flags = P->flags;
   a.num_sms = sms;
+  a.marks = Marks{P->timing_events, P->n_timing_events};
+  a.marks.at(0, st);
   rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedKV, a.sched_kv, status, true, st));
   if (rc != FAPK_OK) return rc;
+  a.marks.at(1, st);
   rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedQ, a.sched_q, status, false, st));
   if (rc != FAPK_OK) return rc;
+  a.marks.at(2, st);
   rc = cuda_status(launch_convert_f16(k, a.k16, (long long)P->T * P->Hkv * P->d, status, sms, st));
   if (rc != FAPK_OK) return rc;
   return cuda_status(launch_bwd_bf16(a, st));

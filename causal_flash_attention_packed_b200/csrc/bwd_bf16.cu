@@ -670,6 +670,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
       !make_tmap_thd(&tv, a.v16, a.T, a.Hkv, D, true) || !make_tmap_thd(&tdo, a.do16, a.T, a.Hq, D, true))
     return cudaErrorInvalidValue;
   // 1. D
+  a.marks.at(3, stream);
   {
     constexpr int rows_per_block = 256 / (D / 8);
     const long long rows = (long long)a.T * a.Hq;
@@ -695,6 +696,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
   p.scale_log2 = a.scale * kLog2e;
   p.grad_bf16 = a.grad_bf16;
   // 2. dK, dV
+  a.marks.at(4, stream);
   {
     using C = KvCfg<D>;
     cudaError_t e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -712,6 +714,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   // 3. dQ
+  a.marks.at(5, stream);
   {
     using C = QCfg<D>;
     cudaError_t e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -728,6 +731,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  a.marks.at(6, stream);
   return cudaSuccess;
 }
 

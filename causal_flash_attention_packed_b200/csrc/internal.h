@@ -12,6 +12,15 @@ namespace fapk {
 
 struct DeviceStatus;
 
+// Optional CUDA events recorded between a call's kernel launches (profiling).
+struct Marks {
+  void* const* ev = nullptr;
+  int n = 0;
+  void at(int i, cudaStream_t s) const {
+    if (ev && i < n && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
+  }
+};
+
 // Work-list modes of the scheduler (schedule.cu).  An item is (doc, tile)
 // with tile in [0, ceil(L / rows)); items are ordered by a cost level,
 // highest first, so that persistent CTAs take the longest work first (LPT).
@@ -79,6 +88,7 @@ struct BwdArgs {
   int grad_bf16;
   SchedBuf sched_kv;
   SchedBuf sched_q;
+  Marks marks;  // [3] before D, [4] before dK/dV, [5] before dQ, [6] after
   DeviceStatus* status;
   uint64_t timeout_ns;
   int flags;

@@ -65,6 +65,8 @@ class Problem(ctypes.Structure):
         ("grad_dtype", ctypes.c_int),
         ("flags", ctypes.c_int),
         ("timeout_ms", ctypes.c_int),
+        ("timing_events", ctypes.c_void_p),
+        ("n_timing_events", ctypes.c_int),
     ]
 
 
@@ -158,7 +160,32 @@ def make_problem(seq: Seqlens, Hq: int, Hkv: int, d: int, scale: float, prec: in
     P.grad_dtype = grad_dtype
     P.flags = flags
     P.timeout_ms = timeout_ms
+    P.timing_events = None
+    P.n_timing_events = 0
     return P
+
+
+class KernelTimer:
+    """CUDA events that a call records between its kernel launches
+    (fapk_problem_t.timing_events): ``with_events(P)`` returns a copy of the
+    problem that records into this timer's events; ``durations_ms()`` returns
+    the time between consecutive events."""
+
+    def __init__(self, n: int):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in self.events:  # create the underlying cudaEvent_t
+            e.record()
+        torch.cuda.synchronize()
+        self._handles = (ctypes.c_void_p * n)(*[e.cuda_event for e in self.events])
+
+    def with_events(self, P: Problem) -> Problem:
+        Q = Problem.from_buffer_copy(P)
+        Q.timing_events = ctypes.cast(self._handles, ctypes.c_void_p)
+        Q.n_timing_events = len(self.events)
+        return Q
+
+    def durations_ms(self):
+        return [a.elapsed_time(b) for a, b in zip(self.events[:-1], self.events[1:])]
 
 
 def workspace_size(P: Problem, which: int) -> int:

@@ -122,6 +122,15 @@ typedef struct {
   int grad_dtype;                /* fapk_grad_dtype_t of dq, dk, dv */
   int flags;                     /* debug flags, 0 in normal use */
   int timeout_ms;                /* device watchdog per wait; <= 0 selects 2000 ms */
+  void* const* timing_events;    /* optional profiling hook: cudaEvent_t handles that a call
+                                    records on its stream before each of its kernel launches
+                                    and after the last one (entries beyond n_timing_events or
+                                    NULL are skipped).  fapk_attn_fwd: [0] schedule, [1] fp16
+                                    copy of V, [2] forward kernel, [3] end.  fapk_attn_bwd:
+                                    [0] key-tile schedule, [1] query-tile schedule, [2] fp16
+                                    copy of K, [3] D and fp16 dO/Q, [4] dK/dV kernel, [5] dQ
+                                    kernel, [6] end. */
+  int n_timing_events;
 } fapk_problem_t;
 
 /* Bytes of workspace the forward (which = FAPK_FWD) or backward
