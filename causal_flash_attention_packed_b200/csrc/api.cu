@@ -121,13 +121,16 @@ SchedBuf sched_buf(void* ws, const SchedLayout& s) {
 constexpr int kFwdRows = 256;  // query rows per forward work item (two 128-row tiles)
 constexpr int kBwdRows = 128;  // rows per backward work item
 
+constexpr int kFwdRowsMx = 128;  // query rows per MXFP8 forward work item (one tile)
+
 struct FwdLayout {
   SchedLayout sched;
   size_t total;
 };
 FwdLayout fwd_layout(const fapk_problem_t* P) {
   FwdLayout L;
-  L.sched = sched_layout(kAlign, P->T, P->n_docs, P->max_seqlen, kFwdRows);
+  L.sched = sched_layout(kAlign, P->T, P->n_docs, P->max_seqlen,
+                         P->prec == FAPK_MXFP8 ? kFwdRowsMx : kFwdRows);
   L.total = L.sched.end;
   return L;
 }
@@ -157,14 +160,43 @@ BwdLayout bwd_layout(const fapk_problem_t* P) {
 //           the 8 of the bf16 output;
 //  v16:     fp16 copy of V [T][Hkv][d], the B operand of O += P V (and of the
 //           backward's dP = dO V^T).
+//  MXFP8 path, instead of v16: the quantiser's forms of Q, K and V (codes and
+//  scales, token-block and per-token), reused by the backward in both
+//  orientations, and V's per-token form dequantised to bf16.
+struct MxForms {
+  size_t vtb, stb, vpt, spt;  // offsets of codes / scales
+};
 struct CtxLayout {
   size_t o_resid, v16, total;
+  MxForms q, k, v;
+  size_t v_deq_pt;
 };
 CtxLayout ctx_layout(const fapk_problem_t* P) {
   CtxLayout L;
   L.o_resid = 0;
-  L.v16 = align_up(sizeof(uint16_t) * (size_t)P->T * P->Hq * P->d);
-  L.total = align_up(L.v16 + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
+  size_t off = align_up(sizeof(uint16_t) * (size_t)P->T * P->Hq * P->d);
+  if (P->prec != FAPK_MXFP8) {
+    L.v16 = off;
+    L.total = align_up(L.v16 + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
+    return L;
+  }
+  L.v16 = 0;
+  const size_t slots = (size_t)P->T / 32 + P->n_docs;
+  auto forms = [&](int H) {
+    MxForms f;
+    const size_t n = (size_t)P->T * H * P->d;
+    f.vtb = off;
+    f.stb = align_up(f.vtb + n);
+    f.vpt = align_up(f.stb + slots * H * (P->d / 32));
+    f.spt = align_up(f.vpt + n);
+    off = align_up(f.spt + (size_t)P->T * H * (P->d / 32));
+    return f;
+  };
+  L.q = forms(P->Hq);
+  L.k = forms(P->Hkv);
+  L.v = forms(P->Hkv);
+  L.v_deq_pt = off;
+  L.total = align_up(off + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
   return L;
 }
 
@@ -173,6 +205,18 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? FAPK_OK : FAPK_ERR_CU
 }  // namespace
 
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {128, (cuuint64_t)H * 128};
+  const cuuint32_t box[3] = {128, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16) {
   EncodeTiledFn enc = encode_fn();
@@ -186,6 +230,64 @@ bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
+
+// MXFP8 forward: quantise Q, K, V into ctx (both forms; V also dequantised
+// per token), build the 128-row schedule, run the kernel.
+int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void* v, void* o, float* lse, void* ctx,
+              void* ws, const FwdLayout& L, int sms, cudaStream_t st) {
+  auto* status = static_cast<DeviceStatus*>(ws);
+  const CtxLayout C = ctx_layout(P);
+  char* c = static_cast<char*>(ctx);
+  auto u8 = [&](size_t off) { return reinterpret_cast<uint8_t*>(c + off); };
+  const Marks mk{P->timing_events, P->n_timing_events};
+  FwdMxArgs a;
+  a.sched = sched_buf(ws, L.sched);
+  mk.at(0, st);
+  int rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, kSchedQ, a.sched, status, true, st));
+  if (rc != FAPK_OK) return rc;
+  mk.at(1, st);
+  const int forms = FAPK_FORM_TB | FAPK_FORM_PT;
+  rc = cuda_status(launch_quantize_mxfp8(q, P->T, P->Hq, P->d, P->cu_seqlens_dev, P->n_docs, forms, P->scale_rule,
+                                         u8(C.q.vtb), u8(C.q.stb), u8(C.q.vpt), u8(C.q.spt), st));
+  if (rc != FAPK_OK) return rc;
+  rc = cuda_status(launch_quantize_mxfp8(k, P->T, P->Hkv, P->d, P->cu_seqlens_dev, P->n_docs, forms, P->scale_rule,
+                                         u8(C.k.vtb), u8(C.k.stb), u8(C.k.vpt), u8(C.k.spt), st));
+  if (rc != FAPK_OK) return rc;
+  rc = cuda_status(launch_quantize_mxfp8(v, P->T, P->Hkv, P->d, P->cu_seqlens_dev, P->n_docs, forms, P->scale_rule,
+                                         u8(C.v.vtb), u8(C.v.stb), u8(C.v.vpt), u8(C.v.spt), st,
+                                         c + C.v_deq_pt));
+  if (rc != FAPK_OK) return rc;
+  a.q_vpt = u8(C.q.vpt);
+  a.q_spt = u8(C.q.spt);
+  a.k_vtb = u8(C.k.vtb);
+  a.k_stb = u8(C.k.stb);
+  a.k_vpt = u8(C.k.vpt);
+  a.k_spt = u8(C.k.spt);
+  a.v_vtb = u8(C.v.vtb);
+  a.v_stb = u8(C.v.stb);
+  a.v_deq_pt = c + C.v_deq_pt;
+  a.o = o;
+  a.lse = lse;
+  a.o_resid = c + C.o_resid;
+  a.cu = P->cu_seqlens_dev;
+  a.T = P->T;
+  a.Hq = P->Hq;
+  a.Hkv = P->Hkv;
+  a.n_docs = P->n_docs;
+  a.scale = P->scale;
+  a.rule = P->scale_rule;
+  a.status = status;
+  a.timeout_ns = timeout_ns_of(P);
+  a.num_sms = sms;
+  mk.at(2, st);
+  rc = cuda_status(launch_fwd_mxfp8(a, st));
+  mk.at(3, st);
+  return rc;
+}
+
+}  // namespace
 
 }  // namespace fapk
 
@@ -216,11 +318,12 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
     return FAPK_ERR_INVALID_ARG;
   const FwdLayout L = fwd_layout(P);
   if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
-  if (P->prec != FAPK_BF16) return FAPK_ERR_UNSUPPORTED;
+  if (P->prec == FAPK_MXFP8 && P->d != 128) return FAPK_ERR_UNSUPPORTED;
   const int sms = device_num_sms();
   if (sms <= 0) return FAPK_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto* status = static_cast<DeviceStatus*>(ws);
+  if (P->prec == FAPK_MXFP8) return fwd_mxfp8(P, q, k, v, o, lse, ctx, ws, L, sms, st);
   FwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
   const CtxLayout CL = ctx_layout(P);
@@ -260,7 +363,7 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
     return FAPK_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(P);
   if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
-  if (P->prec != FAPK_BF16) return FAPK_ERR_UNSUPPORTED;
+  if (P->prec != FAPK_BF16) return FAPK_ERR_UNSUPPORTED;  // the MXFP8 backward is not built yet
   const int sms = device_num_sms();
   if (sms <= 0) return FAPK_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

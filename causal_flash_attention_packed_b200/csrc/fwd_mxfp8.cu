@@ -1,0 +1,591 @@
+// Forward of causal packed-document attention, MXFP8 path, for sm_100a
+// (FLAMIA page, sec. "FLAMIA Mimarisi ve Temel Tasarim Ilkeleri": MXFP8
+// operands with shared E8M0 scales, token-block scaling, leak guards,
+// document-local scales; GPT page secs. 3-6 for the attention itself).
+//
+// Operands come from the quantiser (prepass, stored in ctx for the backward):
+// Q per token (one scale per token x 32 channels), K and V in token-block form
+// (one scale per 32 tokens x 32 channels) and per-token form.  Leak guard
+// (rule L): a query of 32-token block b sees keys of earlier blocks through
+// the token-block forms and keys of its own block through the per-token forms,
+// so no shared scale pools a future token.
+//
+// One persistent CTA per SM, 192 threads; work item = (document, 128-row
+// query tile, head).  Warps 0-3: one thread per query row (softmax, P
+// quantisation, epilogue); warp 4: loads (TMA for codes, plain loads for the
+// scale bytes, staged into the 512-byte blocks tcgen05.cp copies to TMEM);
+// warp 5 (one lane): MMAs.
+//  * S = Q K^T for every key tile: block-scaled FP8 MMA (kind::mxf8f6f4,
+//    E8M0 scales in TMEM) with K in token-block form; on the diagonal tile a
+//    second S with K per token, selected on the diagonal 32x32 blocks.
+//  * P: u = 2^(S log2 e - M) with an integer running reference M (moved only
+//    when the row maximum grows by more than 8), quantised per (row, 32-key
+//    block) to E4M3 with an E8M0 scale.  MX quantisation is invariant under
+//    powers of two, so every M yields the same codes as the final one.
+//  * O += P~ V~: block-scaled FP8 MMA with V in token-block form (MN-major);
+//    on the diagonal tile the diagonal 32x32 blocks of P~ are taken out of the
+//    FP8 operand and multiplied exactly with the dequantised per-token V in a
+//    bf16 MMA (per-token V scales vary along the contraction, which an MX
+//    block scale cannot express).
+// TMEM: S buffers [0,128) and [128,256) (the diagonal tile's per-token S uses
+// the buffer the previous tile freed), O [256,384), scale factors from 384.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "mx.cuh"
+#include "ptx.cuh"
+
+namespace fapk {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kLoadWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kSlots = 6;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLn2 = 0.69314718055994530942f;
+
+// shared memory plan (bytes, 1024-aligned tiles)
+constexpr int kCodeTile = 128 * 128;      // 128 rows x 128 fp8 codes
+constexpr int kBf16Tile = 128 * 128 * 2;  // 128 rows x 128 bf16
+constexpr int kBox = 128 * 64 * 2;        // one 64-channel bf16 box
+constexpr int oQ = 0;
+constexpr int oKpt = oQ + kCodeTile;
+constexpr int oVpt = oKpt + kCodeTile;
+constexpr int oP = oVpt + kBf16Tile;
+constexpr int oPd = oP + kCodeTile;
+constexpr int oRing = oPd + kBf16Tile;
+constexpr int oSf = oRing + kSlots * kCodeTile;  // sfQ, sfKpt, sfP, sfRing[kSlots]
+constexpr int kSfBlk = 512;
+constexpr int oBars = oSf + (3 + kSlots) * kSfBlk;
+constexpr int kNumBars = 2 + 2 * kSlots + 8;
+constexpr int kSmemBytes = oBars + kNumBars * 8 + 16 + 1024;
+
+// TMEM columns
+constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256;
+constexpr uint32_t kSfQ = 384, kSfK = 388, kSfKpt = 392, kSfP = 396, kSfV = 400;
+
+struct Params {
+  const int32_t* cu;
+  const int2* list;
+  const int* n_items;
+  const uint8_t* q_spt;   // Q per-token scales [T][Hq][4]
+  const uint8_t* k_stb;   // K token-block scales [slots][Hkv][4]
+  const uint8_t* k_spt;   // K per-token scales [T][Hkv][4]
+  const uint8_t* v_stb;   // V token-block scales [slots][Hkv][4]
+  __nv_bfloat16* o;
+  float* lse;
+  __nv_bfloat16* o_resid;
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+  int T, Hq, Hkv, n_docs;
+  float scale_log2;
+  int rule;
+};
+
+struct Item {
+  int doc, s, e, h, g, q0, n;  // n key tiles 0..n-1, tile n-1 is the diagonal
+};
+
+__device__ __forceinline__ Item decode(const Params& p, int w) {
+  Item it;
+  const int2 pr = p.list[w / p.Hq];
+  it.h = w % p.Hq;
+  it.g = it.h / (p.Hq / p.Hkv);
+  it.doc = pr.x;
+  it.s = p.cu[pr.x];
+  it.e = p.cu[pr.x + 1];
+  it.q0 = it.s + 128 * pr.y;
+  it.n = pr.y + 1;
+  return it;
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > budget_ns) return;
+  }
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd, int where) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
+}
+
+// 4 scale bytes of token t (per-token form), or the neutral byte 127 (2^0)
+// past the end of the tensor.
+__device__ __forceinline__ uint32_t pt_word(const uint8_t* spt, int t, int T, int H, int h) {
+  return t < T ? __ldg(reinterpret_cast<const uint32_t*>(spt + ((size_t)t * H + h) * 4)) : 0x7F7F7F7Fu;
+}
+
+// 4 scale bytes of document-local token block `blk` of document `doc`
+// (token-block form); 127s past the document's last block.
+__device__ __forceinline__ uint32_t tb_word(const uint8_t* stb, int s, int e, int doc, int blk, int H, int g) {
+  if (32 * blk >= e - s) return 0x7F7F7F7Fu;
+  const size_t slot = (size_t)(s >> 5) + doc + blk;
+  return __ldg(reinterpret_cast<const uint32_t*>(stb + (slot * H + g) * 4));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_mxfp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ktb,
+                     const __grid_constant__ CUtensorMap tm_kpt, const __grid_constant__ CUtensorMap tm_vtb,
+                     const __grid_constant__ CUtensorMap tm_vpt16, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + oQ;
+  uint8_t* sKpt = smem + oKpt;
+  uint8_t* sVpt = smem + oVpt;
+  uint8_t* sP = smem + oP;
+  uint8_t* sPd = smem + oPd;
+  uint8_t* sRing = smem + oRing;
+  uint8_t* sfQ = smem + oSf;
+  uint8_t* sfKpt = sfQ + kSfBlk;
+  uint8_t* sfP = sfQ + 2 * kSfBlk;
+  uint8_t* sfRing = sfQ + 3 * kSfBlk;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oBars);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;
+  uint64_t* kv_empty = bars + 2 + kSlots;
+  // one "scores ready" barrier per S buffer: tile j signals s_full[j & 1], so
+  // no barrier ever runs more than one phase ahead of its waiters
+  uint64_t* s_full = bars + 2 + 2 * kSlots;  // [2]
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = s_full + 3;
+  uint64_t* o_full = s_full + 4;
+  uint64_t* o_free = s_full + 5;
+  uint64_t* fin = s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 32);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(kv_full + i, 32);
+      mbar_init(kv_empty + i, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_full + 1, 1);
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(o_full, 1);
+    mbar_init(o_free, 128);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{p.status, abort_flag, p.timeout_ns};
+  const int n_units = (*p.n_items) * p.Hq;
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ loads
+    uint32_t kv_it = 0;
+    int unit_i = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      const Item it = decode(p, w);
+      if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 51)) break;
+      {
+        // scale blocks: row r = lane + 32 r1 -> bytes 16 lane + 4 r1 .. +3
+        uint4 wq, wk;
+        wq.x = pt_word(p.q_spt, it.q0 + lane, p.T, p.Hq, it.h);
+        wq.y = pt_word(p.q_spt, it.q0 + lane + 32, p.T, p.Hq, it.h);
+        wq.z = pt_word(p.q_spt, it.q0 + lane + 64, p.T, p.Hq, it.h);
+        wq.w = pt_word(p.q_spt, it.q0 + lane + 96, p.T, p.Hq, it.h);
+        wk.x = pt_word(p.k_spt, it.q0 + lane, p.T, p.Hkv, it.g);
+        wk.y = pt_word(p.k_spt, it.q0 + lane + 32, p.T, p.Hkv, it.g);
+        wk.z = pt_word(p.k_spt, it.q0 + lane + 64, p.T, p.Hkv, it.g);
+        wk.w = pt_word(p.k_spt, it.q0 + lane + 96, p.T, p.Hkv, it.g);
+        reinterpret_cast<uint4*>(sfQ)[lane] = wq;
+        reinterpret_cast<uint4*>(sfKpt)[lane] = wk;
+        fence_proxy_async_smem();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full, 2 * kCodeTile + kBf16Tile);
+          tma_load_3d(sQ, &tm_q, q_full, 0, it.h, it.q0);
+          tma_load_3d(sKpt, &tm_kpt, q_full, 0, it.g, it.q0);  // the diagonal key tile starts at q0
+          tma_load_3d(sVpt, &tm_vpt16, q_full, 0, it.g, it.q0);
+          tma_load_3d(sVpt + kBox, &tm_vpt16, q_full, 64, it.g, it.q0);
+        } else {
+          mbar_arrive(q_full);
+        }
+      }
+      for (int j = 0; j < it.n && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv, ++kv_it) {
+          const int slot = kv_it % kSlots;
+          const uint32_t use = kv_it / kSlots;
+          if (use > 0 && !warp_wait(kv_empty + slot, (use - 1) & 1, wd, 52)) { ok = false; break; }
+          uint4 wsf;
+          if (kv == 0) {
+            // K rows = keys: the scale word of the key's token block
+            wsf.x = tb_word(p.k_stb, it.s, it.e, it.doc, 4 * j + 0, p.Hkv, it.g);
+            wsf.y = tb_word(p.k_stb, it.s, it.e, it.doc, 4 * j + 1, p.Hkv, it.g);
+            wsf.z = tb_word(p.k_stb, it.s, it.e, it.doc, 4 * j + 2, p.Hkv, it.g);
+            wsf.w = tb_word(p.k_stb, it.s, it.e, it.doc, 4 * j + 3, p.Hkv, it.g);
+          } else {
+            // V as B of P V: rows = channels c = lane + 32 r1 (group r1), K
+            // blocks = the tile's 4 key blocks; byte kb of word r1 is the
+            // token-block scale of (key block 4j + kb, channel group r1)
+            uint32_t wv[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              const uint32_t t = tb_word(p.v_stb, it.s, it.e, it.doc, 4 * j + kb, p.Hkv, it.g);
+#pragma unroll
+              for (int r1 = 0; r1 < 4; ++r1) wv[r1] |= ((t >> (8 * r1)) & 0xFFu) << (8 * kb);
+            }
+            wsf = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+          reinterpret_cast<uint4*>(sfRing + slot * kSfBlk)[lane] = wsf;
+          fence_proxy_async_smem();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(kv_full + slot, kCodeTile);
+            tma_load_3d(sRing + slot * kCodeTile, kv ? &tm_vtb : &tm_ktb, kv_full + slot, 0, it.g, it.s + 128 * j);
+          } else {
+            mbar_arrive(kv_full + slot);
+          }
+        }
+      }
+    }
+    if (lane == 0) {
+      if (unit_i > 0) drain_wait(q_full, (unit_i - 1) & 1, p.timeout_ns);
+      for (uint32_t i = (kv_it > kSlots ? kv_it - kSlots : 0); i < kv_it; ++i)
+        drain_wait(kv_full + (i % kSlots), (i / kSlots) & 1, p.timeout_ns);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      const uint32_t aq = smem_u32(sQ), akpt = smem_u32(sKpt), avpt = smem_u32(sVpt), ap = smem_u32(sP),
+                     apd = smem_u32(sPd), aring = smem_u32(sRing), asf = smem_u32(sfQ);
+      uint32_t kv_it = 0, p_cnt = 0, o_used = 0;
+      int unit_i = 0;
+      bool ok = true;
+      auto kslot_of = [&](int j) { return (int)((kv_it + 2 * j) % kSlots); };
+      auto vslot_of = [&](int j) { return (int)((kv_it + 2 * j + 1) % kSlots); };
+      auto wait_slot = [&](int j, int kv) {
+        const uint32_t idx = kv_it + 2 * j + kv;
+        return mbar_wait(kv_full + (idx % kSlots), (idx / kSlots) & 1, wd, 53);
+      };
+      // S (into buffer col) = Q K^T with K codes at `kaddr` and its scales at TMEM column sfb
+      auto issue_s = [&](uint32_t col, uint32_t kaddr, uint32_t sfb) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_mxf8_ss(tmem + col, sdesc_sw128(aq + kk * 32, 16, 1024), sdesc_sw128(kaddr + kk * 32, 16, 1024),
+                      idesc_mxf8(128, 128, false, kk, kk), (tmem + kSfQ) | ((uint32_t)kk << 30),
+                      (tmem + sfb) | ((uint32_t)kk << 30), kk > 0);
+      };
+      auto issue_s_tile = [&](int j, uint32_t col) {
+        const int ks = kslot_of(j);
+        tmem_cp_sf(tmem + kSfK, asf + (3 + ks) * kSfBlk);
+        issue_s(col, aring + ks * kCodeTile, kSfK);
+      };
+      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+        const Item it = decode(p, w);
+        const int n = it.n;
+        if (!mbar_wait(q_full, unit_i & 1, wd, 54)) break;
+        tc_fence_after();
+        tmem_cp_sf(tmem + kSfQ, asf);
+        tmem_cp_sf(tmem + kSfKpt, asf + kSfBlk);
+        // prologue: S(0) (+ per-token S if tile 0 is the diagonal), S(1)
+        if (!wait_slot(0, 0)) break;
+        tc_fence_after();
+        issue_s_tile(0, kS0);
+        if (n == 1) issue_s(kS1, akpt, kSfKpt);
+        tc_commit(s_full + 0);
+        tc_commit(kv_empty + kslot_of(0));
+        if (n >= 2) {
+          if (!wait_slot(1, 0)) break;
+          tc_fence_after();
+          issue_s_tile(1, kS1);
+          if (n > 2) tc_commit(s_full + 1);  // the diagonal tile commits after its per-token S
+          tc_commit(kv_empty + kslot_of(1));
+        }
+        for (int j = 0; j < n; ++j) {
+          if (!mbar_wait(p_full, p_cnt & 1, wd, 55)) { ok = false; break; }
+          ++p_cnt;
+          if (!wait_slot(j, 1)) { ok = false; break; }
+          if (j == 0 && o_used > 0 && !mbar_wait(o_free, (o_used - 1) & 1, wd, 56)) { ok = false; break; }
+          tc_fence_after();
+          const int vs = vslot_of(j);
+          tmem_cp_sf(tmem + kSfP, asf + 2 * kSfBlk);
+          tmem_cp_sf(tmem + kSfV, asf + (3 + vs) * kSfBlk);
+          const uint32_t av = aring + vs * kCodeTile;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_mxf8_ss(tmem + kO, sdesc_sw128(ap + kk * 32, 16, 1024), sdesc_sw128(av + kk * 4096, 16384, 1024),
+                        idesc_mxf8(128, 128, true, kk, kk), (tmem + kSfP) | ((uint32_t)kk << 30),
+                        (tmem + kSfV) | ((uint32_t)kk << 30), (j > 0 || kk > 0) ? 1u : 0u);
+          if (j == n - 1) {
+            // diagonal 32x32 blocks: exact bf16 P~ times dequantised per-token V
+            constexpr uint32_t idesc_d = idesc_bf16_f32(128, 128, false, true);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_f16_ss(tmem + kO, sdesc_sw128(apd + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024),
+                         sdesc_sw128(avpt + kk * 2048, kBox, 1024), idesc_d, 1u);
+          }
+          tc_commit(pv_done);
+          tc_commit(kv_empty + vs);
+          if (j == n - 1) {
+            tc_commit(o_full);
+            ++o_used;
+          }
+          if (j + 2 < n) {
+            if (!wait_slot(j + 2, 0)) { ok = false; break; }
+            tc_fence_after();
+            issue_s_tile(j + 2, (j & 1) ? kS1 : kS0);
+            if (j + 2 < n - 1) tc_commit(s_full + (j & 1));
+            tc_commit(kv_empty + kslot_of(j + 2));
+          }
+          if (j == n - 2) {
+            // per-token S of the diagonal tile, into the buffer tile n-2 freed
+            issue_s((j & 1) ? kS1 : kS0, akpt, kSfKpt);
+            tc_commit(s_full + ((j + 1) & 1));  // signals tile n-1 = j+1
+          }
+        }
+        if (!ok) break;
+        kv_it += 2 * n;
+        tc_commit(q_empty);
+      }
+      tc_commit(fin);
+      drain_wait(fin, 0, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int row = warp * 32 + lane;  // query row = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    uint32_t s_cnt[2] = {0, 0}, pv_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
+      const Item it = decode(p, w);
+      const int n = it.n;
+      const int q_idx = it.q0 + row;
+      float M = -INFINITY, l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        const int sbi = j & 1;
+        if (!warp_wait(s_full + sbi, (sbi ? s_cnt[1] : s_cnt[0]) & 1, wd, 57)) { ok = false; break; }
+        if (sbi) ++s_cnt[1]; else ++s_cnt[0];
+        tc_fence_after();
+        const bool diag = j == n - 1;
+        const uint32_t sb = lane_base + ((j & 1) ? kS1 : kS0);
+        uint32_t r[128];
+        tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld32(sb + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+        tmem_ld32(sb + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+        if (diag) {
+          // per-token scores of this row's own 32-key block (the warp's block)
+          uint32_t rp[32];
+          tmem_ld32(lane_base + ((j & 1) ? kS0 : kS1) + 32 * warp, rp);
+          tmem_wait_ld(rp);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            // warp-uniform select of the 32 columns of block `warp`
+            if (warp == 0) r[c] = rp[c];
+            else if (warp == 1) r[32 + c] = rp[c];
+            else if (warp == 2) r[64 + c] = rp[c];
+            else r[96 + c] = rp[c];
+          }
+        }
+        float x[128];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const bool vis = !diag || (c <= row);
+          x[c] = vis ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, x[c]);
+        }
+        float alpha = 1.f;
+        if (mx > M + kRescaleThreshold) {
+          const float Mn = ceilf(mx);
+          // 2^(M - Mn), built exactly (0 on the first tile, when M = -inf)
+          const float dk = M - Mn;
+          alpha = (dk >= -126.f) ? mx_pow2((int)dk) : 0.f;
+          l *= alpha;
+          M = Mn;
+        }
+        const bool any_rescale = __any_sync(0xFFFFFFFFu, alpha != 1.f) && j > 0;
+        // u = 2^(x - M), row sum before quantisation, then MX quantisation per 32-key block
+        uint32_t codes[32];
+        uint32_t sfword = 0;
+        float rs = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          float amax = 0.f;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            x[32 * kb + c] = fast_exp2(x[32 * kb + c] - M);
+            rs += x[32 * kb + c];
+            amax = fmaxf(amax, x[32 * kb + c]);
+          }
+          const int X = mx_block_exponent(amax, p.rule);
+          const float sc = mx_pow2_neg(X < -126 ? -126 : X);
+          sfword |= (uint32_t)(X + 127) << (8 * kb);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float* u = &x[32 * kb + 4 * c];
+            codes[8 * kb + c] = mx_e4m3x2(u[0] * sc, u[1] * sc) | (mx_e4m3x2(u[2] * sc, u[3] * sc) << 16);
+          }
+        }
+        l += rs;
+        // bf16 copy of the diagonal 32-block's P~ (exact), and zero FP8 codes there
+        uint32_t pd[16];
+        if (diag) {
+          const int X = (int)((sfword >> (8 * warp)) & 0xFFu) - 127;
+          const float sc = mx_pow2(X < -126 ? -126 : X);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t w4 = 0;
+            if (warp == 0) w4 = codes[c];
+            else if (warp == 1) w4 = codes[8 + c];
+            else if (warp == 2) w4 = codes[16 + c];
+            else w4 = codes[24 + c];
+            float a, b, cc, d;
+            mx_decode2(w4 & 0xFFFFu, a, b);
+            mx_decode2(w4 >> 16, cc, d);
+            pd[2 * c] = pack_bf16x2(a * sc, b * sc);
+            pd[2 * c + 1] = pack_bf16x2(cc * sc, d * sc);
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (warp == 0) codes[c] = 0;
+            else if (warp == 1) codes[8 + c] = 0;
+            else if (warp == 2) codes[16 + c] = 0;
+            else codes[24 + c] = 0;
+          }
+        }
+        // PV(j-1) must be done before P's shared buffer and O are touched
+        if (j > 0) {
+          if (!warp_wait(pv_done, pv_cnt & 1, wd, 58)) { ok = false; break; }
+          ++pv_cnt;
+          tc_fence_after();
+        }
+        // P codes: row `row`, 128 bytes = 8 chunks of 16 bytes, 128-byte swizzle
+        {
+          uint8_t* prow = sP + row * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
+                make_uint4(codes[4 * c], codes[4 * c + 1], codes[4 * c + 2], codes[4 * c + 3]);
+          reinterpret_cast<uint32_t*>(sfP)[(row & 31) * 4 + (row >> 5)] = sfword;
+        }
+        if (diag) {
+          // P_diag: bf16, two 64-key boxes of 128 rows x 128 bytes; only block `warp` is non-zero
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {  // 16 chunks of 8 bf16 over the 128 keys
+            const int box = c >> 3, cc = c & 7;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if ((c >> 2) == warp) {
+              const int q = c & 3;
+              v = make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
+            }
+            *reinterpret_cast<uint4*>(sPd + box * kBox + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
+          }
+        }
+        if (any_rescale) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t t[32];
+            tmem_ld32(lane_base + kO + 32 * c, t);
+            tmem_wait_ld(t);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
+            tmem_st32(lane_base + kO + 32 * c, t);
+          }
+          tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      // epilogue
+      if (!warp_wait(o_full, o_cnt & 1, wd, 59)) break;
+      ++o_cnt;
+      ++pv_cnt;  // the last tile's PV completion is covered by o_full
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool valid = q_idx < it.e;
+      __nv_bfloat16* orow = p.o + ((size_t)q_idx * p.Hq + it.h) * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t t[32];
+        tmem_ld32(lane_base + kO + 32 * c, t);
+        tmem_wait_ld(t);
+        uint32_t ob[16], rb[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float f0 = __uint_as_float(t[2 * e]) * inv_l, f1 = __uint_as_float(t[2 * e + 1]) * inv_l;
+          ob[e] = pack_bf16x2(f0, f1);
+          rb[e] = pack_bf16x2(f0 - __uint_as_float(ob[e] << 16), f1 - __uint_as_float(ob[e] & 0xFFFF0000u));
+        }
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+          uint4* rdst = reinterpret_cast<uint4*>(p.o_resid + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+            rdst[e] = make_uint4(rb[4 * e], rb[4 * e + 1], rb[4 * e + 2], rb[4 * e + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(o_free);
+      if (valid) p.lse[(size_t)it.h * p.T + q_idx] = (M + __log2f(l)) * kLn2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
+  CUtensorMap tq, tktb, tkpt, tvtb, tvpt;
+  if (!make_tmap_codes(&tq, a.q_vpt, a.T, a.Hq) || !make_tmap_codes(&tktb, a.k_vtb, a.T, a.Hkv) ||
+      !make_tmap_codes(&tkpt, a.k_vpt, a.T, a.Hkv) || !make_tmap_codes(&tvtb, a.v_vtb, a.T, a.Hkv) ||
+      !make_tmap_thd(&tvpt, a.v_deq_pt, a.T, a.Hkv, 128))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(fwd_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  Params p;
+  p.cu = a.cu;
+  p.list = a.sched.list;
+  p.n_items = a.sched.n_items;
+  p.q_spt = a.q_spt;
+  p.k_stb = a.k_stb;
+  p.k_spt = a.k_spt;
+  p.v_stb = a.v_stb;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.o_resid = static_cast<__nv_bfloat16*>(a.o_resid);
+  p.status = a.status;
+  p.timeout_ns = a.timeout_ns;
+  p.T = a.T;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.n_docs = a.n_docs;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.rule = a.rule;
+  const long long max_units = (long long)a.sched.max_items * a.Hq;
+  const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
+  fwd_mxfp8_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tktb, tkpt, tvtb, tvpt, p);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace fapk

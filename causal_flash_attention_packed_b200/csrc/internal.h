@@ -41,9 +41,10 @@ struct SchedBuf {
 cudaError_t launch_schedule(const int32_t* cu, int n_docs, int rows, int mode, const SchedBuf& sb,
                             DeviceStatus* status, bool clear_status, cudaStream_t stream);
 
+// deq_pt_bf16 (optional): also write the per-token form dequantised to bf16.
 cudaError_t launch_quantize_mxfp8(const void* x, int T, int H, int d, const int32_t* cu, int n_docs,
                                   int forms, int rule, uint8_t* vtb, uint8_t* stb, uint8_t* vpt,
-                                  uint8_t* spt, cudaStream_t stream);
+                                  uint8_t* spt, cudaStream_t stream, void* deq_pt_bf16 = nullptr);
 
 // Forward, bf16 operands (fwd_bf16.cu).
 struct FwdArgs {
@@ -64,6 +65,35 @@ struct FwdArgs {
   int num_sms;
 };
 cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t stream);
+
+// Forward, MXFP8 path (fwd_mxfp8.cu): codes and scales from the quantiser.
+struct FwdMxArgs {
+  const uint8_t* q_vpt;      // Q per-token codes [T][Hq][128]
+  const uint8_t* q_spt;      // Q per-token scales [T][Hq][4]
+  const uint8_t* k_vtb;      // K token-block codes [T][Hkv][128]
+  const uint8_t* k_stb;      // K token-block scales [T/32 + n_docs][Hkv][4]
+  const uint8_t* k_vpt;      // K per-token codes
+  const uint8_t* k_spt;      // K per-token scales
+  const uint8_t* v_vtb;      // V token-block codes
+  const uint8_t* v_stb;      // V token-block scales
+  const void* v_deq_pt;      // V per-token form dequantised to bf16 [T][Hkv][128]
+  void* o;
+  float* lse;
+  void* o_resid;
+  const int32_t* cu;
+  int T, Hq, Hkv, n_docs;
+  float scale;
+  int rule;
+  SchedBuf sched;
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+  int num_sms;
+};
+cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream);
+
+// Tensor map of E4M3 codes [T][H][128] as (128, H, T), box 128 x 1 x 128,
+// 128-byte swizzle (api.cu).
+bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H);
 
 // Backward, bf16 operands (bwd_bf16.cu).
 struct BwdArgs {

@@ -15,60 +15,37 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "mx.cuh"
 #include "ptx.cuh"
 
 namespace fapk {
 
 namespace {
 
-// Scale exponent X of a block with maximum magnitude `amax` (a non-negative
-// finite float).  floor(log2 amax) is read from the bit pattern.
-//  rule 0 (RCEIL): smallest X with amax * 2^-X <= 448, i.e. one more than
-//                  floor(log2 amax) - 8 when the significand exceeds 1.75.
-//  rule 1 (OCP):   floor(log2 amax) - 8.
-// Clamped to [-127, 127]; amax == 0 gives -127.
-__device__ __forceinline__ int block_exponent(float amax, int rule) {
-  const uint32_t b = __float_as_uint(amax);
-  if (b == 0u) return -127;
-  const int E = (int)((b >> 23) & 0xFFu);
-  const uint32_t M = b & 0x7FFFFFu;
-  int e;
-  bool above;
-  if (E != 0) {
-    e = E - 127;
-    above = M > 0x600000u;  // 1 + M / 2^23 > 1.75
-  } else {                  // subnormal: M * 2^-149
-    const int n = 32 - __clz(M);
-    e = n - 150;
-    above = 4ull * M > (7ull << (n - 1));
-  }
-  int X = e - 8 + ((rule == FAPK_SCALE_RCEIL && above) ? 1 : 0);
-  return X < -127 ? -127 : (X > 127 ? 127 : X);
-}
-
-// 2^-X as a float (X in [-127, 126], so the exponent field stays normal).
-__device__ __forceinline__ float pow2_neg(int X) { return __uint_as_float((uint32_t)(127 - X) << 23); }
-
-// Two E4M3 codes (round to nearest even, saturating to +-448) in the low and
-// high byte.
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// A code whose magnitude is zero becomes 0x00 (no negative zero), bytewise.
-__device__ __forceinline__ uint32_t canon_zero(uint32_t w) {
-  const uint32_t nz = ((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) & 0x80808080u;  // bit 7: low 7 bits != 0
-  return (w & 0x7F7F7F7Fu) | (w & nz);
-}
-
 // Eight values -> eight codes with scale exponent X.
 __device__ __forceinline__ uint2 encode8(const float (&f)[8], int X) {
-  const float s = pow2_neg(X);
-  uint32_t a = e4m3x2(f[0] * s, f[1] * s) | (e4m3x2(f[2] * s, f[3] * s) << 16);
-  uint32_t b = e4m3x2(f[4] * s, f[5] * s) | (e4m3x2(f[6] * s, f[7] * s) << 16);
-  return make_uint2(canon_zero(a), canon_zero(b));
+  const float s = mx_pow2_neg(X);
+  uint32_t a = mx_e4m3x2(f[0] * s, f[1] * s) | (mx_e4m3x2(f[2] * s, f[3] * s) << 16);
+  uint32_t b = mx_e4m3x2(f[4] * s, f[5] * s) | (mx_e4m3x2(f[6] * s, f[7] * s) << 16);
+  return make_uint2(mx_canon_zero(a), mx_canon_zero(b));
+}
+
+// Dequantised values decode(code) * 2^X of eight codes, as bf16 (exact for
+// every value within the bf16 range).
+__device__ __forceinline__ uint4 dequant8_bf16(uint2 codes, int X) {
+  const float sc = mx_pow2(X < -126 ? -126 : X);
+  const float extra = X < -126 ? 0.5f : 1.f;  // X = -127 only for all-zero blocks
+  const uint32_t w[2] = {codes.x, codes.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float a, b, c, d;
+    mx_decode2(w[i] & 0xFFFFu, a, b);
+    mx_decode2(w[i] >> 16, c, d);
+    o[2 * i] = pack_bf16x2(a * sc * extra, b * sc * extra);
+    o[2 * i + 1] = pack_bf16x2(c * sc * extra, d * sc * extra);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
@@ -84,7 +61,7 @@ template <int D>
 __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(
     const __nv_bfloat16* __restrict__ x, int H, const int32_t* __restrict__ cu, int n_docs, int forms,
     int rule, uint8_t* __restrict__ vtb, uint8_t* __restrict__ stb, uint8_t* __restrict__ vpt,
-    uint8_t* __restrict__ spt) {
+    uint8_t* __restrict__ spt, __nv_bfloat16* __restrict__ deq_pt) {
   constexpr int TPR = D / 8;      // threads per token row (8 channels each)
   constexpr int RPP = 128 / TPR;  // token rows per pass
   constexpr int NP = 32 / RPP;    // passes over the 32-token block
@@ -127,9 +104,11 @@ __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(
     a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
     const int row = r0 + p * RPP;
     if ((forms & FAPK_FORM_PT) && row < nb) {
-      const int X = block_exponent(a, rule);
+      const int X = mx_block_exponent(a, rule);
       const size_t t = (size_t)(t0 + row);
-      *reinterpret_cast<uint2*>(vpt + t * row_stride + col) = encode8(f[p], X);
+      const uint2 codes = encode8(f[p], X);
+      *reinterpret_cast<uint2*>(vpt + t * row_stride + col) = codes;
+      if (deq_pt) *reinterpret_cast<uint4*>(deq_pt + t * row_stride + col) = dequant8_bf16(codes, X);
       if ((c8 & 3) == 0) spt[(t * H + h) * NG + (c8 >> 2)] = (uint8_t)(X + 127);
     }
     amax_tb = fmaxf(amax_tb, a);
@@ -144,7 +123,7 @@ __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(
   __syncthreads();
   const int g = c8 >> 2;
   const float a = fmaxf(fmaxf(red[0][g], red[1][g]), fmaxf(red[2][g], red[3][g]));
-  const int X = block_exponent(a, rule);
+  const int X = mx_block_exponent(a, rule);
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int row = r0 + p * RPP;
@@ -154,7 +133,7 @@ __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(
   if (threadIdx.x < NG) {
     const int gg = threadIdx.x;
     const float ag = fmaxf(fmaxf(red[0][gg], red[1][gg]), fmaxf(red[2][gg], red[3][gg]));
-    stb[((size_t)slot * H + h) * NG + gg] = (uint8_t)(block_exponent(ag, rule) + 127);
+    stb[((size_t)slot * H + h) * NG + gg] = (uint8_t)(mx_block_exponent(ag, rule) + 127);
   }
 }
 
@@ -162,13 +141,14 @@ __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(
 
 cudaError_t launch_quantize_mxfp8(const void* x, int T, int H, int d, const int32_t* cu, int n_docs,
                                   int forms, int rule, uint8_t* vtb, uint8_t* stb, uint8_t* vpt,
-                                  uint8_t* spt, cudaStream_t stream) {
+                                  uint8_t* spt, cudaStream_t stream, void* deq_pt_bf16) {
   const dim3 grid((unsigned)(T / 32 + n_docs), (unsigned)H);
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  auto* dq = static_cast<__nv_bfloat16*>(deq_pt_bf16);
   if (d == 128)
-    quantize_mxfp8_kernel<128><<<grid, 128, 0, stream>>>(xb, H, cu, n_docs, forms, rule, vtb, stb, vpt, spt);
+    quantize_mxfp8_kernel<128><<<grid, 128, 0, stream>>>(xb, H, cu, n_docs, forms, rule, vtb, stb, vpt, spt, dq);
   else
-    quantize_mxfp8_kernel<64><<<grid, 128, 0, stream>>>(xb, H, cu, n_docs, forms, rule, vtb, stb, vpt, spt);
+    quantize_mxfp8_kernel<64><<<grid, 128, 0, stream>>>(xb, H, cu, n_docs, forms, rule, vtb, stb, vpt, spt, dq);
   note_launches(1);
   return cudaGetLastError();
 }
