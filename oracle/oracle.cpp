@@ -43,14 +43,18 @@
  *  - token blocks are document-local: block m of document k covers tokens
  *    [s_k + 32m, min(s_k + 32m + 32, e_k)); its scale lives in slot
  *    floor(s_k/32) + k + m of a [T/32 + n_docs] slot array.
- *  - leak guard (rule L): a shared scale may pool only tokens that are
- *    causally visible at every output position it influences.  Operands are
- *    taken in token-block form (32 tokens x 32 channels share one scale) when
- *    the key block and the query block differ, and in per-token form (one
- *    scale per token x 32 channels) on the diagonal block; Q in Q K^T and dO in
- *    dO V^T are always per-token; computed P and dS are quantised per 32-block
- *    along their contraction (P, dS per (query row, key block); P^T, dS^T per
- *    (key row, query block)), from the normalised fp64 P.
+ *  - leak guard (rule L): a shared scale may not pool a token that the output
+ *    it influences must not see.  Key-side operands (K in Q K^T and in
+ *    dQ = dS K, V in P V and in dP = dO V^T) are taken in token-block form
+ *    (32 tokens x 32 channels share one scale) for key blocks before the
+ *    query's block and in per-token form (one scale per token x 32 channels)
+ *    on the diagonal block; Q in Q K^T and dO in dO V^T are always per-token.
+ *    Query-side operands of the query contraction (Q in dK = dS^T Q, dO in
+ *    dV = P^T dO) are in token-block form in every query block: every query
+ *    with a non-zero term there is causally after the key.  Computed P and dS
+ *    are quantised per 32-block along their contraction (P, dS per (query row,
+ *    key block); P^T, dS^T per (key row, query block)), from the normalised
+ *    fp64 P.
  *
  * Parity pins (tests/test_oracle_*.py): Q=0 closed forms, one-token
  * documents, constant V, rows summing to one, torch fp64 SDPA on one
@@ -647,8 +651,8 @@ void orc_mx_attn_fwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
  *   dP_ij = dO~pt_i . V~_j    (V~ by rule L)
  *   dS_ij = P_ij (dP_ij - D_i) in fp64
  *   dQ_i  = scale sum_j dS~_ij K~_j            (dS~ per (row, key block))
- *   dK_j  = scale sum_i dS~T_ji Q~_i           (dS~T per (key, query block),
- *   dV_j  =       sum_i P~T_ji dO~_i            Q~ and dO~ by rule L) */
+ *   dK_j  = scale sum_i dS~T_ji Q~tb_i         (dS~T per (key, query block))
+ *   dV_j  =       sum_i P~T_ji dO~tb_i         (P~T per (key, query block)) */
 void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
                      const double* q, const double* k, const double* v, const double* dout,
                      int flags, double* o, double* lse, double* dq, double* dk, double* dv) {
@@ -724,8 +728,11 @@ void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
           for (int a = 0; a < nb; ++a) {
             const int li = b0 + a;
             if (li < j) continue;  // masked: exactly zero
-            const double* qi = pick(Qtb, Qpt, li, j, d);
-            const double* doi = pick(dOtb, dOpt, li, j, d);
+            // query-side operands of the query contraction: token-block form
+            // in every query block (every query with a non-zero term here is
+            // causally after key j, so no guard is needed)
+            const double* qi = &Qtb[(size_t)li * d];
+            const double* doi = &dOtb[(size_t)li * d];
             for (int r = 0; r < d; ++r) {
               dkj[r] += dc[a] * qi[r];
               dvj[r] += pc[a] * doi[r];
