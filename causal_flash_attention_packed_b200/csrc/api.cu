@@ -137,9 +137,11 @@ FwdLayout fwd_layout(const fapk_problem_t* P) {
 
 // Backward workspace: two work lists, D = rowsum(dO * O) in fp32 and the fp16
 // copies of Q, K and dO that the gradient MMAs read.
+//  MXFP8 path, instead of the fp16 copies: the quantiser's forms of dO.
 struct BwdLayout {
   SchedLayout kv, q;
   size_t delta, q16, k16, do16, total;
+  size_t do_vtb, do_stb, do_vpt, do_spt;
 };
 BwdLayout bwd_layout(const fapk_problem_t* P) {
   BwdLayout L;
@@ -147,7 +149,18 @@ BwdLayout bwd_layout(const fapk_problem_t* P) {
   L.kv = sched_layout(kAlign, P->T, P->n_docs, P->max_seqlen, kBwdRows);
   L.q = sched_layout(L.kv.end, P->T, P->n_docs, P->max_seqlen, kBwdRows);
   L.delta = L.q.end;
-  L.q16 = align_up(L.delta + sizeof(float) * (size_t)P->Hq * (size_t)P->T);
+  const size_t after_delta = align_up(L.delta + sizeof(float) * (size_t)P->Hq * (size_t)P->T);
+  if (P->prec == FAPK_MXFP8) {
+    const size_t slots = (size_t)P->T / 32 + P->n_docs;
+    L.q16 = L.k16 = L.do16 = 0;
+    L.do_vtb = after_delta;
+    L.do_stb = align_up(L.do_vtb + nq);
+    L.do_vpt = align_up(L.do_stb + slots * P->Hq * (P->d / 32));
+    L.do_spt = align_up(L.do_vpt + nq);
+    L.total = align_up(L.do_spt + (size_t)P->T * P->Hq * (P->d / 32));
+    return L;
+  }
+  L.q16 = after_delta;
   L.k16 = align_up(L.q16 + 2 * nq);
   L.do16 = align_up(L.k16 + 2 * nk);
   L.total = align_up(L.do16 + 2 * nq);
@@ -169,7 +182,7 @@ struct MxForms {
 struct CtxLayout {
   size_t o_resid, v16, total;
   MxForms q, k, v;
-  size_t v_deq_pt;
+  size_t v_deq_pt, k_deq_pt;
 };
 CtxLayout ctx_layout(const fapk_problem_t* P) {
   CtxLayout L;
@@ -196,7 +209,8 @@ CtxLayout ctx_layout(const fapk_problem_t* P) {
   L.k = forms(P->Hkv);
   L.v = forms(P->Hkv);
   L.v_deq_pt = off;
-  L.total = align_up(off + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
+  L.k_deq_pt = align_up(L.v_deq_pt + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
+  L.total = align_up(L.k_deq_pt + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
   return L;
 }
 
@@ -253,7 +267,8 @@ int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void*
                                          u8(C.q.vtb), u8(C.q.stb), u8(C.q.vpt), u8(C.q.spt), st));
   if (rc != FAPK_OK) return rc;
   rc = cuda_status(launch_quantize_mxfp8(k, P->T, P->Hkv, P->d, P->cu_seqlens_dev, P->n_docs, forms, P->scale_rule,
-                                         u8(C.k.vtb), u8(C.k.stb), u8(C.k.vpt), u8(C.k.spt), st));
+                                         u8(C.k.vtb), u8(C.k.stb), u8(C.k.vpt), u8(C.k.spt), st,
+                                         c + C.k_deq_pt));
   if (rc != FAPK_OK) return rc;
   rc = cuda_status(launch_quantize_mxfp8(v, P->T, P->Hkv, P->d, P->cu_seqlens_dev, P->n_docs, forms, P->scale_rule,
                                          u8(C.v.vtb), u8(C.v.stb), u8(C.v.vpt), u8(C.v.spt), st,
@@ -285,6 +300,53 @@ int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void*
   rc = cuda_status(launch_fwd_mxfp8(a, st));
   mk.at(3, st);
   return rc;
+}
+
+// MXFP8 backward: quantise dO (both forms) into the workspace, build both
+// schedules, run D, dK/dV and dQ.
+int bwd_mxfp8(const fapk_problem_t* P, const void* o, const float* lse, const void* dout, const void* ctx, void* dq,
+              void* dk, void* dv, void* ws, const BwdLayout& L, int sms, cudaStream_t st) {
+  auto* status = static_cast<DeviceStatus*>(ws);
+  const CtxLayout C = ctx_layout(P);
+  const char* c = static_cast<const char*>(ctx);
+  char* w = static_cast<char*>(ws);
+  auto cu8 = [&](size_t off) { return reinterpret_cast<const uint8_t*>(c + off); };
+  auto wu8 = [&](size_t off) { return reinterpret_cast<uint8_t*>(w + off); };
+  BwdMxArgs a;
+  a.marks = Marks{P->timing_events, P->n_timing_events};
+  a.sched_kv = sched_buf(ws, L.kv);
+  a.sched_q = sched_buf(ws, L.q);
+  a.marks.at(0, st);
+  int rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedKV, a.sched_kv, status, true, st));
+  if (rc != FAPK_OK) return rc;
+  a.marks.at(1, st);
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedQ, a.sched_q, status, false, st));
+  if (rc != FAPK_OK) return rc;
+  a.marks.at(2, st);
+  rc = cuda_status(launch_quantize_mxfp8(dout, P->T, P->Hq, P->d, P->cu_seqlens_dev, P->n_docs,
+                                         FAPK_FORM_TB | FAPK_FORM_PT, P->scale_rule, wu8(L.do_vtb), wu8(L.do_stb),
+                                         wu8(L.do_vpt), wu8(L.do_spt), st));
+  if (rc != FAPK_OK) return rc;
+  a.q_vtb = cu8(C.q.vtb); a.q_stb = cu8(C.q.stb); a.q_vpt = cu8(C.q.vpt); a.q_spt = cu8(C.q.spt);
+  a.k_vtb = cu8(C.k.vtb); a.k_stb = cu8(C.k.stb); a.k_vpt = cu8(C.k.vpt); a.k_spt = cu8(C.k.spt);
+  a.v_vtb = cu8(C.v.vtb); a.v_stb = cu8(C.v.stb); a.v_vpt = cu8(C.v.vpt); a.v_spt = cu8(C.v.spt);
+  a.do_vtb = wu8(L.do_vtb); a.do_stb = wu8(L.do_stb); a.do_vpt = wu8(L.do_vpt); a.do_spt = wu8(L.do_spt);
+  a.k_deq_pt = c + C.k_deq_pt;
+  a.o = o;
+  a.o_resid = c + C.o_resid;
+  a.lse = lse;
+  a.dout = dout;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.delta = reinterpret_cast<float*>(w + L.delta);
+  a.cu = P->cu_seqlens_dev;
+  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv;
+  a.scale = P->scale;
+  a.grad_bf16 = P->grad_dtype == FAPK_GRAD_BF16;
+  a.rule = P->scale_rule;
+  a.status = status;
+  a.timeout_ns = timeout_ns_of(P);
+  a.num_sms = sms;
+  return cuda_status(launch_bwd_mxfp8(a, st));
 }
 
 }  // namespace
@@ -363,10 +425,11 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
     return FAPK_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(P);
   if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
-  if (P->prec != FAPK_BF16) return FAPK_ERR_UNSUPPORTED;  // the MXFP8 backward is not built yet
+  if (P->prec == FAPK_MXFP8 && P->d != 128) return FAPK_ERR_UNSUPPORTED;
   const int sms = device_num_sms();
   if (sms <= 0) return FAPK_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (P->prec == FAPK_MXFP8) return bwd_mxfp8(P, o, lse, dout, ctx, dq, dk, dv, ws, L, sms, st);
   auto* status = static_cast<DeviceStatus*>(ws);
   BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;

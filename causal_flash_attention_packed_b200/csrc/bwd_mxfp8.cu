@@ -1,0 +1,974 @@
+// Backward of causal packed-document attention, MXFP8 path, for sm_100a
+// (FLAMIA page, sec. "FLAMIA Mimarisi ve Temel Tasarim Ilkeleri": MXFP8
+// operands with shared E8M0 scales, quantised operands reused across the
+// forward and backward orientations, leak guards, fwd/bwd consistency).
+//
+// The straight-through gradient of the MXFP8 forward, from the same quantised
+// operands (the forward's ctx holds Q, K, V in both forms; dO is quantised
+// here):
+//   P    = exp(S - LSE), S from Q~pt and K~ (rule L)      D = dO . O
+//   dP   = dO~pt V~^T (rule L on V)                        dS = P (dP - D)
+//   dQ   = scale dS~ K~   (dS~ per (query row, key block); K by rule L)
+//   dK   = scale dS~T Q~tb,  dV = P~T dO~tb   (dS~T, P~T per (key row, query block))
+// Rule L on the key side: token-block forms for key blocks before the query's
+// block, per-token forms on the diagonal 32x32 blocks.
+//
+// Two kernels, deterministic (no atomics), both persistent with 1 CTA per SM:
+//  * dq_mx:   item = (document, 128-query tile, head); one thread per query
+//    row.  Per key tile: S = Q K^T and dP = dO V^T (block-scaled FP8, K and V
+//    in token-block form; on the diagonal tile a second phase with the
+//    per-token forms into the same TMEM columns), dS~ quantised into shared
+//    memory, dQ += dS~ K~tb (FP8, the same K~tb bytes read MN-major) plus, on
+//    the diagonal tile, the diagonal blocks as an exact bf16 MMA with the
+//    dequantised per-token K.
+//  * dkdv_mx: item = (document, 128-key tile, KV head); one thread per key
+//    row, warpgroup w on query columns [64w, 64w + 64).  Per query tile:
+//    S^T then dP^T into one TMEM region in turn (TMEM also holds dV, dK and
+//    the scale factors), P~T and dS~T quantised into shared memory,
+//    dV += P~T dO~tb and dK += dS~T Q~tb as block-scaled FP8 MMAs.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "mx.cuh"
+#include "ptx.cuh"
+
+namespace fapk {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kCode = 128 * 128;      // 128 rows x 128 fp8 codes
+constexpr int kBf16 = 128 * 128 * 2;  // 128 rows x 128 bf16
+constexpr int kBox = 128 * 64 * 2;    // one 64-element bf16 box of 128 rows
+constexpr int kSfBlk = 512;
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > budget_ns) return;
+  }
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd, int where) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
+}
+
+__device__ __forceinline__ uint32_t pt_word(const uint8_t* spt, int t, int T, int H, int h) {
+  return t < T ? __ldg(reinterpret_cast<const uint32_t*>(spt + ((size_t)t * H + h) * 4)) : 0x7F7F7F7Fu;
+}
+
+__device__ __forceinline__ uint32_t tb_word(const uint8_t* stb, int s, int e, int doc, int blk, int H, int g) {
+  if (32 * blk >= e - s) return 0x7F7F7F7Fu;
+  const size_t slot = (size_t)(s >> 5) + doc + blk;
+  return __ldg(reinterpret_cast<const uint32_t*>(stb + (slot * H + g) * 4));
+}
+
+// Scale block of an MN-major operand whose rows are the 128 channels and
+// whose K blocks are the token blocks blk0..blk0+3 (token-block form): byte
+// kb of the word of channel row (lane + 32 r1) is the scale of (block
+// blk0 + kb, channel group r1).
+__device__ __forceinline__ uint4 tb_channel_rows(const uint8_t* stb, int s, int e, int doc, int blk0, int H, int g) {
+  uint32_t wv[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int kb = 0; kb < 4; ++kb) {
+    const uint32_t t = tb_word(stb, s, e, doc, blk0 + kb, H, g);
+#pragma unroll
+    for (int r1 = 0; r1 < 4; ++r1) wv[r1] |= ((t >> (8 * r1)) & 0xFFu) << (8 * kb);
+  }
+  return make_uint4(wv[0], wv[1], wv[2], wv[3]);
+}
+
+__device__ __forceinline__ uint4 pt_rows(const uint8_t* spt, int t0, int lane, int T, int H, int h) {
+  return make_uint4(pt_word(spt, t0 + lane, T, H, h), pt_word(spt, t0 + lane + 32, T, H, h),
+                    pt_word(spt, t0 + lane + 64, T, H, h), pt_word(spt, t0 + lane + 96, T, H, h));
+}
+
+__device__ __forceinline__ uint4 tb_rows(const uint8_t* stb, int s, int e, int doc, int blk0, int H, int g) {
+  return make_uint4(tb_word(stb, s, e, doc, blk0, H, g), tb_word(stb, s, e, doc, blk0 + 1, H, g),
+                    tb_word(stb, s, e, doc, blk0 + 2, H, g), tb_word(stb, s, e, doc, blk0 + 3, H, g));
+}
+
+// MX quantisation of 32 values (one block): 8 code words; returns the scale byte.
+__device__ __forceinline__ uint32_t quant32(const float (&x)[32], int rule, uint32_t (&codes)[8]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) amax = fmaxf(amax, fabsf(x[c]));
+  const int X = mx_block_exponent(amax, rule);
+  const float sc = mx_pow2_neg(X < -126 ? -126 : X);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    codes[c] = mx_canon_zero(mx_e4m3x2(x[4 * c] * sc, x[4 * c + 1] * sc) |
+                             (mx_e4m3x2(x[4 * c + 2] * sc, x[4 * c + 3] * sc) << 16));
+  return (uint32_t)(X + 127);
+}
+
+// Exact bf16 of the dequantised block: 16 words of packed bf16 pairs.
+__device__ __forceinline__ void dequant32_bf16(const uint32_t (&codes)[8], uint32_t sbyte, uint32_t (&out)[16]) {
+  const int X = (int)sbyte - 127;
+  const float sc = mx_pow2(X < -126 ? -126 : X);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float a, b, cc, d;
+    mx_decode2(codes[c] & 0xFFFFu, a, b);
+    mx_decode2(codes[c] >> 16, cc, d);
+    out[2 * c] = pack_bf16x2(a * sc, b * sc);
+    out[2 * c + 1] = pack_bf16x2(cc * sc, d * sc);
+  }
+}
+
+// 8 code words (32 codes) into row `row` of a K-major FP8 tile at 16-byte
+// chunks c0, c0+1 (128-byte swizzle).
+__device__ __forceinline__ void store_codes32(uint8_t* tile, int row, int c0, const uint32_t (&w)[8]) {
+  uint8_t* prow = tile + row * 128;
+  *reinterpret_cast<uint4*>(prow + ((c0 ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(prow + (((c0 + 1) ^ (row & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// 32 bf16 (16 words) into row `row` of a K-major bf16 tile (two 64-element
+// boxes) at element offset 32 q (q = 0..3).
+__device__ __forceinline__ void store_bf16_32(uint8_t* tile, int row, int q, const uint32_t (&w)[16]) {
+  const int box = q >> 1, c0 = (q & 1) * 4;
+  uint8_t* prow = tile + box * kBox + row * 128;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    *reinterpret_cast<uint4*>(prow + (((c0 + c) ^ (row & 7)) << 4)) =
+        make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+}
+
+__device__ __forceinline__ void zero_bf16_row(uint8_t* tile, int row) {
+#pragma unroll
+  for (int box = 0; box < 2; ++box)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(tile + box * kBox + row * 128 + (c << 4)) = make_uint4(0, 0, 0, 0);
+}
+
+// ---------------------------------------------------------------------------
+// D = rowsum(dO * (o + o_resid)), fp32 [Hq][T]
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) delta_mx_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ o_resid,
+                                                       const __nv_bfloat16* __restrict__ dout,
+                                                       float* __restrict__ delta, int T, int Hq) {
+  const long long row = (long long)blockIdx.x * 16 + threadIdx.x / 16;
+  const int c8 = threadIdx.x % 16;
+  float acc = 0.f;
+  if (row < (long long)T * Hq) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + row * 128) + c8);
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(o_resid + row * 128) + c8);
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * 128) + c8);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wr[4] = {r.x, r.y, r.z, r.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc += (__uint_as_float(wa[i] << 16) + __uint_as_float(wr[i] << 16)) * __uint_as_float(wb[i] << 16);
+      acc += (__uint_as_float(wa[i] & 0xFFFF0000u) + __uint_as_float(wr[i] & 0xFFFF0000u)) *
+             __uint_as_float(wb[i] & 0xFFFF0000u);
+    }
+  }
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+  if (row < (long long)T * Hq && c8 == 0) delta[(row % Hq) * T + row / Hq] = acc;
+}
+
+struct MxParams {
+  const int32_t* cu;
+  const int2* list;
+  const int* n_items;
+  const float* lse;
+  const float* delta;
+  const uint8_t *q_stb, *q_spt, *k_stb, *k_spt, *v_stb, *v_spt, *do_stb, *do_spt;
+  void* out0;  // dq | dk
+  void* out1;  // -  | dv
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+  int T, Hq, Hkv;
+  float scale, scale_log2;
+  int grad_bf16;
+  int rule;
+};
+
+__device__ __forceinline__ void store_row32(void* base, size_t elem_off, const uint32_t (&t)[32], float mul,
+                                            bool bf16) {
+  if (bf16) {
+    uint32_t ob[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      ob[e] = pack_bf16x2(__uint_as_float(t[2 * e]) * mul, __uint_as_float(t[2 * e + 1]) * mul);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + elem_off);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+  } else {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(base) + elem_off);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      dst[e] = make_float4(__uint_as_float(t[4 * e]) * mul, __uint_as_float(t[4 * e + 1]) * mul,
+                           __uint_as_float(t[4 * e + 2]) * mul, __uint_as_float(t[4 * e + 3]) * mul);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ
+// ---------------------------------------------------------------------------
+namespace dqk {
+constexpr int kThreads = 192, kLoad = 4, kMma = 5, kStages = 2;
+constexpr int oQ = 0, oDO = oQ + kCode, oRing = oDO + kCode;  // ring stage: K^tb, V^tb codes
+constexpr int oKpt = oRing + kStages * 2 * kCode, oVpt = oKpt + kCode, oKd = oVpt + kCode;  // diag
+constexpr int oDS = oKd + kBf16, oDSd = oDS + kCode;
+constexpr int oSf = oDSd + kBf16;  // sfQ, sfDO, sfKpt, sfVpt, sfDS, per stage {sfK, sfV, sfKdq}
+constexpr int kNumSf = 5 + 3 * kStages;
+constexpr int oBars = oSf + kNumSf * kSfBlk;
+constexpr int kNumBars = 2 + 2 * kStages + 7;
+constexpr int kSmem = oBars + kNumBars * 8 + 16 + 1024;
+constexpr uint32_t tS = 0, tDP = 128, tDQ = 256;
+constexpr uint32_t tSfQ = 384, tSfDO = 388, tSfK = 392, tSfV = 396, tSfKpt = 400, tSfVpt = 404, tSfDS = 408,
+                   tSfKdq = 412;
+}  // namespace dqk
+
+__global__ void __launch_bounds__(dqk::kThreads, 1)
+    dq_mx_kernel(const __grid_constant__ CUtensorMap tm_qpt, const __grid_constant__ CUtensorMap tm_dopt,
+                 const __grid_constant__ CUtensorMap tm_ktb, const __grid_constant__ CUtensorMap tm_vtb,
+                 const __grid_constant__ CUtensorMap tm_kpt, const __grid_constant__ CUtensorMap tm_vpt,
+                 const __grid_constant__ CUtensorMap tm_kd16, const MxParams p) {
+  using namespace dqk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sf = smem + oSf;  // 512-byte scale blocks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oBars);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* st_full = bars + 2;
+  uint64_t* st_empty = bars + 2 + kStages;
+  uint64_t* s_full = bars + 2 + 2 * kStages;
+  uint64_t* s_read = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* dq_done = s_full + 3;
+  uint64_t* acc_full = s_full + 4;
+  uint64_t* acc_free = s_full + 5;
+  uint64_t* fin = s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto sfb = [&](int i) { return sf + i * kSfBlk; };  // 0 Q, 1 dO, 2 Kpt, 3 Vpt, 4 dS, 5+3s+{0,1,2} stage
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 32);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(st_full + i, 32);
+      mbar_init(st_empty + i, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 128);
+    mbar_init(p_full, 128);
+    mbar_init(dq_done, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_free, 128);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMma) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{p.status, abort_flag, p.timeout_ns};
+  const int n_units = (*p.n_items) * p.Hq;
+  auto decode = [&](int w, int& doc, int& s, int& e, int& h, int& g, int& q0, int& n) {
+    const int2 pr = p.list[w / p.Hq];
+    h = w % p.Hq;
+    g = h / (p.Hq / p.Hkv);
+    doc = pr.x;
+    s = p.cu[doc];
+    e = p.cu[doc + 1];
+    q0 = s + 128 * pr.y;
+    n = pr.y + 1;
+  };
+
+  if (warp == kLoad) {
+    uint32_t st_it = 0;
+    int unit_i = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      int doc, s, e, h, g, q0, n;
+      decode(w, doc, s, e, h, g, q0, n);
+      if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 71)) break;
+      reinterpret_cast<uint4*>(sfb(0))[lane] = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
+      reinterpret_cast<uint4*>(sfb(1))[lane] = pt_rows(p.do_spt, q0, lane, p.T, p.Hq, h);
+      reinterpret_cast<uint4*>(sfb(2))[lane] = pt_rows(p.k_spt, q0, lane, p.T, p.Hkv, g);
+      reinterpret_cast<uint4*>(sfb(3))[lane] = pt_rows(p.v_spt, q0, lane, p.T, p.Hkv, g);
+      fence_proxy_async_smem();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, 4 * kCode + kBf16);
+        tma_load_3d(smem + oQ, &tm_qpt, q_full, 0, h, q0);
+        tma_load_3d(smem + oDO, &tm_dopt, q_full, 0, h, q0);
+        tma_load_3d(smem + oKpt, &tm_kpt, q_full, 0, g, q0);  // the diagonal key tile starts at q0
+        tma_load_3d(smem + oVpt, &tm_vpt, q_full, 0, g, q0);
+        tma_load_3d(smem + oKd, &tm_kd16, q_full, 0, g, q0);
+        tma_load_3d(smem + oKd + kBox, &tm_kd16, q_full, 64, g, q0);
+      } else {
+        mbar_arrive(q_full);
+      }
+      for (int v = 0; v < n; ++v, ++st_it) {
+        const int stg = st_it % kStages;
+        const uint32_t use = st_it / kStages;
+        if (use > 0 && !warp_wait(st_empty + stg, (use - 1) & 1, wd, 72)) { ok = false; break; }
+        reinterpret_cast<uint4*>(sfb(5 + 3 * stg))[lane] = tb_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
+        reinterpret_cast<uint4*>(sfb(6 + 3 * stg))[lane] = tb_rows(p.v_stb, s, e, doc, 4 * v, p.Hkv, g);
+        reinterpret_cast<uint4*>(sfb(7 + 3 * stg))[lane] = tb_channel_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
+        fence_proxy_async_smem();
+        if (lane == 0) {
+          uint8_t* st = smem + oRing + stg * 2 * kCode;
+          mbar_arrive_expect_tx(st_full + stg, 2 * kCode);
+          tma_load_3d(st, &tm_ktb, st_full + stg, 0, g, s + 128 * v);
+          tma_load_3d(st + kCode, &tm_vtb, st_full + stg, 0, g, s + 128 * v);
+        } else {
+          mbar_arrive(st_full + stg);
+        }
+      }
+    }
+    if (lane == 0) {
+      if (unit_i > 0) drain_wait(q_full, (unit_i - 1) & 1, p.timeout_ns);
+      for (uint32_t i = (st_it > kStages ? st_it - kStages : 0); i < st_it; ++i)
+        drain_wait(st_full + (i % kStages), (i / kStages) & 1, p.timeout_ns);
+    }
+  } else if (warp == kMma) {
+    if (lane == 0) {
+      const uint32_t aQ = smem_u32(smem + oQ), aDO = smem_u32(smem + oDO), aRing = smem_u32(smem + oRing),
+                     aKpt = smem_u32(smem + oKpt), aVpt = smem_u32(smem + oVpt), aKd = smem_u32(smem + oKd),
+                     aDS = smem_u32(smem + oDS), aDSd = smem_u32(smem + oDSd), aSf = smem_u32(sf);
+      uint32_t st_it = 0, p_cnt = 0, sr_cnt = 0;
+      int unit_i = 0;
+      bool ok = true;
+      // D (tmem col) = A B^T, both K-major codes, block scales at TMEM cols sfa/sfb
+      auto mx_kk = [&](uint32_t dcol, uint32_t a, uint32_t b, uint32_t sfa, uint32_t sfbc, bool b_mn,
+                       bool acc_first) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_mxf8_ss(tmem + dcol, sdesc_sw128(a + kk * 32, 16, 1024),
+                      b_mn ? sdesc_sw128(b + kk * 4096, 16384, 1024) : sdesc_sw128(b + kk * 32, 16, 1024),
+                      idesc_mxf8(128, 128, b_mn, kk, kk), (tmem + sfa) | ((uint32_t)kk << 30),
+                      (tmem + sfbc) | ((uint32_t)kk << 30), (acc_first || kk > 0) ? 1u : 0u);
+      };
+      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+        int doc, s, e, h, g, q0, n;
+        decode(w, doc, s, e, h, g, q0, n);
+        if (!mbar_wait(q_full, unit_i & 1, wd, 73)) break;
+        tc_fence_after();
+        tmem_cp_sf(tmem + tSfQ, aSf + 0 * kSfBlk);
+        tmem_cp_sf(tmem + tSfDO, aSf + 1 * kSfBlk);
+        tmem_cp_sf(tmem + tSfKpt, aSf + 2 * kSfBlk);
+        tmem_cp_sf(tmem + tSfVpt, aSf + 3 * kSfBlk);
+        for (int v = 0; v < n; ++v, ++st_it) {
+          const int stg = st_it % kStages;
+          if (!mbar_wait(st_full + stg, (st_it / kStages) & 1, wd, 74)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t ak = aRing + stg * 2 * kCode, av = ak + kCode;
+          tmem_cp_sf(tmem + tSfK, aSf + (5 + 3 * stg) * kSfBlk);
+          tmem_cp_sf(tmem + tSfV, aSf + (6 + 3 * stg) * kSfBlk);
+          mx_kk(tS, aQ, ak, tSfQ, tSfK, false, false);
+          mx_kk(tDP, aDO, av, tSfDO, tSfV, false, false);
+          tc_commit(s_full);
+          if (v == n - 1) {
+            // diagonal tile: per-token K and V into the same columns once read
+            if (!mbar_wait(s_read, sr_cnt & 1, wd, 75)) { ok = false; break; }
+            ++sr_cnt;
+            tc_fence_after();
+            mx_kk(tS, aQ, aKpt, tSfQ, tSfKpt, false, false);
+            mx_kk(tDP, aDO, aVpt, tSfDO, tSfVpt, false, false);
+            tc_commit(s_full);
+          }
+          if (!mbar_wait(p_full, p_cnt & 1, wd, 76)) { ok = false; break; }
+          ++p_cnt;
+          if (v == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 77)) { ok = false; break; }
+          tc_fence_after();
+          tmem_cp_sf(tmem + tSfDS, aSf + 4 * kSfBlk);
+          tmem_cp_sf(tmem + tSfKdq, aSf + (7 + 3 * stg) * kSfBlk);
+          mx_kk(tDQ, aDS, ak, tSfDS, tSfKdq, true, v > 0);
+          if (v == n - 1) {
+            constexpr uint32_t idesc_d = idesc_bf16_f32(128, 128, false, true);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_f16_ss(tmem + tDQ, sdesc_sw128(aDSd + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024),
+                         sdesc_sw128(aKd + kk * 2048, kBox, 1024), idesc_d, 1u);
+          }
+          tc_commit(dq_done);
+          tc_commit(st_empty + stg);
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        tc_commit(q_empty);
+      }
+      tc_commit(fin);
+      drain_wait(fin, 0, p.timeout_ns);
+    }
+  } else {
+    // one thread per query row
+    const int row = warp * 32 + lane;
+    const uint32_t lb = tmem + ((uint32_t)(warp * 32) << 16);
+    uint8_t* sDS = smem + oDS;
+    uint8_t* sDSd = smem + oDSd;
+    uint32_t s_cnt = 0, dq_cnt = 0;
+    int unit_i = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      int doc, s, e, h, g, q0, n;
+      decode(w, doc, s, e, h, g, q0, n);
+      const int i = q0 + row;
+      const bool valid = i < e;
+      // rows past the document end get P = 0
+      const float l2 = valid ? p.lse[(size_t)h * p.T + i] * kLog2e : INFINITY;
+      const float dl = valid ? p.delta[(size_t)h * p.T + i] : 0.f;
+      for (int v = 0; v < n; ++v) {
+        if (!warp_wait(s_full, s_cnt & 1, wd, 77)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        const bool diag = v == n - 1;
+        uint32_t codes[32];
+        uint32_t sfword = 0;
+        uint32_t pd[16];
+        // key blocks of this tile; on the diagonal tile block `warp` is the
+        // diagonal block (per-token operands, second phase) and later blocks
+        // are future keys (dS = 0)
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          float ds[32];
+          if (diag && kb > warp) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ds[c] = 0.f;
+          } else if (diag && kb == warp) {
+            continue;  // second phase below
+          } else {
+            uint32_t rs[32], rd[32];
+            tmem_ld32(lb + tS + 32 * kb, rs);
+            tmem_ld32(lb + tDP + 32 * kb, rd);
+            tmem_wait_ld(rs);
+            tmem_wait_ld(rd);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float pp = fast_exp2(__uint_as_float(rs[c]) * p.scale_log2 - l2);
+              ds[c] = pp * (__uint_as_float(rd[c]) - dl);
+            }
+          }
+          uint32_t cw[8];
+          const uint32_t sb = quant32(ds, p.rule, cw);
+          sfword |= sb << (8 * kb);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) codes[8 * kb + c] = cw[c];
+        }
+        if (diag) {
+          tc_fence_before();
+          mbar_arrive(s_read);
+          if (!warp_wait(s_full, s_cnt & 1, wd, 78)) { ok = false; break; }
+          ++s_cnt;
+          tc_fence_after();
+          uint32_t rs[32], rd[32];
+          tmem_ld32(lb + tS + 32 * warp, rs);
+          tmem_ld32(lb + tDP + 32 * warp, rd);
+          tmem_wait_ld(rs);
+          tmem_wait_ld(rd);
+          float ds[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float pp = (32 * warp + c <= row) ? fast_exp2(__uint_as_float(rs[c]) * p.scale_log2 - l2) : 0.f;
+            ds[c] = pp * (__uint_as_float(rd[c]) - dl);
+          }
+          uint32_t cw[8];
+          const uint32_t sb = quant32(ds, p.rule, cw);
+          sfword |= sb << (8 * warp);
+          dequant32_bf16(cw, sb, pd);
+          // the diagonal block leaves the FP8 operand (it goes through the bf16 MMA)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (warp == 0) codes[c] = 0;
+            else if (warp == 1) codes[8 + c] = 0;
+            else if (warp == 2) codes[16 + c] = 0;
+            else codes[24 + c] = 0;
+          }
+        }
+        // dQ of the previous tile must have read the dS buffers
+        if (v > 0) {
+          if (!warp_wait(dq_done, dq_cnt & 1, wd, 79)) { ok = false; break; }
+          ++dq_cnt;
+        }
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          uint32_t cw[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cw[c] = codes[8 * kb + c];
+          store_codes32(sDS, row, 2 * kb, cw);
+        }
+        reinterpret_cast<uint32_t*>(smem + oSf + 4 * kSfBlk)[(row & 31) * 4 + (row >> 5)] = sfword;
+        if (diag) {
+          zero_bf16_row(sDSd, row);
+          store_bf16_32(sDSd, row, warp, pd);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      if (!warp_wait(acc_full, unit_i & 1, wd, 80)) break;
+      ++dq_cnt;  // the last tile's dQ completion is covered by acc_full
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t t[32];
+        tmem_ld32(lb + tDQ + 32 * c, t);
+        tmem_wait_ld(t);
+        if (valid) store_row32(p.out0, ((size_t)i * p.Hq + h) * 128 + 32 * c, t, p.scale, p.grad_bf16);
+      }
+      tc_fence_before();
+      mbar_arrive(acc_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMma) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV
+// ---------------------------------------------------------------------------
+namespace kvk {
+constexpr int kThreads = 320, kLoad = 8, kMma = 9;
+// per item: K^tb, K^pt, V^tb, V^pt codes; per query tile (one stage): Q^pt,
+// Q^tb, dO^pt, dO^tb codes, lse*log2e[128], D[128]; P~T and dS~T codes
+constexpr int oKtb = 0, oKpt = oKtb + kCode, oVtb = oKpt + kCode, oVpt = oVtb + kCode;
+constexpr int oQpt = oVpt + kCode, oQtb = oQpt + kCode, oDOpt = oQtb + kCode, oDOtb = oDOpt + kCode;
+constexpr int oP = oDOtb + kCode, oDS = oP + kCode;
+constexpr int oLse = oDS + kCode, oSf = oLse + 1024;
+// scale blocks: 0 Ktb, 1 Kpt, 2 Vtb, 3 Vpt, 4 Qpt, 5 dOpt, 6 dOtb(dv), 7 Qtb(dk), 8 P, 9 dS
+constexpr int kNumSf = 10;
+constexpr int oBars = oSf + kNumSf * kSfBlk;
+constexpr int kNumBars = 11;
+constexpr int kSmem = oBars + kNumBars * 8 + 16 + 1024;
+constexpr uint32_t tSP = 0, tDV = 128, tDK = 256;
+constexpr uint32_t tSfKtb = 384, tSfKpt = 388, tSfVtb = 392, tSfVpt = 396, tSfQpt = 400, tSfDOpt = 404, tSfP = 408,
+                   tSfDS = 412, tSfDOtb = 416, tSfQtb = 420;
+}  // namespace kvk
+
+__global__ void __launch_bounds__(kvk::kThreads, 1)
+    dkdv_mx_kernel(const __grid_constant__ CUtensorMap tm_ktb, const __grid_constant__ CUtensorMap tm_kpt,
+                   const __grid_constant__ CUtensorMap tm_vtb, const __grid_constant__ CUtensorMap tm_vpt,
+                   const __grid_constant__ CUtensorMap tm_qpt, const __grid_constant__ CUtensorMap tm_qtb,
+                   const __grid_constant__ CUtensorMap tm_dopt, const __grid_constant__ CUtensorMap tm_dotb,
+                   const MxParams p) {
+  using namespace kvk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sf = smem + oSf;
+  auto sfb = [&](int i) { return sf + i * kSfBlk; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oBars);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* st_full = bars + 2;
+  uint64_t* st_empty = bars + 3;
+  uint64_t* s_full = bars + 4;
+  uint64_t* s_read = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* acc_full = bars + 7;
+  uint64_t* acc_free = bars + 8;
+  uint64_t* fin = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 32);
+    mbar_init(kv_empty, 1);
+    mbar_init(st_full, 32);
+    mbar_init(st_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 256);
+    mbar_init(p_full, 256);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_free, 256);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMma) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{p.status, abort_flag, p.timeout_ns};
+  const int n_units = (*p.n_items) * p.Hkv;
+  const int G = p.Hq / p.Hkv;
+  auto decode = [&](int w, int& doc, int& s, int& e, int& g, int& v, int& k0, int& nq) {
+    const int2 pr = p.list[w / p.Hkv];
+    g = w % p.Hkv;
+    doc = pr.x;
+    s = p.cu[doc];
+    e = p.cu[doc + 1];
+    v = pr.y;
+    k0 = s + 128 * v;
+    nq = (e - s + 127) / 128;
+  };
+
+  if (warp == kLoad) {
+    uint32_t st_it = 0;
+    int unit_i = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      int doc, s, e, g, v, k0, nq;
+      decode(w, doc, s, e, g, v, k0, nq);
+      if (unit_i > 0 && !warp_wait(kv_empty, (unit_i - 1) & 1, wd, 81)) break;
+      reinterpret_cast<uint4*>(sfb(0))[lane] = tb_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
+      reinterpret_cast<uint4*>(sfb(1))[lane] = pt_rows(p.k_spt, k0, lane, p.T, p.Hkv, g);
+      reinterpret_cast<uint4*>(sfb(2))[lane] = tb_rows(p.v_stb, s, e, doc, 4 * v, p.Hkv, g);
+      reinterpret_cast<uint4*>(sfb(3))[lane] = pt_rows(p.v_spt, k0, lane, p.T, p.Hkv, g);
+      fence_proxy_async_smem();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(kv_full, 4 * kCode);
+        tma_load_3d(smem + oKtb, &tm_ktb, kv_full, 0, g, k0);
+        tma_load_3d(smem + oKpt, &tm_kpt, kv_full, 0, g, k0);
+        tma_load_3d(smem + oVtb, &tm_vtb, kv_full, 0, g, k0);
+        tma_load_3d(smem + oVpt, &tm_vpt, kv_full, 0, g, k0);
+      } else {
+        mbar_arrive(kv_full);
+      }
+      for (int h = g * G; h < (g + 1) * G && ok; ++h) {
+        for (int m = v; m < nq; ++m, ++st_it) {
+          if (st_it > 0 && !warp_wait(st_empty, (st_it - 1) & 1, wd, 82)) { ok = false; break; }
+          const int q0 = s + 128 * m;
+          reinterpret_cast<uint4*>(sfb(4))[lane] = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
+          reinterpret_cast<uint4*>(sfb(5))[lane] = pt_rows(p.do_spt, q0, lane, p.T, p.Hq, h);
+          reinterpret_cast<uint4*>(sfb(6))[lane] = tb_channel_rows(p.do_stb, s, e, doc, 4 * m, p.Hq, h);
+          reinterpret_cast<uint4*>(sfb(7))[lane] = tb_channel_rows(p.q_stb, s, e, doc, 4 * m, p.Hq, h);
+          float* lse2 = reinterpret_cast<float*>(smem + oLse);
+          float* dl = lse2 + 128;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int i = q0 + lane * 4 + r;
+            const bool in = i < e;  // queries past the document end get P = 0 (lse2 = +inf)
+            lse2[lane * 4 + r] = in ? p.lse[(size_t)h * p.T + i] * kLog2e : INFINITY;
+            dl[lane * 4 + r] = in ? p.delta[(size_t)h * p.T + i] : 0.f;
+          }
+          fence_proxy_async_smem();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(st_full, 4 * kCode);
+            tma_load_3d(smem + oQpt, &tm_qpt, st_full, 0, h, q0);
+            tma_load_3d(smem + oQtb, &tm_qtb, st_full, 0, h, q0);
+            tma_load_3d(smem + oDOpt, &tm_dopt, st_full, 0, h, q0);
+            tma_load_3d(smem + oDOtb, &tm_dotb, st_full, 0, h, q0);
+          } else {
+            mbar_arrive(st_full);
+          }
+        }
+      }
+    }
+    if (lane == 0) {
+      if (unit_i > 0) drain_wait(kv_full, (unit_i - 1) & 1, p.timeout_ns);
+      if (st_it > 0) drain_wait(st_full, (st_it - 1) & 1, p.timeout_ns);
+    }
+  } else if (warp == kMma) {
+    if (lane == 0) {
+      const uint32_t aKtb = smem_u32(smem + oKtb), aKpt = smem_u32(smem + oKpt), aVtb = smem_u32(smem + oVtb),
+                     aVpt = smem_u32(smem + oVpt), aQpt = smem_u32(smem + oQpt), aQtb = smem_u32(smem + oQtb),
+                     aDOpt = smem_u32(smem + oDOpt), aDOtb = smem_u32(smem + oDOtb), aP = smem_u32(smem + oP),
+                     aDS = smem_u32(smem + oDS), aSf = smem_u32(sf);
+      uint32_t st_it = 0, sr_cnt = 0, p_cnt = 0;
+      int unit_i = 0;
+      bool ok = true;
+      auto mx_kk = [&](uint32_t dcol, uint32_t a, uint32_t b, uint32_t sfa, uint32_t sfbc, bool b_mn,
+                       bool acc_first) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_mxf8_ss(tmem + dcol, sdesc_sw128(a + kk * 32, 16, 1024),
+                      b_mn ? sdesc_sw128(b + kk * 4096, 16384, 1024) : sdesc_sw128(b + kk * 32, 16, 1024),
+                      idesc_mxf8(128, 128, b_mn, kk, kk), (tmem + sfa) | ((uint32_t)kk << 30),
+                      (tmem + sfbc) | ((uint32_t)kk << 30), (acc_first || kk > 0) ? 1u : 0u);
+      };
+      auto wait_read = [&]() {
+        const bool r = mbar_wait(s_read, sr_cnt & 1, wd, 83);
+        ++sr_cnt;
+        tc_fence_after();
+        return r;
+      };
+      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+        int doc, s, e, g, v, k0, nq;
+        decode(w, doc, s, e, g, v, k0, nq);
+        if (!mbar_wait(kv_full, unit_i & 1, wd, 84)) break;
+        if (unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 85)) break;
+        tc_fence_after();
+        tmem_cp_sf(tmem + tSfKtb, aSf + 0 * kSfBlk);
+        tmem_cp_sf(tmem + tSfKpt, aSf + 1 * kSfBlk);
+        tmem_cp_sf(tmem + tSfVtb, aSf + 2 * kSfBlk);
+        tmem_cp_sf(tmem + tSfVpt, aSf + 3 * kSfBlk);
+        bool first = true;
+        for (int h = g * G; h < (g + 1) * G && ok; ++h) {
+          for (int m = v; m < nq; ++m, ++st_it) {
+            const bool diag = m == v;
+            if (!mbar_wait(st_full, st_it & 1, wd, 86)) { ok = false; break; }
+            tc_fence_after();
+            tmem_cp_sf(tmem + tSfQpt, aSf + 4 * kSfBlk);
+            tmem_cp_sf(tmem + tSfDOpt, aSf + 5 * kSfBlk);
+            // S^T (token-block K), then on the diagonal the per-token K
+            mx_kk(tSP, aKtb, aQpt, tSfKtb, tSfQpt, false, false);
+            tc_commit(s_full);
+            if (!wait_read()) { ok = false; break; }
+            if (diag) {
+              mx_kk(tSP, aKpt, aQpt, tSfKpt, tSfQpt, false, false);
+              tc_commit(s_full);
+              if (!wait_read()) { ok = false; break; }
+            }
+            // P~T is in shared memory: dV += P~T dO~tb
+            tmem_cp_sf(tmem + tSfP, aSf + 8 * kSfBlk);
+            tmem_cp_sf(tmem + tSfDOtb, aSf + 6 * kSfBlk);
+            mx_kk(tDV, aP, aDOtb, tSfP, tSfDOtb, true, !first);
+            // dP^T (token-block V), then on the diagonal the per-token V
+            mx_kk(tSP, aVtb, aDOpt, tSfVtb, tSfDOpt, false, false);
+            tc_commit(s_full);
+            if (diag) {
+              if (!wait_read()) { ok = false; break; }
+              mx_kk(tSP, aVpt, aDOpt, tSfVpt, tSfDOpt, false, false);
+              tc_commit(s_full);
+            }
+            if (!mbar_wait(p_full, p_cnt & 1, wd, 87)) { ok = false; break; }
+            ++p_cnt;
+            tc_fence_after();
+            tmem_cp_sf(tmem + tSfDS, aSf + 9 * kSfBlk);
+            tmem_cp_sf(tmem + tSfQtb, aSf + 7 * kSfBlk);
+            mx_kk(tDK, aDS, aQtb, tSfDS, tSfQtb, true, !first);
+            first = false;
+            tc_commit(st_empty);
+          }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        tc_commit(kv_empty);
+      }
+      tc_commit(fin);
+      drain_wait(fin, 0, p.timeout_ns);
+    }
+  } else {
+    // one thread per key row; warpgroup wg on query quarters 2 wg, 2 wg + 1
+    const int wg = warp >> 2, quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lb = tmem + ((uint32_t)(quarter * 32) << 16);
+    uint8_t* sP = smem + oP;
+    uint8_t* sDS = smem + oDS;
+    uint8_t* sfP = sfb(8);
+    uint8_t* sfDS = sfb(9);
+    const float* lse2 = reinterpret_cast<const float*>(smem + oLse);
+    const float* dl = lse2 + 128;
+    uint32_t s_cnt = 0;
+    int unit_i = 0;
+    bool ok = true;
+    auto wait_s = [&]() {
+      const bool r = warp_wait(s_full, s_cnt & 1, wd, 88);
+      ++s_cnt;
+      tc_fence_after();
+      return r;
+    };
+    uint32_t st_cnt = 0;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      int doc, s, e, g, v, k0, nq;
+      decode(w, doc, s, e, g, v, k0, nq);
+      const int j = k0 + row;
+      for (int h = g * G; h < (g + 1) * G && ok; ++h) {
+        for (int m = v; m < nq; ++m, ++st_cnt) {
+          const bool diag = m == v;
+          const int i0 = s + 128 * m;  // query index of column 0
+          // the stage's LSE and D were written by the load warp: wait for the
+          // stage directly (not only through the MMA thread's commits)
+          if (!warp_wait(st_full, st_cnt & 1, wd, 90)) { ok = false; break; }
+          // ---- S^T -> P (kept in registers), P~T into shared memory
+          if (!wait_s()) { ok = false; break; }
+          float pr[64];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qq = 2 * wg + u;
+            uint32_t rs[32];
+            tmem_ld32(lb + tSP + 32 * qq, rs);
+            tmem_wait_ld(rs);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pr[32 * u + c] = __uint_as_float(rs[c]);
+          }
+          if (diag) {
+            tc_fence_before();
+            mbar_arrive(s_read);
+            if (!wait_s()) { ok = false; break; }
+            if ((quarter >> 1) == wg) {  // this row's diagonal query block lies in our half
+              uint32_t rs[32];
+              tmem_ld32(lb + tSP + 32 * quarter, rs);
+              tmem_wait_ld(rs);
+              const int u = quarter & 1;
+#pragma unroll
+              for (int c = 0; c < 32; ++c) pr[32 * u + c] = __uint_as_float(rs[c]);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qq = 2 * wg + u;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int cc = 32 * qq + c;
+              const bool vis = !diag || (cc >= row);  // query i0 + cc >= key j (same tile base)
+              pr[32 * u + c] = vis ? fast_exp2(pr[32 * u + c] * p.scale_log2 - lse2[cc]) : 0.f;
+            }
+            float blk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) blk[c] = pr[32 * u + c];
+            uint32_t cw[8];
+            const uint32_t sb = quant32(blk, p.rule, cw);
+            store_codes32(sP, row, 2 * qq, cw);
+            sfP[(row & 31) * 16 + (row >> 5) * 4 + qq] = (uint8_t)sb;
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(s_read);
+          // ---- dP^T -> dS~T into shared memory
+          if (!wait_s()) { ok = false; break; }
+          float dp[64];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qq = 2 * wg + u;
+            uint32_t rd[32];
+            tmem_ld32(lb + tSP + 32 * qq, rd);
+            tmem_wait_ld(rd);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) dp[32 * u + c] = __uint_as_float(rd[c]);
+          }
+          if (diag) {
+            tc_fence_before();
+            mbar_arrive(s_read);
+            if (!wait_s()) { ok = false; break; }
+            if ((quarter >> 1) == wg) {
+              uint32_t rd[32];
+              tmem_ld32(lb + tSP + 32 * quarter, rd);
+              tmem_wait_ld(rd);
+              const int u = quarter & 1;
+#pragma unroll
+              for (int c = 0; c < 32; ++c) dp[32 * u + c] = __uint_as_float(rd[c]);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qq = 2 * wg + u;
+            float blk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) blk[c] = pr[32 * u + c] * (dp[32 * u + c] - dl[32 * qq + c]);
+            uint32_t cw[8];
+            const uint32_t sb = quant32(blk, p.rule, cw);
+            store_codes32(sDS, row, 2 * qq, cw);
+            sfDS[(row & 31) * 16 + (row >> 5) * 4 + qq] = (uint8_t)sb;
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(p_full);
+          (void)i0;
+        }
+      }
+      if (!ok) break;
+      // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK * scale
+      if (!warp_wait(acc_full, unit_i & 1, wd, 89)) break;
+      tc_fence_after();
+      const bool valid = j < e;
+      const uint32_t acc = lb + (wg ? tDK : tDV);
+      void* out = wg ? p.out0 : p.out1;
+      const float mul = wg ? p.scale : 1.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t t[32];
+        tmem_ld32(acc + 32 * c, t);
+        tmem_wait_ld(t);
+        if (valid) store_row32(out, ((size_t)j * p.Hkv + g) * 128 + 32 * c, t, mul, p.grad_bf16);
+      }
+      tc_fence_before();
+      mbar_arrive(acc_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMma) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
+  // 1. D
+  a.marks.at(3, stream);
+  {
+    const long long rows = (long long)a.T * a.Hq;
+    delta_mx_kernel<<<(unsigned)((rows + 15) / 16), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.o_resid),
+        static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.T, a.Hq);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap tqpt, tqtb, tktb, tkpt, tvtb, tvpt, tdopt, tdotb, tkd;
+  if (!make_tmap_codes(&tqpt, a.q_vpt, a.T, a.Hq) || !make_tmap_codes(&tqtb, a.q_vtb, a.T, a.Hq) ||
+      !make_tmap_codes(&tktb, a.k_vtb, a.T, a.Hkv) || !make_tmap_codes(&tkpt, a.k_vpt, a.T, a.Hkv) ||
+      !make_tmap_codes(&tvtb, a.v_vtb, a.T, a.Hkv) || !make_tmap_codes(&tvpt, a.v_vpt, a.T, a.Hkv) ||
+      !make_tmap_codes(&tdopt, a.do_vpt, a.T, a.Hq) || !make_tmap_codes(&tdotb, a.do_vtb, a.T, a.Hq) ||
+      !make_tmap_thd(&tkd, a.k_deq_pt, a.T, a.Hkv, 128))
+    return cudaErrorInvalidValue;
+  MxParams p;
+  p.cu = a.cu;
+  p.lse = a.lse;
+  p.delta = a.delta;
+  p.q_stb = a.q_stb; p.q_spt = a.q_spt;
+  p.k_stb = a.k_stb; p.k_spt = a.k_spt;
+  p.v_stb = a.v_stb; p.v_spt = a.v_spt;
+  p.do_stb = a.do_stb; p.do_spt = a.do_spt;
+  p.status = a.status;
+  p.timeout_ns = a.timeout_ns;
+  p.T = a.T;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * kLog2e;
+  p.grad_bf16 = a.grad_bf16;
+  p.rule = a.rule;
+  // 2. dK, dV
+  a.marks.at(4, stream);
+  {
+    cudaError_t e = cudaFuncSetAttribute(dkdv_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvk::kSmem);
+    if (e != cudaSuccess) return e;
+    MxParams pk = p;
+    pk.list = a.sched_kv.list;
+    pk.n_items = a.sched_kv.n_items;
+    pk.out0 = a.dk;
+    pk.out1 = a.dv;
+    const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
+    const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
+    dkdv_mx_kernel<<<grid, kvk::kThreads, kvk::kSmem, stream>>>(tktb, tkpt, tvtb, tvpt, tqpt, tqtb, tdopt, tdotb, pk);
+    note_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // 3. dQ
+  a.marks.at(5, stream);
+  {
+    cudaError_t e = cudaFuncSetAttribute(dq_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::kSmem);
+    if (e != cudaSuccess) return e;
+    MxParams pq = p;
+    pq.list = a.sched_q.list;
+    pq.n_items = a.sched_q.n_items;
+    pq.out0 = a.dq;
+    pq.out1 = nullptr;
+    const long long max_units = (long long)a.sched_q.max_items * a.Hq;
+    const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
+    dq_mx_kernel<<<grid, dqk::kThreads, dqk::kSmem, stream>>>(tqpt, tdopt, tktb, tvtb, tkpt, tvpt, tkd, pq);
+    note_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  a.marks.at(6, stream);
+  return cudaSuccess;
+}
+
+}  // namespace fapk

@@ -91,6 +91,35 @@ struct FwdMxArgs {
 };
 cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream);
 
+// Backward, MXFP8 path (bwd_mxfp8.cu).
+struct BwdMxArgs {
+  const uint8_t *q_vtb, *q_stb, *q_vpt, *q_spt;     // quantised Q (ctx)
+  const uint8_t *k_vtb, *k_stb, *k_vpt, *k_spt;     // quantised K (ctx)
+  const uint8_t *v_vtb, *v_stb, *v_vpt, *v_spt;     // quantised V (ctx)
+  const uint8_t *do_vtb, *do_stb, *do_vpt, *do_spt; // quantised dO (workspace)
+  const void* k_deq_pt;                             // K per-token form dequantised to bf16 (ctx)
+  const void* o;
+  const void* o_resid;
+  const float* lse;
+  const void* dout;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* delta;
+  const int32_t* cu;
+  int T, Hq, Hkv;
+  float scale;
+  int grad_bf16;
+  int rule;
+  SchedBuf sched_kv;
+  SchedBuf sched_q;
+  Marks marks;
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+  int num_sms;
+};
+cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream);
+
 // Tensor map of E4M3 codes [T][H][128] as (128, H, T), box 128 x 1 x 128,
 // 128-byte swizzle (api.cu).
 bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H);
