@@ -188,6 +188,119 @@ def run_reference(args, w, world, rank):
     print(json.dumps(line), flush=True)
 
 
+KERNELS = {
+    # per path: names of the intervals between the events the library records
+    "bf16": (["schedule_fwd", "convert_v_f16", "fwd_kernel"],
+             ["schedule_kv", "schedule_q", "convert_k_f16", "delta_kernel", "dkdv_kernel", "dq_kernel"]),
+    "mxfp8": (["schedule_fwd", "quantize_qkv", "fwd_kernel"],
+              ["schedule_kv", "schedule_q", "quantize_do", "delta_kernel", "dkdv_kernel", "dq_kernel"]),
+}
+# algorithmic tensor work of each attention kernel per visible (query, key)
+# pair and query head, in units of d: forward S and PV = 4; dK/dV kernel S,
+# dP, dV, dK = 8; dQ kernel S, dP, dQ = 6
+KERNEL_FLOPS = {"fwd_kernel": 4.0, "dkdv_kernel": 8.0, "dq_kernel": 6.0}
+
+
+class Path:
+    """Buffers and one timed fwd+bwd step of one precision path."""
+
+    def __init__(self, fapk, w, prec, dev, tensors):
+        self.fapk, self.w, self.prec, self.dev = fapk, w, prec, dev
+        self.qd, self.kd, self.vd, self.dod = tensors
+        seq = fapk.Seqlens(w.cu, dev)
+        self.seq = seq
+        self.P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale,
+                                   prec=fapk.MXFP8 if prec == "mxfp8" else fapk.BF16)
+        self.ws_f = fapk.workspace(self.P, fapk.FWD, dev)
+        self.ws_b = fapk.workspace(self.P, fapk.BWD, dev)
+        self.o = torch.empty((w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((w.Hq, w.T), dtype=torch.float32, device=dev)
+        self.dq = torch.empty((w.T, w.Hq, w.d), dtype=torch.float32, device=dev)
+        self.dk = torch.empty((w.T, w.Hkv, w.d), dtype=torch.float32, device=dev)
+        self.dv = torch.empty((w.T, w.Hkv, w.d), dtype=torch.float32, device=dev)
+        self.ctx = torch.empty(max(fapk.ctx_size(self.P), 256), dtype=torch.uint8, device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+
+    def step(self, timers=None):
+        f = self.fapk
+        Pf = timers[0].with_events(self.P) if timers else self.P
+        Pb = timers[1].with_events(self.P) if timers else self.P
+        f.attn_fwd(Pf, self.qd, self.kd, self.vd, o=self.o, lse=self.lse, ctx=self.ctx, ws=self.ws_f,
+                   stream=self.stream)
+        f.attn_bwd(Pb, self.qd, self.kd, self.vd, self.o, self.lse, self.dod, ctx=self.ctx, dq=self.dq,
+                   dk=self.dk, dv=self.dv, ws=self.ws_b, stream=self.stream)
+
+    def status_ok(self):
+        return self.fapk.status(self.ws_f) == 0 and self.fapk.status(self.ws_b) == 0
+
+    def timed(self, steps, warmup, world):
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize(self.dev)
+        if not self.status_ok():
+            raise RuntimeError(f"{self.prec}: device status {self.fapk.status(self.ws_f)}/{self.fapk.status(self.ws_b)}")
+        timers = [(self.fapk.KernelTimer(4), self.fapk.KernelTimer(7)) for _ in range(steps)]
+        launches0 = self.fapk.launch_count()
+        barrier(world)
+        torch.cuda.synchronize(self.dev)
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(self.stream)
+        for i in range(steps):
+            self.step(timers[i])
+        end.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        barrier(world)
+        launches = self.fapk.launch_count() - launches0
+        total_ms = max_over_ranks(start.elapsed_time(end), world, self.dev)
+        names = KERNELS[self.prec][0] + KERNELS[self.prec][1]
+        per = [tf.durations_ms() + tb.durations_ms() for tf, tb in timers]
+        kern_ms = {n: max_over_ranks(statistics.mean(row[i] for row in per), world, self.dev)
+                   for i, n in enumerate(names)}
+        return total_ms / steps, kern_ms, launches
+
+
+def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks):
+    flops = w.flops()
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    pairs = w.pairs()
+    fwd_names, bwd_names = KERNELS[prec]
+    fwd_ms = sum(kern_ms[n] for n in fwd_names)
+    bwd_ms = sum(kern_ms[n] for n in bwd_names)
+    dom = max(KERNEL_FLOPS, key=lambda n: kern_ms[n])
+    dom_flops = KERNEL_FLOPS[dom] * w.d * w.Hq * pairs
+    achieved = dom_flops / (kern_ms[dom] * 1e-3) / 1e12
+    if prec == "bf16":
+        peak, peak_src, dense = peaks["bf16_tflops_sustained"], \
+            f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)", DENSE_BF16_TFLOPS
+    else:
+        # no FP8 GEMM is measured on this pool: the measured bf16 sustained
+        # peak times the nominal FP8/bf16 ratio of 2
+        peak, peak_src, dense = 2.0 * peaks["bf16_tflops_sustained"], \
+            f"2 x {peaks['source']} bf16 sustained (MEASURED_PEAKS.json), nominal FP8/bf16 ratio", DENSE_FP8_TFLOPS
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": dom, "peak_source": peak_src,
+                "kernels_ms": kern_ms,
+                "kernels_tflops": {n: KERNEL_FLOPS[n] * w.d * w.Hq * pairs / (kern_ms[n] * 1e-3) / 1e12
+                                   for n in KERNEL_FLOPS},
+                "fwd": {"ms": fwd_ms, "tflops": 4.0 * w.d * w.Hq * pairs / (fwd_ms * 1e-3) / 1e12},
+                "bwd": {"ms": bwd_ms, "tflops": 10.0 * w.d * w.Hq * pairs / (bwd_ms * 1e-3) / 1e12}}
+    out = {"value": value, "ms_per_step": ms_per_step, "pct_of_dense_peak": 100.0 * (value / world) / dense,
+           "dense_peak_tflops": dense, "roofline": roofline, "gpu_launches": launches}
+    if prec == "mxfp8":
+        # quantize launches of the forward (HBM bound): per element 2 B read,
+        # two code forms (2 B), a per-token scale per 32 channels (1/32 B) and
+        # a token-block scale per 32 x 32 (1/1024 B) written; K and V also
+        # write their per-token dequantised copy (2 B)
+        qbytes = (w.T * w.Hq * w.d * (4.0 + 1.0 / 32 + 1.0 / 1024)
+                  + 2 * w.T * w.Hkv * w.d * (6.0 + 1.0 / 32 + 1.0 / 1024))
+        gbs = qbytes / (kern_ms["quantize_qkv"] * 1e-3) / 1e9
+        out["roofline_quantize"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                                    "kernel": "quantize_mxfp8_kernel (Q, K, V; both forms)"}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -196,6 +309,7 @@ def main():
     ap.add_argument("--impl", default="fapk", choices=["fapk", "reference"])
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--paths", default="bf16,mxfp8")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -219,125 +333,71 @@ def main():
     peaks = load_peaks()
 
     q, k, v, do = w.tensors()
-    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
-    seq = fapk.Seqlens(w.cu, dev)
-    P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale)
-    ws_f = fapk.workspace(P, fapk.FWD, dev)
-    ws_b = fapk.workspace(P, fapk.BWD, dev)
-    o = torch.empty((w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((w.Hq, w.T), dtype=torch.float32, device=dev)
-    dq = torch.empty((w.T, w.Hq, w.d), dtype=torch.float32, device=dev)
-    dk = torch.empty((w.T, w.Hkv, w.d), dtype=torch.float32, device=dev)
-    dv = torch.empty((w.T, w.Hkv, w.d), dtype=torch.float32, device=dev)
-    ctx = torch.empty(max(fapk.ctx_size(P), 256), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def step(timers=None):
-        Pf = timers[0].with_events(P) if timers else P
-        Pb = timers[1].with_events(P) if timers else P
-        fapk.attn_fwd(Pf, qd, kd, vd, o=o, lse=lse, ctx=ctx, ws=ws_f, stream=stream)
-        fapk.attn_bwd(Pb, qd, kd, vd, o, lse, dod, ctx=ctx, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    assert fapk.status(ws_f) == 0 and fapk.status(ws_b) == 0
+    dev_tensors = tuple(t.to(dev) for t in (q, k, v, do))
+    paths = [p for p in args.paths.split(",") if p]
+    runners = {p: Path(fapk, w, p, dev, dev_tensors) for p in paths}
 
     clocks = ClockSampler(local) if rank == 0 else None
-    # the library records these events between its own kernel launches
-    timers = [(fapk.KernelTimer(4), fapk.KernelTimer(7)) for _ in range(args.steps)]
-    launches0 = fapk.launch_count()
-    barrier(world)
-    torch.cuda.synchronize(dev)
     if clocks:
         clocks.start()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(args.steps):
-        step(timers[i])
-    end.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
+    results = {}
+    for p in paths:
+        ms, kern_ms, launches = runners[p].timed(args.steps, args.warmup, world)
+        results[p] = path_report(w, p, ms, kern_ms, launches, world, peaks)
     clk = clocks.stop() if clocks else None
-    launches = fapk.launch_count() - launches0
-    st_ok = fapk.status(ws_f) == 0 and fapk.status(ws_b) == 0
-    total_ms = max_over_ranks(start.elapsed_time(end), world, dev)
-    names = ["schedule_fwd", "convert_v_f16", "fwd_kernel", "schedule_kv", "schedule_q", "convert_k_f16",
-             "delta_kernel", "dkdv_kernel", "dq_kernel"]
-    per = [tf.durations_ms() + tb.durations_ms() for tf, tb in timers]
-    kern_ms = {n: max_over_ranks(statistics.mean(row[i] for row in per), world, dev) for i, n in enumerate(names)}
-    fwd_ms = sum(kern_ms[n] for n in names[:3])
-    bwd_ms = sum(kern_ms[n] for n in names[3:])
-    ms_per_step = total_ms / args.steps
-    flops = w.flops()
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    st_ok = all(r.status_ok() for r in runners.values())
 
     # end to end through the C ABI with host buffers (pinned), copies included
     e2e = None
+    main_path = paths[0]
     if args.e2e_steps > 0:
+        R = runners[main_path]
         hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
-        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        hdq = torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True)
-        hdk = torch.empty(dk.shape, dtype=dk.dtype, pin_memory=True)
-        hdv = torch.empty(dv.shape, dtype=dv.dtype, pin_memory=True)
+        outs = (R.o, R.dq, R.dk, R.dv)
+        houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-        d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdk, hdv))
+        d2h = sum(t.numel() * t.element_size() for t in houts)
         barrier(world)
         torch.cuda.synchronize(dev)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        e0.record(R.stream)
         for _ in range(args.e2e_steps):
-            for src, dst in ((hq, qd), (hk, kd), (hv, vd), (hdo, dod)):
+            for src, dst in zip((hq, hk, hv, hdo), dev_tensors):
                 dst.copy_(src, non_blocking=True)
-            step()
-            for src, dst in ((o, ho), (dq, hdq), (dk, hdk), (dv, hdv)):
+            R.step()
+            for src, dst in zip(outs, houts):
                 dst.copy_(src, non_blocking=True)
-        e1.record(stream)
+        e1.record(R.stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
-        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        e2e = {"value": w.flops() * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "path": main_path}
 
     if rank != 0:
         if world > 1:
             torch.distributed.destroy_process_group()
         return
 
-    fwd_flops = 4.0 * w.d * w.Hq * w.pairs()
-    bwd_flops = 10.0 * w.d * w.Hq * w.pairs()
-    # algorithmic tensor work of each attention kernel (per visible pair and
-    # query head): forward S and PV = 4 d; dK/dV kernel S, dP, dV, dK = 8 d;
-    # dQ kernel S, dP, dQ = 6 d
-    kern_flops = {"fwd_kernel": 4.0, "dkdv_kernel": 8.0, "dq_kernel": 6.0}
-    dom = max(kern_flops, key=lambda n: kern_ms[n])
-    dom_flops = kern_flops[dom] * w.d * w.Hq * w.pairs()
-    achieved = dom_flops / (kern_ms[dom] * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": dom,
-                "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)",
-                "kernels_ms": kern_ms,
-                "kernels_tflops": {n: kern_flops[n] * w.d * w.Hq * w.pairs() / (kern_ms[n] * 1e-3) / 1e12
-                                   for n in kern_flops},
-                "fwd": {"ms": fwd_ms, "tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12},
-                "bwd": {"ms": bwd_ms, "tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12}}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         v_cpu, cores, text, _ = cpu_oracle_sample(w, target_s=15.0)
         cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": text}
+    head = results[main_path]
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {**w.describe(), "path": "bf16", "parallelism": f"replicas x{world}",
+        "metric": METRIC, "value": head["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if main_path == "bf16" else "e4m3/e8m0", "data": "synthetic",
+        "config": {**w.describe(), "path": main_path, "parallelism": f"replicas x{world}",
                    "l2": f"inputs {sum(t.numel() * 2 for t in (q, k, v, do)) / 1e9:.2f} GB > 126 MB L2, no flush"},
-        "pct_of_dense_bf16_peak": 100.0 * (value / world) / DENSE_BF16_TFLOPS,
-        "pct_of_measured_bf16_peak": 100.0 * (value / world) / peaks["bf16_tflops"],
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "pct_of_dense_bf16_peak": head["pct_of_dense_peak"] if main_path == "bf16" else None,
+        "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
         "clocks": clk, "status_ok": st_ok,
     }
+    for p in paths[1:]:
+        line[p] = results[p]
     print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
