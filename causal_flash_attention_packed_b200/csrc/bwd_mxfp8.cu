@@ -535,19 +535,31 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
 // dK, dV
 // ---------------------------------------------------------------------------
 namespace kvk {
-constexpr int kThreads = 320, kLoad = 8, kMma = 9;
-// per item: K^tb, K^pt, V^tb, V^pt codes; per query tile (one stage): Q^pt,
-// Q^tb, dO^pt, dO^tb codes, lse*log2e[128], D[128]; P~T and dS~T codes
+// warps 0-7: one thread per key row (warpgroup w on query columns
+// [64w, 64w + 64)); warp 8: K/V, Q^pt, dO^pt, lse and D loads; warp 9: MMA
+// issue; warp 10: dO^tb and Q^tb loads
+constexpr int kThreads = 352, kLoadA = 8, kMma = 9, kLoadB = 10;
+// per item: K^tb, K^pt, V^tb, V^pt codes; per query tile one buffer per
+// operand (Q^pt, dO^pt, dO^tb, Q^tb codes), each released as soon as its last
+// MMA has read it; P~T and dS~T codes; lse*log2e[128] and D[128] of the query
+// tile in two buffers
 constexpr int oKtb = 0, oKpt = oKtb + kCode, oVtb = oKpt + kCode, oVpt = oVtb + kCode;
-constexpr int oQpt = oVpt + kCode, oQtb = oQpt + kCode, oDOpt = oQtb + kCode, oDOtb = oDOpt + kCode;
-constexpr int oP = oDOtb + kCode, oDS = oP + kCode;
-constexpr int oLse = oDS + kCode, oSf = oLse + 1024;
-// scale blocks: 0 Ktb, 1 Kpt, 2 Vtb, 3 Vpt, 4 Qpt, 5 dOpt, 6 dOtb(dv), 7 Qtb(dk), 8 P, 9 dS
+constexpr int oQpt = oVpt + kCode, oDOpt = oQpt + kCode, oDOtb = oDOpt + kCode, oQtb = oDOtb + kCode;
+constexpr int oP = oQtb + kCode, oDS = oP + kCode;
+constexpr int oAux = oDS + kCode;
+constexpr int oSf = oAux + 2 * 1024;
+// scale blocks: 0 Ktb, 1 Kpt, 2 Vtb, 3 Vpt, 4 Qpt, 5 dOpt, 6 dOtb (channel rows), 7 Qtb (channel rows), 8 P, 9 dS
 constexpr int kNumSf = 10;
 constexpr int oBars = oSf + kNumSf * kSfBlk;
-constexpr int kNumBars = 11;
+// operand buffers, in the order the MMAs release them
+constexpr int kQpt = 0, kDOpt = 1, kDOtb = 2, kQtb = 3;
+constexpr int bKvFull = 0, bKvEmpty = 1, bOpFull = 2, bOpEmpty = 6, bAuxFull = 10, bAuxEmpty = 12, bSFull = 14,
+              bSFree = 15, bPFull = 16, bPEmpty = 17, bDsFull = 18, bDsEmpty = 19, bAccFull = 20, bAccFree = 21,
+              bFin = 22, kNumBars = 23;
 constexpr int kSmem = oBars + kNumBars * 8 + 16 + 1024;
-constexpr uint32_t tSP = 0, tDV = 128, tDK = 256;
+// TMEM: one 128-column region that holds S^T and dP^T in turn (each read out
+// into registers and released before the next), dV, dK, scale factors
+constexpr uint32_t tSD = 0, tDV = 128, tDK = 256;
 constexpr uint32_t tSfKtb = 384, tSfKpt = 388, tSfVtb = 392, tSfVpt = 396, tSfQpt = 400, tSfDOpt = 404, tSfP = 408,
                    tSfDS = 412, tSfDOtb = 416, tSfQtb = 420;
 }  // namespace kvk
@@ -564,16 +576,21 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   uint8_t* sf = smem + oSf;
   auto sfb = [&](int i) { return sf + i * kSfBlk; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oBars);
-  uint64_t* kv_full = bars + 0;
-  uint64_t* kv_empty = bars + 1;
-  uint64_t* st_full = bars + 2;
-  uint64_t* st_empty = bars + 3;
-  uint64_t* s_full = bars + 4;
-  uint64_t* s_read = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* acc_full = bars + 7;
-  uint64_t* acc_free = bars + 8;
-  uint64_t* fin = bars + 9;
+  uint64_t* kv_full = bars + bKvFull;
+  uint64_t* kv_empty = bars + bKvEmpty;
+  uint64_t* op_full = bars + bOpFull;
+  uint64_t* op_empty = bars + bOpEmpty;
+  uint64_t* aux_full = bars + bAuxFull;
+  uint64_t* aux_empty = bars + bAuxEmpty;
+  uint64_t* s_full = bars + bSFull;
+  uint64_t* s_free = bars + bSFree;
+  uint64_t* p_full = bars + bPFull;
+  uint64_t* p_empty = bars + bPEmpty;
+  uint64_t* ds_full = bars + bDsFull;
+  uint64_t* ds_empty = bars + bDsEmpty;
+  uint64_t* acc_full = bars + bAccFull;
+  uint64_t* acc_free = bars + bAccFree;
+  uint64_t* fin = bars + bFin;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -581,11 +598,20 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 32);
     mbar_init(kv_empty, 1);
-    mbar_init(st_full, 32);
-    mbar_init(st_empty, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(op_full + i, 32);  // lane 0's expect_tx arrive + 31 lanes after their scale stores
+      mbar_init(op_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(aux_full + i, 32);
+      mbar_init(aux_empty + i, 256);
+    }
     mbar_init(s_full, 1);
-    mbar_init(s_read, 256);
+    mbar_init(s_free, 256);
     mbar_init(p_full, 256);
+    mbar_init(p_empty, 1);
+    mbar_init(ds_full, 256);
+    mbar_init(ds_empty, 1);
     mbar_init(acc_full, 1);
     mbar_init(acc_free, 256);
     mbar_init(fin, 1);
@@ -613,9 +639,25 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     k0 = s + 128 * v;
     nq = (e - s + 127) / 128;
   };
+  // one operand buffer of query tile t: wait until the MMAs of tile t - 1 released
+  // it, store its scale block, then copy the codes
+  auto load_op = [&](int op, uint32_t t, const CUtensorMap* tm, int h, int q0, const uint4& sfw, int where) {
+    if (t > 0 && !warp_wait(op_empty + op, (t - 1) & 1, wd, where)) return false;
+    reinterpret_cast<uint4*>(sfb(4 + op))[lane] = sfw;
+    fence_proxy_async_smem();
+    const int off = op == kQpt ? oQpt : op == kDOpt ? oDOpt : op == kDOtb ? oDOtb : oQtb;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(op_full + op, kCode);
+      tma_load_3d(smem + off, tm, op_full + op, 0, h, q0);
+    } else {
+      mbar_arrive(op_full + op);
+    }
+    return true;
+  };
 
-  if (warp == kLoad) {
-    uint32_t st_it = 0;
+  if (warp == kLoadA) {
+    // ------------------------------------------------- K, V; Q^pt, dO^pt; lse, D
+    uint32_t t = 0;
     int unit_i = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
@@ -637,46 +679,66 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
         mbar_arrive(kv_full);
       }
       for (int h = g * G; h < (g + 1) * G && ok; ++h) {
-        for (int m = v; m < nq; ++m, ++st_it) {
-          if (st_it > 0 && !warp_wait(st_empty, (st_it - 1) & 1, wd, 82)) { ok = false; break; }
+        for (int m = v; m < nq; ++m, ++t) {
           const int q0 = s + 128 * m;
-          reinterpret_cast<uint4*>(sfb(4))[lane] = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
-          reinterpret_cast<uint4*>(sfb(5))[lane] = pt_rows(p.do_spt, q0, lane, p.T, p.Hq, h);
-          reinterpret_cast<uint4*>(sfb(6))[lane] = tb_channel_rows(p.do_stb, s, e, doc, 4 * m, p.Hq, h);
-          reinterpret_cast<uint4*>(sfb(7))[lane] = tb_channel_rows(p.q_stb, s, e, doc, 4 * m, p.Hq, h);
-          float* lse2 = reinterpret_cast<float*>(smem + oLse);
-          float* dl = lse2 + 128;
+          // all global reads of the tile first, so that their latencies overlap
+          const uint4 sq = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
+          const uint4 sdo = pt_rows(p.do_spt, q0, lane, p.T, p.Hq, h);
+          float l4[4], d4[4];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const int i = q0 + lane * 4 + r;
             const bool in = i < e;  // queries past the document end get P = 0 (lse2 = +inf)
-            lse2[lane * 4 + r] = in ? p.lse[(size_t)h * p.T + i] * kLog2e : INFINITY;
-            dl[lane * 4 + r] = in ? p.delta[(size_t)h * p.T + i] : 0.f;
+            l4[r] = in ? p.lse[(size_t)h * p.T + i] * kLog2e : INFINITY;
+            d4[r] = in ? p.delta[(size_t)h * p.T + i] : 0.f;
           }
-          fence_proxy_async_smem();
-          if (lane == 0) {
-            mbar_arrive_expect_tx(st_full, 4 * kCode);
-            tma_load_3d(smem + oQpt, &tm_qpt, st_full, 0, h, q0);
-            tma_load_3d(smem + oQtb, &tm_qtb, st_full, 0, h, q0);
-            tma_load_3d(smem + oDOpt, &tm_dopt, st_full, 0, h, q0);
-            tma_load_3d(smem + oDOtb, &tm_dotb, st_full, 0, h, q0);
-          } else {
-            mbar_arrive(st_full);
-          }
+          const int ab = t & 1;
+          if (t >= 2 && !warp_wait(aux_empty + ab, ((t >> 1) - 1) & 1, wd, 82)) { ok = false; break; }
+          float* lse2 = reinterpret_cast<float*>(smem + oAux + ab * 1024);
+          reinterpret_cast<float4*>(lse2)[lane] = make_float4(l4[0], l4[1], l4[2], l4[3]);
+          reinterpret_cast<float4*>(lse2 + 128)[lane] = make_float4(d4[0], d4[1], d4[2], d4[3]);
+          mbar_arrive(aux_full + ab);
+          if (!load_op(kQpt, t, &tm_qpt, h, q0, sq, 83)) { ok = false; break; }
+          if (!load_op(kDOpt, t, &tm_dopt, h, q0, sdo, 84)) { ok = false; break; }
         }
       }
     }
     if (lane == 0) {
       if (unit_i > 0) drain_wait(kv_full, (unit_i - 1) & 1, p.timeout_ns);
-      if (st_it > 0) drain_wait(st_full, (st_it - 1) & 1, p.timeout_ns);
+      if (t > 0) {
+        drain_wait(op_full + kQpt, (t - 1) & 1, p.timeout_ns);
+        drain_wait(op_full + kDOpt, (t - 1) & 1, p.timeout_ns);
+      }
+    }
+  } else if (warp == kLoadB) {
+    // ------------------------------------------------- dO^tb, Q^tb
+    uint32_t t = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
+      int doc, s, e, g, v, k0, nq;
+      decode(w, doc, s, e, g, v, k0, nq);
+      for (int h = g * G; h < (g + 1) * G && ok; ++h) {
+        for (int m = v; m < nq; ++m, ++t) {
+          const int q0 = s + 128 * m;
+          const uint4 sdo = tb_channel_rows(p.do_stb, s, e, doc, 4 * m, p.Hq, h);
+          const uint4 sq = tb_channel_rows(p.q_stb, s, e, doc, 4 * m, p.Hq, h);
+          if (!load_op(kDOtb, t, &tm_dotb, h, q0, sdo, 85)) { ok = false; break; }
+          if (!load_op(kQtb, t, &tm_qtb, h, q0, sq, 86)) { ok = false; break; }
+        }
+      }
+    }
+    if (lane == 0 && t > 0) {
+      drain_wait(op_full + kDOtb, (t - 1) & 1, p.timeout_ns);
+      drain_wait(op_full + kQtb, (t - 1) & 1, p.timeout_ns);
     }
   } else if (warp == kMma) {
+    // ------------------------------------------------- MMA issue
     if (lane == 0) {
       const uint32_t aKtb = smem_u32(smem + oKtb), aKpt = smem_u32(smem + oKpt), aVtb = smem_u32(smem + oVtb),
                      aVpt = smem_u32(smem + oVpt), aQpt = smem_u32(smem + oQpt), aQtb = smem_u32(smem + oQtb),
                      aDOpt = smem_u32(smem + oDOpt), aDOtb = smem_u32(smem + oDOtb), aP = smem_u32(smem + oP),
                      aDS = smem_u32(smem + oDS), aSf = smem_u32(sf);
-      uint32_t st_it = 0, sr_cnt = 0, p_cnt = 0;
+      uint32_t t = 0, s_uses = 0;
       int unit_i = 0;
       bool ok = true;
       auto mx_kk = [&](uint32_t dcol, uint32_t a, uint32_t b, uint32_t sfa, uint32_t sfbc, bool b_mn,
@@ -688,70 +750,100 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
                       idesc_mxf8(128, 128, b_mn, kk, kk), (tmem + sfa) | ((uint32_t)kk << 30),
                       (tmem + sfbc) | ((uint32_t)kk << 30), (acc_first || kk > 0) ? 1u : 0u);
       };
-      auto wait_read = [&]() {
-        const bool r = mbar_wait(s_read, sr_cnt & 1, wd, 83);
-        ++sr_cnt;
+      // the S/dP region: wait until the compute warps have read out its previous use
+      auto region = [&]() {
+        if (s_uses > 0 && !mbar_wait(s_free, (s_uses - 1) & 1, wd, 87)) return false;
         tc_fence_after();
-        return r;
+        return true;
+      };
+      auto region_done = [&]() {
+        tc_commit(s_full);
+        ++s_uses;
+      };
+      auto wait_op = [&](int op, uint32_t tt, int where) {
+        if (!mbar_wait(op_full + op, tt & 1, wd, where)) return false;
+        tc_fence_after();
+        return true;
+      };
+      // S^T of tile tt with token-block K (every key block of the tile)
+      auto s_tb = [&](uint32_t tt) {
+        if (!wait_op(kQpt, tt, 88)) return false;
+        tmem_cp_sf(tmem + tSfQpt, aSf + 4 * kSfBlk);
+        if (!region()) return false;
+        mx_kk(tSD, aKtb, aQpt, tSfKtb, tSfQpt, false, false);
+        region_done();
+        return true;
       };
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
         int doc, s, e, g, v, k0, nq;
         decode(w, doc, s, e, g, v, k0, nq);
-        if (!mbar_wait(kv_full, unit_i & 1, wd, 84)) break;
-        if (unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 85)) break;
+        if (!mbar_wait(kv_full, unit_i & 1, wd, 89)) break;
+        if (unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 90)) break;
         tc_fence_after();
         tmem_cp_sf(tmem + tSfKtb, aSf + 0 * kSfBlk);
         tmem_cp_sf(tmem + tSfKpt, aSf + 1 * kSfBlk);
         tmem_cp_sf(tmem + tSfVtb, aSf + 2 * kSfBlk);
         tmem_cp_sf(tmem + tSfVpt, aSf + 3 * kSfBlk);
-        bool first = true;
-        for (int h = g * G; h < (g + 1) * G && ok; ++h) {
-          for (int m = v; m < nq; ++m, ++st_it) {
-            const bool diag = m == v;
-            if (!mbar_wait(st_full, st_it & 1, wd, 86)) { ok = false; break; }
-            tc_fence_after();
-            tmem_cp_sf(tmem + tSfQpt, aSf + 4 * kSfBlk);
-            tmem_cp_sf(tmem + tSfDOpt, aSf + 5 * kSfBlk);
-            // S^T (token-block K), then on the diagonal the per-token K
-            mx_kk(tSP, aKtb, aQpt, tSfKtb, tSfQpt, false, false);
-            tc_commit(s_full);
-            if (!wait_read()) { ok = false; break; }
-            if (diag) {
-              mx_kk(tSP, aKpt, aQpt, tSfKpt, tSfQpt, false, false);
-              tc_commit(s_full);
-              if (!wait_read()) { ok = false; break; }
-            }
-            // P~T is in shared memory: dV += P~T dO~tb
-            tmem_cp_sf(tmem + tSfP, aSf + 8 * kSfBlk);
-            tmem_cp_sf(tmem + tSfDOtb, aSf + 6 * kSfBlk);
-            mx_kk(tDV, aP, aDOtb, tSfP, tSfDOtb, true, !first);
-            // dP^T (token-block V), then on the diagonal the per-token V
-            mx_kk(tSP, aVtb, aDOpt, tSfVtb, tSfDOpt, false, false);
-            tc_commit(s_full);
-            if (diag) {
-              if (!wait_read()) { ok = false; break; }
-              mx_kk(tSP, aVpt, aDOpt, tSfVpt, tSfDOpt, false, false);
-              tc_commit(s_full);
-            }
-            if (!mbar_wait(p_full, p_cnt & 1, wd, 87)) { ok = false; break; }
-            ++p_cnt;
-            tc_fence_after();
-            tmem_cp_sf(tmem + tSfDS, aSf + 9 * kSfBlk);
-            tmem_cp_sf(tmem + tSfQtb, aSf + 7 * kSfBlk);
-            mx_kk(tDK, aDS, aQtb, tSfDS, tSfQtb, true, !first);
-            first = false;
-            tc_commit(st_empty);
+        const int nt = nq - v, R = G * nt;
+        bool ahead = false;  // S^T (token-block K) of tile t already issued
+        for (int r = 0; r < R; ++r, ++t) {
+          const bool diag = (r % nt) == 0;  // first query tile of each head: the diagonal tile
+          const bool last = r == R - 1;
+          if (!ahead && !s_tb(t)) { ok = false; break; }
+          if (diag) {
+            // diagonal tile: S^T again with the per-token K; the compute warps
+            // take its diagonal 32x32 blocks
+            if (!region()) { ok = false; break; }
+            mx_kk(tSD, aKpt, aQpt, tSfKpt, tSfQpt, false, false);
+            region_done();
           }
+          tc_commit(op_empty + kQpt);
+          // dP^T (token-block V), on the diagonal tile then the per-token V
+          if (!wait_op(kDOpt, t, 91)) { ok = false; break; }
+          tmem_cp_sf(tmem + tSfDOpt, aSf + 5 * kSfBlk);
+          if (!region()) { ok = false; break; }
+          mx_kk(tSD, aVtb, aDOpt, tSfVtb, tSfDOpt, false, false);
+          region_done();
+          if (diag) {
+            if (!region()) { ok = false; break; }
+            mx_kk(tSD, aVpt, aDOpt, tSfVpt, tSfDOpt, false, false);
+            region_done();
+          }
+          tc_commit(op_empty + kDOpt);
+          if (last) tc_commit(kv_empty);  // the item's last read of K and V has been issued
+          // dV += P~T dO~tb
+          if (!mbar_wait(p_full, t & 1, wd, 92)) { ok = false; break; }
+          if (!wait_op(kDOtb, t, 93)) { ok = false; break; }
+          tmem_cp_sf(tmem + tSfP, aSf + 8 * kSfBlk);
+          tmem_cp_sf(tmem + tSfDOtb, aSf + 6 * kSfBlk);
+          mx_kk(tDV, aP, aDOtb, tSfP, tSfDOtb, true, r > 0);
+          tc_commit(p_empty);
+          tc_commit(op_empty + kDOtb);
+          // the next tile's S^T goes ahead of dK, so that it is ready when the
+          // compute warps finish dS~ of this tile
+          ahead = false;
+          if (!last) {
+            if (!s_tb(t + 1)) { ok = false; break; }
+            ahead = true;
+          }
+          // dK += dS~T Q~tb
+          if (!mbar_wait(ds_full, t & 1, wd, 94)) { ok = false; break; }
+          if (!wait_op(kQtb, t, 95)) { ok = false; break; }
+          tmem_cp_sf(tmem + tSfDS, aSf + 9 * kSfBlk);
+          tmem_cp_sf(tmem + tSfQtb, aSf + 7 * kSfBlk);
+          mx_kk(tDK, aDS, aQtb, tSfDS, tSfQtb, true, r > 0);
+          tc_commit(ds_empty);
+          tc_commit(op_empty + kQtb);
         }
         if (!ok) break;
         tc_commit(acc_full);
-        tc_commit(kv_empty);
       }
       tc_commit(fin);
       drain_wait(fin, 0, p.timeout_ns);
     }
-  } else {
-    // one thread per key row; warpgroup wg on query quarters 2 wg, 2 wg + 1
+  } else if (warp < 8) {
+    // ------------------------------------------------- P~T, dS~T
+    // one thread per key row; warpgroup wg on query columns [64 wg, 64 wg + 64)
     const int wg = warp >> 2, quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lb = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -759,119 +851,118 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     uint8_t* sDS = smem + oDS;
     uint8_t* sfP = sfb(8);
     uint8_t* sfDS = sfb(9);
-    const float* lse2 = reinterpret_cast<const float*>(smem + oLse);
-    const float* dl = lse2 + 128;
-    uint32_t s_cnt = 0;
+    // this row's diagonal query block (columns [32 quarter, 32 quarter + 32))
+    // lies in this warpgroup's half iff quarter >> 1 == wg
+    const bool own_diag = (quarter >> 1) == wg;
+    uint32_t s_cnt = 0, t = 0;
     int unit_i = 0;
     bool ok = true;
-    auto wait_s = [&]() {
-      const bool r = warp_wait(s_full, s_cnt & 1, wd, 88);
+    auto take = [&]() {
+      const bool r = warp_wait(s_full, s_cnt & 1, wd, 96);
       ++s_cnt;
       tc_fence_after();
       return r;
     };
-    uint32_t st_cnt = 0;
+    auto release = [&]() {
+      tc_fence_before();
+      mbar_arrive(s_free);
+    };
+    // the 64 values of this row in this warpgroup's half of the region
+    auto read_half = [&](float (&x)[64]) {
+      uint32_t a[32], b[32];
+      tmem_ld32(lb + tSD + 64 * wg, a);
+      tmem_ld32(lb + tSD + 64 * wg + 32, b);
+      tmem_wait_ld(a);
+      tmem_wait_ld(b);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        x[c] = __uint_as_float(a[c]);
+        x[32 + c] = __uint_as_float(b[c]);
+      }
+    };
+    // the diagonal block from the per-token phase replaces the token-block values
+    auto read_diag = [&](float (&x)[64]) {
+      if (!own_diag) return;
+      uint32_t a[32];
+      tmem_ld32(lb + tSD + 32 * quarter, a);
+      tmem_wait_ld(a);
+      if (quarter & 1) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[32 + c] = __uint_as_float(a[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(a[c]);
+      }
+    };
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
       int doc, s, e, g, v, k0, nq;
       decode(w, doc, s, e, g, v, k0, nq);
       const int j = k0 + row;
       for (int h = g * G; h < (g + 1) * G && ok; ++h) {
-        for (int m = v; m < nq; ++m, ++st_cnt) {
+        for (int m = v; m < nq; ++m, ++t) {
           const bool diag = m == v;
-          const int i0 = s + 128 * m;  // query index of column 0
-          // the stage's LSE and D were written by the load warp: wait for the
-          // stage directly (not only through the MMA thread's commits)
-          if (!warp_wait(st_full, st_cnt & 1, wd, 90)) { ok = false; break; }
-          // ---- S^T -> P (kept in registers), P~T into shared memory
-          if (!wait_s()) { ok = false; break; }
+          const int ab = t & 1;
+          if (!warp_wait(aux_full + ab, (t >> 1) & 1, wd, 97)) { ok = false; break; }
+          const float* lse2 = reinterpret_cast<const float*>(smem + oAux + ab * 1024) + 64 * wg;
+          const float* dl = lse2 + 128;
+          // ---- S^T -> P, P~T into shared memory
           float pr[64];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qq = 2 * wg + u;
-            uint32_t rs[32];
-            tmem_ld32(lb + tSP + 32 * qq, rs);
-            tmem_wait_ld(rs);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) pr[32 * u + c] = __uint_as_float(rs[c]);
-          }
+          if (!take()) { ok = false; break; }
+          read_half(pr);
+          release();
           if (diag) {
-            tc_fence_before();
-            mbar_arrive(s_read);
-            if (!wait_s()) { ok = false; break; }
-            if ((quarter >> 1) == wg) {  // this row's diagonal query block lies in our half
-              uint32_t rs[32];
-              tmem_ld32(lb + tSP + 32 * quarter, rs);
-              tmem_wait_ld(rs);
-              const int u = quarter & 1;
-#pragma unroll
-              for (int c = 0; c < 32; ++c) pr[32 * u + c] = __uint_as_float(rs[c]);
-            }
+            if (!take()) { ok = false; break; }
+            read_diag(pr);
+            release();
           }
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qq = 2 * wg + u;
+          for (int c = 0; c < 64; ++c) {
+            // on the diagonal tile query column 64 wg + c is visible iff it is >= the key row
+            const bool vis = !diag || (64 * wg + c >= row);
+            pr[c] = vis ? fast_exp2(pr[c] * p.scale_log2 - lse2[c]) : 0.f;
+          }
+          if (t > 0 && !warp_wait(p_empty, (t - 1) & 1, wd, 98)) { ok = false; break; }
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const int cc = 32 * qq + c;
-              const bool vis = !diag || (cc >= row);  // query i0 + cc >= key j (same tile base)
-              pr[32 * u + c] = vis ? fast_exp2(pr[32 * u + c] * p.scale_log2 - lse2[cc]) : 0.f;
-            }
+          for (int u = 0; u < 2; ++u) {
             float blk[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) blk[c] = pr[32 * u + c];
             uint32_t cw[8];
             const uint32_t sb = quant32(blk, p.rule, cw);
-            store_codes32(sP, row, 2 * qq, cw);
-            sfP[(row & 31) * 16 + (row >> 5) * 4 + qq] = (uint8_t)sb;
+            store_codes32(sP, row, 2 * (2 * wg + u), cw);
+            sfP[(row & 31) * 16 + (row >> 5) * 4 + 2 * wg + u] = (uint8_t)sb;
           }
           fence_proxy_async_smem();
-          tc_fence_before();
-          mbar_arrive(s_read);
+          mbar_arrive(p_full);
           // ---- dP^T -> dS~T into shared memory
-          if (!wait_s()) { ok = false; break; }
           float dp[64];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qq = 2 * wg + u;
-            uint32_t rd[32];
-            tmem_ld32(lb + tSP + 32 * qq, rd);
-            tmem_wait_ld(rd);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) dp[32 * u + c] = __uint_as_float(rd[c]);
-          }
+          if (!take()) { ok = false; break; }
+          read_half(dp);
+          release();
           if (diag) {
-            tc_fence_before();
-            mbar_arrive(s_read);
-            if (!wait_s()) { ok = false; break; }
-            if ((quarter >> 1) == wg) {
-              uint32_t rd[32];
-              tmem_ld32(lb + tSP + 32 * quarter, rd);
-              tmem_wait_ld(rd);
-              const int u = quarter & 1;
-#pragma unroll
-              for (int c = 0; c < 32; ++c) dp[32 * u + c] = __uint_as_float(rd[c]);
-            }
+            if (!take()) { ok = false; break; }
+            read_diag(dp);
+            release();
           }
+          if (t > 0 && !warp_wait(ds_empty, (t - 1) & 1, wd, 99)) { ok = false; break; }
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int qq = 2 * wg + u;
             float blk[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) blk[c] = pr[32 * u + c] * (dp[32 * u + c] - dl[32 * qq + c]);
+            for (int c = 0; c < 32; ++c) blk[c] = pr[32 * u + c] * (dp[32 * u + c] - dl[32 * u + c]);
             uint32_t cw[8];
             const uint32_t sb = quant32(blk, p.rule, cw);
-            store_codes32(sDS, row, 2 * qq, cw);
-            sfDS[(row & 31) * 16 + (row >> 5) * 4 + qq] = (uint8_t)sb;
+            store_codes32(sDS, row, 2 * (2 * wg + u), cw);
+            sfDS[(row & 31) * 16 + (row >> 5) * 4 + 2 * wg + u] = (uint8_t)sb;
           }
           fence_proxy_async_smem();
-          tc_fence_before();
-          mbar_arrive(p_full);
-          (void)i0;
+          mbar_arrive(ds_full);
+          mbar_arrive(aux_empty + ab);
         }
       }
       if (!ok) break;
       // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK * scale
-      if (!warp_wait(acc_full, unit_i & 1, wd, 89)) break;
+      if (!warp_wait(acc_full, unit_i & 1, wd, 100)) break;
       tc_fence_after();
       const bool valid = j < e;
       const uint32_t acc = lb + (wg ? tDK : tDV);
@@ -879,10 +970,10 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
       const float mul = wg ? p.scale : 1.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t t[32];
-        tmem_ld32(acc + 32 * c, t);
-        tmem_wait_ld(t);
-        if (valid) store_row32(out, ((size_t)j * p.Hkv + g) * 128 + 32 * c, t, mul, p.grad_bf16);
+        uint32_t tt[32];
+        tmem_ld32(acc + 32 * c, tt);
+        tmem_wait_ld(tt);
+        if (valid) store_row32(out, ((size_t)j * p.Hkv + g) * 128 + 32 * c, tt, mul, p.grad_bf16);
       }
       tc_fence_before();
       mbar_arrive(acc_free);
