@@ -140,7 +140,7 @@ FwdLayout fwd_layout(const fapk_problem_t* P) {
 //  MXFP8 path, instead of the fp16 copies: the quantiser's forms of dO.
 struct BwdLayout {
   SchedLayout kv, q;
-  size_t delta, q16, k16, do16, total;
+  size_t delta, q16, k16, do16, nl2, total;
   size_t do_vtb, do_stb, do_vpt, do_spt;
 };
 BwdLayout bwd_layout(const fapk_problem_t* P) {
@@ -163,7 +163,8 @@ BwdLayout bwd_layout(const fapk_problem_t* P) {
   L.q16 = after_delta;
   L.k16 = align_up(L.q16 + 2 * nq);
   L.do16 = align_up(L.k16 + 2 * nk);
-  L.total = align_up(L.do16 + 2 * nq);
+  L.nl2 = align_up(L.do16 + 2 * nq);
+  L.total = align_up(L.nl2 + sizeof(float) * (size_t)P->Hq * (size_t)P->T);
   return L;
 }
 
@@ -232,12 +233,24 @@ bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16) {
+bool make_tmap_flat_f32(CUtensorMap* map, const float* base, long long n, int box) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[1] = {(cuuint64_t)n};
+  const cuuint64_t strides[1] = {4};  // unused for a 1-D map
+  const cuuint32_t boxd[1] = {(cuuint32_t)box};
+  const cuuint32_t estr[1] = {1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<float*>(base), dims, strides, boxd, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
-  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
              const_cast<void*>(base), dims, strides, box, estr,
@@ -441,6 +454,7 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   a.do16 = static_cast<char*>(ws) + L.do16;
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.delta = reinterpret_cast<float*>(static_cast<char*>(ws) + L.delta);
+  a.nl2 = reinterpret_cast<float*>(static_cast<char*>(ws) + L.nl2);
   a.cu = P->cu_seqlens_dev;
   a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.d = P->d;
   a.scale = P->scale;

@@ -89,14 +89,16 @@ __device__ __forceinline__ uint32_t split_a_col(uint32_t base, int kk) {
 // ---------------------------------------------------------------------------
 // O is taken as o + o_resid, the forward's bf16 output plus its rounding
 // residual (about 16 significant bits).
-// The same pass writes the fp16 copies of dO and Q used by the gradient MMAs.
+// The same pass writes the fp16 copies of dO and Q used by the gradient MMAs
+// and -LSE log2(e), the exponent offset of P in base 2.
 template <int D>
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o,
                                                     const __nv_bfloat16* __restrict__ o_resid,
                                                     const __nv_bfloat16* __restrict__ dout,
                                                     const __nv_bfloat16* __restrict__ q,
                                                     uint4* __restrict__ do16, uint4* __restrict__ q16,
-                                                    float* __restrict__ delta, int T, int Hq,
+                                                    const float* __restrict__ lse, float* __restrict__ delta,
+                                                    float* __restrict__ nl2, int T, int Hq,
                                                     DeviceStatus* status) {
   constexpr int TPR = D / 8;  // threads per (token, head) row
   const long long row = (long long)blockIdx.x * (256 / TPR) + threadIdx.x / TPR;
@@ -135,6 +137,7 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
   if (row < (long long)T * Hq && c8 == 0) {
     const long long t = row / Hq, h = row % Hq;
     delta[h * T + t] = acc;
+    nl2[h * T + t] = -(lse[h * T + t] * kLog2e);
   }
   if (!__all_sync(0xFFFFFFFFu, in_range) && (threadIdx.x & 31) == 0) record_error(status, kStatusRange, 41);
 }
@@ -145,6 +148,7 @@ struct BwdParams {
   const int* n_items;
   const float* lse;
   const float* delta;
+  const float* nl2;  // -LSE log2(e), [Hq][T]
   void* out0;  // dkdv: dk;  dq: dq
   void* out1;  // dkdv: dv
   DeviceStatus* status;
@@ -178,20 +182,34 @@ __device__ __forceinline__ void store_row32(void* base, size_t elem_off, const u
 // ---------------------------------------------------------------------------
 // 2. dK, dV
 // ---------------------------------------------------------------------------
+// TMEM holds dV, dK, one 128-column region that S^T and dP^T of a query tile
+// use in turn, and one region for the tile's P^T and dS^T (fp16).  The compute
+// warps read S^T (then dP^T) out into registers and release the region at
+// once, so the MMAs run in the order S(t), dP(t), dV(t), S(t+1), dK(t),
+// dP(t+1), ... and the tensor pipe has the next independent MMA group queued
+// while the exponentials of a tile are computed.  16 compute warps:
+// warpgroup wg owns query columns [32 wg, 32 wg + 32) of every tile.
+constexpr int kKvThreads = 576;
+constexpr int kKvLoadWarp = 16;
+constexpr int kKvMmaWarp = 17;
+constexpr int kKvCompute = 512;
+
 template <int D>
 struct KvCfg : Geo<D> {
-  static constexpr int kStages = (D == 128) ? 2 : 3;
-  static constexpr int kStageBytes = 2 * Geo<D>::kTileBytes + 1024;  // Q, dO, LSE*log2e[128], D[128]
+  static constexpr int kStages = 2;
+  static constexpr int kStageBytes = 2 * Geo<D>::kTileBytes + 1024;  // Q, dO, nl2[128], D[128]
+  static constexpr int kNl2Off = 2 * Geo<D>::kTileBytes, kDeltaOff = kNl2Off + 512;
   static constexpr int kSmemTiles = 2 * Geo<D>::kTileBytes + kStages * kStageBytes;
-  // TMEM: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D)
-  static constexpr uint32_t kS = 0, kDP = 128, kDV = 256, kDK = 256 + D;
-  // bars: kv_full, kv_empty, st_full[S], st_empty[S], s_full, p_full, acc_full, acc_free, fin
-  static constexpr int kNumBars = 2 + 2 * kStages + 5;
+  // TMEM: dV [0,D), dK [128,128+D), S^T / dP^T [256,384), P^T [384,448), dS^T [448,512)
+  static constexpr uint32_t kDV = 0, kDK = 128, kSD = 256, kP = 384, kDS = 448;
+  // bars: kv_full, kv_empty, st_full[S], st_empty[S], s_full, s_free, p_ready, ds_ready,
+  //       dv_done, dk_done, acc_full, acc_free, fin
+  static constexpr int kNumBars = 2 + 2 * kStages + 9;
   static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
 };
 
 struct KvItem {
-  int s, e, v, g, k0, nq;  // k0: first key of the tile; nq: query tiles v..nq-1
+  int s, e, v, g, k0, nq;  // k0: first key of the tile; query tiles v..nq-1
 };
 
 __device__ __forceinline__ KvItem kv_decode(const BwdParams& p, int w) {
@@ -206,8 +224,17 @@ __device__ __forceinline__ KvItem kv_decode(const BwdParams& p, int w) {
   return it;
 }
 
+// 32 values of one TMEM row -> registers.
+__device__ __forceinline__ void ld_row32(uint32_t taddr, float (&x)[32]) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+  tmem_wait_ld(r);
+#pragma unroll
+  for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(r[c]);
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kKvThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const BwdParams p) {
@@ -216,17 +243,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = smem + C::kTileBytes;
-  uint8_t* sStage = smem + 2 * C::kTileBytes;  // per stage: Q tile, dO tile, lse2[128], delta[128]
+  uint8_t* sStage = smem + 2 * C::kTileBytes;  // per stage: Q tile, dO tile, nl2[128], D[128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
   uint64_t* st_full = bars + 2;
   uint64_t* st_empty = bars + 2 + C::kStages;
   uint64_t* s_full = bars + 2 + 2 * C::kStages;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* acc_full = s_full + 2;
-  uint64_t* acc_free = s_full + 3;
-  uint64_t* fin = s_full + 4;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_ready = s_full + 2;
+  uint64_t* ds_ready = s_full + 3;
+  uint64_t* dv_done = s_full + 4;
+  uint64_t* dk_done = s_full + 5;
+  uint64_t* acc_full = s_full + 6;
+  uint64_t* acc_free = s_full + 7;
+  uint64_t* fin = s_full + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -235,18 +266,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
     for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(st_full + i, 32);  // lane 0's expect_tx arrive + 31 lanes after their smem stores
+      mbar_init(st_full + i, 33);  // lane 0's expect_tx arrive + 32 lanes' cp.async completions
       mbar_init(st_empty + i, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 256);
+    mbar_init(s_free, kKvCompute);
+    mbar_init(p_ready, kKvCompute);
+    mbar_init(ds_ready, kKvCompute);
+    mbar_init(dv_done, 1);
+    mbar_init(dk_done, 1);
     mbar_init(acc_full, 1);
-    mbar_init(acc_free, 256);
+    mbar_init(acc_free, kKvCompute);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kKvMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -258,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_units = (*p.n_items) * p.Hkv;
   const int G = p.Hq / p.Hkv;
 
-  if (warp == kLoadWarp) {
+  if (warp == kKvLoadWarp) {
     // ------------------------------------------------------------ loads
     uint32_t st_it = 0;
     int unit_i = 0;
@@ -277,81 +312,109 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int m = it.v; m < it.nq; ++m, ++st_it) {
           const int stage = st_it % C::kStages;
           const uint32_t use = st_it / C::kStages;
+          const int q0 = it.s + 128 * m;
           if (use > 0 && !warp_wait(st_empty + stage, (use - 1) & 1, wd, 22)) { ok = false; break; }
           uint8_t* sb = sStage + stage * C::kStageBytes;
-          const int q0 = it.s + 128 * m;
-          float* lse2 = reinterpret_cast<float*>(sb + 2 * C::kTileBytes);
-          float* dl = lse2 + 128;
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int i = q0 + lane * 4 + r;
-            const bool in = i < p.T;
-            lse2[lane * 4 + r] = in ? p.lse[(size_t)h * p.T + i] * kLog2e : 0.f;
-            dl[lane * 4 + r] = in ? p.delta[(size_t)h * p.T + i] : 0.f;
-          }
           if (lane == 0) {
             mbar_arrive_expect_tx(st_full + stage, 2 * C::kTileBytes);
             for (int b = 0; b < C::kNumBox; ++b) {
               tma_load_3d(sb + b * C::kBoxBytes, &tm_q, st_full + stage, 64 * b, h, q0);
               tma_load_3d(sb + C::kTileBytes + b * C::kBoxBytes, &tm_do, st_full + stage, 64 * b, h, q0);
             }
-          } else {
-            mbar_arrive(st_full + stage);
           }
+          // -LSE log2(e) and D of the tile's 128 queries (zeros past the tensor end)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int c = 4 * lane + r, i = q0 + c;
+            const bool in = i < p.T;
+            const size_t off = in ? (size_t)h * p.T + i : 0;
+            cp_async_4(sb + C::kNl2Off + 4 * c, p.nl2 + off, in ? 4 : 0);
+            cp_async_4(sb + C::kDeltaOff + 4 * c, p.delta + off, in ? 4 : 0);
+          }
+          cp_async_mbar_arrive(st_full + stage);
         }
       }
     }
     if (lane == 0) {
-      // teardown: let this thread's copies land before the CTA exits
+      // teardown: let this warp's copies land before the CTA exits
       if (unit_i > 0) drain_wait(kv_full, (unit_i - 1) & 1, p.timeout_ns);
       for (uint32_t i = (st_it > C::kStages ? st_it - C::kStages : 0); i < st_it; ++i)
         drain_wait(st_full + (i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kKvMmaWarp) {
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);  // K-major x K-major
       constexpr uint32_t idesc_g = idesc_f16_f32(128, D, false, true);     // TMEM A x MN-major B
-      const uint32_t sk = smem_u32(sK), sv = smem_u32(sV), sst = smem_u32(sStage);
-      uint32_t st_it = 0, p_cnt = 0;
+      const uint32_t sst = smem_u32(sStage);
+      // descriptors: base + (byte offset >> 4) in the start-address field
+      const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024), dv0 = sdesc_sw128(smem_u32(sV), 16, 1024);
+      uint32_t t = 0, s_uses = 0;  // query tiles started; uses of the S^T / dP^T region
       int unit_i = 0;
       bool ok = true;
+      auto region = [&]() {  // the compute warps have read out the region's previous use
+        if (s_uses > 0 && !mbar_wait(s_free, (s_uses - 1) & 1, wd, 25)) return false;
+        tc_fence_after();
+        return true;
+      };
+      auto region_done = [&]() {
+        tc_commit(s_full);
+        ++s_uses;
+      };
+      // S^T (kv = 0) or dP^T (kv = 1) of tile tt into the region
+      auto score = [&](uint32_t tt, int kv) {
+        if (!region()) return false;
+        const uint32_t sq = sst + (tt % C::kStages) * C::kStageBytes;
+        const uint64_t da = kv ? dv0 : dk0, db = sdesc_sw128(kv ? sq + C::kTileBytes : sq, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+          mma_f16_ss(tmem + C::kSD, da + o, db + o, idesc_s, kk > 0);
+        }
+        region_done();
+        return true;
+      };
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
         const KvItem it = kv_decode(p, w);
+        const int R = G * (it.nq - it.v);
         if (!mbar_wait(kv_full, unit_i & 1, wd, 23)) break;
-        if (unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 24)) break;
         tc_fence_after();
-        bool first = true;
-        for (int h = it.g * G; h < (it.g + 1) * G && ok; ++h) {
-          for (int m = it.v; m < it.nq; ++m, ++st_it) {
-            const int stage = st_it % C::kStages;
-            if (!mbar_wait(st_full + stage, (st_it / C::kStages) & 1, wd, 25)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t sq = sst + stage * C::kStageBytes, sdo = sq + C::kTileBytes;
+        const uint32_t t_first = t;
+        if (!mbar_wait(st_full + (t % C::kStages), (t / C::kStages) & 1, wd, 26)) break;
+        tc_fence_after();
+        if (!score(t, 0)) break;
+        for (int r = 0; r < R; ++r, ++t) {
+          const uint32_t sq = sst + (t % C::kStages) * C::kStageBytes;
+          if (!score(t, 1)) { ok = false; break; }
+          // dV += P^T dO
+          if (r == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 24)) { ok = false; break; }
+          if (!mbar_wait(p_ready, t & 1, wd, 27)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ddo = sdesc_sw128(sq + C::kTileBytes, C::kBoxBytes, 1024);
+          const uint64_t dq = sdesc_sw128(sq, C::kBoxBytes, 1024);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              mma_f16_ss(tmem + C::kS, kmajor_desc(sk, kk, C::kBoxBytes), kmajor_desc(sq, kk, C::kBoxBytes),
-                         idesc_s, kk > 0);
-              mma_f16_ss(tmem + C::kDP, kmajor_desc(sv, kk, C::kBoxBytes), kmajor_desc(sdo, kk, C::kBoxBytes),
-                         idesc_s, kk > 0);
-            }
-            tc_commit(s_full);
-            if (!mbar_wait(p_full, p_cnt & 1, wd, 26)) { ok = false; break; }
-            ++p_cnt;
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16_ts(tmem + C::kDV, tmem + C::kP + 8 * kk, ddo + ((kk * 2048) >> 4), idesc_g,
+                       (r > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(dv_done);
+          // the next tile's S^T goes ahead of dK (its region was released when dP^T was read)
+          if (r + 1 < R) {
+            if (!mbar_wait(st_full + ((t + 1) % C::kStages), ((t + 1) / C::kStages) & 1, wd, 28)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-              mma_f16_ts(tmem + C::kDV, split_a_col(tmem + C::kS, kk), mnmajor_desc(sdo, kk, C::kBoxBytes),
-                         idesc_g, acc);
-              mma_f16_ts(tmem + C::kDK, split_a_col(tmem + C::kDP, kk), mnmajor_desc(sq, kk, C::kBoxBytes),
-                         idesc_g, acc);
-            }
-            first = false;
-            tc_commit(st_empty + stage);
+            if (!score(t + 1, 0)) { ok = false; break; }
           }
+          // dK += dS^T Q
+          if (!mbar_wait(ds_ready, t & 1, wd, 29)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16_ts(tmem + C::kDK, tmem + C::kDS + 8 * kk, dq + ((kk * 2048) >> 4), idesc_g,
+                       (r > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(dk_done);
+          tc_commit(st_empty + (t % C::kStages));
         }
         if (!ok) break;
+        (void)t_first;
         tc_commit(acc_full);
         tc_commit(kv_empty);
       }
@@ -363,71 +426,105 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = warp >> 2, quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key row of the tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t s_addr = lane_base + C::kS + 64 * wg;   // S^T columns of this warpgroup
-    const uint32_t dp_addr = lane_base + C::kDP + 64 * wg;
-    uint32_t s_cnt = 0, st_it = 0;
+    const uint32_t sd_addr = lane_base + C::kSD + 32 * wg;  // this warpgroup's 32 query columns
+    uint32_t t = 0, s_cnt = 0;
     int unit_i = 0;
     bool ok = true;
+    auto take = [&](float (&x)[32]) {
+      if (!warp_wait(s_full, s_cnt & 1, wd, 30)) return false;
+      ++s_cnt;
+      tc_fence_after();
+      ld_row32(sd_addr, x);
+      tc_fence_before();
+      mbar_arrive(s_free);
+      return true;
+    };
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
       const KvItem it = kv_decode(p, w);
       const int j = it.k0 + row;  // key index
       for (int h = it.g * G; h < (it.g + 1) * G && ok; ++h) {
-        for (int m = it.v; m < it.nq; ++m, ++st_it) {
-          const int stage = st_it % C::kStages;
-          if (!warp_wait(s_full, s_cnt & 1, wd, 27)) { ok = false; break; }
-          ++s_cnt;
-          tc_fence_after();
-          const float* lse2 = reinterpret_cast<const float*>(sStage + stage * C::kStageBytes + 2 * C::kTileBytes);
-          const float* dl = lse2 + 128;
-          uint32_t sr[64], dr[64];
-          tmem_ld64(s_addr, sr);
-          tmem_ld64(dp_addr, dr);
-          const int i0 = it.s + 128 * m + 64 * wg;  // query index of column 0 of this half
+        for (int m = it.v; m < it.nq; ++m, ++t) {
+          const int stage = t % C::kStages;
+          // -LSE log2(e) and D came with the stage: wait for the stage itself
+          if (!warp_wait(st_full + stage, (t / C::kStages) & 1, wd, 31)) { ok = false; break; }
+          const uint8_t* sb = sStage + stage * C::kStageBytes;
+          const float* nl2 = reinterpret_cast<const float*>(sb + C::kNl2Off) + 32 * wg;
+          const float* dl = reinterpret_cast<const float*>(sb + C::kDeltaOff) + 32 * wg;
           // visible iff j <= i < e; only the diagonal and the last query tile need the test
           const bool full = (m > it.v) && (it.s + 128 * m + 128 <= it.e);
-          uint32_t pk[32], dk[32];
-          float dmax = 0.f;
+          const int i0 = it.s + 128 * m + 32 * wg;  // query index of this thread's column 0
+          // ---- P
+          float x[32];
+          if (!take(x)) { ok = false; break; }
 #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            float pv[2], dv[2];
+          for (int c = 0; c < 32; c += 4) {
+            const float4 n4 = *reinterpret_cast<const float4*>(nl2 + c);
+            x[c] = fast_exp2(fmaf(x[c], p.scale_log2, n4.x));
+            x[c + 1] = fast_exp2(fmaf(x[c + 1], p.scale_log2, n4.y));
+            x[c + 2] = fast_exp2(fmaf(x[c + 2], p.scale_log2, n4.z));
+            x[c + 3] = fast_exp2(fmaf(x[c + 3], p.scale_log2, n4.w));
+          }
+          if (!full) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int cc = c + u;
-              const float l2 = lse2[64 * wg + cc];
-              float pp = fast_exp2(__uint_as_float(sr[cc]) * p.scale_log2 - l2);
-              if (!full) {
-                const int i = i0 + cc;
-                if (i < j || i >= it.e) pp = 0.f;
-              }
-              pv[u] = pp;
-              dv[u] = pp * (__uint_as_float(dr[cc]) - dl[64 * wg + cc]);
-              dmax = fmaxf(dmax, fabsf(dv[u]));
+            for (int c = 0; c < 32; ++c) {
+              const int i = i0 + c;
+              if (i < j || i >= it.e) x[c] = 0.f;
             }
-            pk[c / 2] = pack_f16x2(pv[0], pv[1]);
-            dk[c / 2] = pack_f16x2(dv[0], dv[1]);
+          }
+          {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk[c] = pack_f16x2(x[2 * c], x[2 * c + 1]);
+            if (t > 0 && !warp_wait(dv_done, (t - 1) & 1, wd, 32)) { ok = false; break; }
+            tc_fence_after();
+            tmem_st16(lane_base + C::kP + 16 * wg, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(p_ready);
+          }
+          // ---- dS = P (dP - D)
+          float y[32];
+          if (!take(y)) { ok = false; break; }
+          float dmax = 0.f;
+          uint32_t dk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(dl + c);
+            y[c] = x[c] * (y[c] - d4.x);
+            y[c + 1] = x[c + 1] * (y[c + 1] - d4.y);
+            y[c + 2] = x[c + 2] * (y[c + 2] - d4.z);
+            y[c + 3] = x[c + 3] * (y[c + 3] - d4.w);
+          }
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            dmax = fmaxf(dmax, fmaxf(fabsf(y[2 * c]), fabsf(y[2 * c + 1])));
+            dk[c] = pack_f16x2(y[2 * c], y[2 * c + 1]);
           }
           if (!(dmax < kF16Max)) record_error(p.status, kStatusRange, 42);
-          tmem_st32(s_addr, pk);    // P^T  -> columns [64 wg, 64 wg + 32) of S^T
-          tmem_st32(dp_addr, dk);   // dS^T -> columns [64 wg, 64 wg + 32) of dP^T
+          if (t > 0 && !warp_wait(dk_done, (t - 1) & 1, wd, 33)) { ok = false; break; }
+          tc_fence_after();
+          tmem_st16(lane_base + C::kDS + 16 * wg, dk);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(p_full);
+          mbar_arrive(ds_ready);
         }
       }
       if (!ok) break;
-      // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK * scale
-      if (!warp_wait(acc_full, unit_i & 1, wd, 28)) break;
+      // epilogue: warpgroups 0, 1 write halves of dV, warpgroups 2, 3 halves of dK * scale
+      if (!warp_wait(acc_full, unit_i & 1, wd, 34)) break;
       tc_fence_after();
       const bool valid = j < it.e;
-      const uint32_t acc_addr = lane_base + (wg ? C::kDK : C::kDV);
-      void* out = wg ? p.out0 : p.out1;
-      const float mul = wg ? p.scale : 1.f;
+      const bool is_k = wg >= 2;
+      const int c0 = (wg & 1) * (D / 2);
+      const uint32_t acc_addr = lane_base + (is_k ? C::kDK : C::kDV) + c0;
+      void* out = is_k ? p.out0 : p.out1;
+      const float mul = is_k ? p.scale : 1.f;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t t[32];
-        tmem_ld32(acc_addr + 32 * c, t);
-        tmem_wait_ld(t);
-        if (valid) store_row32(out, ((size_t)j * p.Hkv + it.g) * D + 32 * c, t, mul, p.grad_bf16);
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t tt[32];
+        tmem_ld32(acc_addr + 32 * c, tt);
+        tmem_wait_ld(tt);
+        if (valid) store_row32(out, ((size_t)j * p.Hkv + it.g) * D + c0 + 32 * c, tt, mul, p.grad_bf16);
       }
       tc_fence_before();
       mbar_arrive(acc_free);
@@ -437,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  if (warp == kKvMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
@@ -678,7 +775,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     delta_kernel<D><<<grid, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.o_resid),
         static_cast<const __nv_bfloat16*>(a.dout), static_cast<const __nv_bfloat16*>(a.q),
-        static_cast<uint4*>(a.do16), static_cast<uint4*>(a.q16), a.delta, a.T, a.Hq, a.status);
+        static_cast<uint4*>(a.do16), static_cast<uint4*>(a.q16), a.lse, a.delta, a.nl2, a.T, a.Hq, a.status);
     note_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -687,6 +784,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
   p.cu = a.cu;
   p.lse = a.lse;
   p.delta = a.delta;
+  p.nl2 = a.nl2;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
   p.T = a.T;
@@ -708,7 +806,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     pk.out1 = a.dv;
     const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
     const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
-    dkdv_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, pk);
+    dkdv_kernel<D><<<grid, kKvThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, pk);
     note_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

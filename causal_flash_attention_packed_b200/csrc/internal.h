@@ -123,6 +123,10 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream);
 // Tensor map of E4M3 codes [T][H][128] as (128, H, T), box 128 x 1 x 128,
 // 128-byte swizzle (api.cu).
 bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H);
+// Tensor map of `n` contiguous fp32 values viewed as one dimension (the
+// per-head rows of a [H][T] tensor back to back): boxes of `box` values, no
+// swizzle.  A load starts at a multiple of 4 values (16 bytes).
+bool make_tmap_flat_f32(CUtensorMap* map, const float* base, long long n, int box);
 
 // Backward, bf16 operands (bwd_bf16.cu).
 struct BwdArgs {
@@ -141,6 +145,7 @@ struct BwdArgs {
   void* dk;
   void* dv;
   float* delta;  // [Hq][T] fp32 scratch: D_i = dO_i . O_i
+  float* nl2;    // [Hq][T] fp32 scratch: -LSE_i log2(e)
   const int32_t* cu;
   int T, Hq, Hkv, d;
   float scale;
@@ -158,7 +163,9 @@ cudaError_t launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream);
 // Tensor map of a 16-bit [T][H][d] tensor (bf16, or fp16 when `f16`) as a 3-D
 // (d, H, T) view with a box of 64 channels x 1 head x 128 tokens and 128-byte
 // swizzle (api.cu).
-bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16 = false);
+// Tensor map of a [T][H][d] 16-bit tensor: boxes of 64 channels x 1 head x
+// `box_rows` tokens, 128-byte swizzle.
+bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16 = false, int box_rows = 128);
 
 // bf16 -> fp16 copy of n elements (n a multiple of 8); magnitudes >= 65504
 // record kStatusRange (convert.cu).
