@@ -519,6 +519,7 @@ const char* fapk_strerror(int status) {
     case FAPK_ERR_CUDA: return "CUDA runtime error";
     case FAPK_ERR_DEVICE_TIMEOUT: return "device watchdog timeout in a pipeline wait";
     case FAPK_ERR_RANGE: return "a value reached 65504, the fp16 range of the P/dS operand path";
+    case FAPK_ERR_INTERNAL: return "kernel shared-memory layout check failed";
     default: return "unknown status";
   }
 }

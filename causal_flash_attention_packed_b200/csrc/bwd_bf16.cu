@@ -8,19 +8,21 @@
 // over visible pairs only (j <= i, same document).
 //
 // Three kernels, all deterministic (no atomics, fixed summation order):
-//  1. delta_kernel: D for every (token, head).
+//  1. delta_kernel: D and -LSE log2(e) for every (token, head).
 //  2. dkdv kernel: one work item per (document, 128-key tile, KV head).  For
 //     each query head of the group and each query tile at or after the key
 //     tile: S^T = K Q^T and dP^T = V dO^T into TMEM (one thread per key row),
-//     P^T and dS^T written back into TMEM as bf16, then dV += P^T dO and
+//     P^T and dS^T written back into TMEM as fp16, then dV += P^T dO and
 //     dK += dS^T Q with A read from TMEM.  dK, dV accumulate in TMEM across
 //     the whole item (query heads of the group included) and are written once.
 //  3. dq kernel: one work item per (document, 128-query tile, query head).
 //     For each key tile at or before it: S = Q K^T, dP = dO V^T, dS in TMEM,
 //     dQ += dS K.
-// Warp roles as in the forward: warp 8 loads (TMA), warp 9 issues tcgen05
-// MMAs, warps 0-7 compute P and dS (warpgroup 0 on columns 0-63, warpgroup 1
-// on columns 64-127 of each 128x128 tile, every thread owning one TMEM lane).
+// Warp roles in both gradient kernels: warp 16 loads (TMA), warp 17 issues
+// tcgen05 MMAs, warps 0-15 compute P and dS (warpgroup wg on 32 columns of
+// each 128x128 tile, every thread owning one TMEM lane).  Scores are read out
+// of TMEM into registers and their columns released at once, so the MMAs of
+// the next tile overlap the exponentials of the current one.
 // Every MMA of the backward runs on fp16 operands: the prepass copies Q, K, dO
 // to fp16 (V comes from the forward's ctx), which is lossless for bf16 values
 // below 65504, and P and dS are packed to fp16 (11 significant bits, where
@@ -34,9 +36,6 @@ namespace fapk {
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -58,30 +57,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
 }
 
-// 64 TMEM columns of this thread's lane -> registers.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
-  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-  tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-  tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-}
-
-// K-major operand (rows of 128 bytes, 64 bf16 along K per box): descriptor of
-// the kk-th 16-element K step.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk, int box_bytes) {
-  return sdesc_sw128(tile + (kk >> 2) * box_bytes + (kk & 3) * 32, 16, 1024);
-}
-// MN-major operand (rows = K index, 64 bf16 along MN per 128-byte row, boxes
-// 16 KB apart along MN): descriptor of the kk-th 16-row K step.
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk, int box_bytes) {
-  return sdesc_sw128(tile + kk * 2048, box_bytes, 1024);
-}
-
-// Column of the kk-th 16-element K step of a bf16 A operand that the two
-// warpgroups wrote into TMEM: steps 0-3 (elements 0-63) at base + 8 kk,
-// steps 4-7 (elements 64-127) at base + 64 + 8 (kk - 4).
-__device__ __forceinline__ uint32_t split_a_col(uint32_t base, int kk) {
-  return base + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4));
+// One arrival per warp: every lane's prior tcgen05 and shared-memory work is
+// ordered before lane 0's arrive by the warp barrier.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // ---------------------------------------------------------------------------
@@ -192,20 +172,25 @@ __device__ __forceinline__ void store_row32(void* base, size_t elem_off, const u
 constexpr int kKvThreads = 576;
 constexpr int kKvLoadWarp = 16;
 constexpr int kKvMmaWarp = 17;
-constexpr int kKvCompute = 512;
+constexpr int kKvComputeWarps = 16;
 
 template <int D>
 struct KvCfg : Geo<D> {
-  static constexpr int kStages = 2;
-  static constexpr int kStageBytes = 2 * Geo<D>::kTileBytes + 1024;  // Q, dO, nl2[128], D[128]
-  static constexpr int kNl2Off = 2 * Geo<D>::kTileBytes, kDeltaOff = kNl2Off + 512;
-  static constexpr int kSmemTiles = 2 * Geo<D>::kTileBytes + kStages * kStageBytes;
+  // Q and dO stream through separate rings: dO (with the tile's -LSE log2(e)
+  // and D) is free once dV and dS are done, Q only after dK, so Q gets one
+  // stage more
+  static constexpr int kQStages = 3, kOStages = 2;
+  static constexpr int kOStageBytes = Geo<D>::kTileBytes + 1024;  // dO, nl2[128], D[128]
+  static constexpr int kNl2Off = Geo<D>::kTileBytes, kDeltaOff = kNl2Off + 512;
+  static constexpr int kSmemTiles = (2 + kQStages) * Geo<D>::kTileBytes + kOStages * kOStageBytes;
   // TMEM: dV [0,D), dK [128,128+D), S^T / dP^T [256,384), P^T [384,448), dS^T [448,512)
   static constexpr uint32_t kDV = 0, kDK = 128, kSD = 256, kP = 384, kDS = 448;
-  // bars: kv_full, kv_empty, st_full[S], st_empty[S], s_full, s_free, p_ready, ds_ready,
-  //       dv_done, dk_done, acc_full, acc_free, fin
-  static constexpr int kNumBars = 2 + 2 * kStages + 9;
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
+  // bars: kv_full, kv_empty, q_full[Q], q_empty[Q], o_full[O], o_empty[O], s_full, s_free, p_ready,
+  //       ds_ready, dv_done, dk_done, acc_full, acc_free, fin
+  static constexpr int kNumBars = 2 + 2 * kQStages + 2 * kOStages + 9;
+  // no alignment slack: the kernel checks that dynamic shared memory starts
+  // on a 1024-byte boundary
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16;
 };
 
 struct KvItem {
@@ -240,16 +225,23 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 const BwdParams p) {
   using C = KvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw;
+  if ((smem_u32(smem) & 1023u) != 0) {  // 128-byte swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) record_error(p.status, kStatusInternal, 20);
+    return;
+  }
   uint8_t* sK = smem;
   uint8_t* sV = smem + C::kTileBytes;
-  uint8_t* sStage = smem + 2 * C::kTileBytes;  // per stage: Q tile, dO tile, nl2[128], D[128]
+  uint8_t* sQr = smem + 2 * C::kTileBytes;             // Q ring
+  uint8_t* sOr = sQr + C::kQStages * C::kTileBytes;    // dO ring: dO tile, nl2[128], D[128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* st_full = bars + 2;
-  uint64_t* st_empty = bars + 2 + C::kStages;
-  uint64_t* s_full = bars + 2 + 2 * C::kStages;
+  uint64_t* q_full = bars + 2;
+  uint64_t* q_empty = q_full + C::kQStages;
+  uint64_t* o_full = q_empty + C::kQStages;
+  uint64_t* o_empty = o_full + C::kOStages;
+  uint64_t* s_full = o_empty + C::kOStages;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_ready = s_full + 2;
   uint64_t* ds_ready = s_full + 3;
@@ -265,18 +257,22 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(st_full + i, 33);  // lane 0's expect_tx arrive + 32 lanes' cp.async completions
-      mbar_init(st_empty + i, 1);
+    for (int i = 0; i < C::kQStages; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(q_empty + i, 1);
+    }
+    for (int i = 0; i < C::kOStages; ++i) {
+      mbar_init(o_full + i, 33);                   // lane 0's expect_tx arrive + 32 lanes' cp.async completions
+      mbar_init(o_empty + i, 1 + kKvComputeWarps);  // dV's commit + every compute warp after dS
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, kKvCompute);
-    mbar_init(p_ready, kKvCompute);
-    mbar_init(ds_ready, kKvCompute);
+    mbar_init(s_free, kKvComputeWarps);
+    mbar_init(p_ready, kKvComputeWarps);
+    mbar_init(ds_ready, kKvComputeWarps);
     mbar_init(dv_done, 1);
     mbar_init(dk_done, 1);
     mbar_init(acc_full, 1);
-    mbar_init(acc_free, kKvCompute);
+    mbar_init(acc_free, kKvComputeWarps);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -295,7 +291,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 
   if (warp == kKvLoadWarp) {
     // ------------------------------------------------------------ loads
-    uint32_t st_it = 0;
+    uint32_t t = 0;  // query tiles loaded so far
     int unit_i = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
@@ -309,18 +305,22 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
       }
       for (int h = it.g * G; h < (it.g + 1) * G && ok; ++h) {
-        for (int m = it.v; m < it.nq; ++m, ++st_it) {
-          const int stage = st_it % C::kStages;
-          const uint32_t use = st_it / C::kStages;
+        for (int m = it.v; m < it.nq; ++m, ++t) {
+          const int qs = t % C::kQStages, os = t % C::kOStages;
+          const uint32_t qu = t / C::kQStages, ou = t / C::kOStages;
           const int q0 = it.s + 128 * m;
-          if (use > 0 && !warp_wait(st_empty + stage, (use - 1) & 1, wd, 22)) { ok = false; break; }
-          uint8_t* sb = sStage + stage * C::kStageBytes;
+          if (qu > 0 && !warp_wait(q_empty + qs, (qu - 1) & 1, wd, 22)) { ok = false; break; }
           if (lane == 0) {
-            mbar_arrive_expect_tx(st_full + stage, 2 * C::kTileBytes);
-            for (int b = 0; b < C::kNumBox; ++b) {
-              tma_load_3d(sb + b * C::kBoxBytes, &tm_q, st_full + stage, 64 * b, h, q0);
-              tma_load_3d(sb + C::kTileBytes + b * C::kBoxBytes, &tm_do, st_full + stage, 64 * b, h, q0);
-            }
+            mbar_arrive_expect_tx(q_full + qs, C::kTileBytes);
+            for (int b = 0; b < C::kNumBox; ++b)
+              tma_load_3d(sQr + qs * C::kTileBytes + b * C::kBoxBytes, &tm_q, q_full + qs, 64 * b, h, q0);
+          }
+          if (ou > 0 && !warp_wait(o_empty + os, (ou - 1) & 1, wd, 20)) { ok = false; break; }
+          uint8_t* ob = sOr + os * C::kOStageBytes;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(o_full + os, C::kTileBytes);
+            for (int b = 0; b < C::kNumBox; ++b)
+              tma_load_3d(ob + b * C::kBoxBytes, &tm_do, o_full + os, 64 * b, h, q0);
           }
           // -LSE log2(e) and D of the tile's 128 queries (zeros past the tensor end)
 #pragma unroll
@@ -328,25 +328,27 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             const int c = 4 * lane + r, i = q0 + c;
             const bool in = i < p.T;
             const size_t off = in ? (size_t)h * p.T + i : 0;
-            cp_async_4(sb + C::kNl2Off + 4 * c, p.nl2 + off, in ? 4 : 0);
-            cp_async_4(sb + C::kDeltaOff + 4 * c, p.delta + off, in ? 4 : 0);
+            cp_async_4(ob + C::kNl2Off + 4 * c, p.nl2 + off, in ? 4 : 0);
+            cp_async_4(ob + C::kDeltaOff + 4 * c, p.delta + off, in ? 4 : 0);
           }
-          cp_async_mbar_arrive(st_full + stage);
+          cp_async_mbar_arrive(o_full + os);
         }
       }
     }
     if (lane == 0) {
       // teardown: let this warp's copies land before the CTA exits
       if (unit_i > 0) drain_wait(kv_full, (unit_i - 1) & 1, p.timeout_ns);
-      for (uint32_t i = (st_it > C::kStages ? st_it - C::kStages : 0); i < st_it; ++i)
-        drain_wait(st_full + (i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
+      for (uint32_t i = (t > C::kQStages ? t - C::kQStages : 0); i < t; ++i)
+        drain_wait(q_full + (i % C::kQStages), (i / C::kQStages) & 1, p.timeout_ns);
+      for (uint32_t i = (t > C::kOStages ? t - C::kOStages : 0); i < t; ++i)
+        drain_wait(o_full + (i % C::kOStages), (i / C::kOStages) & 1, p.timeout_ns);
     }
   } else if (warp == kKvMmaWarp) {
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);  // K-major x K-major
       constexpr uint32_t idesc_g = idesc_f16_f32(128, D, false, true);     // TMEM A x MN-major B
-      const uint32_t sst = smem_u32(sStage);
+      const uint32_t sqr = smem_u32(sQr), sor = smem_u32(sOr);
       // descriptors: base + (byte offset >> 4) in the start-address field
       const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024), dv0 = sdesc_sw128(smem_u32(sV), 16, 1024);
       uint32_t t = 0, s_uses = 0;  // query tiles started; uses of the S^T / dP^T region
@@ -363,9 +365,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       };
       // S^T (kv = 0) or dP^T (kv = 1) of tile tt into the region
       auto score = [&](uint32_t tt, int kv) {
+        if (kv == 0 && !mbar_wait(q_full + (tt % C::kQStages), (tt / C::kQStages) & 1, wd, 26)) return false;
+        if (kv == 1 && !mbar_wait(o_full + (tt % C::kOStages), (tt / C::kOStages) & 1, wd, 28)) return false;
         if (!region()) return false;
-        const uint32_t sq = sst + (tt % C::kStages) * C::kStageBytes;
-        const uint64_t da = kv ? dv0 : dk0, db = sdesc_sw128(kv ? sq + C::kTileBytes : sq, 16, 1024);
+        const uint32_t b_op = kv ? sor + (tt % C::kOStages) * C::kOStageBytes : sqr + (tt % C::kQStages) * C::kTileBytes;
+        const uint64_t da = kv ? dv0 : dk0, db = sdesc_sw128(b_op, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t o = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
@@ -379,30 +383,23 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const int R = G * (it.nq - it.v);
         if (!mbar_wait(kv_full, unit_i & 1, wd, 23)) break;
         tc_fence_after();
-        const uint32_t t_first = t;
-        if (!mbar_wait(st_full + (t % C::kStages), (t / C::kStages) & 1, wd, 26)) break;
-        tc_fence_after();
         if (!score(t, 0)) break;
         for (int r = 0; r < R; ++r, ++t) {
-          const uint32_t sq = sst + (t % C::kStages) * C::kStageBytes;
           if (!score(t, 1)) { ok = false; break; }
           // dV += P^T dO
           if (r == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 24)) { ok = false; break; }
           if (!mbar_wait(p_ready, t & 1, wd, 27)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t ddo = sdesc_sw128(sq + C::kTileBytes, C::kBoxBytes, 1024);
-          const uint64_t dq = sdesc_sw128(sq, C::kBoxBytes, 1024);
+          const uint64_t ddo = sdesc_sw128(sor + (t % C::kOStages) * C::kOStageBytes, C::kBoxBytes, 1024);
+          const uint64_t dq = sdesc_sw128(sqr + (t % C::kQStages) * C::kTileBytes, C::kBoxBytes, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_f16_ts(tmem + C::kDV, tmem + C::kP + 8 * kk, ddo + ((kk * 2048) >> 4), idesc_g,
                        (r > 0 || kk > 0) ? 1u : 0u);
           tc_commit(dv_done);
+          tc_commit(o_empty + (t % C::kOStages));  // dV was the MMAs' last read of dO
           // the next tile's S^T goes ahead of dK (its region was released when dP^T was read)
-          if (r + 1 < R) {
-            if (!mbar_wait(st_full + ((t + 1) % C::kStages), ((t + 1) / C::kStages) & 1, wd, 28)) { ok = false; break; }
-            tc_fence_after();
-            if (!score(t + 1, 0)) { ok = false; break; }
-          }
+          if (r + 1 < R && !score(t + 1, 0)) { ok = false; break; }
           // dK += dS^T Q
           if (!mbar_wait(ds_ready, t & 1, wd, 29)) { ok = false; break; }
           tc_fence_after();
@@ -411,10 +408,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             mma_f16_ts(tmem + C::kDK, tmem + C::kDS + 8 * kk, dq + ((kk * 2048) >> 4), idesc_g,
                        (r > 0 || kk > 0) ? 1u : 0u);
           tc_commit(dk_done);
-          tc_commit(st_empty + (t % C::kStages));
+          tc_commit(q_empty + (t % C::kQStages));
         }
         if (!ok) break;
-        (void)t_first;
         tc_commit(acc_full);
         tc_commit(kv_empty);
       }
@@ -436,7 +432,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       tc_fence_after();
       ld_row32(sd_addr, x);
       tc_fence_before();
-      mbar_arrive(s_free);
+      warp_arrive(s_free);
       return true;
     };
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
@@ -444,10 +440,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const int j = it.k0 + row;  // key index
       for (int h = it.g * G; h < (it.g + 1) * G && ok; ++h) {
         for (int m = it.v; m < it.nq; ++m, ++t) {
-          const int stage = t % C::kStages;
-          // -LSE log2(e) and D came with the stage: wait for the stage itself
-          if (!warp_wait(st_full + stage, (t / C::kStages) & 1, wd, 31)) { ok = false; break; }
-          const uint8_t* sb = sStage + stage * C::kStageBytes;
+          const int os = t % C::kOStages;
+          // -LSE log2(e) and D came with the dO stage: wait for the stage itself
+          if (!warp_wait(o_full + os, (t / C::kOStages) & 1, wd, 31)) { ok = false; break; }
+          const uint8_t* sb = sOr + os * C::kOStageBytes;
           const float* nl2 = reinterpret_cast<const float*>(sb + C::kNl2Off) + 32 * wg;
           const float* dl = reinterpret_cast<const float*>(sb + C::kDeltaOff) + 32 * wg;
           // visible iff j <= i < e; only the diagonal and the last query tile need the test
@@ -480,7 +476,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             tmem_st16(lane_base + C::kP + 16 * wg, pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_ready);
+            warp_arrive(p_ready);
           }
           // ---- dS = P (dP - D)
           float y[32];
@@ -501,12 +497,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             dk[c] = pack_f16x2(y[2 * c], y[2 * c + 1]);
           }
           if (!(dmax < kF16Max)) record_error(p.status, kStatusRange, 42);
+          warp_arrive(o_empty + os);  // done with this tile's -LSE log2(e) and D
           if (t > 0 && !warp_wait(dk_done, (t - 1) & 1, wd, 33)) { ok = false; break; }
           tc_fence_after();
           tmem_st16(lane_base + C::kDS + 16 * wg, dk);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(ds_ready);
+          warp_arrive(ds_ready);
         }
       }
       if (!ok) break;
@@ -527,7 +524,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (valid) store_row32(out, ((size_t)j * p.Hkv + it.g) * D + c0 + 32 * c, tt, mul, p.grad_bf16);
       }
       tc_fence_before();
-      mbar_arrive(acc_free);
+      warp_arrive(acc_free);
     }
   }
 
@@ -540,15 +537,27 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 // ---------------------------------------------------------------------------
 // 3. dQ
 // ---------------------------------------------------------------------------
+// TMEM holds dQ, S, dP and the tile's dS (fp16).  The compute warps read S and
+// dP out into registers and release them at once, so S and dP of key tile
+// v + 1 are computed while dS of tile v is formed; dQ += dS K takes dS from
+// TMEM.  16 compute warps: warpgroup wg owns key columns [32 wg, 32 wg + 32)
+// of every tile; each thread owns one query row.
+constexpr int kQThreads = 576;
+constexpr int kQLoadWarp = 16;
+constexpr int kQMmaWarp = 17;
+constexpr int kQComputeWarps = 16;
+
 template <int D>
 struct QCfg : Geo<D> {
-  static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kStageBytes = 2 * Geo<D>::kTileBytes;  // K, V
-  static constexpr int kSmemTiles = 2 * Geo<D>::kTileBytes + kStages * kStageBytes;
-  // TMEM: S [0,128), dP [128,256), dQ [256,256+D)
-  static constexpr uint32_t kS = 0, kDP = 128, kDQ = 256;
-  // bars: q_full, q_empty, st_full[S], st_empty[S], s_full, p_full, acc_full, acc_free, fin
-  static constexpr int kNumBars = 2 + 2 * kStages + 5;
+  // K and V stream through separate rings: V is released as soon as dP has
+  // read it, K only after dQ, so K gets one stage more
+  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr int kSmemTiles = (2 + kKStages + kVStages) * Geo<D>::kTileBytes;  // Q, dO, K ring, V ring
+  // TMEM: dQ [0,D), S [128,256), dP [256,384), dS [384,448)
+  static constexpr uint32_t kDQ = 0, kS = 128, kDP = 256, kDS = 384;
+  // bars: q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full, s_free, dp_full, dp_free,
+  //       ds_ready, dq_done, acc_full, acc_free, fin
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 9;
   static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
 };
 
@@ -569,7 +578,7 @@ __device__ __forceinline__ QItem q_decode(const BwdParams& p, int w) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kQThreads, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const BwdParams p) {
@@ -578,17 +587,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sDO = smem + C::kTileBytes;
-  uint8_t* sStage = smem + 2 * C::kTileBytes;  // per stage: K tile, V tile
+  uint8_t* sKr = smem + 2 * C::kTileBytes;                  // K ring
+  uint8_t* sVr = sKr + C::kKStages * C::kTileBytes;          // V ring
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* st_full = bars + 2;
-  uint64_t* st_empty = bars + 2 + C::kStages;
-  uint64_t* s_full = bars + 2 + 2 * C::kStages;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* acc_full = s_full + 2;
-  uint64_t* acc_free = s_full + 3;
-  uint64_t* fin = s_full + 4;
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = k_full + C::kKStages;
+  uint64_t* v_full = k_empty + C::kKStages;
+  uint64_t* v_empty = v_full + C::kVStages;
+  uint64_t* s_full = v_empty + C::kVStages;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* dp_full = s_full + 2;
+  uint64_t* dp_free = s_full + 3;
+  uint64_t* ds_ready = s_full + 4;
+  uint64_t* dq_done = s_full + 5;
+  uint64_t* acc_full = s_full + 6;
+  uint64_t* acc_free = s_full + 7;
+  uint64_t* fin = s_full + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -596,19 +612,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(st_full + i, 1);
-      mbar_init(st_empty + i, 1);
+    for (int i = 0; i < C::kKStages; ++i) {
+      mbar_init(k_full + i, 1);
+      mbar_init(k_empty + i, 1);
+    }
+    for (int i = 0; i < C::kVStages; ++i) {
+      mbar_init(v_full + i, 1);
+      mbar_init(v_empty + i, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 256);
+    mbar_init(s_free, kQComputeWarps);
+    mbar_init(dp_full, 1);
+    mbar_init(dp_free, kQComputeWarps);
+    mbar_init(ds_ready, kQComputeWarps);
+    mbar_init(dq_done, 1);
     mbar_init(acc_full, 1);
-    mbar_init(acc_free, 256);
+    mbar_init(acc_free, kQComputeWarps);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kQMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -619,9 +643,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
   const int n_units = (*p.n_items) * p.Hq;
 
-  if (warp == kLoadWarp) {
+  if (warp == kQLoadWarp) {
     if (lane == 0) {
-      uint32_t st_it = 0;
+      uint32_t kt = 0;  // key tiles loaded (all units)
       int unit_i = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
@@ -632,57 +656,79 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(sQ + b * C::kBoxBytes, &tm_q, q_full, 64 * b, it.h, it.q0);
           tma_load_3d(sDO + b * C::kBoxBytes, &tm_do, q_full, 64 * b, it.h, it.q0);
         }
-        for (int v = 0; v <= it.m; ++v, ++st_it) {
-          const int stage = st_it % C::kStages;
-          const uint32_t use = st_it / C::kStages;
-          if (use > 0 && !mbar_wait(st_empty + stage, (use - 1) & 1, wd, 32)) { ok = false; break; }
-          uint8_t* sb = sStage + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(st_full + stage, 2 * C::kTileBytes);
-          for (int b = 0; b < C::kNumBox; ++b) {
-            tma_load_3d(sb + b * C::kBoxBytes, &tm_k, st_full + stage, 64 * b, it.g, it.s + 128 * v);
-            tma_load_3d(sb + C::kTileBytes + b * C::kBoxBytes, &tm_v, st_full + stage, 64 * b, it.g,
-                        it.s + 128 * v);
-          }
+        for (int v = 0; v <= it.m; ++v, ++kt) {
+          const int ks = kt % C::kKStages, vs = kt % C::kVStages;
+          const uint32_t ku = kt / C::kKStages, vu = kt / C::kVStages;
+          const int k0 = it.s + 128 * v;
+          if (ku > 0 && !mbar_wait(k_empty + ks, (ku - 1) & 1, wd, 32)) { ok = false; break; }
+          mbar_arrive_expect_tx(k_full + ks, C::kTileBytes);
+          for (int b = 0; b < C::kNumBox; ++b)
+            tma_load_3d(sKr + ks * C::kTileBytes + b * C::kBoxBytes, &tm_k, k_full + ks, 64 * b, it.g, k0);
+          if (vu > 0 && !mbar_wait(v_empty + vs, (vu - 1) & 1, wd, 30)) { ok = false; break; }
+          mbar_arrive_expect_tx(v_full + vs, C::kTileBytes);
+          for (int b = 0; b < C::kNumBox; ++b)
+            tma_load_3d(sVr + vs * C::kTileBytes + b * C::kBoxBytes, &tm_v, v_full + vs, 64 * b, it.g, k0);
         }
       }
       if (unit_i > 0) drain_wait(q_full, (unit_i - 1) & 1, p.timeout_ns);
-      for (uint32_t i = (st_it > C::kStages ? st_it - C::kStages : 0); i < st_it; ++i)
-        drain_wait(st_full + (i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
+      for (uint32_t i = (kt > C::kKStages ? kt - C::kKStages : 0); i < kt; ++i)
+        drain_wait(k_full + (i % C::kKStages), (i / C::kKStages) & 1, p.timeout_ns);
+      for (uint32_t i = (kt > C::kVStages ? kt - C::kVStages : 0); i < kt; ++i)
+        drain_wait(v_full + (i % C::kVStages), (i / C::kVStages) & 1, p.timeout_ns);
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kQMmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);
       constexpr uint32_t idesc_g = idesc_f16_f32(128, D, false, true);
-      const uint32_t sq = smem_u32(sQ), sdo = smem_u32(sDO), sst = smem_u32(sStage);
-      uint32_t st_it = 0, p_cnt = 0;
+      const uint32_t skr = smem_u32(sKr), svr = smem_u32(sVr);
+      const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024), ddo0 = sdesc_sw128(smem_u32(sDO), 16, 1024);
+      uint32_t st_it = 0;  // key tiles started (all units)
       int unit_i = 0;
       bool ok = true;
+      // S and dP of key tile number kt (global count) into their regions
+      auto scores = [&](uint32_t kt) {
+        const int ks = kt % C::kKStages, vs = kt % C::kVStages;
+        if (!mbar_wait(k_full + ks, (kt / C::kKStages) & 1, wd, 35)) return false;
+        const uint64_t dk = sdesc_sw128(skr + ks * C::kTileBytes, 16, 1024);
+        const uint64_t dv = sdesc_sw128(svr + vs * C::kTileBytes, 16, 1024);
+        if (kt > 0 && !mbar_wait(s_free, (kt - 1) & 1, wd, 36)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+          mma_f16_ss(tmem + C::kS, dq0 + o, dk + o, idesc_s, kk > 0);
+        }
+        tc_commit(s_full);
+        if (kt > 0 && !mbar_wait(dp_free, (kt - 1) & 1, wd, 37)) return false;
+        if (!mbar_wait(v_full + vs, (kt / C::kVStages) & 1, wd, 44)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+          mma_f16_ss(tmem + C::kDP, ddo0 + o, dv + o, idesc_s, kk > 0);
+        }
+        tc_commit(dp_full);
+        tc_commit(v_empty + vs);  // V is read only by dP
+        return true;
+      };
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
         const QItem it = q_decode(p, w);
         if (!mbar_wait(q_full, unit_i & 1, wd, 33)) break;
-        if (unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 34)) break;
         tc_fence_after();
+        if (!scores(st_it)) break;
         for (int v = 0; v <= it.m; ++v, ++st_it) {
-          const int stage = st_it % C::kStages;
-          if (!mbar_wait(st_full + stage, (st_it / C::kStages) & 1, wd, 35)) { ok = false; break; }
+          // the next key tile's S and dP go ahead of this tile's dQ
+          if (v < it.m && !scores(st_it + 1)) { ok = false; break; }
+          if (v == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 34)) { ok = false; break; }
+          if (!mbar_wait(ds_ready, st_it & 1, wd, 38)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sk = sst + stage * C::kStageBytes, sv = sk + C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            mma_f16_ss(tmem + C::kS, kmajor_desc(sq, kk, C::kBoxBytes), kmajor_desc(sk, kk, C::kBoxBytes),
-                       idesc_s, kk > 0);
-            mma_f16_ss(tmem + C::kDP, kmajor_desc(sdo, kk, C::kBoxBytes), kmajor_desc(sv, kk, C::kBoxBytes),
-                       idesc_s, kk > 0);
-          }
-          tc_commit(s_full);
-          if (!mbar_wait(p_full, p_cnt & 1, wd, 36)) { ok = false; break; }
-          ++p_cnt;
-          tc_fence_after();
+          const uint64_t dkm = sdesc_sw128(skr + (st_it % C::kKStages) * C::kTileBytes, C::kBoxBytes, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_f16_ts(tmem + C::kDQ, split_a_col(tmem + C::kS, kk), mnmajor_desc(sk, kk, C::kBoxBytes), idesc_g,
+            mma_f16_ts(tmem + C::kDQ, tmem + C::kDS + 8 * kk, dkm + ((kk * 2048) >> 4), idesc_g,
                        (v > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(st_empty + stage);
+          tc_commit(dq_done);
+          tc_commit(k_empty + (st_it % C::kKStages));
         }
         if (!ok) break;
         tc_commit(acc_full);
@@ -695,9 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = warp >> 2, quarter = warp & 3;
     const int row = quarter * 32 + lane;  // query row of the tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t s_addr = lane_base + C::kS + 64 * wg;
-    const uint32_t dp_addr = lane_base + C::kDP + 64 * wg;
-    uint32_t s_cnt = 0;
+    uint32_t kt = 0;  // key tiles processed (all units)
     int unit_i = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
@@ -705,59 +749,65 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i = it.q0 + row;
       const bool valid = i < it.e;
       // rows past the document end (the tail of the last tile) get P = 0
-      const float l2 = valid ? p.lse[(size_t)it.h * p.T + i] * kLog2e : INFINITY;
+      const float nl2 = valid ? p.nl2[(size_t)it.h * p.T + i] : -INFINITY;
       const float dl = valid ? p.delta[(size_t)it.h * p.T + i] : 0.f;
-      for (int v = 0; v <= it.m; ++v) {
-        if (!warp_wait(s_full, s_cnt & 1, wd, 37)) { ok = false; break; }
-        ++s_cnt;
+      for (int v = 0; v <= it.m; ++v, ++kt) {
+        float x[32], y[32];
+        if (!warp_wait(s_full, kt & 1, wd, 39)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[64], dr[64];
-        tmem_ld64(s_addr, sr);
-        tmem_ld64(dp_addr, dr);
-        const int j0 = it.s + 128 * v + 64 * wg;  // key index of column 0 of this half
+        ld_row32(lane_base + C::kS + 32 * wg, x);
+        tc_fence_before();
+        warp_arrive(s_free);
+        if (!warp_wait(dp_full, kt & 1, wd, 40)) { ok = false; break; }
+        tc_fence_after();
+        ld_row32(lane_base + C::kDP + 32 * wg, y);
+        tc_fence_before();
+        warp_arrive(dp_free);
+        const int j0 = it.s + 128 * v + 32 * wg;  // key index of this thread's column 0
         const bool diag = v == it.m;
-        uint32_t dk[32];
+        uint32_t dk[16];
         float dmax = 0.f;
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
+        for (int c = 0; c < 32; c += 2) {
           float dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int cc = c + u;
-            float pp = fast_exp2(__uint_as_float(sr[cc]) * p.scale_log2 - l2);
+            float pp = fast_exp2(fmaf(x[cc], p.scale_log2, nl2));
             if (diag && j0 + cc > i) pp = 0.f;
-            dv[u] = pp * (__uint_as_float(dr[cc]) - dl);
+            dv[u] = pp * (y[cc] - dl);
             dmax = fmaxf(dmax, fabsf(dv[u]));
           }
           dk[c / 2] = pack_f16x2(dv[0], dv[1]);
         }
         if (!(dmax < kF16Max)) record_error(p.status, kStatusRange, 43);
-        tmem_st32(s_addr, dk);  // dS -> columns [64 wg, 64 wg + 32) of S
+        if (kt > 0 && !warp_wait(dq_done, (kt - 1) & 1, wd, 41)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st16(lane_base + C::kDS + 16 * wg, dk);  // dS -> columns [16 wg, 16 wg + 16)
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full);
+        warp_arrive(ds_ready);
       }
       if (!ok) break;
-      if (!warp_wait(acc_full, unit_i & 1, wd, 38)) break;
+      if (!warp_wait(acc_full, unit_i & 1, wd, 42)) break;
       tc_fence_after();
-      // warpgroup wg writes channels [wg D/2, (wg+1) D/2) of dQ * scale
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      // warpgroup wg writes channels [wg D/4, (wg+1) D/4) of dQ * scale
+      if (D == 128 || wg < 2) {
         uint32_t t[32];
-        const int col = wg * (D / 2) + 32 * c;
+        const int col = wg * 32;
         tmem_ld32(lane_base + C::kDQ + col, t);
         tmem_wait_ld(t);
         if (valid) store_row32(p.out0, ((size_t)i * p.Hq + it.h) * D + col, t, p.scale, p.grad_bf16);
       }
       tc_fence_before();
-      mbar_arrive(acc_free);
+      warp_arrive(acc_free);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  if (warp == kQMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 template <int D>
@@ -824,7 +874,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     pq.out1 = nullptr;
     const long long max_units = (long long)a.sched_q.max_items * a.Hq;
     const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
-    dq_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, pq);
+    dq_kernel<D><<<grid, kQThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, pq);
     note_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -13,7 +13,7 @@ namespace fapk {
 // ---------------------------------------------------------------------------
 // Status word in the workspace (device errors) and the CTA abort flag.
 // ---------------------------------------------------------------------------
-enum : int { kStatusOk = 0, kStatusBadSeqlens = 3, kStatusTimeout = 6, kStatusRange = 7 };
+enum : int { kStatusOk = 0, kStatusBadSeqlens = 3, kStatusTimeout = 6, kStatusRange = 7, kStatusInternal = 8 };
 
 struct DeviceStatus {
   int code;       // first error recorded (0 = none)

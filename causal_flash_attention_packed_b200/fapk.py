@@ -29,6 +29,7 @@ ERR_WORKSPACE_TOO_SMALL = 4
 ERR_CUDA = 5
 ERR_DEVICE_TIMEOUT = 6
 ERR_RANGE = 7
+ERR_INTERNAL = 8
 
 BF16 = 0
 MXFP8 = 1

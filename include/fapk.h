@@ -73,9 +73,11 @@ typedef enum {
   FAPK_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below fapk_workspace_size() */
   FAPK_ERR_CUDA = 5,                /* a CUDA runtime call failed (launch, no device) */
   FAPK_ERR_DEVICE_TIMEOUT = 6,      /* a bounded device-side wait gave up */
-  FAPK_ERR_RANGE = 7                /* an input or a computed gradient operand reached
+  FAPK_ERR_RANGE = 7,               /* an input or a computed gradient operand reached
                                        65504, the fp16 range of the bf16 path's
                                        P/dS operands (see fapk_attn_fwd) */
+  FAPK_ERR_INTERNAL = 8             /* a kernel found its dynamic shared memory not
+                                       1024-byte aligned and computed nothing */
 } fapk_status_t;
 
 /* Operand precision of the attention path. */
