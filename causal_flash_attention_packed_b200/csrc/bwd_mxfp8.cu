@@ -135,13 +135,6 @@ __device__ __forceinline__ void store_bf16_32(uint8_t* tile, int row, int q, con
         make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
 }
 
-__device__ __forceinline__ void zero_bf16_row(uint8_t* tile, int row) {
-#pragma unroll
-  for (int box = 0; box < 2; ++box)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(tile + box * kBox + row * 128 + (c << 4)) = make_uint4(0, 0, 0, 0);
-}
-
 // ---------------------------------------------------------------------------
 // D = rowsum(dO * (o + o_resid)), fp32 [Hq][T]
 // ---------------------------------------------------------------------------
@@ -209,19 +202,30 @@ __device__ __forceinline__ void store_row32(void* base, size_t elem_off, const u
 // dQ
 // ---------------------------------------------------------------------------
 namespace dqk {
-constexpr int kThreads = 192, kLoad = 4, kMma = 5, kStages = 2;
+// warps 0-15: one thread per (query row, 32-key block): warpgroup wg on key
+// block wg of every tile (one MX scale block of dS~); warp 16: loads; warp 17: MMA
+constexpr int kThreads = 576, kLoad = 16, kMma = 17, kComputeWarps = 16, kStages = 2;
 constexpr int oQ = 0, oDO = oQ + kCode, oRing = oDO + kCode;  // ring stage: K^tb, V^tb codes
 constexpr int oKpt = oRing + kStages * 2 * kCode, oVpt = oKpt + kCode, oKd = oVpt + kCode;  // diag
 constexpr int oDS = oKd + kBf16, oDSd = oDS + kCode;
 constexpr int oSf = oDSd + kBf16;  // sfQ, sfDO, sfKpt, sfVpt, sfDS, per stage {sfK, sfV, sfKdq}
 constexpr int kNumSf = 5 + 3 * kStages;
 constexpr int oBars = oSf + kNumSf * kSfBlk;
-constexpr int kNumBars = 2 + 2 * kStages + 7;
+// bars: q_full, q_empty, st_full[S], st_empty[S], s_full, s_free, dp_full, dp_free, ds_ready, dq_done,
+//       acc_full, acc_free, fin
+constexpr int kNumBars = 2 + 2 * kStages + 9;
 constexpr int kSmem = oBars + kNumBars * 8 + 16 + 1024;
+// TMEM: S and dP regions (each read out into registers and released at
+// once), dQ, scale factors
 constexpr uint32_t tS = 0, tDP = 128, tDQ = 256;
 constexpr uint32_t tSfQ = 384, tSfDO = 388, tSfK = 392, tSfV = 396, tSfKpt = 400, tSfVpt = 404, tSfDS = 408,
                    tSfKdq = 412;
 }  // namespace dqk
+
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
 
 __global__ void __launch_bounds__(dqk::kThreads, 1)
     dq_mx_kernel(const __grid_constant__ CUtensorMap tm_qpt, const __grid_constant__ CUtensorMap tm_dopt,
@@ -238,12 +242,14 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   uint64_t* st_full = bars + 2;
   uint64_t* st_empty = bars + 2 + kStages;
   uint64_t* s_full = bars + 2 + 2 * kStages;
-  uint64_t* s_read = s_full + 1;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* dq_done = s_full + 3;
-  uint64_t* acc_full = s_full + 4;
-  uint64_t* acc_free = s_full + 5;
-  uint64_t* fin = s_full + 6;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* dp_full = s_full + 2;
+  uint64_t* dp_free = s_full + 3;
+  uint64_t* ds_ready = s_full + 4;
+  uint64_t* dq_done = s_full + 5;
+  uint64_t* acc_full = s_full + 6;
+  uint64_t* acc_free = s_full + 7;
+  uint64_t* fin = s_full + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto sfb = [&](int i) { return sf + i * kSfBlk; };  // 0 Q, 1 dO, 2 Kpt, 3 Vpt, 4 dS, 5+3s+{0,1,2} stage
@@ -257,11 +263,13 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       mbar_init(st_empty + i, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_read, 128);
-    mbar_init(p_full, 128);
+    mbar_init(s_free, kComputeWarps);
+    mbar_init(dp_full, 1);
+    mbar_init(dp_free, kComputeWarps);
+    mbar_init(ds_ready, kComputeWarps);
     mbar_init(dq_done, 1);
     mbar_init(acc_full, 1);
-    mbar_init(acc_free, 128);
+    mbar_init(acc_free, kComputeWarps);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -314,10 +322,14 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       for (int v = 0; v < n; ++v, ++st_it) {
         const int stg = st_it % kStages;
         const uint32_t use = st_it / kStages;
+        // scale words first, so that their global reads overlap the wait
+        const uint4 wk = tb_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
+        const uint4 wv = tb_rows(p.v_stb, s, e, doc, 4 * v, p.Hkv, g);
+        const uint4 wkc = tb_channel_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
         if (use > 0 && !warp_wait(st_empty + stg, (use - 1) & 1, wd, 72)) { ok = false; break; }
-        reinterpret_cast<uint4*>(sfb(5 + 3 * stg))[lane] = tb_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
-        reinterpret_cast<uint4*>(sfb(6 + 3 * stg))[lane] = tb_rows(p.v_stb, s, e, doc, 4 * v, p.Hkv, g);
-        reinterpret_cast<uint4*>(sfb(7 + 3 * stg))[lane] = tb_channel_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
+        reinterpret_cast<uint4*>(sfb(5 + 3 * stg))[lane] = wk;
+        reinterpret_cast<uint4*>(sfb(6 + 3 * stg))[lane] = wv;
+        reinterpret_cast<uint4*>(sfb(7 + 3 * stg))[lane] = wkc;
         fence_proxy_async_smem();
         if (lane == 0) {
           uint8_t* st = smem + oRing + stg * 2 * kCode;
@@ -339,7 +351,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       const uint32_t aQ = smem_u32(smem + oQ), aDO = smem_u32(smem + oDO), aRing = smem_u32(smem + oRing),
                      aKpt = smem_u32(smem + oKpt), aVpt = smem_u32(smem + oVpt), aKd = smem_u32(smem + oKd),
                      aDS = smem_u32(smem + oDS), aDSd = smem_u32(smem + oDSd), aSf = smem_u32(sf);
-      uint32_t st_it = 0, p_cnt = 0, sr_cnt = 0;
+      uint32_t kt = 0, s_uses = 0, dp_uses = 0;
       int unit_i = 0;
       bool ok = true;
       // D (tmem col) = A B^T, both K-major codes, block scales at TMEM cols sfa/sfb
@@ -352,42 +364,70 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
                       idesc_mxf8(128, 128, b_mn, kk, kk), (tmem + sfa) | ((uint32_t)kk << 30),
                       (tmem + sfbc) | ((uint32_t)kk << 30), (acc_first || kk > 0) ? 1u : 0u);
       };
+      auto region_s = [&]() {
+        if (s_uses > 0 && !mbar_wait(s_free, (s_uses - 1) & 1, wd, 73)) return false;
+        tc_fence_after();
+        return true;
+      };
+      auto region_dp = [&]() {
+        if (dp_uses > 0 && !mbar_wait(dp_free, (dp_uses - 1) & 1, wd, 74)) return false;
+        tc_fence_after();
+        return true;
+      };
+      // S and dP of key tile number tt (token-block K and V)
+      auto scores_tb = [&](uint32_t tt) {
+        const int stg = tt % kStages;
+        if (!mbar_wait(st_full + stg, (tt / kStages) & 1, wd, 75)) return false;
+        const uint32_t ak = aRing + stg * 2 * kCode, av = ak + kCode;
+        if (!region_s()) return false;
+        tmem_cp_sf(tmem + tSfK, aSf + (5 + 3 * stg) * kSfBlk);
+        mx_kk(tS, aQ, ak, tSfQ, tSfK, false, false);
+        tc_commit(s_full);
+        ++s_uses;
+        if (!region_dp()) return false;
+        tmem_cp_sf(tmem + tSfV, aSf + (6 + 3 * stg) * kSfBlk);
+        mx_kk(tDP, aDO, av, tSfDO, tSfV, false, false);
+        tc_commit(dp_full);
+        ++dp_uses;
+        return true;
+      };
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
         int doc, s, e, h, g, q0, n;
         decode(w, doc, s, e, h, g, q0, n);
-        if (!mbar_wait(q_full, unit_i & 1, wd, 73)) break;
+        if (!mbar_wait(q_full, unit_i & 1, wd, 76)) break;
         tc_fence_after();
         tmem_cp_sf(tmem + tSfQ, aSf + 0 * kSfBlk);
         tmem_cp_sf(tmem + tSfDO, aSf + 1 * kSfBlk);
         tmem_cp_sf(tmem + tSfKpt, aSf + 2 * kSfBlk);
         tmem_cp_sf(tmem + tSfVpt, aSf + 3 * kSfBlk);
-        for (int v = 0; v < n; ++v, ++st_it) {
-          const int stg = st_it % kStages;
-          if (!mbar_wait(st_full + stg, (st_it / kStages) & 1, wd, 74)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t ak = aRing + stg * 2 * kCode, av = ak + kCode;
-          tmem_cp_sf(tmem + tSfK, aSf + (5 + 3 * stg) * kSfBlk);
-          tmem_cp_sf(tmem + tSfV, aSf + (6 + 3 * stg) * kSfBlk);
-          mx_kk(tS, aQ, ak, tSfQ, tSfK, false, false);
-          mx_kk(tDP, aDO, av, tSfDO, tSfV, false, false);
-          tc_commit(s_full);
-          if (v == n - 1) {
-            // diagonal tile: per-token K and V into the same columns once read
-            if (!mbar_wait(s_read, sr_cnt & 1, wd, 75)) { ok = false; break; }
-            ++sr_cnt;
-            tc_fence_after();
+        if (!scores_tb(kt)) break;
+        for (int v = 0; v < n; ++v, ++kt) {
+          const int stg = kt % kStages;
+          const bool diag = v == n - 1;
+          if (diag) {
+            // diagonal tile: per-token K and V into the regions once the
+            // token-block scores were read
+            if (!region_s()) { ok = false; break; }
             mx_kk(tS, aQ, aKpt, tSfQ, tSfKpt, false, false);
-            mx_kk(tDP, aDO, aVpt, tSfDO, tSfVpt, false, false);
             tc_commit(s_full);
+            ++s_uses;
+            if (!region_dp()) { ok = false; break; }
+            mx_kk(tDP, aDO, aVpt, tSfDO, tSfVpt, false, false);
+            tc_commit(dp_full);
+            ++dp_uses;
+          } else if (!scores_tb(kt + 1)) {  // the next key tile goes ahead of this tile's dQ
+            ok = false;
+            break;
           }
-          if (!mbar_wait(p_full, p_cnt & 1, wd, 76)) { ok = false; break; }
-          ++p_cnt;
           if (v == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 77)) { ok = false; break; }
+          if (!mbar_wait(ds_ready, kt & 1, wd, 78)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t ak = aRing + stg * 2 * kCode;
           tmem_cp_sf(tmem + tSfDS, aSf + 4 * kSfBlk);
           tmem_cp_sf(tmem + tSfKdq, aSf + (7 + 3 * stg) * kSfBlk);
           mx_kk(tDQ, aDS, ak, tSfDS, tSfKdq, true, v > 0);
-          if (v == n - 1) {
+          if (diag) {
+            // diagonal 32x32 blocks: exact bf16 dS~ times dequantised per-token K
             constexpr uint32_t idesc_d = idesc_bf16_f32(128, 128, false, true);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
@@ -404,15 +444,29 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       tc_commit(fin);
       drain_wait(fin, 0, p.timeout_ns);
     }
-  } else {
-    // one thread per query row
-    const int row = warp * 32 + lane;
-    const uint32_t lb = tmem + ((uint32_t)(warp * 32) << 16);
+  } else if (warp < kComputeWarps) {
+    // one thread per (query row, key block wg)
+    const int wg = warp >> 2, quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lb = tmem + ((uint32_t)(quarter * 32) << 16);
     uint8_t* sDS = smem + oDS;
     uint8_t* sDSd = smem + oDSd;
-    uint32_t s_cnt = 0, dq_cnt = 0;
+    uint8_t* sfDS = sfb(4);
+    uint32_t s_cnt = 0, dp_cnt = 0, kt = 0;
     int unit_i = 0;
     bool ok = true;
+    auto take = [&](uint64_t* full, uint64_t* free_bar, uint32_t& cnt, uint32_t col, bool load, uint32_t (&r)[32]) {
+      if (!warp_wait(full, cnt & 1, wd, 79)) return false;
+      ++cnt;
+      tc_fence_after();
+      if (load) {
+        tmem_ld32(lb + col + 32 * wg, r);
+        tmem_wait_ld(r);
+      }
+      tc_fence_before();
+      warp_arrive(free_bar);
+      return true;
+    };
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
       int doc, s, e, h, g, q0, n;
       decode(w, doc, s, e, h, g, q0, n);
@@ -421,107 +475,68 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       // rows past the document end get P = 0
       const float l2 = valid ? p.lse[(size_t)h * p.T + i] * kLog2e : INFINITY;
       const float dl = valid ? p.delta[(size_t)h * p.T + i] : 0.f;
-      for (int v = 0; v < n; ++v) {
-        if (!warp_wait(s_full, s_cnt & 1, wd, 77)) { ok = false; break; }
-        ++s_cnt;
-        tc_fence_after();
+      for (int v = 0; v < n; ++v, ++kt) {
         const bool diag = v == n - 1;
-        uint32_t codes[32];
-        uint32_t sfword = 0;
-        uint32_t pd[16];
-        // key blocks of this tile; on the diagonal tile block `warp` is the
-        // diagonal block (per-token operands, second phase) and later blocks
-        // are future keys (dS = 0)
+        // on the diagonal tile block `quarter` of this row is its own 32-key
+        // block (per-token operands, second phase); later blocks are future keys
+        const bool own = diag && wg == quarter;
+        const bool future = diag && wg > quarter;
+        uint32_t r[32];
+        float ds[32];
+        // ---- S -> P (in place)
+        if (!take(s_full, s_free, s_cnt, tS, !own && !future, r)) { ok = false; break; }
+        if (diag && !take(s_full, s_free, s_cnt, tS, own, r)) { ok = false; break; }
+        if (future) {
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          float ds[32];
-          if (diag && kb > warp) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) ds[c] = 0.f;
-          } else if (diag && kb == warp) {
-            continue;  // second phase below
-          } else {
-            uint32_t rs[32], rd[32];
-            tmem_ld32(lb + tS + 32 * kb, rs);
-            tmem_ld32(lb + tDP + 32 * kb, rd);
-            tmem_wait_ld(rs);
-            tmem_wait_ld(rd);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float pp = fast_exp2(__uint_as_float(rs[c]) * p.scale_log2 - l2);
-              ds[c] = pp * (__uint_as_float(rd[c]) - dl);
-            }
-          }
-          uint32_t cw[8];
-          const uint32_t sb = quant32(ds, p.rule, cw);
-          sfword |= sb << (8 * kb);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) codes[8 * kb + c] = cw[c];
-        }
-        if (diag) {
-          tc_fence_before();
-          mbar_arrive(s_read);
-          if (!warp_wait(s_full, s_cnt & 1, wd, 78)) { ok = false; break; }
-          ++s_cnt;
-          tc_fence_after();
-          uint32_t rs[32], rd[32];
-          tmem_ld32(lb + tS + 32 * warp, rs);
-          tmem_ld32(lb + tDP + 32 * warp, rd);
-          tmem_wait_ld(rs);
-          tmem_wait_ld(rd);
-          float ds[32];
+          for (int c = 0; c < 32; ++c) ds[c] = 0.f;
+        } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float pp = (32 * warp + c <= row) ? fast_exp2(__uint_as_float(rs[c]) * p.scale_log2 - l2) : 0.f;
-            ds[c] = pp * (__uint_as_float(rd[c]) - dl);
+            const float pp = fast_exp2(__uint_as_float(r[c]) * p.scale_log2 - l2);
+            ds[c] = (!own || c <= lane) ? pp : 0.f;
           }
-          uint32_t cw[8];
-          const uint32_t sb = quant32(ds, p.rule, cw);
-          sfword |= sb << (8 * warp);
-          dequant32_bf16(cw, sb, pd);
-          // the diagonal block leaves the FP8 operand (it goes through the bf16 MMA)
+        }
+        // ---- dP -> dS = P (dP - D)
+        if (!take(dp_full, dp_free, dp_cnt, tDP, !own && !future, r)) { ok = false; break; }
+        if (diag && !take(dp_full, dp_free, dp_cnt, tDP, own, r)) { ok = false; break; }
+        if (!future) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            if (warp == 0) codes[c] = 0;
-            else if (warp == 1) codes[8 + c] = 0;
-            else if (warp == 2) codes[16 + c] = 0;
-            else codes[24 + c] = 0;
-          }
+          for (int c = 0; c < 32; ++c) ds[c] = ds[c] * (__uint_as_float(r[c]) - dl);
+        }
+        uint32_t cw[8];
+        const uint32_t sb = quant32(ds, p.rule, cw);
+        uint32_t pd[16];
+        if (own) {
+          // the diagonal block leaves the FP8 operand (it goes through the bf16 MMA)
+          dequant32_bf16(cw, sb, pd);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cw[c] = 0;
         }
         // dQ of the previous tile must have read the dS buffers
-        if (v > 0) {
-          if (!warp_wait(dq_done, dq_cnt & 1, wd, 79)) { ok = false; break; }
-          ++dq_cnt;
-        }
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          uint32_t cw[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) cw[c] = codes[8 * kb + c];
-          store_codes32(sDS, row, 2 * kb, cw);
-        }
-        reinterpret_cast<uint32_t*>(smem + oSf + 4 * kSfBlk)[(row & 31) * 4 + (row >> 5)] = sfword;
+        if (kt > 0 && !warp_wait(dq_done, (kt - 1) & 1, wd, 80)) { ok = false; break; }
+        store_codes32(sDS, row, 2 * wg, cw);
+        sfDS[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)sb;
         if (diag) {
-          zero_bf16_row(sDSd, row);
-          store_bf16_32(sDSd, row, warp, pd);
+          if (!own) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pd[c] = 0;
+          }
+          store_bf16_32(sDSd, row, wg, pd);
         }
         fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(p_full);
+        warp_arrive(ds_ready);
       }
       if (!ok) break;
-      if (!warp_wait(acc_full, unit_i & 1, wd, 80)) break;
-      ++dq_cnt;  // the last tile's dQ completion is covered by acc_full
+      if (!warp_wait(acc_full, unit_i & 1, wd, 81)) break;
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      {
         uint32_t t[32];
-        tmem_ld32(lb + tDQ + 32 * c, t);
+        tmem_ld32(lb + tDQ + 32 * wg, t);
         tmem_wait_ld(t);
-        if (valid) store_row32(p.out0, ((size_t)i * p.Hq + h) * 128 + 32 * c, t, p.scale, p.grad_bf16);
+        if (valid) store_row32(p.out0, ((size_t)i * p.Hq + h) * 128 + 32 * wg, t, p.scale, p.grad_bf16);
       }
       tc_fence_before();
-      mbar_arrive(acc_free);
+      warp_arrive(acc_free);
     }
   }
 
