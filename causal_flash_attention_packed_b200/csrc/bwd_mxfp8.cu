@@ -550,10 +550,10 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
 // dK, dV
 // ---------------------------------------------------------------------------
 namespace kvk {
-// warps 0-7: one thread per key row (warpgroup w on query columns
-// [64w, 64w + 64)); warp 8: K/V, Q^pt, dO^pt, lse and D loads; warp 9: MMA
-// issue; warp 10: dO^tb and Q^tb loads
-constexpr int kThreads = 352, kLoadA = 8, kMma = 9, kLoadB = 10;
+// warps 0-15: one thread per (key row, 32-query block): warpgroup wg on query
+// block wg of every tile (one MX scale block of P~T and dS~T); warp 16: K/V,
+// Q^pt, dO^pt, lse and D loads; warp 17: MMA issue; warp 18: dO^tb and Q^tb loads
+constexpr int kThreads = 608, kLoadA = 16, kMma = 17, kLoadB = 18, kComputeWarps = 16;
 // per item: K^tb, K^pt, V^tb, V^pt codes; per query tile one buffer per
 // operand (Q^pt, dO^pt, dO^tb, Q^tb codes), each released as soon as its last
 // MMA has read it; P~T and dS~T codes; lse*log2e[128] and D[128] of the query
@@ -619,16 +619,16 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(aux_full + i, 32);
-      mbar_init(aux_empty + i, 256);
+      mbar_init(aux_empty + i, kComputeWarps);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 256);
-    mbar_init(p_full, 256);
+    mbar_init(s_free, kComputeWarps);
+    mbar_init(p_full, kComputeWarps);
     mbar_init(p_empty, 1);
-    mbar_init(ds_full, 256);
+    mbar_init(ds_full, kComputeWarps);
     mbar_init(ds_empty, 1);
     mbar_init(acc_full, 1);
-    mbar_init(acc_free, 256);
+    mbar_init(acc_free, kComputeWarps);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -856,9 +856,9 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
       tc_commit(fin);
       drain_wait(fin, 0, p.timeout_ns);
     }
-  } else if (warp < 8) {
+  } else if (warp < kComputeWarps) {
     // ------------------------------------------------- P~T, dS~T
-    // one thread per key row; warpgroup wg on query columns [64 wg, 64 wg + 64)
+    // one thread per (key row, query block wg)
     const int wg = warp >> 2, quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lb = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -866,48 +866,22 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     uint8_t* sDS = smem + oDS;
     uint8_t* sfP = sfb(8);
     uint8_t* sfDS = sfb(9);
-    // this row's diagonal query block (columns [32 quarter, 32 quarter + 32))
-    // lies in this warpgroup's half iff quarter >> 1 == wg
-    const bool own_diag = (quarter >> 1) == wg;
     uint32_t s_cnt = 0, t = 0;
     int unit_i = 0;
     bool ok = true;
-    auto take = [&]() {
-      const bool r = warp_wait(s_full, s_cnt & 1, wd, 96);
+    // one use of the S/dP region: wait for it, read this thread's block if
+    // `load`, release it
+    auto take = [&](bool load, uint32_t (&r)[32]) {
+      if (!warp_wait(s_full, s_cnt & 1, wd, 96)) return false;
       ++s_cnt;
       tc_fence_after();
-      return r;
-    };
-    auto release = [&]() {
+      if (load) {
+        tmem_ld32(lb + tSD + 32 * wg, r);
+        tmem_wait_ld(r);
+      }
       tc_fence_before();
-      mbar_arrive(s_free);
-    };
-    // the 64 values of this row in this warpgroup's half of the region
-    auto read_half = [&](float (&x)[64]) {
-      uint32_t a[32], b[32];
-      tmem_ld32(lb + tSD + 64 * wg, a);
-      tmem_ld32(lb + tSD + 64 * wg + 32, b);
-      tmem_wait_ld(a);
-      tmem_wait_ld(b);
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(a[c]);
-        x[32 + c] = __uint_as_float(b[c]);
-      }
-    };
-    // the diagonal block from the per-token phase replaces the token-block values
-    auto read_diag = [&](float (&x)[64]) {
-      if (!own_diag) return;
-      uint32_t a[32];
-      tmem_ld32(lb + tSD + 32 * quarter, a);
-      tmem_wait_ld(a);
-      if (quarter & 1) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[32 + c] = __uint_as_float(a[c]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(a[c]);
-      }
+      warp_arrive(s_free);
+      return true;
     };
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
       int doc, s, e, g, v, k0, nq;
@@ -916,82 +890,77 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
       for (int h = g * G; h < (g + 1) * G && ok; ++h) {
         for (int m = v; m < nq; ++m, ++t) {
           const bool diag = m == v;
+          // on the diagonal tile query block `quarter` is this key row's own
+          // 32-query block (per-token operands, second phase); earlier query
+          // blocks precede the key (P = 0)
+          const bool own = diag && wg == quarter;
+          const bool past = diag && wg < quarter;
           const int ab = t & 1;
           if (!warp_wait(aux_full + ab, (t >> 1) & 1, wd, 97)) { ok = false; break; }
-          const float* lse2 = reinterpret_cast<const float*>(smem + oAux + ab * 1024) + 64 * wg;
+          const float* lse2 = reinterpret_cast<const float*>(smem + oAux + ab * 1024) + 32 * wg;
           const float* dl = lse2 + 128;
-          // ---- S^T -> P, P~T into shared memory
-          float pr[64];
-          if (!take()) { ok = false; break; }
-          read_half(pr);
-          release();
-          if (diag) {
-            if (!take()) { ok = false; break; }
-            read_diag(pr);
-            release();
-          }
+          uint32_t r[32];
+          float pr[32];
+          // ---- S^T -> P (kept in registers), P~T into shared memory
+          if (!take(!own && !past, r)) { ok = false; break; }
+          if (diag && !take(own, r)) { ok = false; break; }
+          if (past) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            // on the diagonal tile query column 64 wg + c is visible iff it is >= the key row
-            const bool vis = !diag || (64 * wg + c >= row);
-            pr[c] = vis ? fast_exp2(pr[c] * p.scale_log2 - lse2[c]) : 0.f;
+            for (int c = 0; c < 32; ++c) pr[c] = 0.f;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              // on the own block query column c is visible iff it is >= the key row
+              const float pp = fast_exp2(__uint_as_float(r[c]) * p.scale_log2 - lse2[c]);
+              pr[c] = (!own || c >= lane) ? pp : 0.f;
+            }
           }
           if (t > 0 && !warp_wait(p_empty, (t - 1) & 1, wd, 98)) { ok = false; break; }
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            float blk[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) blk[c] = pr[32 * u + c];
+          {
             uint32_t cw[8];
-            const uint32_t sb = quant32(blk, p.rule, cw);
-            store_codes32(sP, row, 2 * (2 * wg + u), cw);
-            sfP[(row & 31) * 16 + (row >> 5) * 4 + 2 * wg + u] = (uint8_t)sb;
+            const uint32_t sb = quant32(pr, p.rule, cw);
+            store_codes32(sP, row, 2 * wg, cw);
+            sfP[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)sb;
           }
           fence_proxy_async_smem();
-          mbar_arrive(p_full);
+          warp_arrive(p_full);
           // ---- dP^T -> dS~T into shared memory
-          float dp[64];
-          if (!take()) { ok = false; break; }
-          read_half(dp);
-          release();
-          if (diag) {
-            if (!take()) { ok = false; break; }
-            read_diag(dp);
-            release();
-          }
+          if (!take(!own && !past, r)) { ok = false; break; }
+          if (diag && !take(own, r)) { ok = false; break; }
           if (t > 0 && !warp_wait(ds_empty, (t - 1) & 1, wd, 99)) { ok = false; break; }
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
+          {
             float blk[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) blk[c] = pr[32 * u + c] * (dp[32 * u + c] - dl[32 * u + c]);
+            for (int c = 0; c < 32; ++c) blk[c] = past ? 0.f : pr[c] * (__uint_as_float(r[c]) - dl[c]);
             uint32_t cw[8];
             const uint32_t sb = quant32(blk, p.rule, cw);
-            store_codes32(sDS, row, 2 * (2 * wg + u), cw);
-            sfDS[(row & 31) * 16 + (row >> 5) * 4 + 2 * wg + u] = (uint8_t)sb;
+            store_codes32(sDS, row, 2 * wg, cw);
+            sfDS[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)sb;
           }
           fence_proxy_async_smem();
-          mbar_arrive(ds_full);
-          mbar_arrive(aux_empty + ab);
+          warp_arrive(ds_full);
+          warp_arrive(aux_empty + ab);
         }
       }
       if (!ok) break;
-      // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK * scale
+      // epilogue: warpgroups 0, 1 write halves of dV, warpgroups 2, 3 halves of dK * scale
       if (!warp_wait(acc_full, unit_i & 1, wd, 100)) break;
       tc_fence_after();
       const bool valid = j < e;
-      const uint32_t acc = lb + (wg ? tDK : tDV);
-      void* out = wg ? p.out0 : p.out1;
-      const float mul = wg ? p.scale : 1.f;
+      const bool is_k = wg >= 2;
+      const int c0 = (wg & 1) * 64;
+      const uint32_t acc = lb + (is_k ? tDK : tDV) + c0;
+      void* out = is_k ? p.out0 : p.out1;
+      const float mul = is_k ? p.scale : 1.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t tt[32];
         tmem_ld32(acc + 32 * c, tt);
         tmem_wait_ld(tt);
-        if (valid) store_row32(out, ((size_t)j * p.Hkv + g) * 128 + 32 * c, tt, mul, p.grad_bf16);
+        if (valid) store_row32(out, ((size_t)j * p.Hkv + g) * 128 + c0 + 32 * c, tt, mul, p.grad_bf16);
       }
       tc_fence_before();
-      mbar_arrive(acc_free);
+      warp_arrive(acc_free);
     }
   }
 
