@@ -10,11 +10,15 @@
 // the token-block forms and keys of its own block through the per-token forms,
 // so no shared scale pools a future token.
 //
-// One persistent CTA per SM, 192 threads; work item = (document, 128-row
-// query tile, head).  Warps 0-3: one thread per query row (softmax, P
-// quantisation, epilogue); warp 4: loads (TMA for codes, plain loads for the
-// scale bytes, staged into the 512-byte blocks tcgen05.cp copies to TMEM);
-// warp 5 (one lane): MMAs.
+// One persistent CTA per SM, 576 threads; work item = (document, 128-row
+// query tile, head).  Warps 0-15: one thread per (query row, 32-key block):
+// warpgroup wg takes key block wg of every tile, i.e. one MX scale block of
+// P~ (softmax, P quantisation, epilogue of O columns [32 wg, 32 wg + 32));
+// the four threads of a row exchange their block maxima through shared
+// memory (an mbarrier per row quarter, bounded waits) so they all move the
+// reference M alike, and add their partial row sums at the end.  Warp 16:
+// loads (TMA for codes, plain loads for the scale bytes, staged into the
+// 512-byte blocks tcgen05.cp copies to TMEM); warp 17 (one lane): MMAs.
 //  * S = Q K^T for every key tile: block-scaled FP8 MMA (kind::mxf8f6f4,
 //    E8M0 scales in TMEM) with K in token-block form; on the diagonal tile a
 //    second S with K per token, selected on the diagonal 32x32 blocks.
@@ -39,9 +43,10 @@ namespace fapk {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kLoadWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kThreads = 576;
+constexpr int kLoadWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kComputeWarps = 16;
 constexpr int kSlots = 6;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -58,8 +63,10 @@ constexpr int oPd = oP + kCodeTile;
 constexpr int oRing = oPd + kBf16Tile;
 constexpr int oSf = oRing + kSlots * kCodeTile;  // sfQ, sfKpt, sfP, sfRing[kSlots]
 constexpr int kSfBlk = 512;
-constexpr int oBars = oSf + (3 + kSlots) * kSfBlk;
-constexpr int kNumBars = 2 + 2 * kSlots + 8;
+constexpr int oXmax = oSf + (3 + kSlots) * kSfBlk;  // block maxima [2][4][128] (by tile parity)
+constexpr int oLsum = oXmax + 2 * 4 * 128 * 4;       // partial row sums [4][128]
+constexpr int oBars = oLsum + 4 * 128 * 4;
+constexpr int kNumBars = 2 + 2 * kSlots + 8 + 4;  // + one row-exchange barrier per row quarter
 constexpr int kSmemBytes = oBars + kNumBars * 8 + 16 + 1024;
 
 // TMEM columns
@@ -112,6 +119,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
 }
 
+// One arrival per warp, after every lane's prior work (warp barrier first).
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // 4 scale bytes of token t (per-token form), or the neutral byte 127 (2^0)
 // past the end of the tensor.
 __device__ __forceinline__ uint32_t pt_word(const uint8_t* spt, int t, int T, int H, int h) {
@@ -155,6 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_full = s_full + 4;
   uint64_t* o_free = s_full + 5;
   uint64_t* fin = s_full + 6;
+  uint64_t* xbar = s_full + 7;  // [4]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -168,11 +182,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_full + 1, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, kComputeWarps);
     mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
-    mbar_init(o_free, 128);
+    mbar_init(o_free, kComputeWarps);
     mbar_init(fin, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(xbar + i, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -357,55 +372,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(fin);
       drain_wait(fin, 0, p.timeout_ns);
     }
-  } else {
+  } else if (warp < kComputeWarps) {
     // ------------------------------------------------------------ softmax
-    const int row = warp * 32 + lane;  // query row = TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    uint32_t s_cnt[2] = {0, 0}, pv_cnt = 0, o_cnt = 0;
+    const int wg = warp >> 2, quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // query row = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    float* xmax = reinterpret_cast<float*>(smem + oXmax);
+    float* lsum = reinterpret_cast<float*>(smem + oLsum);
+    // the four warps that share this row quarter meet here (bounded wait)
+    uint32_t x_cnt = 0;
+    auto row_sync = [&]() {
+      warp_arrive(xbar + quarter);
+      const bool r = warp_wait(xbar + quarter, x_cnt & 1, wd, 60);
+      ++x_cnt;
+      return r;
+    };
+    uint32_t s_cnt[2] = {0, 0}, pv_cnt = 0, o_cnt = 0, tiles = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
       const Item it = decode(p, w);
       const int n = it.n;
       const int q_idx = it.q0 + row;
-      float M = -INFINITY, l = 0.f;
-      for (int j = 0; j < n; ++j) {
+      float M = -INFINITY, l = 0.f;  // l: this thread's share of the row sum
+      for (int j = 0; j < n; ++j, ++tiles) {
         const int sbi = j & 1;
         if (!warp_wait(s_full + sbi, (sbi ? s_cnt[1] : s_cnt[0]) & 1, wd, 57)) { ok = false; break; }
         if (sbi) ++s_cnt[1]; else ++s_cnt[0];
         tc_fence_after();
         const bool diag = j == n - 1;
-        const uint32_t sb = lane_base + ((j & 1) ? kS1 : kS0);
-        uint32_t r[128];
-        tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_ld32(sb + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-        tmem_ld32(sb + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
-        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[96]));
-        if (diag) {
-          // per-token scores of this row's own 32-key block (the warp's block)
-          uint32_t rp[32];
-          tmem_ld32(lane_base + ((j & 1) ? kS0 : kS1) + 32 * warp, rp);
-          tmem_wait_ld(rp);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            // warp-uniform select of the 32 columns of block `warp`
-            if (warp == 0) r[c] = rp[c];
-            else if (warp == 1) r[32 + c] = rp[c];
-            else if (warp == 2) r[64 + c] = rp[c];
-            else r[96 + c] = rp[c];
-          }
+        // on the diagonal tile key block `quarter` is this row's own block
+        // (per-token scores, from the other buffer); later blocks are future keys
+        const bool own = diag && wg == quarter;
+        const bool future = diag && wg > quarter;
+        uint32_t r[32];
+        if (!future) {
+          tmem_ld32(lane_base + (own ? ((j & 1) ? kS0 : kS1) : ((j & 1) ? kS1 : kS0)) + 32 * wg, r);
+          tmem_wait_ld(r);
         }
-        float x[128];
-        float mx = -INFINITY;
+        float x[32];
+        float bmax = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const bool vis = !diag || (c <= row);
+        for (int c = 0; c < 32; ++c) {
+          const bool vis = !future && (!own || c <= lane);
           x[c] = vis ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, x[c]);
+          bmax = fmaxf(bmax, x[c]);
         }
+        float* xm = xmax + (tiles & 1) * 512;
+        xm[wg * 128 + row] = bmax;
+        if (!row_sync()) { ok = false; break; }
+        const float mx = fmaxf(fmaxf(xm[row], xm[128 + row]), fmaxf(xm[256 + row], xm[384 + row]));
         float alpha = 1.f;
         if (mx > M + kRescaleThreshold) {
           const float Mn = ceilf(mx);
@@ -416,53 +431,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           M = Mn;
         }
         const bool any_rescale = __any_sync(0xFFFFFFFFu, alpha != 1.f) && j > 0;
-        // u = 2^(x - M), row sum before quantisation, then MX quantisation per 32-key block
-        uint32_t codes[32];
-        uint32_t sfword = 0;
-        float rs = 0.f;
+        // u = 2^(x - M), row sum before quantisation, MX quantisation of the block
+        float rs = 0.f, amax = 0.f;
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          float amax = 0.f;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            x[32 * kb + c] = fast_exp2(x[32 * kb + c] - M);
-            rs += x[32 * kb + c];
-            amax = fmaxf(amax, x[32 * kb + c]);
-          }
-          const int X = mx_block_exponent(amax, p.rule);
-          const float sc = mx_pow2_neg(X < -126 ? -126 : X);
-          sfword |= (uint32_t)(X + 127) << (8 * kb);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float* u = &x[32 * kb + 4 * c];
-            codes[8 * kb + c] = mx_e4m3x2(u[0] * sc, u[1] * sc) | (mx_e4m3x2(u[2] * sc, u[3] * sc) << 16);
-          }
+        for (int c = 0; c < 32; ++c) {
+          x[c] = fast_exp2(x[c] - M);
+          rs += x[c];
+          amax = fmaxf(amax, x[c]);
         }
         l += rs;
-        // bf16 copy of the diagonal 32-block's P~ (exact), and zero FP8 codes there
+        const int X = mx_block_exponent(amax, p.rule);
+        const float sc = mx_pow2_neg(X < -126 ? -126 : X);
+        uint32_t codes[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          codes[c] = mx_e4m3x2(x[4 * c] * sc, x[4 * c + 1] * sc) | (mx_e4m3x2(x[4 * c + 2] * sc, x[4 * c + 3] * sc) << 16);
+        // bf16 copy of the own block's P~ (exact); its FP8 codes are zeroed
         uint32_t pd[16];
-        if (diag) {
-          const int X = (int)((sfword >> (8 * warp)) & 0xFFu) - 127;
-          const float sc = mx_pow2(X < -126 ? -126 : X);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pd[c] = 0;
+        if (own) {
+          const float scd = mx_pow2(X < -126 ? -126 : X);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            uint32_t w4 = 0;
-            if (warp == 0) w4 = codes[c];
-            else if (warp == 1) w4 = codes[8 + c];
-            else if (warp == 2) w4 = codes[16 + c];
-            else w4 = codes[24 + c];
             float a, b, cc, d;
-            mx_decode2(w4 & 0xFFFFu, a, b);
-            mx_decode2(w4 >> 16, cc, d);
-            pd[2 * c] = pack_bf16x2(a * sc, b * sc);
-            pd[2 * c + 1] = pack_bf16x2(cc * sc, d * sc);
-          }
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            if (warp == 0) codes[c] = 0;
-            else if (warp == 1) codes[8 + c] = 0;
-            else if (warp == 2) codes[16 + c] = 0;
-            else codes[24 + c] = 0;
+            mx_decode2(codes[c] & 0xFFFFu, a, b);
+            mx_decode2(codes[c] >> 16, cc, d);
+            pd[2 * c] = pack_bf16x2(a * scd, b * scd);
+            pd[2 * c + 1] = pack_bf16x2(cc * scd, d * scd);
+            codes[c] = 0;
           }
         }
         // PV(j-1) must be done before P's shared buffer and O are touched
@@ -471,57 +468,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++pv_cnt;
           tc_fence_after();
         }
-        // P codes: row `row`, 128 bytes = 8 chunks of 16 bytes, 128-byte swizzle
+        // P codes: row `row`, 16-byte chunks 2 wg, 2 wg + 1 (128-byte swizzle)
         {
           uint8_t* prow = sP + row * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
-                make_uint4(codes[4 * c], codes[4 * c + 1], codes[4 * c + 2], codes[4 * c + 3]);
-          reinterpret_cast<uint32_t*>(sfP)[(row & 31) * 4 + (row >> 5)] = sfword;
+          *reinterpret_cast<uint4*>(prow + (((2 * wg) ^ (row & 7)) << 4)) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+          *reinterpret_cast<uint4*>(prow + (((2 * wg + 1) ^ (row & 7)) << 4)) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+          sfP[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)(X + 127);
         }
         if (diag) {
-          // P_diag: bf16, two 64-key boxes of 128 rows x 128 bytes; only block `warp` is non-zero
+          // P_diag: bf16, two 64-key boxes of 128 rows x 128 bytes; only the own block is non-zero
+          const int box = wg >> 1, c0 = (wg & 1) * 4;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {  // 16 chunks of 8 bf16 over the 128 keys
-            const int box = c >> 3, cc = c & 7;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if ((c >> 2) == warp) {
-              const int q = c & 3;
-              v = make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
-            }
-            *reinterpret_cast<uint4*>(sPd + box * kBox + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
-          }
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(sPd + box * kBox + row * 128 + (((c0 + c) ^ (row & 7)) << 4)) =
+                make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
         }
         if (any_rescale) {
+          uint32_t t[32];
+          tmem_ld32(lane_base + kO + 32 * wg, t);
+          tmem_wait_ld(t);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t t[32];
-            tmem_ld32(lane_base + kO + 32 * c, t);
-            tmem_wait_ld(t);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
-            tmem_st32(lane_base + kO + 32 * c, t);
-          }
+          for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
+          tmem_st32(lane_base + kO + 32 * wg, t);
           tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(p_full);
+        warp_arrive(p_full);
       }
       if (!ok) break;
-      // epilogue
+      // epilogue: the row sum from the four block shares, O columns [32 wg, 32 wg + 32)
+      lsum[wg * 128 + row] = l;
+      if (!row_sync()) break;
+      const float lt = (lsum[row] + lsum[128 + row]) + (lsum[256 + row] + lsum[384 + row]);
       if (!warp_wait(o_full, o_cnt & 1, wd, 59)) break;
       ++o_cnt;
       ++pv_cnt;  // the last tile's PV completion is covered by o_full
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = 1.f / lt;
       const bool valid = q_idx < it.e;
-      __nv_bfloat16* orow = p.o + ((size_t)q_idx * p.Hq + it.h) * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      {
         uint32_t t[32];
-        tmem_ld32(lane_base + kO + 32 * c, t);
+        tmem_ld32(lane_base + kO + 32 * wg, t);
         tmem_wait_ld(t);
         uint32_t ob[16], rb[16];
 #pragma unroll
@@ -531,8 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           rb[e] = pack_bf16x2(f0 - __uint_as_float(ob[e] << 16), f1 - __uint_as_float(ob[e] & 0xFFFF0000u));
         }
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-          uint4* rdst = reinterpret_cast<uint4*>(p.o_resid + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * c);
+          uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * wg);
+          uint4* rdst = reinterpret_cast<uint4*>(p.o_resid + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * wg);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
@@ -541,8 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(o_free);
-      if (valid) p.lse[(size_t)it.h * p.T + q_idx] = (M + __log2f(l)) * kLn2;
+      warp_arrive(o_free);
+      if (valid && wg == 0) p.lse[(size_t)it.h * p.T + q_idx] = (M + __log2f(lt)) * kLn2;
     }
   }
 
