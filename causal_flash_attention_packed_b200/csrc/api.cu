@@ -92,7 +92,7 @@ uint64_t timeout_ns_of(const fapk_problem_t* P) {
 
 // --- workspace layout ---
 struct SchedLayout {
-  size_t level_off, n_items, list, end;
+  size_t scratch, docs, counts, next, end;
   int max_levels, max_items;
 };
 
@@ -100,19 +100,21 @@ SchedLayout sched_layout(size_t base, int T, int n_docs, int max_seqlen, int row
   SchedLayout s;
   s.max_levels = (max_seqlen + rows - 1) / rows;
   s.max_items = T / rows + n_docs + 1;
-  s.level_off = align_up(base);
-  s.n_items = align_up(s.level_off + sizeof(int) * (size_t)(s.max_levels + 2));
-  s.list = align_up(s.n_items + sizeof(int));
-  s.end = align_up(s.list + sizeof(int2) * (size_t)s.max_items);
+  s.scratch = align_up(base);
+  s.docs = align_up(s.scratch + sizeof(int) * 3 * (size_t)(s.max_levels + 2));
+  s.counts = align_up(s.docs + sizeof(int2) * (size_t)(n_docs > 0 ? n_docs : 1));
+  s.next = align_up(s.counts + 2 * sizeof(int));
+  s.end = align_up(s.next + sizeof(int));
   return s;
 }
 
 SchedBuf sched_buf(void* ws, const SchedLayout& s) {
   char* w = static_cast<char*>(ws);
   SchedBuf b;
-  b.level_off = reinterpret_cast<int*>(w + s.level_off);
-  b.n_items = reinterpret_cast<int*>(w + s.n_items);
-  b.list = reinterpret_cast<int2*>(w + s.list);
+  b.scratch = reinterpret_cast<int*>(w + s.scratch);
+  b.docs = reinterpret_cast<int2*>(w + s.docs);
+  b.counts = reinterpret_cast<int*>(w + s.counts);
+  b.next = reinterpret_cast<int*>(w + s.next);
   b.max_levels = s.max_levels;
   b.max_items = s.max_items;
   return b;
@@ -233,24 +235,12 @@ bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_tmap_flat_f32(CUtensorMap* map, const float* base, long long n, int box) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[1] = {(cuuint64_t)n};
-  const cuuint64_t strides[1] = {4};  // unused for a 1-D map
-  const cuuint32_t boxd[1] = {(cuuint32_t)box};
-  const cuuint32_t estr[1] = {1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<float*>(base), dims, strides, boxd, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16, int box_rows) {
+bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
-  const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  const cuuint32_t box[3] = {64, 1, 128};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
              const_cast<void*>(base), dims, strides, box, estr,
@@ -272,7 +262,7 @@ int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void*
   FwdMxArgs a;
   a.sched = sched_buf(ws, L.sched);
   mk.at(0, st);
-  int rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, kSchedQ, a.sched, status, true, st));
+  int rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, a.sched, status, true, st));
   if (rc != FAPK_OK) return rc;
   mk.at(1, st);
   const int forms = FAPK_FORM_TB | FAPK_FORM_PT;
@@ -330,10 +320,10 @@ int bwd_mxfp8(const fapk_problem_t* P, const void* o, const float* lse, const vo
   a.sched_kv = sched_buf(ws, L.kv);
   a.sched_q = sched_buf(ws, L.q);
   a.marks.at(0, st);
-  int rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedKV, a.sched_kv, status, true, st));
+  int rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, a.sched_kv, status, true, st));
   if (rc != FAPK_OK) return rc;
   a.marks.at(1, st);
-  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedQ, a.sched_q, status, false, st));
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, a.sched_q, status, false, st));
   if (rc != FAPK_OK) return rc;
   a.marks.at(2, st);
   rc = cuda_status(launch_quantize_mxfp8(dout, P->T, P->Hq, P->d, P->cu_seqlens_dev, P->n_docs,
@@ -414,7 +404,7 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
   a.num_sms = sms;
   const Marks mk{P->timing_events, P->n_timing_events};
   mk.at(0, st);
-  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRows, kSchedQ, a.sched, status, true, st));
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRows, a.sched, status, true, st));
   if (rc != FAPK_OK) return rc;
   mk.at(1, st);
   rc = cuda_status(launch_convert_f16(v, a.v16, (long long)P->T * P->Hkv * P->d, status, sms, st));
@@ -467,10 +457,10 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   a.num_sms = sms;
   a.marks = Marks{P->timing_events, P->n_timing_events};
   a.marks.at(0, st);
-  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedKV, a.sched_kv, status, true, st));
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, a.sched_kv, status, true, st));
   if (rc != FAPK_OK) return rc;
   a.marks.at(1, st);
-  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, kSchedQ, a.sched_q, status, false, st));
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, a.sched_q, status, false, st));
   if (rc != FAPK_OK) return rc;
   a.marks.at(2, st);
   rc = cuda_status(launch_convert_f16(k, a.k16, (long long)P->T * P->Hkv * P->d, status, sms, st));

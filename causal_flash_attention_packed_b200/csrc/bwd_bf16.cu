@@ -31,6 +31,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "sched.cuh"
 
 namespace fapk {
 
@@ -124,8 +125,7 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
 
 struct BwdParams {
   const int32_t* cu;
-  const int2* list;
-  const int* n_items;
+  SchedView sched;
   const float* lse;
   const float* delta;
   const float* nl2;  // -LSE log2(e), [Hq][T]
@@ -187,23 +187,23 @@ struct KvCfg : Geo<D> {
   static constexpr uint32_t kDV = 0, kDK = 128, kSD = 256, kP = 384, kDS = 448;
   // bars: kv_full, kv_empty, q_full[Q], q_empty[Q], o_full[O], o_empty[O], s_full, s_free, p_ready,
   //       ds_ready, dv_done, dk_done, acc_full, acc_free, fin
-  static constexpr int kNumBars = 2 + 2 * kQStages + 2 * kOStages + 9;
+  // + the unit ring's full[8] and empty[8]
+  static constexpr int kNumBars = 2 + 2 * kQStages + 2 * kOStages + 9 + 2 * kUnitRing;
   // no alignment slack: the kernel checks that dynamic shared memory starts
   // on a 1024-byte boundary
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 4 * kUnitRing;
 };
 
 struct KvItem {
   int s, e, v, g, k0, nq;  // k0: first key of the tile; query tiles v..nq-1
 };
 
-__device__ __forceinline__ KvItem kv_decode(const BwdParams& p, int w) {
+__device__ __forceinline__ KvItem kv_decode(const BwdParams& p, const UnitSpace& us, int w) {
   KvItem it;
-  const int2 pr = p.list[w / p.Hkv];
-  it.g = w % p.Hkv;
-  it.s = p.cu[pr.x];
-  it.e = p.cu[pr.x + 1];
-  it.v = pr.y;
+  int doc;
+  unit_decode(us, w, doc, it.v, it.g);
+  it.s = p.cu[doc];
+  it.e = p.cu[doc + 1];
   it.k0 = it.s + 128 * it.v;
   it.nq = (it.e - it.s + 127) / 128;
   return it;
@@ -250,6 +250,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   uint64_t* acc_full = s_full + 6;
   uint64_t* acc_free = s_full + 7;
   uint64_t* fin = s_full + 8;
+  const UnitRing ring{reinterpret_cast<int*>(bars + C::kNumBars) + 4, bars + C::kNumBars - 2 * kUnitRing,
+                      bars + C::kNumBars - kUnitRing};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -274,6 +276,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kKvComputeWarps);
     mbar_init(fin, 1);
+    unit_ring_init(ring, 1 + kKvComputeWarps);  // the MMA thread and the compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -286,7 +289,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
-  const int n_units = (*p.n_items) * p.Hkv;
+  const UnitSpace us = unit_space(p.sched, p.Hkv, kSchedKV);
+  const int n_units = us.n_units();
   const int G = p.Hq / p.Hkv;
 
   if (warp == kKvLoadWarp) {
@@ -294,8 +298,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     uint32_t t = 0;  // query tiles loaded so far
     int unit_i = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
-      const KvItem it = kv_decode(p, w);
+    for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+      int w = 0;
+      if (lane == 0) w = unit_produce(ring, p.sched.next, uk, wd);
+      w = __shfl_sync(0xFFFFFFFFu, w, 0);
+      if (w < 0 || w >= n_units) break;
+      const KvItem it = kv_decode(p, us, w);
       if (unit_i > 0 && !warp_wait(kv_empty, (unit_i - 1) & 1, wd, 21)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
@@ -378,8 +386,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         region_done();
         return true;
       };
-      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
-        const KvItem it = kv_decode(p, w);
+      for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+        const int w = unit_take(ring, uk, wd);
+        if (w < 0 || w >= n_units) break;
+        const KvItem it = kv_decode(p, us, w);
         const int R = G * (it.nq - it.v);
         if (!mbar_wait(kv_full, unit_i & 1, wd, 23)) break;
         tc_fence_after();
@@ -435,8 +445,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       warp_arrive(s_free);
       return true;
     };
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
-      const KvItem it = kv_decode(p, w);
+    for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+      const int w = unit_take_warp(ring, uk, wd);
+      if (w < 0 || w >= n_units) break;
+      const KvItem it = kv_decode(p, us, w);
       const int j = it.k0 + row;  // key index
       for (int h = it.g * G; h < (it.g + 1) * G && ok; ++h) {
         for (int m = it.v; m < it.nq; ++m, ++t) {
@@ -557,22 +569,22 @@ struct QCfg : Geo<D> {
   static constexpr uint32_t kDQ = 0, kS = 128, kDP = 256, kDS = 384;
   // bars: q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full, s_free, dp_full, dp_free,
   //       ds_ready, dq_done, acc_full, acc_free, fin
-  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 9;
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
+  // + the unit ring's full[8] and empty[8]
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 9 + 2 * kUnitRing;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
 };
 
 struct QItem {
   int s, e, m, h, g, q0;  // key tiles 0..m
 };
 
-__device__ __forceinline__ QItem q_decode(const BwdParams& p, int w) {
+__device__ __forceinline__ QItem q_decode(const BwdParams& p, const UnitSpace& us, int w) {
   QItem it;
-  const int2 pr = p.list[w / p.Hq];
-  it.h = w % p.Hq;
+  int doc;
+  unit_decode(us, w, doc, it.m, it.h);
   it.g = it.h / (p.Hq / p.Hkv);
-  it.s = p.cu[pr.x];
-  it.e = p.cu[pr.x + 1];
-  it.m = pr.y;
+  it.s = p.cu[doc];
+  it.e = p.cu[doc + 1];
   it.q0 = it.s + 128 * it.m;
   return it;
 }
@@ -605,6 +617,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
   uint64_t* acc_full = s_full + 6;
   uint64_t* acc_free = s_full + 7;
   uint64_t* fin = s_full + 8;
+  const UnitRing ring{reinterpret_cast<int*>(bars + C::kNumBars) + 4, bars + C::kNumBars - 2 * kUnitRing,
+                      bars + C::kNumBars - kUnitRing};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -629,6 +643,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kQComputeWarps);
     mbar_init(fin, 1);
+    unit_ring_init(ring, 1 + kQComputeWarps);  // the MMA thread and the compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -641,15 +656,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
-  const int n_units = (*p.n_items) * p.Hq;
+  const UnitSpace us = unit_space(p.sched, p.Hq, kSchedQ);
+  const int n_units = us.n_units();
 
   if (warp == kQLoadWarp) {
     if (lane == 0) {
       uint32_t kt = 0;  // key tiles loaded (all units)
       int unit_i = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
-        const QItem it = q_decode(p, w);
+      for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+        const int w = unit_produce(ring, p.sched.next, uk, wd);
+        if (w < 0 || w >= n_units) break;
+        const QItem it = q_decode(p, us, w);
         if (unit_i > 0 && !mbar_wait(q_empty, (unit_i - 1) & 1, wd, 31)) break;
         mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
         for (int b = 0; b < C::kNumBox; ++b) {
@@ -711,8 +729,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
         tc_commit(v_empty + vs);  // V is read only by dP
         return true;
       };
-      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
-        const QItem it = q_decode(p, w);
+      for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+        const int w = unit_take(ring, uk, wd);
+        if (w < 0 || w >= n_units) break;
+        const QItem it = q_decode(p, us, w);
         if (!mbar_wait(q_full, unit_i & 1, wd, 33)) break;
         tc_fence_after();
         if (!scores(st_it)) break;
@@ -744,8 +764,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
     uint32_t kt = 0;  // key tiles processed (all units)
     int unit_i = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
-      const QItem it = q_decode(p, w);
+    for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+      const int w = unit_take_warp(ring, uk, wd);
+      if (w < 0 || w >= n_units) break;
+      const QItem it = q_decode(p, us, w);
       const int i = it.q0 + row;
       const bool valid = i < it.e;
       // rows past the document end (the tail of the last tile) get P = 0
@@ -850,8 +872,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     BwdParams pk = p;
-    pk.list = a.sched_kv.list;
-    pk.n_items = a.sched_kv.n_items;
+    pk.sched = sched_view(a.sched_kv);
     pk.out0 = a.dk;
     pk.out1 = a.dv;
     const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
@@ -868,8 +889,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     BwdParams pq = p;
-    pq.list = a.sched_q.list;
-    pq.n_items = a.sched_q.n_items;
+    pq.sched = sched_view(a.sched_q);
     pq.out0 = a.dq;
     pq.out1 = nullptr;
     const long long max_units = (long long)a.sched_q.max_items * a.Hq;

@@ -31,6 +31,7 @@
 #include "internal.h"
 #include "mx.cuh"
 #include "ptx.cuh"
+#include "sched.cuh"
 
 namespace fapk {
 
@@ -164,8 +165,7 @@ __global__ void __launch_bounds__(256) delta_mx_kernel(const __nv_bfloat16* __re
 
 struct MxParams {
   const int32_t* cu;
-  const int2* list;
-  const int* n_items;
+  SchedView sched;
   const float* lse;
   const float* delta;
   const uint8_t *q_stb, *q_spt, *k_stb, *k_spt, *v_stb, *v_spt, *do_stb, *do_spt;
@@ -213,8 +213,9 @@ constexpr int kNumSf = 5 + 3 * kStages;
 constexpr int oBars = oSf + kNumSf * kSfBlk;
 // bars: q_full, q_empty, st_full[S], st_empty[S], s_full, s_free, dp_full, dp_free, ds_ready, dq_done,
 //       acc_full, acc_free, fin
-constexpr int kNumBars = 2 + 2 * kStages + 9;
-constexpr int kSmem = oBars + kNumBars * 8 + 16 + 1024;
+// + the unit ring's full[8] and empty[8]
+constexpr int kNumBars = 2 + 2 * kStages + 9 + 2 * kUnitRing;
+constexpr int kSmem = oBars + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
 // TMEM: S and dP regions (each read out into registers and released at
 // once), dQ, scale factors
 constexpr uint32_t tS = 0, tDP = 128, tDQ = 256;
@@ -250,6 +251,8 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   uint64_t* acc_full = s_full + 6;
   uint64_t* acc_free = s_full + 7;
   uint64_t* fin = s_full + 8;
+  const UnitRing ring{reinterpret_cast<int*>(bars + kNumBars) + 4, bars + kNumBars - 2 * kUnitRing,
+                      bars + kNumBars - kUnitRing};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto sfb = [&](int i) { return sf + i * kSfBlk; };  // 0 Q, 1 dO, 2 Kpt, 3 Vpt, 4 dS, 5+3s+{0,1,2} stage
@@ -271,6 +274,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kComputeWarps);
     mbar_init(fin, 1);
+    unit_ring_init(ring, 1 + kComputeWarps);  // the MMA thread and the compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -283,23 +287,27 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
-  const int n_units = (*p.n_items) * p.Hq;
+  const UnitSpace us = unit_space(p.sched, p.Hq, kSchedQ);
+  const int n_units = us.n_units();
   auto decode = [&](int w, int& doc, int& s, int& e, int& h, int& g, int& q0, int& n) {
-    const int2 pr = p.list[w / p.Hq];
-    h = w % p.Hq;
+    int m;
+    unit_decode(us, w, doc, m, h);
     g = h / (p.Hq / p.Hkv);
-    doc = pr.x;
     s = p.cu[doc];
     e = p.cu[doc + 1];
-    q0 = s + 128 * pr.y;
-    n = pr.y + 1;
+    q0 = s + 128 * m;
+    n = m + 1;
   };
 
   if (warp == kLoad) {
     uint32_t st_it = 0;
     int unit_i = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+    for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+      int w = 0;
+      if (lane == 0) w = unit_produce(ring, p.sched.next, uk, wd);
+      w = __shfl_sync(0xFFFFFFFFu, w, 0);
+      if (w < 0 || w >= n_units) break;
       int doc, s, e, h, g, q0, n;
       decode(w, doc, s, e, h, g, q0, n);
       if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 71)) break;
@@ -391,7 +399,9 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         ++dp_uses;
         return true;
       };
-      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+        const int w = unit_take(ring, uk, wd);
+        if (w < 0 || w >= n_units) break;
         int doc, s, e, h, g, q0, n;
         decode(w, doc, s, e, h, g, q0, n);
         if (!mbar_wait(q_full, unit_i & 1, wd, 76)) break;
@@ -467,7 +477,9 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       warp_arrive(free_bar);
       return true;
     };
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+    for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+      const int w = unit_take_warp(ring, uk, wd);
+      if (w < 0 || w >= n_units) break;
       int doc, s, e, h, g, q0, n;
       decode(w, doc, s, e, h, g, q0, n);
       const int i = q0 + row;
@@ -570,8 +582,8 @@ constexpr int oBars = oSf + kNumSf * kSfBlk;
 constexpr int kQpt = 0, kDOpt = 1, kDOtb = 2, kQtb = 3;
 constexpr int bKvFull = 0, bKvEmpty = 1, bOpFull = 2, bOpEmpty = 6, bAuxFull = 10, bAuxEmpty = 12, bSFull = 14,
               bSFree = 15, bPFull = 16, bPEmpty = 17, bDsFull = 18, bDsEmpty = 19, bAccFull = 20, bAccFree = 21,
-              bFin = 22, kNumBars = 23;
-constexpr int kSmem = oBars + kNumBars * 8 + 16 + 1024;
+              bFin = 22, bRing = 23, kNumBars = 23 + 2 * kUnitRing;
+constexpr int kSmem = oBars + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
 // TMEM: one 128-column region that holds S^T and dP^T in turn (each read out
 // into registers and released before the next), dV, dK, scale factors
 constexpr uint32_t tSD = 0, tDV = 128, tDK = 256;
@@ -606,6 +618,8 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   uint64_t* acc_full = bars + bAccFull;
   uint64_t* acc_free = bars + bAccFree;
   uint64_t* fin = bars + bFin;
+  const UnitRing ring{reinterpret_cast<int*>(bars + kNumBars) + 4, bars + kNumBars - 2 * kUnitRing,
+                      bars + kNumBars - kUnitRing};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -630,6 +644,7 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kComputeWarps);
     mbar_init(fin, 1);
+    unit_ring_init(ring, 2 + kComputeWarps);  // loader B, the MMA thread and the compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -642,15 +657,13 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
-  const int n_units = (*p.n_items) * p.Hkv;
+  const UnitSpace us = unit_space(p.sched, p.Hkv, kSchedKV);
+  const int n_units = us.n_units();
   const int G = p.Hq / p.Hkv;
   auto decode = [&](int w, int& doc, int& s, int& e, int& g, int& v, int& k0, int& nq) {
-    const int2 pr = p.list[w / p.Hkv];
-    g = w % p.Hkv;
-    doc = pr.x;
+    unit_decode(us, w, doc, v, g);
     s = p.cu[doc];
     e = p.cu[doc + 1];
-    v = pr.y;
     k0 = s + 128 * v;
     nq = (e - s + 127) / 128;
   };
@@ -675,7 +688,11 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     uint32_t t = 0;
     int unit_i = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+    for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+      int w = 0;
+      if (lane == 0) w = unit_produce(ring, p.sched.next, uk, wd);
+      w = __shfl_sync(0xFFFFFFFFu, w, 0);
+      if (w < 0 || w >= n_units) break;
       int doc, s, e, g, v, k0, nq;
       decode(w, doc, s, e, g, v, k0, nq);
       if (unit_i > 0 && !warp_wait(kv_empty, (unit_i - 1) & 1, wd, 81)) break;
@@ -729,7 +746,9 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     // ------------------------------------------------- dO^tb, Q^tb
     uint32_t t = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
+    for (uint32_t uk = 0; ok; ++uk) {
+      const int w = unit_take_warp(ring, uk, wd);
+      if (w < 0 || w >= n_units) break;
       int doc, s, e, g, v, k0, nq;
       decode(w, doc, s, e, g, v, k0, nq);
       for (int h = g * G; h < (g + 1) * G && ok; ++h) {
@@ -789,7 +808,9 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
         region_done();
         return true;
       };
-      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+      for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+        const int w = unit_take(ring, uk, wd);
+        if (w < 0 || w >= n_units) break;
         int doc, s, e, g, v, k0, nq;
         decode(w, doc, s, e, g, v, k0, nq);
         if (!mbar_wait(kv_full, unit_i & 1, wd, 89)) break;
@@ -883,7 +904,9 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
       warp_arrive(s_free);
       return true;
     };
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
+    for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+      const int w = unit_take_warp(ring, uk, wd);
+      if (w < 0 || w >= n_units) break;
       int doc, s, e, g, v, k0, nq;
       decode(w, doc, s, e, g, v, k0, nq);
       const int j = k0 + row;
@@ -1014,8 +1037,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(dkdv_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvk::kSmem);
     if (e != cudaSuccess) return e;
     MxParams pk = p;
-    pk.list = a.sched_kv.list;
-    pk.n_items = a.sched_kv.n_items;
+    pk.sched = sched_view(a.sched_kv);
     pk.out0 = a.dk;
     pk.out1 = a.dv;
     const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
@@ -1031,8 +1053,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(dq_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::kSmem);
     if (e != cudaSuccess) return e;
     MxParams pq = p;
-    pq.list = a.sched_q.list;
-    pq.n_items = a.sched_q.n_items;
+    pq.sched = sched_view(a.sched_q);
     pq.out0 = a.dq;
     pq.out1 = nullptr;
     const long long max_units = (long long)a.sched_q.max_items * a.Hq;

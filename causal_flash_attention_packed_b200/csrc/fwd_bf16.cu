@@ -30,6 +30,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "sched.cuh"
 
 namespace fapk {
 
@@ -53,14 +54,14 @@ struct Cfg {
   static constexpr uint32_t kTmemCols = 512;
   // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2],
   // o_full[2], o_free[2], final
-  static constexpr int kNumBars = 2 + 2 * kSlots + 8 + 1;
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
+  // + the unit ring's full[8] and empty[8]
+  static constexpr int kNumBars = 2 + 2 * kSlots + 8 + 1 + 2 * kUnitRing;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
 };
 
 struct Params {
   const int32_t* cu;
-  const int2* list;
-  const int* n_items;
+  SchedView sched;
   __nv_bfloat16* o;
   float* lse;
   __nv_bfloat16* o_resid;
@@ -75,14 +76,13 @@ struct Item {
   int s, e, u, h, g, q0, n0, n1, nkv;
 };
 
-__device__ __forceinline__ Item decode(const Params& p, int w) {
+__device__ __forceinline__ Item decode(const Params& p, const UnitSpace& us, int w) {
   Item it;
-  const int2 pr = p.list[w / p.Hq];
-  it.h = w % p.Hq;
+  int doc;
+  unit_decode(us, w, doc, it.u, it.h);
   it.g = it.h / (p.Hq / p.Hkv);
-  it.s = p.cu[pr.x];
-  it.e = p.cu[pr.x + 1];
-  it.u = pr.y;
+  it.s = p.cu[doc];
+  it.e = p.cu[doc + 1];
   it.q0 = it.s + 256 * it.u;
   it.n0 = 2 * it.u + 1;                               // key tiles 0..2u for query tile 0
   it.n1 = (it.q0 + 128 < it.e) ? 2 * it.u + 2 : 0;    // key tiles 0..2u+1 for query tile 1
@@ -130,6 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_full = s_full + 4;                   // [2]
   uint64_t* o_free = s_full + 6;                   // [2]
   uint64_t* fin = s_full + 8;
+  const UnitRing ring{reinterpret_cast<int*>(bars + C::kNumBars) + 4, bars + C::kNumBars - 2 * kUnitRing,
+                      bars + C::kNumBars - kUnitRing};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(o_free + i, 128);
     }
     mbar_init(fin, 1);
+    unit_ring_init(ring, 1 + 8);  // the MMA thread and the 8 softmax warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -165,7 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
-  const int n_units = (*p.n_items) * p.Hq;
+  const UnitSpace us = unit_space(p.sched, p.Hq, kSchedQ);
+  const int n_units = us.n_units();
 
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ TMA loads
@@ -173,8 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kv_it = 0;
       int unit_i = 0;
       int last_q_phase = -1;
-      for (int w = blockIdx.x; w < n_units; w += gridDim.x, ++unit_i) {
-        const Item it = decode(p, w);
+      for (uint32_t uk = 0;; ++uk, ++unit_i) {
+        const int w = unit_produce(ring, p.sched.next, uk, wd);
+        if (w < 0 || w >= n_units) break;
+        const Item it = decode(p, us, w);
         if (unit_i > 0 && !mbar_wait(q_empty, (unit_i - 1) & 1, wd, 1)) break;
         mbar_arrive_expect_tx(q_full, (it.n1 ? 2 : 1) * C::kTileBytes);
         last_q_phase = unit_i & 1;
@@ -189,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t use = kv_it / C::kSlots;
             if (use > 0 && !mbar_wait(kv_empty + slot, (use - 1) & 1, wd, 2)) { ok = false; break; }
             mbar_arrive_expect_tx(kv_full + slot, C::kTileBytes);
-            const bool drop = (p.flags & FAPK_FLAG_INJECT_DROP_LOAD) && blockIdx.x == 0 && kv_it == 3;
+            // injected fault: the CTA that takes the first (longest) unit drops its fourth copy
+            const bool drop = (p.flags & FAPK_FLAG_INJECT_DROP_LOAD) && w == 0 && kv_it == 3;
             if (!drop) {
               const CUtensorMap* tm = kv ? &tm_v : &tm_k;
               for (int b = 0; b < C::kNumBox; ++b)
@@ -236,8 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_f16_ts(tmem + (i ? C::kOCol1 : C::kOCol0), pcol + kk * 8,
                      sdesc_sw128(va + kk * 2048, C::kBoxBytes, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
       };
-      for (int w = blockIdx.x; w < n_units; w += gridDim.x, ++unit_i) {
-        const Item it = decode(p, w);
+      for (uint32_t uk = 0;; ++uk, ++unit_i) {
+        const int w = unit_take(ring, uk, wd);
+        if (w < 0 || w >= n_units) break;
+        const Item it = decode(p, us, w);
         if (!mbar_wait(q_full, unit_i & 1, wd, 3)) break;
         int kslot = kv_it % C::kSlots;
         if (!mbar_wait(kv_full + kslot, (kv_it / C::kSlots) & 1, wd, 4)) break;
@@ -300,8 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_addr = lane_base + (wg ? C::kSCol1 : C::kSCol0);
     const uint32_t o_addr = lane_base + (wg ? C::kOCol1 : C::kOCol0);
     uint32_t s_cnt = 0, o_cnt = 0;
-    for (int w = blockIdx.x; w < n_units; w += gridDim.x) {
-      const Item it = decode(p, w);
+    for (uint32_t uk = 0;; ++uk) {
+      const int w = unit_take_warp(ring, uk, wd);
+      if (w < 0 || w >= n_units) break;
+      const Item it = decode(p, us, w);
       const int n = wg ? it.n1 : it.n0;
       if (n == 0) continue;
       const int q_idx = it.q0 + 128 * wg + row;
@@ -419,8 +430,7 @@ cudaError_t launch_d(const FwdArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   Params p;
   p.cu = a.cu;
-  p.list = a.sched.list;
-  p.n_items = a.sched.n_items;
+  p.sched = sched_view(a.sched);
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.lse = a.lse;
   p.o_resid = static_cast<__nv_bfloat16*>(a.o_resid);

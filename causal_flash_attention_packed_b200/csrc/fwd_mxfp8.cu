@@ -38,6 +38,7 @@
 #include "internal.h"
 #include "mx.cuh"
 #include "ptx.cuh"
+#include "sched.cuh"
 
 namespace fapk {
 
@@ -66,8 +67,9 @@ constexpr int kSfBlk = 512;
 constexpr int oXmax = oSf + (3 + kSlots) * kSfBlk;  // block maxima [2][4][128] (by tile parity)
 constexpr int oLsum = oXmax + 2 * 4 * 128 * 4;       // partial row sums [4][128]
 constexpr int oBars = oLsum + 4 * 128 * 4;
-constexpr int kNumBars = 2 + 2 * kSlots + 8 + 4;  // + one row-exchange barrier per row quarter
-constexpr int kSmemBytes = oBars + kNumBars * 8 + 16 + 1024;
+// + one row-exchange barrier per row quarter, the unit ring's full[8] and empty[8]
+constexpr int kNumBars = 2 + 2 * kSlots + 8 + 4 + 2 * kUnitRing;
+constexpr int kSmemBytes = oBars + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
 
 // TMEM columns
 constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256;
@@ -75,8 +77,7 @@ constexpr uint32_t kSfQ = 384, kSfK = 388, kSfKpt = 392, kSfP = 396, kSfV = 400;
 
 struct Params {
   const int32_t* cu;
-  const int2* list;
-  const int* n_items;
+  SchedView sched;
   const uint8_t* q_spt;   // Q per-token scales [T][Hq][4]
   const uint8_t* k_stb;   // K token-block scales [slots][Hkv][4]
   const uint8_t* k_spt;   // K per-token scales [T][Hkv][4]
@@ -95,16 +96,15 @@ struct Item {
   int doc, s, e, h, g, q0, n;  // n key tiles 0..n-1, tile n-1 is the diagonal
 };
 
-__device__ __forceinline__ Item decode(const Params& p, int w) {
+__device__ __forceinline__ Item decode(const Params& p, const UnitSpace& us, int w) {
   Item it;
-  const int2 pr = p.list[w / p.Hq];
-  it.h = w % p.Hq;
+  int m;
+  unit_decode(us, w, it.doc, m, it.h);
   it.g = it.h / (p.Hq / p.Hkv);
-  it.doc = pr.x;
-  it.s = p.cu[pr.x];
-  it.e = p.cu[pr.x + 1];
-  it.q0 = it.s + 128 * pr.y;
-  it.n = pr.y + 1;
+  it.s = p.cu[it.doc];
+  it.e = p.cu[it.doc + 1];
+  it.q0 = it.s + 128 * m;
+  it.n = m + 1;
   return it;
 }
 
@@ -169,6 +169,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_free = s_full + 5;
   uint64_t* fin = s_full + 6;
   uint64_t* xbar = s_full + 7;  // [4]
+  const UnitRing ring{reinterpret_cast<int*>(bars + kNumBars) + 4, bars + kNumBars - 2 * kUnitRing,
+                      bars + kNumBars - kUnitRing};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -187,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(o_full, 1);
     mbar_init(o_free, kComputeWarps);
     mbar_init(fin, 1);
+    unit_ring_init(ring, 1 + kComputeWarps);  // the MMA thread and the softmax warps
     for (int i = 0; i < 4; ++i) mbar_init(xbar + i, 4);
     *abort_flag = 0;
     fence_mbar_init();
@@ -200,15 +203,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
-  const int n_units = (*p.n_items) * p.Hq;
+  const UnitSpace us = unit_space(p.sched, p.Hq, kSchedQ);
+  const int n_units = us.n_units();
 
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ loads
     uint32_t kv_it = 0;
     int unit_i = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
-      const Item it = decode(p, w);
+    for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+      int w = 0;
+      if (lane == 0) w = unit_produce(ring, p.sched.next, uk, wd);
+      w = __shfl_sync(0xFFFFFFFFu, w, 0);
+      if (w < 0 || w >= n_units) break;
+      const Item it = decode(p, us, w);
       if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 51)) break;
       {
         // scale blocks: row r = lane + 32 r1 -> bytes 16 lane + 4 r1 .. +3
@@ -302,8 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_cp_sf(tmem + kSfK, asf + (3 + ks) * kSfBlk);
         issue_s(col, aring + ks * kCodeTile, kSfK);
       };
-      for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x, ++unit_i) {
-        const Item it = decode(p, w);
+      for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+        const int w = unit_take(ring, uk, wd);
+        if (w < 0 || w >= n_units) break;
+        const Item it = decode(p, us, w);
         const int n = it.n;
         if (!mbar_wait(q_full, unit_i & 1, wd, 54)) break;
         tc_fence_after();
@@ -389,8 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     uint32_t s_cnt[2] = {0, 0}, pv_cnt = 0, o_cnt = 0, tiles = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
-      const Item it = decode(p, w);
+    for (uint32_t uk = 0; ok; ++uk) {
+      const int w = unit_take_warp(ring, uk, wd);
+      if (w < 0 || w >= n_units) break;
+      const Item it = decode(p, us, w);
       const int n = it.n;
       const int q_idx = it.q0 + row;
       float M = -INFINITY, l = 0.f;  // l: this thread's share of the row sum
@@ -552,8 +564,7 @@ cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   Params p;
   p.cu = a.cu;
-  p.list = a.sched.list;
-  p.n_items = a.sched.n_items;
+  p.sched = sched_view(a.sched);
   p.q_spt = a.q_spt;
   p.k_stb = a.k_stb;
   p.k_spt = a.k_spt;

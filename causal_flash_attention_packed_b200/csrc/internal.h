@@ -21,25 +21,39 @@ struct Marks {
   }
 };
 
-// Work-list modes of the scheduler (schedule.cu).  An item is (doc, tile)
-// with tile in [0, ceil(L / rows)); items are ordered by a cost level,
-// highest first, so that persistent CTAs take the longest work first (LPT).
-//  kSchedQ:  level = tile               (a later query tile sees more keys)
-//  kSchedKV: level = ntiles - 1 - tile  (an earlier key tile is seen by more
-//                                        queries)
+// Work order of the persistent kernels (schedule.cu).  Each document of
+// length L has ceil(L / rows) tiles; a work unit is (document, head, tile).
+// Units are numbered document by document (longest documents first), and
+// within a document head by head, each head's tiles longest work first:
+//  kSchedQ:  query tiles, last tile first (a later query tile sees more keys)
+//  kSchedKV: key tiles, first tile first  (an earlier key tile is seen by
+//                                          more queries)
+// so the units that run side by side share their streamed K/V (or Q/dO)
+// tiles through L2.  The CTAs take units in this order from an atomic
+// counter, so the short units of the smallest documents come last.
 enum SchedMode : int { kSchedQ = 0, kSchedKV = 1 };
 
-// Scratch of one work list inside the workspace.
+// Scratch of one work order inside the workspace.
 struct SchedBuf {
-  int* level_off;  // [max_levels + 2]
-  int2* list;      // [max_items]
-  int* n_items;    // 1 int
+  int* scratch;   // [3 * (max_levels + 2)]: tile-count histogram and offsets
+  int2* docs;     // [n_docs]: {document, index of its first tile}, longest first
+  int* counts;    // [0] documents with at least one tile, [1] tiles in all
+  int* next;      // the units handed out so far (reset by the scheduler)
   int max_levels;
-  int max_items;
+  int max_items;  // upper bound of the tile count (grid sizing)
 };
 
-cudaError_t launch_schedule(const int32_t* cu, int n_docs, int rows, int mode, const SchedBuf& sb,
-                            DeviceStatus* status, bool clear_status, cudaStream_t stream);
+// What the kernels read of a work order.
+struct SchedView {
+  const int2* docs;
+  const int* counts;
+  int* next;
+};
+
+inline SchedView sched_view(const SchedBuf& b) { return SchedView{b.docs, b.counts, b.next}; }
+
+cudaError_t launch_schedule(const int32_t* cu, int n_docs, int rows, const SchedBuf& sb, DeviceStatus* status,
+                            bool clear_status, cudaStream_t stream);
 
 // deq_pt_bf16 (optional): also write the per-token form dequantised to bf16.
 cudaError_t launch_quantize_mxfp8(const void* x, int T, int H, int d, const int32_t* cu, int n_docs,
@@ -123,10 +137,6 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream);
 // Tensor map of E4M3 codes [T][H][128] as (128, H, T), box 128 x 1 x 128,
 // 128-byte swizzle (api.cu).
 bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H);
-// Tensor map of `n` contiguous fp32 values viewed as one dimension (the
-// per-head rows of a [H][T] tensor back to back): boxes of `box` values, no
-// swizzle.  A load starts at a multiple of 4 values (16 bytes).
-bool make_tmap_flat_f32(CUtensorMap* map, const float* base, long long n, int box);
 
 // Backward, bf16 operands (bwd_bf16.cu).
 struct BwdArgs {
@@ -164,8 +174,8 @@ cudaError_t launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream);
 // (d, H, T) view with a box of 64 channels x 1 head x 128 tokens and 128-byte
 // swizzle (api.cu).
 // Tensor map of a [T][H][d] 16-bit tensor: boxes of 64 channels x 1 head x
-// `box_rows` tokens, 128-byte swizzle.
-bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16 = false, int box_rows = 128);
+// 128 tokens, 128-byte swizzle.
+bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool f16 = false);
 
 // bf16 -> fp16 copy of n elements (n a multiple of 8); magnitudes >= 65504
 // record kStatusRange (convert.cu).

@@ -101,20 +101,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), CTA-local destinations, no multicast.
-// The innermost coordinate of every 3-D load here is a channel offset that is
-// a multiple of 64 elements (128 bytes); 1-D fp32 loads start at a multiple
-// of 4 values.  Both meet the 16-byte rule.
+// The innermost coordinate of every load here is a channel offset that is a
+// multiple of 64 elements (128 bytes), so it always meets the 16-byte rule.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-__device__ __forceinline__ void tma_load_1d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0) {
-  asm volatile(
-      "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0)
-      : "memory");
 }
 
 // Asynchronous 4-byte copy global -> shared; `bytes` = 0 writes a zero
@@ -244,20 +235,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
-// 32 lanes x 16 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : FAPK_R8(0), FAPK_R8(8)
-      : "r"(taddr)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" : FAPK_U8(0), FAPK_U8(8) : : "memory");
-}
-
 // Completes every outstanding tcgen05.ld of the thread; the register operands
 // tie the loaded values to this point so no use is scheduled above it.
 __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
@@ -283,12 +260,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
       FAPK_W8(0), FAPK_W8(8)
       : "memory");
-}
-
-// 32 lanes x 8 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), FAPK_W8(0)
-               : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_st() {

@@ -1,32 +1,36 @@
-// Workload-aware scheduling of packed documents (FLAMIA page, sec. "FLAMIA
+// Workload-aware work order for packed documents (FLAMIA page, sec. "FLAMIA
 // Mimarisi ve Temel Tasarim Ilkeleri": documents are processed in their packed
 // layout without repacking, and the schedule is workload-aware).
 //
-// Each document of length L contributes ceil(L / rows) tiles.  The work of a
-// tile under the causal mask grows with its query index (or, for key tiles,
-// with the number of later query tiles), so tiles are bucketed by a cost level
-// and emitted highest level first: persistent CTAs that take items in list
-// order get the longest work first (longest-processing-time-first balancing).
-// Within one level the order is whatever the atomics give; every item's
-// computation is independent of which CTA runs it, so results are unaffected.
+// Documents are counting-sorted by their tile count, longest first; the
+// sorted table records each document and the index of its first tile (a
+// document's tiles follow those of all longer documents).  The kernels number
+// their work units over this table (see unit_decode in sched.cuh) and take
+// them from an atomic counter, which this kernel resets.  Documents of equal
+// length land in whatever order the atomics give; every unit's computation is
+// independent of which CTA runs it and when, so results are unaffected.
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace fapk {
 
-__global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restrict__ cu, int n_docs,
-                                                        int rows, int mode, SchedBuf sb,
-                                                        DeviceStatus* status, int clear_status) {
+__global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restrict__ cu, int n_docs, int rows,
+                                                        SchedBuf sb, DeviceStatus* status, int clear_status) {
   const int tid = threadIdx.x;
-  int* off = sb.level_off;  // histogram, then running level offsets
-  if (tid == 0 && clear_status) {
-    status->code = 0;
-    status->where = 0;
-    status->block = 0;
+  const int L1 = sb.max_levels + 2;
+  int* hist = sb.scratch;           // documents per tile count, then running positions
+  int* doc_off = sb.scratch + L1;   // first sorted position of each tile count
+  int* tile_off = sb.scratch + 2 * L1;  // first tile index of each tile count
+  if (tid == 0) {
+    if (clear_status) {
+      status->code = 0;
+      status->where = 0;
+      status->block = 0;
+    }
+    *sb.next = 0;
   }
-  for (int i = tid; i < sb.max_levels + 2; i += blockDim.x) off[i] = 0;
+  for (int i = tid; i < L1; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  // histogram of tiles per document: off[nt] += 1
   for (int k = tid; k < n_docs; k += blockDim.x) {
     const int L = cu[k + 1] - cu[k];
     const int nt = (L + rows - 1) / rows;
@@ -34,40 +38,36 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restric
       record_error(status, kStatusBadSeqlens, 1);
       continue;
     }
-    if (nt > 0) atomicAdd(&off[nt], 1);
+    if (nt > 0) atomicAdd(&hist[nt], 1);
   }
   __syncthreads();
   if (tid == 0) {
-    // count[l] = number of documents with more than l tiles = sum_{n > l} hist[n];
-    // levels are emitted highest first: offset[l] = sum_{l' > l} count[l'].
-    int suffix = 0;  // running count[l]
-    int total = 0;   // items of levels above l
+    // longest documents first: offsets of each tile count, counted from the top
+    int docs = 0, tiles = 0;
     for (int l = sb.max_levels; l >= 1; --l) {
-      suffix += off[l];  // documents with exactly l tiles join count[l - 1]
-      const int c = suffix;
-      off[l] = total;    // reuse slot l as the offset of level l - 1
-      total += c;
+      const int c = hist[l];
+      doc_off[l] = docs;
+      tile_off[l] = tiles;
+      hist[l] = docs;
+      docs += c;
+      tiles += c * l;
     }
-    off[0] = 0;
-    *sb.n_items = total;
+    sb.counts[0] = docs;
+    sb.counts[1] = tiles;
   }
   __syncthreads();
-  // place: level lvl's offset sits in off[lvl + 1]
   for (int k = tid; k < n_docs; k += blockDim.x) {
     const int L = cu[k + 1] - cu[k];
     const int nt = (L + rows - 1) / rows;
     if (L <= 0 || nt > sb.max_levels) continue;
-    for (int t = 0; t < nt; ++t) {
-      const int lvl = (mode == kSchedQ) ? t : (nt - 1 - t);
-      const int pos = atomicAdd(&off[lvl + 1], 1);
-      if (pos < sb.max_items) sb.list[pos] = make_int2(k, t);
-    }
+    const int pos = atomicAdd(&hist[nt], 1);
+    sb.docs[pos] = make_int2(k, tile_off[nt] + (pos - doc_off[nt]) * nt);
   }
 }
 
-cudaError_t launch_schedule(const int32_t* cu, int n_docs, int rows, int mode, const SchedBuf& sb,
-                            DeviceStatus* status, bool clear_status, cudaStream_t stream) {
-  schedule_kernel<<<1, 1024, 0, stream>>>(cu, n_docs, rows, mode, sb, status, clear_status ? 1 : 0);
+cudaError_t launch_schedule(const int32_t* cu, int n_docs, int rows, const SchedBuf& sb, DeviceStatus* status,
+                            bool clear_status, cudaStream_t stream) {
+  schedule_kernel<<<1, 1024, 0, stream>>>(cu, n_docs, rows, sb, status, clear_status ? 1 : 0);
   note_launches(1);
   return cudaGetLastError();
 }
