@@ -199,6 +199,14 @@ KERNELS = {
 # pair and query head, in units of d: forward S and PV = 4; dK/dV kernel S,
 # dP, dV, dK = 8; dQ kernel S, dP, dQ = 6
 KERNEL_FLOPS = {"fwd_kernel": 4.0, "dkdv_kernel": 8.0, "dq_kernel": 6.0}
+# DRAM bytes (read + written) of one launch of each attention kernel on the
+# 32K workload (config 4), from dram__bytes_read.sum + dram__bytes_write.sum
+# of an ncu capture of the kernels as they stand; None where not measured.
+# These must be taken again whenever a kernel changes.
+MEASURED_TRAFFIC = {
+    4: {"bf16": {"fwd_kernel": 1.336e9, "dkdv_kernel": 2.134e9, "dq_kernel": 1.607e9},
+        "mxfp8": {"fwd_kernel": 1.335e9, "dkdv_kernel": 2.157e9, "dq_kernel": 1.630e9}},
+}
 
 
 class Path:
@@ -260,7 +268,7 @@ class Path:
         return total_ms / steps, kern_ms, launches
 
 
-def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks):
+def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, config=None):
     flops = w.flops()
     value = flops * world / (ms_per_step * 1e-3) / 1e12
     pairs = w.pairs()
@@ -278,8 +286,10 @@ def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks):
         # peak times the nominal FP8/bf16 ratio of 2
         peak, peak_src, dense = 2.0 * peaks["bf16_tflops_sustained"], \
             f"2 x {peaks['source']} bf16 sustained (MEASURED_PEAKS.json), nominal FP8/bf16 ratio", DENSE_FP8_TFLOPS
+    traffic = MEASURED_TRAFFIC.get(config, {}).get(prec, {}).get(dom)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": dom, "peak_source": peak_src,
+                "frac": achieved / peak, "traffic": traffic, "traffic_unit": "bytes per launch",
+                "kernel": dom, "peak_source": peak_src,
                 "kernels_ms": kern_ms,
                 "kernels_tflops": {n: KERNEL_FLOPS[n] * w.d * w.Hq * pairs / (kern_ms[n] * 1e-3) / 1e12
                                    for n in KERNEL_FLOPS},
@@ -343,7 +353,7 @@ def main():
     results = {}
     for p in paths:
         ms, kern_ms, launches = runners[p].timed(args.steps, args.warmup, world)
-        results[p] = path_report(w, p, ms, kern_ms, launches, world, peaks)
+        results[p] = path_report(w, p, ms, kern_ms, launches, world, peaks, config=args.config)
     clk = clocks.stop() if clocks else None
     st_ok = all(r.status_ok() for r in runners.values())
 
