@@ -238,6 +238,29 @@ class Path:
         f.attn_bwd(Pb, self.qd, self.kd, self.vd, self.o, self.lse, self.dod, ctx=self.ctx, dq=self.dq,
                    dk=self.dk, dv=self.dv, ws=self.ws_b, stream=self.stream)
 
+    def balance(self, num_sms):
+        """One untimed fwd + bwd with per-CTA time records: mean / max of the
+        CTAs' busy times (start of the earliest CTA to each CTA's end), per
+        persistent kernel, next to the same ratio of causal tile work when the
+        units are handed out in order to the SM that frees up first."""
+        f = self.fapk
+        P = f.make_problem(self.seq, self.w.Hq, self.w.Hkv, self.w.d, self.w.scale,
+                           prec=f.MXFP8 if self.prec == "mxfp8" else f.BF16, flags=f.FLAG_CTA_TIMES)
+        f.attn_fwd(P, self.qd, self.kd, self.vd, o=self.o, lse=self.lse, ctx=self.ctx, ws=self.ws_f,
+                   stream=self.stream)
+        fwd = f.cta_times(P, f.FWD, 0, self.ws_f, self.stream)
+        f.attn_bwd(P, self.qd, self.kd, self.vd, self.o, self.lse, self.dod, ctx=self.ctx, dq=self.dq,
+                   dk=self.dk, dv=self.dv, ws=self.ws_b, stream=self.stream)
+        kv = f.cta_times(P, f.BWD, 0, self.ws_b, self.stream)
+        qk = f.cta_times(P, f.BWD, 1, self.ws_b, self.stream)
+        ana = analytic_balance(self.w, self.prec, num_sms)
+        out = {}
+        for name, t in (("fwd_kernel", fwd), ("dkdv_kernel", kv), ("dq_kernel", qk)):
+            busy = (t[:, 1] - t[:, 0].min()).astype(np.float64)
+            out[name] = {"measured": float(busy.mean() / busy.max()), "analytic": ana[name], "ctas": int(len(t)),
+                         "max_ms": float(busy.max() / 1e6)}
+        return out
+
     def status_ok(self):
         return self.fapk.status(self.ws_f) == 0 and self.fapk.status(self.ws_b) == 0
 
@@ -266,6 +289,51 @@ class Path:
         kern_ms = {n: max_over_ranks(statistics.mean(row[i] for row in per), world, self.dev)
                    for i, n in enumerate(names)}
         return total_ms / steps, kern_ms, launches
+
+
+def analytic_balance(w, prec, num_sms):
+    """Mean / max per-SM causal tile work (128 x 128 tile pairs) of each
+    persistent kernel when its units, in the scheduler's order (documents by
+    tile count, longest first; head by head; each head's tiles longest work
+    first), go one by one to the SM that frees up first."""
+    import heapq
+    lengths = np.diff(w.cu.astype(np.int64))
+    G = w.Hq // w.Hkv
+
+    def units(rows, H, work_of):
+        nts = [int((L + rows - 1) // rows) for L in lengths]
+        order = sorted([k for k in range(len(lengths)) if nts[k] > 0], key=lambda k: -nts[k])
+        for k in order:
+            for _ in range(H):
+                for r in range(nts[k]):
+                    yield work_of(k, nts[k], r)
+
+    def fwd_pair(k, nt, r):  # 256-row unit: query tiles 2u (and 2u + 1 if present)
+        u = nt - 1 - r
+        n0 = 2 * u + 1
+        n1 = 2 * u + 2 if 256 * u + 128 < lengths[k] else 0
+        return n0 + n1
+
+    def ratio(gen):
+        heap = [(0.0, i) for i in range(num_sms)]
+        loads = [0.0] * num_sms
+        n = 0
+        for work in gen:
+            t, i = heapq.heappop(heap)
+            loads[i] += work
+            heapq.heappush(heap, (t + work, i))
+            n += 1
+        used = loads[: min(n, num_sms)]
+        return float(np.mean(used) / max(used)) if used and max(used) > 0 else 1.0
+
+    if prec == "mxfp8":
+        fwd = ratio(units(128, w.Hq, lambda k, nt, r: nt - r))
+    else:
+        fwd = ratio(units(256, w.Hq, fwd_pair))
+    nq = lambda k: (lengths[k] + 127) // 128
+    return {"fwd_kernel": fwd,
+            "dkdv_kernel": ratio(units(128, w.Hkv, lambda k, nt, r: G * (nt - r))),
+            "dq_kernel": ratio(units(128, w.Hq, lambda k, nt, r: nt - r))}
 
 
 def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, config=None):
@@ -356,6 +424,9 @@ def main():
         results[p] = path_report(w, p, ms, kern_ms, launches, world, peaks, config=args.config)
     clk = clocks.stop() if clocks else None
     st_ok = all(r.status_ok() for r in runners.values())
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    balance = {p: runners[p].balance(num_sms) for p in paths}
+    st_ok = st_ok and all(r.status_ok() for r in runners.values())
 
     # end to end through the C ABI with host buffers (pinned), copies included
     e2e = None
@@ -405,6 +476,7 @@ def main():
         "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
         "clocks": clk, "status_ok": st_ok,
+        "scheduler_balance": balance,
     }
     for p in paths[1:]:
         line[p] = results[p]

@@ -127,13 +127,14 @@ constexpr int kFwdRowsMx = 128;  // query rows per MXFP8 forward work item (one 
 
 struct FwdLayout {
   SchedLayout sched;
-  size_t total;
+  size_t cta_times, total;
 };
 FwdLayout fwd_layout(const fapk_problem_t* P) {
   FwdLayout L;
   L.sched = sched_layout(kAlign, P->T, P->n_docs, P->max_seqlen,
                          P->prec == FAPK_MXFP8 ? kFwdRowsMx : kFwdRows);
-  L.total = L.sched.end;
+  L.cta_times = align_up(L.sched.end);
+  L.total = align_up(L.cta_times + sizeof(unsigned long long) * kCtaTimesWords);
   return L;
 }
 
@@ -142,7 +143,7 @@ FwdLayout fwd_layout(const fapk_problem_t* P) {
 //  MXFP8 path, instead of the fp16 copies: the quantiser's forms of dO.
 struct BwdLayout {
   SchedLayout kv, q;
-  size_t delta, q16, k16, do16, nl2, total;
+  size_t delta, q16, k16, do16, nl2, cta_times, total;
   size_t do_vtb, do_stb, do_vpt, do_spt;
 };
 BwdLayout bwd_layout(const fapk_problem_t* P) {
@@ -159,14 +160,16 @@ BwdLayout bwd_layout(const fapk_problem_t* P) {
     L.do_stb = align_up(L.do_vtb + nq);
     L.do_vpt = align_up(L.do_stb + slots * P->Hq * (P->d / 32));
     L.do_spt = align_up(L.do_vpt + nq);
-    L.total = align_up(L.do_spt + (size_t)P->T * P->Hq * (P->d / 32));
+    L.cta_times = align_up(L.do_spt + (size_t)P->T * P->Hq * (P->d / 32));
+    L.total = align_up(L.cta_times + 2 * sizeof(unsigned long long) * kCtaTimesWords);
     return L;
   }
   L.q16 = after_delta;
   L.k16 = align_up(L.q16 + 2 * nq);
   L.do16 = align_up(L.k16 + 2 * nk);
   L.nl2 = align_up(L.do16 + 2 * nq);
-  L.total = align_up(L.nl2 + sizeof(float) * (size_t)P->Hq * (size_t)P->T);
+  L.cta_times = align_up(L.nl2 + sizeof(float) * (size_t)P->Hq * (size_t)P->T);
+  L.total = align_up(L.cta_times + 2 * sizeof(unsigned long long) * kCtaTimesWords);
   return L;
 }
 
@@ -297,6 +300,8 @@ int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void*
   a.scale = P->scale;
   a.rule = P->scale_rule;
   a.status = status;
+  if (P->flags & FAPK_FLAG_CTA_TIMES)
+    a.cta_times[0] = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + L.cta_times);
   a.timeout_ns = timeout_ns_of(P);
   a.num_sms = sms;
   mk.at(2, st);
@@ -347,6 +352,11 @@ int bwd_mxfp8(const fapk_problem_t* P, const void* o, const float* lse, const vo
   a.grad_bf16 = P->grad_dtype == FAPK_GRAD_BF16;
   a.rule = P->scale_rule;
   a.status = status;
+  if (P->flags & FAPK_FLAG_CTA_TIMES) {
+    auto* ct = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + L.cta_times);
+    a.cta_times[0] = ct;
+    a.cta_times[1] = ct + kCtaTimesWords;
+  }
   a.timeout_ns = timeout_ns_of(P);
   a.num_sms = sms;
   return cuda_status(launch_bwd_mxfp8(a, st));
@@ -399,6 +409,8 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
   a.scale = P->scale;
   a.sched = sched_buf(ws, L.sched);
   a.status = status;
+  if (P->flags & FAPK_FLAG_CTA_TIMES)
+    a.cta_times[0] = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + L.cta_times);
   a.timeout_ns = timeout_ns_of(P);
   a.flags = P->flags;
   a.num_sms = sms;
@@ -452,6 +464,11 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   a.sched_kv = sched_buf(ws, L.kv);
   a.sched_q = sched_buf(ws, L.q);
   a.status = status;
+  if (P->flags & FAPK_FLAG_CTA_TIMES) {
+    auto* ct = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + L.cta_times);
+    a.cta_times[0] = ct;
+    a.cta_times[1] = ct + kCtaTimesWords;
+  }
   a.timeout_ns = timeout_ns_of(P);
   a.flags = P->flags;
   a.num_sms = sms;
@@ -489,6 +506,26 @@ int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const int32_t* 
   }
   return cuda_status(launch_quantize_mxfp8(x_bf16, T, H, d, cu_seqlens_dev, n_docs, forms, scale_rule, val_tb,
                                            scale_tb, val_pt, scale_pt, static_cast<cudaStream_t>(stream)));
+}
+
+int fapk_cta_times(const fapk_problem_t* P, int which, int kernel, const void* ws, void* stream,
+                   unsigned long long* out_pairs, int max_ctas, int* n_ctas) {
+  if (!P || !ws || !n_ctas || (max_ctas > 0 && !out_pairs) || max_ctas < 0) return FAPK_ERR_INVALID_ARG;
+  if (which != FAPK_FWD && which != FAPK_BWD) return FAPK_ERR_INVALID_ARG;
+  if (kernel < 0 || kernel > (which == FAPK_FWD ? 0 : 1)) return FAPK_ERR_INVALID_ARG;
+  const size_t off = (which == FAPK_FWD ? fwd_layout(P).cta_times : bwd_layout(P).cta_times) +
+                     sizeof(unsigned long long) * kCtaTimesWords * (size_t)kernel;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FAPK_ERR_CUDA;
+  const char* base = static_cast<const char*>(ws) + off;
+  unsigned long long count = 0;
+  if (cudaMemcpy(&count, base, sizeof(count), cudaMemcpyDeviceToHost) != cudaSuccess) return FAPK_ERR_CUDA;
+  if (count > (unsigned long long)kMaxCtaTimes) count = kMaxCtaTimes;
+  *n_ctas = (int)count;
+  const int n = (int)count < max_ctas ? (int)count : max_ctas;
+  if (n > 0 && cudaMemcpy(out_pairs, base + sizeof(unsigned long long), 2 * sizeof(unsigned long long) * (size_t)n,
+                          cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FAPK_ERR_CUDA;
+  return FAPK_OK;
 }
 
 int fapk_status(const void* ws, void* stream) {

@@ -137,6 +137,7 @@ struct BwdParams {
   float scale;       // softmax scale (dK, dQ factor)
   float scale_log2;  // scale * log2(e)
   int grad_bf16;
+  unsigned long long* cta_times;  // per-CTA (start, end) records, or null
 };
 
 // Store 32 fp32 values (times `mul`) of one row as fp32 or bf16.
@@ -288,6 +289,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) {  // scheduler balance record
+    if (blockIdx.x == 0) p.cta_times[0] = gridDim.x;
+    p.cta_times[1 + 2 * blockIdx.x] = globaltimer_ns();
+  }
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
   const UnitSpace us = unit_space(p.sched, p.Hkv, kSchedKV);
   const int n_units = us.n_units();
@@ -543,6 +548,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) p.cta_times[2 + 2 * blockIdx.x] = globaltimer_ns();
   if (warp == kKvMmaWarp) tmem_dealloc(tmem, 512);
 }
 
@@ -655,6 +661,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) {  // scheduler balance record
+    if (blockIdx.x == 0) p.cta_times[0] = gridDim.x;
+    p.cta_times[1 + 2 * blockIdx.x] = globaltimer_ns();
+  }
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
   const UnitSpace us = unit_space(p.sched, p.Hq, kSchedQ);
   const int n_units = us.n_units();
@@ -829,6 +839,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) p.cta_times[2 + 2 * blockIdx.x] = globaltimer_ns();
   if (warp == kQMmaWarp) tmem_dealloc(tmem, 512);
 }
 
@@ -873,6 +884,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     BwdParams pk = p;
     pk.sched = sched_view(a.sched_kv);
+    pk.cta_times = a.cta_times[0];
     pk.out0 = a.dk;
     pk.out1 = a.dv;
     const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
@@ -890,6 +902,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     BwdParams pq = p;
     pq.sched = sched_view(a.sched_q);
+    pq.cta_times = a.cta_times[1];
     pq.out0 = a.dq;
     pq.out1 = nullptr;
     const long long max_units = (long long)a.sched_q.max_items * a.Hq;

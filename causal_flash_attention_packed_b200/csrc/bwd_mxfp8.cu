@@ -177,6 +177,7 @@ struct MxParams {
   float scale, scale_log2;
   int grad_bf16;
   int rule;
+  unsigned long long* cta_times;  // per-CTA (start, end) records, or null
 };
 
 __device__ __forceinline__ void store_row32(void* base, size_t elem_off, const uint32_t (&t)[32], float mul,
@@ -286,6 +287,10 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) {  // scheduler balance record
+    if (blockIdx.x == 0) p.cta_times[0] = gridDim.x;
+    p.cta_times[1 + 2 * blockIdx.x] = globaltimer_ns();
+  }
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
   const UnitSpace us = unit_space(p.sched, p.Hq, kSchedQ);
   const int n_units = us.n_units();
@@ -555,6 +560,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) p.cta_times[2 + 2 * blockIdx.x] = globaltimer_ns();
   if (warp == kMma) tmem_dealloc(tmem, 512);
 }
 
@@ -656,6 +662,10 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) {  // scheduler balance record
+    if (blockIdx.x == 0) p.cta_times[0] = gridDim.x;
+    p.cta_times[1 + 2 * blockIdx.x] = globaltimer_ns();
+  }
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
   const UnitSpace us = unit_space(p.sched, p.Hkv, kSchedKV);
   const int n_units = us.n_units();
@@ -990,6 +1000,7 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) p.cta_times[2 + 2 * blockIdx.x] = globaltimer_ns();
   if (warp == kMma) tmem_dealloc(tmem, 512);
 }
 
@@ -1038,6 +1049,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     MxParams pk = p;
     pk.sched = sched_view(a.sched_kv);
+    pk.cta_times = a.cta_times[0];
     pk.out0 = a.dk;
     pk.out1 = a.dv;
     const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
@@ -1054,6 +1066,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     MxParams pq = p;
     pq.sched = sched_view(a.sched_q);
+    pq.cta_times = a.cta_times[1];
     pq.out0 = a.dq;
     pq.out1 = nullptr;
     const long long max_units = (long long)a.sched_q.max_items * a.Hq;

@@ -70,6 +70,7 @@ struct Params {
   int T, Hq, Hkv;
   float scale_log2;
   int flags;
+  unsigned long long* cta_times;  // per-CTA (start, end) records, or null
 };
 
 struct Item {
@@ -167,6 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) {  // scheduler balance record
+    if (blockIdx.x == 0) p.cta_times[0] = gridDim.x;
+    p.cta_times[1 + 2 * blockIdx.x] = globaltimer_ns();
+  }
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
   const UnitSpace us = unit_space(p.sched, p.Hq, kSchedQ);
   const int n_units = us.n_units();
@@ -416,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) p.cta_times[2 + 2 * blockIdx.x] = globaltimer_ns();
   if (warp == kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
 }
 
@@ -431,6 +437,7 @@ cudaError_t launch_d(const FwdArgs& a, cudaStream_t stream) {
   Params p;
   p.cu = a.cu;
   p.sched = sched_view(a.sched);
+  p.cta_times = a.cta_times[0];
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.lse = a.lse;
   p.o_resid = static_cast<__nv_bfloat16*>(a.o_resid);

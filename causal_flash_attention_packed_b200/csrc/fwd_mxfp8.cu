@@ -90,6 +90,7 @@ struct Params {
   int T, Hq, Hkv, n_docs;
   float scale_log2;
   int rule;
+  unsigned long long* cta_times;  // per-CTA (start, end) records, or null
 };
 
 struct Item {
@@ -202,6 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) {  // scheduler balance record
+    if (blockIdx.x == 0) p.cta_times[0] = gridDim.x;
+    p.cta_times[1 + 2 * blockIdx.x] = globaltimer_ns();
+  }
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
   const UnitSpace us = unit_space(p.sched, p.Hq, kSchedQ);
   const int n_units = us.n_units();
@@ -549,6 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (p.cta_times && threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) p.cta_times[2 + 2 * blockIdx.x] = globaltimer_ns();
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
@@ -565,6 +571,7 @@ cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
   Params p;
   p.cu = a.cu;
   p.sched = sched_view(a.sched);
+  p.cta_times = a.cta_times[0];
   p.q_spt = a.q_spt;
   p.k_stb = a.k_stb;
   p.k_spt = a.k_spt;

@@ -60,8 +60,14 @@ cudaError_t launch_quantize_mxfp8(const void* x, int T, int H, int d, const int3
                                   int forms, int rule, uint8_t* vtb, uint8_t* stb, uint8_t* vpt,
                                   uint8_t* spt, cudaStream_t stream, void* deq_pt_bf16 = nullptr);
 
+// Per-CTA (start, end) %globaltimer records of one persistent kernel launch:
+// [0] = CTA count, then one pair per CTA (kMaxCtaTimes CTAs at most).
+constexpr int kMaxCtaTimes = 1024;
+constexpr size_t kCtaTimesWords = 1 + 2 * (size_t)kMaxCtaTimes;
+
 // Forward, bf16 operands (fwd_bf16.cu).
 struct FwdArgs {
+  unsigned long long* cta_times[2] = {nullptr, nullptr};  // per kernel, or null
   const void* q;
   const void* k;
   const void* v;
@@ -82,6 +88,7 @@ cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t stream);
 
 // Forward, MXFP8 path (fwd_mxfp8.cu): codes and scales from the quantiser.
 struct FwdMxArgs {
+  unsigned long long* cta_times[2] = {nullptr, nullptr};  // per kernel, or null
   const uint8_t* q_vpt;      // Q per-token codes [T][Hq][128]
   const uint8_t* q_spt;      // Q per-token scales [T][Hq][4]
   const uint8_t* k_vtb;      // K token-block codes [T][Hkv][128]
@@ -107,6 +114,7 @@ cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream);
 
 // Backward, MXFP8 path (bwd_mxfp8.cu).
 struct BwdMxArgs {
+  unsigned long long* cta_times[2] = {nullptr, nullptr};  // per kernel, or null
   const uint8_t *q_vtb, *q_stb, *q_vpt, *q_spt;     // quantised Q (ctx)
   const uint8_t *k_vtb, *k_stb, *k_vpt, *k_spt;     // quantised K (ctx)
   const uint8_t *v_vtb, *v_stb, *v_vpt, *v_spt;     // quantised V (ctx)
@@ -140,6 +148,7 @@ bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H);
 
 // Backward, bf16 operands (bwd_bf16.cu).
 struct BwdArgs {
+  unsigned long long* cta_times[2] = {nullptr, nullptr};  // per kernel, or null
   const void* q;
   const void* k;
   const void* v;

@@ -42,6 +42,7 @@ BWD = 1
 FORM_TB = 1
 FORM_PT = 2
 FLAG_INJECT_DROP_LOAD = 1
+FLAG_CTA_TIMES = 2
 
 
 class FapkError(RuntimeError):
@@ -99,6 +100,8 @@ def lib() -> ctypes.CDLL:
     L.fapk_quantize_mxfp8.restype = i
     L.fapk_status.argtypes = [vp, vp]
     L.fapk_status.restype = i
+    L.fapk_cta_times.argtypes = [PP, i, i, vp, vp, ctypes.POINTER(ctypes.c_ulonglong), i, ctypes.POINTER(i)]
+    L.fapk_cta_times.restype = i
     L.fapk_strerror.argtypes = [i]
     L.fapk_strerror.restype = ctypes.c_char_p
     L.fapk_launch_count.argtypes = []
@@ -281,6 +284,18 @@ def quantize_mxfp8(x: torch.Tensor, seq: Seqlens, forms: int = FORM_TB | FORM_PT
                                    _stream(stream))
     _check(rc, "fapk_quantize_mxfp8")
     return out
+
+
+def cta_times(P: Problem, which: int, kernel: int, ws: torch.Tensor, stream=None):
+    """Per-CTA (start, end) %globaltimer pairs (ns, int64 array [n, 2]) of
+    persistent kernel `kernel` of the last call made with FLAG_CTA_TIMES on
+    workspace `ws` (forward: 0; backward: 0 = dK/dV, 1 = dQ)."""
+    import numpy as np
+    out = (ctypes.c_ulonglong * (2 * 1024))()
+    n = ctypes.c_int(0)
+    _check(lib().fapk_cta_times(ctypes.byref(P), which, kernel, _ptr(ws), _stream(stream), out, 1024,
+                                ctypes.byref(n)), "fapk_cta_times")
+    return np.array(out[: 2 * n.value], dtype=np.int64).reshape(-1, 2)
 
 
 def status(ws: torch.Tensor, stream=None) -> int:

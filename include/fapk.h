@@ -107,7 +107,11 @@ enum {
    * one K/V tile copy, so the consumer's bounded wait runs out and the call
    * reports FAPK_ERR_DEVICE_TIMEOUT through fapk_status.  No fault, trap or
    * hang is involved. */
-  FAPK_FLAG_INJECT_DROP_LOAD = 1 << 0
+  FAPK_FLAG_INJECT_DROP_LOAD = 1 << 0,
+  /* Scheduler balance: every CTA of the call's persistent attention kernels
+   * records the %globaltimer (ns) when it starts and when it has finished its
+   * work units, in the workspace; read them back with fapk_cta_times. */
+  FAPK_FLAG_CTA_TIMES = 1 << 1
 };
 
 /* One attention problem.  All fields are read during the call only. */
@@ -211,6 +215,18 @@ FAPK_API int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const 
  *  - The device status word of these calls is not readable by the caller. */
 FAPK_API int fapk_attn_fwd_noalloc(const fapk_problem_t* prob, const void* q, const void* k,
                                    const void* v, void* o, float* lse, void* ctx, void* stream);
+
+/* Scheduler balance (the pages have no counterpart): after a call made with
+ * FAPK_FLAG_CTA_TIMES on workspace `ws` and problem `prob`, synchronises
+ * `stream` and copies, for the call's persistent kernel number `kernel`
+ * (forward, which = FAPK_FWD: 0 = the attention kernel; backward, which =
+ * FAPK_BWD: 0 = dK/dV, 1 = dQ), one (start, end) pair of %globaltimer values
+ * in ns per CTA into out_pairs[2 * i], out_pairs[2 * i + 1] for the first
+ * min(CTAs, max_ctas) CTAs; *n_ctas receives the kernel's CTA count.
+ * Host-owned output; FAPK_ERR_INVALID_ARG for a bad kernel number or null
+ * pointer, FAPK_ERR_CUDA if the copy fails. */
+FAPK_API int fapk_cta_times(const fapk_problem_t* prob, int which, int kernel, const void* ws, void* stream,
+                            unsigned long long* out_pairs, int max_ctas, int* n_ctas);
 
 /* Synchronises `stream`, then returns the device status word of the last call
  * that used workspace `ws` (FAPK_OK, FAPK_ERR_DEVICE_TIMEOUT, or

@@ -195,3 +195,50 @@ def test_bwd_dkdv_leak_free_at_block_aligned_t(t_rel):
     _, b = mx_fwd_bwd(w, dev, tensors=_perturb(base, t, 10, zero_dout=True))
     assert torch.equal(a[3][: t + 1], b[3][: t + 1])
     assert torch.equal(a[4][: t + 1], b[4][: t + 1])
+
+
+def _mx_sampled_docs(w, dev, max_tokens=6000, first_doc=0, kv_group=0):
+    """Full-size workload in the launch configuration the benchmark uses; the
+    oracle's MXFP8 emulation reruns whole documents (the scales are
+    document-local, so a document's outputs depend on its own tokens only)
+    for the query heads of one KV group: O, LSE, dQ, dK, dV of those
+    documents and heads against the emulation."""
+    (q, k, v, do), (o, lse, dq, dk, dv) = mx_fwd_bwd(w, dev)
+    cu = w.cu
+    lengths = np.diff(cu)
+    k0 = first_doc
+    k1 = k0
+    while k1 < w.n_docs and cu[k1 + 1] - cu[k0] <= max_tokens:
+        k1 += 1
+    if k1 == k0:  # the first candidate alone is longer than the budget
+        k1 = k0 + 1
+    t0, t1 = int(cu[k0]), int(cu[k1])
+    assert t1 > t0 and lengths[k0:k1].min() >= 0
+    G = w.Hq // w.Hkv
+    hs = list(range(kv_group * G, (kv_group + 1) * G))
+    cu_s = (cu[k0:k1 + 1] - t0).astype(np.int32)
+    sub_q = lambda x: x[t0:t1, hs].double().numpy()
+    sub_k = lambda x: x[t0:t1, kv_group:kv_group + 1].double().numpy()
+    em_o, em_l = oracle.mx_attn_fwd(sub_q(q), sub_k(k), sub_k(v), cu_s, w.scale, flags=oracle.MX_QUANT_P)
+    em = oracle.mx_attn_bwd(sub_q(q), sub_k(k), sub_k(v), sub_q(do), cu_s, w.scale, flags=oracle.MX_QUANT_P)
+    res = {
+        "o": rel_frob(f64(o)[t0:t1, hs], em_o),
+        "dq": rel_frob(f64(dq)[t0:t1, hs], em["dq"]),
+        "dk": rel_frob(f64(dk)[t0:t1, kv_group:kv_group + 1], em["dk"]),
+        "dv": rel_frob(f64(dv)[t0:t1, kv_group:kv_group + 1], em["dv"]),
+    }
+    for name, rf in res.items():
+        assert rf <= MX_REL_FROB, f"{name} rel_frob vs emulation {rf:.3e} (documents {k0}..{k1 - 1})"
+    assert float(np.max(np.abs(f64(lse)[hs, t0:t1] - em_l))) <= LSE_ABS
+    return res
+
+
+def test_full_size_packed_32k_documents_vs_emulation():
+    """The 32768-token benchmark workload (32 heads, 1% x8 outlier tokens)."""
+    _mx_sampled_docs(W.config(4, 0), require_gpu())
+
+
+def test_full_size_gqa_128k_documents_vs_emulation():
+    """131072 tokens with a 65536-token first document, 32 query heads on 8 KV
+    heads; two documents after the long one, KV group 3."""
+    _mx_sampled_docs(W.config(5, 0), require_gpu(), first_doc=4, kv_group=3)
