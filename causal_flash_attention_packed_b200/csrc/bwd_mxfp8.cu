@@ -370,10 +370,10 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       // D (tmem col) = A B^T, both K-major codes, block scales at TMEM cols sfa/sfb
       auto mx_kk = [&](uint32_t dcol, uint32_t a, uint32_t b, uint32_t sfa, uint32_t sfbc, bool b_mn,
                        bool acc_first) {
+        const uint64_t da = sdesc_sw128(a, 16, 1024), db = b_mn ? sdesc_sw128(b, 16384, 1024) : sdesc_sw128(b, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_mxf8_ss(tmem + dcol, sdesc_sw128(a + kk * 32, 16, 1024),
-                      b_mn ? sdesc_sw128(b + kk * 4096, 16384, 1024) : sdesc_sw128(b + kk * 32, 16, 1024),
+          mma_mxf8_ss(tmem + dcol, da + ((kk * 32) >> 4), db + ((b_mn ? kk * 4096 : kk * 32) >> 4),
                       idesc_mxf8(128, 128, b_mn, kk, kk), (tmem + sfa) | ((uint32_t)kk << 30),
                       (tmem + sfbc) | ((uint32_t)kk << 30), (acc_first || kk > 0) ? 1u : 0u);
       };
@@ -787,10 +787,10 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
       bool ok = true;
       auto mx_kk = [&](uint32_t dcol, uint32_t a, uint32_t b, uint32_t sfa, uint32_t sfbc, bool b_mn,
                        bool acc_first) {
+        const uint64_t da = sdesc_sw128(a, 16, 1024), db = b_mn ? sdesc_sw128(b, 16384, 1024) : sdesc_sw128(b, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_mxf8_ss(tmem + dcol, sdesc_sw128(a + kk * 32, 16, 1024),
-                      b_mn ? sdesc_sw128(b + kk * 4096, 16384, 1024) : sdesc_sw128(b + kk * 32, 16, 1024),
+          mma_mxf8_ss(tmem + dcol, da + ((kk * 32) >> 4), db + ((b_mn ? kk * 4096 : kk * 32) >> 4),
                       idesc_mxf8(128, 128, b_mn, kk, kk), (tmem + sfa) | ((uint32_t)kk << 30),
                       (tmem + sfbc) | ((uint32_t)kk << 30), (acc_first || kk > 0) ? 1u : 0u);
       };

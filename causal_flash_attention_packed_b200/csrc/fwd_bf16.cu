@@ -226,27 +226,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sq_addr = smem_u32(sQ), skv_addr = smem_u32(sKV);
       uint32_t kv_it = 0, p_cnt[2] = {0, 0}, o_used[2] = {0, 0};
       int unit_i = 0;
+      // Descriptors are built once per tile and advanced by constant offsets
+      // (start address >> 4 in the low field).
       // S_i = Q_i K^T: D/16 MMAs of K = 16 channels, 32 bytes apart inside a
       // 128-byte swizzle row, 16 KB apart across 64-channel boxes.
+      const uint64_t dq0 = sdesc_sw128(sq_addr, 16, 1024), dq1 = sdesc_sw128(sq_addr + C::kTileBytes, 16, 1024);
       auto issue_s = [&](int i, int kslot) {
-        const uint32_t qa = sq_addr + i * C::kTileBytes, ka = skv_addr + kslot * C::kTileBytes;
+        const uint64_t da = i ? dq1 : dq0, db = sdesc_sw128(skv_addr + kslot * C::kTileBytes, 16, 1024);
+        const uint32_t dcol = tmem + (i ? C::kSCol1 : C::kSCol0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-          mma_f16_ss(tmem + (i ? C::kSCol1 : C::kSCol0), sdesc_sw128(qa + off, 16, 1024),
-                     sdesc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0);
+          const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+          mma_f16_ss(dcol, da + off, db + off, idesc_qk, kk > 0);
         }
       };
       // O_i += P_i V: 8 MMAs of K = 16 keys; P_i from TMEM (8 packed columns
       // per step), V MN-major (16 keys = 2048 bytes per step, 64-channel
       // chunks 16 KB apart).
       auto issue_pv = [&](int i, int vslot, bool acc) {
-        const uint32_t va = skv_addr + vslot * C::kTileBytes;
-        const uint32_t pcol = tmem + (i ? C::kSCol1 : C::kSCol0);
+        const uint64_t dv = sdesc_sw128(skv_addr + vslot * C::kTileBytes, C::kBoxBytes, 1024);
+        const uint32_t pcol = tmem + (i ? C::kSCol1 : C::kSCol0), dcol = tmem + (i ? C::kOCol1 : C::kOCol0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_f16_ts(tmem + (i ? C::kOCol1 : C::kOCol0), pcol + kk * 8,
-                     sdesc_sw128(va + kk * 2048, C::kBoxBytes, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          mma_f16_ts(dcol, pcol + kk * 8, dv + ((kk * 2048) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
       };
       for (uint32_t uk = 0;; ++uk, ++unit_i) {
         const int w = unit_take(ring, uk, wd);

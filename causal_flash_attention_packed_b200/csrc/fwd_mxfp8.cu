@@ -303,12 +303,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         return mbar_wait(kv_full + (idx % kSlots), (idx / kSlots) & 1, wd, 53);
       };
       // S (into buffer col) = Q K^T with K codes at `kaddr` and its scales at TMEM column sfb
+      // descriptors built once per operand tile and advanced by constant
+      // offsets (start address >> 4 in the low field)
+      const uint64_t dq = sdesc_sw128(aq, 16, 1024), dp = sdesc_sw128(ap, 16, 1024);
       auto issue_s = [&](uint32_t col, uint32_t kaddr, uint32_t sfb) {
+        const uint64_t dk = sdesc_sw128(kaddr, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_mxf8_ss(tmem + col, sdesc_sw128(aq + kk * 32, 16, 1024), sdesc_sw128(kaddr + kk * 32, 16, 1024),
-                      idesc_mxf8(128, 128, false, kk, kk), (tmem + kSfQ) | ((uint32_t)kk << 30),
-                      (tmem + sfb) | ((uint32_t)kk << 30), kk > 0);
+          mma_mxf8_ss(tmem + col, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_mxf8(128, 128, false, kk, kk),
+                      (tmem + kSfQ) | ((uint32_t)kk << 30), (tmem + sfb) | ((uint32_t)kk << 30), kk > 0);
       };
       auto issue_s_tile = [&](int j, uint32_t col) {
         const int ks = kslot_of(j);
@@ -347,12 +350,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int vs = vslot_of(j);
           tmem_cp_sf(tmem + kSfP, asf + 2 * kSfBlk);
           tmem_cp_sf(tmem + kSfV, asf + (3 + vs) * kSfBlk);
-          const uint32_t av = aring + vs * kCodeTile;
+          const uint64_t dv = sdesc_sw128(aring + vs * kCodeTile, 16384, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_mxf8_ss(tmem + kO, sdesc_sw128(ap + kk * 32, 16, 1024), sdesc_sw128(av + kk * 4096, 16384, 1024),
-                        idesc_mxf8(128, 128, true, kk, kk), (tmem + kSfP) | ((uint32_t)kk << 30),
-                        (tmem + kSfV) | ((uint32_t)kk << 30), (j > 0 || kk > 0) ? 1u : 0u);
+            mma_mxf8_ss(tmem + kO, dp + ((kk * 32) >> 4), dv + ((kk * 4096) >> 4), idesc_mxf8(128, 128, true, kk, kk),
+                        (tmem + kSfP) | ((uint32_t)kk << 30), (tmem + kSfV) | ((uint32_t)kk << 30),
+                        (j > 0 || kk > 0) ? 1u : 0u);
           if (j == n - 1) {
             // diagonal 32x32 blocks: exact bf16 P~ times dequantised per-token V
             constexpr uint32_t idesc_d = idesc_bf16_f32(128, 128, false, true);
