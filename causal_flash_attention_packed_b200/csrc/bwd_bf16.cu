@@ -168,11 +168,15 @@ __device__ __forceinline__ void store_row32(void* base, size_t elem_off, const u
 // warps read S^T (then dP^T) out into registers and release the region at
 // once, so the MMAs run in the order S(t), dP(t), dV(t), S(t+1), dK(t),
 // dP(t+1), ... and the tensor pipe has the next independent MMA group queued
-// while the exponentials of a tile are computed.  16 compute warps:
-// warpgroup wg owns query columns [32 wg, 32 wg + 32) of every tile.
-constexpr int kKvThreads = 576;
+// while the exponentials of a tile are computed.  Two threads issue the MMAs:
+// warp 17 the scores S^T and dP^T, warp 18 the gradients dV and dK, so that a
+// wait of one never leaves the tensor pipe without the other's queued work.
+// 16 compute warps: warpgroup wg owns query columns [32 wg, 32 wg + 32) of
+// every tile.
+constexpr int kKvThreads = 608;
 constexpr int kKvLoadWarp = 16;
-constexpr int kKvMmaWarp = 17;
+constexpr int kKvMmaWarp = 17;   // S^T, dP^T; owns the TMEM allocation
+constexpr int kKvGradWarp = 18;  // dV, dK
 constexpr int kKvComputeWarps = 16;
 
 template <int D>
@@ -276,8 +280,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     mbar_init(dk_done, 1);
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kKvComputeWarps);
-    mbar_init(fin, 1);
-    unit_ring_init(ring, 1 + kKvComputeWarps);  // the MMA thread and the compute warps
+    mbar_init(fin, 2);
+    unit_ring_init(ring, 2 + kKvComputeWarps);  // both MMA threads and the compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -357,30 +361,22 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         drain_wait(o_full + (i % C::kOStages), (i / C::kOStages) & 1, p.timeout_ns);
     }
   } else if (warp == kKvMmaWarp) {
-    // ------------------------------------------------------------ MMA
+    // ------------------------------------------------------------ MMA: S^T, dP^T
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);  // K-major x K-major
-      constexpr uint32_t idesc_g = idesc_f16_f32(128, D, false, true);     // TMEM A x MN-major B
       const uint32_t sqr = smem_u32(sQr), sor = smem_u32(sOr);
       // descriptors: base + (byte offset >> 4) in the start-address field
       const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024), dv0 = sdesc_sw128(smem_u32(sV), 16, 1024);
       uint32_t t = 0, s_uses = 0;  // query tiles started; uses of the S^T / dP^T region
       int unit_i = 0;
       bool ok = true;
-      auto region = [&]() {  // the compute warps have read out the region's previous use
-        if (s_uses > 0 && !mbar_wait(s_free, (s_uses - 1) & 1, wd, 25)) return false;
-        tc_fence_after();
-        return true;
-      };
-      auto region_done = [&]() {
-        tc_commit(s_full);
-        ++s_uses;
-      };
-      // S^T (kv = 0) or dP^T (kv = 1) of tile tt into the region
+      // S^T (kv = 0) or dP^T (kv = 1) of tile tt into the region, once the
+      // compute warps have read out its previous use
       auto score = [&](uint32_t tt, int kv) {
         if (kv == 0 && !mbar_wait(q_full + (tt % C::kQStages), (tt / C::kQStages) & 1, wd, 26)) return false;
         if (kv == 1 && !mbar_wait(o_full + (tt % C::kOStages), (tt / C::kOStages) & 1, wd, 28)) return false;
-        if (!region()) return false;
+        if (s_uses > 0 && !mbar_wait(s_free, (s_uses - 1) & 1, wd, 25)) return false;
+        tc_fence_after();
         const uint32_t b_op = kv ? sor + (tt % C::kOStages) * C::kOStageBytes : sqr + (tt % C::kQStages) * C::kTileBytes;
         const uint64_t da = kv ? dv0 : dk0, db = sdesc_sw128(b_op, 16, 1024);
 #pragma unroll
@@ -388,7 +384,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           const uint32_t o = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
           mma_f16_ss(tmem + C::kSD, da + o, db + o, idesc_s, kk > 0);
         }
-        region_done();
+        tc_commit(s_full);
+        ++s_uses;
         return true;
       };
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
@@ -397,37 +394,58 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const KvItem it = kv_decode(p, us, w);
         const int R = G * (it.nq - it.v);
         if (!mbar_wait(kv_full, unit_i & 1, wd, 23)) break;
-        tc_fence_after();
-        if (!score(t, 0)) break;
         for (int r = 0; r < R; ++r, ++t) {
-          if (!score(t, 1)) { ok = false; break; }
+          if (!score(t, 0) || !score(t, 1)) { ok = false; break; }
+        }
+        if (!ok) break;
+        tc_commit(kv_empty);  // K and V are read by these MMAs only
+      }
+      tc_commit(fin);
+      drain_wait(fin, 0, p.timeout_ns);
+    }
+  } else if (warp == kKvGradWarp) {
+    // ------------------------------------------------------------ MMA: dV, dK
+    // Q and dO of a tile are released here: the score MMAs that also read them
+    // completed before the compute warps signalled P^T (S^T) and dS^T (dP^T).
+    if (lane == 0) {
+      constexpr uint32_t idesc_g = idesc_f16_f32(128, D, false, true);  // TMEM A x MN-major B
+      const uint32_t sqr = smem_u32(sQr), sor = smem_u32(sOr);
+      uint32_t t = 0;
+      int unit_i = 0;
+      bool ok = true;
+      for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+        const int w = unit_take(ring, uk, wd);
+        if (w < 0 || w >= n_units) break;
+        const KvItem it = kv_decode(p, us, w);
+        const int R = G * (it.nq - it.v);
+        for (int r = 0; r < R; ++r, ++t) {
+          const int qs = t % C::kQStages, os = t % C::kOStages;
           // dV += P^T dO
           if (r == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 24)) { ok = false; break; }
+          if (!mbar_wait(o_full + os, (t / C::kOStages) & 1, wd, 45)) { ok = false; break; }
           if (!mbar_wait(p_ready, t & 1, wd, 27)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t ddo = sdesc_sw128(sor + (t % C::kOStages) * C::kOStageBytes, C::kBoxBytes, 1024);
-          const uint64_t dq = sdesc_sw128(sqr + (t % C::kQStages) * C::kTileBytes, C::kBoxBytes, 1024);
+          const uint64_t ddo = sdesc_sw128(sor + os * C::kOStageBytes, C::kBoxBytes, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_f16_ts(tmem + C::kDV, tmem + C::kP + 8 * kk, ddo + ((kk * 2048) >> 4), idesc_g,
                        (r > 0 || kk > 0) ? 1u : 0u);
           tc_commit(dv_done);
-          tc_commit(o_empty + (t % C::kOStages));  // dV was the MMAs' last read of dO
-          // the next tile's S^T goes ahead of dK (its region was released when dP^T was read)
-          if (r + 1 < R && !score(t + 1, 0)) { ok = false; break; }
+          tc_commit(o_empty + os);
           // dK += dS^T Q
+          if (!mbar_wait(q_full + qs, (t / C::kQStages) & 1, wd, 46)) { ok = false; break; }
           if (!mbar_wait(ds_ready, t & 1, wd, 29)) { ok = false; break; }
           tc_fence_after();
+          const uint64_t dq = sdesc_sw128(sqr + qs * C::kTileBytes, C::kBoxBytes, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_f16_ts(tmem + C::kDK, tmem + C::kDS + 8 * kk, dq + ((kk * 2048) >> 4), idesc_g,
                        (r > 0 || kk > 0) ? 1u : 0u);
           tc_commit(dk_done);
-          tc_commit(q_empty + (t % C::kQStages));
+          tc_commit(q_empty + qs);
         }
         if (!ok) break;
         tc_commit(acc_full);
-        tc_commit(kv_empty);
       }
       tc_commit(fin);
       drain_wait(fin, 0, p.timeout_ns);
@@ -558,11 +576,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 // TMEM holds dQ, S, dP and the tile's dS (fp16).  The compute warps read S and
 // dP out into registers and release them at once, so S and dP of key tile
 // v + 1 are computed while dS of tile v is formed; dQ += dS K takes dS from
-// TMEM.  16 compute warps: warpgroup wg owns key columns [32 wg, 32 wg + 32)
-// of every tile; each thread owns one query row.
-constexpr int kQThreads = 576;
+// TMEM.  Warp 17 issues the score MMAs S and dP, warp 18 the gradient MMA dQ,
+// so that a wait of one never leaves the tensor pipe without the other's
+// queued work.  16 compute warps: warpgroup wg owns key columns
+// [32 wg, 32 wg + 32) of every tile; each thread owns one query row.
+constexpr int kQThreads = 608;
 constexpr int kQLoadWarp = 16;
-constexpr int kQMmaWarp = 17;
+constexpr int kQMmaWarp = 17;   // S, dP; owns the TMEM allocation
+constexpr int kQGradWarp = 18;  // dQ
 constexpr int kQComputeWarps = 16;
 
 template <int D>
@@ -648,8 +669,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
     mbar_init(dq_done, 1);
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kQComputeWarps);
-    mbar_init(fin, 1);
-    unit_ring_init(ring, 1 + kQComputeWarps);  // the MMA thread and the compute warps
+    mbar_init(fin, 2);
+    unit_ring_init(ring, 2 + kQComputeWarps);  // both MMA threads and the compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -705,64 +726,81 @@ __global__ void __launch_bounds__(kQThreads, 1)
         drain_wait(v_full + (i % C::kVStages), (i / C::kVStages) & 1, p.timeout_ns);
     }
   } else if (warp == kQMmaWarp) {
+    // ------------------------------------------------------------ MMA: S, dP
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);
-      constexpr uint32_t idesc_g = idesc_f16_f32(128, D, false, true);
       const uint32_t skr = smem_u32(sKr), svr = smem_u32(sVr);
       const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024), ddo0 = sdesc_sw128(smem_u32(sDO), 16, 1024);
-      uint32_t st_it = 0;  // key tiles started (all units)
+      uint32_t kt = 0;  // key tiles started (all units)
       int unit_i = 0;
       bool ok = true;
-      // S and dP of key tile number kt (global count) into their regions
-      auto scores = [&](uint32_t kt) {
-        const int ks = kt % C::kKStages, vs = kt % C::kVStages;
-        if (!mbar_wait(k_full + ks, (kt / C::kKStages) & 1, wd, 35)) return false;
-        const uint64_t dk = sdesc_sw128(skr + ks * C::kTileBytes, 16, 1024);
-        const uint64_t dv = sdesc_sw128(svr + vs * C::kTileBytes, 16, 1024);
-        if (kt > 0 && !mbar_wait(s_free, (kt - 1) & 1, wd, 36)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
-          mma_f16_ss(tmem + C::kS, dq0 + o, dk + o, idesc_s, kk > 0);
-        }
-        tc_commit(s_full);
-        if (kt > 0 && !mbar_wait(dp_free, (kt - 1) & 1, wd, 37)) return false;
-        if (!mbar_wait(v_full + vs, (kt / C::kVStages) & 1, wd, 44)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
-          mma_f16_ss(tmem + C::kDP, ddo0 + o, dv + o, idesc_s, kk > 0);
-        }
-        tc_commit(dp_full);
-        tc_commit(v_empty + vs);  // V is read only by dP
-        return true;
-      };
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
         const int w = unit_take(ring, uk, wd);
         if (w < 0 || w >= n_units) break;
         const QItem it = q_decode(p, us, w);
         if (!mbar_wait(q_full, unit_i & 1, wd, 33)) break;
-        tc_fence_after();
-        if (!scores(st_it)) break;
-        for (int v = 0; v <= it.m; ++v, ++st_it) {
-          // the next key tile's S and dP go ahead of this tile's dQ
-          if (v < it.m && !scores(st_it + 1)) { ok = false; break; }
-          if (v == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 34)) { ok = false; break; }
-          if (!mbar_wait(ds_ready, st_it & 1, wd, 38)) { ok = false; break; }
+        for (int v = 0; v <= it.m; ++v, ++kt) {
+          // S and dP of key tile kt into their regions, each once the compute
+          // warps have read out its previous use
+          const int ks = kt % C::kKStages, vs = kt % C::kVStages;
+          if (!mbar_wait(k_full + ks, (kt / C::kKStages) & 1, wd, 35)) { ok = false; break; }
+          if (kt > 0 && !mbar_wait(s_free, (kt - 1) & 1, wd, 36)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t dkm = sdesc_sw128(skr + (st_it % C::kKStages) * C::kTileBytes, C::kBoxBytes, 1024);
+          const uint64_t dk = sdesc_sw128(skr + ks * C::kTileBytes, 16, 1024);
+          const uint64_t dv = sdesc_sw128(svr + vs * C::kTileBytes, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t o = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+            mma_f16_ss(tmem + C::kS, dq0 + o, dk + o, idesc_s, kk > 0);
+          }
+          tc_commit(s_full);
+          if (kt > 0 && !mbar_wait(dp_free, (kt - 1) & 1, wd, 37)) { ok = false; break; }
+          if (!mbar_wait(v_full + vs, (kt / C::kVStages) & 1, wd, 44)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t o = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+            mma_f16_ss(tmem + C::kDP, ddo0 + o, dv + o, idesc_s, kk > 0);
+          }
+          tc_commit(dp_full);
+          tc_commit(v_empty + vs);  // V is read only by dP
+        }
+        if (!ok) break;
+        tc_commit(q_empty);  // Q and dO are read only by S and dP
+      }
+      tc_commit(fin);
+      drain_wait(fin, 0, p.timeout_ns);
+    }
+  } else if (warp == kQGradWarp) {
+    // ------------------------------------------------------------ MMA: dQ
+    // K of a tile is released here: S, its other reader, completed before the
+    // compute warps signalled dS.
+    if (lane == 0) {
+      constexpr uint32_t idesc_g = idesc_f16_f32(128, D, false, true);
+      const uint32_t skr = smem_u32(sKr);
+      uint32_t kt = 0;
+      int unit_i = 0;
+      bool ok = true;
+      for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+        const int w = unit_take(ring, uk, wd);
+        if (w < 0 || w >= n_units) break;
+        const QItem it = q_decode(p, us, w);
+        for (int v = 0; v <= it.m; ++v, ++kt) {
+          const int ks = kt % C::kKStages;
+          if (v == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 34)) { ok = false; break; }
+          if (!mbar_wait(k_full + ks, (kt / C::kKStages) & 1, wd, 47)) { ok = false; break; }
+          if (!mbar_wait(ds_ready, kt & 1, wd, 38)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t dkm = sdesc_sw128(skr + ks * C::kTileBytes, C::kBoxBytes, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_f16_ts(tmem + C::kDQ, tmem + C::kDS + 8 * kk, dkm + ((kk * 2048) >> 4), idesc_g,
                        (v > 0 || kk > 0) ? 1u : 0u);
           tc_commit(dq_done);
-          tc_commit(k_empty + (st_it % C::kKStages));
+          tc_commit(k_empty + ks);
         }
         if (!ok) break;
         tc_commit(acc_full);
-        tc_commit(q_empty);
       }
       tc_commit(fin);
       drain_wait(fin, 0, p.timeout_ns);
