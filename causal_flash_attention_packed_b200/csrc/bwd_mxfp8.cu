@@ -204,8 +204,10 @@ __device__ __forceinline__ void store_row32(void* base, size_t elem_off, const u
 // ---------------------------------------------------------------------------
 namespace dqk {
 // warps 0-15: one thread per (query row, 32-key block): warpgroup wg on key
-// block wg of every tile (one MX scale block of dS~); warp 16: loads; warp 17: MMA
-constexpr int kThreads = 576, kLoad = 16, kMma = 17, kComputeWarps = 16, kStages = 2;
+// block wg of every tile (one MX scale block of dS~); warp 16: loads; warp 17:
+// the score MMAs S and dP; warp 18: the dQ MMAs (two issuing threads, so that a
+// wait of one never leaves the tensor pipe without the other's queued work)
+constexpr int kThreads = 608, kLoad = 16, kMma = 17, kGrad = 18, kComputeWarps = 16, kStages = 2;
 constexpr int oQ = 0, oDO = oQ + kCode, oRing = oDO + kCode;  // ring stage: K^tb, V^tb codes
 constexpr int oKpt = oRing + kStages * 2 * kCode, oVpt = oKpt + kCode, oKd = oVpt + kCode;  // diag
 constexpr int oDS = oKd + kBf16, oDSd = oDS + kCode;
@@ -274,8 +276,8 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
     mbar_init(dq_done, 1);
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kComputeWarps);
-    mbar_init(fin, 1);
-    unit_ring_init(ring, 1 + kComputeWarps);  // the MMA thread and the compute warps
+    mbar_init(fin, 2);
+    unit_ring_init(ring, 2 + kComputeWarps);  // both MMA threads and the compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -359,7 +361,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       for (uint32_t i = (st_it > kStages ? st_it - kStages : 0); i < st_it; ++i)
         drain_wait(st_full + (i % kStages), (i / kStages) & 1, p.timeout_ns);
     }
-  } else if (warp == kMma) {
+  } else if (warp == kMma || warp == kGrad) {
     if (lane == 0) {
       const uint32_t aQ = smem_u32(smem + oQ), aDO = smem_u32(smem + oDO), aRing = smem_u32(smem + oRing),
                      aKpt = smem_u32(smem + oKpt), aVpt = smem_u32(smem + oVpt), aKd = smem_u32(smem + oKd),
@@ -377,84 +379,81 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
                       idesc_mxf8(128, 128, b_mn, kk, kk), (tmem + sfa) | ((uint32_t)kk << 30),
                       (tmem + sfbc) | ((uint32_t)kk << 30), (acc_first || kk > 0) ? 1u : 0u);
       };
-      auto region_s = [&]() {
-        if (s_uses > 0 && !mbar_wait(s_free, (s_uses - 1) & 1, wd, 73)) return false;
-        tc_fence_after();
-        return true;
-      };
-      auto region_dp = [&]() {
-        if (dp_uses > 0 && !mbar_wait(dp_free, (dp_uses - 1) & 1, wd, 74)) return false;
-        tc_fence_after();
-        return true;
-      };
-      // S and dP of key tile number tt (token-block K and V)
-      auto scores_tb = [&](uint32_t tt) {
-        const int stg = tt % kStages;
-        if (!mbar_wait(st_full + stg, (tt / kStages) & 1, wd, 75)) return false;
-        const uint32_t ak = aRing + stg * 2 * kCode, av = ak + kCode;
-        if (!region_s()) return false;
-        tmem_cp_sf(tmem + tSfK, aSf + (5 + 3 * stg) * kSfBlk);
-        mx_kk(tS, aQ, ak, tSfQ, tSfK, false, false);
-        tc_commit(s_full);
-        ++s_uses;
-        if (!region_dp()) return false;
-        tmem_cp_sf(tmem + tSfV, aSf + (6 + 3 * stg) * kSfBlk);
-        mx_kk(tDP, aDO, av, tSfDO, tSfV, false, false);
-        tc_commit(dp_full);
-        ++dp_uses;
-        return true;
-      };
-      for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_take(ring, uk, wd);
-        if (w < 0 || w >= n_units) break;
-        int doc, s, e, h, g, q0, n;
-        decode(w, doc, s, e, h, g, q0, n);
-        if (!mbar_wait(q_full, unit_i & 1, wd, 76)) break;
-        tc_fence_after();
-        tmem_cp_sf(tmem + tSfQ, aSf + 0 * kSfBlk);
-        tmem_cp_sf(tmem + tSfDO, aSf + 1 * kSfBlk);
-        tmem_cp_sf(tmem + tSfKpt, aSf + 2 * kSfBlk);
-        tmem_cp_sf(tmem + tSfVpt, aSf + 3 * kSfBlk);
-        if (!scores_tb(kt)) break;
-        for (int v = 0; v < n; ++v, ++kt) {
-          const int stg = kt % kStages;
-          const bool diag = v == n - 1;
-          if (diag) {
-            // diagonal tile: per-token K and V into the regions once the
-            // token-block scores were read
-            if (!region_s()) { ok = false; break; }
-            mx_kk(tS, aQ, aKpt, tSfQ, tSfKpt, false, false);
-            tc_commit(s_full);
-            ++s_uses;
-            if (!region_dp()) { ok = false; break; }
-            mx_kk(tDP, aDO, aVpt, tSfDO, tSfVpt, false, false);
-            tc_commit(dp_full);
-            ++dp_uses;
-          } else if (!scores_tb(kt + 1)) {  // the next key tile goes ahead of this tile's dQ
-            ok = false;
-            break;
-          }
-          if (v == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 77)) { ok = false; break; }
-          if (!mbar_wait(ds_ready, kt & 1, wd, 78)) { ok = false; break; }
+      if (warp == kMma) {
+        // ---------------------------------------------- S, dP
+        // each score MMA goes into its region once the compute warps have read
+        // out the previous use; the regions' reads of Q, dO, the per-token K and
+        // V and the stage's V end here, K^tb is read by dQ too
+        auto score = [&](bool dp, uint32_t a, uint32_t b, uint32_t sfa, uint32_t sfbc) {
+          uint32_t& uses = dp ? dp_uses : s_uses;
+          if (uses > 0 && !mbar_wait(dp ? dp_free : s_free, (uses - 1) & 1, wd, dp ? 74 : 73)) return false;
           tc_fence_after();
-          const uint32_t ak = aRing + stg * 2 * kCode;
-          tmem_cp_sf(tmem + tSfDS, aSf + 4 * kSfBlk);
-          tmem_cp_sf(tmem + tSfKdq, aSf + (7 + 3 * stg) * kSfBlk);
-          mx_kk(tDQ, aDS, ak, tSfDS, tSfKdq, true, v > 0);
-          if (diag) {
-            // diagonal 32x32 blocks: exact bf16 dS~ times dequantised per-token K
-            constexpr uint32_t idesc_d = idesc_bf16_f32(128, 128, false, true);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_f16_ss(tmem + tDQ, sdesc_sw128(aDSd + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024),
-                         sdesc_sw128(aKd + kk * 2048, kBox, 1024), idesc_d, 1u);
+          mx_kk(dp ? tDP : tS, a, b, sfa, sfbc, false, false);
+          tc_commit(dp ? dp_full : s_full);
+          ++uses;
+          return true;
+        };
+        for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+          const int w = unit_take(ring, uk, wd);
+          if (w < 0 || w >= n_units) break;
+          int doc, s, e, h, g, q0, n;
+          decode(w, doc, s, e, h, g, q0, n);
+          if (!mbar_wait(q_full, unit_i & 1, wd, 76)) break;
+          tc_fence_after();
+          tmem_cp_sf(tmem + tSfQ, aSf + 0 * kSfBlk);
+          tmem_cp_sf(tmem + tSfDO, aSf + 1 * kSfBlk);
+          tmem_cp_sf(tmem + tSfKpt, aSf + 2 * kSfBlk);
+          tmem_cp_sf(tmem + tSfVpt, aSf + 3 * kSfBlk);
+          for (int v = 0; v < n; ++v, ++kt) {
+            // token-block S and dP of key tile kt
+            const int stg = kt % kStages;
+            if (!mbar_wait(st_full + stg, (kt / kStages) & 1, wd, 75)) { ok = false; break; }
+            const uint32_t ak = aRing + stg * 2 * kCode, av = ak + kCode;
+            tmem_cp_sf(tmem + tSfK, aSf + (5 + 3 * stg) * kSfBlk);
+            if (!score(false, aQ, ak, tSfQ, tSfK)) { ok = false; break; }
+            tmem_cp_sf(tmem + tSfV, aSf + (6 + 3 * stg) * kSfBlk);
+            if (!score(true, aDO, av, tSfDO, tSfV)) { ok = false; break; }
           }
-          tc_commit(dq_done);
-          tc_commit(st_empty + stg);
+          if (!ok) break;
+          // the diagonal tile again with the per-token K and V
+          if (!score(false, aQ, aKpt, tSfQ, tSfKpt) || !score(true, aDO, aVpt, tSfDO, tSfVpt)) break;
         }
-        if (!ok) break;
-        tc_commit(acc_full);
-        tc_commit(q_empty);
+      } else {
+        // ---------------------------------------------- dQ
+        // the stage and the unit's buffers are released here: the score MMAs
+        // that also read them completed before the compute warps signalled dS~
+        for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
+          const int w = unit_take(ring, uk, wd);
+          if (w < 0 || w >= n_units) break;
+          int doc, s, e, h, g, q0, n;
+          decode(w, doc, s, e, h, g, q0, n);
+          if (!mbar_wait(q_full, unit_i & 1, wd, 101)) break;
+          for (int v = 0; v < n; ++v, ++kt) {
+            const int stg = kt % kStages;
+            const bool diag = v == n - 1;
+            if (v == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 77)) { ok = false; break; }
+            if (!mbar_wait(st_full + stg, (kt / kStages) & 1, wd, 102)) { ok = false; break; }
+            if (!mbar_wait(ds_ready, kt & 1, wd, 78)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t ak = aRing + stg * 2 * kCode;
+            tmem_cp_sf(tmem + tSfDS, aSf + 4 * kSfBlk);
+            tmem_cp_sf(tmem + tSfKdq, aSf + (7 + 3 * stg) * kSfBlk);
+            mx_kk(tDQ, aDS, ak, tSfDS, tSfKdq, true, v > 0);
+            if (diag) {
+              // diagonal 32x32 blocks: exact bf16 dS~ times dequantised per-token K
+              constexpr uint32_t idesc_d = idesc_bf16_f32(128, 128, false, true);
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                mma_f16_ss(tmem + tDQ, sdesc_sw128(aDSd + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024),
+                           sdesc_sw128(aKd + kk * 2048, kBox, 1024), idesc_d, 1u);
+            }
+            tc_commit(dq_done);
+            tc_commit(st_empty + stg);
+          }
+          if (!ok) break;
+          tc_commit(acc_full);
+          tc_commit(q_empty);
+        }
       }
       tc_commit(fin);
       drain_wait(fin, 0, p.timeout_ns);

@@ -332,21 +332,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[128];
         tmem_ld128(s_addr, r);
         float x[128];
-        float mx = -INFINITY;
         const int key0 = it.s + 128 * j;
         if (j == n - 1) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            x[c] = (key0 + c <= q_idx) ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, x[c]);
-          }
+          for (int c = 0; c < 128; ++c) x[c] = (key0 + c <= q_idx) ? __uint_as_float(r[c]) : -INFINITY;
         } else {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            x[c] = __uint_as_float(r[c]) * p.scale_log2;
-            mx = fmaxf(mx, x[c]);
-          }
+          for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(r[c]);
         }
+        // row maximum of the raw scores (the scale is positive) through eight
+        // independent partial maxima, so that no 128-long dependency chain
+        // sits between the scores' arrival and P; column 0 of the last key
+        // tile is the query's own key, so the maximum is finite
+        float pm[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pm[k] = x[k];
+#pragma unroll
+        for (int c = 8; c < 128; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * p.scale_log2;
         const float m_new = fmaxf(m, mx);
         const bool need = m_new > m + kRescaleThreshold;
         float alpha = 1.f;
@@ -356,15 +360,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
           l *= alpha;
         }
+        // P = 2^(s scale log2(e) - m) with one FMA per element; row sum in
+        // four independent partial sums
         uint32_t pk[64];
-        float rs = 0.f;
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        const float nm = -m;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float a = fast_exp2(x[2 * c] - m), b = fast_exp2(x[2 * c + 1] - m);
-          rs += a + b;
+          const float a = fast_exp2(fmaf(x[2 * c], p.scale_log2, nm));
+          const float b = fast_exp2(fmaf(x[2 * c + 1], p.scale_log2, nm));
+          rs[c & 3] += a + b;
           pk[c] = pack_f16x2(a, b);
         }
-        l += rs;
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
         tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
         if (any_need && j > 0) {
