@@ -58,13 +58,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
 }
 
-// One arrival per warp: every lane's prior tcgen05 and shared-memory work is
-// ordered before lane 0's arrive by the warp barrier.
-__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
 // ---------------------------------------------------------------------------
 // 1. D = rowsum(dO * O), fp32 [Hq][T]
 // ---------------------------------------------------------------------------
@@ -137,28 +130,10 @@ struct BwdParams {
   float scale;       // softmax scale (dK, dQ factor)
   float scale_log2;  // scale * log2(e)
   int grad_bf16;
+  int wide;  // every gradient output 32-byte aligned: 32-byte stores
   unsigned long long* cta_times;  // per-CTA (start, end) records, or null
 };
 
-// Store 32 fp32 values (times `mul`) of one row as fp32 or bf16.
-__device__ __forceinline__ void store_row32(void* base, size_t elem_off, const uint32_t (&t)[32], float mul,
-                                            bool bf16) {
-  if (bf16) {
-    uint32_t ob[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e)
-      ob[e] = pack_bf16x2(__uint_as_float(t[2 * e]) * mul, __uint_as_float(t[2 * e + 1]) * mul);
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + elem_off);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
-  } else {
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(base) + elem_off);
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      dst[e] = make_float4(__uint_as_float(t[4 * e]) * mul, __uint_as_float(t[4 * e + 1]) * mul,
-                           __uint_as_float(t[4 * e + 2]) * mul, __uint_as_float(t[4 * e + 3]) * mul);
-  }
-}
 
 // ---------------------------------------------------------------------------
 // 2. dK, dV
@@ -556,7 +531,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         uint32_t tt[32];
         tmem_ld32(acc_addr + 32 * c, tt);
         tmem_wait_ld(tt);
-        if (valid) store_row32(out, ((size_t)j * p.Hkv + it.g) * D + c0 + 32 * c, tt, mul, p.grad_bf16);
+        if (valid) store_row32(out, ((size_t)j * p.Hkv + it.g) * D + c0 + 32 * c, tt, mul, p.grad_bf16, p.wide);
       }
       tc_fence_before();
       warp_arrive(acc_free);
@@ -867,7 +842,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const int col = wg * 32;
         tmem_ld32(lane_base + C::kDQ + col, t);
         tmem_wait_ld(t);
-        if (valid) store_row32(p.out0, ((size_t)i * p.Hq + it.h) * D + col, t, p.scale, p.grad_bf16);
+        if (valid) store_row32(p.out0, ((size_t)i * p.Hq + it.h) * D + col, t, p.scale, p.grad_bf16, p.wide);
       }
       tc_fence_before();
       warp_arrive(acc_free);
@@ -925,6 +900,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     pk.cta_times = a.cta_times[0];
     pk.out0 = a.dk;
     pk.out1 = a.dv;
+    pk.wide = aligned32(a.dk) && aligned32(a.dv);
     const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
     const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
     dkdv_kernel<D><<<grid, kKvThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, pk);
@@ -942,6 +918,7 @@ cudaError_t launch_d(const BwdArgs& a, cudaStream_t stream) {
     pq.sched = sched_view(a.sched_q);
     pq.cta_times = a.cta_times[1];
     pq.out0 = a.dq;
+    pq.wide = aligned32(a.dq);
     pq.out1 = nullptr;
     const long long max_units = (long long)a.sched_q.max_items * a.Hq;
     const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);

@@ -176,28 +176,11 @@ struct MxParams {
   int T, Hq, Hkv;
   float scale, scale_log2;
   int grad_bf16;
+  int wide;  // every gradient output 32-byte aligned: 32-byte stores
   int rule;
   unsigned long long* cta_times;  // per-CTA (start, end) records, or null
 };
 
-__device__ __forceinline__ void store_row32(void* base, size_t elem_off, const uint32_t (&t)[32], float mul,
-                                            bool bf16) {
-  if (bf16) {
-    uint32_t ob[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e)
-      ob[e] = pack_bf16x2(__uint_as_float(t[2 * e]) * mul, __uint_as_float(t[2 * e + 1]) * mul);
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + elem_off);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
-  } else {
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(base) + elem_off);
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      dst[e] = make_float4(__uint_as_float(t[4 * e]) * mul, __uint_as_float(t[4 * e + 1]) * mul,
-                           __uint_as_float(t[4 * e + 2]) * mul, __uint_as_float(t[4 * e + 3]) * mul);
-  }
-}
 
 // ---------------------------------------------------------------------------
 // dQ
@@ -225,11 +208,6 @@ constexpr uint32_t tS = 0, tDP = 128, tDQ = 256;
 constexpr uint32_t tSfQ = 384, tSfDO = 388, tSfK = 392, tSfV = 396, tSfKpt = 400, tSfVpt = 404, tSfDS = 408,
                    tSfKdq = 412;
 }  // namespace dqk
-
-__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
 
 __global__ void __launch_bounds__(dqk::kThreads, 1)
     dq_mx_kernel(const __grid_constant__ CUtensorMap tm_qpt, const __grid_constant__ CUtensorMap tm_dopt,
@@ -549,7 +527,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         uint32_t t[32];
         tmem_ld32(lb + tDQ + 32 * wg, t);
         tmem_wait_ld(t);
-        if (valid) store_row32(p.out0, ((size_t)i * p.Hq + h) * 128 + 32 * wg, t, p.scale, p.grad_bf16);
+        if (valid) store_row32(p.out0, ((size_t)i * p.Hq + h) * 128 + 32 * wg, t, p.scale, p.grad_bf16, p.wide);
       }
       tc_fence_before();
       warp_arrive(acc_free);
@@ -989,7 +967,7 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
         uint32_t tt[32];
         tmem_ld32(acc + 32 * c, tt);
         tmem_wait_ld(tt);
-        if (valid) store_row32(out, ((size_t)j * p.Hkv + g) * 128 + c0 + 32 * c, tt, mul, p.grad_bf16);
+        if (valid) store_row32(out, ((size_t)j * p.Hkv + g) * 128 + c0 + 32 * c, tt, mul, p.grad_bf16, p.wide);
       }
       tc_fence_before();
       warp_arrive(acc_free);
@@ -1051,6 +1029,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     pk.cta_times = a.cta_times[0];
     pk.out0 = a.dk;
     pk.out1 = a.dv;
+    pk.wide = aligned32(a.dk) && aligned32(a.dv);
     const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
     const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
     dkdv_mx_kernel<<<grid, kvk::kThreads, kvk::kSmem, stream>>>(tktb, tkpt, tvtb, tvpt, tqpt, tqtb, tdopt, tdotb, pk);
@@ -1067,6 +1046,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     pq.sched = sched_view(a.sched_q);
     pq.cta_times = a.cta_times[1];
     pq.out0 = a.dq;
+    pq.wide = aligned32(a.dq);
     pq.out1 = nullptr;
     const long long max_units = (long long)a.sched_q.max_items * a.Hq;
     const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);

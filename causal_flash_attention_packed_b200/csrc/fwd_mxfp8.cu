@@ -120,12 +120,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
 }
 
-// One arrival per warp, after every lane's prior work (warp barrier first).
-__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
 // 4 scale bytes of token t (per-token form), or the neutral byte 127 (2^0)
 // past the end of the tensor.
 __device__ __forceinline__ uint32_t pt_word(const uint8_t* spt, int t, int T, int H, int h) {

@@ -10,6 +10,10 @@
 
 namespace fapk {
 
+// 32-byte alignment of an output buffer: kernels then write whole 32-byte
+// sectors per store instruction (null counts as aligned).
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
 struct DeviceStatus;
 
 // Optional CUDA events recorded between a call's kernel launches (profiling).

@@ -101,10 +101,4 @@ __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint32_t smem_block) 
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
 
-// Generic-proxy shared-memory writes made visible to the async proxy
-// (TMA, tcgen05.mma / tcgen05.cp operands).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 }  // namespace fapk

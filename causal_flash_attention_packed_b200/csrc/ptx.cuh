@@ -294,4 +294,67 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 // Largest finite fp16 magnitude: values at or above it cannot be converted.
 constexpr float kF16Max = 65504.0f;
 
+// One arrival per warp: every lane's prior tcgen05 and shared-memory work is
+// ordered before lane 0's arrive by the warp barrier.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// Generic-proxy shared-memory writes made visible to the async proxy
+// (TMA, tcgen05.mma / tcgen05.cp operands).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// max(a, b, c) in one instruction (three-operand max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 32 bytes to global memory in one instruction (st.global.v8, sm_100); the
+// address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_32B(void* ptr, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+// 32 fp32 accumulator columns of one row, times `mul`, to global memory as
+// bf16 or fp32 at element offset elem_off of `base`.  With `wide` (base and
+// offset 32-byte aligned) each instruction writes a whole 32-byte sector.
+__device__ __forceinline__ void store_row32(void* base, size_t elem_off, const uint32_t (&t)[32], float mul,
+                                            bool bf16, bool wide) {
+  if (bf16) {
+    uint32_t ob[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      ob[e] = pack_bf16x2(__uint_as_float(t[2 * e]) * mul, __uint_as_float(t[2 * e + 1]) * mul);
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(base) + elem_off;
+    if (wide) {
+      st_global_32B(dst, ob);
+      st_global_32B(dst + 16, ob + 8);
+    } else {
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d4[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+    }
+  } else {
+    uint32_t of[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) of[e] = __float_as_uint(__uint_as_float(t[e]) * mul);
+    float* dst = static_cast<float*>(base) + elem_off;
+    if (wide) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) st_global_32B(dst + 8 * e, of + 8 * e);
+    } else {
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) d4[e] = make_uint4(of[4 * e], of[4 * e + 1], of[4 * e + 2], of[4 * e + 3]);
+    }
+  }
+}
+
 }  // namespace fapk
