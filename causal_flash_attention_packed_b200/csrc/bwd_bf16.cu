@@ -171,19 +171,21 @@ struct KvCfg : Geo<D> {
   static constexpr int kNumBars = 2 + 2 * kQStages + 2 * kOStages + 9 + 2 * kUnitRing;
   // no alignment slack: the kernel checks that dynamic shared memory starts
   // on a 1024-byte boundary
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 4 * kUnitRing;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + kUnitRingBytes;
 };
+static_assert(KvCfg<128>::kSmemBytes <= 227 * 1024 && KvCfg<64>::kSmemBytes <= 227 * 1024,
+              "shared memory of the dK/dV kernel exceeds the 227 KB a CTA may use");
 
 struct KvItem {
   int s, e, v, g, k0, nq;  // k0: first key of the tile; query tiles v..nq-1
 };
 
-__device__ __forceinline__ KvItem kv_decode(const BwdParams& p, const UnitSpace& us, int w) {
+__device__ __forceinline__ KvItem kv_decode(const UnitInfo& un) {
   KvItem it;
-  int doc;
-  unit_decode(us, w, doc, it.v, it.g);
-  it.s = p.cu[doc];
-  it.e = p.cu[doc + 1];
+  it.v = un.tile;
+  it.g = un.h;
+  it.s = un.s;
+  it.e = un.e;
   it.k0 = it.s + 128 * it.v;
   it.nq = (it.e - it.s + 127) / 128;
   return it;
@@ -283,11 +285,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     int unit_i = 0;
     bool ok = true;
     for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-      int w = 0;
-      if (lane == 0) w = unit_produce(ring, p.sched.next, uk, wd);
-      w = __shfl_sync(0xFFFFFFFFu, w, 0);
+      const UnitInfo un = unit_produce_warp(ring, us, p.cu, p.sched.next, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
-      const KvItem it = kv_decode(p, us, w);
+      const KvItem it = kv_decode(un);
       if (unit_i > 0 && !warp_wait(kv_empty, (unit_i - 1) & 1, wd, 21)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
@@ -364,9 +365,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         return true;
       };
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_take(ring, uk, wd);
+        const UnitInfo un = unit_take(ring, uk, wd);
+        const int w = un.w;
         if (w < 0 || w >= n_units) break;
-        const KvItem it = kv_decode(p, us, w);
+        const KvItem it = kv_decode(un);
         const int R = G * (it.nq - it.v);
         if (!mbar_wait(kv_full, unit_i & 1, wd, 23)) break;
         for (int r = 0; r < R; ++r, ++t) {
@@ -389,9 +391,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       int unit_i = 0;
       bool ok = true;
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_take(ring, uk, wd);
+        const UnitInfo un = unit_take(ring, uk, wd);
+        const int w = un.w;
         if (w < 0 || w >= n_units) break;
-        const KvItem it = kv_decode(p, us, w);
+        const KvItem it = kv_decode(un);
         const int R = G * (it.nq - it.v);
         for (int r = 0; r < R; ++r, ++t) {
           const int qs = t % C::kQStages, os = t % C::kOStages;
@@ -444,9 +447,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       return true;
     };
     for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-      const int w = unit_take_warp(ring, uk, wd);
+      const UnitInfo un = unit_take_warp(ring, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
-      const KvItem it = kv_decode(p, us, w);
+      const KvItem it = kv_decode(un);
       const int j = it.k0 + row;  // key index
       for (int h = it.g * G; h < (it.g + 1) * G && ok; ++h) {
         for (int m = it.v; m < it.nq; ++m, ++t) {
@@ -573,20 +577,22 @@ struct QCfg : Geo<D> {
   //       ds_ready, dq_done, acc_full, acc_free, fin
   // + the unit ring's full[8] and empty[8]
   static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 9 + 2 * kUnitRing;
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
 };
+static_assert(QCfg<128>::kSmemBytes <= 227 * 1024 && QCfg<64>::kSmemBytes <= 227 * 1024,
+              "shared memory of the dQ kernel exceeds the 227 KB a CTA may use");
 
 struct QItem {
   int s, e, m, h, g, q0;  // key tiles 0..m
 };
 
-__device__ __forceinline__ QItem q_decode(const BwdParams& p, const UnitSpace& us, int w) {
+__device__ __forceinline__ QItem q_decode(const BwdParams& p, const UnitInfo& un) {
   QItem it;
-  int doc;
-  unit_decode(us, w, doc, it.m, it.h);
+  it.m = un.tile;
+  it.h = un.h;
   it.g = it.h / (p.Hq / p.Hkv);
-  it.s = p.cu[doc];
-  it.e = p.cu[doc + 1];
+  it.s = un.s;
+  it.e = un.e;
   it.q0 = it.s + 128 * it.m;
   return it;
 }
@@ -671,9 +677,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
       int unit_i = 0;
       bool ok = true;
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_produce(ring, p.sched.next, uk, wd);
+        const UnitInfo un = unit_produce(ring, us, p.cu, p.sched.next, uk, wd);
+        const int w = un.w;
         if (w < 0 || w >= n_units) break;
-        const QItem it = q_decode(p, us, w);
+        const QItem it = q_decode(p, un);
         if (unit_i > 0 && !mbar_wait(q_empty, (unit_i - 1) & 1, wd, 31)) break;
         mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
         for (int b = 0; b < C::kNumBox; ++b) {
@@ -710,9 +717,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
       int unit_i = 0;
       bool ok = true;
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_take(ring, uk, wd);
+        const UnitInfo un = unit_take(ring, uk, wd);
+        const int w = un.w;
         if (w < 0 || w >= n_units) break;
-        const QItem it = q_decode(p, us, w);
+        const QItem it = q_decode(p, un);
         if (!mbar_wait(q_full, unit_i & 1, wd, 33)) break;
         for (int v = 0; v <= it.m; ++v, ++kt) {
           // S and dP of key tile kt into their regions, each once the compute
@@ -757,9 +765,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
       int unit_i = 0;
       bool ok = true;
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_take(ring, uk, wd);
+        const UnitInfo un = unit_take(ring, uk, wd);
+        const int w = un.w;
         if (w < 0 || w >= n_units) break;
-        const QItem it = q_decode(p, us, w);
+        const QItem it = q_decode(p, un);
         for (int v = 0; v <= it.m; ++v, ++kt) {
           const int ks = kt % C::kKStages;
           if (v == 0 && unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 34)) { ok = false; break; }
@@ -788,9 +797,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
     int unit_i = 0;
     bool ok = true;
     for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-      const int w = unit_take_warp(ring, uk, wd);
+      const UnitInfo un = unit_take_warp(ring, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
-      const QItem it = q_decode(p, us, w);
+      const QItem it = q_decode(p, un);
       const int i = it.q0 + row;
       const bool valid = i < it.e;
       // rows past the document end (the tail of the last tile) get P = 0

@@ -201,7 +201,8 @@ constexpr int oBars = oSf + kNumSf * kSfBlk;
 //       acc_full, acc_free, fin
 // + the unit ring's full[8] and empty[8]
 constexpr int kNumBars = 2 + 2 * kStages + 9 + 2 * kUnitRing;
-constexpr int kSmem = oBars + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
+constexpr int kSmem = oBars + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
+static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may use");
 // TMEM: S and dP regions (each read out into registers and released at
 // once), dQ, scale factors
 constexpr uint32_t tS = 0, tDP = 128, tDQ = 256;
@@ -274,12 +275,13 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   const Watchdog wd{p.status, abort_flag, p.timeout_ns};
   const UnitSpace us = unit_space(p.sched, p.Hq, kSchedQ);
   const int n_units = us.n_units();
-  auto decode = [&](int w, int& doc, int& s, int& e, int& h, int& g, int& q0, int& n) {
-    int m;
-    unit_decode(us, w, doc, m, h);
+  auto decode = [&](const UnitInfo& un, int& doc, int& s, int& e, int& h, int& g, int& q0, int& n) {
+    const int m = un.tile;
+    doc = un.doc;
+    h = un.h;
     g = h / (p.Hq / p.Hkv);
-    s = p.cu[doc];
-    e = p.cu[doc + 1];
+    s = un.s;
+    e = un.e;
     q0 = s + 128 * m;
     n = m + 1;
   };
@@ -289,12 +291,11 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
     int unit_i = 0;
     bool ok = true;
     for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-      int w = 0;
-      if (lane == 0) w = unit_produce(ring, p.sched.next, uk, wd);
-      w = __shfl_sync(0xFFFFFFFFu, w, 0);
+      const UnitInfo un = unit_produce_warp(ring, us, p.cu, p.sched.next, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
       int doc, s, e, h, g, q0, n;
-      decode(w, doc, s, e, h, g, q0, n);
+      decode(un, doc, s, e, h, g, q0, n);
       if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 71)) break;
       reinterpret_cast<uint4*>(sfb(0))[lane] = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
       reinterpret_cast<uint4*>(sfb(1))[lane] = pt_rows(p.do_spt, q0, lane, p.T, p.Hq, h);
@@ -372,10 +373,11 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
           return true;
         };
         for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-          const int w = unit_take(ring, uk, wd);
+          const UnitInfo un = unit_take(ring, uk, wd);
+          const int w = un.w;
           if (w < 0 || w >= n_units) break;
           int doc, s, e, h, g, q0, n;
-          decode(w, doc, s, e, h, g, q0, n);
+          decode(un, doc, s, e, h, g, q0, n);
           if (!mbar_wait(q_full, unit_i & 1, wd, 76)) break;
           tc_fence_after();
           tmem_cp_sf(tmem + tSfQ, aSf + 0 * kSfBlk);
@@ -401,10 +403,11 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         // the stage and the unit's buffers are released here: the score MMAs
         // that also read them completed before the compute warps signalled dS~
         for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-          const int w = unit_take(ring, uk, wd);
+          const UnitInfo un = unit_take(ring, uk, wd);
+          const int w = un.w;
           if (w < 0 || w >= n_units) break;
           int doc, s, e, h, g, q0, n;
-          decode(w, doc, s, e, h, g, q0, n);
+          decode(un, doc, s, e, h, g, q0, n);
           if (!mbar_wait(q_full, unit_i & 1, wd, 101)) break;
           for (int v = 0; v < n; ++v, ++kt) {
             const int stg = kt % kStages;
@@ -460,10 +463,11 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       return true;
     };
     for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-      const int w = unit_take_warp(ring, uk, wd);
+      const UnitInfo un = unit_take_warp(ring, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
       int doc, s, e, h, g, q0, n;
-      decode(w, doc, s, e, h, g, q0, n);
+      decode(un, doc, s, e, h, g, q0, n);
       const int i = q0 + row;
       const bool valid = i < e;
       // rows past the document end get P = 0
@@ -566,7 +570,8 @@ constexpr int kQpt = 0, kDOpt = 1, kDOtb = 2, kQtb = 3;
 constexpr int bKvFull = 0, bKvEmpty = 1, bOpFull = 2, bOpEmpty = 6, bAuxFull = 10, bAuxEmpty = 12, bSFull = 14,
               bSFree = 15, bPFull = 16, bPEmpty = 17, bDsFull = 18, bDsEmpty = 19, bAccFull = 20, bAccFree = 21,
               bFin = 22, bRing = 23, kNumBars = 23 + 2 * kUnitRing;
-constexpr int kSmem = oBars + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
+constexpr int kSmem = oBars + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
+static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may use");
 // TMEM: one 128-column region that holds S^T and dP^T in turn (each read out
 // into registers and released before the next), dV, dK, scale factors
 constexpr uint32_t tSD = 0, tDV = 128, tDK = 256;
@@ -647,10 +652,12 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   const UnitSpace us = unit_space(p.sched, p.Hkv, kSchedKV);
   const int n_units = us.n_units();
   const int G = p.Hq / p.Hkv;
-  auto decode = [&](int w, int& doc, int& s, int& e, int& g, int& v, int& k0, int& nq) {
-    unit_decode(us, w, doc, v, g);
-    s = p.cu[doc];
-    e = p.cu[doc + 1];
+  auto decode = [&](const UnitInfo& un, int& doc, int& s, int& e, int& g, int& v, int& k0, int& nq) {
+    doc = un.doc;
+    v = un.tile;
+    g = un.h;
+    s = un.s;
+    e = un.e;
     k0 = s + 128 * v;
     nq = (e - s + 127) / 128;
   };
@@ -676,12 +683,11 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     int unit_i = 0;
     bool ok = true;
     for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-      int w = 0;
-      if (lane == 0) w = unit_produce(ring, p.sched.next, uk, wd);
-      w = __shfl_sync(0xFFFFFFFFu, w, 0);
+      const UnitInfo un = unit_produce_warp(ring, us, p.cu, p.sched.next, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
       int doc, s, e, g, v, k0, nq;
-      decode(w, doc, s, e, g, v, k0, nq);
+      decode(un, doc, s, e, g, v, k0, nq);
       if (unit_i > 0 && !warp_wait(kv_empty, (unit_i - 1) & 1, wd, 81)) break;
       reinterpret_cast<uint4*>(sfb(0))[lane] = tb_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
       reinterpret_cast<uint4*>(sfb(1))[lane] = pt_rows(p.k_spt, k0, lane, p.T, p.Hkv, g);
@@ -734,10 +740,11 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     uint32_t t = 0;
     bool ok = true;
     for (uint32_t uk = 0; ok; ++uk) {
-      const int w = unit_take_warp(ring, uk, wd);
+      const UnitInfo un = unit_take_warp(ring, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
       int doc, s, e, g, v, k0, nq;
-      decode(w, doc, s, e, g, v, k0, nq);
+      decode(un, doc, s, e, g, v, k0, nq);
       for (int h = g * G; h < (g + 1) * G && ok; ++h) {
         for (int m = v; m < nq; ++m, ++t) {
           const int q0 = s + 128 * m;
@@ -796,10 +803,11 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
         return true;
       };
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_take(ring, uk, wd);
+        const UnitInfo un = unit_take(ring, uk, wd);
+          const int w = un.w;
         if (w < 0 || w >= n_units) break;
         int doc, s, e, g, v, k0, nq;
-        decode(w, doc, s, e, g, v, k0, nq);
+        decode(un, doc, s, e, g, v, k0, nq);
         if (!mbar_wait(kv_full, unit_i & 1, wd, 89)) break;
         if (unit_i > 0 && !mbar_wait(acc_free, (unit_i - 1) & 1, wd, 90)) break;
         tc_fence_after();
@@ -892,10 +900,11 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
       return true;
     };
     for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-      const int w = unit_take_warp(ring, uk, wd);
+      const UnitInfo un = unit_take_warp(ring, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
       int doc, s, e, g, v, k0, nq;
-      decode(w, doc, s, e, g, v, k0, nq);
+      decode(un, doc, s, e, g, v, k0, nq);
       const int j = k0 + row;
       for (int h = g * G; h < (g + 1) * G && ok; ++h) {
         for (int m = v; m < nq; ++m, ++t) {

@@ -64,7 +64,7 @@ struct Cfg {
   // s_full[2], s_free[2], p_full[2], p_free[2], o_full[2], o_free[2], fin
   // + the unit ring's full[8] and empty[8]
   static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 12 + 1 + 2 * kUnitRing;
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
 };
 static_assert(Cfg<128>::kSmemBytes <= 227 * 1024 && Cfg<64>::kSmemBytes <= 227 * 1024,
               "shared memory of the forward exceeds the 227 KB a CTA may use");
@@ -88,13 +88,13 @@ struct Item {
   int s, e, u, h, g, q0, n0, n1, nkv;
 };
 
-__device__ __forceinline__ Item decode(const Params& p, const UnitSpace& us, int w) {
+__device__ __forceinline__ Item decode(const Params& p, const UnitInfo& un) {
   Item it;
-  int doc;
-  unit_decode(us, w, doc, it.u, it.h);
+  it.u = un.tile;
+  it.h = un.h;
   it.g = it.h / (p.Hq / p.Hkv);
-  it.s = p.cu[doc];
-  it.e = p.cu[doc + 1];
+  it.s = un.s;
+  it.e = un.e;
   it.q0 = it.s + 256 * it.u;
   it.n0 = 2 * it.u + 1;                               // key tiles 0..2u for query tile 0
   it.n1 = (it.q0 + 128 < it.e) ? 2 * it.u + 2 : 0;    // key tiles 0..2u+1 for query tile 1
@@ -207,9 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last_q_phase = -1;
       bool ok = true;
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_produce(ring, p.sched.next, uk, wd);
+        const UnitInfo un = unit_produce(ring, us, p.cu, p.sched.next, uk, wd);
+        const int w = un.w;
         if (w < 0 || w >= n_units) break;
-        const Item it = decode(p, us, w);
+        const Item it = decode(p, un);
         if (unit_i > 0 && !mbar_wait(q_empty, (unit_i - 1) & 1, wd, 1)) break;
         mbar_arrive_expect_tx(q_full, (it.n1 ? 2 : 1) * C::kTileBytes);
         last_q_phase = unit_i & 1;
@@ -239,9 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t vt = 0;
       bool ok = true;
       for (uint32_t uk = 0; ok; ++uk) {
-        const int w = unit_take(ring, uk, wd);
+        const UnitInfo un = unit_take(ring, uk, wd);
+        const int w = un.w;
         if (w < 0 || w >= n_units) break;
-        const Item it = decode(p, us, w);
+        const Item it = decode(p, un);
         for (int j = 0; j < it.nkv; ++j, ++vt) {
           const int slot = vt % C::kVStages;
           const uint32_t use = vt / C::kVStages;
@@ -325,9 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_take(ring, uk, wd);
+        const UnitInfo un = unit_take(ring, uk, wd);
+        const int w = un.w;
         if (w < 0 || w >= n_units) break;
-        const Item it = decode(p, us, w);
+        const Item it = decode(p, un);
         const int n = i ? it.n1 : it.n0;
         if (!mbar_wait(q_full, unit_i & 1, wd, 3)) break;
         if (!step_k(n > 0)) break;
@@ -359,9 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sw = row & 7;                            // 128-byte swizzle of the row
     uint32_t s_cnt = 0, p_cnt = 0, o_cnt = 0;
     for (uint32_t uk = 0;; ++uk) {
-      const int w = unit_take_warp(ring, uk, wd);
+      const UnitInfo un = unit_take_warp(ring, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
-      const Item it = decode(p, us, w);
+      const Item it = decode(p, un);
       const int n = wg ? it.n1 : it.n0;
       if (n == 0) continue;
       const int q_idx = it.q0 + 128 * wg + row;
@@ -457,11 +461,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = 1.f / l;
       const bool valid = q_idx < it.e;
       __nv_bfloat16* orow = p.o + ((size_t)q_idx * p.Hq + it.h) * D;
+      // the row of O in one batch of TMEM loads and one wait
+      uint32_t ot[D];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(o_addr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&ot[32 * c]));
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&ot[32 * c]));
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t t[32];
-        tmem_ld32(o_addr + 32 * c, t);
-        tmem_wait_ld(t);
+        const uint32_t* t = ot + 32 * c;
         uint32_t ob[16], rb[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {

@@ -69,7 +69,8 @@ constexpr int oLsum = oXmax + 2 * 4 * 128 * 4;       // partial row sums [4][128
 constexpr int oBars = oLsum + 4 * 128 * 4;
 // + one row-exchange barrier per row quarter, the unit ring's full[8] and empty[8]
 constexpr int kNumBars = 2 + 2 * kSlots + 8 + 4 + 2 * kUnitRing;
-constexpr int kSmemBytes = oBars + kNumBars * 8 + 16 + 4 * kUnitRing + 1024;
+constexpr int kSmemBytes = oBars + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may use");
 
 // TMEM columns
 constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256;
@@ -90,6 +91,7 @@ struct Params {
   int T, Hq, Hkv, n_docs;
   float scale_log2;
   int rule;
+  int wide;  // O and its residual 32-byte aligned: 32-byte stores
   unsigned long long* cta_times;  // per-CTA (start, end) records, or null
 };
 
@@ -97,13 +99,14 @@ struct Item {
   int doc, s, e, h, g, q0, n;  // n key tiles 0..n-1, tile n-1 is the diagonal
 };
 
-__device__ __forceinline__ Item decode(const Params& p, const UnitSpace& us, int w) {
+__device__ __forceinline__ Item decode(const Params& p, const UnitInfo& un) {
   Item it;
-  int m;
-  unit_decode(us, w, it.doc, m, it.h);
+  const int m = un.tile;
+  it.doc = un.doc;
+  it.h = un.h;
   it.g = it.h / (p.Hq / p.Hkv);
-  it.s = p.cu[it.doc];
-  it.e = p.cu[it.doc + 1];
+  it.s = un.s;
+  it.e = un.e;
   it.q0 = it.s + 128 * m;
   it.n = m + 1;
   return it;
@@ -211,11 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int unit_i = 0;
     bool ok = true;
     for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-      int w = 0;
-      if (lane == 0) w = unit_produce(ring, p.sched.next, uk, wd);
-      w = __shfl_sync(0xFFFFFFFFu, w, 0);
+      const UnitInfo un = unit_produce_warp(ring, us, p.cu, p.sched.next, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
-      const Item it = decode(p, us, w);
+      const Item it = decode(p, un);
       if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 51)) break;
       {
         // scale blocks: row r = lane + 32 r1 -> bytes 16 lane + 4 r1 .. +3
@@ -313,9 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(col, aring + ks * kCodeTile, kSfK);
       };
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
-        const int w = unit_take(ring, uk, wd);
+        const UnitInfo un = unit_take(ring, uk, wd);
+        const int w = un.w;
         if (w < 0 || w >= n_units) break;
-        const Item it = decode(p, us, w);
+        const Item it = decode(p, un);
         const int n = it.n;
         if (!mbar_wait(q_full, unit_i & 1, wd, 54)) break;
         tc_fence_after();
@@ -402,9 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_cnt[2] = {0, 0}, pv_cnt = 0, o_cnt = 0, tiles = 0;
     bool ok = true;
     for (uint32_t uk = 0; ok; ++uk) {
-      const int w = unit_take_warp(ring, uk, wd);
+      const UnitInfo un = unit_take_warp(ring, uk, wd);
+      const int w = un.w;
       if (w < 0 || w >= n_units) break;
-      const Item it = decode(p, us, w);
+      const Item it = decode(p, un);
       const int n = it.n;
       const int q_idx = it.q0 + row;
       float M = -INFINITY, l = 0.f;  // l: this thread's share of the row sum
@@ -533,12 +537,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           rb[e] = pack_bf16x2(f0 - __uint_as_float(ob[e] << 16), f1 - __uint_as_float(ob[e] & 0xFFFF0000u));
         }
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * wg);
-          uint4* rdst = reinterpret_cast<uint4*>(p.o_resid + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * wg);
+          __nv_bfloat16* orow = p.o + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * wg;
+          __nv_bfloat16* rrow = p.o_resid + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * wg;
+          if (p.wide) {
+            st_global_32B(orow, ob);
+            st_global_32B(orow + 16, ob + 8);
+            st_global_32B(rrow, rb);
+            st_global_32B(rrow + 16, rb + 8);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow);
+            uint4* rdst = reinterpret_cast<uint4*>(rrow);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
-            rdst[e] = make_uint4(rb[4 * e], rb[4 * e + 1], rb[4 * e + 2], rb[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) {
+              dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+              rdst[e] = make_uint4(rb[4 * e], rb[4 * e + 1], rb[4 * e + 2], rb[4 * e + 3]);
+            }
           }
         }
       }
@@ -584,6 +597,7 @@ cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
   p.n_docs = a.n_docs;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.rule = a.rule;
+  p.wide = aligned32(a.o) && aligned32(a.o_resid);
   const long long max_units = (long long)a.sched.max_items * a.Hq;
   const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
   fwd_mxfp8_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tktb, tkpt, tvtb, tvpt, p);
