@@ -427,14 +427,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(lane_base + (own ? ((j & 1) ? kS0 : kS1) : ((j & 1) ? kS1 : kS0)) + 32 * wg, r);
           tmem_wait_ld(r);
         }
+        // raw scores, -inf where not visible (masks only on the diagonal tile)
         float x[32];
-        float bmax = -INFINITY;
+        if (future) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const bool vis = !future && (!own || c <= lane);
-          x[c] = vis ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
-          bmax = fmaxf(bmax, x[c]);
+          for (int c = 0; c < 32; ++c) x[c] = -INFINITY;
+        } else if (own) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = c <= lane ? __uint_as_float(r[c]) : -INFINITY;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(r[c]);
         }
+        // block maximum of the raw scores (the scale is positive), in log2 units
+        float pm[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) pm[k] = fmaxf(x[k], x[4 + k]);
+#pragma unroll
+        for (int c = 8; c < 32; c += 8) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) pm[k] = fmax3(pm[k], x[c + k], x[c + 4 + k]);
+        }
+        const float bmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * p.scale_log2;
         float* xm = xmax + (tiles & 1) * 512;
         xm[wg * 128 + row] = bmax;
         if (!row_sync()) { ok = false; break; }
@@ -449,15 +463,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           M = Mn;
         }
         const bool any_rescale = __any_sync(0xFFFFFFFFu, alpha != 1.f) && j > 0;
-        // u = 2^(x - M), row sum before quantisation, MX quantisation of the block
-        float rs = 0.f, amax = 0.f;
+        // u = 2^(s scale log2(e) - M) with one FMA per element, a quarter of
+        // the exponentials on the FMA pipe; row sum before quantisation and
+        // block maximum of u in four partial chains each; MX quantisation of
+        // the block
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f}, am4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float nM = -M;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          x[c] = fast_exp2(x[c] - M);
-          rs += x[c];
-          amax = fmaxf(amax, x[c]);
+          const float arg = fmaf(x[c], p.scale_log2, nM);
+          x[c] = (c & 3) == 3 ? exp2_poly(arg) : fast_exp2(arg);
+          rs4[c & 3] += x[c];
+          am4[c & 3] = fmaxf(am4[c & 3], x[c]);
         }
-        l += rs;
+        const float amax = fmaxf(fmaxf(am4[0], am4[1]), fmaxf(am4[2], am4[3]));
+        l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         const int X = mx_block_exponent(amax, p.rule);
         const float sc = mx_pow2_neg(X < -126 ? -126 : X);
         uint32_t codes[8];
