@@ -410,10 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
           l *= alpha;
         }
-        // P = 2^(s scale log2(e) - m) with one FMA per element (all on MUFU:
-        // with two softmax warps per SM partition, moving a quarter of them to
-        // the FMA pipe cost more issue slots than it saved); row sum in four
-        // independent partial sums
+        // P = 2^(s scale log2(e) - m) with one FMA per element; row sum in
+        // four independent partial sums
         uint32_t pk[64];
         float rs[4] = {0.f, 0.f, 0.f, 0.f};
         const float nm = -m;

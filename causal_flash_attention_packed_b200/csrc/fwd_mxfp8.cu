@@ -463,16 +463,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           M = Mn;
         }
         const bool any_rescale = __any_sync(0xFFFFFFFFu, alpha != 1.f) && j > 0;
-        // u = 2^(s scale log2(e) - M) with one FMA per element, a quarter of
-        // the exponentials on the FMA pipe; row sum before quantisation and
-        // block maximum of u in four partial chains each; MX quantisation of
-        // the block
+        // u = 2^(s scale log2(e) - M) with one FMA per element; row sum
+        // before quantisation and block maximum of u in four partial chains
+        // each; MX quantisation of the block
         float rs4[4] = {0.f, 0.f, 0.f, 0.f}, am4[4] = {0.f, 0.f, 0.f, 0.f};
         const float nM = -M;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float arg = fmaf(x[c], p.scale_log2, nM);
-          x[c] = (c & 3) == 3 ? exp2_poly(arg) : fast_exp2(arg);
+          x[c] = fast_exp2(arg);
           rs4[c & 3] += x[c];
           am4[c & 3] = fmaxf(am4[c & 3], x[c]);
         }

@@ -357,27 +357,4 @@ __device__ __forceinline__ void store_row32(void* base, size_t elem_off, const u
   }
 }
 
-// 2^x on the FMA pipe, for spreading exponentials between the FMA pipe and
-// the MUFU unit (16 ex2 per cycle per SM; the MXFP8 forward, whose 16 softmax
-// warps leave issue slots free while MUFU is busy).  x = n + f with n the nearest
-// integer (reduction through the rounding constant 1.5 * 2^23, whose low
-// mantissa bits then hold n) and f in [-1/2, 1/2]; 2^f from a degree-3
-// polynomial fitted by Remez exchange for minimax relative error on
-// [-1/2, 1/2] (7.48e-5; the same bound holds for this fp32 evaluation, checked
-// on a dense grid of [-125, 8] by the tests); n is added to the exponent field.
-// Returns 0 for x < -125 (and -inf); x must stay below 2^22.
-constexpr float kExp2C0 = 0.9999280571937561f, kExp2C1 = 0.6932609677314758f,
-                kExp2C2 = 0.2426111251115799f, kExp2C3 = 0.0551716685295105f;
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -125.f);
-  const float t = xc + 12582912.f;
-  const float n = t - 12582912.f;
-  const float f = xc - n;
-  float p = fmaf(kExp2C3, f, kExp2C2);
-  p = fmaf(p, f, kExp2C1);
-  p = fmaf(p, f, kExp2C0);
-  const float r = __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-  return x < -125.f ? 0.f : r;
-}
-
 }  // namespace fapk
