@@ -46,18 +46,6 @@ struct Geo {
   static constexpr int kNumBox = D / 64;
 };
 
-// Bounded wait that ignores the abort flag (teardown: drain what is in flight).
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > budget_ns) return;
-  }
-}
-
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd, int where) {
-  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
-}
-
 // ---------------------------------------------------------------------------
 // 1. D = rowsum(dO * O), fp32 [Hq][T]
 // ---------------------------------------------------------------------------
@@ -133,7 +121,6 @@ struct BwdParams {
   int wide;  // every gradient output 32-byte aligned: 32-byte stores
   unsigned long long* cta_times;  // per-CTA (start, end) records, or null
 };
-
 
 // ---------------------------------------------------------------------------
 // 2. dK, dV

@@ -43,27 +43,6 @@ constexpr int kBf16 = 128 * 128 * 2;  // 128 rows x 128 bf16
 constexpr int kBox = 128 * 64 * 2;    // one 64-element bf16 box of 128 rows
 constexpr int kSfBlk = 512;
 
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > budget_ns) return;
-  }
-}
-
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd, int where) {
-  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
-}
-
-__device__ __forceinline__ uint32_t pt_word(const uint8_t* spt, int t, int T, int H, int h) {
-  return t < T ? __ldg(reinterpret_cast<const uint32_t*>(spt + ((size_t)t * H + h) * 4)) : 0x7F7F7F7Fu;
-}
-
-__device__ __forceinline__ uint32_t tb_word(const uint8_t* stb, int s, int e, int doc, int blk, int H, int g) {
-  if (32 * blk >= e - s) return 0x7F7F7F7Fu;
-  const size_t slot = (size_t)(s >> 5) + doc + blk;
-  return __ldg(reinterpret_cast<const uint32_t*>(stb + (slot * H + g) * 4));
-}
-
 // Scale block of an MN-major operand whose rows are the 128 channels and
 // whose K blocks are the token blocks blk0..blk0+3 (token-block form): byte
 // kb of the word of channel row (lane + 32 r1) is the scale of (block
@@ -180,7 +159,6 @@ struct MxParams {
   int rule;
   unsigned long long* cta_times;  // per-CTA (start, end) records, or null
 };
-
 
 // ---------------------------------------------------------------------------
 // dQ

@@ -115,14 +115,6 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
   tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&r[96]));
 }
 
-// Bounded wait that ignores the abort flag (teardown: drain what is in flight).
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > budget_ns) return;
-  }
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,

@@ -112,31 +112,6 @@ __device__ __forceinline__ Item decode(const Params& p, const UnitInfo& un) {
   return it;
 }
 
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > budget_ns) return;
-  }
-}
-
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd, int where) {
-  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
-}
-
-// 4 scale bytes of token t (per-token form), or the neutral byte 127 (2^0)
-// past the end of the tensor.
-__device__ __forceinline__ uint32_t pt_word(const uint8_t* spt, int t, int T, int H, int h) {
-  return t < T ? __ldg(reinterpret_cast<const uint32_t*>(spt + ((size_t)t * H + h) * 4)) : 0x7F7F7F7Fu;
-}
-
-// 4 scale bytes of document-local token block `blk` of document `doc`
-// (token-block form); 127s past the document's last block.
-__device__ __forceinline__ uint32_t tb_word(const uint8_t* stb, int s, int e, int doc, int blk, int H, int g) {
-  if (32 * blk >= e - s) return 0x7F7F7F7Fu;
-  const size_t slot = (size_t)(s >> 5) + doc + blk;
-  return __ldg(reinterpret_cast<const uint32_t*>(stb + (slot * H + g) * 4));
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_mxfp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ktb,
                      const __grid_constant__ CUtensorMap tm_kpt, const __grid_constant__ CUtensorMap tm_vtb,

@@ -101,4 +101,18 @@ __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint32_t smem_block) 
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
 
+// 4 scale bytes of token t (per-token form), or the neutral byte 127 (2^0)
+// past the end of the tensor.
+__device__ __forceinline__ uint32_t pt_word(const uint8_t* spt, int t, int T, int H, int h) {
+  return t < T ? __ldg(reinterpret_cast<const uint32_t*>(spt + ((size_t)t * H + h) * 4)) : 0x7F7F7F7Fu;
+}
+
+// 4 scale bytes of document-local token block `blk` of document `doc`
+// (token-block form); 127s past the document's last block.
+__device__ __forceinline__ uint32_t tb_word(const uint8_t* stb, int s, int e, int doc, int blk, int H, int g) {
+  if (32 * blk >= e - s) return 0x7F7F7F7Fu;
+  const size_t slot = (size_t)(s >> 5) + doc + blk;
+  return __ldg(reinterpret_cast<const uint32_t*>(stb + (slot * H + g) * 4));
+}
+
 }  // namespace fapk

@@ -357,4 +357,18 @@ __device__ __forceinline__ void store_row32(void* base, size_t elem_off, const u
   }
 }
 
+// Bounded wait that ignores the abort flag (teardown: let what is in flight
+// land before the CTA exits).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > budget_ns) return;
+  }
+}
+
+// A whole warp waits; false for every lane if any lane's wait gave up.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Watchdog& wd, int where) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, wd, where));
+}
+
 }  // namespace fapk
