@@ -27,7 +27,7 @@
  *           a running max/sum reaches exactly the softmax result.  The oracle
  *           does NOT tile: it materialises one score row per query.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent (the choices this oracle makes):
  *  - packed documents: token i of document k=[s_k,e_k) sees keys j with
  *    s_k <= j <= i only; cu_seqlens gives s_k = cu[k], e_k = cu[k+1].
  *  - GQA: query head h reads KV head h / (Hq/Hkv).
