@@ -482,7 +482,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           // ---- dS = P (dP - D)
           float y[32];
           if (!take(y)) { ok = false; break; }
-          float dmax = 0.f;
+          float dm[4] = {0.f, 0.f, 0.f, 0.f};  // range check in four partial chains
           uint32_t dk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
@@ -494,9 +494,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           }
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            dmax = fmaxf(dmax, fmaxf(fabsf(y[2 * c]), fabsf(y[2 * c + 1])));
+            dm[c & 3] = fmaxf(dm[c & 3], fmaxf(fabsf(y[2 * c]), fabsf(y[2 * c + 1])));
             dk[c] = pack_f16x2(y[2 * c], y[2 * c + 1]);
           }
+          const float dmax = fmaxf(fmaxf(dm[0], dm[1]), fmaxf(dm[2], dm[3]));
           if (!(dmax < kF16Max)) record_error(p.status, kStatusRange, 42);
           warp_arrive(o_empty + os);  // done with this tile's -LSE log2(e) and D
           if (t > 0 && !warp_wait(dk_done, (t - 1) & 1, wd, 33)) { ok = false; break; }
@@ -808,7 +809,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const int j0 = it.s + 128 * v + 32 * wg;  // key index of this thread's column 0
         const bool diag = v == it.m;
         uint32_t dk[16];
-        float dmax = 0.f;
+        float dm[4] = {0.f, 0.f, 0.f, 0.f};  // range check in four partial chains
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           float dv[2];
@@ -818,10 +819,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
             float pp = fast_exp2(fmaf(x[cc], p.scale_log2, nl2));
             if (diag && j0 + cc > i) pp = 0.f;
             dv[u] = pp * (y[cc] - dl);
-            dmax = fmaxf(dmax, fabsf(dv[u]));
+            dm[(c / 2) & 3] = fmaxf(dm[(c / 2) & 3], fabsf(dv[u]));
           }
           dk[c / 2] = pack_f16x2(dv[0], dv[1]);
         }
+        const float dmax = fmaxf(fmaxf(dm[0], dm[1]), fmaxf(dm[2], dm[3]));
         if (!(dmax < kF16Max)) record_error(p.status, kStatusRange, 43);
         if (kt > 0 && !warp_wait(dq_done, (kt - 1) & 1, wd, 41)) { ok = false; break; }
         tc_fence_after();
