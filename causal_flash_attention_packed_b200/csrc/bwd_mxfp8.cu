@@ -547,7 +547,7 @@ constexpr int oBars = oSf + kNumSf * kSfBlk;
 constexpr int kQpt = 0, kDOpt = 1, kDOtb = 2, kQtb = 3;
 constexpr int bKvFull = 0, bKvEmpty = 1, bOpFull = 2, bOpEmpty = 6, bAuxFull = 10, bAuxEmpty = 12, bSFull = 14,
               bSFree = 15, bPFull = 16, bPEmpty = 17, bDsFull = 18, bDsEmpty = 19, bAccFull = 20, bAccFree = 21,
-              bFin = 22, bRing = 23, kNumBars = 23 + 2 * kUnitRing;
+              bFin = 22, bRing = 23, kNumBars = bRing + 2 * kUnitRing;  // the unit ring's full[], empty[] from bRing
 constexpr int kSmem = oBars + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
 static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may use");
 // TMEM: one 128-column region that holds S^T and dP^T in turn (each read out
