@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers with bounded waits, TMA
-// tile loads (no cluster multicast anywhere in this library), tcgen05 tensor
+// tile loads (each into the issuing CTA's own shared memory only), tcgen05 tensor
 // memory allocation, MMA, commit, loads and stores, and the shared-memory
 // matrix / instruction descriptors of the 5th-generation tensor cores.
 #pragma once
@@ -100,7 +100,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 // ---------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), CTA-local destinations, no multicast.
+// TMA (cp.async.bulk.tensor) into the issuing CTA's own shared memory.
 // The innermost coordinate of every load here is a channel offset that is a
 // multiple of 64 elements (128 bytes), so it always meets the 16-byte rule.
 // ---------------------------------------------------------------------------
