@@ -43,10 +43,27 @@ def load_peaks():
         with open(path) as f:
             pk = json.load(f)
         return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
-                "bf16_tflops_sustained": pk["bf16_tflops_sustained"], "source": "measured"}
+                "bf16_tflops_sustained": pk["bf16_tflops_sustained"],
+                "sm_max_mhz": float(pk.get("sm_max_mhz", 1965.0)), "source": "measured"}
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-                "source": "fallback"}
+                "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def tensor_peak(peaks, clk, fp8: bool):
+    """Tensor denominator for a kernel timed in a short region: the measured
+    burst bf16 GEMM peak (taken at the maximum SM clock), scaled to the median
+    SM clock sampled during the timed region, times the nominal FP8/bf16 ratio
+    of 2 for the MXFP8 path.  Returns (peak TFLOP/s, description)."""
+    mhz = clk.get("sm_mhz") if clk else None
+    top = peaks["sm_max_mhz"]
+    f = min(1.0, mhz / top) if mhz else 1.0
+    base = peaks["bf16_tflops"] * f
+    desc = (f"{peaks['source']} bf16 burst GEMM peak {peaks['bf16_tflops']:.1f} TFLOP/s (MEASURED_PEAKS.json) "
+            f"x median SM clock {mhz if mhz else 'unknown'} / {top:.0f} MHz")
+    if fp8:
+        return 2.0 * base, "2 x " + desc + " (nominal FP8/bf16 ratio; no FP8 GEMM measured)"
+    return base, desc
 
 
 class ClockSampler:
@@ -173,8 +190,6 @@ def run_reference(args, w, world, rank):
     vals = []
     text = ""
     cores = len(os.sched_getaffinity(0))
-    for _ in range(args.warmup if args.warmup < 1 else 1):
-        pass
     for _ in range(args.steps):
         v, cores, text, _ = cpu_oracle_sample(w, target_s=args.ref_seconds)
         vals.append(v)
@@ -336,7 +351,7 @@ def analytic_balance(w, prec, num_sms):
             "dq_kernel": ratio(units(128, w.Hq, lambda k, nt, r: nt - r))}
 
 
-def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, config=None):
+def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, clk, config=None):
     flops = w.flops()
     value = flops * world / (ms_per_step * 1e-3) / 1e12
     pairs = w.pairs()
@@ -346,18 +361,14 @@ def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, config=No
     dom = max(KERNEL_FLOPS, key=lambda n: kern_ms[n])
     dom_flops = KERNEL_FLOPS[dom] * w.d * w.Hq * pairs
     achieved = dom_flops / (kern_ms[dom] * 1e-3) / 1e12
-    if prec == "bf16":
-        peak, peak_src, dense = peaks["bf16_tflops_sustained"], \
-            f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)", DENSE_BF16_TFLOPS
-    else:
-        # no FP8 GEMM is measured on this machine: the measured bf16 sustained
-        # peak times the nominal FP8/bf16 ratio of 2
-        peak, peak_src, dense = 2.0 * peaks["bf16_tflops_sustained"], \
-            f"2 x {peaks['source']} bf16 sustained (MEASURED_PEAKS.json), nominal FP8/bf16 ratio", DENSE_FP8_TFLOPS
+    peak, peak_src = tensor_peak(peaks, clk, prec != "bf16")
+    dense = DENSE_BF16_TFLOPS if prec == "bf16" else DENSE_FP8_TFLOPS
     traffic = MEASURED_TRAFFIC.get(config, {}).get(prec, {}).get(dom)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic, "traffic_unit": "bytes per launch",
                 "kernel": dom, "peak_source": peak_src,
+                "sm_mhz_median": clk.get("sm_mhz") if clk else None,
+                "frac_of_dense_datasheet": achieved / dense,
                 "kernels_ms": kern_ms,
                 "kernels_tflops": {n: KERNEL_FLOPS[n] * w.d * w.Hq * pairs / (kern_ms[n] * 1e-3) / 1e12
                                    for n in KERNEL_FLOPS},
@@ -366,15 +377,15 @@ def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, config=No
     out = {"value": value, "ms_per_step": ms_per_step, "pct_of_dense_peak": 100.0 * (value / world) / dense,
            "dense_peak_tflops": dense, "roofline": roofline, "gpu_launches": launches}
     if prec == "mxfp8":
-        # quantize launches of the forward (HBM bound): per element 2 B read,
-        # two code forms (2 B), a per-token scale per 32 channels (1/32 B) and
-        # a token-block scale per 32 x 32 (1/1024 B) written; K and V also
-        # write their per-token dequantised copy (2 B)
-        qbytes = (w.T * w.Hq * w.d * (4.0 + 1.0 / 32 + 1.0 / 1024)
-                  + 2 * w.T * w.Hkv * w.d * (6.0 + 1.0 / 32 + 1.0 / 1024))
+        # quantize launches of the forward (HBM bound), algorithmic bytes per
+        # element: 2 B bf16 read, then per form 1 B of E4M3 codes and 1/32 B of
+        # scales written (two forms); extra copies a kernel writes for its own
+        # use are not counted
+        qbytes = (w.T * w.Hq * w.d + 2 * w.T * w.Hkv * w.d) * (2.0 + 2 * (1.0 + 1.0 / 32))
         gbs = qbytes / (kern_ms["quantize_qkv"] * 1e-3) / 1e9
         out["roofline_quantize"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                                    "algorithmic_bytes": qbytes,
                                     "kernel": "quantize_mxfp8_kernel (Q, K, V; both forms)"}
     return out
 
@@ -418,11 +429,11 @@ def main():
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-    results = {}
+    timed = {}
     for p in paths:
-        ms, kern_ms, launches = runners[p].timed(args.steps, args.warmup, world)
-        results[p] = path_report(w, p, ms, kern_ms, launches, world, peaks, config=args.config)
+        timed[p] = runners[p].timed(args.steps, args.warmup, world)
     clk = clocks.stop() if clocks else None
+    results = {p: path_report(w, p, *timed[p], world, peaks, clk, config=args.config) for p in paths}
     st_ok = all(r.status_ok() for r in runners.values())
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     balance = {p: runners[p].balance(num_sms) for p in paths}
@@ -434,7 +445,7 @@ def main():
     if args.e2e_steps > 0:
         R = runners[main_path]
         hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
-        outs = (R.o, R.dq, R.dk, R.dv)
+        outs = (R.o, R.lse, R.dq, R.dk, R.dv)
         houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
         d2h = sum(t.numel() * t.element_size() for t in houts)

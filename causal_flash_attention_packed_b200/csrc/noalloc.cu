@@ -2,22 +2,28 @@
 //
 // Some callers cannot obtain device memory at the point where they run the
 // forward: a plugin that is handed its input and output buffers by a host
-// framework and must not allocate behind its back, code that runs inside a
-// host callback where CUDA API calls that allocate are not allowed, or an
-// embedded runtime that reserves all device memory at start-up.  For them the
-// forward's scratch (the device status word and the scheduler's work list)
-// lives in a fixed array compiled into the library.  Inputs, outputs and the
-// saved-state buffer ctx are still the caller's.
+// framework and must not allocate behind its back, or an embedded runtime
+// that reserves all device memory at start-up.  For them the forward's
+// scratch (the device status word and the scheduler's work list) lives in a
+// fixed array compiled into the library.  Inputs, outputs and the saved-state
+// buffer ctx are still the caller's.  These entry points make CUDA runtime
+// calls (device query, symbol lookup, kernel launches), so, like any CUDA
+// call, they must not be made from inside a stream callback
+// (cudaLaunchHostFunc / cudaStreamAddCallback).
 //
 // The array is file-scope device memory: every GPU that loads the library
-// holds its kNoAllocScratchBytes until the process exits.  Host code may not
-// hand the array's name to a kernel (on the host that name is only a
-// stand-in, not a device address); the device address is looked up once per
-// device with cudaGetSymbolAddress, with that device current, and cached.
-// Every call shares the one array and leaves its contents behind; the
-// forward's scheduler clears the status word and its counters at the start of
-// each call, and calls whose GPU work overlaps (other streams, other host
-// threads) race on the array.
+// holds its kNoAllocScratchBytes until the process exits.  With CUDA's lazy
+// module loading (the default) that memory is taken when this file's module
+// is first loaded on a device, which happens at the first cudaGetSymbolAddress
+// below, i.e. during the first call on that device: make that first call
+// before reserving the rest of the device's memory, and before any stream
+// capture.  Host code may not hand the array's name to a kernel (on the host
+// that name is only a stand-in, not a device address); the device address is
+// looked up once per device with cudaGetSymbolAddress, with that device
+// current, and cached.  Every call shares the one array and leaves its
+// contents behind; the forward's scheduler clears the status word and its
+// counters at the start of each call, and calls whose GPU work overlaps (other
+// streams, other host threads) race on the array.
 #include <mutex>
 
 #include "internal.h"
@@ -61,6 +67,13 @@ int fapk_attn_fwd_noalloc(const fapk_problem_t* prob, const void* q, const void*
   void* ws = scratch_address();
   if (!ws) return FAPK_ERR_CUDA;
   return fapk_attn_fwd(prob, q, k, v, o, lse, ctx, ws, kNoAllocScratchBytes, stream);
+}
+
+int fapk_noalloc_status(void* stream) {
+  void* ws = scratch_address();
+  if (!ws) return FAPK_ERR_CUDA;
+  // the status word sits at the start of the forward's workspace
+  return fapk_status(ws, stream);
 }
 
 }  // extern "C"

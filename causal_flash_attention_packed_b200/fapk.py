@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
     L.fapk_attn_bwd.restype = i
     L.fapk_attn_fwd_noalloc.argtypes = [PP, vp, vp, vp, vp, vp, vp, vp]
     L.fapk_attn_fwd_noalloc.restype = i
+    L.fapk_noalloc_status.argtypes = [vp]
+    L.fapk_noalloc_status.restype = i
     L.fapk_quantize_mxfp8.argtypes = [vp, i, i, i, vp, vp, i, i, i, vp, vp, vp, vp, vp]
     L.fapk_quantize_mxfp8.restype = i
     L.fapk_status.argtypes = [vp, vp]
@@ -301,3 +303,9 @@ def cta_times(P: Problem, which: int, kernel: int, ws: torch.Tensor, stream=None
 def status(ws: torch.Tensor, stream=None) -> int:
     """fapk_status: synchronises the stream and returns the device status word."""
     return int(lib().fapk_status(_ptr(ws), _stream(stream)))
+
+
+def noalloc_status(stream=None) -> int:
+    """fapk_noalloc_status: synchronises the stream and returns the status word
+    of the last fapk_attn_fwd_noalloc call on the current device."""
+    return int(lib().fapk_noalloc_status(_stream(stream)))

@@ -198,23 +198,35 @@ FAPK_API int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const 
 /* Forward that allocates nothing.  The pages have no counterpart: this entry
  * point exists for callers that cannot obtain device memory where they run the
  * forward -- a plugin handed its buffers by a host framework that must not
- * allocate on its own, code inside a host callback, or a runtime that reserves
- * all device memory at start-up.  Same arguments and results as
- * fapk_attn_fwd minus the workspace: inputs, outputs and ctx are still the
- * caller's, and the forward's scratch (status word and work list) is a 1 MiB
- * array of device memory inside the library, which every GPU that loads the
- * library holds until the process exits.
+ * allocate on its own, or a runtime that reserves all device memory at
+ * start-up.  Same arguments and results as fapk_attn_fwd minus the workspace:
+ * inputs, outputs and ctx are still the caller's, and the forward's scratch
+ * (status word and work list) is a 1 MiB array of device memory inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.
  *  - A problem whose forward workspace (fapk_workspace_size(prob, FAPK_FWD))
- *    exceeds 1 MiB is rejected with FAPK_ERR_WORKSPACE_TOO_SMALL; at T = 32768
- *    tokens that size is about 1 KiB plus 8 bytes per document.
+ *    exceeds 1 MiB is rejected with FAPK_ERR_WORKSPACE_TOO_SMALL.  That size
+ *    is about 17 KiB, plus 12 bytes per ceil(max_seqlen / 128) and 8 bytes
+ *    per document: at most about 128 800 documents fit.
  *  - The first call on a device looks up the array's device address with that
- *    device current; make that first call before any stream capture.
+ *    device current; under CUDA's lazy module loading (the default) this is
+ *    also when the array's 1 MiB is taken on that device.  Make that first
+ *    call before any stream capture and before reserving the rest of the
+ *    device's memory.
+ *  - It makes CUDA runtime calls, so it must not be called from inside a
+ *    stream callback (cudaLaunchHostFunc / cudaStreamAddCallback).
  *  - All calls share the array and it keeps the last call's contents; each
  *    call clears the status word and counters it uses when it starts.  Calls
  *    whose GPU work overlaps (different streams or host threads) race on it.
- *  - The device status word of these calls is not readable by the caller. */
+ *  - The device status word is read with fapk_noalloc_status. */
 FAPK_API int fapk_attn_fwd_noalloc(const fapk_problem_t* prob, const void* q, const void* k,
                                    const void* v, void* o, float* lse, void* ctx, void* stream);
+
+/* Device status word of the last fapk_attn_fwd_noalloc call on the current
+ * device: synchronises `stream`, then returns FAPK_OK, FAPK_ERR_DEVICE_TIMEOUT
+ * or FAPK_ERR_BAD_SEQLENS as fapk_status does for a workspace, or
+ * FAPK_ERR_CUDA if the stream reported an error.  Allocates nothing. */
+FAPK_API int fapk_noalloc_status(void* stream);
 
 /* Scheduler balance (the pages have no counterpart): after a call made with
  * FAPK_FLAG_CTA_TIMES on workspace `ws` and problem `prob`, synchronises

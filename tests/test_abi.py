@@ -115,3 +115,25 @@ def test_quantize_validation(L):
     cu = np.array([0, 10, 60], np.int32)
     assert q(x, 64, 2, 64, 16, cu.ctypes.data, 2, 2, 0, None, None, 256, 256, None) == fapk.ERR_BAD_SEQLENS
     assert q(x, 0, 2, 64, None, None, 0, 3, 0, None, None, None, None, None) == fapk.OK
+
+
+@pytest.mark.parametrize("prec,rows", [(fapk.BF16, 256), (fapk.MXFP8, 128)])
+def test_noalloc_size_limit_matches_its_documented_formula(L, prec, rows):
+    """The forward workspace that the no-allocation entry point must fit in its
+    1 MiB array is about 17 KiB + 12 B per ceil(max_seqlen/128) + 8 B per
+    document (as documented): checked here against the library's own sizing,
+    and the limit of about 128 800 documents of one token each."""
+    for T, nd, ml in ((32768, 14, 7545), (131072, 30, 65536), (200000, 200000, 1)):
+        P = _problem(T=T, n_docs=nd, max_seqlen=ml, prec=prec)
+        ws = fapk.workspace_size(P, fapk.FWD)
+        levels = -(-ml // rows)
+        est = 17 * 1024 + 12 * levels + 8 * nd
+        assert abs(ws - est) <= 2048, (T, nd, ml, ws, est)
+    limit = 1 << 20
+    fits = [n for n in (128000, 128800, 129000)
+            if fapk.workspace_size(_problem(T=n, n_docs=n, max_seqlen=1, prec=prec), fapk.FWD) <= limit]
+    assert fits == [128000, 128800]
+    big = _problem(T=200000, n_docs=200000, max_seqlen=1, prec=prec)
+    # rejected on the host, before any CUDA call (dummy aligned pointers)
+    assert L.fapk_attn_fwd_noalloc(ctypes.byref(big), 256, 256, 256, 256, 256, 256, None) == \
+        fapk.ERR_WORKSPACE_TOO_SMALL
