@@ -36,9 +36,13 @@ def _rank_main(rank, world, port, out_dir):
         bench.barrier(world)
         got = bench.max_over_ranks(local_ms, world, dev)
         w = W.config(1, 0)
-        peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 900.0, "hbm_gbs": 6000.0, "source": "measured"}
+        peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 900.0, "hbm_gbs": 6000.0, "sm_max_mhz": 2000.0,
+                 "source": "measured"}
+        clk = {"sm_mhz": 1500.0}
         rep = bench.path_report(w, "bf16", got, {n: 1.0 for n in bench.KERNELS["bf16"][0] + bench.KERNELS["bf16"][1]},
-                                9, world, peaks, config=1)
+                                9, world, peaks, clk, config=1)
+        # the tensor denominator is the burst peak scaled to the sampled clock
+        assert abs(rep["roofline"]["peak"] - 750.0) < 1e-9
         bench.barrier(world)
         with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
             json.dump({"max_ms": got, "value": rep["value"], "flops": w.flops()}, f)
