@@ -12,10 +12,11 @@ the readings taken where the pages are silent.  Arrays are numpy float64 in the
 layouts of the C-ABI: Q/O/dO ``[T, Hq, d]``, K/V ``[T, Hkv, d]``, LSE
 ``[Hq, T]``, ``cu_seqlens`` int32 ``[n_docs + 1]``.
 
-The MXFP8 emulation (``mx_attn_fwd`` / ``mx_attn_bwd``) is pinned only by
-properties (its exact limit on on-grid inputs, its cosine to the exact path,
-the leak tests run on it and a hand-checked operand selection); beyond those,
-its element-level parity is unpinned.
+The MXFP8 emulation (``mx_attn_fwd`` / ``mx_attn_bwd``) is pinned by its
+exact limit on on-grid inputs, its cosine to the exact path, the leak tests run
+on it, hand-derived cases of the operand selection (forward and backward) and
+of the forward's P~, and element-by-element read-outs of the blocks in which
+dS~, P~T and dS~T are quantised (tests/test_oracle_mx*.py).
 """
 from __future__ import annotations
 

@@ -35,11 +35,16 @@
  *  - backward = analytic derivative (the pages give no formulas):
  *    D_i = dO_i . O_i, dP_ij = dO_i . V_j, dS_ij = P_ij (dP_ij - D_i),
  *    dQ_i = s sum_j dS_ij K_j, dK_j = s sum_i dS_ij Q_i, dV_j = sum_i P_ij dO_i.
- *  - MXFP8: E4M3 element codes, E8M0 shared scale per 32 elements, scale
- *    exponent X = clamp(floor(log2 amax) - 8, -127, 127) (X = -127 for an
- *    all-zero block), element code = RNE(x * 2^-X) saturated to +-448, scale
- *    byte X + 127.  (Block size and formats from the benchmark spec, the
- *    exponent rule from the OCP Microscaling v1.0 definition.)
+ *  - MXFP8: E4M3 element codes, E8M0 shared scale per 32 elements, element
+ *    code = RNE(x * 2^-X) saturated to +-448, scale byte X + 127.  Scale
+ *    exponent (block_exponent below), clamped to [-127, 127], X = -127 for an
+ *    all-zero block:
+ *      RULE_RCEIL (the default): X = ceil(log2(amax / 448)), the smallest
+ *        exponent at which the block maximum does not saturate;
+ *      RULE_OCP (flag MX_RULE_OCP): X = floor(log2 amax) - 8, the OCP
+ *        Microscaling v1.0 rule, under which block maxima whose significand
+ *        exceeds 1.75 saturate to 448.
+ *    (Block size and formats from the benchmark spec.)
  *  - token blocks are document-local: block m of document k covers tokens
  *    [s_k + 32m, min(s_k + 32m + 32, e_k)); its scale lives in slot
  *    floor(s_k/32) + k + m of a [T/32 + n_docs] slot array.
@@ -61,7 +66,11 @@
  * document, packing and permutation invariance, central finite differences
  * of the backward, brute force of the quantiser over every finite bf16 value,
  * the E4M3 round trip, worked quantiser values, the MXFP8 emulation's
- * exact limit, its cosine to the exact path and the leak properties.
+ * exact limit, its cosine to the exact path and the leak properties; the
+ * forward P~ of a hand-derived row and its independence of the integer
+ * reference; the blocks of dS~, P~T and dS~T read out element by element
+ * (document-local, along the contraction); the operand forms of dP (dO per
+ * token) and of dK, dV (Q, dO in token-block form) in hand-derived cases.
  */
 #include <algorithm>
 #include <cfenv>
