@@ -66,6 +66,9 @@ int validate_problem(const fapk_problem_t* P) {
   if (P->Hq % P->Hkv != 0) return FAPK_ERR_UNSUPPORTED;
   if (P->prec != FAPK_BF16 && P->prec != FAPK_MXFP8) return FAPK_ERR_UNSUPPORTED;
   if (P->scale_rule != FAPK_SCALE_RCEIL && P->scale_rule != FAPK_SCALE_OCP) return FAPK_ERR_UNSUPPORTED;
+  // the attention path quantises with RCEIL only: under OCP the computed
+  // operands quantise discontinuously near powers of two (see fapk.h)
+  if (P->prec == FAPK_MXFP8 && P->scale_rule != FAPK_SCALE_RCEIL) return FAPK_ERR_UNSUPPORTED;
   if (P->grad_dtype != FAPK_GRAD_F32 && P->grad_dtype != FAPK_GRAD_BF16) return FAPK_ERR_UNSUPPORTED;
   if (!std::isfinite(P->scale)) return FAPK_ERR_INVALID_ARG;
   if (P->T > 0) {

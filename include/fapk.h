@@ -92,7 +92,13 @@ typedef enum { FAPK_GRAD_F32 = 0, FAPK_GRAD_BF16 = 1 } fapk_grad_dtype_t;
  *  FAPK_SCALE_OCP: X = floor(log2(amax)) - 8 (OCP Microscaling v1.0);
  *    block maxima whose mantissa exceeds 1.75 saturate to 448.
  * Both clamp X to [-127, 127]; an all-zero block takes X = -127.  The scale
- * byte is X + 127. */
+ * byte is X + 127.  fapk_quantize_mxfp8 takes either rule.  The MXFP8
+ * attention path takes RCEIL only (FAPK_ERR_UNSUPPORTED otherwise): under
+ * OCP a computed P or dS block whose maximum lies just below a power of two
+ * saturates (up to 12.5% error) while one just above does not, so the
+ * gradients jump with tiny changes of P (a 1e-6 relative change of P moved
+ * dV by 2.8% in a measured case), and OCP is further from exact fp64 than
+ * RCEIL on every output. */
 typedef enum { FAPK_SCALE_RCEIL = 0, FAPK_SCALE_OCP = 1 } fapk_scale_rule_t;
 
 /* Which pass a workspace is sized for. */

@@ -33,6 +33,11 @@ _lib = None
 
 MX_QUANT_P = 1   # quantise the computed P and dS operands (the method's rule)
 MX_RULE_OCP = 2  # use the OCP floor(log2 amax) - 8 scale rule instead of RCEIL
+# accuracy-study switches (each takes one quantisation out of the emulation)
+MX_KEEP_INPUTS = 4   # Q, K, V, dO unquantised
+MX_KEEP_P = 8        # P~ and P~T unquantised
+MX_KEEP_DS = 16      # dS~ and dS~T unquantised
+MX_SYM_GUARD = 32    # Q and dO per token on the diagonal query block of dK and dV
 RULE_RCEIL = 0   # scale exponent X = ceil(log2(amax / 448)): never saturates
 RULE_OCP = 1     # scale exponent X = floor(log2 amax) - 8: may saturate to 448
 

@@ -275,11 +275,17 @@ uint8_t quant_block(const double* x, int n, size_t stride, uint8_t* codes, size_
 }
 
 /* Token-block (tb) and per-token (pt) dequantised forms of one (document,
- * head) slice, row-major [L][d] in doc-local token order. */
+ * head) slice, row-major [L][d] in doc-local token order.  With `exact` (an
+ * accuracy-study switch) both forms are the unquantised values. */
 void mx_forms(const double* x, int s, int L, int h, int H, int d, int rule,
-              std::vector<double>& tb, std::vector<double>& pt) {
+              std::vector<double>& tb, std::vector<double>& pt, bool exact = false) {
   std::vector<double> xs;
   slice_n(x, s, L, h, H, d, xs);
+  if (exact) {
+    tb = xs;
+    pt = xs;
+    return;
+  }
   tb.assign((size_t)L * d, 0.0);
   pt.assign((size_t)L * d, 0.0);
   for (int j = 0; j < L; ++j)
@@ -319,12 +325,20 @@ void quant_along(std::vector<double>& p, int n, bool on, int rule) {
   }
 }
 
-/* flags of the MXFP8 emulation */
+/* flags of the MXFP8 emulation.  MX_QUANT_P is the method; the others are
+ * accuracy-study switches that each take one quantisation out (or, for
+ * MX_SYM_GUARD, apply the per-token guard to the query side of dK and dV). */
 enum {
-  MX_QUANT_P = 1,  // quantise the computed P and dS operands (the method's rule)
-  MX_RULE_OCP = 2  // use RULE_OCP for every scale instead of RULE_RCEIL
+  MX_QUANT_P = 1,     // quantise the computed P and dS operands (the method's rule)
+  MX_RULE_OCP = 2,    // use RULE_OCP for every scale instead of RULE_RCEIL
+  MX_KEEP_INPUTS = 4, // study: Q, K, V, dO unquantised
+  MX_KEEP_P = 8,      // study: P~ (forward) and P~T (backward) unquantised
+  MX_KEEP_DS = 16,    // study: dS~ and dS~T unquantised
+  MX_SYM_GUARD = 32   // study: Q and dO per token on the diagonal query block of dK, dV
 };
 inline int rule_of(int flags) { return (flags & MX_RULE_OCP) ? RULE_OCP : RULE_RCEIL; }
+inline bool quant_p(int flags) { return (flags & MX_QUANT_P) && !(flags & MX_KEEP_P); }
+inline bool quant_ds(int flags) { return (flags & MX_QUANT_P) && !(flags & MX_KEEP_DS); }
 
 /* P~ of the forward: the row's probabilities are quantised in the form
  *   u_ij = 2^(S_ij log2(e) - M_i),  M_i = ceil(max_j S_ij log2(e)),
@@ -626,16 +640,16 @@ void orc_mx_attn_fwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
                      double* lse) {
   const Problem P{T, nd, Hq, Hkv, d, cu, scale};
   const std::vector<Task> tasks = head_doc_tasks(P, Hq);
-  const bool qp = flags & MX_QUANT_P;
+  const bool qp = quant_p(flags), ex = flags & MX_KEEP_INPUTS;
   const int rule = rule_of(flags);
 #pragma omp parallel for schedule(dynamic, 1)
   for (long ti = 0; ti < (long)tasks.size(); ++ti) {
     const int kdoc = tasks[ti].doc, h = tasks[ti].h, g = h / P.G();
     const int s = cu[kdoc], L = cu[kdoc + 1] - cu[kdoc];
     std::vector<double> Qtb, Qpt, Ktb, Kpt, Vtb, Vpt, srow, p, pq, orow(d);
-    mx_forms(q, s, L, h, Hq, d, rule, Qtb, Qpt);
-    mx_forms(k, s, L, g, Hkv, d, rule, Ktb, Kpt);
-    mx_forms(v, s, L, g, Hkv, d, rule, Vtb, Vpt);
+    mx_forms(q, s, L, h, Hq, d, rule, Qtb, Qpt, ex);
+    mx_forms(k, s, L, g, Hkv, d, rule, Ktb, Kpt, ex);
+    mx_forms(v, s, L, g, Hkv, d, rule, Vtb, Vpt, ex);
     for (int li = 0; li < L; ++li) {
       double m, l;
       const int n = mx_score_row(&Qpt[(size_t)li * d], Ktb, Kpt, li, d, scale, srow, p, m, l);
@@ -667,7 +681,8 @@ void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
                      int flags, double* o, double* lse, double* dq, double* dk, double* dv) {
   const Problem P{T, nd, Hq, Hkv, d, cu, scale};
   const int G = P.G();
-  const bool qp = flags & MX_QUANT_P;
+  const bool qp = quant_p(flags), qds = quant_ds(flags), ex = flags & MX_KEEP_INPUTS;
+  const bool sym = flags & MX_SYM_GUARD;
   const int rule = rule_of(flags);
   const std::vector<Task> tasks = head_doc_tasks(P, Hkv);
 #pragma omp parallel for schedule(dynamic, 1)
@@ -675,12 +690,12 @@ void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
     const int kdoc = tasks[ti].doc, g = tasks[ti].h;
     const int s = cu[kdoc], L = cu[kdoc + 1] - cu[kdoc];
     std::vector<double> Ktb, Kpt, Vtb, Vpt, Qtb, Qpt, dOtb, dOpt, srow, p, pq, orow(d);
-    mx_forms(k, s, L, g, Hkv, d, rule, Ktb, Kpt);
-    mx_forms(v, s, L, g, Hkv, d, rule, Vtb, Vpt);
+    mx_forms(k, s, L, g, Hkv, d, rule, Ktb, Kpt, ex);
+    mx_forms(v, s, L, g, Hkv, d, rule, Vtb, Vpt, ex);
     std::vector<double> dK((size_t)L * d, 0.0), dV((size_t)L * d, 0.0);
     for (int h = g * G; h < (g + 1) * G; ++h) {
-      mx_forms(q, s, L, h, Hq, d, rule, Qtb, Qpt);
-      mx_forms(dout, s, L, h, Hq, d, rule, dOtb, dOpt);
+      mx_forms(q, s, L, h, Hq, d, rule, Qtb, Qpt, ex);
+      mx_forms(dout, s, L, h, Hq, d, rule, dOtb, dOpt, ex);
       // rows are processed in 32-row query blocks so that P^T and dS^T can be
       // quantised per (key row, query block)
       for (int b0 = 0; b0 < L; b0 += 32) {
@@ -713,7 +728,7 @@ void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
           }
           // dQ_i = scale sum_j dS~_ij K~_j
           std::vector<double> dsq(ds);
-          quant_along(dsq, n, qp, rule);
+          quant_along(dsq, n, qds, rule);
           std::vector<double> dqrow(d, 0.0);
           for (int j = 0; j < n; ++j) {
             const double* kj = pick(Ktb, Kpt, j, li, d);
@@ -728,10 +743,8 @@ void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
             pc[a] = Pblk[(size_t)a * ncol + j];
             dc[a] = dSblk[(size_t)a * ncol + j];
           }
-          if (qp) {
-            quant_block(pc.data(), nb, 1, nullptr, 0, pc.data(), 1, rule);
-            quant_block(dc.data(), nb, 1, nullptr, 0, dc.data(), 1, rule);
-          }
+          if (qp) quant_block(pc.data(), nb, 1, nullptr, 0, pc.data(), 1, rule);
+          if (qds) quant_block(dc.data(), nb, 1, nullptr, 0, dc.data(), 1, rule);
           double* dkj = &dK[(size_t)j * d];
           double* dvj = &dV[(size_t)j * d];
           for (int a = 0; a < nb; ++a) {
@@ -740,8 +753,9 @@ void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
             // query-side operands of the query contraction: token-block form
             // in every query block (every query with a non-zero term here is
             // causally after key j, so no guard is needed)
-            const double* qi = &Qtb[(size_t)li * d];
-            const double* doi = &dOtb[(size_t)li * d];
+            const bool pt_side = sym && (li >> 5) == (j >> 5);
+            const double* qi = pt_side ? &Qpt[(size_t)li * d] : &Qtb[(size_t)li * d];
+            const double* doi = pt_side ? &dOpt[(size_t)li * d] : &dOtb[(size_t)li * d];
             for (int r = 0; r < d; ++r) {
               dkj[r] += dc[a] * qi[r];
               dvj[r] += pc[a] * doi[r];

@@ -77,6 +77,8 @@ def test_host_validation_codes(L):
     assert _fwd(L, _problem(d=96)) == fapk.ERR_UNSUPPORTED
     assert _fwd(L, _problem(Hq=3, Hkv=2)) == fapk.ERR_UNSUPPORTED
     assert _fwd(L, _problem(prec=7)) == fapk.ERR_UNSUPPORTED
+    assert _fwd(L, _problem(prec=fapk.MXFP8, scale_rule=fapk.SCALE_OCP)) == fapk.ERR_UNSUPPORTED
+    assert _fwd(L, _problem(prec=fapk.MXFP8, scale_rule=7)) == fapk.ERR_UNSUPPORTED
     assert _fwd(L, _problem(Hq=0)) == fapk.ERR_INVALID_ARG
     assert _fwd(L, _problem(T=-1)) == fapk.ERR_INVALID_ARG
     assert _fwd(L, _problem(max_seqlen=0)) == fapk.ERR_INVALID_ARG

@@ -61,10 +61,9 @@ def test_single_tile_and_ragged_documents():
     _check(w, require_gpu())
 
 
-@pytest.mark.parametrize("rule", [fapk.SCALE_RCEIL, fapk.SCALE_OCP])
-def test_gqa_and_both_scale_rules(rule):
+def test_gqa():
     w = W.custom([513, 64, 1000], Hq=4, Hkv=2, d=128, seed=62)
-    _check(w, require_gpu(), rule)
+    _check(w, require_gpu())
 
 
 def test_outlier_channels_16k_full():
@@ -108,23 +107,11 @@ def mx_fwd_bwd(w, dev, tensors=None, rule=fapk.SCALE_RCEIL):
     return (q, k, v, do), (o, lse, dq, dk, dv)
 
 
-# The OCP scale rule saturates a block maximum whose significand exceeds 1.75
-# (up to 12.5% error) but not one just above a power of two, so P or dS values
-# near a power of two (P ~ 1 on peaked rows, P = 1 at every document's first
-# query) quantise discontinuously: on the GQA case below a 1e-6 relative
-# perturbation of P moves the emulated dV by 2.8% under OCP and by 0.017%
-# under RCEIL (CPU measurement).  The kernel's fp32 P and the emulation's fp64
-# P differ at that level, so under OCP the backward is compared at 5e-2; the
-# default RCEIL rule keeps the 1e-2 bar.
-OCP_BWD_REL_FROB = 5e-2
-
-
-def _check_bwd(w, dev, rule=fapk.SCALE_RCEIL):
-    (q, k, v, do), (o, lse, dq, dk, dv) = mx_fwd_bwd(w, dev, rule=rule)
-    bar = MX_REL_FROB if rule == fapk.SCALE_RCEIL else OCP_BWD_REL_FROB
+def _check_bwd(w, dev):
+    (q, k, v, do), (o, lse, dq, dk, dv) = mx_fwd_bwd(w, dev)
+    bar = MX_REL_FROB
     args = [t.double().numpy() for t in (q, k, v, do)]
-    flags = oracle.MX_QUANT_P | (oracle.MX_RULE_OCP if rule == fapk.SCALE_OCP else 0)
-    em = oracle.mx_attn_bwd(*args, w.cu, w.scale, flags=flags)
+    em = oracle.mx_attn_bwd(*args, w.cu, w.scale, flags=oracle.MX_QUANT_P)
     ex = oracle.attn_bwd(*args, w.cu, w.scale)
     out = {}
     for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
@@ -143,10 +130,9 @@ def test_bwd_ragged_documents():
     _check_bwd(w, require_gpu())
 
 
-@pytest.mark.parametrize("rule", [fapk.SCALE_RCEIL, fapk.SCALE_OCP])
-def test_bwd_gqa_and_both_rules(rule):
+def test_bwd_gqa():
     w = W.custom([513, 64, 1000], Hq=4, Hkv=2, d=128, seed=72)
-    _check_bwd(w, require_gpu(), rule)
+    _check_bwd(w, require_gpu())
 
 
 def test_bwd_outlier_channels_16k_full():
@@ -242,3 +228,28 @@ def test_full_size_gqa_128k_documents_vs_emulation():
     """131072 tokens with a 65536-token first document, 32 query heads on 8 KV
     heads; two documents after the long one, KV group 3."""
     _mx_sampled_docs(W.config(5, 0), require_gpu(), first_doc=4, kv_group=3)
+
+
+@pytest.mark.parametrize("t_rel", [13, 100, 200])
+def test_bwd_dkdv_at_unaligned_t_measured(t_rel):
+    """T3 at a t that is not the end of a 32-token block (the reading of the
+    leak test that the quantisation rule cannot meet bit for bit): the query
+    block holding t shares one Q~tb scale (and one P~T / dS~T scale per key)
+    with the randomised queries after t, so dK and dV at positions <= t may
+    move by range effects (values that turn subnormal or flush).  The oracle's
+    emulation measures 40 to 2347 of 0.8e5 to 1.9e5 dK elements moving, by at
+    most 7.4e-4 of the RMS of dK, and no dV element.  The kernel must stay
+    within 2e-3 of the RMS; the counts are printed."""
+    dev = require_gpu()
+    w = W.custom([300, 513, 200], Hq=2, Hkv=2, d=128, seed=74)
+    base = list(w.tensors())
+    t = 300 + t_rel
+    base[3][t + 1:] = 0
+    _, a = mx_fwd_bwd(w, dev, tensors=base)
+    _, b = mx_fwd_bwd(w, dev, tensors=_perturb(base, t, 10, zero_dout=True))
+    for name, x, y in (("dk", a[3], b[3]), ("dv", a[4], b[4])):
+        x, y = f64(x[: t + 1]), f64(y[: t + 1])
+        n = int(np.count_nonzero(x != y))
+        rel = float(np.max(np.abs(x - y)) / np.sqrt(np.mean(x * x)))
+        print(f"T3 t_rel={t_rel} {name}: {n} of {x.size} elements differ, max diff {rel:.2e} of RMS")
+        assert rel <= 2e-3, (name, n, rel)

@@ -343,3 +343,30 @@ def test_dk_uses_token_block_q_and_dv_token_block_do(orc):
     assert out["dk"][0, 0, 0] == 0.0439453125
     out = orc.mx_attn_bwd(zeros, zeros, zeros, sel, _cu([T]), 1.0)
     assert out["dv"][0, 0, 0] == 0.0537109375
+
+
+def test_study_switches_reach_the_exact_oracle(orc):
+    """The accuracy-study switches of the emulation (oracle/mx_accuracy_study.py)
+    each take one quantisation out; with all three out (inputs, P~/P~T,
+    dS~/dS~T) the emulation is the exact oracle on any inputs.  With the
+    symmetric guard, dK on the diagonal query block uses the per-token Q: in
+    the hand case of test_dk_uses_token_block_q_and_dv_token_block_do that is
+    0.140625 * 0.28125."""
+    rng = np.random.default_rng(5)
+    cu = _cu([45, 1, 70, 33])
+    T, Hq, Hkv, d, sc = cu[-1], 4, 2, 64, 0.125
+    q, k, v, do = (rng.standard_normal((T, H, d)) for H in (Hq, Hkv, Hkv, Hq))
+    ex = orc.attn_bwd(q, k, v, do, cu, sc)
+    flags = orc.MX_QUANT_P | orc.MX_KEEP_INPUTS | orc.MX_KEEP_P | orc.MX_KEEP_DS
+    mx = orc.mx_attn_bwd(q, k, v, do, cu, sc, flags=flags)
+    for key in ex:
+        np.testing.assert_allclose(mx[key], ex[key], rtol=0, atol=1e-12, err_msg=key)
+    T, d = 40, 32
+    sel = _selection_rows(T, d)
+    zeros = np.zeros((T, 1, d))
+    v = np.zeros((T, 1, d))
+    v[0, 0, 2] = 1.0
+    do = np.zeros((T, 1, d))
+    do[5, 0, 2] = 1.0
+    out = orc.mx_attn_bwd(sel, zeros, v, do, _cu([T]), 1.0, flags=orc.MX_QUANT_P | orc.MX_SYM_GUARD)
+    assert out["dk"][0, 0, 0] == 0.140625 * 0.28125
