@@ -69,6 +69,7 @@ def _load():
     lib.orc_attn_bwd.argtypes = head + [P, P, P, P, P, P, P, P, P]
     lib.orc_attn_rows.argtypes = head + [P, P, P, P, i, P, P, P, P, P]
     lib.orc_attn_kv_cols.argtypes = head + [P, P, P, P, i, P, P, P, P]
+    lib.orc_attn_kv_cols_from_rows.argtypes = head + [P, P, P, P, P, P, i, P, P, P, P]
     lib.orc_e4m3_encode.argtypes = [dbl]
     lib.orc_e4m3_encode.restype = ctypes.c_uint8
     lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -156,6 +157,54 @@ def attn_kv_cols(q, k, v, do, cu, scale, tok, kvhead):
     dk, dv = np.zeros((n, d)), np.zeros((n, d))
     _load().orc_attn_kv_cols(T, nd, _ptr(cu), Hq, Hkv, d, float(scale), _ptr(q), _ptr(k),
                              _ptr(v), _ptr(do), n, _ptr(tok), _ptr(kvhead), _ptr(dk), _ptr(dv))
+    return dk, dv
+
+
+def attn_fwd_doc(q, k, v, cu, scale, doc, head, chunk: int = 2048):
+    """Exact O [L,d] and LSE [L] of every query of document `doc` for query
+    head `head`, for one long document (where the per-(document, head) tasks
+    of attn_fwd leave most cores idle).  Plain fp64 torch CPU ops, row by row
+    as the definition reads ("GPT Kernel Programlama" page secs. 3-6): the
+    score row S_i = scale q_i K^T over the document's keys, the causal mask
+    j > i, the stable softmax and O_i = P_i V; rows are handed to the matmul
+    `chunk` at a time, each row on its own, so that the library's threads
+    share the work."""
+    import torch
+    cu = _i32(cu)
+    T, Hq, d = q.shape
+    G = Hq // k.shape[1]
+    s, e = int(cu[doc]), int(cu[doc + 1])
+    L = e - s
+    Q = torch.from_numpy(_f64(q[s:e, head]))
+    K = torch.from_numpy(_f64(k[s:e, head // G]))
+    V = torch.from_numpy(_f64(v[s:e, head // G]))
+    o = torch.empty((L, d), dtype=torch.float64)
+    lse = torch.empty(L, dtype=torch.float64)
+    for i0 in range(0, L, chunk):
+        i1 = min(L, i0 + chunk)
+        S = (Q[i0:i1] @ K[:i1].T) * float(scale)
+        S.masked_fill_(torch.arange(i1)[None, :] > torch.arange(i0, i1)[:, None], float("-inf"))
+        m = S.amax(dim=1, keepdim=True)
+        S.sub_(m).exp_()
+        ell = S.sum(dim=1, keepdim=True)
+        o[i0:i1] = (S @ V[:i1]) / ell
+        lse[i0:i1] = (m + torch.log(ell))[:, 0]
+    return o.numpy(), lse.numpy()
+
+
+def attn_kv_cols_from_rows(q, k, v, do, o, lse, cu, scale, tok, kvhead):
+    """Exact dK, dV of selected (token, kv-head) keys, given the exact O
+    [T,Hq,d] and LSE [Hq,T] of every query that sees them (from attn_fwd or
+    attn_fwd_doc); no query row is recomputed."""
+    q, k, v, do, o, lse, cu = _f64(q), _f64(k), _f64(v), _f64(do), _f64(o), _f64(lse), _i32(cu)
+    T, nd, Hq, Hkv, d = _dims(q, k, cu)
+    assert o.shape == q.shape and lse.shape == (Hq, T)
+    tok, kvhead = _i32(tok), _i32(kvhead)
+    n = len(tok)
+    dk, dv = np.zeros((n, d)), np.zeros((n, d))
+    _load().orc_attn_kv_cols_from_rows(T, nd, _ptr(cu), Hq, Hkv, d, float(scale), _ptr(q), _ptr(k),
+                                       _ptr(v), _ptr(do), _ptr(o), _ptr(lse), n, _ptr(tok), _ptr(kvhead),
+                                       _ptr(dk), _ptr(dv))
     return dk, dv
 
 

@@ -571,6 +571,53 @@ void orc_attn_kv_cols(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, 
   }
 }
 
+/* Exact dK and dV of selected (token, kv head) keys from the exact forward
+ * rows of the queries that see them: o [T][Hq][d] and lse [Hq][T] must hold
+ * the exact O_i and LSE_i of every query i >= j of key j's document for the
+ * query heads of its group (other entries are not read).  Same sums as
+ * orc_attn_kv_cols, with P_ij = exp(S_ij - LSE_i) (the normalised softmax, by
+ * the definition of LSE) and D_i = dO_i . O_i, so no query row is recomputed.
+ * dk/dv: [n][d]. */
+void orc_attn_kv_cols_from_rows(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
+                                const double* q, const double* k, const double* v, const double* dout,
+                                const double* o, const double* lse, int n, const int32_t* tok,
+                                const int32_t* kvhead, double* dk, double* dv) {
+  const Problem P{T, nd, Hq, Hkv, d, cu, scale};
+  const int G = P.G();
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int si = 0; si < n; ++si) {
+    const int j = tok[si], g = kvhead[si];
+    const int kdoc = (int)(std::upper_bound(cu, cu + nd + 1, j) - cu) - 1;
+    const int e = cu[kdoc + 1];
+    const double* kj = &k[idx3(j, g, 0, Hkv, d)];
+    const double* vj = &v[idx3(j, g, 0, Hkv, d)];
+    std::vector<double> dkj(d, 0.0), dvj(d, 0.0);
+    for (int h = g * G; h < (g + 1) * G; ++h) {
+      for (int i = j; i < e; ++i) {
+        const double* qi = &q[idx3(i, h, 0, Hq, d)];
+        const double* doi = &dout[idx3(i, h, 0, Hq, d)];
+        const double* oi = &o[idx3(i, h, 0, Hq, d)];
+        double sij = 0.0, dpj = 0.0, D = 0.0;
+        for (int r = 0; r < d; ++r) {
+          sij += qi[r] * kj[r];
+          dpj += doi[r] * vj[r];
+          D += doi[r] * oi[r];
+        }
+        const double pij = std::exp(scale * sij - lse[(size_t)h * T + i]);
+        const double ds = pij * (dpj - D);
+        for (int r = 0; r < d; ++r) {
+          dkj[r] += ds * qi[r];
+          dvj[r] += pij * doi[r];
+        }
+      }
+    }
+    for (int r = 0; r < d; ++r) {
+      dk[(size_t)si * d + r] = scale * dkj[r];
+      dv[(size_t)si * d + r] = dvj[r];
+    }
+  }
+}
+
 /* ---- MXFP8 quantiser -------------------------------------------------- */
 
 uint8_t orc_e4m3_encode(double y) { return e4m3_encode(y); }

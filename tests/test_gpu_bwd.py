@@ -67,12 +67,16 @@ def test_packed_8k_full():
     _full_check(W.config(2, 0), require_gpu())
 
 
-def _sampled_check(w, dev, n_rows=96, n_cols=24, seed=0):
+def _sampled_check(w, dev, n_rows=96, n_cols=24, seed=0, long_doc=None):
     """Full-size workload in the launch configuration the benchmark uses;
     the oracle computes sampled rows (O, LSE, dQ) and sampled keys (dK, dV) one
     by one.  Keys are drawn near document ends, where the exact dK/dV needs few
-    query rows."""
+    query rows, and, with `long_doc` = (document, KV head, doc-local key
+    positions), at the start of a long document, where every later query of
+    every query head of the group adds to them (the longest accumulations)."""
     (q, k, v, do), (o, lse, dq, dk, dv) = run_fwd_bwd(w, dev)
+    if long_doc is not None:
+        _long_doc_keys(w, (q, k, v, do), dk, dv, *long_doc)
     rng = np.random.default_rng(seed)
     cu = w.cu
     tok = rng.integers(0, w.T, n_rows)
@@ -93,14 +97,43 @@ def _sampled_check(w, dev, n_rows=96, n_cols=24, seed=0):
     check_close("dV", f64(dv)[ktok, kvh], rdv)
 
 
+def _long_doc_keys(w, tensors, dk, dv, doc, kv_head, key_locals):
+    """dK, dV of keys of one document and KV head against the oracle: the
+    exact forward rows (O, LSE) of every query of the document for the group's
+    query heads, then each key's sums over all queries after it."""
+    q, k, v, do = tensors
+    s, e = int(w.cu[doc]), int(w.cu[doc + 1])
+    G = w.Hq // w.Hkv
+    hq = slice(kv_head * G, (kv_head + 1) * G)
+    qs, dos = (x[s:e, hq].double().numpy() for x in (q, do))
+    ks, vs = (x[s:e, kv_head:kv_head + 1].double().numpy() for x in (k, v))
+    cu_s = np.array([0, e - s], np.int32)
+    o_s = np.zeros_like(qs)
+    lse_s = np.zeros((G, e - s))
+    for h in range(G):
+        o_s[:, h], lse_s[h] = oracle.attn_fwd_doc(qs, ks, vs, cu_s, w.scale, 0, h)
+    tok = np.asarray(key_locals, dtype=np.int32)
+    rdk, rdv = oracle.attn_kv_cols_from_rows(qs, ks, vs, dos, o_s, lse_s, cu_s, w.scale, tok,
+                                             np.zeros_like(tok))
+    check_close("dK (long document)", f64(dk)[s + tok, kv_head], rdk)
+    check_close("dV (long document)", f64(dv)[s + tok, kv_head], rdv)
+
+
 def test_full_size_packed_32k_sampled():
-    """32768 tokens, log-normal lengths, 32 heads (the benchmark workload)."""
-    _sampled_check(W.config(4, 0), require_gpu())
+    """32768 tokens, log-normal lengths, 32 heads (the benchmark workload);
+    plus 16 keys in the first 256 tokens of its longest document (7545
+    tokens), KV head 5."""
+    w = W.config(4, 0)
+    doc = int(np.argmax(np.diff(w.cu)))
+    keys = np.random.default_rng(3).choice(256, 16, replace=False)
+    _sampled_check(w, require_gpu(), long_doc=(doc, 5, keys))
 
 
 def test_full_size_gqa_128k_sampled():
-    """131072 tokens with a 65536-token document, 32 query heads on 8 KV heads."""
-    _sampled_check(W.config(5, 0), require_gpu(), n_rows=48, n_cols=12)
+    """131072 tokens with a 65536-token document, 32 query heads on 8 KV heads;
+    plus 3 keys at the start of the 65536-token document (KV head 1, so the
+    sums run over 4 query heads x up to 65536 queries)."""
+    _sampled_check(W.config(5, 0), require_gpu(), n_rows=48, n_cols=12, long_doc=(0, 1, [0, 37, 300]))
 
 
 def test_deterministic():

@@ -219,9 +219,13 @@ def _mx_sampled_docs(w, dev, max_tokens=6000, first_doc=0, kv_group=0):
     return res
 
 
-def test_full_size_packed_32k_documents_vs_emulation():
-    """The 32768-token benchmark workload (32 heads, 1% x8 outlier tokens)."""
-    _mx_sampled_docs(W.config(4, 0), require_gpu())
+@pytest.mark.parametrize("first_doc,max_tokens,kv_group", [(0, 6000, 0), (6, 13000, 9)])
+def test_full_size_packed_32k_documents_vs_emulation(first_doc, max_tokens, kv_group):
+    """The 32768-token benchmark workload (32 heads, 1% x8 outlier tokens):
+    its first two documents (2322 and 1795 tokens), and its two longest
+    (7545 and 5280 tokens, documents 6 and 7)."""
+    _mx_sampled_docs(W.config(4, 0), require_gpu(), max_tokens=max_tokens, first_doc=first_doc,
+                     kv_group=kv_group)
 
 
 def test_full_size_gqa_128k_documents_vs_emulation():

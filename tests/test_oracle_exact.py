@@ -206,6 +206,19 @@ def test_sampled_rows_and_columns_match_full(orc):
     dk, dv = orc.attn_kv_cols(q, k, v, do, cu, sc, tok, kvh)
     np.testing.assert_allclose(dk, full["dk"][tok, kvh], atol=1e-12)
     np.testing.assert_allclose(dv, full["dv"][tok, kvh], atol=1e-12)
+    # the forward rows alone, and the keys' gradients from the full oracle's
+    # forward rows (P = exp(S - LSE), D = dO . O, no row recomputed)
+    for doc in range(len(cu) - 1):
+        for h in range(Hq):
+            o2, lse2 = orc.attn_fwd_doc(q, k, v, cu, sc, doc, h)
+            np.testing.assert_allclose(o2, full["o"][cu[doc]:cu[doc + 1], h], atol=1e-12)
+            np.testing.assert_allclose(lse2, full["lse"][h, cu[doc]:cu[doc + 1]], atol=1e-12)
+    dk2, dv2 = orc.attn_kv_cols_from_rows(q, k, v, do, full["o"], full["lse"], cu, sc, tok, kvh)
+    np.testing.assert_allclose(dk2, full["dk"][tok, kvh], atol=1e-12)
+    np.testing.assert_allclose(dv2, full["dv"][tok, kvh], atol=1e-12)
+    # a wrong row state moves them: the planted mistake of an LSE off by 0.1
+    dk3, _ = orc.attn_kv_cols_from_rows(q, k, v, do, full["o"], full["lse"] + 0.1, cu, sc, tok, kvh)
+    assert np.max(np.abs(dk3 - full["dk"][tok, kvh])) > 1e-3
 
 
 def test_future_perturbation_leaves_past_bit_identical(orc):
