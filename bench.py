@@ -207,8 +207,8 @@ KERNELS = {
     # per path: names of the intervals between the events the library records
     "bf16": (["schedule_fwd", "convert_v_f16", "fwd_kernel"],
              ["schedule_kv", "schedule_q", "convert_k_f16", "delta_kernel", "dkdv_kernel", "dq_kernel"]),
-    "mxfp8": (["schedule_fwd", "quantize_qkv", "fwd_kernel"],
-              ["schedule_kv", "schedule_q", "quantize_do", "delta_kernel", "dkdv_kernel", "dq_kernel"]),
+    "mxfp8": (["schedule_fwd", "quantize_kv", "fwd_kernel"],
+              ["schedule_kv", "schedule_q", "delta_quantize_do", "dkdv_kernel", "dq_kernel"]),
 }
 # algorithmic tensor work of each attention kernel per visible (query, key)
 # pair and query head, in units of d: forward S and PV = 4; dK/dV kernel S,
@@ -285,7 +285,8 @@ class Path:
         torch.cuda.synchronize(self.dev)
         if not self.status_ok():
             raise RuntimeError(f"{self.prec}: device status {self.fapk.status(self.ws_f)}/{self.fapk.status(self.ws_b)}")
-        timers = [(self.fapk.KernelTimer(4), self.fapk.KernelTimer(7)) for _ in range(steps)]
+        nf, nb = (len(x) + 1 for x in KERNELS[self.prec])
+        timers = [(self.fapk.KernelTimer(nf), self.fapk.KernelTimer(nb)) for _ in range(steps)]
         launches0 = self.fapk.launch_count()
         barrier(world)
         torch.cuda.synchronize(self.dev)
@@ -377,16 +378,24 @@ def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, clk, conf
     out = {"value": value, "ms_per_step": ms_per_step, "pct_of_dense_peak": 100.0 * (value / world) / dense,
            "dense_peak_tflops": dense, "roofline": roofline, "gpu_launches": launches}
     if prec == "mxfp8":
-        # quantize launches of the forward (HBM bound), algorithmic bytes per
-        # element: 2 B bf16 read, then per form 1 B of E4M3 codes and 1/32 B of
-        # scales written (two forms); extra copies a kernel writes for its own
-        # use are not counted
-        qbytes = (w.T * w.Hq * w.d + 2 * w.T * w.Hkv * w.d) * (2.0 + 2 * (1.0 + 1.0 / 32))
-        gbs = qbytes / (kern_ms["quantize_qkv"] * 1e-3) / 1e9
+        # the standalone quantisation launch of the forward (K and V, both
+        # forms; HBM bound), algorithmic bytes per element: 2 B bf16 read, then
+        # per form 1 B of E4M3 codes and 1/32 B of scales written.  Q is
+        # quantised on load inside the forward kernel, dO inside the D pass.
+        qbytes = 2 * w.T * w.Hkv * w.d * (2.0 + 2 * (1.0 + 1.0 / 32))
+        gbs = qbytes / (kern_ms["quantize_kv"] * 1e-3) / 1e9
         out["roofline_quantize"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                                     "algorithmic_bytes": qbytes,
-                                    "kernel": "quantize_mxfp8_kernel (Q, K, V; both forms)"}
+                                    "kernel": "quantize_mxfp8_kernel (K and V in one launch; both forms)"}
+        # the D pass with dO's quantisation: reads dO, O and O's residual
+        # (6 B), writes dO's two forms (2 + 1/16 B) per element and D
+        dbytes = w.T * w.Hq * w.d * (6.0 + 2 * (1.0 + 1.0 / 32)) + 4.0 * w.T * w.Hq
+        gbs = dbytes / (kern_ms["delta_quantize_do"] * 1e-3) / 1e9
+        out["roofline_delta_quantize_do"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                                             "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                                             "algorithmic_bytes": dbytes}
+        out["quantize_ms_per_step"] = kern_ms["quantize_kv"] + kern_ms["delta_quantize_do"]
     return out
 
 

@@ -182,16 +182,16 @@ BwdLayout bwd_layout(const fapk_problem_t* P) {
 //           the 8 of the bf16 output;
 //  v16:     fp16 copy of V [T][Hkv][d], the B operand of O += P V (and of the
 //           backward's dP = dO V^T).
-//  MXFP8 path, instead of v16: the quantiser's forms of Q, K and V (codes and
-//  scales, token-block and per-token), reused by the backward in both
-//  orientations, and V's per-token form dequantised to bf16.
+//  MXFP8 path, instead of v16: the MX forms of Q, K and V (codes and scales,
+//  token-block and per-token), reused by the backward in both orientations;
+//  Q's are written by the forward kernel, which quantises Q on load, K's and
+//  V's by the quantiser's prepass.
 struct MxForms {
   size_t vtb, stb, vpt, spt;  // offsets of codes / scales
 };
 struct CtxLayout {
   size_t o_resid, v16, total;
   MxForms q, k, v;
-  size_t v_deq_pt, k_deq_pt;
 };
 CtxLayout ctx_layout(const fapk_problem_t* P) {
   CtxLayout L;
@@ -217,9 +217,7 @@ CtxLayout ctx_layout(const fapk_problem_t* P) {
   L.q = forms(P->Hq);
   L.k = forms(P->Hkv);
   L.v = forms(P->Hkv);
-  L.v_deq_pt = off;
-  L.k_deq_pt = align_up(L.v_deq_pt + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
-  L.total = align_up(L.k_deq_pt + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
+  L.total = off;
   return L;
 }
 
@@ -256,8 +254,9 @@ bool make_tmap_thd(CUtensorMap* map, const void* base, int T, int H, int d, bool
 
 namespace {
 
-// MXFP8 forward: quantise Q, K, V into ctx (both forms; V also dequantised
-// per token), build the 128-row schedule, run the kernel.
+// MXFP8 forward: build the 128-row schedule, quantise K and V into ctx (both
+// forms, one launch), run the kernel (which quantises Q on load and writes its
+// forms into ctx).
 int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void* v, void* o, float* lse, void* ctx,
               void* ws, const FwdLayout& L, int sms, cudaStream_t st) {
   auto* status = static_cast<DeviceStatus*>(ws);
@@ -271,27 +270,27 @@ int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void*
   int rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, a.sched, status, true, st));
   if (rc != FAPK_OK) return rc;
   mk.at(1, st);
-  const int forms = FAPK_FORM_TB | FAPK_FORM_PT;
-  rc = cuda_status(launch_quantize_mxfp8(q, P->T, P->Hq, P->d, P->cu_seqlens_dev, P->n_docs, forms, P->scale_rule,
-                                         u8(C.q.vtb), u8(C.q.stb), u8(C.q.vpt), u8(C.q.spt), st));
+  QuantJobs jobs;
+  jobs.job[0] = QuantJob{static_cast<const __nv_bfloat16*>(k), P->Hkv, u8(C.k.vtb), u8(C.k.stb), u8(C.k.vpt),
+                         u8(C.k.spt), nullptr};
+  jobs.job[1] = QuantJob{static_cast<const __nv_bfloat16*>(v), P->Hkv, u8(C.v.vtb), u8(C.v.stb), u8(C.v.vpt),
+                         u8(C.v.spt), nullptr};
+  rc = cuda_status(launch_quantize_jobs(jobs, 2, P->T, P->d, P->cu_seqlens_dev, P->n_docs,
+                                        FAPK_FORM_TB | FAPK_FORM_PT, P->scale_rule, st));
   if (rc != FAPK_OK) return rc;
-  rc = cuda_status(launch_quantize_mxfp8(k, P->T, P->Hkv, P->d, P->cu_seqlens_dev, P->n_docs, forms, P->scale_rule,
-                                         u8(C.k.vtb), u8(C.k.stb), u8(C.k.vpt), u8(C.k.spt), st,
-                                         c + C.k_deq_pt));
-  if (rc != FAPK_OK) return rc;
-  rc = cuda_status(launch_quantize_mxfp8(v, P->T, P->Hkv, P->d, P->cu_seqlens_dev, P->n_docs, forms, P->scale_rule,
-                                         u8(C.v.vtb), u8(C.v.stb), u8(C.v.vpt), u8(C.v.spt), st,
-                                         c + C.v_deq_pt));
-  if (rc != FAPK_OK) return rc;
+  a.q = q;
   a.q_vpt = u8(C.q.vpt);
   a.q_spt = u8(C.q.spt);
+  a.q_vtb = u8(C.q.vtb);
+  a.q_stb = u8(C.q.stb);
   a.k_vtb = u8(C.k.vtb);
   a.k_stb = u8(C.k.stb);
   a.k_vpt = u8(C.k.vpt);
   a.k_spt = u8(C.k.spt);
   a.v_vtb = u8(C.v.vtb);
   a.v_stb = u8(C.v.stb);
-  a.v_deq_pt = c + C.v_deq_pt;
+  a.v_vpt = u8(C.v.vpt);
+  a.v_spt = u8(C.v.spt);
   a.o = o;
   a.lse = lse;
   a.o_resid = c + C.o_resid;
@@ -313,8 +312,8 @@ int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void*
   return rc;
 }
 
-// MXFP8 backward: quantise dO (both forms) into the workspace, build both
-// schedules, run D, dK/dV and dQ.
+// MXFP8 backward: build both schedules, then D together with dO's two MX
+// forms (one pass over dO, into the workspace), dK/dV and dQ.
 int bwd_mxfp8(const fapk_problem_t* P, const void* o, const float* lse, const void* dout, const void* ctx, void* dq,
               void* dk, void* dv, void* ws, const BwdLayout& L, int sms, cudaStream_t st) {
   auto* status = static_cast<DeviceStatus*>(ws);
@@ -333,16 +332,10 @@ int bwd_mxfp8(const fapk_problem_t* P, const void* o, const float* lse, const vo
   a.marks.at(1, st);
   rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kBwdRows, a.sched_q, status, false, st));
   if (rc != FAPK_OK) return rc;
-  a.marks.at(2, st);
-  rc = cuda_status(launch_quantize_mxfp8(dout, P->T, P->Hq, P->d, P->cu_seqlens_dev, P->n_docs,
-                                         FAPK_FORM_TB | FAPK_FORM_PT, P->scale_rule, wu8(L.do_vtb), wu8(L.do_stb),
-                                         wu8(L.do_vpt), wu8(L.do_spt), st));
-  if (rc != FAPK_OK) return rc;
   a.q_vtb = cu8(C.q.vtb); a.q_stb = cu8(C.q.stb); a.q_vpt = cu8(C.q.vpt); a.q_spt = cu8(C.q.spt);
   a.k_vtb = cu8(C.k.vtb); a.k_stb = cu8(C.k.stb); a.k_vpt = cu8(C.k.vpt); a.k_spt = cu8(C.k.spt);
   a.v_vtb = cu8(C.v.vtb); a.v_stb = cu8(C.v.stb); a.v_vpt = cu8(C.v.vpt); a.v_spt = cu8(C.v.spt);
   a.do_vtb = wu8(L.do_vtb); a.do_stb = wu8(L.do_stb); a.do_vpt = wu8(L.do_vpt); a.do_spt = wu8(L.do_spt);
-  a.k_deq_pt = c + C.k_deq_pt;
   a.o = o;
   a.o_resid = c + C.o_resid;
   a.lse = lse;
@@ -350,7 +343,7 @@ int bwd_mxfp8(const fapk_problem_t* P, const void* o, const float* lse, const vo
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.delta = reinterpret_cast<float*>(w + L.delta);
   a.cu = P->cu_seqlens_dev;
-  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv;
+  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.n_docs = P->n_docs;
   a.scale = P->scale;
   a.grad_bf16 = P->grad_dtype == FAPK_GRAD_BF16;
   a.rule = P->scale_rule;

@@ -20,7 +20,8 @@
 //    per-token forms into the same TMEM columns), dS~ quantised into shared
 //    memory, dQ += dS~ K~tb (FP8, the same K~tb bytes read MN-major) plus, on
 //    the diagonal tile, the diagonal blocks as an exact bf16 MMA with the
-//    dequantised per-token K.
+//    per-token K, which the compute warps dequantise on load at the start of
+//    each item.
 //  * dkdv_mx: item = (document, 128-key tile, KV head); one thread per key
 //    row, warpgroup w on query columns [64w, 64w + 64).  Per query tile:
 //    S^T then dP^T into one TMEM region in turn (TMEM also holds dV, dK and
@@ -115,33 +116,6 @@ __device__ __forceinline__ void store_bf16_32(uint8_t* tile, int row, int q, con
         make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
 }
 
-// ---------------------------------------------------------------------------
-// D = rowsum(dO * (o + o_resid)), fp32 [Hq][T]
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) delta_mx_kernel(const __nv_bfloat16* __restrict__ o,
-                                                       const __nv_bfloat16* __restrict__ o_resid,
-                                                       const __nv_bfloat16* __restrict__ dout,
-                                                       float* __restrict__ delta, int T, int Hq) {
-  const long long row = (long long)blockIdx.x * 16 + threadIdx.x / 16;
-  const int c8 = threadIdx.x % 16;
-  float acc = 0.f;
-  if (row < (long long)T * Hq) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + row * 128) + c8);
-    const uint4 r = __ldg(reinterpret_cast<const uint4*>(o_resid + row * 128) + c8);
-    const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * 128) + c8);
-    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wr[4] = {r.x, r.y, r.z, r.w}, wb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc += (__uint_as_float(wa[i] << 16) + __uint_as_float(wr[i] << 16)) * __uint_as_float(wb[i] << 16);
-      acc += (__uint_as_float(wa[i] & 0xFFFF0000u) + __uint_as_float(wr[i] & 0xFFFF0000u)) *
-             __uint_as_float(wb[i] & 0xFFFF0000u);
-    }
-  }
-#pragma unroll
-  for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-  if (row < (long long)T * Hq && c8 == 0) delta[(row % Hq) * T + row / Hq] = acc;
-}
-
 struct MxParams {
   const int32_t* cu;
   SchedView sched;
@@ -176,9 +150,9 @@ constexpr int oSf = oDSd + kBf16;  // sfQ, sfDO, sfKpt, sfVpt, sfDS, per stage {
 constexpr int kNumSf = 5 + 3 * kStages;
 constexpr int oBars = oSf + kNumSf * kSfBlk;
 // bars: q_full, q_empty, st_full[S], st_empty[S], s_full, s_free, dp_full, dp_free, ds_ready, dq_done,
-//       acc_full, acc_free, fin
+//       acc_full, acc_free, fin, kd_full
 // + the unit ring's full[8] and empty[8]
-constexpr int kNumBars = 2 + 2 * kStages + 9 + 2 * kUnitRing;
+constexpr int kNumBars = 2 + 2 * kStages + 10 + 2 * kUnitRing;
 constexpr int kSmem = oBars + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
 static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may use");
 // TMEM: S and dP regions (each read out into registers and released at
@@ -192,7 +166,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
     dq_mx_kernel(const __grid_constant__ CUtensorMap tm_qpt, const __grid_constant__ CUtensorMap tm_dopt,
                  const __grid_constant__ CUtensorMap tm_ktb, const __grid_constant__ CUtensorMap tm_vtb,
                  const __grid_constant__ CUtensorMap tm_kpt, const __grid_constant__ CUtensorMap tm_vpt,
-                 const __grid_constant__ CUtensorMap tm_kd16, const MxParams p) {
+                 const MxParams p) {
   using namespace dqk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -211,6 +185,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
   uint64_t* acc_full = s_full + 6;
   uint64_t* acc_free = s_full + 7;
   uint64_t* fin = s_full + 8;
+  uint64_t* kd_full = s_full + 9;  // the diagonal per-token K dequantised to bf16 (compute warps)
   const UnitRing ring{reinterpret_cast<int*>(bars + kNumBars) + 4, bars + kNumBars - 2 * kUnitRing,
                       bars + kNumBars - kUnitRing};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
@@ -234,6 +209,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kComputeWarps);
     mbar_init(fin, 2);
+    mbar_init(kd_full, kComputeWarps);
     unit_ring_init(ring, 2 + kComputeWarps);  // both MMA threads and the compute warps
     *abort_flag = 0;
     fence_mbar_init();
@@ -281,13 +257,11 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       reinterpret_cast<uint4*>(sfb(3))[lane] = pt_rows(p.v_spt, q0, lane, p.T, p.Hkv, g);
       fence_proxy_async_smem();
       if (lane == 0) {
-        mbar_arrive_expect_tx(q_full, 4 * kCode + kBf16);
+        mbar_arrive_expect_tx(q_full, 4 * kCode);
         tma_load_3d(smem + oQ, &tm_qpt, q_full, 0, h, q0);
         tma_load_3d(smem + oDO, &tm_dopt, q_full, 0, h, q0);
         tma_load_3d(smem + oKpt, &tm_kpt, q_full, 0, g, q0);  // the diagonal key tile starts at q0
         tma_load_3d(smem + oVpt, &tm_vpt, q_full, 0, g, q0);
-        tma_load_3d(smem + oKd, &tm_kd16, q_full, 0, g, q0);
-        tma_load_3d(smem + oKd + kBox, &tm_kd16, q_full, 64, g, q0);
       } else {
         mbar_arrive(q_full);
       }
@@ -400,6 +374,8 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
             mx_kk(tDQ, aDS, ak, tSfDS, tSfKdq, true, v > 0);
             if (diag) {
               // diagonal 32x32 blocks: exact bf16 dS~ times dequantised per-token K
+              if (!mbar_wait(kd_full, unit_i & 1, wd, 103)) { ok = false; break; }
+              tc_fence_after();
               constexpr uint32_t idesc_d = idesc_bf16_f32(128, 128, false, true);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
@@ -448,6 +424,23 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       decode(un, doc, s, e, h, g, q0, n);
       const int i = q0 + row;
       const bool valid = i < e;
+      {
+        // the diagonal per-token K, dequantised to bf16 for the exact
+        // diagonal-block product: this thread's key row `row`, channels
+        // 32 wg .. 32 wg + 31.  The previous item's dQ MMAs have completed
+        // (q_full of this item follows the loader's wait on q_empty).
+        if (!warp_wait(q_full, unit_i & 1, wd, 104)) break;
+        const uint8_t* krow = smem + oKpt + row * 128;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(krow + (((2 * wg) ^ (row & 7)) << 4));
+        const uint4 c1 = *reinterpret_cast<const uint4*>(krow + (((2 * wg + 1) ^ (row & 7)) << 4));
+        const uint32_t codes[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        uint32_t kd[16];
+        dequant32_bf16(codes, sfb(2)[16 * lane + 4 * quarter + wg], kd);
+        store_bf16_32(smem + oKd, row, wg, kd);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        warp_arrive(kd_full);
+      }
       // rows past the document end get P = 0
       const float l2 = valid ? p.lse[(size_t)h * p.T + i] * kLog2e : INFINITY;
       const float dl = valid ? p.delta[(size_t)h * p.T + i] : 0.f;
@@ -971,23 +964,25 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
 }  // namespace
 
 cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
-  // 1. D
-  a.marks.at(3, stream);
+  // 1. D = rowsum(dO * (o + residual)) and dO's two MX forms, in one read of dO
+  a.marks.at(2, stream);
   {
-    const long long rows = (long long)a.T * a.Hq;
-    delta_mx_kernel<<<(unsigned)((rows + 15) / 16), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.o_resid),
-        static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.T, a.Hq);
-    note_launches(1);
-    cudaError_t e = cudaGetLastError();
+    QuantJob job{static_cast<const __nv_bfloat16*>(a.dout), a.Hq, const_cast<uint8_t*>(a.do_vtb),
+                 const_cast<uint8_t*>(a.do_stb), const_cast<uint8_t*>(a.do_vpt), const_cast<uint8_t*>(a.do_spt),
+                 nullptr};
+    DeltaArgs da;
+    da.o = static_cast<const __nv_bfloat16*>(a.o);
+    da.o_resid = static_cast<const __nv_bfloat16*>(a.o_resid);
+    da.delta = a.delta;
+    da.T = a.T;
+    cudaError_t e = launch_quantize_with_delta(job, a.T, 128, a.cu, a.n_docs, a.rule, da, stream);
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap tqpt, tqtb, tktb, tkpt, tvtb, tvpt, tdopt, tdotb, tkd;
+  CUtensorMap tqpt, tqtb, tktb, tkpt, tvtb, tvpt, tdopt, tdotb;
   if (!make_tmap_codes(&tqpt, a.q_vpt, a.T, a.Hq) || !make_tmap_codes(&tqtb, a.q_vtb, a.T, a.Hq) ||
       !make_tmap_codes(&tktb, a.k_vtb, a.T, a.Hkv) || !make_tmap_codes(&tkpt, a.k_vpt, a.T, a.Hkv) ||
       !make_tmap_codes(&tvtb, a.v_vtb, a.T, a.Hkv) || !make_tmap_codes(&tvpt, a.v_vpt, a.T, a.Hkv) ||
-      !make_tmap_codes(&tdopt, a.do_vpt, a.T, a.Hq) || !make_tmap_codes(&tdotb, a.do_vtb, a.T, a.Hq) ||
-      !make_tmap_thd(&tkd, a.k_deq_pt, a.T, a.Hkv, 128))
+      !make_tmap_codes(&tdopt, a.do_vpt, a.T, a.Hq) || !make_tmap_codes(&tdotb, a.do_vtb, a.T, a.Hq))
     return cudaErrorInvalidValue;
   MxParams p;
   p.cu = a.cu;
@@ -1007,7 +1002,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
   p.grad_bf16 = a.grad_bf16;
   p.rule = a.rule;
   // 2. dK, dV
-  a.marks.at(4, stream);
+  a.marks.at(3, stream);
   {
     cudaError_t e = cudaFuncSetAttribute(dkdv_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvk::kSmem);
     if (e != cudaSuccess) return e;
@@ -1025,7 +1020,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   // 3. dQ
-  a.marks.at(5, stream);
+  a.marks.at(4, stream);
   {
     cudaError_t e = cudaFuncSetAttribute(dq_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::kSmem);
     if (e != cudaSuccess) return e;
@@ -1037,12 +1032,12 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     pq.out1 = nullptr;
     const long long max_units = (long long)a.sched_q.max_items * a.Hq;
     const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
-    dq_mx_kernel<<<grid, dqk::kThreads, dqk::kSmem, stream>>>(tqpt, tdopt, tktb, tvtb, tkpt, tvpt, tkd, pq);
+    dq_mx_kernel<<<grid, dqk::kThreads, dqk::kSmem, stream>>>(tqpt, tdopt, tktb, tvtb, tkpt, tvpt, pq);
     note_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  a.marks.at(6, stream);
+  a.marks.at(5, stream);
   return cudaSuccess;
 }
 

@@ -3,12 +3,16 @@
 // operands with shared E8M0 scales, token-block scaling, leak guards,
 // document-local scales; GPT page secs. 3-6 for the attention itself).
 //
-// Operands come from the quantiser (prepass, stored in ctx for the backward):
-// Q per token (one scale per token x 32 channels), K and V in token-block form
-// (one scale per 32 tokens x 32 channels) and per-token form.  Leak guard
-// (rule L): a query of 32-token block b sees keys of earlier blocks through
-// the token-block forms and keys of its own block through the per-token forms,
-// so no shared scale pools a future token.
+// Fused quantisation: Q is quantised on load by this kernel (each query tile
+// is read by exactly one work item), per token for the scores, and written to
+// ctx in both forms for the backward; K and V, which every later query tile
+// of the document streams again, come from a prepass in token-block form (one
+// scale per 32 tokens x 32 channels) and per-token form (one scale per token x
+// 32 channels), and the diagonal tile's per-token V is dequantised on load for
+// its exact bf16 product.  Leak guard (rule L): a query of 32-token block b
+// sees keys of earlier blocks through the token-block forms and keys of its
+// own block through the per-token forms, so no shared scale pools a future
+// token.
 //
 // One persistent CTA per SM, 576 threads; work item = (document, 128-row
 // query tile, head).  Warps 0-15: one thread per (query row, 32-key block):
@@ -16,9 +20,11 @@
 // P~ (softmax, P quantisation, epilogue of O columns [32 wg, 32 wg + 32));
 // the four threads of a row exchange their block maxima through shared
 // memory (an mbarrier per row quarter, bounded waits) so they all move the
-// reference M alike, and add their partial row sums at the end.  Warp 16:
-// loads (TMA for codes, plain loads for the scale bytes, staged into the
-// 512-byte blocks tcgen05.cp copies to TMEM); warp 17 (one lane): MMAs.
+// reference M alike, and add their partial row sums at the end.  At the start
+// of an item the same threads, as (query row, 32-channel group), quantise the
+// item's Q and dequantise its diagonal V.  Warp 16: loads (TMA for K and V
+// codes, plain loads for their scale bytes, staged into the 512-byte blocks
+// tcgen05.cp copies to TMEM); warp 17 (one lane): MMAs.
 //  * S = Q K^T for every key tile: block-scaled FP8 MMA (kind::mxf8f6f4,
 //    E8M0 scales in TMEM) with K in token-block form; on the diagonal tile a
 //    second S with K per token, selected on the diagonal 32x32 blocks.
@@ -79,7 +85,13 @@ constexpr uint32_t kSfQ = 384, kSfK = 388, kSfKpt = 392, kSfP = 396, kSfV = 400;
 struct Params {
   const int32_t* cu;
   SchedView sched;
-  const uint8_t* q_spt;   // Q per-token scales [T][Hq][4]
+  const __nv_bfloat16* q;  // Q [T][Hq][128] (bf16 input, quantised on load)
+  uint8_t* q_vpt;          // out: Q per-token codes [T][Hq][128] (ctx)
+  uint8_t* q_spt;          // out: Q per-token scales [T][Hq][4]
+  uint8_t* q_vtb;          // out: Q token-block codes [T][Hq][128]
+  uint8_t* q_stb;          // out: Q token-block scales [slots][Hq][4]
+  const uint8_t* v_vpt;    // V per-token codes [T][Hkv][128] (diagonal tile)
+  const uint8_t* v_spt;    // V per-token scales [T][Hkv][4]
   const uint8_t* k_stb;   // K token-block scales [slots][Hkv][4]
   const uint8_t* k_spt;   // K per-token scales [T][Hkv][4]
   const uint8_t* v_stb;   // V token-block scales [slots][Hkv][4]
@@ -96,7 +108,7 @@ struct Params {
 };
 
 struct Item {
-  int doc, s, e, h, g, q0, n;  // n key tiles 0..n-1, tile n-1 is the diagonal
+  int doc, s, e, h, g, q0, m, n;  // query tile m; n = m + 1 key tiles, tile n-1 is the diagonal
 };
 
 __device__ __forceinline__ Item decode(const Params& p, const UnitInfo& un) {
@@ -108,14 +120,94 @@ __device__ __forceinline__ Item decode(const Params& p, const UnitInfo& un) {
   it.s = un.s;
   it.e = un.e;
   it.q0 = it.s + 128 * m;
+  it.m = m;
   it.n = m + 1;
   return it;
 }
 
+// Start of an item, one thread per (row, 32-channel group wg) of its 128 rows
+// (tokens q0 + row; rows past the document end are zeros and are not stored):
+//  * Q quantised per token into the MMA operand sQ (K-major FP8, 128-byte
+//    swizzle) and its scale block sfQ, and, for the backward, into ctx in
+//    per-token and token-block form (the warp's 32 rows are one
+//    document-local token block, since tiles start at the document start);
+//  * the diagonal tile's per-token V (its keys are the same tokens)
+//    dequantised to bf16 into sVpt (two 64-channel boxes, 128-byte swizzle).
+__device__ __forceinline__ void stage_item(const Params& p, const Item& it, int row, int wg, uint8_t* sQ,
+                                           uint8_t* sfQ, uint8_t* sVpt) {
+  const int t = it.q0 + row;
+  const bool in_doc = t < it.e;
+  float f[32];
+  uint4 vc[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  uint32_t vs = 127u;
+  if (in_doc) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)t * p.Hq + it.h) * 128 + 32 * wg);
+    uint4 raw[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) raw[c] = __ldg(src + c);
+    const uint4* vsrc = reinterpret_cast<const uint4*>(p.v_vpt + ((size_t)t * p.Hkv + it.g) * 128 + 32 * wg);
+    vc[0] = __ldg(vsrc);
+    vc[1] = __ldg(vsrc + 1);
+    vs = __ldg(p.v_spt + ((size_t)t * p.Hkv + it.g) * 4 + wg);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) unpack8(raw[c], *reinterpret_cast<float(*)[8]>(&f[8 * c]));
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) f[c] = 0.f;
+  }
+  // per-token form
+  float a = 0.f;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) a = fmaxf(a, fabsf(f[c]));
+  const int X = mx_block_exponent(a, p.rule);
+  uint2 cw[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) cw[c] = encode8(*reinterpret_cast<const float(*)[8]>(&f[8 * c]), X);
+  uint8_t* prow = sQ + row * 128;
+  *reinterpret_cast<uint4*>(prow + (((2 * wg) ^ (row & 7)) << 4)) = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+  *reinterpret_cast<uint4*>(prow + (((2 * wg + 1) ^ (row & 7)) << 4)) = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+  sfQ[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)(X + 127);
+  const size_t qo = ((size_t)t * p.Hq + it.h) * 128 + 32 * wg;
+  if (in_doc) {
+    uint4* dst = reinterpret_cast<uint4*>(p.q_vpt + qo);
+    dst[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+    dst[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+    p.q_spt[((size_t)t * p.Hq + it.h) * 4 + wg] = (uint8_t)(X + 127);
+  }
+  // token-block form: the warp's 32 rows, this channel group
+  float atb = a;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) atb = fmaxf(atb, __shfl_xor_sync(0xFFFFFFFFu, atb, off));
+  const int Xtb = mx_block_exponent(atb, p.rule);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) cw[c] = encode8(*reinterpret_cast<const float(*)[8]>(&f[8 * c]), Xtb);
+  if (in_doc) {
+    uint4* dst = reinterpret_cast<uint4*>(p.q_vtb + qo);
+    dst[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+    dst[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+  }
+  const int quarter = row >> 5;
+  if ((row & 31) == 0 && it.q0 + 32 * quarter < it.e) {
+    const size_t slot = (size_t)(it.s >> 5) + it.doc + 4 * it.m + quarter;
+    p.q_stb[(slot * p.Hq + it.h) * 4 + wg] = (uint8_t)(Xtb + 127);
+  }
+  // diagonal V: per-token codes -> bf16 (exact), channels 32 wg .. 32 wg + 31
+  const int Xv = (int)vs - 127;
+  const uint4 d0 = dequant8_bf16(make_uint2(vc[0].x, vc[0].y), Xv);
+  const uint4 d1 = dequant8_bf16(make_uint2(vc[0].z, vc[0].w), Xv);
+  const uint4 d2 = dequant8_bf16(make_uint2(vc[1].x, vc[1].y), Xv);
+  const uint4 d3 = dequant8_bf16(make_uint2(vc[1].z, vc[1].w), Xv);
+  uint8_t* vrow = sVpt + (wg >> 1) * kBox + row * 128;
+  const int c0 = (wg & 1) * 4;
+  *reinterpret_cast<uint4*>(vrow + (((c0 + 0) ^ (row & 7)) << 4)) = d0;
+  *reinterpret_cast<uint4*>(vrow + (((c0 + 1) ^ (row & 7)) << 4)) = d1;
+  *reinterpret_cast<uint4*>(vrow + (((c0 + 2) ^ (row & 7)) << 4)) = d2;
+  *reinterpret_cast<uint4*>(vrow + (((c0 + 3) ^ (row & 7)) << 4)) = d3;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    fwd_mxfp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ktb,
-                     const __grid_constant__ CUtensorMap tm_kpt, const __grid_constant__ CUtensorMap tm_vtb,
-                     const __grid_constant__ CUtensorMap tm_vpt16, const Params p) {
+    fwd_mxfp8_kernel(const __grid_constant__ CUtensorMap tm_ktb, const __grid_constant__ CUtensorMap tm_kpt,
+                     const __grid_constant__ CUtensorMap tm_vtb, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + oQ;
@@ -149,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 32);
+    mbar_init(q_full, 32 + kComputeWarps);  // the loader's lanes (K^pt) and the compute warps (Q, diagonal V)
     mbar_init(q_empty, 1);
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(kv_full + i, 32);
@@ -195,25 +287,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = decode(p, un);
       if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 51)) break;
       {
-        // scale blocks: row r = lane + 32 r1 -> bytes 16 lane + 4 r1 .. +3
-        uint4 wq, wk;
-        wq.x = pt_word(p.q_spt, it.q0 + lane, p.T, p.Hq, it.h);
-        wq.y = pt_word(p.q_spt, it.q0 + lane + 32, p.T, p.Hq, it.h);
-        wq.z = pt_word(p.q_spt, it.q0 + lane + 64, p.T, p.Hq, it.h);
-        wq.w = pt_word(p.q_spt, it.q0 + lane + 96, p.T, p.Hq, it.h);
+        // scale block of the diagonal per-token K: row r = lane + 32 r1 ->
+        // bytes 16 lane + 4 r1 .. +3 (Q and the diagonal V are staged by the
+        // compute warps)
+        uint4 wk;
         wk.x = pt_word(p.k_spt, it.q0 + lane, p.T, p.Hkv, it.g);
         wk.y = pt_word(p.k_spt, it.q0 + lane + 32, p.T, p.Hkv, it.g);
         wk.z = pt_word(p.k_spt, it.q0 + lane + 64, p.T, p.Hkv, it.g);
         wk.w = pt_word(p.k_spt, it.q0 + lane + 96, p.T, p.Hkv, it.g);
-        reinterpret_cast<uint4*>(sfQ)[lane] = wq;
         reinterpret_cast<uint4*>(sfKpt)[lane] = wk;
         fence_proxy_async_smem();
         if (lane == 0) {
-          mbar_arrive_expect_tx(q_full, 2 * kCodeTile + kBf16Tile);
-          tma_load_3d(sQ, &tm_q, q_full, 0, it.h, it.q0);
+          mbar_arrive_expect_tx(q_full, kCodeTile);
           tma_load_3d(sKpt, &tm_kpt, q_full, 0, it.g, it.q0);  // the diagonal key tile starts at q0
-          tma_load_3d(sVpt, &tm_vpt16, q_full, 0, it.g, it.q0);
-          tma_load_3d(sVpt + kBox, &tm_vpt16, q_full, 64, it.g, it.q0);
         } else {
           mbar_arrive(q_full);
         }
@@ -386,6 +472,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = decode(p, un);
       const int n = it.n;
       const int q_idx = it.q0 + row;
+      // the previous item's MMAs have completed (its epilogue waited for
+      // o_full), so sQ, sfQ and sVpt may be rewritten
+      stage_item(p, it, row, wg, smem + oQ, smem + oSf, smem + oVpt);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      warp_arrive(q_full);
       float M = -INFINITY, l = 0.f;  // l: this thread's share of the row sum
       for (int j = 0; j < n; ++j, ++tiles) {
         const int sbi = j & 1;
@@ -565,10 +657,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
-  CUtensorMap tq, tktb, tkpt, tvtb, tvpt;
-  if (!make_tmap_codes(&tq, a.q_vpt, a.T, a.Hq) || !make_tmap_codes(&tktb, a.k_vtb, a.T, a.Hkv) ||
-      !make_tmap_codes(&tkpt, a.k_vpt, a.T, a.Hkv) || !make_tmap_codes(&tvtb, a.v_vtb, a.T, a.Hkv) ||
-      !make_tmap_thd(&tvpt, a.v_deq_pt, a.T, a.Hkv, 128))
+  CUtensorMap tktb, tkpt, tvtb;
+  if (!make_tmap_codes(&tktb, a.k_vtb, a.T, a.Hkv) || !make_tmap_codes(&tkpt, a.k_vpt, a.T, a.Hkv) ||
+      !make_tmap_codes(&tvtb, a.v_vtb, a.T, a.Hkv))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -576,7 +667,13 @@ cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
   p.cu = a.cu;
   p.sched = sched_view(a.sched);
   p.cta_times = a.cta_times[0];
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.q_vpt = a.q_vpt;
   p.q_spt = a.q_spt;
+  p.q_vtb = a.q_vtb;
+  p.q_stb = a.q_stb;
+  p.v_vpt = a.v_vpt;
+  p.v_spt = a.v_spt;
   p.k_stb = a.k_stb;
   p.k_spt = a.k_spt;
   p.v_stb = a.v_stb;
@@ -594,7 +691,7 @@ cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
   p.wide = aligned32(a.o) && aligned32(a.o_resid);
   const long long max_units = (long long)a.sched.max_items * a.Hq;
   const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
-  fwd_mxfp8_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tktb, tkpt, tvtb, tvpt, p);
+  fwd_mxfp8_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tktb, tkpt, tvtb, p);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -64,6 +65,31 @@ cudaError_t launch_quantize_mxfp8(const void* x, int T, int H, int d, const int3
                                   int forms, int rule, uint8_t* vtb, uint8_t* stb, uint8_t* vpt,
                                   uint8_t* spt, cudaStream_t stream, void* deq_pt_bf16 = nullptr);
 
+// One tensor of a quantisation launch: bf16 x [T][H][d] and its forms.
+struct QuantJob {
+  const __nv_bfloat16* x;
+  int H;
+  uint8_t *vtb, *stb, *vpt, *spt;
+  __nv_bfloat16* deq;  // per-token form dequantised to bf16, or null
+};
+struct QuantJobs {
+  QuantJob job[2];
+};
+// D_i = dO_i . (o_i + o_resid_i), fp32 [Hq][T], computed by the quantisation
+// launch of dO (x = dO) in the same pass.
+struct DeltaArgs {
+  const __nv_bfloat16* o = nullptr;
+  const __nv_bfloat16* o_resid = nullptr;
+  float* delta = nullptr;
+  int T = 0;
+};
+// Up to two tensors of the same T and d in one launch (blockIdx.z = job).
+cudaError_t launch_quantize_jobs(const QuantJobs& jobs, int n_jobs, int T, int d, const int32_t* cu, int n_docs,
+                                 int forms, int rule, cudaStream_t stream);
+// dO: both forms, and D in the same read.
+cudaError_t launch_quantize_with_delta(const QuantJob& job, int T, int d, const int32_t* cu, int n_docs, int rule,
+                                       const DeltaArgs& da, cudaStream_t stream);
+
 // Per-CTA (start, end) %globaltimer records of one persistent kernel launch:
 // [0] = CTA count, then one pair per CTA (kMaxCtaTimes CTAs at most).
 constexpr int kMaxCtaTimes = 1024;
@@ -90,18 +116,24 @@ struct FwdArgs {
 };
 cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t stream);
 
-// Forward, MXFP8 path (fwd_mxfp8.cu): codes and scales from the quantiser.
+// Forward, MXFP8 path (fwd_mxfp8.cu): Q is quantised on load by the kernel
+// (and its forms written to ctx); K and V codes and scales come from the
+// quantiser's prepass.
 struct FwdMxArgs {
   unsigned long long* cta_times[2] = {nullptr, nullptr};  // per kernel, or null
-  const uint8_t* q_vpt;      // Q per-token codes [T][Hq][128]
-  const uint8_t* q_spt;      // Q per-token scales [T][Hq][4]
+  const void* q;             // Q bf16 [T][Hq][128], quantised on load
+  uint8_t* q_vpt;            // out: Q per-token codes [T][Hq][128]
+  uint8_t* q_spt;            // out: Q per-token scales [T][Hq][4]
+  uint8_t* q_vtb;            // out: Q token-block codes [T][Hq][128]
+  uint8_t* q_stb;            // out: Q token-block scales [T/32 + n_docs][Hq][4]
   const uint8_t* k_vtb;      // K token-block codes [T][Hkv][128]
   const uint8_t* k_stb;      // K token-block scales [T/32 + n_docs][Hkv][4]
   const uint8_t* k_vpt;      // K per-token codes
   const uint8_t* k_spt;      // K per-token scales
   const uint8_t* v_vtb;      // V token-block codes
   const uint8_t* v_stb;      // V token-block scales
-  const void* v_deq_pt;      // V per-token form dequantised to bf16 [T][Hkv][128]
+  const uint8_t* v_vpt;      // V per-token codes (diagonal tiles, dequantised on load)
+  const uint8_t* v_spt;      // V per-token scales
   void* o;
   float* lse;
   void* o_resid;
@@ -122,8 +154,7 @@ struct BwdMxArgs {
   const uint8_t *q_vtb, *q_stb, *q_vpt, *q_spt;     // quantised Q (ctx)
   const uint8_t *k_vtb, *k_stb, *k_vpt, *k_spt;     // quantised K (ctx)
   const uint8_t *v_vtb, *v_stb, *v_vpt, *v_spt;     // quantised V (ctx)
-  const uint8_t *do_vtb, *do_stb, *do_vpt, *do_spt; // quantised dO (workspace)
-  const void* k_deq_pt;                             // K per-token form dequantised to bf16 (ctx)
+  const uint8_t *do_vtb, *do_stb, *do_vpt, *do_spt; // quantised dO (workspace; written by the D pass)
   const void* o;
   const void* o_resid;
   const float* lse;
@@ -133,7 +164,7 @@ struct BwdMxArgs {
   void* dv;
   float* delta;
   const int32_t* cu;
-  int T, Hq, Hkv;
+  int T, Hq, Hkv, n_docs;
   float scale;
   int grad_bf16;
   int rule;

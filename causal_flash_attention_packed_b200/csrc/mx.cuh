@@ -62,6 +62,41 @@ __device__ __forceinline__ void mx_decode2(uint32_t c2, float& lo, float& hi) {
   hi = __high2float(h);
 }
 
+// Eight values -> eight codes with scale exponent X.
+__device__ __forceinline__ uint2 encode8(const float (&f)[8], int X) {
+  const float s = mx_pow2_neg(X);
+  uint32_t a = mx_e4m3x2(f[0] * s, f[1] * s) | (mx_e4m3x2(f[2] * s, f[3] * s) << 16);
+  uint32_t b = mx_e4m3x2(f[4] * s, f[5] * s) | (mx_e4m3x2(f[6] * s, f[7] * s) << 16);
+  return make_uint2(mx_canon_zero(a), mx_canon_zero(b));
+}
+
+// Dequantised values decode(code) * 2^X of eight codes, as bf16 (exact for
+// every value within the bf16 range).
+__device__ __forceinline__ uint4 dequant8_bf16(uint2 codes, int X) {
+  const float sc = mx_pow2(X < -126 ? -126 : X);
+  const float extra = X < -126 ? 0.5f : 1.f;  // X = -127 only for all-zero blocks
+  const uint32_t w[2] = {codes.x, codes.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float a, b, c, d;
+    mx_decode2(w[i] & 0xFFFFu, a, b);
+    mx_decode2(w[i] >> 16, c, d);
+    o[2 * i] = pack_bf16x2(a * sc * extra, b * sc * extra);
+    o[2 * i + 1] = pack_bf16x2(c * sc * extra, d * sc * extra);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
 // Instruction descriptor of kind::mxf8f6f4.block_scale with E4M3 A and B,
 // E8M0 scales, fp32 accumulation: [4,6) B scale-factor id, [7,10) A format
 // (0 = E4M3), [10,13) B format, bit 15 A major, bit 16 B major (1 = MN),

@@ -138,10 +138,13 @@ typedef struct {
                                     records on its stream before each of its kernel launches
                                     and after the last one (entries beyond n_timing_events or
                                     NULL are skipped).  fapk_attn_fwd: [0] schedule, [1] fp16
-                                    copy of V, [2] forward kernel, [3] end.  fapk_attn_bwd:
+                                    copy of V (FAPK_MXFP8: MX quantisation of K and V),
+                                    [2] forward kernel, [3] end.  fapk_attn_bwd, FAPK_BF16:
                                     [0] key-tile schedule, [1] query-tile schedule, [2] fp16
                                     copy of K, [3] D and fp16 dO/Q, [4] dK/dV kernel, [5] dQ
-                                    kernel, [6] end. */
+                                    kernel, [6] end; FAPK_MXFP8: [0] key-tile schedule,
+                                    [1] query-tile schedule, [2] D and MX quantisation of dO,
+                                    [3] dK/dV kernel, [4] dQ kernel, [5] end. */
   int n_timing_events;
 } fapk_problem_t;
 
@@ -154,8 +157,9 @@ FAPK_API size_t fapk_workspace_size(const fapk_problem_t* prob, int which);
 /* Bytes of the saved-state buffer `ctx` that the forward fills and the
  * backward reads.  It holds the bf16 rounding residual of O (O_fp32 minus its
  * bf16 rounding, [T][Hq][d] bf16), so that the backward's D_i = dO_i . O_i
- * sees O to about 16 significant bits; the MXFP8 path adds its quantised
- * token-block operands, reused across orientations (FLAMIA page: "token-block
+ * sees O to about 16 significant bits; the bf16 path adds an fp16 copy of V,
+ * the MXFP8 path the MX forms (codes and scales, token-block and per-token) of
+ * Q, K and V, reused across orientations (FLAMIA page: "token-block
  * scaling"). */
 FAPK_API size_t fapk_ctx_size(const fapk_problem_t* prob);
 
