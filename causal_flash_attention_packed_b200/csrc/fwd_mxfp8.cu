@@ -73,8 +73,9 @@ constexpr int kSfBlk = 512;
 constexpr int oXmax = oSf + (3 + kSlots) * kSfBlk;  // block maxima [2][4][128] (by tile parity)
 constexpr int oLsum = oXmax + 2 * 4 * 128 * 4;       // partial row sums [4][128]
 constexpr int oBars = oLsum + 4 * 128 * 4;
-// + one row-exchange barrier per row quarter, the unit ring's full[8] and empty[8]
-constexpr int kNumBars = 2 + 2 * kSlots + 8 + 4 + 2 * kUnitRing;
+// q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full, pv_done, o_full, o_free, fin,
+// one row-exchange barrier per row quarter, kpt_full, vd_full, the unit ring's full[8] and empty[8]
+constexpr int kNumBars = 2 + 2 * kSlots + 13 + 2 * kUnitRing;
 constexpr int kSmemBytes = oBars + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may use");
 
@@ -125,30 +126,34 @@ __device__ __forceinline__ Item decode(const Params& p, const UnitInfo& un) {
   return it;
 }
 
-// Start of an item, one thread per (row, 32-channel group wg) of its 128 rows
-// (tokens q0 + row; rows past the document end are zeros and are not stored):
-//  * Q quantised per token into the MMA operand sQ (K-major FP8, 128-byte
-//    swizzle) and its scale block sfQ, and, for the backward, into ctx in
-//    per-token and token-block form (the warp's 32 rows are one
+// Per item, one thread per (row, 32-channel group wg) of its 128 rows (tokens
+// q0 + row; rows past the document end are zeros and are not stored):
+//  * stage_q: Q quantised per token into the MMA operand sQ (K-major FP8,
+//    128-byte swizzle) and its scale block sfQ, and, for the backward, into
+//    ctx in per-token and token-block form (the warp's 32 rows are one
 //    document-local token block, since tiles start at the document start);
-//  * the diagonal tile's per-token V (its keys are the same tokens)
-//    dequantised to bf16 into sVpt (two 64-channel boxes, 128-byte swizzle).
-__device__ __forceinline__ void stage_item(const Params& p, const Item& it, int row, int wg, uint8_t* sQ,
-                                           uint8_t* sfQ, uint8_t* sVpt) {
+//  * stage_v: the diagonal tile's per-token V (its keys are the same tokens)
+//    dequantised to bf16 into sVpt (two 64-channel boxes, 128-byte swizzle);
+//  * prefetch: the item's Q row and diagonal V codes into L2, ahead of both.
+__device__ __forceinline__ void prefetch_item(const Params& p, const Item& it, int row, int wg) {
+  const int t = it.q0 + row;
+  if (t >= it.e) return;
+  const __nv_bfloat16* q = p.q + ((size_t)t * p.Hq + it.h) * 128 + 32 * wg;
+  const uint8_t* v = p.v_vpt + ((size_t)t * p.Hkv + it.g) * 128 + 32 * wg;
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(q));
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(v));
+}
+
+__device__ __forceinline__ void stage_q(const Params& p, const Item& it, int row, int wg, uint8_t* sQ,
+                                        uint8_t* sfQ) {
   const int t = it.q0 + row;
   const bool in_doc = t < it.e;
   float f[32];
-  uint4 vc[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-  uint32_t vs = 127u;
   if (in_doc) {
     const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)t * p.Hq + it.h) * 128 + 32 * wg);
     uint4 raw[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) raw[c] = __ldg(src + c);
-    const uint4* vsrc = reinterpret_cast<const uint4*>(p.v_vpt + ((size_t)t * p.Hkv + it.g) * 128 + 32 * wg);
-    vc[0] = __ldg(vsrc);
-    vc[1] = __ldg(vsrc + 1);
-    vs = __ldg(p.v_spt + ((size_t)t * p.Hkv + it.g) * 4 + wg);
 #pragma unroll
     for (int c = 0; c < 4; ++c) unpack8(raw[c], *reinterpret_cast<float(*)[8]>(&f[8 * c]));
   } else {
@@ -191,7 +196,19 @@ __device__ __forceinline__ void stage_item(const Params& p, const Item& it, int 
     const size_t slot = (size_t)(it.s >> 5) + it.doc + 4 * it.m + quarter;
     p.q_stb[(slot * p.Hq + it.h) * 4 + wg] = (uint8_t)(Xtb + 127);
   }
-  // diagonal V: per-token codes -> bf16 (exact), channels 32 wg .. 32 wg + 31
+}
+
+__device__ __forceinline__ void stage_v(const Params& p, const Item& it, int row, int wg, uint8_t* sVpt) {
+  const int t = it.q0 + row;
+  uint4 vc[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  uint32_t vs = 127u;
+  if (t < it.e) {
+    const uint4* vsrc = reinterpret_cast<const uint4*>(p.v_vpt + ((size_t)t * p.Hkv + it.g) * 128 + 32 * wg);
+    vc[0] = __ldg(vsrc);
+    vc[1] = __ldg(vsrc + 1);
+    vs = __ldg(p.v_spt + ((size_t)t * p.Hkv + it.g) * 4 + wg);
+  }
+  // per-token codes -> bf16 (exact), channels 32 wg .. 32 wg + 31
   const int Xv = (int)vs - 127;
   const uint4 d0 = dequant8_bf16(make_uint2(vc[0].x, vc[0].y), Xv);
   const uint4 d1 = dequant8_bf16(make_uint2(vc[0].z, vc[0].w), Xv);
@@ -234,6 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_free = s_full + 5;
   uint64_t* fin = s_full + 6;
   uint64_t* xbar = s_full + 7;  // [4]
+  uint64_t* kpt_full = s_full + 11;  // the diagonal per-token K and its scales (loader)
+  uint64_t* vd_full = s_full + 12;   // the diagonal V dequantised to bf16 (compute warps)
   const UnitRing ring{reinterpret_cast<int*>(bars + kNumBars) + 4, bars + kNumBars - 2 * kUnitRing,
                       bars + kNumBars - kUnitRing};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
@@ -241,7 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 32 + kComputeWarps);  // the loader's lanes (K^pt) and the compute warps (Q, diagonal V)
+    mbar_init(q_full, kComputeWarps);  // Q staged by the compute warps
+    mbar_init(kpt_full, 32);
+    mbar_init(vd_full, kComputeWarps);
     mbar_init(q_empty, 1);
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(kv_full + i, 32);
@@ -277,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ loads
-    uint32_t kv_it = 0;
+    uint32_t kv_it = 0, kpt_loads = 0;
     int unit_i = 0;
     bool ok = true;
     for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
@@ -285,25 +306,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int w = un.w;
       if (w < 0 || w >= n_units) break;
       const Item it = decode(p, un);
-      if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 51)) break;
-      {
-        // scale block of the diagonal per-token K: row r = lane + 32 r1 ->
-        // bytes 16 lane + 4 r1 .. +3 (Q and the diagonal V are staged by the
-        // compute warps)
-        uint4 wk;
-        wk.x = pt_word(p.k_spt, it.q0 + lane, p.T, p.Hkv, it.g);
-        wk.y = pt_word(p.k_spt, it.q0 + lane + 32, p.T, p.Hkv, it.g);
-        wk.z = pt_word(p.k_spt, it.q0 + lane + 64, p.T, p.Hkv, it.g);
-        wk.w = pt_word(p.k_spt, it.q0 + lane + 96, p.T, p.Hkv, it.g);
-        reinterpret_cast<uint4*>(sfKpt)[lane] = wk;
-        fence_proxy_async_smem();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(q_full, kCodeTile);
-          tma_load_3d(sKpt, &tm_kpt, q_full, 0, it.g, it.q0);  // the diagonal key tile starts at q0
-        } else {
-          mbar_arrive(q_full);
-        }
-      }
       for (int j = 0; j < it.n && ok; ++j) {
         for (int kv = 0; kv < 2; ++kv, ++kv_it) {
           const int slot = kv_it % kSlots;
@@ -338,10 +340,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(kv_full + slot);
           }
         }
+        if (j == it.n - 1 && ok) {
+          // the diagonal per-token K and its scale block (row r = lane + 32 r1
+          // -> bytes 16 lane + 4 r1 .. +3), once every MMA of the previous
+          // item has read the previous ones; after the item's last K and V
+          // (the per-token scores come last), so that the item's streamed
+          // tiles never wait for the previous item to finish
+          if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 51)) { ok = false; break; }
+          uint4 wk;
+          wk.x = pt_word(p.k_spt, it.q0 + lane, p.T, p.Hkv, it.g);
+          wk.y = pt_word(p.k_spt, it.q0 + lane + 32, p.T, p.Hkv, it.g);
+          wk.z = pt_word(p.k_spt, it.q0 + lane + 64, p.T, p.Hkv, it.g);
+          wk.w = pt_word(p.k_spt, it.q0 + lane + 96, p.T, p.Hkv, it.g);
+          reinterpret_cast<uint4*>(sfKpt)[lane] = wk;
+          fence_proxy_async_smem();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(kpt_full, kCodeTile);
+            tma_load_3d(sKpt, &tm_kpt, kpt_full, 0, it.g, it.q0);  // the diagonal key tile starts at q0
+          } else {
+            mbar_arrive(kpt_full);
+          }
+          ++kpt_loads;
+        }
       }
     }
     if (lane == 0) {
-      if (unit_i > 0) drain_wait(q_full, (unit_i - 1) & 1, p.timeout_ns);
+      if (kpt_loads > 0) drain_wait(kpt_full, (kpt_loads - 1) & 1, p.timeout_ns);
       for (uint32_t i = (kv_it > kSlots ? kv_it - kSlots : 0); i < kv_it; ++i)
         drain_wait(kv_full + (i % kSlots), (i / kSlots) & 1, p.timeout_ns);
     }
@@ -384,12 +408,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(q_full, unit_i & 1, wd, 54)) break;
         tc_fence_after();
         tmem_cp_sf(tmem + kSfQ, asf);
-        tmem_cp_sf(tmem + kSfKpt, asf + kSfBlk);
+        // the diagonal per-token K (and its scales) arrive on their own barrier
+        auto wait_kpt = [&]() {
+          if (!mbar_wait(kpt_full, unit_i & 1, wd, 61)) return false;
+          tc_fence_after();
+          tmem_cp_sf(tmem + kSfKpt, asf + kSfBlk);
+          return true;
+        };
         // prologue: S(0) (+ per-token S if tile 0 is the diagonal), S(1)
         if (!wait_slot(0, 0)) break;
         tc_fence_after();
         issue_s_tile(0, kS0);
-        if (n == 1) issue_s(kS1, akpt, kSfKpt);
+        if (n == 1) {
+          if (!wait_kpt()) break;
+          issue_s(kS1, akpt, kSfKpt);
+        }
         tc_commit(s_full + 0);
         tc_commit(kv_empty + kslot_of(0));
         if (n >= 2) {
@@ -416,6 +449,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         (j > 0 || kk > 0) ? 1u : 0u);
           if (j == n - 1) {
             // diagonal 32x32 blocks: exact bf16 P~ times dequantised per-token V
+            if (!mbar_wait(vd_full, unit_i & 1, wd, 62)) { ok = false; break; }
+            tc_fence_after();
             constexpr uint32_t idesc_d = idesc_bf16_f32(128, 128, false, true);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
@@ -437,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (j == n - 2) {
             // per-token S of the diagonal tile, into the buffer tile n-2 freed
+            if (!wait_kpt()) { ok = false; break; }
             issue_s((j & 1) ? kS1 : kS0, akpt, kSfKpt);
             tc_commit(s_full + ((j + 1) & 1));  // signals tile n-1 = j+1
           }
@@ -465,21 +501,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     uint32_t s_cnt[2] = {0, 0}, pv_cnt = 0, o_cnt = 0, tiles = 0;
     bool ok = true;
-    for (uint32_t uk = 0; ok; ++uk) {
-      const UnitInfo un = unit_take_warp(ring, uk, wd);
-      const int w = un.w;
-      if (w < 0 || w >= n_units) break;
-      const Item it = decode(p, un);
-      const int n = it.n;
-      const int q_idx = it.q0 + row;
-      // the previous item's MMAs have completed (its epilogue waited for
-      // o_full), so sQ, sfQ and sVpt may be rewritten
-      stage_item(p, it, row, wg, smem + oQ, smem + oSf, smem + oVpt);
+    // Q of an item is staged before the previous item's epilogue (its first
+    // scores then overlap that epilogue), its diagonal V after it (the
+    // previous item's last P V reads sVpt until o_full)
+    uint32_t uk = 0;
+    UnitInfo un = unit_take_warp(ring, uk++, wd);
+    bool have = un.w >= 0 && un.w < n_units;
+    if (have) {
+      stage_q(p, decode(p, un), row, wg, smem + oQ, smem + oSf);
       fence_proxy_async_smem();
       tc_fence_before();
       warp_arrive(q_full);
+    }
+    while (have && ok) {
+      const Item it = decode(p, un);
+      const int n = it.n;
+      const int q_idx = it.q0 + row;
+      stage_v(p, it, row, wg, smem + oVpt);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      warp_arrive(vd_full);
+      UnitInfo nx{-1, 0, 0, 0, 0, 0};
+      bool have_next = false;
       float M = -INFINITY, l = 0.f;  // l: this thread's share of the row sum
       for (int j = 0; j < n; ++j, ++tiles) {
+        if (j == n - 1) {
+          // the next item, taken now so that its Q reaches L2 during this tile
+          nx = unit_take_warp(ring, uk++, wd);
+          have_next = nx.w >= 0 && nx.w < n_units;
+          if (have_next) prefetch_item(p, decode(p, nx), row, wg);
+        }
         const int sbi = j & 1;
         if (!warp_wait(s_full + sbi, (sbi ? s_cnt[1] : s_cnt[0]) & 1, wd, 57)) { ok = false; break; }
         if (sbi) ++s_cnt[1]; else ++s_cnt[0];
@@ -601,6 +652,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         warp_arrive(p_full);
       }
       if (!ok) break;
+      if (have_next) {
+        // every S MMA of this item has completed (its last scores were read
+        // above), so sQ and sfQ may take the next item's Q
+        stage_q(p, decode(p, nx), row, wg, smem + oQ, smem + oSf);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        warp_arrive(q_full);
+      }
       // epilogue: the row sum from the four block shares, O columns [32 wg, 32 wg + 32)
       lsum[wg * 128 + row] = l;
       if (!row_sync()) break;
@@ -644,6 +703,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       warp_arrive(o_free);
       if (valid && wg == 0) p.lse[(size_t)it.h * p.T + q_idx] = (M + __log2f(lt)) * kLn2;
+      un = nx;
+      have = have_next;
     }
   }
 
