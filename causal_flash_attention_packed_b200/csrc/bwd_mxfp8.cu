@@ -524,30 +524,23 @@ namespace kvk {
 // block wg of every tile (one MX scale block of P~T and dS~T); warp 16: K/V,
 // Q^pt, dO^pt, lse and D loads; warp 17: MMA issue; warp 18: dO^tb and Q^tb loads
 constexpr int kThreads = 608, kLoadA = 16, kMma = 17, kLoadB = 18, kComputeWarps = 16;
-// per item: K^tb, K^pt, V^tb, V^pt codes; per query tile the operands Q^pt,
-// dO^pt, dO^tb, Q^tb (codes), each released as soon as its last MMA has read
-// it: Q^pt, dO^pt and dO^tb in two buffers each (tile t in buffer t & 1), so
-// that the next tile's copy is in flight while this tile's MMAs read the
-// other buffer, Q^tb (read last) in one; P~T and dS~T codes; lse*log2e[128]
-// and D[128] of the query tile in two buffers
-constexpr int kQpt = 0, kDOpt = 1, kDOtb = 2, kQtb = 3;  // operands, in the order the MMAs release them
-constexpr int kNumOpBufs = 7;                            // buffers: Qpt x2, dOpt x2, dOtb x2, Qtb
-__host__ __device__ constexpr int op_nbuf(int op) { return op == kQtb ? 1 : 2; }
-__host__ __device__ constexpr int op_first(int op) { return 2 * op; }  // first buffer index of an operand
+// per item: K^tb, K^pt, V^tb, V^pt codes; per query tile one buffer per
+// operand (Q^pt, dO^pt, dO^tb, Q^tb codes), each released as soon as its last
+// MMA has read it; P~T and dS~T codes; lse*log2e[128] and D[128] of the query
+// tile in two buffers
 constexpr int oKtb = 0, oKpt = oKtb + kCode, oVtb = oKpt + kCode, oVpt = oVtb + kCode;
-constexpr int oOps = oVpt + kCode;  // kNumOpBufs code buffers
-constexpr int oP = oOps + kNumOpBufs * kCode, oDS = oP + kCode;
+constexpr int oQpt = oVpt + kCode, oDOpt = oQpt + kCode, oDOtb = oDOpt + kCode, oQtb = oDOtb + kCode;
+constexpr int oP = oQtb + kCode, oDS = oP + kCode;
 constexpr int oAux = oDS + kCode;
 constexpr int oSf = oAux + 2 * 1024;
-// scale blocks: 0 Ktb, 1 Kpt, 2 Vtb, 3 Vpt, 4..10 the operand buffers (dOtb and Qtb by channel rows), 11 P, 12 dS
-constexpr int kSfOp = 4, kSfP = kSfOp + kNumOpBufs, kSfDS = kSfP + 1;
-constexpr int kNumSf = kSfDS + 1;
+// scale blocks: 0 Ktb, 1 Kpt, 2 Vtb, 3 Vpt, 4 Qpt, 5 dOpt, 6 dOtb (channel rows), 7 Qtb (channel rows), 8 P, 9 dS
+constexpr int kNumSf = 10;
 constexpr int oBars = oSf + kNumSf * kSfBlk;
-constexpr int bKvFull = 0, bKvEmpty = 1, bOpFull = 2, bOpEmpty = bOpFull + kNumOpBufs, bAuxFull = bOpEmpty + kNumOpBufs,
-              bAuxEmpty = bAuxFull + 2, bSFull = bAuxEmpty + 2, bSFree = bSFull + 1, bPFull = bSFree + 1,
-              bPEmpty = bPFull + 1, bDsFull = bPEmpty + 1, bDsEmpty = bDsFull + 1, bAccFull = bDsEmpty + 1,
-              bAccFree = bAccFull + 1, bFin = bAccFree + 1, bRing = bFin + 1,
-              kNumBars = bRing + 2 * kUnitRing;  // the unit ring's full[], empty[] from bRing
+// operand buffers, in the order the MMAs release them
+constexpr int kQpt = 0, kDOpt = 1, kDOtb = 2, kQtb = 3;
+constexpr int bKvFull = 0, bKvEmpty = 1, bOpFull = 2, bOpEmpty = 6, bAuxFull = 10, bAuxEmpty = 12, bSFull = 14,
+              bSFree = 15, bPFull = 16, bPEmpty = 17, bDsFull = 18, bDsEmpty = 19, bAccFull = 20, bAccFree = 21,
+              bFin = 22, bRing = 23, kNumBars = bRing + 2 * kUnitRing;  // the unit ring's full[], empty[] from bRing
 constexpr int kSmem = oBars + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
 static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may use");
 // TMEM: one 128-column region that holds S^T and dP^T in turn (each read out
@@ -593,7 +586,7 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 32);
     mbar_init(kv_empty, 1);
-    for (int i = 0; i < kNumOpBufs; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(op_full + i, 32);  // lane 0's expect_tx arrive + 31 lanes after their scale stores
       mbar_init(op_empty + i, 1);
     }
@@ -639,29 +632,20 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     k0 = s + 128 * v;
     nq = (e - s + 127) / 128;
   };
-  // buffer of operand `op` for query tile t, and the use count of that buffer
-  auto op_buf = [](int op, uint32_t t) { return op_first(op) + (op_nbuf(op) == 2 ? (int)(t & 1) : 0); };
-  auto op_use = [](int op, uint32_t t) { return op_nbuf(op) == 2 ? t >> 1 : t; };
-  // one operand buffer of query tile t: wait until the MMAs of its previous use
-  // released it, store its scale block, then copy the codes
+  // one operand buffer of query tile t: wait until the MMAs of tile t - 1 released
+  // it, store its scale block, then copy the codes
   auto load_op = [&](int op, uint32_t t, const CUtensorMap* tm, int h, int q0, const uint4& sfw, int where) {
-    const int b = op_buf(op, t);
-    const uint32_t u = op_use(op, t);
-    if (u > 0 && !warp_wait(op_empty + b, (u - 1) & 1, wd, where)) return false;
-    reinterpret_cast<uint4*>(sfb(kSfOp + b))[lane] = sfw;
+    if (t > 0 && !warp_wait(op_empty + op, (t - 1) & 1, wd, where)) return false;
+    reinterpret_cast<uint4*>(sfb(4 + op))[lane] = sfw;
     fence_proxy_async_smem();
+    const int off = op == kQpt ? oQpt : op == kDOpt ? oDOpt : op == kDOtb ? oDOtb : oQtb;
     if (lane == 0) {
-      mbar_arrive_expect_tx(op_full + b, kCode);
-      tma_load_3d(smem + oOps + b * kCode, tm, op_full + b, 0, h, q0);
+      mbar_arrive_expect_tx(op_full + op, kCode);
+      tma_load_3d(smem + off, tm, op_full + op, 0, h, q0);
     } else {
-      mbar_arrive(op_full + b);
+      mbar_arrive(op_full + op);
     }
     return true;
-  };
-  // teardown: let the last copy of every buffer of `op` land
-  auto drain_op = [&](int op, uint32_t t_end) {
-    for (uint32_t t = (t_end > (uint32_t)op_nbuf(op) ? t_end - op_nbuf(op) : 0); t < t_end; ++t)
-      drain_wait(op_full + op_buf(op, t), op_use(op, t) & 1, p.timeout_ns);
   };
 
   if (warp == kLoadA) {
@@ -717,8 +701,10 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     }
     if (lane == 0) {
       if (unit_i > 0) drain_wait(kv_full, (unit_i - 1) & 1, p.timeout_ns);
-      drain_op(kQpt, t);
-      drain_op(kDOpt, t);
+      if (t > 0) {
+        drain_wait(op_full + kQpt, (t - 1) & 1, p.timeout_ns);
+        drain_wait(op_full + kDOpt, (t - 1) & 1, p.timeout_ns);
+      }
     }
   } else if (warp == kLoadB) {
     // ------------------------------------------------- dO^tb, Q^tb
@@ -740,20 +726,17 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
         }
       }
     }
-    if (lane == 0) {
-      drain_op(kDOtb, t);
-      drain_op(kQtb, t);
+    if (lane == 0 && t > 0) {
+      drain_wait(op_full + kDOtb, (t - 1) & 1, p.timeout_ns);
+      drain_wait(op_full + kQtb, (t - 1) & 1, p.timeout_ns);
     }
   } else if (warp == kMma) {
     // ------------------------------------------------- MMA issue
     if (lane == 0) {
       const uint32_t aKtb = smem_u32(smem + oKtb), aKpt = smem_u32(smem + oKpt), aVtb = smem_u32(smem + oVtb),
-                     aVpt = smem_u32(smem + oVpt), aOps = smem_u32(smem + oOps), aP = smem_u32(smem + oP),
+                     aVpt = smem_u32(smem + oVpt), aQpt = smem_u32(smem + oQpt), aQtb = smem_u32(smem + oQtb),
+                     aDOpt = smem_u32(smem + oDOpt), aDOtb = smem_u32(smem + oDOtb), aP = smem_u32(smem + oP),
                      aDS = smem_u32(smem + oDS), aSf = smem_u32(sf);
-      // codes and scale block of operand `op` for query tile tt
-      auto op_addr = [&](int op, uint32_t tt) { return aOps + op_buf(op, tt) * kCode; };
-      auto op_sf = [&](int op, uint32_t tt) { return aSf + (kSfOp + op_buf(op, tt)) * kSfBlk; };
-      auto op_release = [&](int op, uint32_t tt) { tc_commit(op_empty + op_buf(op, tt)); };
       uint32_t t = 0, s_uses = 0;
       int unit_i = 0;
       bool ok = true;
@@ -777,16 +760,16 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
         ++s_uses;
       };
       auto wait_op = [&](int op, uint32_t tt, int where) {
-        if (!mbar_wait(op_full + op_buf(op, tt), op_use(op, tt) & 1, wd, where)) return false;
+        if (!mbar_wait(op_full + op, tt & 1, wd, where)) return false;
         tc_fence_after();
         return true;
       };
       // S^T of tile tt with token-block K (every key block of the tile)
       auto s_tb = [&](uint32_t tt) {
         if (!wait_op(kQpt, tt, 88)) return false;
-        tmem_cp_sf(tmem + tSfQpt, op_sf(kQpt, tt));
+        tmem_cp_sf(tmem + tSfQpt, aSf + 4 * kSfBlk);
         if (!region()) return false;
-        mx_kk(tSD, aKtb, op_addr(kQpt, tt), tSfKtb, tSfQpt, false, false);
+        mx_kk(tSD, aKtb, aQpt, tSfKtb, tSfQpt, false, false);
         region_done();
         return true;
       };
@@ -813,31 +796,31 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
             // diagonal tile: S^T again with the per-token K; the compute warps
             // take its diagonal 32x32 blocks
             if (!region()) { ok = false; break; }
-            mx_kk(tSD, aKpt, op_addr(kQpt, t), tSfKpt, tSfQpt, false, false);
+            mx_kk(tSD, aKpt, aQpt, tSfKpt, tSfQpt, false, false);
             region_done();
           }
-          op_release(kQpt, t);
+          tc_commit(op_empty + kQpt);
           // dP^T (token-block V), on the diagonal tile then the per-token V
           if (!wait_op(kDOpt, t, 91)) { ok = false; break; }
-          tmem_cp_sf(tmem + tSfDOpt, op_sf(kDOpt, t));
+          tmem_cp_sf(tmem + tSfDOpt, aSf + 5 * kSfBlk);
           if (!region()) { ok = false; break; }
-          mx_kk(tSD, aVtb, op_addr(kDOpt, t), tSfVtb, tSfDOpt, false, false);
+          mx_kk(tSD, aVtb, aDOpt, tSfVtb, tSfDOpt, false, false);
           region_done();
           if (diag) {
             if (!region()) { ok = false; break; }
-            mx_kk(tSD, aVpt, op_addr(kDOpt, t), tSfVpt, tSfDOpt, false, false);
+            mx_kk(tSD, aVpt, aDOpt, tSfVpt, tSfDOpt, false, false);
             region_done();
           }
-          op_release(kDOpt, t);
+          tc_commit(op_empty + kDOpt);
           if (last) tc_commit(kv_empty);  // the item's last read of K and V has been issued
           // dV += P~T dO~tb
           if (!mbar_wait(p_full, t & 1, wd, 92)) { ok = false; break; }
           if (!wait_op(kDOtb, t, 93)) { ok = false; break; }
-          tmem_cp_sf(tmem + tSfP, aSf + kSfP * kSfBlk);
-          tmem_cp_sf(tmem + tSfDOtb, op_sf(kDOtb, t));
-          mx_kk(tDV, aP, op_addr(kDOtb, t), tSfP, tSfDOtb, true, r > 0);
+          tmem_cp_sf(tmem + tSfP, aSf + 8 * kSfBlk);
+          tmem_cp_sf(tmem + tSfDOtb, aSf + 6 * kSfBlk);
+          mx_kk(tDV, aP, aDOtb, tSfP, tSfDOtb, true, r > 0);
           tc_commit(p_empty);
-          op_release(kDOtb, t);
+          tc_commit(op_empty + kDOtb);
           // the next tile's S^T goes ahead of dK, so that it is ready when the
           // compute warps finish dS~ of this tile
           ahead = false;
@@ -848,11 +831,11 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           // dK += dS~T Q~tb
           if (!mbar_wait(ds_full, t & 1, wd, 94)) { ok = false; break; }
           if (!wait_op(kQtb, t, 95)) { ok = false; break; }
-          tmem_cp_sf(tmem + tSfDS, aSf + kSfDS * kSfBlk);
-          tmem_cp_sf(tmem + tSfQtb, op_sf(kQtb, t));
-          mx_kk(tDK, aDS, op_addr(kQtb, t), tSfDS, tSfQtb, true, r > 0);
+          tmem_cp_sf(tmem + tSfDS, aSf + 9 * kSfBlk);
+          tmem_cp_sf(tmem + tSfQtb, aSf + 7 * kSfBlk);
+          mx_kk(tDK, aDS, aQtb, tSfDS, tSfQtb, true, r > 0);
           tc_commit(ds_empty);
-          op_release(kQtb, t);
+          tc_commit(op_empty + kQtb);
         }
         if (!ok) break;
         tc_commit(acc_full);
@@ -868,8 +851,8 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     const uint32_t lb = tmem + ((uint32_t)(quarter * 32) << 16);
     uint8_t* sP = smem + oP;
     uint8_t* sDS = smem + oDS;
-    uint8_t* sfP = sfb(kSfP);
-    uint8_t* sfDS = sfb(kSfDS);
+    uint8_t* sfP = sfb(8);
+    uint8_t* sfDS = sfb(9);
     uint32_t s_cnt = 0, t = 0;
     int unit_i = 0;
     bool ok = true;
