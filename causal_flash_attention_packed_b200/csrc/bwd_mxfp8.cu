@@ -684,8 +684,8 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const int i = q0 + lane * 4 + r;
-            const bool in = i < e;  // queries past the document end get P = 0 (lse2 = +inf)
-            l4[r] = in ? p.lse[(size_t)h * p.T + i] * kLog2e : INFINITY;
+            const bool in = i < e;  // queries past the document end get P = 0 (-lse log2 e = -inf)
+            l4[r] = in ? -p.lse[(size_t)h * p.T + i] * kLog2e : -INFINITY;
             d4[r] = in ? p.delta[(size_t)h * p.T + i] : 0.f;
           }
           const int ab = t & 1;
@@ -887,28 +887,45 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           const bool past = diag && wg < quarter;
           const int ab = t & 1;
           if (!warp_wait(aux_full + ab, (t >> 1) & 1, wd, 97)) { ok = false; break; }
-          const float* lse2 = reinterpret_cast<const float*>(smem + oAux + ab * 1024) + 32 * wg;
-          const float* dl = lse2 + 128;
+          // -lse log2 e and D of this block's 32 queries (identical across the warp)
+          const float4* nl4 = reinterpret_cast<const float4*>(smem + oAux + ab * 1024) + 8 * wg;
+          const float4* dl4 = nl4 + 32;
           uint32_t r[32];
-          float pr[32];
+          uint64_t pr2[16];  // P of this thread's 32 queries, in pairs (kept for dS)
           // ---- S^T -> P (kept in registers), P~T into shared memory
           if (!take(!own && !past, r)) { ok = false; break; }
           if (diag && !take(own, r)) { ok = false; break; }
           if (past) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) pr[c] = 0.f;
+            for (int i = 0; i < 16; ++i) pr2[i] = 0ull;
           } else {
+            // P = 2^(S scale log2 e - lse log2 e): one packed FMA per pair
+            const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int q = 0; q < 8; ++q) {
+              const float4 n = nl4[q];
+              float a0, a1, a2, a3;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), sl2,
+                               f2_pack(n.x, n.y)), a0, a1);
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), sl2,
+                               f2_pack(n.z, n.w)), a2, a3);
+              pr2[2 * q] = f2_pack(fast_exp2(a0), fast_exp2(a1));
+              pr2[2 * q + 1] = f2_pack(fast_exp2(a2), fast_exp2(a3));
+            }
+            if (own) {
               // on the own block query column c is visible iff it is >= the key row
-              const float pp = fast_exp2(__uint_as_float(r[c]) * p.scale_log2 - lse2[c]);
-              pr[c] = (!own || c >= lane) ? pp : 0.f;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float lo, hi;
+                f2_unpack(pr2[i], lo, hi);
+                pr2[i] = f2_pack(2 * i >= lane ? lo : 0.f, 2 * i + 1 >= lane ? hi : 0.f);
+              }
             }
           }
           if (t > 0 && !warp_wait(p_empty, (t - 1) & 1, wd, 98)) { ok = false; break; }
           {
             uint32_t cw[8];
-            const uint32_t sb = quant32(pr, p.rule, cw);
+            const uint32_t sb = mx_quant32_pairs<true>(pr2, p.rule, cw);
             store_codes32(sP, row, 2 * wg, cw);
             sfP[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)sb;
           }
@@ -919,11 +936,20 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           if (diag && !take(own, r)) { ok = false; break; }
           if (t > 0 && !warp_wait(ds_empty, (t - 1) & 1, wd, 99)) { ok = false; break; }
           {
-            float blk[32];
+            // dS = P (dP - D), packed, in place of P (P is not needed after this)
+            if (!past) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) blk[c] = past ? 0.f : pr[c] * (__uint_as_float(r[c]) - dl[c]);
+              for (int q = 0; q < 8; ++q) {
+                const float4 dd = dl4[q];
+                pr2[2 * q] = f2_mul(pr2[2 * q], f2_sub(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])),
+                                                      f2_pack(dd.x, dd.y)));
+                pr2[2 * q + 1] = f2_mul(pr2[2 * q + 1], f2_sub(f2_pack(__uint_as_float(r[4 * q + 2]),
+                                                                      __uint_as_float(r[4 * q + 3])),
+                                                              f2_pack(dd.z, dd.w)));
+              }
+            }
             uint32_t cw[8];
-            const uint32_t sb = quant32(blk, p.rule, cw);
+            const uint32_t sb = mx_quant32_pairs<false>(pr2, p.rule, cw);
             store_codes32(sDS, row, 2 * wg, cw);
             sfDS[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)sb;
           }

@@ -97,6 +97,90 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
   }
 }
 
+// Pairs of fp32 in one 64-bit register, for sm_100's packed f32x2
+// arithmetic (one instruction per pair, round to nearest like the scalar
+// forms).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// max(|a|, |b|) in magnitude (the sign of the result is that of neither; take
+// its absolute value at the end of a chain).
+__device__ __forceinline__ float max_abs_xs(float a, float b) {
+  float r;
+  asm("max.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// MX quantisation of one 32-value block of a computed operand (P or dS of the
+// attention kernels), held as 16 packed pairs: 8 code words and the scale
+// byte.  Same codes as the quantiser except that a value that rounds to zero
+// from below keeps the code 0x80 (-0), which adds nothing to an MMA.
+// kNonneg: every value is >= 0, so the block maximum needs no |.|.
+template <bool kNonneg>
+__device__ __forceinline__ uint32_t mx_quant32_pairs(const uint64_t (&v)[16], int rule, uint32_t (&codes)[8]) {
+  float x[32];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) f2_unpack(v[i], x[2 * i], x[2 * i + 1]);
+  float amax;
+  if (kNonneg) {
+    float m[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = fmaxf(x[k], x[4 + k]);
+#pragma unroll
+    for (int c = 8; c < 32; c += 8) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float r;
+        asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m[k]), "f"(x[c + k]), "f"(x[c + 4 + k]));
+        m[k] = r;
+      }
+    }
+    amax = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+  } else {
+    float m[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = max_abs_xs(x[k], x[4 + k]);
+#pragma unroll
+    for (int c = 8; c < 32; c += 4) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) m[k] = max_abs_xs(m[k], x[c + k]);
+    }
+    amax = fabsf(max_abs_xs(max_abs_xs(m[0], m[1]), max_abs_xs(m[2], m[3])));
+  }
+  const int X = mx_block_exponent(amax, rule);
+  const float sc = mx_pow2_neg(X < -126 ? -126 : X);
+  const uint64_t sc2 = f2_pack(sc, sc);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float a, b, c, d;
+    f2_unpack(f2_mul(v[2 * i], sc2), a, b);
+    f2_unpack(f2_mul(v[2 * i + 1], sc2), c, d);
+    codes[i] = mx_e4m3x2(a, b) | (mx_e4m3x2(c, d) << 16);
+  }
+  return (uint32_t)(X + 127);
+}
+
 // Instruction descriptor of kind::mxf8f6f4.block_scale with E4M3 A and B,
 // E8M0 scales, fp32 accumulation: [4,6) B scale-factor id, [7,10) A format
 // (0 = E4M3), [10,13) B format, bit 15 A major, bit 16 B major (1 = MN),
