@@ -159,11 +159,13 @@ BwdLayout bwd_layout(const fapk_problem_t* P) {
   if (P->prec == FAPK_MXFP8) {
     const size_t slots = (size_t)P->T / 32 + P->n_docs;
     L.q16 = L.k16 = L.do16 = 0;
+    // dO's MX forms, 128 codes and 4 scale bytes per (token, head) for any d
+    const size_t nq128 = (size_t)P->T * P->Hq * 128;
     L.do_vtb = after_delta;
-    L.do_stb = align_up(L.do_vtb + nq);
-    L.do_vpt = align_up(L.do_stb + slots * P->Hq * (P->d / 32));
-    L.do_spt = align_up(L.do_vpt + nq);
-    L.cta_times = align_up(L.do_spt + (size_t)P->T * P->Hq * (P->d / 32));
+    L.do_stb = align_up(L.do_vtb + nq128);
+    L.do_vpt = align_up(L.do_stb + slots * P->Hq * 4);
+    L.do_spt = align_up(L.do_vpt + nq128);
+    L.cta_times = align_up(L.do_spt + (size_t)P->T * P->Hq * 4);
     L.total = align_up(L.cta_times + 2 * sizeof(unsigned long long) * kCtaTimesWords);
     return L;
   }
@@ -204,14 +206,16 @@ CtxLayout ctx_layout(const fapk_problem_t* P) {
   }
   L.v16 = 0;
   const size_t slots = (size_t)P->T / 32 + P->n_docs;
+  // 128 codes and 4 scale bytes per (token, head) for any d (d = 64: the
+  // upper half holds zero codes)
   auto forms = [&](int H) {
     MxForms f;
-    const size_t n = (size_t)P->T * H * P->d;
+    const size_t n = (size_t)P->T * H * 128;
     f.vtb = off;
     f.stb = align_up(f.vtb + n);
-    f.vpt = align_up(f.stb + slots * H * (P->d / 32));
+    f.vpt = align_up(f.stb + slots * H * 4);
     f.spt = align_up(f.vpt + n);
-    off = align_up(f.spt + (size_t)P->T * H * (P->d / 32));
+    off = align_up(f.spt + (size_t)P->T * H * 4);
     return f;
   };
   L.q = forms(P->Hq);
@@ -272,9 +276,9 @@ int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void*
   mk.at(1, st);
   QuantJobs jobs;
   jobs.job[0] = QuantJob{static_cast<const __nv_bfloat16*>(k), P->Hkv, u8(C.k.vtb), u8(C.k.stb), u8(C.k.vpt),
-                         u8(C.k.spt), nullptr};
+                         u8(C.k.spt), nullptr, true};
   jobs.job[1] = QuantJob{static_cast<const __nv_bfloat16*>(v), P->Hkv, u8(C.v.vtb), u8(C.v.stb), u8(C.v.vpt),
-                         u8(C.v.spt), nullptr};
+                         u8(C.v.spt), nullptr, true};
   rc = cuda_status(launch_quantize_jobs(jobs, 2, P->T, P->d, P->cu_seqlens_dev, P->n_docs,
                                         FAPK_FORM_TB | FAPK_FORM_PT, P->scale_rule, st));
   if (rc != FAPK_OK) return rc;
@@ -299,6 +303,7 @@ int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void*
   a.Hq = P->Hq;
   a.Hkv = P->Hkv;
   a.n_docs = P->n_docs;
+  a.d = P->d;
   a.scale = P->scale;
   a.rule = P->scale_rule;
   a.status = status;
@@ -343,7 +348,7 @@ int bwd_mxfp8(const fapk_problem_t* P, const void* o, const float* lse, const vo
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.delta = reinterpret_cast<float*>(w + L.delta);
   a.cu = P->cu_seqlens_dev;
-  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.n_docs = P->n_docs;
+  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.n_docs = P->n_docs; a.d = P->d;
   a.scale = P->scale;
   a.grad_bf16 = P->grad_dtype == FAPK_GRAD_BF16;
   a.rule = P->scale_rule;
@@ -389,7 +394,6 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
     return FAPK_ERR_INVALID_ARG;
   const FwdLayout L = fwd_layout(P);
   if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
-  if (P->prec == FAPK_MXFP8 && P->d != 128) return FAPK_ERR_UNSUPPORTED;
   const int sms = device_num_sms();
   if (sms <= 0) return FAPK_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -436,7 +440,6 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
     return FAPK_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(P);
   if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
-  if (P->prec == FAPK_MXFP8 && P->d != 128) return FAPK_ERR_UNSUPPORTED;
   const int sms = device_num_sms();
   if (sms <= 0) return FAPK_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

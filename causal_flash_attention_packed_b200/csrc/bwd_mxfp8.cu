@@ -127,6 +127,7 @@ struct MxParams {
   DeviceStatus* status;
   uint64_t timeout_ns;
   int T, Hq, Hkv;
+  int d;  // head dimension of the bf16/fp32 tensors (64 or 128); the codes always have 128 per row
   float scale, scale_log2;
   int grad_bf16;
   int wide;  // every gradient output 32-byte aligned: 32-byte stores
@@ -502,7 +503,8 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         uint32_t t[32];
         tmem_ld32(lb + tDQ + 32 * wg, t);
         tmem_wait_ld(t);
-        if (valid) store_row32(p.out0, ((size_t)i * p.Hq + h) * 128 + 32 * wg, t, p.scale, p.grad_bf16, p.wide);
+        if (valid && 32 * wg < p.d)
+          store_row32(p.out0, ((size_t)i * p.Hq + h) * p.d + 32 * wg, t, p.scale, p.grad_bf16, p.wide);
       }
       tc_fence_before();
       warp_arrive(acc_free);
@@ -973,7 +975,8 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
         uint32_t tt[32];
         tmem_ld32(acc + 32 * c, tt);
         tmem_wait_ld(tt);
-        if (valid) store_row32(out, ((size_t)j * p.Hkv + g) * 128 + c0 + 32 * c, tt, mul, p.grad_bf16, p.wide);
+        if (valid && c0 + 32 * c < p.d)
+          store_row32(out, ((size_t)j * p.Hkv + g) * p.d + c0 + 32 * c, tt, mul, p.grad_bf16, p.wide);
       }
       tc_fence_before();
       warp_arrive(acc_free);
@@ -995,13 +998,13 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
   {
     QuantJob job{static_cast<const __nv_bfloat16*>(a.dout), a.Hq, const_cast<uint8_t*>(a.do_vtb),
                  const_cast<uint8_t*>(a.do_stb), const_cast<uint8_t*>(a.do_vpt), const_cast<uint8_t*>(a.do_spt),
-                 nullptr};
+                 nullptr, true};
     DeltaArgs da;
     da.o = static_cast<const __nv_bfloat16*>(a.o);
     da.o_resid = static_cast<const __nv_bfloat16*>(a.o_resid);
     da.delta = a.delta;
     da.T = a.T;
-    cudaError_t e = launch_quantize_with_delta(job, a.T, 128, a.cu, a.n_docs, a.rule, da, stream);
+    cudaError_t e = launch_quantize_with_delta(job, a.T, a.d, a.cu, a.n_docs, a.rule, da, stream);
     if (e != cudaSuccess) return e;
   }
   CUtensorMap tqpt, tqtb, tktb, tkpt, tvtb, tvpt, tdopt, tdotb;
@@ -1023,6 +1026,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
   p.T = a.T;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
+  p.d = a.d;
   p.scale = a.scale;
   p.scale_log2 = a.scale * kLog2e;
   p.grad_bf16 = a.grad_bf16;

@@ -102,6 +102,7 @@ struct Params {
   DeviceStatus* status;
   uint64_t timeout_ns;
   int T, Hq, Hkv, n_docs;
+  int d;  // head dimension of Q and O (64 or 128); the codes always have 128 per row
   float scale_log2;
   int rule;
   int wide;  // O and its residual 32-byte aligned: 32-byte stores
@@ -149,8 +150,8 @@ __device__ __forceinline__ void stage_q(const Params& p, const Item& it, int row
   const int t = it.q0 + row;
   const bool in_doc = t < it.e;
   float f[32];
-  if (in_doc) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)t * p.Hq + it.h) * 128 + 32 * wg);
+  if (in_doc && 32 * wg < p.d) {  // channels past d (d = 64) are zeros
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)t * p.Hq + it.h) * p.d + 32 * wg);
     uint4 raw[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) raw[c] = __ldg(src + c);
@@ -669,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++pv_cnt;  // the last tile's PV completion is covered by o_full
       tc_fence_after();
       const float inv_l = 1.f / lt;
-      const bool valid = q_idx < it.e;
+      const bool valid = q_idx < it.e && 32 * wg < p.d;
       {
         uint32_t t[32];
         tmem_ld32(lane_base + kO + 32 * wg, t);
@@ -682,8 +683,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           rb[e] = pack_bf16x2(f0 - __uint_as_float(ob[e] << 16), f1 - __uint_as_float(ob[e] & 0xFFFF0000u));
         }
         if (valid) {
-          __nv_bfloat16* orow = p.o + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * wg;
-          __nv_bfloat16* rrow = p.o_resid + ((size_t)q_idx * p.Hq + it.h) * 128 + 32 * wg;
+          __nv_bfloat16* orow = p.o + ((size_t)q_idx * p.Hq + it.h) * p.d + 32 * wg;
+          __nv_bfloat16* rrow = p.o_resid + ((size_t)q_idx * p.Hq + it.h) * p.d + 32 * wg;
           if (p.wide) {
             st_global_32B(orow, ob);
             st_global_32B(orow + 16, ob + 8);
@@ -702,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       warp_arrive(o_free);
-      if (valid && wg == 0) p.lse[(size_t)it.h * p.T + q_idx] = (M + __log2f(lt)) * kLn2;
+      if (q_idx < it.e && wg == 0) p.lse[(size_t)it.h * p.T + q_idx] = (M + __log2f(lt)) * kLn2;
       un = nx;
       have = have_next;
     }
@@ -746,6 +747,7 @@ cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
   p.T = a.T;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
+  p.d = a.d;
   p.n_docs = a.n_docs;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.rule = a.rule;

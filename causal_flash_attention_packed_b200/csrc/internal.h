@@ -66,11 +66,17 @@ cudaError_t launch_quantize_mxfp8(const void* x, int T, int H, int d, const int3
                                   uint8_t* spt, cudaStream_t stream, void* deq_pt_bf16 = nullptr);
 
 // One tensor of a quantisation launch: bf16 x [T][H][d] and its forms.
+// padded: the forms are laid out with 128 codes and 4 scale bytes per
+// (token, head) whatever d -- the layout the MXFP8 attention kernels read --
+// so that for d = 64 channels 64..127 hold zero codes (scale byte 127): an
+// all-zero 32-channel group contributes nothing to any product and leaves
+// the real groups' scales alone.
 struct QuantJob {
   const __nv_bfloat16* x;
   int H;
   uint8_t *vtb, *stb, *vpt, *spt;
   __nv_bfloat16* deq;  // per-token form dequantised to bf16, or null
+  bool padded;
 };
 struct QuantJobs {
   QuantJob job[2];
@@ -138,7 +144,7 @@ struct FwdMxArgs {
   float* lse;
   void* o_resid;
   const int32_t* cu;
-  int T, Hq, Hkv, n_docs;
+  int T, Hq, Hkv, n_docs, d;
   float scale;
   int rule;
   SchedBuf sched;
@@ -164,7 +170,7 @@ struct BwdMxArgs {
   void* dv;
   float* delta;
   const int32_t* cu;
-  int T, Hq, Hkv, n_docs;
+  int T, Hq, Hkv, n_docs, d;
   float scale;
   int grad_bf16;
   int rule;

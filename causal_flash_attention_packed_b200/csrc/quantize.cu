@@ -53,6 +53,13 @@ __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(const QuantJobs job
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const size_t row_stride = (size_t)H * D;
   const size_t col = (size_t)h * D + c8 * 8;
+  // the forms may be laid out with a row of 128 codes and 4 scale groups per
+  // (token, head) whatever D (job.padded): channels D..127 then hold zero
+  // codes and their groups the scale byte 127
+  const bool pad = job.padded && D < 128;
+  const size_t cstride = pad ? (size_t)H * 128 : row_stride;
+  const size_t ccol = pad ? (size_t)h * 128 + c8 * 8 : col;
+  const int sgroups = pad ? 4 : NG;
 
   uint4 raw[NP];
 #pragma unroll
@@ -98,9 +105,13 @@ __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(const QuantJobs job
       const int X = mx_block_exponent(a, rule);
       const size_t t = (size_t)(t0 + row);
       const uint2 codes = encode8(f[p], X);
-      *reinterpret_cast<uint2*>(job.vpt + t * row_stride + col) = codes;
+      *reinterpret_cast<uint2*>(job.vpt + t * cstride + ccol) = codes;
+      if (pad) {
+        *reinterpret_cast<uint2*>(job.vpt + t * cstride + ccol + D) = make_uint2(0u, 0u);
+        if ((c8 & 3) == 0) job.spt[(t * H + h) * sgroups + NG + (c8 >> 2)] = (uint8_t)127;
+      }
       if (job.deq) *reinterpret_cast<uint4*>(job.deq + t * row_stride + col) = dequant8_bf16(codes, X);
-      if ((c8 & 3) == 0) job.spt[(t * H + h) * NG + (c8 >> 2)] = (uint8_t)(X + 127);
+      if ((c8 & 3) == 0) job.spt[(t * H + h) * sgroups + (c8 >> 2)] = (uint8_t)(X + 127);
     }
     amax_tb = fmaxf(amax_tb, a);
   }
@@ -118,13 +129,16 @@ __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(const QuantJobs job
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int row = r0 + p * RPP;
-    if (row < nb)
-      *reinterpret_cast<uint2*>(job.vtb + (size_t)(t0 + row) * row_stride + col) = encode8(f[p], X);
+    if (row < nb) {
+      *reinterpret_cast<uint2*>(job.vtb + (size_t)(t0 + row) * cstride + ccol) = encode8(f[p], X);
+      if (pad) *reinterpret_cast<uint2*>(job.vtb + (size_t)(t0 + row) * cstride + ccol + D) = make_uint2(0u, 0u);
+    }
   }
   if (threadIdx.x < NG) {
     const int gg = threadIdx.x;
     const float ag = fmaxf(fmaxf(red[0][gg], red[1][gg]), fmaxf(red[2][gg], red[3][gg]));
-    job.stb[((size_t)slot * H + h) * NG + gg] = (uint8_t)(mx_block_exponent(ag, rule) + 127);
+    job.stb[((size_t)slot * H + h) * sgroups + gg] = (uint8_t)(mx_block_exponent(ag, rule) + 127);
+    if (pad) job.stb[((size_t)slot * H + h) * sgroups + NG + gg] = (uint8_t)127;
   }
 }
 
@@ -149,7 +163,7 @@ cudaError_t launch_quantize_mxfp8(const void* x, int T, int H, int d, const int3
                                   uint8_t* spt, cudaStream_t stream, void* deq_pt_bf16) {
   QuantJobs jobs;
   jobs.job[0] = QuantJob{static_cast<const __nv_bfloat16*>(x), H, vtb, stb, vpt, spt,
-                         static_cast<__nv_bfloat16*>(deq_pt_bf16)};
+                         static_cast<__nv_bfloat16*>(deq_pt_bf16), false};
   return launch_jobs<false>(jobs, 1, T, d, cu, n_docs, forms, rule, DeltaArgs{}, stream);
 }
 

@@ -66,6 +66,14 @@ def test_gqa():
     _check(w, require_gpu())
 
 
+@pytest.mark.parametrize("G", [1, 2])
+def test_head_dim_64_ragged_documents(G):
+    """d = 64: the MX forms keep 128 codes per row with a zero upper half, which
+    changes no real block's scale; against the emulation at d = 64."""
+    w = W.custom([1, 31, 32, 33, 127, 128, 129, 300, 700], Hq=2 * G, Hkv=2, d=64, seed=64)
+    _check(w, require_gpu())
+
+
 def test_outlier_channels_16k_full():
     """The 16384-token MXFP8 workload (x20 outlier channels), full size."""
     _check(W.config(3, 0), require_gpu())
@@ -133,6 +141,26 @@ def test_bwd_ragged_documents():
 def test_bwd_gqa():
     w = W.custom([513, 64, 1000], Hq=4, Hkv=2, d=128, seed=72)
     _check_bwd(w, require_gpu())
+
+
+@pytest.mark.parametrize("G", [1, 2])
+def test_bwd_head_dim_64_ragged_documents(G):
+    w = W.custom([1, 31, 32, 33, 127, 128, 129, 300, 700], Hq=2 * G, Hkv=2, d=64, seed=75)
+    _check_bwd(w, require_gpu())
+
+
+@pytest.mark.parametrize("t_rel", [13, 31, 200])
+def test_head_dim_64_leak_free(t_rel):
+    """T1/T2 at d = 64: O, LSE and dQ at positions <= t are bit-identical when
+    everything after t is randomised."""
+    dev = require_gpu()
+    w = W.custom([300, 513, 200], Hq=2, Hkv=2, d=64, seed=76)
+    base = w.tensors()
+    t = 300 + t_rel
+    _, a = mx_fwd_bwd(w, dev, tensors=base)
+    _, b = mx_fwd_bwd(w, dev, tensors=_perturb(base, t, 11))
+    for x, y in zip(a[:3], b[:3]):
+        assert torch.equal(x[: t + 1] if x.dim() == 3 else x[:, : t + 1], y[: t + 1] if y.dim() == 3 else y[:, : t + 1])
 
 
 def test_bwd_outlier_channels_16k_full():
