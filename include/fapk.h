@@ -30,7 +30,9 @@
  *   lse            : fp32 [Hq][T]    cu_seqlens   : int32 [n_docs + 1]
  * with cu[0] = 0, cu non-decreasing, cu[n_docs] = T; document k holds tokens
  * [cu[k], cu[k+1]); zero-length documents are allowed and produce nothing.
- * Query head h reads KV head h / (Hq / Hkv).  d must be 64 or 128.
+ * Query head h reads KV head h / (Hq / Hkv).  d must be 64 or 128 (both
+ * paths; the MXFP8 path keeps its internal code rows 128 wide and for d = 64
+ * fills the upper half with zero codes, which change no real block's scale).
  *
  * Ownership and threading.  The caller owns every buffer (inputs, outputs,
  * workspace, ctx).  The library allocates no device memory and keeps no
