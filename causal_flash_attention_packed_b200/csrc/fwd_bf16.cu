@@ -402,19 +402,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
           l *= alpha;
         }
-        // P = 2^(s scale log2(e) - m) with one FMA per element; row sum in
-        // four independent partial sums
+        // P = 2^(s scale log2(e) - m): one packed FMA per pair of elements;
+        // row sum in four independent packed partial sums
         uint32_t pk[64];
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
-        const float nm = -m;
+        uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+        const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-m, -m);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float a = fast_exp2(fmaf(x[2 * c], p.scale_log2, nm));
-          const float b = fast_exp2(fmaf(x[2 * c + 1], p.scale_log2, nm));
-          rs[c & 3] += a + b;
+          float a, b;
+          f2_unpack(f2_fma(f2_pack(x[2 * c], x[2 * c + 1]), sl2, nm2), a, b);
+          a = fast_exp2(a);
+          b = fast_exp2(b);
+          const uint64_t ab = f2_pack(a, b);
+          rs2[c & 3] = (c < 4) ? ab : f2_add(rs2[c & 3], ab);
           pk[c] = pack_f16x2(a, b);
         }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        {
+          float s0, s1, s2, s3;
+          f2_unpack(f2_add(rs2[0], rs2[1]), s0, s1);
+          f2_unpack(f2_add(rs2[2], rs2[3]), s2, s3);
+          l += (s0 + s2) + (s1 + s3);
+        }
         // the previous P V of this tile has completed: P's buffer is free and
         // O is settled for the rescale
         if (p_cnt > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(p_free + wg, (p_cnt - 1) & 1, wd, 13))) {
