@@ -453,13 +453,17 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           // ---- P
           float x[32];
           if (!take(x)) { ok = false; break; }
+          {
+            // P = 2^(S scale log2(e) - LSE log2(e)): one packed FMA per pair
+            const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            const float4 n4 = *reinterpret_cast<const float4*>(nl2 + c);
-            x[c] = fast_exp2(fmaf(x[c], p.scale_log2, n4.x));
-            x[c + 1] = fast_exp2(fmaf(x[c + 1], p.scale_log2, n4.y));
-            x[c + 2] = fast_exp2(fmaf(x[c + 2], p.scale_log2, n4.z));
-            x[c + 3] = fast_exp2(fmaf(x[c + 3], p.scale_log2, n4.w));
+            for (int c = 0; c < 32; c += 4) {
+              const float4 n4 = *reinterpret_cast<const float4*>(nl2 + c);
+              f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), sl2, f2_pack(n4.x, n4.y)), x[c], x[c + 1]);
+              f2_unpack(f2_fma(f2_pack(x[c + 2], x[c + 3]), sl2, f2_pack(n4.z, n4.w)), x[c + 2], x[c + 3]);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) x[c + u] = fast_exp2(x[c + u]);
+            }
           }
           if (!full) {
 #pragma unroll
@@ -486,11 +490,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           uint32_t dk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
+            // dS = P (dP - D), packed pairs
             const float4 d4 = *reinterpret_cast<const float4*>(dl + c);
-            y[c] = x[c] * (y[c] - d4.x);
-            y[c + 1] = x[c + 1] * (y[c + 1] - d4.y);
-            y[c + 2] = x[c + 2] * (y[c + 2] - d4.z);
-            y[c + 3] = x[c + 3] * (y[c + 3] - d4.w);
+            f2_unpack(f2_mul(f2_pack(x[c], x[c + 1]), f2_sub(f2_pack(y[c], y[c + 1]), f2_pack(d4.x, d4.y))), y[c],
+                      y[c + 1]);
+            f2_unpack(f2_mul(f2_pack(x[c + 2], x[c + 3]), f2_sub(f2_pack(y[c + 2], y[c + 3]), f2_pack(d4.z, d4.w))),
+                      y[c + 2], y[c + 3]);
           }
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
@@ -810,17 +815,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const bool diag = v == it.m;
         uint32_t dk[16];
         float dm[4] = {0.f, 0.f, 0.f, 0.f};  // range check in four partial chains
+        const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2), nl22 = f2_pack(nl2, nl2), dl2 = f2_pack(dl, dl);
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
+          // P = 2^(S scale log2(e) - LSE log2(e)), dS = P (dP - D): packed pairs
+          float a0, a1;
+          f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), sl2, nl22), a0, a1);
+          float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+          if (diag && j0 + c > i) p0 = 0.f;
+          if (diag && j0 + c + 1 > i) p1 = 0.f;
           float dv[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int cc = c + u;
-            float pp = fast_exp2(fmaf(x[cc], p.scale_log2, nl2));
-            if (diag && j0 + cc > i) pp = 0.f;
-            dv[u] = pp * (y[cc] - dl);
-            dm[(c / 2) & 3] = fmaxf(dm[(c / 2) & 3], fabsf(dv[u]));
-          }
+          f2_unpack(f2_mul(f2_pack(p0, p1), f2_sub(f2_pack(y[c], y[c + 1]), dl2)), dv[0], dv[1]);
+          dm[(c / 2) & 3] = fmaxf(dm[(c / 2) & 3], fmaxf(fabsf(dv[0]), fabsf(dv[1])));
           dk[c / 2] = pack_f16x2(dv[0], dv[1]);
         }
         const float dmax = fmaxf(fmaxf(dm[0], dm[1]), fmaxf(dm[2], dm[3]));

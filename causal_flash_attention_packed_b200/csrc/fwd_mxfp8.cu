@@ -585,23 +585,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // u = 2^(s scale log2(e) - M) with one FMA per element; row sum
         // before quantisation and block maximum of u in four partial chains
         // each; MX quantisation of the block
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f}, am4[4] = {0.f, 0.f, 0.f, 0.f};
-        const float nM = -M;
+        // (packed pairs: one FMA per pair for the arguments, one add per pair
+        // for the row sum, and the block quantisation on pairs)
+        uint64_t u2[16], rs2[2] = {0ull, 0ull};
+        {
+          const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2), nM2 = f2_pack(-M, -M);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float arg = fmaf(x[c], p.scale_log2, nM);
-          x[c] = fast_exp2(arg);
-          rs4[c & 3] += x[c];
-          am4[c & 3] = fmaxf(am4[c & 3], x[c]);
+          for (int c = 0; c < 16; ++c) {
+            float a, b;
+            f2_unpack(f2_fma(f2_pack(x[2 * c], x[2 * c + 1]), sl2, nM2), a, b);
+            u2[c] = f2_pack(fast_exp2(a), fast_exp2(b));
+            rs2[c & 1] = (c < 2) ? u2[c] : f2_add(rs2[c & 1], u2[c]);
+          }
+          float s0, s1, s2, s3;
+          f2_unpack(rs2[0], s0, s1);
+          f2_unpack(rs2[1], s2, s3);
+          l += (s0 + s1) + (s2 + s3);
         }
-        const float amax = fmaxf(fmaxf(am4[0], am4[1]), fmaxf(am4[2], am4[3]));
-        l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-        const int X = mx_block_exponent(amax, p.rule);
-        const float sc = mx_pow2_neg(X < -126 ? -126 : X);
         uint32_t codes[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          codes[c] = mx_e4m3x2(x[4 * c] * sc, x[4 * c + 1] * sc) | (mx_e4m3x2(x[4 * c + 2] * sc, x[4 * c + 3] * sc) << 16);
+        const int X = (int)mx_quant32_pairs<true>(u2, p.rule, codes) - 127;
         // bf16 copy of the own block's P~ (exact); its FP8 codes are zeroed
         uint32_t pd[16];
 #pragma unroll
