@@ -69,6 +69,27 @@ __device__ __forceinline__ uint4 tb_rows(const uint8_t* stb, int s, int e, int d
                     tb_word(stb, s, e, doc, blk0 + 2, H, g), tb_word(stb, s, e, doc, blk0 + 3, H, g));
 }
 
+// MX quantisation of 32 values (one block of a computed operand): 8 code
+// words; returns the scale byte.  A value that rounds to zero from below keeps
+// the code 0x80 (-0), which adds nothing to an MMA.
+__device__ __forceinline__ uint32_t quant32(const float (&x)[32], int rule, uint32_t (&codes)[8]) {
+  float m[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) m[k] = max_abs_xs(x[k], x[4 + k]);
+#pragma unroll
+  for (int c = 8; c < 32; c += 4) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = max_abs_xs(m[k], x[c + k]);
+  }
+  const float amax = fabsf(max_abs_xs(max_abs_xs(m[0], m[1]), max_abs_xs(m[2], m[3])));
+  const int X = mx_block_exponent(amax, rule);
+  const float sc = mx_pow2_neg(X < -126 ? -126 : X);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    codes[c] = mx_e4m3x2(x[4 * c] * sc, x[4 * c + 1] * sc) | (mx_e4m3x2(x[4 * c + 2] * sc, x[4 * c + 3] * sc) << 16);
+  return (uint32_t)(X + 127);
+}
+
 // Exact bf16 of the dequantised block: 16 words of packed bf16 pairs.
 __device__ __forceinline__ void dequant32_bf16(const uint32_t (&codes)[8], uint32_t sbyte, uint32_t (&out)[16]) {
   const int X = (int)sbyte - 127;
@@ -438,39 +459,29 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         const bool own = diag && wg == quarter;
         const bool future = diag && wg > quarter;
         uint32_t r[32];
-        uint64_t ds2[16];  // P, then dS, of this thread's 32 keys in packed pairs
+        float ds[32];
         // ---- S -> P (in place)
         if (!take(s_full, s_free, s_cnt, tS, !own && !future, r)) { ok = false; break; }
         if (diag && !take(s_full, s_free, s_cnt, tS, own, r)) { ok = false; break; }
         if (future) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) ds2[c] = 0ull;
+          for (int c = 0; c < 32; ++c) ds[c] = 0.f;
         } else {
-          const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(-l2, -l2);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float a, b;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2, nl2), a, b);
-            a = fast_exp2(a);
-            b = fast_exp2(b);
-            if (own) {
-              if (2 * c > lane) a = 0.f;
-              if (2 * c + 1 > lane) b = 0.f;
-            }
-            ds2[c] = f2_pack(a, b);
+          for (int c = 0; c < 32; ++c) {
+            const float pp = fast_exp2(__uint_as_float(r[c]) * p.scale_log2 - l2);
+            ds[c] = (!own || c <= lane) ? pp : 0.f;
           }
         }
         // ---- dP -> dS = P (dP - D)
         if (!take(dp_full, dp_free, dp_cnt, tDP, !own && !future, r)) { ok = false; break; }
         if (diag && !take(dp_full, dp_free, dp_cnt, tDP, own, r)) { ok = false; break; }
         if (!future) {
-          const uint64_t dl2 = f2_pack(dl, dl);
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            ds2[c] = f2_mul(ds2[c], f2_sub(f2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), dl2));
+          for (int c = 0; c < 32; ++c) ds[c] = ds[c] * (__uint_as_float(r[c]) - dl);
         }
         uint32_t cw[8];
-        const uint32_t sb = mx_quant32_pairs<false>(ds2, p.rule, cw);
+        const uint32_t sb = quant32(ds, p.rule, cw);
         uint32_t pd[16];
         if (own) {
           // the diagonal block leaves the FP8 operand (it goes through the bf16 MMA)
