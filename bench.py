@@ -219,8 +219,9 @@ KERNEL_FLOPS = {"fwd_kernel": 4.0, "dkdv_kernel": 8.0, "dq_kernel": 6.0}
 # of an ncu capture of the kernels as they stand; None where not measured.
 # These must be taken again whenever a kernel changes.
 MEASURED_TRAFFIC = {
-    4: {"bf16": {"fwd_kernel": 1.337e9, "dkdv_kernel": 2.132e9, "dq_kernel": 1.610e9},
-        "mxfp8": {"fwd_kernel": None, "dkdv_kernel": 2.169e9, "dq_kernel": 1.637e9}},
+    4: {"bf16": {"fwd_kernel": 1.325e9, "dkdv_kernel": 2.131e9, "dq_kernel": 1.610e9},
+        "mxfp8": {"fwd_kernel": 1.594e9, "dkdv_kernel": 2.198e9, "dq_kernel": 1.354e9,
+                  "quantize_kv": 1.033e9, "delta_quantize_do": 1.052e9}},
 }
 
 
@@ -384,8 +385,9 @@ def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, clk, conf
         # quantised on load inside the forward kernel, dO inside the D pass.
         qbytes = 2 * w.T * w.Hkv * w.d * (2.0 + 2 * (1.0 + 1.0 / 32))
         gbs = qbytes / (kern_ms["quantize_kv"] * 1e-3) / 1e9
+        qtraffic = MEASURED_TRAFFIC.get(config, {}).get(prec, {})
         out["roofline_quantize"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                    "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                                    "frac": gbs / peaks["hbm_gbs"], "traffic": qtraffic.get("quantize_kv"),
                                     "algorithmic_bytes": qbytes,
                                     "kernel": "quantize_mxfp8_kernel (K and V in one launch; both forms)"}
         # the D pass with dO's quantisation: reads dO, O and O's residual
@@ -394,6 +396,7 @@ def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, clk, conf
         gbs = dbytes / (kern_ms["delta_quantize_do"] * 1e-3) / 1e9
         out["roofline_delta_quantize_do"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                                              "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                                             "traffic": qtraffic.get("delta_quantize_do"),
                                              "algorithmic_bytes": dbytes}
         out["quantize_ms_per_step"] = kern_ms["quantize_kv"] + kern_ms["delta_quantize_do"]
     return out
