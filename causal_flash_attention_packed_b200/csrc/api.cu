@@ -484,6 +484,58 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   return cuda_status(launch_bwd_bf16(a, st));
 }
 
+int fapk_attn_fwd_quantized_kv(const fapk_problem_t* P, const void* q, const uint8_t* k_val_tb,
+                               const uint8_t* k_scale_tb, const uint8_t* k_val_pt, const uint8_t* k_scale_pt,
+                               const uint8_t* v_val_tb, const uint8_t* v_scale_tb, const uint8_t* v_val_pt,
+                               const uint8_t* v_scale_pt, void* o, float* lse, void* ws, size_t ws_bytes,
+                               void* stream) {
+  int rc = validate_problem(P);
+  if (rc != FAPK_OK) return rc;
+  if (P->prec != FAPK_MXFP8 || P->d != 128) return FAPK_ERR_UNSUPPORTED;
+  if (P->T == 0) return FAPK_OK;
+  if (!q || !k_val_tb || !k_scale_tb || !k_val_pt || !k_scale_pt || !v_val_tb || !v_scale_tb || !v_val_pt ||
+      !v_scale_pt || !o || !lse || !ws)
+    return FAPK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || !aligned16(k_val_tb) || !aligned16(k_val_pt) ||
+      !aligned16(v_val_tb) || !aligned16(v_val_pt) || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+    return FAPK_ERR_INVALID_ARG;
+  // scale rows are read 4 bytes at a time
+  for (const uint8_t* sp : {k_scale_tb, k_scale_pt, v_scale_tb, v_scale_pt})
+    if (reinterpret_cast<uintptr_t>(sp) & 3u) return FAPK_ERR_INVALID_ARG;
+  const FwdLayout L = fwd_layout(P);
+  if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
+  const int sms = device_num_sms();
+  if (sms <= 0) return FAPK_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* status = static_cast<DeviceStatus*>(ws);
+  const Marks mk{P->timing_events, P->n_timing_events};
+  FwdMxArgs a;
+  a.sched = sched_buf(ws, L.sched);
+  mk.at(0, st);
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, a.sched, status, true, st));
+  if (rc != FAPK_OK) return rc;
+  a.q = q;
+  a.q_vpt = a.q_spt = a.q_vtb = a.q_stb = nullptr;  // no saved state: nothing for a backward
+  a.k_vtb = k_val_tb; a.k_stb = k_scale_tb; a.k_vpt = k_val_pt; a.k_spt = k_scale_pt;
+  a.v_vtb = v_val_tb; a.v_stb = v_scale_tb; a.v_vpt = v_val_pt; a.v_spt = v_scale_pt;
+  a.o = o;
+  a.lse = lse;
+  a.o_resid = nullptr;
+  a.cu = P->cu_seqlens_dev;
+  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.n_docs = P->n_docs; a.d = P->d;
+  a.scale = P->scale;
+  a.rule = P->scale_rule;
+  a.status = status;
+  if (P->flags & FAPK_FLAG_CTA_TIMES)
+    a.cta_times[0] = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + L.cta_times);
+  a.timeout_ns = timeout_ns_of(P);
+  a.num_sms = sms;
+  mk.at(1, st);
+  rc = cuda_status(launch_fwd_mxfp8(a, st));
+  mk.at(2, st);
+  return rc;
+}
+
 int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const int32_t* cu_seqlens_dev,
                         const int32_t* cu_seqlens_host, int n_docs, int forms, int scale_rule,
                         uint8_t* val_tb, uint8_t* scale_tb, uint8_t* val_pt, uint8_t* scale_pt,

@@ -87,7 +87,8 @@ struct Params {
   const int32_t* cu;
   SchedView sched;
   const __nv_bfloat16* q;  // Q [T][Hq][128] (bf16 input, quantised on load)
-  uint8_t* q_vpt;          // out: Q per-token codes [T][Hq][128] (ctx)
+  uint8_t* q_vpt;          // out: Q per-token codes [T][Hq][128] (ctx); null: no saved state
+                           // for a backward (then q_spt.. and o_resid are not written either)
   uint8_t* q_spt;          // out: Q per-token scales [T][Hq][4]
   uint8_t* q_vtb;          // out: Q token-block codes [T][Hq][128]
   uint8_t* q_stb;          // out: Q token-block scales [slots][Hq][4]
@@ -173,6 +174,7 @@ __device__ __forceinline__ void stage_q(const Params& p, const Item& it, int row
   *reinterpret_cast<uint4*>(prow + (((2 * wg) ^ (row & 7)) << 4)) = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
   *reinterpret_cast<uint4*>(prow + (((2 * wg + 1) ^ (row & 7)) << 4)) = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
   sfQ[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)(X + 127);
+  if (!p.q_vpt) return;  // inference: Q's forms are not kept
   const size_t qo = ((size_t)t * p.Hq + it.h) * 128 + 32 * wg;
   if (in_doc) {
     uint4* dst = reinterpret_cast<uint4*>(p.q_vpt + qo);
@@ -686,19 +688,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (valid) {
           __nv_bfloat16* orow = p.o + ((size_t)q_idx * p.Hq + it.h) * p.d + 32 * wg;
-          __nv_bfloat16* rrow = p.o_resid + ((size_t)q_idx * p.Hq + it.h) * p.d + 32 * wg;
+          __nv_bfloat16* rrow = p.o_resid ? p.o_resid + ((size_t)q_idx * p.Hq + it.h) * p.d + 32 * wg : nullptr;
           if (p.wide) {
             st_global_32B(orow, ob);
             st_global_32B(orow + 16, ob + 8);
-            st_global_32B(rrow, rb);
-            st_global_32B(rrow + 16, rb + 8);
+            if (rrow) {
+              st_global_32B(rrow, rb);
+              st_global_32B(rrow + 16, rb + 8);
+            }
           } else {
             uint4* dst = reinterpret_cast<uint4*>(orow);
-            uint4* rdst = reinterpret_cast<uint4*>(rrow);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
-              rdst[e] = make_uint4(rb[4 * e], rb[4 * e + 1], rb[4 * e + 2], rb[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+            if (rrow) {
+              uint4* rdst = reinterpret_cast<uint4*>(rrow);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) rdst[e] = make_uint4(rb[4 * e], rb[4 * e + 1], rb[4 * e + 2], rb[4 * e + 3]);
             }
           }
         }

@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
     L.fapk_attn_bwd.restype = i
     L.fapk_attn_fwd_noalloc.argtypes = [PP, vp, vp, vp, vp, vp, vp, vp]
     L.fapk_attn_fwd_noalloc.restype = i
+    L.fapk_attn_fwd_quantized_kv.argtypes = [PP] + [vp] * 11 + [sz, vp]
+    L.fapk_attn_fwd_quantized_kv.restype = i
     L.fapk_noalloc_status.argtypes = [vp]
     L.fapk_noalloc_status.restype = i
     L.fapk_quantize_mxfp8.argtypes = [vp, i, i, i, vp, vp, i, i, i, vp, vp, vp, vp, vp]
@@ -237,6 +239,25 @@ def attn_fwd_noalloc(P: Problem, q, k, v, o, lse, ctx, stream=None):
                                      _ptr(ctx), _stream(stream))
     _check(rc, "fapk_attn_fwd_noalloc")
     return o, lse, ctx
+
+
+def attn_fwd_quantized_kv(P: Problem, q, k_forms: dict, v_forms: dict, o=None, lse=None, ws=None, stream=None):
+    """fapk_attn_fwd_quantized_kv: MXFP8 forward over K and V given in both MX
+    forms (dicts with val_tb, scale_tb, val_pt, scale_pt as quantize_mxfp8
+    returns them).  Returns (o, lse)."""
+    dev = q.device
+    if o is None:
+        o = torch.empty((P.T, P.Hq, P.d), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((P.Hq, P.T), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(P, FWD, dev)
+    f = [k_forms[n] for n in ("val_tb", "scale_tb", "val_pt", "scale_pt")] + \
+        [v_forms[n] for n in ("val_tb", "scale_tb", "val_pt", "scale_pt")]
+    rc = lib().fapk_attn_fwd_quantized_kv(ctypes.byref(P), _ptr(q), *[_ptr(t) for t in f], _ptr(o), _ptr(lse),
+                                          _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "fapk_attn_fwd_quantized_kv")
+    return o, lse
 
 
 def attn_bwd(P: Problem, q, k, v, o, lse, dout, ctx=None, dq=None, dk=None, dv=None, ws=None,

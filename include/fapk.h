@@ -207,6 +207,30 @@ FAPK_API int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const 
                         uint8_t* val_tb, uint8_t* scale_tb, uint8_t* val_pt, uint8_t* scale_pt,
                         void* stream);
 
+/* MXFP8 forward over already-quantised K and V ("Flash Attention" glossary
+ * page on local inference engines, secs. "Tanim" and the KV-cache table: a
+ * quantised KV cache, read directly by the fused attention kernel, holds the
+ * keys and values in half the bytes of f16).  Q is bf16 and quantised on load
+ * as in fapk_attn_fwd; K and V arrive in both MX forms exactly as
+ * fapk_quantize_mxfp8 writes them (forms = FAPK_FORM_TB | FAPK_FORM_PT, for
+ * example once into a cache and then reused by many calls), so the call
+ * launches no quantisation of its own.  Inference only: no ctx, no backward.
+ *  - prob->prec must be FAPK_MXFP8, prob->d 128 (FAPK_ERR_UNSUPPORTED
+ *    otherwise); the forms must have been made with prob's cu_seqlens and
+ *    scale rule.
+ *  - k_val_tb, k_val_pt, v_val_tb, v_val_pt: codes [T][Hkv][128], 16-byte
+ *    aligned; k_scale_tb, v_scale_tb: [T/32 + n_docs][Hkv][4];
+ *    k_scale_pt, v_scale_pt: [T][Hkv][4]; scales 4-byte aligned.
+ *  - q, o, lse, ws and errors as in fapk_attn_fwd.  With the forms of
+ *    fapk_quantize_mxfp8, O and LSE are bit-identical to fapk_attn_fwd's in
+ *    the MXFP8 path. */
+FAPK_API int fapk_attn_fwd_quantized_kv(const fapk_problem_t* prob, const void* q, const uint8_t* k_val_tb,
+                                        const uint8_t* k_scale_tb, const uint8_t* k_val_pt,
+                                        const uint8_t* k_scale_pt, const uint8_t* v_val_tb,
+                                        const uint8_t* v_scale_tb, const uint8_t* v_val_pt,
+                                        const uint8_t* v_scale_pt, void* o, float* lse, void* ws,
+                                        size_t ws_bytes, void* stream);
+
 /* Forward that allocates nothing.  The pages have no counterpart: this entry
  * point exists for callers that cannot obtain device memory where they run the
  * forward -- a plugin handed its buffers by a host framework that must not

@@ -106,6 +106,18 @@ def test_bad_seqlens_detected_on_host(L, cu, maxlen):
     assert _fwd(L, P) == fapk.ERR_BAD_SEQLENS
 
 
+def test_quantized_kv_forward_validation(L):
+    """The forward from pre-quantised K/V takes the MXFP8 path at d = 128 only."""
+    f = L.fapk_attn_fwd_quantized_kv
+    ptrs = [256] * 11
+    assert f(ctypes.byref(_problem(prec=fapk.BF16)), *ptrs, 256, 1 << 30, None) == fapk.ERR_UNSUPPORTED
+    assert f(ctypes.byref(_problem(prec=fapk.MXFP8, d=64)), *ptrs, 256, 1 << 30, None) == fapk.ERR_UNSUPPORTED
+    bad = list(ptrs)
+    bad[2] = 258  # a scale array not 4-byte aligned
+    assert f(ctypes.byref(_problem(prec=fapk.MXFP8)), *bad, 256, 1 << 30, None) == fapk.ERR_INVALID_ARG
+    assert f(ctypes.byref(_problem(prec=fapk.MXFP8)), *ptrs, 256, 16, None) == fapk.ERR_WORKSPACE_TOO_SMALL
+
+
 def test_quantize_validation(L):
     q = L.fapk_quantize_mxfp8
     x = 256

@@ -192,3 +192,10 @@ def test_leak_T3(t_rel):
     _, b = run_fwd_bwd(w, dev, tensors=_perturbed(base, t, 8, keep_dout_zero=True))
     assert torch.equal(a[3][: t + 1], b[3][: t + 1])
     assert torch.equal(a[4][: t + 1], b[4][: t + 1])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_multi_query_attention(d):
+    """MQA: every query head reads the one KV head (Hkv = 1), so dK and dV sum
+    over all eight query heads; full outputs against the oracle."""
+    _full_check(W.custom([1, 129, 300, 700, 64], Hq=8, Hkv=1, d=d, seed=23), require_gpu())

@@ -285,3 +285,34 @@ def test_bwd_dkdv_at_unaligned_t_measured(t_rel):
         rel = float(np.max(np.abs(x - y)) / np.sqrt(np.mean(x * x)))
         print(f"T3 t_rel={t_rel} {name}: {n} of {x.size} elements differ, max diff {rel:.2e} of RMS")
         assert rel <= 2e-3, (name, n, rel)
+
+
+def test_forward_from_quantised_kv_matches_the_mxfp8_forward():
+    """fapk_attn_fwd_quantized_kv: K and V quantised once by fapk_quantize_mxfp8
+    (as a quantised KV cache would hold them) and reused by two calls with
+    different Q; each call's O and LSE are bit-identical to the MXFP8 forward
+    on the bf16 K and V, and within the bar of the oracle's emulation."""
+    dev = require_gpu()
+    w = W.custom([1, 31, 33, 127, 129, 300, 700], Hq=4, Hkv=2, d=128, seed=77)
+    (q, k, v, _), (qd, kd, vd, _) = to_dev(w, dev, with_dout=False)
+    seq = fapk.Seqlens(w.cu, dev)
+    P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale, prec=fapk.MXFP8)
+    kf = fapk.quantize_mxfp8(kd, seq)
+    vf = fapk.quantize_mxfp8(vd, seq)
+    g = torch.Generator().manual_seed(78)
+    q2 = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    for qq in (q, q2):
+        qqd = qq.to(dev)
+        o1, l1 = fapk.attn_fwd_quantized_kv(P, qqd, kf, vf)
+        o2, l2, _ = fapk.attn_fwd(P, qqd, kd, vd)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        eo, _ = oracle.mx_attn_fwd(qq.double().numpy(), k.double().numpy(), v.double().numpy(), w.cu, w.scale)
+        assert rel_frob(f64(o1), eo) <= MX_REL_FROB
+
+
+def test_multi_query_attention_fwd_bwd():
+    """MQA in the MXFP8 path (Hkv = 1, eight query heads)."""
+    w = W.custom([1, 129, 300, 700, 64], Hq=8, Hkv=1, d=128, seed=79)
+    _check(w, require_gpu())
+    _check_bwd(w, require_gpu())
