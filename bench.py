@@ -402,6 +402,35 @@ def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, clk, conf
     return out
 
 
+def time_qkv_proj(fapk, w, dev, peaks, clk, warmup, steps):
+    """CUDA-event time of fapk_qkv_proj_mxfp8 on the workload's tokens: x
+    [T, Hq d] bf16 against w [(Hq + 2 Hkv) d, Hq d]; 2 T d_model N FLOP."""
+    g = torch.Generator(device=dev).manual_seed(5)
+    Dm = w.Hq * w.d
+    N = (w.Hq + 2 * w.Hkv) * w.d
+    x = torch.randn((w.T, Dm), generator=g, device=dev).to(torch.bfloat16)
+    wt = (torch.randn((N, Dm), generator=g, device=dev) / Dm ** 0.5).to(torch.bfloat16)
+    seq = fapk.Seqlens(w.cu, dev)
+    P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale, prec=fapk.MXFP8)
+    ws = fapk.workspace(P, fapk.FWD, dev)
+    for _ in range(warmup):
+        fapk.qkv_proj_mxfp8(P, x, wt, ws=ws)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fapk.qkv_proj_mxfp8(P, x, wt, ws=ws)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    flops = 2.0 * w.T * Dm * N
+    tf = flops / (ms * 1e-3) / 1e12
+    peak, src = tensor_peak(peaks, clk, False)
+    return {"ms": ms, "tflops": tf, "frac": tf / peak, "peak": peak, "peak_source": src,
+            "shape": {"tokens": w.T, "d_model": Dm, "n_out": N}, "status_ok": fapk.status(ws) == 0,
+            "note": "includes the schedule launch and the MX forms of K and V written by the epilogue"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -414,6 +443,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--qkv-proj", type=int, default=1, help="also time the fused QKV projection (0: skip)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -450,6 +480,13 @@ def main():
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     balance = {p: runners[p].balance(num_sms) for p in paths}
     st_ok = st_ok and all(r.status_ok() for r in runners.values())
+
+    # the fused QKV projection with K's and V's MX quantisation in its epilogue,
+    # on the same tokens (d_model = Hq d, as for a model whose heads span it);
+    # timed on its own: it precedes the attention step in a training step
+    proj = None
+    if args.qkv_proj and w.d == 128:
+        proj = time_qkv_proj(fapk, w, dev, peaks, clk, args.warmup, min(args.steps, 20))
 
     # end to end through the C ABI with host buffers (pinned), copies included
     e2e = None
@@ -498,7 +535,7 @@ def main():
         "pct_of_dense_bf16_peak": head["pct_of_dense_peak"] if main_path == "bf16" else None,
         "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
-        "clocks": clk, "status_ok": st_ok,
+        "clocks": clk, "status_ok": st_ok, "qkv_proj": proj,
         "scheduler_balance": balance,
     }
     for p in paths[1:]:

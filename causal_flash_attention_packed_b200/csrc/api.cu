@@ -536,6 +536,51 @@ int fapk_attn_fwd_quantized_kv(const fapk_problem_t* P, const void* q, const uin
   return rc;
 }
 
+int fapk_qkv_proj_mxfp8(const fapk_problem_t* P, const void* x, int d_model, const void* w, void* q, void* k,
+                        void* v, uint8_t* k_val_tb, uint8_t* k_scale_tb, uint8_t* k_val_pt, uint8_t* k_scale_pt,
+                        uint8_t* v_val_tb, uint8_t* v_scale_tb, uint8_t* v_val_pt, uint8_t* v_scale_pt, void* ws,
+                        size_t ws_bytes, void* stream) {
+  int rc = validate_problem(P);
+  if (rc != FAPK_OK) return rc;
+  if (P->prec != FAPK_MXFP8 || P->d != 128) return FAPK_ERR_UNSUPPORTED;
+  if (d_model <= 0 || d_model % 8 != 0) return FAPK_ERR_INVALID_ARG;
+  if (P->T == 0) return FAPK_OK;
+  if (!x || !w || !q || !k || !v || !k_val_tb || !k_scale_tb || !k_val_pt || !k_scale_pt || !v_val_tb ||
+      !v_scale_tb || !v_val_pt || !v_scale_pt || !ws)
+    return FAPK_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_val_tb) ||
+      !aligned16(k_val_pt) || !aligned16(v_val_tb) || !aligned16(v_val_pt) ||
+      (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+    return FAPK_ERR_INVALID_ARG;
+  // 64-bit offsets throughout; keep the weight rows inside the TMA coordinate range
+  if ((long long)(P->Hq + 2 * P->Hkv) * 128 > 0x7FFFFFFFLL) return FAPK_ERR_UNSUPPORTED;
+  const FwdLayout L = fwd_layout(P);  // the MXFP8 forward's work order: 128-row tiles per document
+  if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
+  const int sms = device_num_sms();
+  if (sms <= 0) return FAPK_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* status = static_cast<DeviceStatus*>(ws);
+  QkvProjArgs a;
+  a.sched = sched_buf(ws, L.sched);
+  const Marks mk{P->timing_events, P->n_timing_events};
+  mk.at(0, st);
+  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, a.sched, status, true, st));
+  if (rc != FAPK_OK) return rc;
+  a.x = x; a.w = w; a.q = q; a.k = k; a.v = v;
+  a.k_vtb = k_val_tb; a.k_stb = k_scale_tb; a.k_vpt = k_val_pt; a.k_spt = k_scale_pt;
+  a.v_vtb = v_val_tb; a.v_stb = v_scale_tb; a.v_vpt = v_val_pt; a.v_spt = v_scale_pt;
+  a.cu = P->cu_seqlens_dev;
+  a.T = P->T; a.Dm = d_model; a.Hq = P->Hq; a.Hkv = P->Hkv;
+  a.rule = P->scale_rule;
+  a.status = status;
+  a.timeout_ns = timeout_ns_of(P);
+  a.num_sms = sms;
+  mk.at(1, st);
+  rc = cuda_status(launch_qkv_proj(a, st));
+  mk.at(2, st);
+  return rc;
+}
+
 int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const int32_t* cu_seqlens_dev,
                         const int32_t* cu_seqlens_host, int n_docs, int forms, int scale_rule,
                         uint8_t* val_tb, uint8_t* scale_tb, uint8_t* val_pt, uint8_t* scale_pt,

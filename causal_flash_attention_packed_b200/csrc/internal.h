@@ -183,6 +183,25 @@ struct BwdMxArgs {
 };
 cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream);
 
+// Fused QKV projection with the MX quantisation of K and V in its epilogue
+// (qkv_proj.cu).  x [T][Dm] bf16, w [(Hq + 2 Hkv) 128][Dm] bf16; outputs q
+// [T][Hq][128], k, v [T][Hkv][128] bf16 and K's and V's MX forms.
+struct QkvProjArgs {
+  const void* x;
+  const void* w;
+  void *q, *k, *v;
+  uint8_t *k_vtb, *k_stb, *k_vpt, *k_spt;
+  uint8_t *v_vtb, *v_stb, *v_vpt, *v_spt;
+  const int32_t* cu;
+  int T, Dm, Hq, Hkv;
+  int rule;
+  SchedBuf sched;  // 128-row tiles per document
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+  int num_sms;
+};
+cudaError_t launch_qkv_proj(const QkvProjArgs& a, cudaStream_t stream);
+
 // Tensor map of E4M3 codes [T][H][128] as (128, H, T), box 128 x 1 x 128,
 // 128-byte swizzle (api.cu).
 bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H);

@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
     L.fapk_attn_fwd_noalloc.restype = i
     L.fapk_attn_fwd_quantized_kv.argtypes = [PP] + [vp] * 11 + [sz, vp]
     L.fapk_attn_fwd_quantized_kv.restype = i
+    L.fapk_qkv_proj_mxfp8.argtypes = [PP, vp, i, vp, vp, vp, vp] + [vp] * 8 + [vp, sz, vp]
+    L.fapk_qkv_proj_mxfp8.restype = i
     L.fapk_noalloc_status.argtypes = [vp]
     L.fapk_noalloc_status.restype = i
     L.fapk_quantize_mxfp8.argtypes = [vp, i, i, i, vp, vp, i, i, i, vp, vp, vp, vp, vp]
@@ -258,6 +260,35 @@ def attn_fwd_quantized_kv(P: Problem, q, k_forms: dict, v_forms: dict, o=None, l
                                           _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "fapk_attn_fwd_quantized_kv")
     return o, lse
+
+
+def qkv_proj_mxfp8(P: Problem, x: torch.Tensor, w: torch.Tensor, ws=None, stream=None):
+    """fapk_qkv_proj_mxfp8: [Q | K | V] = x w^T with K's and V's MX forms from
+    the epilogue.  x [T, d_model] bf16, w [(Hq + 2 Hkv) d, d_model] bf16.
+    Returns (q, k, v, k_forms, v_forms); the forms are dicts like
+    quantize_mxfp8's, ready for attn_fwd_quantized_kv."""
+    dev = x.device
+    T, Dm = x.shape
+    q = torch.empty((T, P.Hq, P.d), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((T, P.Hkv, P.d), dtype=torch.bfloat16, device=dev)
+    v = torch.empty((T, P.Hkv, P.d), dtype=torch.bfloat16, device=dev)
+
+    def forms():
+        return {"val_tb": torch.empty((T, P.Hkv, P.d), dtype=torch.uint8, device=dev),
+                "scale_tb": torch.full((tb_slots(T, P.n_docs), P.Hkv, P.d // 32), 0xFF, dtype=torch.uint8,
+                                       device=dev),
+                "val_pt": torch.empty((T, P.Hkv, P.d), dtype=torch.uint8, device=dev),
+                "scale_pt": torch.empty((T, P.Hkv, P.d // 32), dtype=torch.uint8, device=dev)}
+
+    kf, vf = forms(), forms()
+    if ws is None:
+        ws = workspace(P, FWD, dev)
+    f = [kf[n] for n in ("val_tb", "scale_tb", "val_pt", "scale_pt")] + \
+        [vf[n] for n in ("val_tb", "scale_tb", "val_pt", "scale_pt")]
+    rc = lib().fapk_qkv_proj_mxfp8(ctypes.byref(P), _ptr(x), Dm, _ptr(w), _ptr(q), _ptr(k), _ptr(v),
+                                   *[_ptr(t) for t in f], _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "fapk_qkv_proj_mxfp8")
+    return q, k, v, kf, vf
 
 
 def attn_bwd(P: Problem, q, k, v, o, lse, dout, ctx=None, dq=None, dk=None, dv=None, ws=None,

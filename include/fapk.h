@@ -231,6 +231,32 @@ FAPK_API int fapk_attn_fwd_quantized_kv(const fapk_problem_t* prob, const void* 
                                         const uint8_t* v_scale_pt, void* o, float* lse, void* ws,
                                         size_t ws_bytes, void* stream);
 
+/* Fused QKV projection with MXFP8 quantisation of K and V in its epilogue
+ * ("GPT Kernel Programlama: MatMul, Softmax ve Attention Hesabi", sec. 2: the
+ * three projections as one fused QKV projection; FLAMIA page, sec. "FLAMIA
+ * Mimarisi ve Temel Tasarim Ilkeleri": fused quantisation, document-local
+ * scales over packed layouts).  One tensor-core GEMM [Q | K | V] = X W^T over
+ * the packed tokens:
+ *   x: [T][d_model] bf16 (d_model a multiple of 8);
+ *   w: [(Hq + 2 Hkv) d][d_model] bf16, the rows of the Q heads, then the K
+ *      heads, then the V heads (the usual out x in layout of a linear layer);
+ *   q: [T][Hq][d], k, v: [T][Hkv][d] bf16, the fp32 products rounded to
+ *      nearest even;
+ *   K's and V's token-block and per-token MX forms, quantised from those bf16
+ *   values with prob's cu_seqlens and scale rule, in the layout of
+ *   fapk_quantize_mxfp8 (codes [T][Hkv][128], 16-byte aligned; scales
+ *   [T/32 + n_docs][Hkv][4] and [T][Hkv][4]), ready for
+ *   fapk_attn_fwd_quantized_kv, which then launches no quantisation.
+ * prob->prec must be FAPK_MXFP8 and prob->d 128 (FAPK_ERR_UNSUPPORTED
+ * otherwise).  ws: at least fapk_workspace_size(prob, FAPK_FWD) bytes (the
+ * same work order as the MXFP8 forward).  Asynchronous like the other calls;
+ * the device status word is read with fapk_status(ws). */
+FAPK_API int fapk_qkv_proj_mxfp8(const fapk_problem_t* prob, const void* x, int d_model, const void* w,
+                                 void* q, void* k, void* v, uint8_t* k_val_tb, uint8_t* k_scale_tb,
+                                 uint8_t* k_val_pt, uint8_t* k_scale_pt, uint8_t* v_val_tb,
+                                 uint8_t* v_scale_tb, uint8_t* v_val_pt, uint8_t* v_scale_pt, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 /* Forward that allocates nothing.  The pages have no counterpart: this entry
  * point exists for callers that cannot obtain device memory where they run the
  * forward -- a plugin handed its buffers by a host framework that must not

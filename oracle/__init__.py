@@ -208,6 +208,22 @@ def attn_kv_cols_from_rows(q, k, v, do, o, lse, cu, scale, tok, kvhead):
     return dk, dv
 
 
+def qkv_proj(x, w, Hq: int, Hkv: int, d: int):
+    """Fused QKV projection, exact ("GPT Kernel Programlama" page, sec. 2: the
+    three projections of X as one): Y = X W^T in fp64 (a library matmul), its
+    columns split into the Q heads, then the K heads, then the V heads.
+    x [T, d_model], w [(Hq + 2 Hkv) d, d_model]; returns q [T, Hq, d],
+    k, v [T, Hkv, d]."""
+    x, w = _f64(x), _f64(w)
+    T = x.shape[0]
+    assert w.shape == ((Hq + 2 * Hkv) * d, x.shape[1])
+    y = x @ w.T
+    q = y[:, : Hq * d].reshape(T, Hq, d)
+    k = y[:, Hq * d: (Hq + Hkv) * d].reshape(T, Hkv, d)
+    v = y[:, (Hq + Hkv) * d:].reshape(T, Hkv, d)
+    return q, k, v
+
+
 # ---- MXFP8 quantiser ----------------------------------------------------
 
 def e4m3_encode(y: float) -> int:

@@ -246,3 +246,27 @@ def test_future_perturbation_leaves_past_bit_identical(orc):
     b = orc.attn_bwd(q2, k2, v2, do2, cu, sc)
     for key in ("dk", "dv"):
         np.testing.assert_array_equal(a[key][: t + 1], b[key][: t + 1])
+
+
+def test_qkv_projection_split(orc):
+    """The projection's head split: with d_model = (Hq + 2 Hkv) d and W the
+    identity, q, k and v are consecutive column slices of x (Q heads first,
+    then K, then V); a permutation of W's rows permutes the outputs the same
+    way.  Fails a wrong head order or a transposed W."""
+    rng = np.random.default_rng(12)
+    Hq, Hkv, d, T = 2, 1, 4, 5
+    n = (Hq + 2 * Hkv) * d
+    x = rng.standard_normal((T, n))
+    q, k, v = orc.qkv_proj(x, np.eye(n), Hq, Hkv, d)
+    np.testing.assert_array_equal(q.reshape(T, -1), x[:, : Hq * d])
+    np.testing.assert_array_equal(k.reshape(T, -1), x[:, Hq * d: (Hq + Hkv) * d])
+    np.testing.assert_array_equal(v.reshape(T, -1), x[:, (Hq + Hkv) * d:])
+    perm = rng.permutation(n)
+    q2, k2, v2 = orc.qkv_proj(x, np.eye(n)[perm], Hq, Hkv, d)
+    y2 = np.concatenate([q2.reshape(T, -1), k2.reshape(T, -1), v2.reshape(T, -1)], axis=1)
+    np.testing.assert_array_equal(y2, x[:, perm])
+    # a non-square W: row r of W gives output column r
+    w = rng.standard_normal((n, 3))
+    x3 = rng.standard_normal((T, 3))
+    q3, _, _ = orc.qkv_proj(x3, w, Hq, Hkv, d)
+    assert abs(q3[2, 1, 3] - float(x3[2] @ w[1 * d + 3])) < 1e-13
