@@ -316,3 +316,30 @@ def test_multi_query_attention_fwd_bwd():
     w = W.custom([1, 129, 300, 700, 64], Hq=8, Hkv=1, d=128, seed=79)
     _check(w, require_gpu())
     _check_bwd(w, require_gpu())
+
+
+def test_zero_length_and_one_token_documents():
+    """Zero-length documents produce nothing and one-token documents attend to
+    themselves only (O = their own V~): forward and backward against the
+    emulation, with every other output finite."""
+    w = W.custom([0, 1, 40, 0, 0, 1, 257, 1, 0], Hq=2, Hkv=1, d=128, seed=80)
+    _check(w, require_gpu())
+    _check_bwd(w, require_gpu())
+
+
+def test_bf16_gradient_output():
+    """grad_dtype = bf16 in the MXFP8 path: the gradients are the fp32 ones
+    rounded to bf16 (within half a bf16 ulp of the fp32-output run)."""
+    dev = require_gpu()
+    w = W.custom([200, 513, 64], Hq=4, Hkv=2, d=128, seed=81)
+    (q, k, v, do), (qd, kd, vd, dod) = to_dev(w, dev)
+    seq = fapk.Seqlens(w.cu, dev)
+    outs = []
+    for gdt in (fapk.GRAD_F32, fapk.GRAD_BF16):
+        P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale, prec=fapk.MXFP8, grad_dtype=gdt)
+        o, lse, ctx = fapk.attn_fwd(P, qd, kd, vd)
+        outs.append(fapk.attn_bwd(P, qd, kd, vd, o, lse, dod, ctx=ctx))
+    torch.cuda.synchronize()
+    for a, b in zip(*outs):
+        assert b.dtype == torch.bfloat16
+        assert torch.equal(a.to(torch.bfloat16), b)
