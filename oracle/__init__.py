@@ -16,7 +16,11 @@ The MXFP8 emulation (``mx_attn_fwd`` / ``mx_attn_bwd``) is pinned by its
 exact limit on on-grid inputs, its cosine to the exact path, the leak tests run
 on it, hand-derived cases of the operand selection (forward and backward) and
 of the forward's P~, and element-by-element read-outs of the blocks in which
-dS~, P~T and dS~T are quantised (tests/test_oracle_mx*.py).
+dS~, P~T and dS~T are quantised (tests/test_oracle_mx*.py).  The mixed
+NVFP4/FP8 path (``nvmx_attn_fwd`` / ``nvmx_attn_bwd``: the scores from NVFP4 Q
+and K) and its quantiser are pinned by the E2M1 and E4M3 grids, hand-worked
+blocks, the exact limit on on-grid inputs and a hand-derived score
+(tests/test_oracle_nvfp4.py).
 """
 from __future__ import annotations
 
@@ -81,6 +85,16 @@ def _load():
     lib.orc_quantize_mxfp8.argtypes = [P, i, i, i, P, i, i, i, P, P, P, P]
     lib.orc_mx_attn_fwd.argtypes = head + [P, P, P, i, P, P]
     lib.orc_mx_attn_bwd.argtypes = head + [P, P, P, P, i, P, P, P, P, P]
+    f32 = ctypes.c_float
+    lib.orc_e2m1_encode.argtypes = [dbl]
+    lib.orc_e2m1_encode.restype = ctypes.c_uint8
+    lib.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+    lib.orc_e2m1_decode.restype = dbl
+    lib.orc_nv_quant_block.argtypes = [P, i, f32, P, P]
+    lib.orc_nv_quant_block.restype = ctypes.c_uint8
+    lib.orc_quantize_nvfp4.argtypes = [P, i, i, i, f32, P, P]
+    lib.orc_nvmx_attn_fwd.argtypes = head + [P, P, P, i, f32, f32, P, P]
+    lib.orc_nvmx_attn_bwd.argtypes = head + [P, P, P, P, i, f32, f32, P, P, P, P, P]
     _lib = lib
     return lib
 
@@ -293,6 +307,59 @@ def mx_attn_bwd(q, k, v, do, cu, scale, flags: int = MX_QUANT_P):
     _load().orc_mx_attn_bwd(T, nd, _ptr(cu), Hq, Hkv, d, float(scale), _ptr(q), _ptr(k),
                             _ptr(v), _ptr(do), int(flags), _ptr(out["o"]), _ptr(out["lse"]),
                             _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]))
+    return out
+
+
+# ---- mixed NVFP4/FP8 path --------------------------------------------------
+
+def e2m1_encode(y: float) -> int:
+    return int(_load().orc_e2m1_encode(float(y)))
+
+
+def e2m1_decode(code: int) -> float:
+    return float(_load().orc_e2m1_decode(int(code)))
+
+
+def nv_quant_block(x, g: float = 1.0):
+    """One NVFP4 block: returns (E2M1 codes uint8[n], dequantised f64[n], E4M3 scale byte)."""
+    x = _f64(x)
+    codes = np.zeros(len(x), np.uint8)
+    deq = np.zeros(len(x))
+    sb = _load().orc_nv_quant_block(_ptr(x), len(x), float(g), _ptr(codes), _ptr(deq))
+    return codes, deq, int(sb)
+
+
+def quantize_nvfp4(x, g: float = 1.0):
+    """NVFP4 of a [T,H,d] bf16-valued tensor: (codes uint8 [T,H,d/2], channel
+    2i in the low nibble; scales uint8 [T,H,d/16])."""
+    x = _f64(x)
+    T, H, d = x.shape
+    codes = np.zeros((T, H, d // 2), np.uint8)
+    scales = np.zeros((T, H, d // 16), np.uint8)
+    _load().orc_quantize_nvfp4(_ptr(x), T, H, d, float(g), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def nvmx_attn_fwd(q, k, v, cu, scale, flags: int = MX_QUANT_P, gq: float = 1.0, gk: float = 1.0):
+    """Mixed NVFP4/FP8 emulation forward: (O, LSE) in fp64."""
+    q, k, v, cu = _f64(q), _f64(k), _f64(v), _i32(cu)
+    T, nd, Hq, Hkv, d = _dims(q, k, cu)
+    o = np.zeros((T, Hq, d))
+    lse = np.zeros((Hq, T))
+    _load().orc_nvmx_attn_fwd(T, nd, _ptr(cu), Hq, Hkv, d, float(scale), _ptr(q), _ptr(k), _ptr(v),
+                              int(flags), float(gq), float(gk), _ptr(o), _ptr(lse))
+    return o, lse
+
+
+def nvmx_attn_bwd(q, k, v, do, cu, scale, flags: int = MX_QUANT_P, gq: float = 1.0, gk: float = 1.0):
+    """Mixed NVFP4/FP8 emulation forward + backward: dict o, lse, dq, dk, dv."""
+    q, k, v, do, cu = _f64(q), _f64(k), _f64(v), _f64(do), _i32(cu)
+    T, nd, Hq, Hkv, d = _dims(q, k, cu)
+    out = dict(o=np.zeros((T, Hq, d)), lse=np.zeros((Hq, T)), dq=np.zeros((T, Hq, d)),
+               dk=np.zeros((T, Hkv, d)), dv=np.zeros((T, Hkv, d)))
+    _load().orc_nvmx_attn_bwd(T, nd, _ptr(cu), Hq, Hkv, d, float(scale), _ptr(q), _ptr(k),
+                              _ptr(v), _ptr(do), int(flags), float(gq), float(gk), _ptr(out["o"]),
+                              _ptr(out["lse"]), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]))
     return out
 
 

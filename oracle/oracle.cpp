@@ -45,6 +45,20 @@
  *        Microscaling v1.0 rule, under which block maxima whose significand
  *        exceeds 1.75 saturate to 448.
  *    (Block size and formats from the benchmark spec.)
+ *  - mixed NVFP4/FP8 path ([FLAMIA] names "mixed NVFP4/FP8 training paths"
+ *    without giving the split): the scores S = Q K^T, in the forward and in
+ *    the backward's recomputation alike (fwd/bwd consistency), take Q and K
+ *    in NVFP4; every other product is the MXFP8 path's.  NVFP4 is NVIDIA's
+ *    published format (the pages only name it): E2M1 element codes, one
+ *    unsigned E4M3 scale per 16 consecutive channels of one token, and one
+ *    fp32 decode scale g per tensor, x ~ code * scale * g.  Quantisation of a
+ *    block with largest magnitude a, in fp32 arithmetic (each step rounded to
+ *    nearest even):  s = E4M3(a / (6 g)) (saturating at 448),
+ *    r = 1 / (decode(s) g) (0 when that is 0), code_i = E2M1(x_i r)
+ *    (saturating at 6; a zero result is code 0).  g is the caller's (a
+ *    tensor-wide amax of this batch would let later tokens set the scale of
+ *    earlier ones); the blocks lie along channels inside one token, so no
+ *    leak guard is needed for them.
  *  - token blocks are document-local: block m of document k covers tokens
  *    [s_k + 32m, min(s_k + 32m + 32, e_k)); its scale lives in slot
  *    floor(s_k/32) + k + m of a [T/32 + n_docs] slot array.
@@ -307,6 +321,76 @@ void mx_forms(const double* x, int s, int L, int h, int H, int d, int rule,
     }
   }
 }
+
+/* ---- NVFP4 (mixed path) ------------------------------------------------- */
+
+/* E2M1 code of y: round to nearest, ties to the even code, saturate to +-6;
+ * 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit: magnitudes
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6 for codes 0..7.  A zero result is code 0. */
+uint8_t e2m1_encode(double y) {
+  const double a = std::fabs(y);
+  double qv;
+  if (a >= 6.0) {
+    qv = 6.0;
+  } else {
+    const int e = a < 1.0 ? 0 : floor_log2(a);     // below 1: the subnormal quantum 0.5
+    const double quantum = std::ldexp(1.0, e - 1);  // one mantissa bit
+    qv = std::min(6.0, rne(a / quantum) * quantum);
+  }
+  if (qv == 0.0) return 0;
+  uint8_t mag;
+  if (qv < 1.0)
+    mag = 1;  // 0.5, subnormal
+  else {
+    const int e2 = floor_log2(qv);
+    mag = (uint8_t)(((e2 + 1) << 1) | (qv > std::ldexp(1.0, e2) ? 1 : 0));
+  }
+  return (uint8_t)((y < 0.0 ? 8 : 0) | mag);
+}
+
+double e2m1_decode(uint8_t c) {
+  const int mag = c & 7, e = mag >> 1, m = mag & 1;
+  const double v = e == 0 ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, e - 1);
+  return (c & 8) ? -v : v;
+}
+
+/* One NVFP4 block of n (16) values x[0..n) (bf16 values, exact in fp32) with
+ * the tensor's decode scale g: codes (E2M1, one per value), dequantised
+ * values code * decode(s) * g (fp64), returns the E4M3 scale byte s.  The
+ * arithmetic is fp32, step by step as the format's quantisation states it. */
+uint8_t nv_quant_block(const double* x, int n, float g, uint8_t* codes, double* deq) {
+  float a = 0.f;
+  for (int i = 0; i < n; ++i) a = std::max(a, std::fabs((float)x[i]));
+  const float six_g = 6.0f * g;
+  const float t = a / six_g;
+  const uint8_t sbyte = e4m3_encode((double)t);  // t >= 0: an unsigned E4M3
+  const float sg = (float)e4m3_decode(sbyte) * g;
+  const float r = sg > 0.f ? 1.0f / sg : 0.f;
+  for (int i = 0; i < n; ++i) {
+    const float y = (float)x[i] * r;
+    const uint8_t c = e2m1_encode((double)y);
+    if (codes) codes[i] = c;
+    if (deq) deq[i] = e2m1_decode(c) * e4m3_decode(sbyte) * (double)g;
+  }
+  return sbyte;
+}
+
+/* Dequantised NVFP4 form of one (document, head) slice: [L][d], per token,
+ * 16-channel blocks. */
+void nv_form(const double* x, int s, int L, int h, int H, int d, float g, std::vector<double>& out) {
+  std::vector<double> xs;
+  slice_n(x, s, L, h, H, d, xs);
+  out.assign((size_t)L * d, 0.0);
+  for (int j = 0; j < L; ++j)
+    for (int c0 = 0; c0 < d; c0 += 16)
+      nv_quant_block(&xs[(size_t)j * d + c0], 16, g, nullptr, &out[(size_t)j * d + c0]);
+}
+
+/* The mixed path's option: S from NVFP4 Q and K with decode scales gq, gk. */
+struct NvOpt {
+  bool on;
+  float gq, gk;
+};
 
 /* Rule L operand selection: per-token form on the diagonal block, token-block
  * form elsewhere. */
@@ -682,9 +766,13 @@ void orc_quantize_mxfp8(const double* x, int T, int H, int d, const int32_t* cu,
  * (row, key block) in the integer-power-of-two form of fwd_p_tilde when
  * flags & MX_QUANT_P; O = sum_j P~_ij V~_j (rule L); LSE from the quantised
  * S.  Every scale uses rule_of(flags). */
-void orc_mx_attn_fwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
-                     const double* q, const double* k, const double* v, int flags, double* o,
-                     double* lse) {
+}  // extern "C"
+
+namespace {
+
+void mx_attn_fwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
+                 const double* q, const double* k, const double* v, int flags, const NvOpt& nv,
+                 double* o, double* lse) {
   const Problem P{T, nd, Hq, Hkv, d, cu, scale};
   const std::vector<Task> tasks = head_doc_tasks(P, Hq);
   const bool qp = quant_p(flags), ex = flags & MX_KEEP_INPUTS;
@@ -697,9 +785,16 @@ void orc_mx_attn_fwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
     mx_forms(q, s, L, h, Hq, d, rule, Qtb, Qpt, ex);
     mx_forms(k, s, L, g, Hkv, d, rule, Ktb, Kpt, ex);
     mx_forms(v, s, L, g, Hkv, d, rule, Vtb, Vpt, ex);
+    // the scores' operands: Q~pt and K~ by rule L, or NVFP4 Q and K (mixed path)
+    std::vector<double> Qs, Ks;
+    if (nv.on) {
+      nv_form(q, s, L, h, Hq, d, nv.gq, Qs);
+      nv_form(k, s, L, g, Hkv, d, nv.gk, Ks);
+    }
     for (int li = 0; li < L; ++li) {
       double m, l;
-      const int n = mx_score_row(&Qpt[(size_t)li * d], Ktb, Kpt, li, d, scale, srow, p, m, l);
+      const int n = nv.on ? mx_score_row(&Qs[(size_t)li * d], Ks, Ks, li, d, scale, srow, p, m, l)
+                          : mx_score_row(&Qpt[(size_t)li * d], Ktb, Kpt, li, d, scale, srow, p, m, l);
       fwd_p_tilde(srow, n, qp, rule, pq);
       std::fill(orow.begin(), orow.end(), 0.0);
       for (int j = 0; j < n; ++j) {
@@ -723,9 +818,9 @@ void orc_mx_attn_fwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
  *   dQ_i  = scale sum_j dS~_ij K~_j            (dS~ per (row, key block))
  *   dK_j  = scale sum_i dS~T_ji Q~tb_i         (dS~T per (key, query block))
  *   dV_j  =       sum_i P~T_ji dO~tb_i         (P~T per (key, query block)) */
-void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
-                     const double* q, const double* k, const double* v, const double* dout,
-                     int flags, double* o, double* lse, double* dq, double* dk, double* dv) {
+void mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
+                 const double* q, const double* k, const double* v, const double* dout, int flags,
+                 const NvOpt& nv, double* o, double* lse, double* dq, double* dk, double* dv) {
   const Problem P{T, nd, Hq, Hkv, d, cu, scale};
   const int G = P.G();
   const bool qp = quant_p(flags), qds = quant_ds(flags), ex = flags & MX_KEEP_INPUTS;
@@ -736,13 +831,15 @@ void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
   for (long ti = 0; ti < (long)tasks.size(); ++ti) {
     const int kdoc = tasks[ti].doc, g = tasks[ti].h;
     const int s = cu[kdoc], L = cu[kdoc + 1] - cu[kdoc];
-    std::vector<double> Ktb, Kpt, Vtb, Vpt, Qtb, Qpt, dOtb, dOpt, srow, p, pq, orow(d);
+    std::vector<double> Ktb, Kpt, Vtb, Vpt, Qtb, Qpt, dOtb, dOpt, srow, p, pq, orow(d), Qs, Ks;
     mx_forms(k, s, L, g, Hkv, d, rule, Ktb, Kpt, ex);
     mx_forms(v, s, L, g, Hkv, d, rule, Vtb, Vpt, ex);
+    if (nv.on) nv_form(k, s, L, g, Hkv, d, nv.gk, Ks);
     std::vector<double> dK((size_t)L * d, 0.0), dV((size_t)L * d, 0.0);
     for (int h = g * G; h < (g + 1) * G; ++h) {
       mx_forms(q, s, L, h, Hq, d, rule, Qtb, Qpt, ex);
       mx_forms(dout, s, L, h, Hq, d, rule, dOtb, dOpt, ex);
+      if (nv.on) nv_form(q, s, L, h, Hq, d, nv.gq, Qs);
       // rows are processed in 32-row query blocks so that P^T and dS^T can be
       // quantised per (key row, query block)
       for (int b0 = 0; b0 < L; b0 += 32) {
@@ -752,7 +849,9 @@ void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
         for (int a = 0; a < nb; ++a) {
           const int li = b0 + a, i = s + li;
           double m, l;
-          const int n = mx_score_row(&Qpt[(size_t)li * d], Ktb, Kpt, li, d, scale, srow, p, m, l);
+          // the same scores as the forward's (NVFP4 Q and K on the mixed path)
+          const int n = nv.on ? mx_score_row(&Qs[(size_t)li * d], Ks, Ks, li, d, scale, srow, p, m, l)
+                              : mx_score_row(&Qpt[(size_t)li * d], Ktb, Kpt, li, d, scale, srow, p, m, l);
           fwd_p_tilde(srow, n, qp, rule, pq);
           std::fill(orow.begin(), orow.end(), 0.0);
           for (int j = 0; j < n; ++j) {
@@ -817,6 +916,65 @@ void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, d
         dv[idx3(s + j, g, r, Hkv, d)] = dV[(size_t)j * d + r];
       }
   }
+}
+
+}  // namespace
+
+extern "C" {
+
+void orc_mx_attn_fwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
+                     const double* q, const double* k, const double* v, int flags, double* o,
+                     double* lse) {
+  mx_attn_fwd(T, nd, cu, Hq, Hkv, d, scale, q, k, v, flags, NvOpt{false, 1.f, 1.f}, o, lse);
+}
+
+void orc_mx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
+                     const double* q, const double* k, const double* v, const double* dout,
+                     int flags, double* o, double* lse, double* dq, double* dk, double* dv) {
+  mx_attn_bwd(T, nd, cu, Hq, Hkv, d, scale, q, k, v, dout, flags, NvOpt{false, 1.f, 1.f}, o, lse, dq,
+              dk, dv);
+}
+
+/* ---- mixed NVFP4/FP8 path ------------------------------------------------ */
+
+uint8_t orc_e2m1_encode(double y) { return e2m1_encode(y); }
+double orc_e2m1_decode(uint8_t c) { return e2m1_decode(c); }
+
+/* One NVFP4 block of n values with decode scale g: codes (one per value),
+ * dequantised values; returns the E4M3 scale byte. */
+uint8_t orc_nv_quant_block(const double* x, int n, float g, uint8_t* codes, double* deq) {
+  return nv_quant_block(x, n, g, codes, deq);
+}
+
+/* NVFP4 of a bf16-valued [T][H][d] tensor (exact doubles), decode scale g:
+ * codes [T][H][d/2] (channel 2i in the low nibble of byte i, 2i + 1 in the
+ * high nibble), scales [T][H][d/16]. */
+void orc_quantize_nvfp4(const double* x, int T, int H, int d, float g, uint8_t* codes, uint8_t* scales) {
+#pragma omp parallel for schedule(static)
+  for (long t = 0; t < (long)T; ++t)
+    for (int h = 0; h < H; ++h)
+      for (int b = 0; b < d / 16; ++b) {
+        uint8_t c[16];
+        const size_t o = idx3((int)t, h, 16 * b, H, d);
+        scales[((size_t)t * H + h) * (d / 16) + b] = nv_quant_block(&x[o], 16, g, c, nullptr);
+        for (int i = 0; i < 8; ++i) codes[o / 2 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+      }
+}
+
+/* The mixed path's forward and backward: the MXFP8 emulation with the scores
+ * taken from NVFP4 Q and K (decode scales gq, gk), in both passes. */
+void orc_nvmx_attn_fwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
+                       const double* q, const double* k, const double* v, int flags, float gq, float gk,
+                       double* o, double* lse) {
+  mx_attn_fwd(T, nd, cu, Hq, Hkv, d, scale, q, k, v, flags, NvOpt{true, gq, gk}, o, lse);
+}
+
+void orc_nvmx_attn_bwd(int T, int nd, const int32_t* cu, int Hq, int Hkv, int d, double scale,
+                       const double* q, const double* k, const double* v, const double* dout,
+                       int flags, float gq, float gk, double* o, double* lse, double* dq, double* dk,
+                       double* dv) {
+  mx_attn_bwd(T, nd, cu, Hq, Hkv, d, scale, q, k, v, dout, flags, NvOpt{true, gq, gk}, o, lse, dq, dk,
+              dv);
 }
 
 }  // extern "C"
