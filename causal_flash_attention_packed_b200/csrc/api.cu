@@ -59,16 +59,28 @@ int device_num_sms() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // --- problem validation ---
+// The MXFP8 machinery (quantised forms in ctx, the MX kernels) serves both
+// low-precision paths.
+bool is_mx(const fapk_problem_t* P) { return P->prec == FAPK_MXFP8 || P->prec == FAPK_NVFP4_MIXED; }
+// An NVFP4 decode scale: 0 (selects 1) or a finite value in [2^-100, 2^100],
+// so that no step of the quantisation overflows fp32.
+bool nv_scale_ok(float g) { return g == 0.f || (std::isfinite(g) && g >= 0x1p-100f && g <= 0x1p100f); }
+float nv_scale_of(float g) { return g == 0.f ? 1.f : g; }
+
 int validate_problem(const fapk_problem_t* P) {
   if (!P) return FAPK_ERR_INVALID_ARG;
   if (P->T < 0 || P->n_docs < 0 || P->Hq <= 0 || P->Hkv <= 0) return FAPK_ERR_INVALID_ARG;
   if (P->d != 64 && P->d != 128) return FAPK_ERR_UNSUPPORTED;
   if (P->Hq % P->Hkv != 0) return FAPK_ERR_UNSUPPORTED;
-  if (P->prec != FAPK_BF16 && P->prec != FAPK_MXFP8) return FAPK_ERR_UNSUPPORTED;
+  if (P->prec != FAPK_BF16 && P->prec != FAPK_MXFP8 && P->prec != FAPK_NVFP4_MIXED) return FAPK_ERR_UNSUPPORTED;
   if (P->scale_rule != FAPK_SCALE_RCEIL && P->scale_rule != FAPK_SCALE_OCP) return FAPK_ERR_UNSUPPORTED;
   // the attention path quantises with RCEIL only: under OCP the computed
   // operands quantise discontinuously near powers of two (see fapk.h)
-  if (P->prec == FAPK_MXFP8 && P->scale_rule != FAPK_SCALE_RCEIL) return FAPK_ERR_UNSUPPORTED;
+  if (is_mx(P) && P->scale_rule != FAPK_SCALE_RCEIL) return FAPK_ERR_UNSUPPORTED;
+  if (P->prec == FAPK_NVFP4_MIXED) {
+    if (P->d != 128) return FAPK_ERR_UNSUPPORTED;
+    if (!nv_scale_ok(P->nv_scale_q) || !nv_scale_ok(P->nv_scale_k)) return FAPK_ERR_INVALID_ARG;
+  }
   if (P->grad_dtype != FAPK_GRAD_F32 && P->grad_dtype != FAPK_GRAD_BF16) return FAPK_ERR_UNSUPPORTED;
   if (!std::isfinite(P->scale)) return FAPK_ERR_INVALID_ARG;
   if (P->T > 0) {
@@ -135,7 +147,7 @@ struct FwdLayout {
 FwdLayout fwd_layout(const fapk_problem_t* P) {
   FwdLayout L;
   L.sched = sched_layout(kAlign, P->T, P->n_docs, P->max_seqlen,
-                         P->prec == FAPK_MXFP8 ? kFwdRowsMx : kFwdRows);
+                         is_mx(P) ? kFwdRowsMx : kFwdRows);
   L.cta_times = align_up(L.sched.end);
   L.total = align_up(L.cta_times + sizeof(unsigned long long) * kCtaTimesWords);
   return L;
@@ -156,7 +168,7 @@ BwdLayout bwd_layout(const fapk_problem_t* P) {
   L.q = sched_layout(L.kv.end, P->T, P->n_docs, P->max_seqlen, kBwdRows);
   L.delta = L.q.end;
   const size_t after_delta = align_up(L.delta + sizeof(float) * (size_t)P->Hq * (size_t)P->T);
-  if (P->prec == FAPK_MXFP8) {
+  if (is_mx(P)) {
     const size_t slots = (size_t)P->T / 32 + P->n_docs;
     L.q16 = L.k16 = L.do16 = 0;
     // dO's MX forms, 128 codes and 4 scale bytes per (token, head) for any d
@@ -194,12 +206,14 @@ struct MxForms {
 struct CtxLayout {
   size_t o_resid, v16, total;
   MxForms q, k, v;
+  // mixed NVFP4/FP8 path: NVFP4 codes [T][H][64] and scales [T][H][8] of Q and K
+  size_t q_nvv = 0, q_nvs = 0, k_nvv = 0, k_nvs = 0;
 };
 CtxLayout ctx_layout(const fapk_problem_t* P) {
   CtxLayout L;
   L.o_resid = 0;
   size_t off = align_up(sizeof(uint16_t) * (size_t)P->T * P->Hq * P->d);
-  if (P->prec != FAPK_MXFP8) {
+  if (!is_mx(P)) {
     L.v16 = off;
     L.total = align_up(L.v16 + sizeof(uint16_t) * (size_t)P->T * P->Hkv * P->d);
     return L;
@@ -221,6 +235,13 @@ CtxLayout ctx_layout(const fapk_problem_t* P) {
   L.q = forms(P->Hq);
   L.k = forms(P->Hkv);
   L.v = forms(P->Hkv);
+  if (P->prec == FAPK_NVFP4_MIXED) {
+    L.q_nvv = off;
+    L.q_nvs = align_up(L.q_nvv + (size_t)P->T * P->Hq * 64);
+    L.k_nvv = align_up(L.q_nvs + (size_t)P->T * P->Hq * 8);
+    L.k_nvs = align_up(L.k_nvv + (size_t)P->T * P->Hkv * 64);
+    off = align_up(L.k_nvs + (size_t)P->T * P->Hkv * 8);
+  }
   L.total = off;
   return L;
 }
@@ -240,6 +261,18 @@ bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H) {
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_nv(CUtensorMap* map, const void* base, int T, int H) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {64, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {64, (cuuint64_t)H * 64};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -279,6 +312,21 @@ int fwd_mxfp8(const fapk_problem_t* P, const void* q, const void* k, const void*
                          u8(C.k.spt), nullptr, true};
   jobs.job[1] = QuantJob{static_cast<const __nv_bfloat16*>(v), P->Hkv, u8(C.v.vtb), u8(C.v.stb), u8(C.v.vpt),
                          u8(C.v.spt), nullptr, true};
+  const bool nv = P->prec == FAPK_NVFP4_MIXED;
+  if (nv) {
+    // K's NVFP4 form for the scores, in the same pass
+    jobs.job[0].nvv = u8(C.k_nvv);
+    jobs.job[0].nvs = u8(C.k_nvs);
+    jobs.job[0].nv_g = nv_scale_of(P->nv_scale_k);
+    jobs.job[0].nv_six_g = 6.0f * jobs.job[0].nv_g;
+    a.nv = true;
+    a.k_nvv = u8(C.k_nvv);
+    a.k_nvs = u8(C.k_nvs);
+    a.q_nvv = u8(C.q_nvv);
+    a.q_nvs = u8(C.q_nvs);
+    a.nv_g_q = nv_scale_of(P->nv_scale_q);
+    a.nv_g_k = nv_scale_of(P->nv_scale_k);
+  }
   rc = cuda_status(launch_quantize_jobs(jobs, 2, P->T, P->d, P->cu_seqlens_dev, P->n_docs,
                                         FAPK_FORM_TB | FAPK_FORM_PT, P->scale_rule, st));
   if (rc != FAPK_OK) return rc;
@@ -341,6 +389,12 @@ int bwd_mxfp8(const fapk_problem_t* P, const void* o, const float* lse, const vo
   a.k_vtb = cu8(C.k.vtb); a.k_stb = cu8(C.k.stb); a.k_vpt = cu8(C.k.vpt); a.k_spt = cu8(C.k.spt);
   a.v_vtb = cu8(C.v.vtb); a.v_stb = cu8(C.v.stb); a.v_vpt = cu8(C.v.vpt); a.v_spt = cu8(C.v.spt);
   a.do_vtb = wu8(L.do_vtb); a.do_stb = wu8(L.do_stb); a.do_vpt = wu8(L.do_vpt); a.do_spt = wu8(L.do_spt);
+  if (P->prec == FAPK_NVFP4_MIXED) {
+    a.nv = true;
+    a.q_nvv = cu8(C.q_nvv); a.q_nvs = cu8(C.q_nvs); a.k_nvv = cu8(C.k_nvv); a.k_nvs = cu8(C.k_nvs);
+    a.nv_g_q = nv_scale_of(P->nv_scale_q);
+    a.nv_g_k = nv_scale_of(P->nv_scale_k);
+  }
   a.o = o;
   a.o_resid = c + C.o_resid;
   a.lse = lse;
@@ -398,7 +452,7 @@ int fapk_attn_fwd(const fapk_problem_t* P, const void* q, const void* k, const v
   if (sms <= 0) return FAPK_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto* status = static_cast<DeviceStatus*>(ws);
-  if (P->prec == FAPK_MXFP8) return fwd_mxfp8(P, q, k, v, o, lse, ctx, ws, L, sms, st);
+  if (is_mx(P)) return fwd_mxfp8(P, q, k, v, o, lse, ctx, ws, L, sms, st);
   FwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
   const CtxLayout CL = ctx_layout(P);
@@ -443,7 +497,7 @@ int fapk_attn_bwd(const fapk_problem_t* P, const void* q, const void* k, const v
   const int sms = device_num_sms();
   if (sms <= 0) return FAPK_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (P->prec == FAPK_MXFP8) return bwd_mxfp8(P, o, lse, dout, ctx, dq, dk, dv, ws, L, sms, st);
+  if (is_mx(P)) return bwd_mxfp8(P, o, lse, dout, ctx, dq, dk, dv, ws, L, sms, st);
   auto* status = static_cast<DeviceStatus*>(ws);
   BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
@@ -602,6 +656,18 @@ int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const int32_t* 
   }
   return cuda_status(launch_quantize_mxfp8(x_bf16, T, H, d, cu_seqlens_dev, n_docs, forms, scale_rule, val_tb,
                                            scale_tb, val_pt, scale_pt, static_cast<cudaStream_t>(stream)));
+}
+
+int fapk_quantize_nvfp4(const void* x_bf16, int T, int H, int d, float g, uint8_t* codes, uint8_t* scales,
+                        void* stream) {
+  if (T < 0 || H <= 0) return FAPK_ERR_INVALID_ARG;
+  if (d != 128) return FAPK_ERR_UNSUPPORTED;
+  if (g == 0.f || !nv_scale_ok(g)) return FAPK_ERR_INVALID_ARG;
+  if (T == 0) return FAPK_OK;
+  if (!x_bf16 || !codes || !scales || !aligned16(x_bf16) || (reinterpret_cast<uintptr_t>(codes) & 7u))
+    return FAPK_ERR_INVALID_ARG;
+  if ((long long)T * H * 8 > 0x7FFFFFFFLL * 256) return FAPK_ERR_UNSUPPORTED;
+  return cuda_status(launch_quantize_nvfp4(x_bf16, T, H, g, codes, scales, static_cast<cudaStream_t>(stream)));
 }
 
 int fapk_cta_times(const fapk_problem_t* P, int which, int kernel, const void* ws, void* stream,

@@ -27,10 +27,17 @@
 //    S^T then dP^T into one TMEM region in turn (TMEM also holds dV, dK and
 //    the scale factors), P~T and dS~T quantised into shared memory,
 //    dV += P~T dO~tb and dK += dS~T Q~tb as block-scaled FP8 MMAs.
+//
+// Mixed NVFP4/FP8 path (kNv): the scores are recomputed from the forward's
+// NVFP4 Q and K (kind::mxf4nvf4, two MMAs of K = 64 per tile), the same
+// product the forward took; the diagonal tile's second score phase repeats
+// it on the same tiles (NVFP4 blocks never pool tokens), so the compute
+// warps run unchanged.  dP and the gradient products are the MXFP8 path's.
 #include <cuda_bf16.h>
 
 #include "internal.h"
 #include "mx.cuh"
+#include "nv.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
 
@@ -129,6 +136,8 @@ struct MxParams {
   const float* lse;
   const float* delta;
   const uint8_t *q_stb, *q_spt, *k_stb, *k_spt, *v_stb, *v_spt, *do_stb, *do_spt;
+  const uint8_t *q_nvs, *k_nvs;  // mixed path: NVFP4 scales of Q [T][Hq][8] and K [T][Hkv][8]
+  const uint8_t* k_vpt;          // mixed path: K per-token codes (dQ's diagonal, read directly)
   void* out0;  // dq | dk
   void* out1;  // -  | dv
   DeviceStatus* status;
@@ -155,7 +164,11 @@ constexpr int oQ = 0, oDO = oQ + kCode, oRing = oDO + kCode;  // ring stage: K^t
 constexpr int oKpt = oRing + kStages * 2 * kCode, oVpt = oKpt + kCode, oKd = oVpt + kCode;  // diag
 constexpr int oDS = oKd + kBf16, oDSd = oDS + kCode;
 constexpr int oSf = oDSd + kBf16;  // sfQ, sfDO, sfKpt, sfVpt, sfDS, per stage {sfK, sfV, sfKdq}
-constexpr int kNumSf = 5 + 3 * kStages;
+// mixed path: the NVFP4 K tile of stage s at oKpt + s kNvTile (the per-token K
+// tile is not loaded: its dequantised copy is read from global memory); Q's
+// second scale block in the sfKpt slot, stage s's second K block at 5 + 3 kStages + s
+constexpr int kNvTile = 128 * 64;
+constexpr int kNumSf = 5 + 4 * kStages;
 constexpr int oBars = oSf + kNumSf * kSfBlk;
 // bars: q_full, q_empty, st_full[S], st_empty[S], s_full, s_free, dp_full, dp_free, ds_ready, dq_done,
 //       acc_full, acc_free, fin, kd_full
@@ -167,14 +180,16 @@ static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may u
 // once), dQ, scale factors
 constexpr uint32_t tS = 0, tDP = 128, tDQ = 256;
 constexpr uint32_t tSfQ = 384, tSfDO = 388, tSfK = 392, tSfV = 396, tSfKpt = 400, tSfVpt = 404, tSfDS = 408,
-                   tSfKdq = 412;
+                   tSfKdq = 412, tSfK2 = 416;  // mixed path: tSfKpt holds Q's second block, tSfK2 K's
 }  // namespace dqk
 
+// kNv: tm_qpt maps Q's NVFP4 codes, tm_knv K's (tm_kpt is not read)
+template <bool kNv>
 __global__ void __launch_bounds__(dqk::kThreads, 1)
     dq_mx_kernel(const __grid_constant__ CUtensorMap tm_qpt, const __grid_constant__ CUtensorMap tm_dopt,
                  const __grid_constant__ CUtensorMap tm_ktb, const __grid_constant__ CUtensorMap tm_vtb,
                  const __grid_constant__ CUtensorMap tm_kpt, const __grid_constant__ CUtensorMap tm_vpt,
-                 const MxParams p) {
+                 const __grid_constant__ CUtensorMap tm_knv, const MxParams p) {
   using namespace dqk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -259,16 +274,25 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       int doc, s, e, h, g, q0, n;
       decode(un, doc, s, e, h, g, q0, n);
       if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 71)) break;
-      reinterpret_cast<uint4*>(sfb(0))[lane] = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
+      if constexpr (kNv) {
+        const uint2 w0 = nv_scale_words(p.q_nvs, q0 + lane, p.T, p.Hq, h);
+        const uint2 w1 = nv_scale_words(p.q_nvs, q0 + lane + 32, p.T, p.Hq, h);
+        const uint2 w2 = nv_scale_words(p.q_nvs, q0 + lane + 64, p.T, p.Hq, h);
+        const uint2 w3 = nv_scale_words(p.q_nvs, q0 + lane + 96, p.T, p.Hq, h);
+        reinterpret_cast<uint4*>(sfb(0))[lane] = make_uint4(w0.x, w1.x, w2.x, w3.x);
+        reinterpret_cast<uint4*>(sfb(2))[lane] = make_uint4(w0.y, w1.y, w2.y, w3.y);
+      } else {
+        reinterpret_cast<uint4*>(sfb(0))[lane] = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
+        reinterpret_cast<uint4*>(sfb(2))[lane] = pt_rows(p.k_spt, q0, lane, p.T, p.Hkv, g);
+      }
       reinterpret_cast<uint4*>(sfb(1))[lane] = pt_rows(p.do_spt, q0, lane, p.T, p.Hq, h);
-      reinterpret_cast<uint4*>(sfb(2))[lane] = pt_rows(p.k_spt, q0, lane, p.T, p.Hkv, g);
       reinterpret_cast<uint4*>(sfb(3))[lane] = pt_rows(p.v_spt, q0, lane, p.T, p.Hkv, g);
       fence_proxy_async_smem();
       if (lane == 0) {
-        mbar_arrive_expect_tx(q_full, 4 * kCode);
+        mbar_arrive_expect_tx(q_full, kNv ? kNvTile + 2 * kCode : 4 * kCode);
         tma_load_3d(smem + oQ, &tm_qpt, q_full, 0, h, q0);
         tma_load_3d(smem + oDO, &tm_dopt, q_full, 0, h, q0);
-        tma_load_3d(smem + oKpt, &tm_kpt, q_full, 0, g, q0);  // the diagonal key tile starts at q0
+        if (!kNv) tma_load_3d(smem + oKpt, &tm_kpt, q_full, 0, g, q0);  // the diagonal key tile starts at q0
         tma_load_3d(smem + oVpt, &tm_vpt, q_full, 0, g, q0);
       } else {
         mbar_arrive(q_full);
@@ -277,19 +301,33 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         const int stg = st_it % kStages;
         const uint32_t use = st_it / kStages;
         // scale words first, so that their global reads overlap the wait
-        const uint4 wk = tb_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
+        uint4 wk, wk2;
+        if constexpr (kNv) {
+          // the NVFP4 scale words of the tile's keys (scores)
+          const int k0 = s + 128 * v;
+          const uint2 w0 = nv_scale_words(p.k_nvs, k0 + lane, p.T, p.Hkv, g);
+          const uint2 w1 = nv_scale_words(p.k_nvs, k0 + lane + 32, p.T, p.Hkv, g);
+          const uint2 w2 = nv_scale_words(p.k_nvs, k0 + lane + 64, p.T, p.Hkv, g);
+          const uint2 w3 = nv_scale_words(p.k_nvs, k0 + lane + 96, p.T, p.Hkv, g);
+          wk = make_uint4(w0.x, w1.x, w2.x, w3.x);
+          wk2 = make_uint4(w0.y, w1.y, w2.y, w3.y);
+        } else {
+          wk = tb_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
+        }
         const uint4 wv = tb_rows(p.v_stb, s, e, doc, 4 * v, p.Hkv, g);
         const uint4 wkc = tb_channel_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
         if (use > 0 && !warp_wait(st_empty + stg, (use - 1) & 1, wd, 72)) { ok = false; break; }
         reinterpret_cast<uint4*>(sfb(5 + 3 * stg))[lane] = wk;
         reinterpret_cast<uint4*>(sfb(6 + 3 * stg))[lane] = wv;
         reinterpret_cast<uint4*>(sfb(7 + 3 * stg))[lane] = wkc;
+        if (kNv) reinterpret_cast<uint4*>(sfb(5 + 3 * kStages + stg))[lane] = wk2;
         fence_proxy_async_smem();
         if (lane == 0) {
           uint8_t* st = smem + oRing + stg * 2 * kCode;
-          mbar_arrive_expect_tx(st_full + stg, 2 * kCode);
+          mbar_arrive_expect_tx(st_full + stg, kNv ? 2 * kCode + kNvTile : 2 * kCode);
           tma_load_3d(st, &tm_ktb, st_full + stg, 0, g, s + 128 * v);
           tma_load_3d(st + kCode, &tm_vtb, st_full + stg, 0, g, s + 128 * v);
+          if (kNv) tma_load_3d(smem + oKpt + stg * kNvTile, &tm_knv, st_full + stg, 0, g, s + 128 * v);
         } else {
           mbar_arrive(st_full + stg);
         }
@@ -323,11 +361,20 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         // each score MMA goes into its region once the compute warps have read
         // out the previous use; the regions' reads of Q, dO, the per-token K and
         // V and the stage's V end here, K^tb is read by dQ too
+        // (mixed path: S from the NVFP4 Q and the stage's NVFP4 K, whose
+        // second scale blocks sit at tSfKpt and tSfK2)
         auto score = [&](bool dp, uint32_t a, uint32_t b, uint32_t sfa, uint32_t sfbc) {
           uint32_t& uses = dp ? dp_uses : s_uses;
           if (uses > 0 && !mbar_wait(dp ? dp_free : s_free, (uses - 1) & 1, wd, dp ? 74 : 73)) return false;
           tc_fence_after();
-          mx_kk(dp ? tDP : tS, a, b, sfa, sfbc, false, false);
+          if (kNv && !dp) {
+            const uint64_t da = sdesc_sw64(a), db = sdesc_sw64(b);
+            constexpr uint32_t idn = idesc_nvf4(128, 128);
+            mma_nvf4_ss(tmem + tS, da, db, idn, tmem + sfa, tmem + sfbc, 0u);
+            mma_nvf4_ss(tmem + tS, da + 2, db + 2, idn, tmem + tSfKpt, tmem + tSfK2, 1u);
+          } else {
+            mx_kk(dp ? tDP : tS, a, b, sfa, sfbc, false, false);
+          }
           tc_commit(dp ? dp_full : s_full);
           ++uses;
           return true;
@@ -350,13 +397,17 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
             if (!mbar_wait(st_full + stg, (kt / kStages) & 1, wd, 75)) { ok = false; break; }
             const uint32_t ak = aRing + stg * 2 * kCode, av = ak + kCode;
             tmem_cp_sf(tmem + tSfK, aSf + (5 + 3 * stg) * kSfBlk);
-            if (!score(false, aQ, ak, tSfQ, tSfK)) { ok = false; break; }
+            if (kNv) tmem_cp_sf(tmem + tSfK2, aSf + (5 + 3 * kStages + stg) * kSfBlk);
+            if (!score(false, aQ, kNv ? aKpt + stg * kNvTile : ak, tSfQ, tSfK)) { ok = false; break; }
             tmem_cp_sf(tmem + tSfV, aSf + (6 + 3 * stg) * kSfBlk);
             if (!score(true, aDO, av, tSfDO, tSfV)) { ok = false; break; }
           }
           if (!ok) break;
-          // the diagonal tile again with the per-token K and V
-          if (!score(false, aQ, aKpt, tSfQ, tSfKpt) || !score(true, aDO, aVpt, tSfDO, tSfVpt)) break;
+          // the diagonal tile again with the per-token K and V (mixed path:
+          // the same NVFP4 scores again, from the last stage, which stays
+          // loaded until the dQ MMAs of this tile release it)
+          const uint32_t s2 = kNv ? aKpt + ((kt - 1) % kStages) * kNvTile : aKpt;
+          if (!score(false, aQ, s2, tSfQ, kNv ? tSfK : tSfKpt) || !score(true, aDO, aVpt, tSfDO, tSfVpt)) break;
         }
       } else {
         // ---------------------------------------------- dQ
@@ -438,12 +489,28 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         // 32 wg .. 32 wg + 31.  The previous item's dQ MMAs have completed
         // (q_full of this item follows the loader's wait on q_empty).
         if (!warp_wait(q_full, unit_i & 1, wd, 104)) break;
-        const uint8_t* krow = smem + oKpt + row * 128;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(krow + (((2 * wg) ^ (row & 7)) << 4));
-        const uint4 c1 = *reinterpret_cast<const uint4*>(krow + (((2 * wg + 1) ^ (row & 7)) << 4));
+        uint4 c0, c1;
+        uint32_t ksb;
+        if constexpr (kNv) {
+          // (mixed path: from global memory; the shared tile holds NVFP4 K)
+          const int t = q0 + row;
+          c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
+          ksb = 127u;
+          if (t < p.T) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.k_vpt + ((size_t)t * p.Hkv + g) * 128 + 32 * wg);
+            c0 = __ldg(src);
+            c1 = __ldg(src + 1);
+            ksb = __ldg(p.k_spt + ((size_t)t * p.Hkv + g) * 4 + wg);
+          }
+        } else {
+          const uint8_t* krow = smem + oKpt + row * 128;
+          c0 = *reinterpret_cast<const uint4*>(krow + (((2 * wg) ^ (row & 7)) << 4));
+          c1 = *reinterpret_cast<const uint4*>(krow + (((2 * wg + 1) ^ (row & 7)) << 4));
+          ksb = sfb(2)[16 * lane + 4 * quarter + wg];
+        }
         const uint32_t codes[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         uint32_t kd[16];
-        dequant32_bf16(codes, sfb(2)[16 * lane + 4 * quarter + wg], kd);
+        dequant32_bf16(codes, ksb, kd);
         store_bf16_32(smem + oKd, row, wg, kd);
         fence_proxy_async_smem();
         tc_fence_before();
@@ -542,8 +609,11 @@ constexpr int oQpt = oVpt + kCode, oDOpt = oQpt + kCode, oDOtb = oDOpt + kCode, 
 constexpr int oP = oQtb + kCode, oDS = oP + kCode;
 constexpr int oAux = oDS + kCode;
 constexpr int oSf = oAux + 2 * 1024;
-// scale blocks: 0 Ktb, 1 Kpt, 2 Vtb, 3 Vpt, 4 Qpt, 5 dOpt, 6 dOtb (channel rows), 7 Qtb (channel rows), 8 P, 9 dS
-constexpr int kNumSf = 10;
+// scale blocks: 0 Ktb, 1 Kpt, 2 Vtb, 3 Vpt, 4 Qpt, 5 dOpt, 6 dOtb (channel rows), 7 Qtb (channel rows), 8 P, 9 dS,
+// 10 (mixed path) Q's second NVFP4 block.  Mixed path: the NVFP4 K tile at oKtb with its two
+// blocks in 0 and 1 (the per-token K is not loaded), the NVFP4 Q tile at oQpt
+constexpr int kNumSf = 11;
+constexpr int kNvTile = 128 * 64;
 constexpr int oBars = oSf + kNumSf * kSfBlk;
 // operand buffers, in the order the MMAs release them
 constexpr int kQpt = 0, kDOpt = 1, kDOtb = 2, kQtb = 3;
@@ -556,9 +626,11 @@ static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may u
 // into registers and released before the next), dV, dK, scale factors
 constexpr uint32_t tSD = 0, tDV = 128, tDK = 256;
 constexpr uint32_t tSfKtb = 384, tSfKpt = 388, tSfVtb = 392, tSfVpt = 396, tSfQpt = 400, tSfDOpt = 404, tSfP = 408,
-                   tSfDS = 412, tSfDOtb = 416, tSfQtb = 420;
+                   tSfDS = 412, tSfDOtb = 416, tSfQtb = 420, tSfQ2 = 424;
 }  // namespace kvk
 
+// kNv: tm_ktb and tm_kpt map K's NVFP4 codes (only tm_ktb is read), tm_qpt Q's
+template <bool kNv>
 __global__ void __launch_bounds__(kvk::kThreads, 1)
     dkdv_mx_kernel(const __grid_constant__ CUtensorMap tm_ktb, const __grid_constant__ CUtensorMap tm_kpt,
                    const __grid_constant__ CUtensorMap tm_vtb, const __grid_constant__ CUtensorMap tm_vpt,
@@ -643,13 +715,16 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   };
   // one operand buffer of query tile t: wait until the MMAs of tile t - 1 released
   // it, store its scale block, then copy the codes
-  auto load_op = [&](int op, uint32_t t, const CUtensorMap* tm, int h, int q0, const uint4& sfw, int where) {
+  // (mixed path, Q^pt buffer: Q's NVFP4 tile, its second scale block sfw2 in block 10)
+  auto load_op = [&](int op, uint32_t t, const CUtensorMap* tm, int h, int q0, const uint4& sfw, int where,
+                     const uint4* sfw2 = nullptr) {
     if (t > 0 && !warp_wait(op_empty + op, (t - 1) & 1, wd, where)) return false;
     reinterpret_cast<uint4*>(sfb(4 + op))[lane] = sfw;
+    if (sfw2) reinterpret_cast<uint4*>(sfb(10))[lane] = *sfw2;
     fence_proxy_async_smem();
     const int off = op == kQpt ? oQpt : op == kDOpt ? oDOpt : op == kDOtb ? oDOtb : oQtb;
     if (lane == 0) {
-      mbar_arrive_expect_tx(op_full + op, kCode);
+      mbar_arrive_expect_tx(op_full + op, (kNv && op == kQpt) ? kNvTile : kCode);
       tma_load_3d(smem + off, tm, op_full + op, 0, h, q0);
     } else {
       mbar_arrive(op_full + op);
@@ -669,15 +744,24 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
       int doc, s, e, g, v, k0, nq;
       decode(un, doc, s, e, g, v, k0, nq);
       if (unit_i > 0 && !warp_wait(kv_empty, (unit_i - 1) & 1, wd, 81)) break;
-      reinterpret_cast<uint4*>(sfb(0))[lane] = tb_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
-      reinterpret_cast<uint4*>(sfb(1))[lane] = pt_rows(p.k_spt, k0, lane, p.T, p.Hkv, g);
+      if constexpr (kNv) {
+        const uint2 w0 = nv_scale_words(p.k_nvs, k0 + lane, p.T, p.Hkv, g);
+        const uint2 w1 = nv_scale_words(p.k_nvs, k0 + lane + 32, p.T, p.Hkv, g);
+        const uint2 w2 = nv_scale_words(p.k_nvs, k0 + lane + 64, p.T, p.Hkv, g);
+        const uint2 w3 = nv_scale_words(p.k_nvs, k0 + lane + 96, p.T, p.Hkv, g);
+        reinterpret_cast<uint4*>(sfb(0))[lane] = make_uint4(w0.x, w1.x, w2.x, w3.x);
+        reinterpret_cast<uint4*>(sfb(1))[lane] = make_uint4(w0.y, w1.y, w2.y, w3.y);
+      } else {
+        reinterpret_cast<uint4*>(sfb(0))[lane] = tb_rows(p.k_stb, s, e, doc, 4 * v, p.Hkv, g);
+        reinterpret_cast<uint4*>(sfb(1))[lane] = pt_rows(p.k_spt, k0, lane, p.T, p.Hkv, g);
+      }
       reinterpret_cast<uint4*>(sfb(2))[lane] = tb_rows(p.v_stb, s, e, doc, 4 * v, p.Hkv, g);
       reinterpret_cast<uint4*>(sfb(3))[lane] = pt_rows(p.v_spt, k0, lane, p.T, p.Hkv, g);
       fence_proxy_async_smem();
       if (lane == 0) {
-        mbar_arrive_expect_tx(kv_full, 4 * kCode);
+        mbar_arrive_expect_tx(kv_full, kNv ? kNvTile + 2 * kCode : 4 * kCode);
         tma_load_3d(smem + oKtb, &tm_ktb, kv_full, 0, g, k0);
-        tma_load_3d(smem + oKpt, &tm_kpt, kv_full, 0, g, k0);
+        if (!kNv) tma_load_3d(smem + oKpt, &tm_kpt, kv_full, 0, g, k0);
         tma_load_3d(smem + oVtb, &tm_vtb, kv_full, 0, g, k0);
         tma_load_3d(smem + oVpt, &tm_vpt, kv_full, 0, g, k0);
       } else {
@@ -687,7 +771,17 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
         for (int m = v; m < nq; ++m, ++t) {
           const int q0 = s + 128 * m;
           // all global reads of the tile first, so that their latencies overlap
-          const uint4 sq = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
+          uint4 sq, sq2;
+          if constexpr (kNv) {
+            const uint2 w0 = nv_scale_words(p.q_nvs, q0 + lane, p.T, p.Hq, h);
+            const uint2 w1 = nv_scale_words(p.q_nvs, q0 + lane + 32, p.T, p.Hq, h);
+            const uint2 w2 = nv_scale_words(p.q_nvs, q0 + lane + 64, p.T, p.Hq, h);
+            const uint2 w3 = nv_scale_words(p.q_nvs, q0 + lane + 96, p.T, p.Hq, h);
+            sq = make_uint4(w0.x, w1.x, w2.x, w3.x);
+            sq2 = make_uint4(w0.y, w1.y, w2.y, w3.y);
+          } else {
+            sq = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
+          }
           const uint4 sdo = pt_rows(p.do_spt, q0, lane, p.T, p.Hq, h);
           float l4[4], d4[4];
 #pragma unroll
@@ -703,7 +797,7 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           reinterpret_cast<float4*>(lse2)[lane] = make_float4(l4[0], l4[1], l4[2], l4[3]);
           reinterpret_cast<float4*>(lse2 + 128)[lane] = make_float4(d4[0], d4[1], d4[2], d4[3]);
           mbar_arrive(aux_full + ab);
-          if (!load_op(kQpt, t, &tm_qpt, h, q0, sq, 83)) { ok = false; break; }
+          if (!load_op(kQpt, t, &tm_qpt, h, q0, sq, 83, kNv ? &sq2 : nullptr)) { ok = false; break; }
           if (!load_op(kDOpt, t, &tm_dopt, h, q0, sdo, 84)) { ok = false; break; }
         }
       }
@@ -773,12 +867,23 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
         tc_fence_after();
         return true;
       };
+      // mixed path: S^T from the NVFP4 K (scale blocks at tSfKtb, tSfKpt) and Q (tSfQpt, tSfQ2)
+      auto nv_st = [&]() {
+        const uint64_t da = sdesc_sw64(aKtb), db = sdesc_sw64(aQpt);
+        constexpr uint32_t idn = idesc_nvf4(128, 128);
+        mma_nvf4_ss(tmem + tSD, da, db, idn, tmem + tSfKtb, tmem + tSfQpt, 0u);
+        mma_nvf4_ss(tmem + tSD, da + 2, db + 2, idn, tmem + tSfKpt, tmem + tSfQ2, 1u);
+      };
       // S^T of tile tt with token-block K (every key block of the tile)
       auto s_tb = [&](uint32_t tt) {
         if (!wait_op(kQpt, tt, 88)) return false;
         tmem_cp_sf(tmem + tSfQpt, aSf + 4 * kSfBlk);
+        if (kNv) tmem_cp_sf(tmem + tSfQ2, aSf + 10 * kSfBlk);
         if (!region()) return false;
-        mx_kk(tSD, aKtb, aQpt, tSfKtb, tSfQpt, false, false);
+        if (kNv)
+          nv_st();
+        else
+          mx_kk(tSD, aKtb, aQpt, tSfKtb, tSfQpt, false, false);
         region_done();
         return true;
       };
@@ -804,8 +909,12 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           if (diag) {
             // diagonal tile: S^T again with the per-token K; the compute warps
             // take its diagonal 32x32 blocks
+            // (mixed path: the same NVFP4 product again)
             if (!region()) { ok = false; break; }
-            mx_kk(tSD, aKpt, aQpt, tSfKpt, tSfQpt, false, false);
+            if (kNv)
+              nv_st();
+            else
+              mx_kk(tSD, aKpt, aQpt, tSfKpt, tSfQpt, false, false);
             region_done();
           }
           tc_commit(op_empty + kQpt);
@@ -1014,12 +1123,21 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     cudaError_t e = launch_quantize_with_delta(job, a.T, a.d, a.cu, a.n_docs, a.rule, da, stream);
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap tqpt, tqtb, tktb, tkpt, tvtb, tvpt, tdopt, tdotb;
-  if (!make_tmap_codes(&tqpt, a.q_vpt, a.T, a.Hq) || !make_tmap_codes(&tqtb, a.q_vtb, a.T, a.Hq) ||
-      !make_tmap_codes(&tktb, a.k_vtb, a.T, a.Hkv) || !make_tmap_codes(&tkpt, a.k_vpt, a.T, a.Hkv) ||
-      !make_tmap_codes(&tvtb, a.v_vtb, a.T, a.Hkv) || !make_tmap_codes(&tvpt, a.v_vpt, a.T, a.Hkv) ||
-      !make_tmap_codes(&tdopt, a.do_vpt, a.T, a.Hq) || !make_tmap_codes(&tdotb, a.do_vtb, a.T, a.Hq))
+  CUtensorMap tqpt, tqtb, tktb, tkpt, tvtb, tvpt, tdopt, tdotb, tqnv, tknv;
+  if (!make_tmap_codes(&tqtb, a.q_vtb, a.T, a.Hq) || !make_tmap_codes(&tktb, a.k_vtb, a.T, a.Hkv) ||
+      !make_tmap_codes(&tkpt, a.k_vpt, a.T, a.Hkv) || !make_tmap_codes(&tvtb, a.v_vtb, a.T, a.Hkv) ||
+      !make_tmap_codes(&tvpt, a.v_vpt, a.T, a.Hkv) || !make_tmap_codes(&tdopt, a.do_vpt, a.T, a.Hq) ||
+      !make_tmap_codes(&tdotb, a.do_vtb, a.T, a.Hq))
     return cudaErrorInvalidValue;
+  if (a.nv) {
+    // the scores' operands: NVFP4 Q and K (Q's per-token MXFP8 form is not kept)
+    if (!make_tmap_nv(&tqnv, a.q_nvv, a.T, a.Hq) || !make_tmap_nv(&tknv, a.k_nvv, a.T, a.Hkv))
+      return cudaErrorInvalidValue;
+    tqpt = tqnv;
+  } else {
+    if (!make_tmap_codes(&tqpt, a.q_vpt, a.T, a.Hq)) return cudaErrorInvalidValue;
+    tknv = tkpt;  // not read
+  }
   MxParams p;
   p.cu = a.cu;
   p.lse = a.lse;
@@ -1028,6 +1146,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
   p.k_stb = a.k_stb; p.k_spt = a.k_spt;
   p.v_stb = a.v_stb; p.v_spt = a.v_spt;
   p.do_stb = a.do_stb; p.do_spt = a.do_spt;
+  p.q_nvs = a.q_nvs; p.k_nvs = a.k_nvs; p.k_vpt = a.k_vpt;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
   p.T = a.T;
@@ -1035,13 +1154,15 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
   p.Hkv = a.Hkv;
   p.d = a.d;
   p.scale = a.scale;
-  p.scale_log2 = a.scale * kLog2e;
+  // mixed path: the scores' MMAs leave out the decode scales of Q and K
+  p.scale_log2 = a.scale * kLog2e * (a.nv ? a.nv_g_q * a.nv_g_k : 1.f);
   p.grad_bf16 = a.grad_bf16;
   p.rule = a.rule;
   // 2. dK, dV
   a.marks.at(3, stream);
   {
-    cudaError_t e = cudaFuncSetAttribute(dkdv_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvk::kSmem);
+    const auto kern = a.nv ? dkdv_mx_kernel<true> : dkdv_mx_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kvk::kSmem);
     if (e != cudaSuccess) return e;
     MxParams pk = p;
     pk.sched = sched_view(a.sched_kv);
@@ -1051,7 +1172,10 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     pk.wide = aligned32(a.dk) && aligned32(a.dv);
     const long long max_units = (long long)a.sched_kv.max_items * a.Hkv;
     const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
-    dkdv_mx_kernel<<<grid, kvk::kThreads, kvk::kSmem, stream>>>(tktb, tkpt, tvtb, tvpt, tqpt, tqtb, tdopt, tdotb, pk);
+    if (a.nv)
+      kern<<<grid, kvk::kThreads, kvk::kSmem, stream>>>(tknv, tknv, tvtb, tvpt, tqpt, tqtb, tdopt, tdotb, pk);
+    else
+      kern<<<grid, kvk::kThreads, kvk::kSmem, stream>>>(tktb, tkpt, tvtb, tvpt, tqpt, tqtb, tdopt, tdotb, pk);
     note_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -1059,7 +1183,8 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
   // 3. dQ
   a.marks.at(4, stream);
   {
-    cudaError_t e = cudaFuncSetAttribute(dq_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::kSmem);
+    const auto kern = a.nv ? dq_mx_kernel<true> : dq_mx_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::kSmem);
     if (e != cudaSuccess) return e;
     MxParams pq = p;
     pq.sched = sched_view(a.sched_q);
@@ -1069,7 +1194,7 @@ cudaError_t launch_bwd_mxfp8(const BwdMxArgs& a, cudaStream_t stream) {
     pq.out1 = nullptr;
     const long long max_units = (long long)a.sched_q.max_items * a.Hq;
     const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
-    dq_mx_kernel<<<grid, dqk::kThreads, dqk::kSmem, stream>>>(tqpt, tdopt, tktb, tvtb, tkpt, tvpt, pq);
+    kern<<<grid, dqk::kThreads, dqk::kSmem, stream>>>(tqpt, tdopt, tktb, tvtb, tkpt, tvpt, tknv, pq);
     note_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -39,10 +39,19 @@
 //    block scale cannot express).
 // TMEM: S buffers [0,128) and [128,256) (the diagonal tile's per-token S uses
 // the buffer the previous tile freed), O [256,384), scale factors from 384.
+//
+// Mixed NVFP4/FP8 path (kNv): the scores take Q and K in NVFP4 (E2M1 codes,
+// one E4M3 scale per 16 channels of one token, kind::mxf4nvf4 MMAs, two per
+// tile with K = 64); Q is quantised on load to NVFP4 (its token-block MXFP8
+// form and its NVFP4 form go to ctx for the backward), K's NVFP4 tiles come
+// from the prepass.  NVFP4 blocks lie inside one token, so the diagonal
+// tile's second S (the "per-token" one) is the same product on the diagonal
+// key tile and the softmax warps run unchanged; P~ V is the MXFP8 path's.
 #include <cuda_bf16.h>
 
 #include "internal.h"
 #include "mx.cuh"
+#include "nv.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
 
@@ -70,7 +79,9 @@ constexpr int oPd = oP + kCodeTile;
 constexpr int oRing = oPd + kBf16Tile;
 constexpr int oSf = oRing + kSlots * kCodeTile;  // sfQ, sfKpt, sfP, sfRing[kSlots]
 constexpr int kSfBlk = 512;
-constexpr int oXmax = oSf + (3 + kSlots) * kSfBlk;  // block maxima [2][4][128] (by tile parity)
+// mixed path: the second scale block (channels 64..127) of sfQ, sfKpt, sfRing[kSlots]
+constexpr int oSf2 = oSf + (3 + kSlots) * kSfBlk;
+constexpr int oXmax = oSf2 + (2 + kSlots) * kSfBlk;  // block maxima [2][4][128] (by tile parity)
 constexpr int oLsum = oXmax + 2 * 4 * 128 * 4;       // partial row sums [4][128]
 constexpr int oBars = oLsum + 4 * 128 * 4;
 // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full, pv_done, o_full, o_free, fin,
@@ -82,6 +93,8 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory exceeds the 227 KB a CTA 
 // TMEM columns
 constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256;
 constexpr uint32_t kSfQ = 384, kSfK = 388, kSfKpt = 392, kSfP = 396, kSfV = 400;
+constexpr uint32_t kSfQ2 = 404, kSfK2 = 408, kSfKpt2 = 412;  // mixed path: channels 64..127
+constexpr int kNvTile = 128 * 64;  // 128 rows x 128 E2M1 codes
 
 struct Params {
   const int32_t* cu;
@@ -97,6 +110,11 @@ struct Params {
   const uint8_t* k_stb;   // K token-block scales [slots][Hkv][4]
   const uint8_t* k_spt;   // K per-token scales [T][Hkv][4]
   const uint8_t* v_stb;   // V token-block scales [slots][Hkv][4]
+  // mixed path
+  const uint8_t* k_nvs;   // K NVFP4 scales [T][Hkv][8]
+  uint8_t* q_nvv;         // out: Q NVFP4 codes [T][Hq][64] (ctx); null: no saved state
+  uint8_t* q_nvs;         // out: Q NVFP4 scales [T][Hq][8]
+  float nv_g_q, nv_six_g_q;  // Q's decode scale g and fp32(6 g)
   __nv_bfloat16* o;
   float* lse;
   __nv_bfloat16* o_resid;
@@ -146,6 +164,7 @@ __device__ __forceinline__ void prefetch_item(const Params& p, const Item& it, i
   asm volatile("prefetch.global.L2 [%0];" ::"l"(v));
 }
 
+template <bool kNv>
 __device__ __forceinline__ void stage_q(const Params& p, const Item& it, int row, int wg, uint8_t* sQ,
                                         uint8_t* sfQ) {
   const int t = it.q0 + row;
@@ -162,26 +181,44 @@ __device__ __forceinline__ void stage_q(const Params& p, const Item& it, int row
 #pragma unroll
     for (int c = 0; c < 32; ++c) f[c] = 0.f;
   }
-  // per-token form
   float a = 0.f;
 #pragma unroll
   for (int c = 0; c < 32; ++c) a = fmaxf(a, fabsf(f[c]));
-  const int X = mx_block_exponent(a, p.rule);
   uint2 cw[4];
+  if constexpr (kNv) {
+    // NVFP4 for the scores: channels 32 wg .. 32 wg + 31 are two 16-channel
+    // blocks, 16 bytes of codes = chunk wg of the 64-byte row; their scale
+    // bytes 2 wg, 2 wg + 1 go to the word of MMA k-step wg >> 1
+    uint32_t c0[2], c1[2];
+    const uint32_t s0 = nv_quant16(&f[0], p.nv_six_g_q, p.nv_g_q, c0);
+    const uint32_t s1 = nv_quant16(&f[16], p.nv_six_g_q, p.nv_g_q, c1);
+    const uint4 codes = make_uint4(c0[0], c0[1], c1[0], c1[1]);
+    *reinterpret_cast<uint4*>(sQ + sw64_chunk(row, wg)) = codes;
+    const uint16_t sw = (uint16_t)(s0 | (s1 << 8));
+    *reinterpret_cast<uint16_t*>(sfQ + (wg >> 1) * (oSf2 - oSf) + (row & 31) * 16 + (row >> 5) * 4 + 2 * (wg & 1)) = sw;
+    if (!p.q_nvv) return;  // inference: Q's forms are not kept
+    if (in_doc) {
+      *reinterpret_cast<uint4*>(p.q_nvv + ((size_t)t * p.Hq + it.h) * 64 + 16 * wg) = codes;
+      *reinterpret_cast<uint16_t*>(p.q_nvs + ((size_t)t * p.Hq + it.h) * 8 + 2 * wg) = sw;
+    }
+  } else {
+    // per-token form
+    const int X = mx_block_exponent(a, p.rule);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) cw[c] = encode8(*reinterpret_cast<const float(*)[8]>(&f[8 * c]), X);
-  uint8_t* prow = sQ + row * 128;
-  *reinterpret_cast<uint4*>(prow + (((2 * wg) ^ (row & 7)) << 4)) = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
-  *reinterpret_cast<uint4*>(prow + (((2 * wg + 1) ^ (row & 7)) << 4)) = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
-  sfQ[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)(X + 127);
-  if (!p.q_vpt) return;  // inference: Q's forms are not kept
-  const size_t qo = ((size_t)t * p.Hq + it.h) * 128 + 32 * wg;
-  if (in_doc) {
-    uint4* dst = reinterpret_cast<uint4*>(p.q_vpt + qo);
-    dst[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
-    dst[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
-    p.q_spt[((size_t)t * p.Hq + it.h) * 4 + wg] = (uint8_t)(X + 127);
+    for (int c = 0; c < 4; ++c) cw[c] = encode8(*reinterpret_cast<const float(*)[8]>(&f[8 * c]), X);
+    uint8_t* prow = sQ + row * 128;
+    *reinterpret_cast<uint4*>(prow + (((2 * wg) ^ (row & 7)) << 4)) = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+    *reinterpret_cast<uint4*>(prow + (((2 * wg + 1) ^ (row & 7)) << 4)) = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+    sfQ[(row & 31) * 16 + (row >> 5) * 4 + wg] = (uint8_t)(X + 127);
+    if (!p.q_vpt) return;  // inference: Q's forms are not kept
+    if (in_doc) {
+      uint4* dst = reinterpret_cast<uint4*>(p.q_vpt + ((size_t)t * p.Hq + it.h) * 128 + 32 * wg);
+      dst[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+      dst[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+      p.q_spt[((size_t)t * p.Hq + it.h) * 4 + wg] = (uint8_t)(X + 127);
+    }
   }
+  const size_t qo = ((size_t)t * p.Hq + it.h) * 128 + 32 * wg;
   // token-block form: the warp's 32 rows, this channel group
   float atb = a;
 #pragma unroll
@@ -225,6 +262,9 @@ __device__ __forceinline__ void stage_v(const Params& p, const Item& it, int row
   *reinterpret_cast<uint4*>(vrow + (((c0 + 3) ^ (row & 7)) << 4)) = d3;
 }
 
+// tm_ktb, tm_kpt: K's token-block and per-token MXFP8 codes, or (kNv) both
+// K's NVFP4 codes
+template <bool kNv>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_mxfp8_kernel(const __grid_constant__ CUtensorMap tm_ktb, const __grid_constant__ CUtensorMap tm_kpt,
                      const __grid_constant__ CUtensorMap tm_vtb, const Params p) {
@@ -240,6 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sfKpt = sfQ + kSfBlk;
   uint8_t* sfP = sfQ + 2 * kSfBlk;
   uint8_t* sfRing = sfQ + 3 * kSfBlk;
+  uint8_t* sfKpt2 = smem + oSf2 + kSfBlk;   // mixed path: second scale blocks
+  uint8_t* sfRing2 = smem + oSf2 + 2 * kSfBlk;
+  constexpr uint32_t kKBytes = kNv ? kNvTile : kCodeTile;  // bytes of one K tile
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oBars);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
@@ -315,7 +358,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t use = kv_it / kSlots;
           if (use > 0 && !warp_wait(kv_empty + slot, (use - 1) & 1, wd, 52)) { ok = false; break; }
           uint4 wsf;
-          if (kv == 0) {
+          if (kNv && kv == 0) {
+            // K rows = keys: the NVFP4 scale words (channels 0..63, 64..127) of each key
+            const int k0 = it.s + 128 * j;
+            const uint2 w0 = nv_scale_words(p.k_nvs, k0 + lane, p.T, p.Hkv, it.g);
+            const uint2 w1 = nv_scale_words(p.k_nvs, k0 + lane + 32, p.T, p.Hkv, it.g);
+            const uint2 w2 = nv_scale_words(p.k_nvs, k0 + lane + 64, p.T, p.Hkv, it.g);
+            const uint2 w3 = nv_scale_words(p.k_nvs, k0 + lane + 96, p.T, p.Hkv, it.g);
+            wsf = make_uint4(w0.x, w1.x, w2.x, w3.x);
+            reinterpret_cast<uint4*>(sfRing2 + slot * kSfBlk)[lane] = make_uint4(w0.y, w1.y, w2.y, w3.y);
+          } else if (kv == 0) {
             // K rows = keys: the scale word of the key's token block
             wsf.x = tb_word(p.k_stb, it.s, it.e, it.doc, 4 * j + 0, p.Hkv, it.g);
             wsf.y = tb_word(p.k_stb, it.s, it.e, it.doc, 4 * j + 1, p.Hkv, it.g);
@@ -337,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           reinterpret_cast<uint4*>(sfRing + slot * kSfBlk)[lane] = wsf;
           fence_proxy_async_smem();
           if (lane == 0) {
-            mbar_arrive_expect_tx(kv_full + slot, kCodeTile);
+            mbar_arrive_expect_tx(kv_full + slot, kv ? kCodeTile : kKBytes);
             tma_load_3d(sRing + slot * kCodeTile, kv ? &tm_vtb : &tm_ktb, kv_full + slot, 0, it.g, it.s + 128 * j);
           } else {
             mbar_arrive(kv_full + slot);
@@ -351,14 +403,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           // tiles never wait for the previous item to finish
           if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 51)) { ok = false; break; }
           uint4 wk;
-          wk.x = pt_word(p.k_spt, it.q0 + lane, p.T, p.Hkv, it.g);
-          wk.y = pt_word(p.k_spt, it.q0 + lane + 32, p.T, p.Hkv, it.g);
-          wk.z = pt_word(p.k_spt, it.q0 + lane + 64, p.T, p.Hkv, it.g);
-          wk.w = pt_word(p.k_spt, it.q0 + lane + 96, p.T, p.Hkv, it.g);
+          if constexpr (kNv) {
+            // the diagonal key tile's NVFP4 codes and scales (the same scores
+            // as the ring's copy of that tile)
+            const uint2 w0 = nv_scale_words(p.k_nvs, it.q0 + lane, p.T, p.Hkv, it.g);
+            const uint2 w1 = nv_scale_words(p.k_nvs, it.q0 + lane + 32, p.T, p.Hkv, it.g);
+            const uint2 w2 = nv_scale_words(p.k_nvs, it.q0 + lane + 64, p.T, p.Hkv, it.g);
+            const uint2 w3 = nv_scale_words(p.k_nvs, it.q0 + lane + 96, p.T, p.Hkv, it.g);
+            wk = make_uint4(w0.x, w1.x, w2.x, w3.x);
+            reinterpret_cast<uint4*>(sfKpt2)[lane] = make_uint4(w0.y, w1.y, w2.y, w3.y);
+          } else {
+            wk.x = pt_word(p.k_spt, it.q0 + lane, p.T, p.Hkv, it.g);
+            wk.y = pt_word(p.k_spt, it.q0 + lane + 32, p.T, p.Hkv, it.g);
+            wk.z = pt_word(p.k_spt, it.q0 + lane + 64, p.T, p.Hkv, it.g);
+            wk.w = pt_word(p.k_spt, it.q0 + lane + 96, p.T, p.Hkv, it.g);
+          }
           reinterpret_cast<uint4*>(sfKpt)[lane] = wk;
           fence_proxy_async_smem();
           if (lane == 0) {
-            mbar_arrive_expect_tx(kpt_full, kCodeTile);
+            mbar_arrive_expect_tx(kpt_full, kKBytes);
             tma_load_3d(sKpt, &tm_kpt, kpt_full, 0, it.g, it.q0);  // the diagonal key tile starts at q0
           } else {
             mbar_arrive(kpt_full);
@@ -390,17 +453,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       // descriptors built once per operand tile and advanced by constant
       // offsets (start address >> 4 in the low field)
       const uint64_t dq = sdesc_sw128(aq, 16, 1024), dp = sdesc_sw128(ap, 16, 1024);
-      auto issue_s = [&](uint32_t col, uint32_t kaddr, uint32_t sfb) {
-        const uint64_t dk = sdesc_sw128(kaddr, 16, 1024);
+      // (mixed path: two NVFP4 MMAs of K = 64, scale words of channels
+      // 0..63 at sfb and 64..127 at sfb2; both tiles 64-byte swizzled)
+      auto issue_s = [&](uint32_t col, uint32_t kaddr, uint32_t sfb, uint32_t sfb2) {
+        if constexpr (kNv) {
+          const uint64_t dqn = sdesc_sw64(aq), dkn = sdesc_sw64(kaddr);
+          constexpr uint32_t idn = idesc_nvf4(128, 128);
+          mma_nvf4_ss(tmem + col, dqn, dkn, idn, tmem + kSfQ, tmem + sfb, 0u);
+          mma_nvf4_ss(tmem + col, dqn + 2, dkn + 2, idn, tmem + kSfQ2, tmem + sfb2, 1u);  // +32 bytes
+        } else {
+          const uint64_t dk = sdesc_sw128(kaddr, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_mxf8_ss(tmem + col, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_mxf8(128, 128, false, kk, kk),
-                      (tmem + kSfQ) | ((uint32_t)kk << 30), (tmem + sfb) | ((uint32_t)kk << 30), kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_mxf8_ss(tmem + col, dq + ((kk * 32) >> 4), dk + ((kk * 32) >> 4), idesc_mxf8(128, 128, false, kk, kk),
+                        (tmem + kSfQ) | ((uint32_t)kk << 30), (tmem + sfb) | ((uint32_t)kk << 30), kk > 0);
+        }
       };
       auto issue_s_tile = [&](int j, uint32_t col) {
         const int ks = kslot_of(j);
         tmem_cp_sf(tmem + kSfK, asf + (3 + ks) * kSfBlk);
-        issue_s(col, aring + ks * kCodeTile, kSfK);
+        if constexpr (kNv) tmem_cp_sf(tmem + kSfK2, smem_u32(sfRing2) + ks * kSfBlk);
+        issue_s(col, aring + ks * kCodeTile, kSfK, kSfK2);
       };
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
         const UnitInfo un = unit_take(ring, uk, wd);
@@ -411,11 +484,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(q_full, unit_i & 1, wd, 54)) break;
         tc_fence_after();
         tmem_cp_sf(tmem + kSfQ, asf);
+        if constexpr (kNv) tmem_cp_sf(tmem + kSfQ2, smem_u32(smem + oSf2));
         // the diagonal per-token K (and its scales) arrive on their own barrier
         auto wait_kpt = [&]() {
           if (!mbar_wait(kpt_full, unit_i & 1, wd, 61)) return false;
           tc_fence_after();
           tmem_cp_sf(tmem + kSfKpt, asf + kSfBlk);
+          if constexpr (kNv) tmem_cp_sf(tmem + kSfKpt2, smem_u32(sfKpt2));
           return true;
         };
         // prologue: S(0) (+ per-token S if tile 0 is the diagonal), S(1)
@@ -424,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s_tile(0, kS0);
         if (n == 1) {
           if (!wait_kpt()) break;
-          issue_s(kS1, akpt, kSfKpt);
+          issue_s(kS1, akpt, kSfKpt, kSfKpt2);
         }
         tc_commit(s_full + 0);
         tc_commit(kv_empty + kslot_of(0));
@@ -476,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j == n - 2) {
             // per-token S of the diagonal tile, into the buffer tile n-2 freed
             if (!wait_kpt()) { ok = false; break; }
-            issue_s((j & 1) ? kS1 : kS0, akpt, kSfKpt);
+            issue_s((j & 1) ? kS1 : kS0, akpt, kSfKpt, kSfKpt2);
             tc_commit(s_full + ((j + 1) & 1));  // signals tile n-1 = j+1
           }
         }
@@ -511,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     UnitInfo un = unit_take_warp(ring, uk++, wd);
     bool have = un.w >= 0 && un.w < n_units;
     if (have) {
-      stage_q(p, decode(p, un), row, wg, smem + oQ, smem + oSf);
+      stage_q<kNv>(p, decode(p, un), row, wg, smem + oQ, smem + oSf);
       fence_proxy_async_smem();
       tc_fence_before();
       warp_arrive(q_full);
@@ -660,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (have_next) {
         // every S MMA of this item has completed (its last scores were read
         // above), so sQ and sfQ may take the next item's Q
-        stage_q(p, decode(p, nx), row, wg, smem + oQ, smem + oSf);
+        stage_q<kNv>(p, decode(p, nx), row, wg, smem + oQ, smem + oSf);
         fence_proxy_async_smem();
         tc_fence_before();
         warp_arrive(q_full);
@@ -727,10 +802,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
   CUtensorMap tktb, tkpt, tvtb;
-  if (!make_tmap_codes(&tktb, a.k_vtb, a.T, a.Hkv) || !make_tmap_codes(&tkpt, a.k_vpt, a.T, a.Hkv) ||
-      !make_tmap_codes(&tvtb, a.v_vtb, a.T, a.Hkv))
+  if (a.nv) {
+    if (!make_tmap_nv(&tktb, a.k_nvv, a.T, a.Hkv) || !make_tmap_nv(&tkpt, a.k_nvv, a.T, a.Hkv))
+      return cudaErrorInvalidValue;
+  } else if (!make_tmap_codes(&tktb, a.k_vtb, a.T, a.Hkv) || !make_tmap_codes(&tkpt, a.k_vpt, a.T, a.Hkv)) {
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  }
+  if (!make_tmap_codes(&tvtb, a.v_vtb, a.T, a.Hkv)) return cudaErrorInvalidValue;
+  const auto kern = a.nv ? fwd_mxfp8_kernel<true> : fwd_mxfp8_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   Params p;
   p.cu = a.cu;
@@ -746,6 +826,11 @@ cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
   p.k_stb = a.k_stb;
   p.k_spt = a.k_spt;
   p.v_stb = a.v_stb;
+  p.k_nvs = a.k_nvs;
+  p.q_nvv = a.q_nvv;
+  p.q_nvs = a.q_nvs;
+  p.nv_g_q = a.nv_g_q;
+  p.nv_six_g_q = 6.0f * a.nv_g_q;
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.lse = a.lse;
   p.o_resid = static_cast<__nv_bfloat16*>(a.o_resid);
@@ -756,12 +841,13 @@ cudaError_t launch_fwd_mxfp8(const FwdMxArgs& a, cudaStream_t stream) {
   p.Hkv = a.Hkv;
   p.d = a.d;
   p.n_docs = a.n_docs;
-  p.scale_log2 = a.scale * 1.4426950408889634f;
+  // mixed path: the scores' MMAs leave out the decode scales of Q and K
+  p.scale_log2 = a.scale * 1.4426950408889634f * (a.nv ? a.nv_g_q * a.nv_g_k : 1.f);
   p.rule = a.rule;
   p.wide = aligned32(a.o) && aligned32(a.o_resid);
   const long long max_units = (long long)a.sched.max_items * a.Hq;
   const int grid = (int)(max_units < a.num_sms ? max_units : a.num_sms);
-  fwd_mxfp8_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tktb, tkpt, tvtb, p);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(tktb, tkpt, tvtb, p);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -77,6 +77,11 @@ struct QuantJob {
   uint8_t *vtb, *stb, *vpt, *spt;
   __nv_bfloat16* deq;  // per-token form dequantised to bf16, or null
   bool padded;
+  // NVFP4 form (d = 128 only), or null: codes [T][H][64], scales [T][H][8],
+  // decode scale g (six_g = fp32(6 g))
+  uint8_t* nvv = nullptr;
+  uint8_t* nvs = nullptr;
+  float nv_g = 1.f, nv_six_g = 6.f;
 };
 struct QuantJobs {
   QuantJob job[2];
@@ -92,6 +97,9 @@ struct DeltaArgs {
 // Up to two tensors of the same T and d in one launch (blockIdx.z = job).
 cudaError_t launch_quantize_jobs(const QuantJobs& jobs, int n_jobs, int T, int d, const int32_t* cu, int n_docs,
                                  int forms, int rule, cudaStream_t stream);
+// NVFP4 of a bf16 [T][H][128] tensor alone: codes [T][H][64], scales [T][H][8].
+cudaError_t launch_quantize_nvfp4(const void* x, int T, int H, float g, uint8_t* codes, uint8_t* scales,
+                                  cudaStream_t stream);
 // dO: both forms, and D in the same read.
 cudaError_t launch_quantize_with_delta(const QuantJob& job, int T, int d, const int32_t* cu, int n_docs, int rule,
                                        const DeltaArgs& da, cudaStream_t stream);
@@ -140,6 +148,14 @@ struct FwdMxArgs {
   const uint8_t* v_stb;      // V token-block scales
   const uint8_t* v_vpt;      // V per-token codes (diagonal tiles, dequantised on load)
   const uint8_t* v_spt;      // V per-token scales
+  // mixed NVFP4/FP8 path (nv): the scores from NVFP4 Q (quantised on load,
+  // written to q_nvv/q_nvs unless null) and K (k_nvv, k_nvs, from the prepass)
+  bool nv = false;
+  const uint8_t* k_nvv = nullptr;  // K NVFP4 codes [T][Hkv][64]
+  const uint8_t* k_nvs = nullptr;  // K NVFP4 scales [T][Hkv][8]
+  uint8_t* q_nvv = nullptr;        // out: Q NVFP4 codes [T][Hq][64]
+  uint8_t* q_nvs = nullptr;        // out: Q NVFP4 scales [T][Hq][8]
+  float nv_g_q = 1.f, nv_g_k = 1.f;  // decode scales
   void* o;
   float* lse;
   void* o_resid;
@@ -161,6 +177,10 @@ struct BwdMxArgs {
   const uint8_t *k_vtb, *k_stb, *k_vpt, *k_spt;     // quantised K (ctx)
   const uint8_t *v_vtb, *v_stb, *v_vpt, *v_spt;     // quantised V (ctx)
   const uint8_t *do_vtb, *do_stb, *do_vpt, *do_spt; // quantised dO (workspace; written by the D pass)
+  // mixed NVFP4/FP8 path (nv): the scores from the forward's NVFP4 Q and K (ctx)
+  bool nv = false;
+  const uint8_t *q_nvv = nullptr, *q_nvs = nullptr, *k_nvv = nullptr, *k_nvs = nullptr;
+  float nv_g_q = 1.f, nv_g_k = 1.f;
   const void* o;
   const void* o_resid;
   const float* lse;
@@ -204,6 +224,8 @@ cudaError_t launch_qkv_proj(const QkvProjArgs& a, cudaStream_t stream);
 
 // Tensor map of E4M3 codes [T][H][128] as (128, H, T), box 128 x 1 x 128,
 // 128-byte swizzle (api.cu).
+// NVFP4 codes [T][H][64 bytes]: boxes of 128 rows x 64 bytes, 64-byte swizzle.
+bool make_tmap_nv(CUtensorMap* map, const void* base, int T, int H);
 bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H);
 
 // Backward, bf16 operands (bwd_bf16.cu).

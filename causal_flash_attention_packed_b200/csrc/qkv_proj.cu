@@ -46,7 +46,7 @@ namespace fapk {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kLoadWarp = 0, kMmaWarp = 1, kEpiWarp0 = 2;
+constexpr int kLoadWarp = 0, kMmaWarp = 1;  // warps 2-5: epilogue
 constexpr int kStages = 4;
 constexpr int kBoxBytes = 128 * 64 * 2;     // 128 rows x 64 bf16
 constexpr int kStageBytes = 3 * kBoxBytes;  // X tile and two W boxes (256 rows)

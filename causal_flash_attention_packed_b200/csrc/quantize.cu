@@ -13,13 +13,15 @@
 // One launch can quantise two tensors of the same shape (K and V): blockIdx.z
 // picks the job.  The backward's variant also reads O and its bf16 residual in
 // the same pass and writes D_i = dO_i . (O_i + residual_i), so that dO is read
-// once for D and for its quantisation.
+// once for D and for its quantisation.  The mixed NVFP4/FP8 path's K job also
+// writes K's NVFP4 form (16-channel blocks inside one token) in the same pass.
 // The kernel is bound by HBM traffic: 2 bytes read and 1 + 1/32 bytes written
 // per element and form (plus 4 bytes read per element of O for D).
 #include <cuda_bf16.h>
 
 #include "internal.h"
 #include "mx.cuh"
+#include "nv.cuh"
 #include "ptx.cuh"
 
 namespace fapk {
@@ -97,10 +99,20 @@ __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(const QuantJobs job
     float a = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(f[p][i]));
-    // the 4 threads of one 32-channel group are adjacent lanes
+    // the 4 threads of one 32-channel group are adjacent lanes; a lane pair
+    // holds one 16-channel block
     a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
     const int row = r0 + p * RPP;
+    if (D == 128 && job.nvv && row < nb) {
+      // NVFP4 form: both lanes of the pair derive the same scale from the
+      // block maximum; each writes its 8 codes, the even lane the scale byte
+      float r;
+      const uint32_t sb = nv_block_scale(a, job.nv_six_g, job.nv_g, r);
+      const size_t t = (size_t)(t0 + row);
+      *reinterpret_cast<uint32_t*>(job.nvv + (t * H + h) * 64 + c8 * 4) = nv_codes8(f[p], r);
+      if ((c8 & 1) == 0) job.nvs[(t * H + h) * 8 + (c8 >> 1)] = (uint8_t)sb;
+    }
+    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
     if ((forms & FAPK_FORM_PT) && row < nb) {
       const int X = mx_block_exponent(a, rule);
       const size_t t = (size_t)(t0 + row);
@@ -156,7 +168,32 @@ cudaError_t launch_jobs(const QuantJobs& jobs, int n_jobs, int T, int d, const i
   return cudaGetLastError();
 }
 
+// NVFP4 of a [T][H][128] tensor: one thread per (token, head, 16-channel block).
+__global__ void __launch_bounds__(256) quantize_nvfp4_kernel(const __nv_bfloat16* __restrict__ x, long long n_blocks,
+                                                             float six_g, float g, uint8_t* __restrict__ codes,
+                                                             uint8_t* __restrict__ scales) {
+  const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= n_blocks) return;
+  const uint4* src = reinterpret_cast<const uint4*>(x + b * 16);
+  float f[16];
+  unpack8(__ldg(src), *reinterpret_cast<float(*)[8]>(&f[0]));
+  unpack8(__ldg(src + 1), *reinterpret_cast<float(*)[8]>(&f[8]));
+  uint32_t c[2];
+  scales[b] = (uint8_t)nv_quant16(f, six_g, g, c);
+  *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(c[0], c[1]);
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_nvfp4(const void* x, int T, int H, float g, uint8_t* codes, uint8_t* scales,
+                                  cudaStream_t stream) {
+  const long long n_blocks = (long long)T * H * 8;
+  if (n_blocks == 0) return cudaSuccess;
+  quantize_nvfp4_kernel<<<(unsigned)((n_blocks + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), n_blocks, 6.0f * g, g, codes, scales);
+  note_launches(1);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_mxfp8(const void* x, int T, int H, int d, const int32_t* cu, int n_docs,
                                   int forms, int rule, uint8_t* vtb, uint8_t* stb, uint8_t* vpt,

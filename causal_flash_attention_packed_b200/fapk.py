@@ -6,7 +6,7 @@ the current stream.  There is no fallback: if ``libfapk.so`` is missing or
 cannot be loaded, every call raises ``FapkError``.
 
 Names follow the C ABI without the ``fapk_`` prefix: ``attn_fwd``,
-``attn_bwd``, ``quantize_mxfp8``, ``workspace_size``, ``ctx_size``,
+``attn_bwd``, ``quantize_mxfp8``, ``quantize_nvfp4``, ``workspace_size``, ``ctx_size``,
 ``status``, ``strerror``.
 """
 from __future__ import annotations
@@ -33,6 +33,7 @@ ERR_INTERNAL = 8
 
 BF16 = 0
 MXFP8 = 1
+NVFP4_MIXED = 2
 GRAD_F32 = 0
 GRAD_BF16 = 1
 SCALE_RCEIL = 0
@@ -69,6 +70,8 @@ class Problem(ctypes.Structure):
         ("timeout_ms", ctypes.c_int),
         ("timing_events", ctypes.c_void_p),
         ("n_timing_events", ctypes.c_int),
+        ("nv_scale_q", ctypes.c_float),
+        ("nv_scale_k", ctypes.c_float),
     ]
 
 
@@ -104,6 +107,8 @@ def lib() -> ctypes.CDLL:
     L.fapk_noalloc_status.restype = i
     L.fapk_quantize_mxfp8.argtypes = [vp, i, i, i, vp, vp, i, i, i, vp, vp, vp, vp, vp]
     L.fapk_quantize_mxfp8.restype = i
+    L.fapk_quantize_nvfp4.argtypes = [vp, i, i, i, ctypes.c_float, vp, vp, vp]
+    L.fapk_quantize_nvfp4.restype = i
     L.fapk_status.argtypes = [vp, vp]
     L.fapk_status.restype = i
     L.fapk_cta_times.argtypes = [PP, i, i, vp, vp, ctypes.POINTER(ctypes.c_ulonglong), i, ctypes.POINTER(i)]
@@ -156,7 +161,8 @@ class Seqlens:
 
 def make_problem(seq: Seqlens, Hq: int, Hkv: int, d: int, scale: float, prec: int = BF16,
                  grad_dtype: int = GRAD_F32, scale_rule: int = SCALE_RCEIL, flags: int = 0,
-                 timeout_ms: int = 0, validate_host: bool = True) -> Problem:
+                 timeout_ms: int = 0, validate_host: bool = True, nv_scale_q: float = 0.0,
+                 nv_scale_k: float = 0.0) -> Problem:
     P = Problem()
     P.T = seq.T
     P.n_docs = seq.n_docs
@@ -172,6 +178,9 @@ def make_problem(seq: Seqlens, Hq: int, Hkv: int, d: int, scale: float, prec: in
     P.timeout_ms = timeout_ms
     P.timing_events = None
     P.n_timing_events = 0
+    P.nv_scale_q = float(nv_scale_q)
+    P.nv_scale_k = float(nv_scale_k)
+    P._seqlens = seq  # the problem points at seq's device array: keep it alive with the problem
     return P
 
 
@@ -190,6 +199,7 @@ class KernelTimer:
 
     def with_events(self, P: Problem) -> Problem:
         Q = Problem.from_buffer_copy(P)
+        Q._seqlens = getattr(P, "_seqlens", None)
         Q.timing_events = ctypes.cast(self._handles, ctypes.c_void_p)
         Q.n_timing_events = len(self.events)
         return Q
@@ -338,6 +348,18 @@ def quantize_mxfp8(x: torch.Tensor, seq: Seqlens, forms: int = FORM_TB | FORM_PT
                                    _stream(stream))
     _check(rc, "fapk_quantize_mxfp8")
     return out
+
+
+def quantize_nvfp4(x: torch.Tensor, g: float = 1.0, stream=None):
+    """fapk_quantize_nvfp4 of x [T,H,128] bf16 with decode scale g.  Returns
+    (codes uint8 [T,H,64], channel 2i in the low nibble of byte i; scales
+    uint8 [T,H,8], E4M3)."""
+    T, H, d = x.shape
+    codes = torch.empty((T, H, d // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((T, H, d // 16), dtype=torch.uint8, device=x.device)
+    _check(lib().fapk_quantize_nvfp4(_ptr(x), T, H, d, float(g), _ptr(codes), _ptr(scales), _stream(stream)),
+           "fapk_quantize_nvfp4")
+    return codes, scales
 
 
 def cta_times(P: Problem, which: int, kernel: int, ws: torch.Tensor, stream=None):

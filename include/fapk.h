@@ -82,8 +82,16 @@ typedef enum {
                                        1024-byte aligned and computed nothing */
 } fapk_status_t;
 
-/* Operand precision of the attention path. */
-typedef enum { FAPK_BF16 = 0, FAPK_MXFP8 = 1 } fapk_prec_t;
+/* Operand precision of the attention path.
+ *  FAPK_NVFP4_MIXED: the mixed NVFP4/FP8 path (FLAMIA page, sec. "FLAMIA
+ *    Mimarisi ve Temel Tasarim Ilkeleri", which names mixed NVFP4/FP8 training
+ *    paths beside MXFP8).  The scores S = Q K^T, in the forward and in the
+ *    backward's recomputation alike, take Q and K in NVFP4 (E2M1 codes, one
+ *    E4M3 scale per 16 channels of one token, the per-tensor decode scales
+ *    nv_scale_q and nv_scale_k; see fapk_quantize_nvfp4); every other
+ *    product is the MXFP8 path's (P~ V, dO V^T, and the gradient products
+ *    with the MXFP8 forms of K, Q and dO).  d = 128 only. */
+typedef enum { FAPK_BF16 = 0, FAPK_MXFP8 = 1, FAPK_NVFP4_MIXED = 2 } fapk_prec_t;
 
 /* Element type of dq, dk, dv. */
 typedef enum { FAPK_GRAD_F32 = 0, FAPK_GRAD_BF16 = 1 } fapk_grad_dtype_t;
@@ -148,6 +156,12 @@ typedef struct {
                                     [1] query-tile schedule, [2] D and MX quantisation of dO,
                                     [3] dK/dV kernel, [4] dQ kernel, [5] end. */
   int n_timing_events;
+  float nv_scale_q, nv_scale_k;  /* FAPK_NVFP4_MIXED: per-tensor fp32 decode scales g of
+                                    Q and K (0 selects 1; else within [2^-100, 2^100],
+                                    FAPK_ERR_INVALID_ARG otherwise).  They are the
+                                    caller's, e.g. from earlier steps' maxima: a scale
+                                    taken from this batch's tensor-wide maximum would
+                                    let later tokens set the codes of earlier ones. */
 } fapk_problem_t;
 
 /* Bytes of workspace the forward (which = FAPK_FWD) or backward
@@ -162,7 +176,7 @@ FAPK_API size_t fapk_workspace_size(const fapk_problem_t* prob, int which);
  * sees O to about 16 significant bits; the bf16 path adds an fp16 copy of V,
  * the MXFP8 path the MX forms (codes and scales, token-block and per-token) of
  * Q, K and V, reused across orientations (FLAMIA page: "token-block
- * scaling"). */
+ * scaling"); the mixed NVFP4/FP8 path adds the NVFP4 forms of Q and K. */
 FAPK_API size_t fapk_ctx_size(const fapk_problem_t* prob);
 
 /* Forward.  Reads q, k, v (bf16); writes o (bf16) and lse (fp32, natural
@@ -206,6 +220,23 @@ FAPK_API int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const 
                         const int32_t* cu_seqlens_host, int n_docs, int forms, int scale_rule,
                         uint8_t* val_tb, uint8_t* scale_tb, uint8_t* val_pt, uint8_t* scale_pt,
                         void* stream);
+
+/* NVFP4 quantisation of a bf16 tensor x [T][H][d] (d = 128), the operand
+ * form of the mixed NVFP4/FP8 path's scores.  NVFP4 is NVIDIA's published
+ * format (the FLAMIA page only names it): E2M1 codes, one unsigned E4M3
+ * scale per 16 consecutive channels of one token, and the per-tensor fp32
+ * decode scale g, x ~ code * scale * g.  A block with largest magnitude a is
+ * quantised in fp32 arithmetic, each step rounded to nearest even:
+ *   s = E4M3(a / (6 g))     (saturating at 448; 0 for an all-zero block),
+ *   r = 1 / (decode(s) g)   (0 when that product is 0),
+ *   code_i = E2M1(x_i r)    (saturating at +-6; a zero result is code 0).
+ * codes [T][H][d/2] (channel 2i in the low nibble of byte i), 8-byte
+ * aligned; scales [T][H][d/16].  g must be finite and within [2^-100,
+ * 2^100] (FAPK_ERR_INVALID_ARG); x 16-byte aligned.  The attention path's
+ * own NVFP4 operands are computed with the same arithmetic (K by its
+ * prepass, Q on load by the forward kernel). */
+FAPK_API int fapk_quantize_nvfp4(const void* x_bf16, int T, int H, int d, float g, uint8_t* codes,
+                                 uint8_t* scales, void* stream);
 
 /* MXFP8 forward over already-quantised K and V ("Flash Attention" glossary
  * page on local inference engines, secs. "Tanim" and the KV-cache table: a

@@ -131,6 +131,31 @@ def test_quantize_validation(L):
     assert q(x, 0, 2, 64, None, None, 0, 3, 0, None, None, None, None, None) == fapk.OK
 
 
+def test_nvfp4_mixed_validation(L):
+    """The mixed NVFP4/FP8 path: d = 128 and RCEIL only, decode scales 0 (=1)
+    or finite within [2^-100, 2^100]; its ctx adds Q's and K's NVFP4 forms
+    (64 code bytes and 8 scale bytes per token and head) to the MXFP8 ctx."""
+    nv = dict(prec=fapk.NVFP4_MIXED)
+    assert _fwd(L, _problem(d=64, **nv)) == fapk.ERR_UNSUPPORTED
+    assert _fwd(L, _problem(scale_rule=fapk.SCALE_OCP, **nv)) == fapk.ERR_UNSUPPORTED
+    for bad in (float("nan"), float("inf"), -1.0, 2.0 ** -101, 2.0 ** 101):
+        assert _fwd(L, _problem(nv_scale_q=bad, **nv)) == fapk.ERR_INVALID_ARG
+        assert _fwd(L, _problem(nv_scale_k=bad, **nv)) == fapk.ERR_INVALID_ARG
+    assert _fwd(L, _problem(T=0, n_docs=0, nv_scale_q=0.5, nv_scale_k=4.0, **nv)) == fapk.OK
+    P, M = _problem(**nv), _problem(prec=fapk.MXFP8)
+    T, Hq, Hkv = P.T, P.Hq, P.Hkv
+    assert fapk.ctx_size(P) >= fapk.ctx_size(M) + T * (Hq + Hkv) * 72
+    assert fapk.workspace_size(P, fapk.FWD) == fapk.workspace_size(M, fapk.FWD)
+    assert fapk.workspace_size(P, fapk.BWD) == fapk.workspace_size(M, fapk.BWD)
+    q = L.fapk_quantize_nvfp4
+    assert q(256, 64, 2, 64, ctypes.c_float(1.0), 256, 256, None) == fapk.ERR_UNSUPPORTED
+    assert q(256, 64, 2, 128, ctypes.c_float(0.0), 256, 256, None) == fapk.ERR_INVALID_ARG
+    assert q(256, 64, 2, 128, ctypes.c_float(float("nan")), 256, 256, None) == fapk.ERR_INVALID_ARG
+    assert q(264, 64, 2, 128, ctypes.c_float(1.0), 256, 256, None) == fapk.ERR_INVALID_ARG  # x alignment
+    assert q(256, 64, 2, 128, ctypes.c_float(1.0), 260, 256, None) == fapk.ERR_INVALID_ARG  # codes alignment
+    assert q(256, 0, 2, 128, ctypes.c_float(1.0), None, None, None) == fapk.OK
+
+
 @pytest.mark.parametrize("prec,rows", [(fapk.BF16, 256), (fapk.MXFP8, 128)])
 def test_noalloc_size_limit_matches_its_documented_formula(L, prec, rows):
     """The forward workspace that the no-allocation entry point must fit in its
