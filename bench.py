@@ -33,6 +33,13 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 METRIC = "causal fwd+bwd attention TFLOP/s (bf16, MXFP8 incl. quant) & % of B200 tensor peak"
+# the library's precision constant of each path name
+PREC = {"bf16": "BF16", "mxfp8": "MXFP8", "nvfp4": "NVFP4_MIXED"}
+# mixed NVFP4/FP8 path: the scores' MMAs run FP4 (twice the FP8 rate), the
+# other products FP8; the time-weighted peak of each kernel in units of the
+# FP8 peak: forward S + PV = 2 + 2 -> 4 / (1 + 2); dK/dV S, dP, dV, dK ->
+# 8 / (1 + 6); dQ S, dP, dQ -> 6 / (1 + 4)
+NV_PEAK_FACTOR = {"fwd_kernel": 4.0 / 3.0, "dkdv_kernel": 8.0 / 7.0, "dq_kernel": 6.0 / 5.0}
 DENSE_BF16_TFLOPS = 2250.0   # NVIDIA B200 datasheet, dense
 DENSE_FP8_TFLOPS = 4500.0
 
@@ -210,6 +217,7 @@ KERNELS = {
     "mxfp8": (["schedule_fwd", "quantize_kv", "fwd_kernel"],
               ["schedule_kv", "schedule_q", "delta_quantize_do", "dkdv_kernel", "dq_kernel"]),
 }
+KERNELS["nvfp4"] = KERNELS["mxfp8"]  # the same launches (the K pass also writes K's NVFP4 form)
 # algorithmic tensor work of each attention kernel per visible (query, key)
 # pair and query head, in units of d: forward S and PV = 4; dK/dV kernel S,
 # dP, dV, dK = 8; dQ kernel S, dP, dQ = 6
@@ -233,8 +241,7 @@ class Path:
         self.qd, self.kd, self.vd, self.dod = tensors
         seq = fapk.Seqlens(w.cu, dev)
         self.seq = seq
-        self.P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale,
-                                   prec=fapk.MXFP8 if prec == "mxfp8" else fapk.BF16)
+        self.P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale, prec=getattr(fapk, PREC[prec]))
         self.ws_f = fapk.workspace(self.P, fapk.FWD, dev)
         self.ws_b = fapk.workspace(self.P, fapk.BWD, dev)
         self.o = torch.empty((w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
@@ -261,7 +268,7 @@ class Path:
         units are handed out in order to the SM that frees up first."""
         f = self.fapk
         P = f.make_problem(self.seq, self.w.Hq, self.w.Hkv, self.w.d, self.w.scale,
-                           prec=f.MXFP8 if self.prec == "mxfp8" else f.BF16, flags=f.FLAG_CTA_TIMES)
+                           prec=getattr(f, PREC[self.prec]), flags=f.FLAG_CTA_TIMES)
         f.attn_fwd(P, self.qd, self.kd, self.vd, o=self.o, lse=self.lse, ctx=self.ctx, ws=self.ws_f,
                    stream=self.stream)
         fwd = f.cta_times(P, f.FWD, 0, self.ws_f, self.stream)
@@ -343,7 +350,7 @@ def analytic_balance(w, prec, num_sms):
         used = loads[: min(n, num_sms)]
         return float(np.mean(used) / max(used)) if used and max(used) > 0 else 1.0
 
-    if prec == "mxfp8":
+    if prec != "bf16":
         fwd = ratio(units(128, w.Hq, lambda k, nt, r: nt - r))
     else:
         fwd = ratio(units(256, w.Hq, fwd_pair))
@@ -364,6 +371,11 @@ def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, clk, conf
     dom_flops = KERNEL_FLOPS[dom] * w.d * w.Hq * pairs
     achieved = dom_flops / (kern_ms[dom] * 1e-3) / 1e12
     peak, peak_src = tensor_peak(peaks, clk, prec != "bf16")
+    kpeak = {n: peak * (NV_PEAK_FACTOR[n] if prec == "nvfp4" else 1.0) for n in KERNEL_FLOPS}
+    if prec == "nvfp4":
+        peak *= NV_PEAK_FACTOR[dom]
+        peak_src = (f"{NV_PEAK_FACTOR[dom]:.4f} x " + peak_src + " (the scores' FP4 MMAs at twice the FP8 "
+                    "rate, weighted by the kernel's products)")
     dense = DENSE_BF16_TFLOPS if prec == "bf16" else DENSE_FP8_TFLOPS
     traffic = MEASURED_TRAFFIC.get(config, {}).get(prec, {}).get(dom)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -374,16 +386,20 @@ def path_report(w, prec, ms_per_step, kern_ms, launches, world, peaks, clk, conf
                 "kernels_ms": kern_ms,
                 "kernels_tflops": {n: KERNEL_FLOPS[n] * w.d * w.Hq * pairs / (kern_ms[n] * 1e-3) / 1e12
                                    for n in KERNEL_FLOPS},
+                "kernels_frac": {n: KERNEL_FLOPS[n] * w.d * w.Hq * pairs / (kern_ms[n] * 1e-3) / 1e12 / kpeak[n]
+                                 for n in KERNEL_FLOPS},
                 "fwd": {"ms": fwd_ms, "tflops": 4.0 * w.d * w.Hq * pairs / (fwd_ms * 1e-3) / 1e12},
                 "bwd": {"ms": bwd_ms, "tflops": 10.0 * w.d * w.Hq * pairs / (bwd_ms * 1e-3) / 1e12}}
     out = {"value": value, "ms_per_step": ms_per_step, "pct_of_dense_peak": 100.0 * (value / world) / dense,
            "dense_peak_tflops": dense, "roofline": roofline, "gpu_launches": launches}
-    if prec == "mxfp8":
+    if prec != "bf16":
         # the standalone quantisation launch of the forward (K and V, both
         # forms; HBM bound), algorithmic bytes per element: 2 B bf16 read, then
         # per form 1 B of E4M3 codes and 1/32 B of scales written.  Q is
         # quantised on load inside the forward kernel, dO inside the D pass.
         qbytes = 2 * w.T * w.Hkv * w.d * (2.0 + 2 * (1.0 + 1.0 / 32))
+        if prec == "nvfp4":  # K's NVFP4 form too: 1/2 B of codes and 1/16 B of scales per element
+            qbytes += w.T * w.Hkv * w.d * (0.5 + 1.0 / 16)
         gbs = qbytes / (kern_ms["quantize_kv"] * 1e-3) / 1e9
         qtraffic = MEASURED_TRAFFIC.get(config, {}).get(prec, {})
         out["roofline_quantize"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -439,7 +455,7 @@ def main():
     ap.add_argument("--impl", default="fapk", choices=["fapk", "reference"])
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--paths", default="bf16,mxfp8")
+    ap.add_argument("--paths", default="bf16,mxfp8,nvfp4")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

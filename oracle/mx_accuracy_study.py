@@ -9,7 +9,8 @@ Prints two markdown tables.
    Temel Tasarim Ilkeleri": MXFP8 operands, token-block scaling, leak guards)
    and with one quantisation taken out at a time (inputs Q, K, V, dO; the
    computed P~/P~T; the computed dS~/dS~T), with the OCP scale rule, and with
-   the symmetric diagonal guard.  Workloads: the 16384-token outlier-channel
+   the symmetric diagonal guard, and for the mixed NVFP4/FP8 path (scores
+   from NVFP4 Q and K, decode scales 1).  Workloads: the 16384-token outlier-channel
    workload (all 16 heads) and the first documents of the 32768-token
    log-normal workload (KV heads 0-7).
 2. The leak test T3 at document-local token positions t that are not the end
@@ -43,6 +44,7 @@ VARIANTS = [
     ("only inputs quantised", oracle.MX_QUANT_P | oracle.MX_KEEP_P | oracle.MX_KEEP_DS),
     ("OCP scale rule", oracle.MX_QUANT_P | oracle.MX_RULE_OCP),
     ("symmetric diagonal guard", oracle.MX_QUANT_P | oracle.MX_SYM_GUARD),
+    ("mixed NVFP4/FP8 (NVFP4 scores)", None),
 ]
 
 
@@ -73,7 +75,10 @@ def cosine_table():
         args, cu, n, T = _subset(w, max_tokens, kvh)
         ex = oracle.attn_bwd(*args, cu, w.scale)
         for name, flags in VARIANTS:
-            em = oracle.mx_attn_bwd(*args, cu, w.scale, flags=flags)
+            if flags is None:
+                em = oracle.nvmx_attn_bwd(*args, cu, w.scale, flags=oracle.MX_QUANT_P)
+            else:
+                em = oracle.mx_attn_bwd(*args, cu, w.scale, flags=flags)
             rows.append((f"{title} ({n} docs, {T} tokens)", name,
                          *(_cos(em[key], ex[key]) for key in ("o", "dq", "dk", "dv"))))
     out = ["| workload | emulation | O | dQ | dK | dV |", "|---|---|---|---|---|---|"]
