@@ -78,7 +78,6 @@ int validate_problem(const fapk_problem_t* P) {
   // operands quantise discontinuously near powers of two (see fapk.h)
   if (is_mx(P) && P->scale_rule != FAPK_SCALE_RCEIL) return FAPK_ERR_UNSUPPORTED;
   if (P->prec == FAPK_NVFP4_MIXED) {
-    if (P->d != 128) return FAPK_ERR_UNSUPPORTED;
     if (!nv_scale_ok(P->nv_scale_q) || !nv_scale_ok(P->nv_scale_k)) return FAPK_ERR_INVALID_ARG;
   }
   if (P->grad_dtype != FAPK_GRAD_F32 && P->grad_dtype != FAPK_GRAD_BF16) return FAPK_ERR_UNSUPPORTED;

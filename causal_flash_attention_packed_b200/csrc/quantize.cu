@@ -103,14 +103,20 @@ __global__ void __launch_bounds__(128) quantize_mxfp8_kernel(const QuantJobs job
     // holds one 16-channel block
     a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
     const int row = r0 + p * RPP;
-    if (D == 128 && job.nvv && row < nb) {
+    if (job.nvv && row < nb) {
       // NVFP4 form: both lanes of the pair derive the same scale from the
-      // block maximum; each writes its 8 codes, the even lane the scale byte
+      // block maximum; each writes its 8 codes, the even lane the scale byte.
+      // The row always has 128 channels: for D = 64 channels 64..127 are zero
+      // codes with scale 0, which add nothing to a product.
       float r;
       const uint32_t sb = nv_block_scale(a, job.nv_six_g, job.nv_g, r);
       const size_t t = (size_t)(t0 + row);
       *reinterpret_cast<uint32_t*>(job.nvv + (t * H + h) * 64 + c8 * 4) = nv_codes8(f[p], r);
       if ((c8 & 1) == 0) job.nvs[(t * H + h) * 8 + (c8 >> 1)] = (uint8_t)sb;
+      if (D < 128) {
+        *reinterpret_cast<uint32_t*>(job.nvv + (t * H + h) * 64 + D / 2 + c8 * 4) = 0u;
+        if ((c8 & 1) == 0) job.nvs[(t * H + h) * 8 + D / 16 + (c8 >> 1)] = 0;
+      }
     }
     a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
     if ((forms & FAPK_FORM_PT) && row < nb) {

@@ -90,7 +90,8 @@ typedef enum {
  *    E4M3 scale per 16 channels of one token, the per-tensor decode scales
  *    nv_scale_q and nv_scale_k; see fapk_quantize_nvfp4); every other
  *    product is the MXFP8 path's (P~ V, dO V^T, and the gradient products
- *    with the MXFP8 forms of K, Q and dO).  d = 128 only. */
+ *    with the MXFP8 forms of K, Q and dO).  d = 64 or 128 (the NVFP4 rows keep
+ *    128 channels; for d = 64 the upper 64 are zero codes with scale 0). */
 typedef enum { FAPK_BF16 = 0, FAPK_MXFP8 = 1, FAPK_NVFP4_MIXED = 2 } fapk_prec_t;
 
 /* Element type of dq, dk, dv. */

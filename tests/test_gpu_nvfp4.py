@@ -125,6 +125,14 @@ def test_gqa_and_decode_scales():
     _check(w, require_gpu(), gq=0.37, gk=3.5)
 
 
+@pytest.mark.parametrize("G", [1, 2])
+def test_head_dim_64_ragged_documents(G):
+    """d = 64: the NVFP4 rows keep 128 channels with a zero upper half (scale
+    0), which adds nothing to the scores; against the emulation at d = 64."""
+    w = W.custom([1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 300, 700], Hq=2 * G, Hkv=2, d=64, seed=84)
+    _check(w, require_gpu())
+
+
 def test_outlier_channels_16k_full():
     """The 16384-token workload with x20 outlier channels, full size."""
     _check(W.config(3, 0), require_gpu())
@@ -175,6 +183,12 @@ def test_bwd_ragged_documents():
 def test_bwd_gqa_and_decode_scales():
     w = W.custom([513, 64, 1000], Hq=4, Hkv=2, d=128, seed=92)
     _check_bwd(w, require_gpu(), gq=2.0, gk=0.3)
+
+
+@pytest.mark.parametrize("G", [1, 2])
+def test_bwd_head_dim_64_ragged_documents(G):
+    w = W.custom([1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 300, 700], Hq=2 * G, Hkv=2, d=64, seed=95)
+    _check_bwd(w, require_gpu())
 
 
 def test_bwd_outlier_channels_16k_full():
