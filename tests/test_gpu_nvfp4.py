@@ -235,3 +235,58 @@ def test_bwd_dkdv_leak_free_at_block_aligned_t(t_rel):
     _, b = nv_fwd_bwd(w, dev, tensors=_perturb(base, t, 10, zero_dout=True))
     assert torch.equal(a[3][: t + 1], b[3][: t + 1])
     assert torch.equal(a[4][: t + 1], b[4][: t + 1])
+
+
+def _nv_sampled_docs(w, dev, max_tokens=6000, first_doc=0, kv_group=0):
+    """Full-size workload in the launch configuration the benchmark uses; the
+    oracle's mixed emulation reruns whole documents (every scale is per token
+    or document-local, so a document's outputs depend on its own tokens only)
+    for the query heads of one KV group: O, LSE, dQ, dK, dV of those documents
+    and heads against the emulation."""
+    (q, k, v, do), (o, lse, dq, dk, dv) = nv_fwd_bwd(w, dev)
+    cu = w.cu
+    k0 = k1 = first_doc
+    while k1 < w.n_docs and cu[k1 + 1] - cu[k0] <= max_tokens:
+        k1 += 1
+    if k1 == k0:  # the first candidate alone is longer than the budget
+        k1 = k0 + 1
+    t0, t1 = int(cu[k0]), int(cu[k1])
+    G = w.Hq // w.Hkv
+    hs = list(range(kv_group * G, (kv_group + 1) * G))
+    cu_s = (cu[k0:k1 + 1] - t0).astype(np.int32)
+    sub_q = lambda x: x[t0:t1, hs].double().numpy()  # noqa: E731
+    sub_k = lambda x: x[t0:t1, kv_group:kv_group + 1].double().numpy()  # noqa: E731
+    em = oracle.nvmx_attn_bwd(sub_q(q), sub_k(k), sub_k(v), sub_q(do), cu_s, w.scale)
+    res = {
+        "o": rel_frob(f64(o)[t0:t1, hs], em["o"]),
+        "dq": rel_frob(f64(dq)[t0:t1, hs], em["dq"]),
+        "dk": rel_frob(f64(dk)[t0:t1, kv_group:kv_group + 1], em["dk"]),
+        "dv": rel_frob(f64(dv)[t0:t1, kv_group:kv_group + 1], em["dv"]),
+    }
+    print(f"documents {k0}..{k1 - 1} ({t1 - t0} tokens), KV group {kv_group}: " +
+          ", ".join(f"{n} {r:.2e}" for n, r in res.items()))
+    for name, rf in res.items():
+        assert rf <= NV_REL_FROB, f"{name} rel_frob vs emulation {rf:.3e} (documents {k0}..{k1 - 1})"
+    assert float(np.max(np.abs(f64(lse)[hs, t0:t1] - em["lse"]))) <= LSE_ABS
+
+
+@pytest.mark.parametrize("first_doc,max_tokens,kv_group", [(0, 6000, 0), (6, 13000, 9)])
+def test_full_size_packed_32k_documents_vs_emulation(first_doc, max_tokens, kv_group):
+    """The 32768-token benchmark workload (32 heads, 1% x8 outlier tokens):
+    its first two documents (2322 and 1795 tokens), and its two longest
+    (7545 and 5280 tokens, documents 6 and 7)."""
+    _nv_sampled_docs(W.config(4, 0), require_gpu(), max_tokens=max_tokens, first_doc=first_doc,
+                     kv_group=kv_group)
+
+
+def test_full_size_gqa_128k_documents_vs_emulation():
+    """131072 tokens with a 65536-token first document, 32 query heads on 8 KV
+    heads; two documents after the long one, KV group 3."""
+    _nv_sampled_docs(W.config(5, 0), require_gpu(), first_doc=4, kv_group=3)
+
+
+def test_zero_length_and_one_token_documents():
+    """Empty documents between others and one-token documents: the empty ones
+    own no tile, the one-token ones are a single visible key."""
+    w = W.custom([0, 1, 0, 0, 37, 1, 0, 200, 1, 0], Hq=2, Hkv=1, d=128, seed=96)
+    _check_bwd(w, require_gpu())
