@@ -290,3 +290,28 @@ def test_zero_length_and_one_token_documents():
     own no tile, the one-token ones are a single visible key."""
     w = W.custom([0, 1, 0, 0, 37, 1, 0, 200, 1, 0], Hq=2, Hkv=1, d=128, seed=96)
     _check_bwd(w, require_gpu())
+
+
+def test_multi_query_attention_fwd_bwd():
+    """MQA in the mixed path (Hkv = 1, eight query heads)."""
+    w = W.custom([1, 129, 300, 700, 64], Hq=8, Hkv=1, d=128, seed=97)
+    _check(w, require_gpu())
+    _check_bwd(w, require_gpu())
+
+
+def test_bf16_gradient_output():
+    """grad_dtype = bf16 in the mixed path: the gradients are the fp32 ones
+    rounded to bf16 (bit for bit)."""
+    dev = require_gpu()
+    w = W.custom([200, 513, 64], Hq=4, Hkv=2, d=128, seed=98)
+    (q, k, v, do), (qd, kd, vd, dod) = to_dev(w, dev)
+    seq = fapk.Seqlens(w.cu, dev)
+    outs = []
+    for gdt in (fapk.GRAD_F32, fapk.GRAD_BF16):
+        P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale, prec=fapk.NVFP4_MIXED, grad_dtype=gdt)
+        o, lse, ctx = fapk.attn_fwd(P, qd, kd, vd)
+        outs.append(fapk.attn_bwd(P, qd, kd, vd, o, lse, dod, ctx=ctx))
+    torch.cuda.synchronize()
+    for a, b in zip(*outs):
+        assert b.dtype == torch.bfloat16
+        assert torch.equal(a.to(torch.bfloat16), b)
