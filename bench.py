@@ -449,6 +449,35 @@ def time_qkv_proj(fapk, w, dev, peaks, clk, warmup, steps):
             "note": "includes the schedule launch and the MX forms of K and V written by the epilogue"}
 
 
+def time_quantized_kv(fapk, w, dev, tensors, peaks, clk, warmup, steps):
+    """CUDA-event time of fapk_attn_fwd_quantized_kv (the MXFP8 forward over
+    K and V given in both MX forms, as a cache would hold them: no
+    quantisation launch) on the workload; 4 d Hq pairs FLOP."""
+    qd, kd, vd = tensors[:3]
+    seq = fapk.Seqlens(w.cu, dev)
+    P = fapk.make_problem(seq, w.Hq, w.Hkv, w.d, w.scale, prec=fapk.MXFP8)
+    kf = fapk.quantize_mxfp8(kd, seq)
+    vf = fapk.quantize_mxfp8(vd, seq)
+    ws = fapk.workspace(P, fapk.FWD, dev)
+    o = torch.empty((w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.Hq, w.T), dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        fapk.attn_fwd_quantized_kv(P, qd, kf, vf, o=o, lse=lse, ws=ws)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fapk.attn_fwd_quantized_kv(P, qd, kf, vf, o=o, lse=lse, ws=ws)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    tf = 4.0 * w.d * w.Hq * w.pairs() / (ms * 1e-3) / 1e12
+    peak, src = tensor_peak(peaks, clk, True)
+    return {"ms": ms, "tflops": tf, "frac": tf / peak, "peak": peak, "peak_source": src,
+            "status_ok": fapk.status(ws) == 0,
+            "note": "forward only, K and V pre-quantised; includes the schedule launch"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -505,6 +534,11 @@ def main():
     proj = None
     if args.qkv_proj and w.d == 128:
         proj = time_qkv_proj(fapk, w, dev, peaks, clk, args.warmup, min(args.steps, 20))
+
+    # the forward over pre-quantised K and V (a quantised KV cache)
+    qkv_cached = None
+    if w.d == 128:
+        qkv_cached = time_quantized_kv(fapk, w, dev, dev_tensors, peaks, clk, args.warmup, min(args.steps, 20))
 
     # end to end through the C ABI with host buffers (pinned), copies included:
     # every step copies its inputs host -> device and its outputs device ->
@@ -579,7 +613,7 @@ def main():
         "pct_of_dense_bf16_peak": head["pct_of_dense_peak"] if main_path == "bf16" else None,
         "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
-        "clocks": clk, "status_ok": st_ok, "qkv_proj": proj,
+        "clocks": clk, "status_ok": st_ok, "qkv_proj": proj, "fwd_quantized_kv": qkv_cached,
         "scheduler_balance": balance,
     }
     for p in paths[1:]:

@@ -597,9 +597,10 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
 // ---------------------------------------------------------------------------
 namespace kvk {
 // warps 0-15: one thread per (key row, 32-query block): warpgroup wg on query
-// block wg of every tile (one MX scale block of P~T and dS~T); warp 16: K/V,
-// Q^pt, dO^pt, lse and D loads; warp 17: MMA issue; warp 18: dO^tb and Q^tb loads
-constexpr int kThreads = 608, kLoadA = 16, kMma = 17, kLoadB = 18, kComputeWarps = 16;
+// block wg of every tile (one MX scale block of P~T and dS~T); warp 16: all
+// loads (K/V; per query tile lse, D, Q^pt, dO^pt, dO^tb, Q^tb); warp 17: MMA
+// issue.  18 warps leave 112 registers per thread (19 would leave 96).
+constexpr int kThreads = 576, kLoadA = 16, kMma = 17, kComputeWarps = 16;
 // per item: K^tb, K^pt, V^tb, V^pt codes; per query tile one buffer per
 // operand (Q^pt, dO^pt, dO^tb, Q^tb codes), each released as soon as its last
 // MMA has read it; P~T and dS~T codes; lse*log2e[128] and D[128] of the query
@@ -684,7 +685,7 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kComputeWarps);
     mbar_init(fin, 1);
-    unit_ring_init(ring, 2 + kComputeWarps);  // loader B, the MMA thread and the compute warps
+    unit_ring_init(ring, 1 + kComputeWarps);  // the MMA thread and the compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -799,6 +800,11 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           mbar_arrive(aux_full + ab);
           if (!load_op(kQpt, t, &tm_qpt, h, q0, sq, 83, kNv ? &sq2 : nullptr)) { ok = false; break; }
           if (!load_op(kDOpt, t, &tm_dopt, h, q0, sdo, 84)) { ok = false; break; }
+          // the query-side operands of dV and dK (token-block form)
+          const uint4 sdotb = tb_channel_rows(p.do_stb, s, e, doc, 4 * m, p.Hq, h);
+          const uint4 sqtb = tb_channel_rows(p.q_stb, s, e, doc, 4 * m, p.Hq, h);
+          if (!load_op(kDOtb, t, &tm_dotb, h, q0, sdotb, 85)) { ok = false; break; }
+          if (!load_op(kQtb, t, &tm_qtb, h, q0, sqtb, 86)) { ok = false; break; }
         }
       }
     }
@@ -807,31 +813,9 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
       if (t > 0) {
         drain_wait(op_full + kQpt, (t - 1) & 1, p.timeout_ns);
         drain_wait(op_full + kDOpt, (t - 1) & 1, p.timeout_ns);
+        drain_wait(op_full + kDOtb, (t - 1) & 1, p.timeout_ns);
+        drain_wait(op_full + kQtb, (t - 1) & 1, p.timeout_ns);
       }
-    }
-  } else if (warp == kLoadB) {
-    // ------------------------------------------------- dO^tb, Q^tb
-    uint32_t t = 0;
-    bool ok = true;
-    for (uint32_t uk = 0; ok; ++uk) {
-      const UnitInfo un = unit_take_warp(ring, uk, wd);
-      const int w = un.w;
-      if (w < 0 || w >= n_units) break;
-      int doc, s, e, g, v, k0, nq;
-      decode(un, doc, s, e, g, v, k0, nq);
-      for (int h = g * G; h < (g + 1) * G && ok; ++h) {
-        for (int m = v; m < nq; ++m, ++t) {
-          const int q0 = s + 128 * m;
-          const uint4 sdo = tb_channel_rows(p.do_stb, s, e, doc, 4 * m, p.Hq, h);
-          const uint4 sq = tb_channel_rows(p.q_stb, s, e, doc, 4 * m, p.Hq, h);
-          if (!load_op(kDOtb, t, &tm_dotb, h, q0, sdo, 85)) { ok = false; break; }
-          if (!load_op(kQtb, t, &tm_qtb, h, q0, sq, 86)) { ok = false; break; }
-        }
-      }
-    }
-    if (lane == 0 && t > 0) {
-      drain_wait(op_full + kDOtb, (t - 1) & 1, p.timeout_ns);
-      drain_wait(op_full + kQtb, (t - 1) & 1, p.timeout_ns);
     }
   } else if (warp == kMma) {
     // ------------------------------------------------- MMA issue
