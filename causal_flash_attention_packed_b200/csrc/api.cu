@@ -416,6 +416,93 @@ int bwd_mxfp8(const fapk_problem_t* P, const void* o, const float* lse, const vo
   return cuda_status(launch_bwd_mxfp8(a, st));
 }
 
+
+// The forward over pre-quantised K and V (no quantisation launch, no saved
+// state): a carries K's forms (MX, or NVFP4 with a.nv); V's MX forms are
+// checked and set here.
+int fwd_quantized_kv(const fapk_problem_t* P, const void* q, FwdMxArgs& a, const uint8_t* v_val_tb,
+                     const uint8_t* v_scale_tb, const uint8_t* v_val_pt, const uint8_t* v_scale_pt, void* o,
+                     float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!q || !v_val_tb || !v_scale_tb || !v_val_pt || !v_scale_pt || !o || !lse || !ws) return FAPK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || !aligned16(v_val_tb) || !aligned16(v_val_pt) ||
+      (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+    return FAPK_ERR_INVALID_ARG;
+  // scale rows are read 4 bytes at a time
+  for (const uint8_t* sp : {v_scale_tb, v_scale_pt})
+    if (reinterpret_cast<uintptr_t>(sp) & 3u) return FAPK_ERR_INVALID_ARG;
+  const FwdLayout L = fwd_layout(P);
+  if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
+  const int sms = device_num_sms();
+  if (sms <= 0) return FAPK_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* status = static_cast<DeviceStatus*>(ws);
+  const Marks mk{P->timing_events, P->n_timing_events};
+  a.sched = sched_buf(ws, L.sched);
+  mk.at(0, st);
+  int rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, a.sched, status, true, st));
+  if (rc != FAPK_OK) return rc;
+  a.q = q;
+  a.q_vpt = a.q_spt = a.q_vtb = a.q_stb = nullptr;  // no saved state: nothing for a backward
+  a.q_nvv = a.q_nvs = nullptr;
+  a.v_vtb = v_val_tb; a.v_stb = v_scale_tb; a.v_vpt = v_val_pt; a.v_spt = v_scale_pt;
+  a.o = o;
+  a.lse = lse;
+  a.o_resid = nullptr;
+  a.cu = P->cu_seqlens_dev;
+  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.n_docs = P->n_docs; a.d = P->d;
+  a.scale = P->scale;
+  a.rule = P->scale_rule;
+  a.status = status;
+  if (P->flags & FAPK_FLAG_CTA_TIMES)
+    a.cta_times[0] = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + L.cta_times);
+  a.timeout_ns = timeout_ns_of(P);
+  a.num_sms = sms;
+  mk.at(1, st);
+  rc = cuda_status(launch_fwd_mxfp8(a, st));
+  mk.at(2, st);
+  return rc;
+}
+
+
+// The fused QKV projection: a carries K's output forms (MX, or NVFP4 when
+// a.k_nvv is set); the rest is checked and set here.
+int qkv_proj(const fapk_problem_t* P, const void* x, int d_model, const void* w, void* q, void* k, void* v,
+             QkvProjArgs& a, uint8_t* v_val_tb, uint8_t* v_scale_tb, uint8_t* v_val_pt, uint8_t* v_scale_pt,
+             void* ws, size_t ws_bytes, void* stream) {
+  if (d_model <= 0 || d_model % 8 != 0) return FAPK_ERR_INVALID_ARG;
+  if (P->T == 0) return FAPK_OK;
+  if (!x || !w || !q || !k || !v || !v_val_tb || !v_scale_tb || !v_val_pt || !v_scale_pt || !ws)
+    return FAPK_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(v_val_tb) ||
+      !aligned16(v_val_pt) || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+    return FAPK_ERR_INVALID_ARG;
+  // 64-bit offsets throughout; keep the weight rows inside the TMA coordinate range
+  if ((long long)(P->Hq + 2 * P->Hkv) * 128 > 0x7FFFFFFFLL) return FAPK_ERR_UNSUPPORTED;
+  const FwdLayout L = fwd_layout(P);  // the MX forward's work order: 128-row tiles per document
+  if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
+  const int sms = device_num_sms();
+  if (sms <= 0) return FAPK_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* status = static_cast<DeviceStatus*>(ws);
+  a.sched = sched_buf(ws, L.sched);
+  const Marks mk{P->timing_events, P->n_timing_events};
+  mk.at(0, st);
+  int rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, a.sched, status, true, st));
+  if (rc != FAPK_OK) return rc;
+  a.x = x; a.w = w; a.q = q; a.k = k; a.v = v;
+  a.v_vtb = v_val_tb; a.v_stb = v_scale_tb; a.v_vpt = v_val_pt; a.v_spt = v_scale_pt;
+  a.cu = P->cu_seqlens_dev;
+  a.T = P->T; a.Dm = d_model; a.Hq = P->Hq; a.Hkv = P->Hkv;
+  a.rule = P->scale_rule;
+  a.status = status;
+  a.timeout_ns = timeout_ns_of(P);
+  a.num_sms = sms;
+  mk.at(1, st);
+  rc = cuda_status(launch_qkv_proj(a, st));
+  mk.at(2, st);
+  return rc;
+}
+
 }  // namespace
 
 }  // namespace fapk
@@ -546,47 +633,32 @@ int fapk_attn_fwd_quantized_kv(const fapk_problem_t* P, const void* q, const uin
   if (rc != FAPK_OK) return rc;
   if (P->prec != FAPK_MXFP8 || P->d != 128) return FAPK_ERR_UNSUPPORTED;
   if (P->T == 0) return FAPK_OK;
-  if (!q || !k_val_tb || !k_scale_tb || !k_val_pt || !k_scale_pt || !v_val_tb || !v_scale_tb || !v_val_pt ||
-      !v_scale_pt || !o || !lse || !ws)
+  if (!k_val_tb || !k_scale_tb || !k_val_pt || !k_scale_pt || !aligned16(k_val_tb) || !aligned16(k_val_pt) ||
+      (reinterpret_cast<uintptr_t>(k_scale_tb) & 3u) || (reinterpret_cast<uintptr_t>(k_scale_pt) & 3u))
     return FAPK_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || !aligned16(k_val_tb) || !aligned16(k_val_pt) ||
-      !aligned16(v_val_tb) || !aligned16(v_val_pt) || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
-    return FAPK_ERR_INVALID_ARG;
-  // scale rows are read 4 bytes at a time
-  for (const uint8_t* sp : {k_scale_tb, k_scale_pt, v_scale_tb, v_scale_pt})
-    if (reinterpret_cast<uintptr_t>(sp) & 3u) return FAPK_ERR_INVALID_ARG;
-  const FwdLayout L = fwd_layout(P);
-  if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
-  const int sms = device_num_sms();
-  if (sms <= 0) return FAPK_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  auto* status = static_cast<DeviceStatus*>(ws);
-  const Marks mk{P->timing_events, P->n_timing_events};
   FwdMxArgs a;
-  a.sched = sched_buf(ws, L.sched);
-  mk.at(0, st);
-  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, a.sched, status, true, st));
-  if (rc != FAPK_OK) return rc;
-  a.q = q;
-  a.q_vpt = a.q_spt = a.q_vtb = a.q_stb = nullptr;  // no saved state: nothing for a backward
   a.k_vtb = k_val_tb; a.k_stb = k_scale_tb; a.k_vpt = k_val_pt; a.k_spt = k_scale_pt;
-  a.v_vtb = v_val_tb; a.v_stb = v_scale_tb; a.v_vpt = v_val_pt; a.v_spt = v_scale_pt;
-  a.o = o;
-  a.lse = lse;
-  a.o_resid = nullptr;
-  a.cu = P->cu_seqlens_dev;
-  a.T = P->T; a.Hq = P->Hq; a.Hkv = P->Hkv; a.n_docs = P->n_docs; a.d = P->d;
-  a.scale = P->scale;
-  a.rule = P->scale_rule;
-  a.status = status;
-  if (P->flags & FAPK_FLAG_CTA_TIMES)
-    a.cta_times[0] = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + L.cta_times);
-  a.timeout_ns = timeout_ns_of(P);
-  a.num_sms = sms;
-  mk.at(1, st);
-  rc = cuda_status(launch_fwd_mxfp8(a, st));
-  mk.at(2, st);
-  return rc;
+  return fwd_quantized_kv(P, q, a, v_val_tb, v_scale_tb, v_val_pt, v_scale_pt, o, lse, ws, ws_bytes, stream);
+}
+
+int fapk_attn_fwd_quantized_kv_nvfp4(const fapk_problem_t* P, const void* q, const uint8_t* k_codes,
+                                     const uint8_t* k_scales, const uint8_t* v_val_tb, const uint8_t* v_scale_tb,
+                                     const uint8_t* v_val_pt, const uint8_t* v_scale_pt, void* o, float* lse,
+                                     void* ws, size_t ws_bytes, void* stream) {
+  int rc = validate_problem(P);
+  if (rc != FAPK_OK) return rc;
+  if (P->prec != FAPK_NVFP4_MIXED || P->d != 128) return FAPK_ERR_UNSUPPORTED;
+  if (P->T == 0) return FAPK_OK;
+  if (!k_codes || !k_scales || !aligned16(k_codes) || (reinterpret_cast<uintptr_t>(k_scales) & 7u))
+    return FAPK_ERR_INVALID_ARG;
+  FwdMxArgs a;
+  a.nv = true;
+  a.k_nvv = k_codes;
+  a.k_nvs = k_scales;
+  a.nv_g_q = nv_scale_of(P->nv_scale_q);
+  a.nv_g_k = nv_scale_of(P->nv_scale_k);
+  a.k_vtb = a.k_stb = a.k_vpt = a.k_spt = nullptr;  // not read on the mixed path
+  return fwd_quantized_kv(P, q, a, v_val_tb, v_scale_tb, v_val_pt, v_scale_pt, o, lse, ws, ws_bytes, stream);
 }
 
 int fapk_qkv_proj_mxfp8(const fapk_problem_t* P, const void* x, int d_model, const void* w, void* q, void* k,
@@ -596,42 +668,28 @@ int fapk_qkv_proj_mxfp8(const fapk_problem_t* P, const void* x, int d_model, con
   int rc = validate_problem(P);
   if (rc != FAPK_OK) return rc;
   if (P->prec != FAPK_MXFP8 || P->d != 128) return FAPK_ERR_UNSUPPORTED;
-  if (d_model <= 0 || d_model % 8 != 0) return FAPK_ERR_INVALID_ARG;
-  if (P->T == 0) return FAPK_OK;
-  if (!x || !w || !q || !k || !v || !k_val_tb || !k_scale_tb || !k_val_pt || !k_scale_pt || !v_val_tb ||
-      !v_scale_tb || !v_val_pt || !v_scale_pt || !ws)
+  if (P->T > 0 && (!k_val_tb || !k_scale_tb || !k_val_pt || !k_scale_pt || !aligned16(k_val_tb) ||
+                   !aligned16(k_val_pt)))
     return FAPK_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_val_tb) ||
-      !aligned16(k_val_pt) || !aligned16(v_val_tb) || !aligned16(v_val_pt) ||
-      (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
-    return FAPK_ERR_INVALID_ARG;
-  // 64-bit offsets throughout; keep the weight rows inside the TMA coordinate range
-  if ((long long)(P->Hq + 2 * P->Hkv) * 128 > 0x7FFFFFFFLL) return FAPK_ERR_UNSUPPORTED;
-  const FwdLayout L = fwd_layout(P);  // the MXFP8 forward's work order: 128-row tiles per document
-  if (ws_bytes < L.total) return FAPK_ERR_WORKSPACE_TOO_SMALL;
-  const int sms = device_num_sms();
-  if (sms <= 0) return FAPK_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  auto* status = static_cast<DeviceStatus*>(ws);
   QkvProjArgs a;
-  a.sched = sched_buf(ws, L.sched);
-  const Marks mk{P->timing_events, P->n_timing_events};
-  mk.at(0, st);
-  rc = cuda_status(launch_schedule(P->cu_seqlens_dev, P->n_docs, kFwdRowsMx, a.sched, status, true, st));
-  if (rc != FAPK_OK) return rc;
-  a.x = x; a.w = w; a.q = q; a.k = k; a.v = v;
   a.k_vtb = k_val_tb; a.k_stb = k_scale_tb; a.k_vpt = k_val_pt; a.k_spt = k_scale_pt;
-  a.v_vtb = v_val_tb; a.v_stb = v_scale_tb; a.v_vpt = v_val_pt; a.v_spt = v_scale_pt;
-  a.cu = P->cu_seqlens_dev;
-  a.T = P->T; a.Dm = d_model; a.Hq = P->Hq; a.Hkv = P->Hkv;
-  a.rule = P->scale_rule;
-  a.status = status;
-  a.timeout_ns = timeout_ns_of(P);
-  a.num_sms = sms;
-  mk.at(1, st);
-  rc = cuda_status(launch_qkv_proj(a, st));
-  mk.at(2, st);
-  return rc;
+  return qkv_proj(P, x, d_model, w, q, k, v, a, v_val_tb, v_scale_tb, v_val_pt, v_scale_pt, ws, ws_bytes, stream);
+}
+
+int fapk_qkv_proj_nvfp4(const fapk_problem_t* P, const void* x, int d_model, const void* w, void* q, void* k,
+                        void* v, uint8_t* k_codes, uint8_t* k_scales, uint8_t* v_val_tb, uint8_t* v_scale_tb,
+                        uint8_t* v_val_pt, uint8_t* v_scale_pt, void* ws, size_t ws_bytes, void* stream) {
+  int rc = validate_problem(P);
+  if (rc != FAPK_OK) return rc;
+  if (P->prec != FAPK_NVFP4_MIXED || P->d != 128) return FAPK_ERR_UNSUPPORTED;
+  if (P->T > 0 && (!k_codes || !k_scales || !aligned16(k_codes) || (reinterpret_cast<uintptr_t>(k_scales) & 1u)))
+    return FAPK_ERR_INVALID_ARG;
+  QkvProjArgs a;
+  a.k_vtb = a.k_stb = a.k_vpt = a.k_spt = nullptr;
+  a.k_nvv = k_codes;
+  a.k_nvs = k_scales;
+  a.nv_g_k = nv_scale_of(P->nv_scale_k);
+  return qkv_proj(P, x, d_model, w, q, k, v, a, v_val_tb, v_scale_tb, v_val_pt, v_scale_pt, ws, ws_bytes, stream);
 }
 
 int fapk_quantize_mxfp8(const void* x_bf16, int T, int H, int d, const int32_t* cu_seqlens_dev,

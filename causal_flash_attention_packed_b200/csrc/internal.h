@@ -212,6 +212,10 @@ struct QkvProjArgs {
   void *q, *k, *v;
   uint8_t *k_vtb, *k_stb, *k_vpt, *k_spt;
   uint8_t *v_vtb, *v_stb, *v_vpt, *v_spt;
+  // K's NVFP4 form (mixed path) instead of its MX forms, or null
+  uint8_t* k_nvv = nullptr;  // codes [T][Hkv][64]
+  uint8_t* k_nvs = nullptr;  // scales [T][Hkv][8]
+  float nv_g_k = 1.f;        // K's decode scale
   const int32_t* cu;
   int T, Dm, Hq, Hkv;
   int rule;
@@ -224,9 +228,9 @@ cudaError_t launch_qkv_proj(const QkvProjArgs& a, cudaStream_t stream);
 
 // Tensor map of E4M3 codes [T][H][128] as (128, H, T), box 128 x 1 x 128,
 // 128-byte swizzle (api.cu).
+bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H);
 // NVFP4 codes [T][H][64 bytes]: boxes of 128 rows x 64 bytes, 64-byte swizzle.
 bool make_tmap_nv(CUtensorMap* map, const void* base, int T, int H);
-bool make_tmap_codes(CUtensorMap* map, const void* base, int T, int H);
 
 // Backward, bf16 operands (bwd_bf16.cu).
 struct BwdArgs {

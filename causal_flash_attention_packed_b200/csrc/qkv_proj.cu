@@ -33,11 +33,13 @@
 //  * warps 2-5: epilogue, one thread per output row (TMEM lane): fp32 -> bf16,
 //    and for K and V heads the per-token form (per 32 channels) and the
 //    token-block form (the warp's 32 rows are one token block) of each
-//    32-channel group.
+//    32-channel group; for the mixed NVFP4/FP8 path K's NVFP4 form (two
+//    16-channel blocks per group) instead of its MX forms.
 #include <cuda_bf16.h>
 
 #include "internal.h"
 #include "mx.cuh"
+#include "nv.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
 
@@ -61,6 +63,8 @@ struct Params {
   __nv_bfloat16 *q, *k, *v;
   uint8_t *k_vtb, *k_stb, *k_vpt, *k_spt;
   uint8_t *v_vtb, *v_stb, *v_vpt, *v_spt;
+  uint8_t *k_nvv, *k_nvs;  // mixed path: K's NVFP4 form instead of its MX forms (null: MX)
+  float nv_g_k, nv_six_g_k;
   DeviceStatus* status;
   uint64_t timeout_ns;
   int T, Dm, Hq, Hkv, n_heads;  // n_heads = Hq + 2 Hkv: the unit's head index runs over Q, K, V heads
@@ -199,21 +203,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(lane_addr + 32 * g, r);
           tmem_wait_ld(r);
           uint32_t b[16];
-  #pragma unroll
+#pragma unroll
           for (int e = 0; e < 16; ++e) b[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
           if (valid) {
             uint4* dst = reinterpret_cast<uint4*>(out + orow + 32 * g);
-  #pragma unroll
+#pragma unroll
             for (int e = 0; e < 4; ++e) dst[e] = make_uint4(b[4 * e], b[4 * e + 1], b[4 * e + 2], b[4 * e + 3]);
           }
           if (is_q) continue;
+          if (is_k && p.k_nvv) {
+            // NVFP4 form of K (two 16-channel blocks), quantised as fapk_quantize_nvfp4 does
+            if (valid) {
+              float f[4][8];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) unpack8(make_uint4(b[4 * c], b[4 * c + 1], b[4 * c + 2], b[4 * c + 3]), f[c]);
+              uint32_t c0[2], c1[2];
+              const uint32_t s0 = nv_quant16(&f[0][0], p.nv_six_g_k, p.nv_g_k, c0);
+              const uint32_t s1 = nv_quant16(&f[2][0], p.nv_six_g_k, p.nv_g_k, c1);
+              const size_t nrow = (size_t)t * H + head;
+              *reinterpret_cast<uint4*>(p.k_nvv + nrow * 64 + 16 * g) = make_uint4(c0[0], c0[1], c1[0], c1[1]);
+              *reinterpret_cast<uint16_t*>(p.k_nvs + nrow * 8 + 2 * g) = (uint16_t)(s0 | (s1 << 8));
+            }
+            continue;
+          }
           // the bf16 values as floats, quantised exactly as fapk_quantize_mxfp8 does
           float f[4][8];
           float a = 0.f;
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < 4; ++c) {
             unpack8(make_uint4(b[4 * c], b[4 * c + 1], b[4 * c + 2], b[4 * c + 3]), f[c]);
-  #pragma unroll
+#pragma unroll
             for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(f[c][i]));
           }
           if (!valid) a = 0.f;  // rows of the next document take no part in this block's scale
@@ -221,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int X = mx_block_exponent(a, p.rule);
           if (valid) {
             uint2 cw[4];
-  #pragma unroll
+#pragma unroll
             for (int c = 0; c < 4; ++c) cw[c] = encode8(f[c], X);
             uint4* dst = reinterpret_cast<uint4*>(vpt + orow + 32 * g);
             dst[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
@@ -230,12 +249,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // token-block form: the warp's 32 rows are one document-local block
           float atb = a;
-  #pragma unroll
+#pragma unroll
           for (int off = 16; off > 0; off >>= 1) atb = fmaxf(atb, __shfl_xor_sync(0xFFFFFFFFu, atb, off));
           const int Xtb = mx_block_exponent(atb, p.rule);
           if (valid) {
             uint2 cw[4];
-  #pragma unroll
+#pragma unroll
             for (int c = 0; c < 4; ++c) cw[c] = encode8(f[c], Xtb);
             uint4* dst = reinterpret_cast<uint4*>(vtb + orow + 32 * g);
             dst[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
@@ -275,6 +294,9 @@ cudaError_t launch_qkv_proj(const QkvProjArgs& a, cudaStream_t stream) {
   p.v = static_cast<__nv_bfloat16*>(a.v);
   p.k_vtb = a.k_vtb; p.k_stb = a.k_stb; p.k_vpt = a.k_vpt; p.k_spt = a.k_spt;
   p.v_vtb = a.v_vtb; p.v_stb = a.v_stb; p.v_vpt = a.v_vpt; p.v_spt = a.v_spt;
+  p.k_nvv = a.k_nvv; p.k_nvs = a.k_nvs;
+  p.nv_g_k = a.nv_g_k;
+  p.nv_six_g_k = 6.0f * a.nv_g_k;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
   p.T = a.T;

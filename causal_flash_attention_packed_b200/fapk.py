@@ -99,10 +99,14 @@ def lib() -> ctypes.CDLL:
     L.fapk_attn_bwd.restype = i
     L.fapk_attn_fwd_noalloc.argtypes = [PP, vp, vp, vp, vp, vp, vp, vp]
     L.fapk_attn_fwd_noalloc.restype = i
-    L.fapk_attn_fwd_quantized_kv.argtypes = [PP] + [vp] * 11 + [sz, vp]
+    L.fapk_attn_fwd_quantized_kv.argtypes = [PP] + [vp] * 12 + [sz, vp]
     L.fapk_attn_fwd_quantized_kv.restype = i
     L.fapk_qkv_proj_mxfp8.argtypes = [PP, vp, i, vp, vp, vp, vp] + [vp] * 8 + [vp, sz, vp]
     L.fapk_qkv_proj_mxfp8.restype = i
+    L.fapk_attn_fwd_quantized_kv_nvfp4.argtypes = [PP] + [vp] * 10 + [sz, vp]
+    L.fapk_attn_fwd_quantized_kv_nvfp4.restype = i
+    L.fapk_qkv_proj_nvfp4.argtypes = [PP, vp, i, vp, vp, vp, vp] + [vp] * 6 + [vp, sz, vp]
+    L.fapk_qkv_proj_nvfp4.restype = i
     L.fapk_noalloc_status.argtypes = [vp]
     L.fapk_noalloc_status.restype = i
     L.fapk_quantize_mxfp8.argtypes = [vp, i, i, i, vp, vp, i, i, i, vp, vp, vp, vp, vp]
@@ -299,6 +303,49 @@ def qkv_proj_mxfp8(P: Problem, x: torch.Tensor, w: torch.Tensor, ws=None, stream
                                    *[_ptr(t) for t in f], _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "fapk_qkv_proj_mxfp8")
     return q, k, v, kf, vf
+
+
+def qkv_proj_nvfp4(P: Problem, x: torch.Tensor, w: torch.Tensor, ws=None, stream=None):
+    """fapk_qkv_proj_nvfp4 (mixed path): [Q | K | V] = x w^T with K's NVFP4
+    form and V's MX forms from the epilogue.  Returns (q, k, v, (k_codes,
+    k_scales), v_forms), ready for attn_fwd_quantized_kv_nvfp4."""
+    dev = x.device
+    T, Dm = x.shape
+    q = torch.empty((T, P.Hq, P.d), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((T, P.Hkv, P.d), dtype=torch.bfloat16, device=dev)
+    v = torch.empty((T, P.Hkv, P.d), dtype=torch.bfloat16, device=dev)
+    kc = torch.empty((T, P.Hkv, P.d // 2), dtype=torch.uint8, device=dev)
+    ks = torch.empty((T, P.Hkv, P.d // 16), dtype=torch.uint8, device=dev)
+    vf = {"val_tb": torch.empty((T, P.Hkv, P.d), dtype=torch.uint8, device=dev),
+          "scale_tb": torch.full((tb_slots(T, P.n_docs), P.Hkv, P.d // 32), 0xFF, dtype=torch.uint8, device=dev),
+          "val_pt": torch.empty((T, P.Hkv, P.d), dtype=torch.uint8, device=dev),
+          "scale_pt": torch.empty((T, P.Hkv, P.d // 32), dtype=torch.uint8, device=dev)}
+    if ws is None:
+        ws = workspace(P, FWD, dev)
+    f = [vf[n] for n in ("val_tb", "scale_tb", "val_pt", "scale_pt")]
+    rc = lib().fapk_qkv_proj_nvfp4(ctypes.byref(P), _ptr(x), Dm, _ptr(w), _ptr(q), _ptr(k), _ptr(v), _ptr(kc),
+                                   _ptr(ks), *[_ptr(t) for t in f], _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "fapk_qkv_proj_nvfp4")
+    return q, k, v, (kc, ks), vf
+
+
+def attn_fwd_quantized_kv_nvfp4(P: Problem, q, k_nv, v_forms: dict, o=None, lse=None, ws=None, stream=None):
+    """fapk_attn_fwd_quantized_kv_nvfp4 (mixed path): the forward over K in
+    NVFP4 (k_nv = (codes, scales) as quantize_nvfp4 returns them) and V in
+    both MX forms.  Returns (o, lse)."""
+    dev = q.device
+    if o is None:
+        o = torch.empty((P.T, P.Hq, P.d), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((P.Hq, P.T), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(P, FWD, dev)
+    f = [v_forms[n] for n in ("val_tb", "scale_tb", "val_pt", "scale_pt")]
+    rc = lib().fapk_attn_fwd_quantized_kv_nvfp4(ctypes.byref(P), _ptr(q), _ptr(k_nv[0]), _ptr(k_nv[1]),
+                                                *[_ptr(t) for t in f], _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                                                _stream(stream))
+    _check(rc, "fapk_attn_fwd_quantized_kv_nvfp4")
+    return o, lse
 
 
 def attn_bwd(P: Problem, q, k, v, o, lse, dout, ctx=None, dq=None, dk=None, dv=None, ws=None,

@@ -289,6 +289,29 @@ FAPK_API int fapk_qkv_proj_mxfp8(const fapk_problem_t* prob, const void* x, int 
                                  uint8_t* v_scale_tb, uint8_t* v_val_pt, uint8_t* v_scale_pt, void* ws,
                                  size_t ws_bytes, void* stream);
 
+/* The mixed NVFP4/FP8 path's counterparts of the two calls above (prob->prec
+ * = FAPK_NVFP4_MIXED, d = 128; otherwise FAPK_ERR_UNSUPPORTED).
+ *  fapk_qkv_proj_nvfp4: the same projection, with K's NVFP4 form in place of
+ *    its MX forms: k_codes [T][Hkv][64] (16-byte aligned) and k_scales
+ *    [T][Hkv][8] (2-byte aligned), quantised from the bf16 K with decode
+ *    scale prob->nv_scale_k exactly as fapk_quantize_nvfp4 would; V's MX
+ *    forms as above.
+ *  fapk_attn_fwd_quantized_kv_nvfp4: the mixed path's forward over K in
+ *    NVFP4 (k_codes, k_scales as fapk_quantize_nvfp4 or the projection write
+ *    them; 16- and 8-byte aligned) and V in both MX forms; Q is quantised on
+ *    load as in fapk_attn_fwd.  No quantisation launch and no saved state;
+ *    the output is bit-identical to fapk_attn_fwd's on the same inputs.
+ * Ownership, workspace, stream and errors as for the MXFP8 calls. */
+FAPK_API int fapk_qkv_proj_nvfp4(const fapk_problem_t* prob, const void* x, int d_model, const void* w,
+                                 void* q, void* k, void* v, uint8_t* k_codes, uint8_t* k_scales,
+                                 uint8_t* v_val_tb, uint8_t* v_scale_tb, uint8_t* v_val_pt,
+                                 uint8_t* v_scale_pt, void* ws, size_t ws_bytes, void* stream);
+FAPK_API int fapk_attn_fwd_quantized_kv_nvfp4(const fapk_problem_t* prob, const void* q,
+                                              const uint8_t* k_codes, const uint8_t* k_scales,
+                                              const uint8_t* v_val_tb, const uint8_t* v_scale_tb,
+                                              const uint8_t* v_val_pt, const uint8_t* v_scale_pt, void* o,
+                                              float* lse, void* ws, size_t ws_bytes, void* stream);
+
 /* Forward that allocates nothing.  The pages have no counterpart: this entry
  * point exists for callers that cannot obtain device memory where they run the
  * forward -- a plugin handed its buffers by a host framework that must not

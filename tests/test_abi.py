@@ -154,6 +154,22 @@ def test_nvfp4_mixed_validation(L):
     assert q(264, 64, 2, 128, ctypes.c_float(1.0), 256, 256, None) == fapk.ERR_INVALID_ARG  # x alignment
     assert q(256, 64, 2, 128, ctypes.c_float(1.0), 260, 256, None) == fapk.ERR_INVALID_ARG  # codes alignment
     assert q(256, 0, 2, 128, ctypes.c_float(1.0), None, None, None) == fapk.OK
+    # the mixed path's quantised-KV forward and QKV projection
+    f = L.fapk_attn_fwd_quantized_kv_nvfp4
+    ptrs = [256] * 9
+    assert f(ctypes.byref(_problem(prec=fapk.MXFP8)), *ptrs, 256, 1 << 30, None) == fapk.ERR_UNSUPPORTED
+    assert f(ctypes.byref(_problem(d=64, **nv)), *ptrs, 256, 1 << 30, None) == fapk.ERR_UNSUPPORTED
+    bad = list(ptrs)
+    bad[2] = 260  # K's scales not 8-byte aligned
+    assert f(ctypes.byref(_problem(**nv)), *bad, 256, 1 << 30, None) == fapk.ERR_INVALID_ARG
+    assert f(ctypes.byref(_problem(**nv)), *ptrs, 256, 16, None) == fapk.ERR_WORKSPACE_TOO_SMALL
+    g = L.fapk_qkv_proj_nvfp4
+    args = [256, 4096, 256, 256, 256, 256, 256, 256, 256, 256, 256, 256, 256]
+    assert g(ctypes.byref(_problem(prec=fapk.MXFP8)), *args, 1 << 30, None) == fapk.ERR_UNSUPPORTED
+    bad = list(args)
+    bad[1] = 4095  # d_model not a multiple of 8
+    assert g(ctypes.byref(_problem(**nv)), *bad, 1 << 30, None) == fapk.ERR_INVALID_ARG
+    assert g(ctypes.byref(_problem(**nv)), *args, 16, None) == fapk.ERR_WORKSPACE_TOO_SMALL
 
 
 @pytest.mark.parametrize("prec,rows", [(fapk.BF16, 256), (fapk.MXFP8, 128)])

@@ -315,3 +315,20 @@ def test_bf16_gradient_output():
     for a, b in zip(*outs):
         assert b.dtype == torch.bfloat16
         assert torch.equal(a.to(torch.bfloat16), b)
+
+
+def test_forward_from_quantised_kv_matches_the_mixed_forward():
+    """fapk_attn_fwd_quantized_kv_nvfp4 over K quantised by fapk_quantize_nvfp4
+    and V by fapk_quantize_mxfp8 (as a cache would hold them) gives O and LSE
+    bit-identical to the mixed forward, twice over the same forms."""
+    dev = require_gpu()
+    w = W.custom([1, 129, 300, 700, 64], Hq=4, Hkv=2, d=128, seed=99)
+    (q, k, v, _), (qd, kd, vd, _) = to_dev(w, dev, with_dout=False)
+    P, seq = _problem(w, dev, 0.7, 1.3)
+    kn = fapk.quantize_nvfp4(kd, 1.3)
+    vf = fapk.quantize_mxfp8(vd, seq)
+    o_ref, l_ref, _ = fapk.attn_fwd(P, qd, kd, vd)
+    for _ in range(2):
+        o, lse = fapk.attn_fwd_quantized_kv_nvfp4(P, qd, kn, vf)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)

@@ -57,3 +57,29 @@ def test_projection_and_forms(lengths, d_model):
     o2, l2, _ = fapk.attn_fwd(P, q, k, v)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("gk", [1.0, 0.4])
+def test_projection_nvfp4_mixed(gk):
+    """fapk_qkv_proj_nvfp4: the same projection with K's NVFP4 form (decode
+    scale gk) in place of its MX forms, bit-exact against the oracle's NVFP4
+    quantiser of the kernel's bf16 K; V's MX forms as above; the mixed path's
+    forward over those forms bit-identical to its forward over the bf16 K, V."""
+    dev = require_gpu()
+    Hq, Hkv = 4, 2
+    lengths, d_model = [1, 31, 33, 127, 129, 300, 700], 384
+    x, w, cu = _inputs(lengths, d_model, Hq, Hkv, seed=91)
+    seq = fapk.Seqlens(cu, dev)
+    P = fapk.make_problem(seq, Hq, Hkv, 128, 128 ** -0.5, prec=fapk.NVFP4_MIXED, nv_scale_q=0.8, nv_scale_k=gk)
+    ws = fapk.workspace(P, fapk.FWD, dev)
+    q, k, v, (kc, ks), vf = fapk.qkv_proj_nvfp4(P, x.to(dev), w.to(dev), ws=ws)
+    assert fapk.status(ws) == fapk.OK
+    ec, es = oracle.quantize_nvfp4(f64(k), gk)
+    assert np.array_equal(kc.cpu().numpy(), ec) and np.array_equal(ks.cpu().numpy(), es)
+    ref = oracle.quantize_mxfp8(f64(v), cu)
+    for key in ("val_tb", "val_pt", "scale_pt"):
+        assert np.array_equal(vf[key].cpu().numpy(), ref[key]), key
+    o1, l1 = fapk.attn_fwd_quantized_kv_nvfp4(P, q, (kc, ks), vf)
+    o2, l2, _ = fapk.attn_fwd(P, q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
