@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         const int stg = st_it % kStages;
         const uint32_t use = st_it / kStages;
         // scale words first, so that their global reads overlap the wait
-        uint4 wk, wk2;
+        uint4 wk, wk2 = make_uint4(0u, 0u, 0u, 0u);
         if constexpr (kNv) {
           // the NVFP4 scale words of the tile's keys (scores)
           const int k0 = s + 128 * v;
