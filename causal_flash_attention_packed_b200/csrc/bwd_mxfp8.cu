@@ -273,20 +273,26 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
       if (w < 0 || w >= n_units) break;
       int doc, s, e, h, g, q0, n;
       decode(un, doc, s, e, h, g, q0, n);
-      if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 71)) break;
+      // the scale words' global reads first, so that their latency overlaps the wait
+      uint4 w_0, w_2;
       if constexpr (kNv) {
         const uint2 w0 = nv_scale_words(p.q_nvs, q0 + lane, p.T, p.Hq, h);
         const uint2 w1 = nv_scale_words(p.q_nvs, q0 + lane + 32, p.T, p.Hq, h);
         const uint2 w2 = nv_scale_words(p.q_nvs, q0 + lane + 64, p.T, p.Hq, h);
         const uint2 w3 = nv_scale_words(p.q_nvs, q0 + lane + 96, p.T, p.Hq, h);
-        reinterpret_cast<uint4*>(sfb(0))[lane] = make_uint4(w0.x, w1.x, w2.x, w3.x);
-        reinterpret_cast<uint4*>(sfb(2))[lane] = make_uint4(w0.y, w1.y, w2.y, w3.y);
+        w_0 = make_uint4(w0.x, w1.x, w2.x, w3.x);
+        w_2 = make_uint4(w0.y, w1.y, w2.y, w3.y);
       } else {
-        reinterpret_cast<uint4*>(sfb(0))[lane] = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
-        reinterpret_cast<uint4*>(sfb(2))[lane] = pt_rows(p.k_spt, q0, lane, p.T, p.Hkv, g);
+        w_0 = pt_rows(p.q_spt, q0, lane, p.T, p.Hq, h);
+        w_2 = pt_rows(p.k_spt, q0, lane, p.T, p.Hkv, g);
       }
-      reinterpret_cast<uint4*>(sfb(1))[lane] = pt_rows(p.do_spt, q0, lane, p.T, p.Hq, h);
-      reinterpret_cast<uint4*>(sfb(3))[lane] = pt_rows(p.v_spt, q0, lane, p.T, p.Hkv, g);
+      const uint4 w_1 = pt_rows(p.do_spt, q0, lane, p.T, p.Hq, h);
+      const uint4 w_3 = pt_rows(p.v_spt, q0, lane, p.T, p.Hkv, g);
+      if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 71)) break;
+      reinterpret_cast<uint4*>(sfb(0))[lane] = w_0;
+      reinterpret_cast<uint4*>(sfb(1))[lane] = w_1;
+      reinterpret_cast<uint4*>(sfb(2))[lane] = w_2;
+      reinterpret_cast<uint4*>(sfb(3))[lane] = w_3;
       fence_proxy_async_smem();
       if (lane == 0) {
         mbar_arrive_expect_tx(q_full, kNv ? kNvTile + 2 * kCode : 4 * kCode);

@@ -356,8 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kv = 0; kv < 2; ++kv, ++kv_it) {
           const int slot = kv_it % kSlots;
           const uint32_t use = kv_it / kSlots;
-          if (use > 0 && !warp_wait(kv_empty + slot, (use - 1) & 1, wd, 52)) { ok = false; break; }
-          uint4 wsf;
+          // the scale words' global reads first, so that their latency overlaps the wait
+          uint4 wsf, wsf2 = make_uint4(0u, 0u, 0u, 0u);
           if (kNv && kv == 0) {
             // K rows = keys: the NVFP4 scale words (channels 0..63, 64..127) of each key
             const int k0 = it.s + 128 * j;
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint2 w2 = nv_scale_words(p.k_nvs, k0 + lane + 64, p.T, p.Hkv, it.g);
             const uint2 w3 = nv_scale_words(p.k_nvs, k0 + lane + 96, p.T, p.Hkv, it.g);
             wsf = make_uint4(w0.x, w1.x, w2.x, w3.x);
-            reinterpret_cast<uint4*>(sfRing2 + slot * kSfBlk)[lane] = make_uint4(w0.y, w1.y, w2.y, w3.y);
+            wsf2 = make_uint4(w0.y, w1.y, w2.y, w3.y);
           } else if (kv == 0) {
             // K rows = keys: the scale word of the key's token block
             wsf.x = tb_word(p.k_stb, it.s, it.e, it.doc, 4 * j + 0, p.Hkv, it.g);
@@ -386,6 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             wsf = make_uint4(wv[0], wv[1], wv[2], wv[3]);
           }
+          if (use > 0 && !warp_wait(kv_empty + slot, (use - 1) & 1, wd, 52)) { ok = false; break; }
+          if (kNv && kv == 0) reinterpret_cast<uint4*>(sfRing2 + slot * kSfBlk)[lane] = wsf2;
           reinterpret_cast<uint4*>(sfRing + slot * kSfBlk)[lane] = wsf;
           fence_proxy_async_smem();
           if (lane == 0) {
@@ -401,8 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // item has read the previous ones; after the item's last K and V
           // (the per-token scores come last), so that the item's streamed
           // tiles never wait for the previous item to finish
-          if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 51)) { ok = false; break; }
-          uint4 wk;
+          uint4 wk, wk2 = make_uint4(0u, 0u, 0u, 0u);
           if constexpr (kNv) {
             // the diagonal key tile's NVFP4 codes and scales (the same scores
             // as the ring's copy of that tile)
@@ -411,13 +412,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint2 w2 = nv_scale_words(p.k_nvs, it.q0 + lane + 64, p.T, p.Hkv, it.g);
             const uint2 w3 = nv_scale_words(p.k_nvs, it.q0 + lane + 96, p.T, p.Hkv, it.g);
             wk = make_uint4(w0.x, w1.x, w2.x, w3.x);
-            reinterpret_cast<uint4*>(sfKpt2)[lane] = make_uint4(w0.y, w1.y, w2.y, w3.y);
+            wk2 = make_uint4(w0.y, w1.y, w2.y, w3.y);
           } else {
             wk.x = pt_word(p.k_spt, it.q0 + lane, p.T, p.Hkv, it.g);
             wk.y = pt_word(p.k_spt, it.q0 + lane + 32, p.T, p.Hkv, it.g);
             wk.z = pt_word(p.k_spt, it.q0 + lane + 64, p.T, p.Hkv, it.g);
             wk.w = pt_word(p.k_spt, it.q0 + lane + 96, p.T, p.Hkv, it.g);
           }
+          // the scale words were read above, so that their latency overlaps this wait
+          if (unit_i > 0 && !warp_wait(q_empty, (unit_i - 1) & 1, wd, 51)) { ok = false; break; }
+          if (kNv) reinterpret_cast<uint4*>(sfKpt2)[lane] = wk2;
           reinterpret_cast<uint4*>(sfKpt)[lane] = wk;
           fence_proxy_async_smem();
           if (lane == 0) {
