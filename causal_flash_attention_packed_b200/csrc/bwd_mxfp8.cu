@@ -625,8 +625,8 @@ constexpr int oBars = oSf + kNumSf * kSfBlk;
 // operand buffers, in the order the MMAs release them
 constexpr int kQpt = 0, kDOpt = 1, kDOtb = 2, kQtb = 3;
 constexpr int bKvFull = 0, bKvEmpty = 1, bOpFull = 2, bOpEmpty = 6, bAuxFull = 10, bAuxEmpty = 12, bSFull = 14,
-              bSFree = 15, bPFull = 16, bPEmpty = 17, bDsFull = 18, bDsEmpty = 19, bAccFull = 20, bAccFree = 21,
-              bFin = 22, bRing = 23, kNumBars = bRing + 2 * kUnitRing;  // the unit ring's full[], empty[] from bRing
+              bSFree = 15, bPFull = 16, bDsFull = 17, bAccFull = 18, bAccFree = 19, bFin = 20, bRing = 21,
+              kNumBars = bRing + 2 * kUnitRing;  // the unit ring's full[], empty[] from bRing
 constexpr int kSmem = oBars + kNumBars * 8 + 16 + kUnitRingBytes + 1024;
 static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may use");
 // TMEM: one 128-column region that holds S^T and dP^T in turn (each read out
@@ -659,9 +659,7 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   uint64_t* s_full = bars + bSFull;
   uint64_t* s_free = bars + bSFree;
   uint64_t* p_full = bars + bPFull;
-  uint64_t* p_empty = bars + bPEmpty;
   uint64_t* ds_full = bars + bDsFull;
-  uint64_t* ds_empty = bars + bDsEmpty;
   uint64_t* acc_full = bars + bAccFull;
   uint64_t* acc_free = bars + bAccFree;
   uint64_t* fin = bars + bFin;
@@ -685,9 +683,7 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
     mbar_init(s_full, 1);
     mbar_init(s_free, kComputeWarps);
     mbar_init(p_full, kComputeWarps);
-    mbar_init(p_empty, 1);
     mbar_init(ds_full, kComputeWarps);
-    mbar_init(ds_empty, 1);
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kComputeWarps);
     mbar_init(fin, 1);
@@ -927,7 +923,6 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           tmem_cp_sf(tmem + tSfP, aSf + 8 * kSfBlk);
           tmem_cp_sf(tmem + tSfDOtb, aSf + 6 * kSfBlk);
           mx_kk(tDV, aP, aDOtb, tSfP, tSfDOtb, true, r > 0);
-          tc_commit(p_empty);
           tc_commit(op_empty + kDOtb);
           // the next tile's S^T goes ahead of dK, so that it is ready when the
           // compute warps finish dS~ of this tile
@@ -942,7 +937,6 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           tmem_cp_sf(tmem + tSfDS, aSf + 9 * kSfBlk);
           tmem_cp_sf(tmem + tSfQtb, aSf + 7 * kSfBlk);
           mx_kk(tDK, aDS, aQtb, tSfDS, tSfQtb, true, r > 0);
-          tc_commit(ds_empty);
           tc_commit(op_empty + kQtb);
         }
         if (!ok) break;
@@ -1030,7 +1024,10 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
               }
             }
           }
-          if (t > 0 && !warp_wait(p_empty, (t - 1) & 1, wd, 98)) { ok = false; break; }
+          // P~T's buffer and scale block are free: this thread has seen S^T of
+          // this tile complete, and the MMA thread issued that S^T after the
+          // previous tile's dV MMA and scale copy (a commit tracks every earlier
+          // tcgen05 operation of its thread)
           {
             uint32_t cw[8];
             const uint32_t sb = mx_quant32_pairs<true>(pr2, p.rule, cw);
@@ -1042,7 +1039,8 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           // ---- dP^T -> dS~T into shared memory
           if (!take(!own && !past, r)) { ok = false; break; }
           if (diag && !take(own, r)) { ok = false; break; }
-          if (t > 0 && !warp_wait(ds_empty, (t - 1) & 1, wd, 99)) { ok = false; break; }
+          // dS~T's buffer is free likewise: dP^T of this tile was issued after
+          // the previous tile's dK MMA
           {
             // dS = P (dP - D), packed, in place of P (P is not needed after this)
             if (!past) {
