@@ -369,10 +369,16 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
         // V and the stage's V end here, K^tb is read by dQ too
         // (mixed path: S from the NVFP4 Q and the stage's NVFP4 K, whose
         // second scale blocks sit at tSfKpt and tSfK2)
-        auto score = [&](bool dp, uint32_t a, uint32_t b, uint32_t sfa, uint32_t sfbc) {
+        // (a stage's K or V scale block is copied into TMEM only after the
+        // region's previous MMA, which read the same scale columns, has been
+        // read out, i.e. has completed; cp_src 0: no copy)
+        auto score = [&](bool dp, uint32_t a, uint32_t b, uint32_t sfa, uint32_t sfbc, uint32_t cp_src = 0,
+                         uint32_t cp_src2 = 0) {
           uint32_t& uses = dp ? dp_uses : s_uses;
           if (uses > 0 && !mbar_wait(dp ? dp_free : s_free, (uses - 1) & 1, wd, dp ? 74 : 73)) return false;
           tc_fence_after();
+          if (cp_src) tmem_cp_sf(tmem + sfbc, cp_src);
+          if (cp_src2) tmem_cp_sf(tmem + tSfK2, cp_src2);
           if (kNv && !dp) {
             const uint64_t da = sdesc_sw64(a), db = sdesc_sw64(b);
             constexpr uint32_t idn = idesc_nvf4(128, 128);
@@ -402,11 +408,9 @@ __global__ void __launch_bounds__(dqk::kThreads, 1)
             const int stg = kt % kStages;
             if (!mbar_wait(st_full + stg, (kt / kStages) & 1, wd, 75)) { ok = false; break; }
             const uint32_t ak = aRing + stg * 2 * kCode, av = ak + kCode;
-            tmem_cp_sf(tmem + tSfK, aSf + (5 + 3 * stg) * kSfBlk);
-            if (kNv) tmem_cp_sf(tmem + tSfK2, aSf + (5 + 3 * kStages + stg) * kSfBlk);
-            if (!score(false, aQ, kNv ? aKpt + stg * kNvTile : ak, tSfQ, tSfK)) { ok = false; break; }
-            tmem_cp_sf(tmem + tSfV, aSf + (6 + 3 * stg) * kSfBlk);
-            if (!score(true, aDO, av, tSfDO, tSfV)) { ok = false; break; }
+            if (!score(false, aQ, kNv ? aKpt + stg * kNvTile : ak, tSfQ, tSfK, aSf + (5 + 3 * stg) * kSfBlk,
+                       kNv ? aSf + (5 + 3 * kStages + stg) * kSfBlk : 0u)) { ok = false; break; }
+            if (!score(true, aDO, av, tSfDO, tSfV, aSf + (6 + 3 * stg) * kSfBlk)) { ok = false; break; }
           }
           if (!ok) break;
           // the diagonal tile again with the per-token K and V (mixed path:
