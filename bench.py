@@ -228,9 +228,10 @@ KERNEL_FLOPS = {"fwd_kernel": 4.0, "dkdv_kernel": 8.0, "dq_kernel": 6.0}
 # These must be taken again whenever a kernel changes.
 MEASURED_TRAFFIC = {
     4: {"bf16": {"fwd_kernel": 1.325e9, "dkdv_kernel": 2.131e9, "dq_kernel": 1.610e9},
-        "mxfp8": {"fwd_kernel": 1.594e9, "dkdv_kernel": 2.188e9, "dq_kernel": 1.354e9,
+        # (the MXFP8 dK/dV kernel changed after its last capture: not measured)
+        "mxfp8": {"fwd_kernel": 1.594e9, "dkdv_kernel": None, "dq_kernel": 1.354e9,
                   "quantize_kv": 1.034e9, "delta_quantize_do": 1.052e9},
-        "nvfp4": {"fwd_kernel": 1.324e9, "dkdv_kernel": 1.909e9, "dq_kernel": 1.368e9,
+        "nvfp4": {"fwd_kernel": 1.324e9, "dkdv_kernel": None, "dq_kernel": 1.368e9,
                   "quantize_kv": 1.111e9, "delta_quantize_do": 1.052e9}},
 }
 

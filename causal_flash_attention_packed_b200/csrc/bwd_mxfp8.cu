@@ -628,6 +628,7 @@ constexpr int kNvTile = 128 * 64;
 constexpr int oBars = oSf + kNumSf * kSfBlk;
 // operand buffers, in the order the MMAs release them
 constexpr int kQpt = 0, kDOpt = 1, kDOtb = 2, kQtb = 3;
+// (bAuxFull, bDsFull: unused slots)
 constexpr int bKvFull = 0, bKvEmpty = 1, bOpFull = 2, bOpEmpty = 6, bAuxFull = 10, bAuxEmpty = 12, bSFull = 14,
               bSFree = 15, bPFull = 16, bDsFull = 17, bAccFull = 18, bAccFree = 19, bFin = 20, bRing = 21,
               kNumBars = bRing + 2 * kUnitRing;  // the unit ring's full[], empty[] from bRing
@@ -658,7 +659,6 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
   uint64_t* kv_empty = bars + bKvEmpty;
   uint64_t* op_full = bars + bOpFull;
   uint64_t* op_empty = bars + bOpEmpty;
-  uint64_t* aux_full = bars + bAuxFull;
   uint64_t* aux_empty = bars + bAuxEmpty;
   uint64_t* s_full = bars + bSFull;
   uint64_t* s_free = bars + bSFree;
@@ -681,7 +681,6 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
       mbar_init(op_empty + i, 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(aux_full + i, 32);
       mbar_init(aux_empty + i, kComputeWarps);
     }
     mbar_init(s_full, 1);
@@ -803,7 +802,10 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           float* lse2 = reinterpret_cast<float*>(smem + oAux + ab * 1024);
           reinterpret_cast<float4*>(lse2)[lane] = make_float4(l4[0], l4[1], l4[2], l4[3]);
           reinterpret_cast<float4*>(lse2 + 128)[lane] = make_float4(d4[0], d4[1], d4[2], d4[3]);
-          mbar_arrive(aux_full + ab);
+          // no barrier of their own: each lane's arrival on Q^pt's barrier
+          // below releases these stores, the MMA thread waits on that barrier
+          // before it issues S^T of this tile, and the compute warps read them
+          // only after they have seen that S^T complete
           if (!load_op(kQpt, t, &tm_qpt, h, q0, sq, 83, kNv ? &sq2 : nullptr)) { ok = false; break; }
           if (!load_op(kDOpt, t, &tm_dopt, h, q0, sdo, 84)) { ok = false; break; }
           // the query-side operands of dV and dK (token-block form)
@@ -992,8 +994,8 @@ __global__ void __launch_bounds__(kvk::kThreads, 1)
           const bool own = diag && wg == quarter;
           const bool past = diag && wg < quarter;
           const int ab = t & 1;
-          if (!warp_wait(aux_full + ab, (t >> 1) & 1, wd, 97)) { ok = false; break; }
-          // -lse log2 e and D of this block's 32 queries (identical across the warp)
+          // -lse log2 e and D of this block's 32 queries (identical across the
+          // warp), read after S^T of this tile has been seen complete
           const float4* nl4 = reinterpret_cast<const float4*>(smem + oAux + ab * 1024) + 8 * wg;
           const float4* dl4 = nl4 + 32;
           uint32_t r[32];
