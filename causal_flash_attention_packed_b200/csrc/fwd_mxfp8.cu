@@ -94,6 +94,10 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory exceeds the 227 KB a CTA 
 constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256;
 constexpr uint32_t kSfQ = 384, kSfK = 388, kSfKpt = 392, kSfP = 396, kSfV = 400;
 constexpr uint32_t kSfQ2 = 404, kSfK2 = 408, kSfKpt2 = 412;  // mixed path: channels 64..127
+// the K scale columns of odd tiles: the copy for S(j + 2) is issued before
+// S(j + 1), which reads the other set, has been seen complete, so it must not
+// overwrite that set (it overwrites S(j)'s, which the softmax warps have read)
+constexpr uint32_t kSfK1 = 416, kSfK21 = 420;
 constexpr int kNvTile = 128 * 64;  // 128 rows x 128 E2M1 codes
 
 struct Params {
@@ -475,9 +479,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_s_tile = [&](int j, uint32_t col) {
         const int ks = kslot_of(j);
-        tmem_cp_sf(tmem + kSfK, asf + (3 + ks) * kSfBlk);
-        if constexpr (kNv) tmem_cp_sf(tmem + kSfK2, smem_u32(sfRing2) + ks * kSfBlk);
-        issue_s(col, aring + ks * kCodeTile, kSfK, kSfK2);
+        const uint32_t sk = (j & 1) ? kSfK1 : kSfK, sk2 = (j & 1) ? kSfK21 : kSfK2;
+        tmem_cp_sf(tmem + sk, asf + (3 + ks) * kSfBlk);
+        if constexpr (kNv) tmem_cp_sf(tmem + sk2, smem_u32(sfRing2) + ks * kSfBlk);
+        issue_s(col, aring + ks * kCodeTile, sk, sk2);
       };
       for (uint32_t uk = 0; ok; ++uk, ++unit_i) {
         const UnitInfo un = unit_take(ring, uk, wd);
