@@ -181,6 +181,8 @@ static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may u
 constexpr uint32_t tS = 0, tDP = 128, tDQ = 256;
 constexpr uint32_t tSfQ = 384, tSfDO = 388, tSfK = 392, tSfV = 396, tSfKpt = 400, tSfVpt = 404, tSfDS = 408,
                    tSfKdq = 412, tSfK2 = 416;  // mixed path: tSfKpt holds Q's second block, tSfK2 K's
+constexpr uint32_t kSfCols[] = {tSfQ, tSfDO, tSfK, tSfV, tSfKpt, tSfVpt, tSfDS, tSfKdq, tSfK2};
+static_assert(sf_cols_ok(kSfCols, tDQ + 128), "dQ kernel TMEM scale columns overlap");
 }  // namespace dqk
 
 // kNv: tm_qpt maps Q's NVFP4 codes, tm_knv K's (tm_kpt is not read)
@@ -639,6 +641,8 @@ static_assert(kSmem <= 227 * 1024, "shared memory exceeds the 227 KB a CTA may u
 constexpr uint32_t tSD = 0, tDV = 128, tDK = 256;
 constexpr uint32_t tSfKtb = 384, tSfKpt = 388, tSfVtb = 392, tSfVpt = 396, tSfQpt = 400, tSfDOpt = 404, tSfP = 408,
                    tSfDS = 412, tSfDOtb = 416, tSfQtb = 420, tSfQ2 = 424;
+constexpr uint32_t kSfCols[] = {tSfKtb, tSfKpt, tSfVtb, tSfVpt, tSfQpt, tSfDOpt, tSfP, tSfDS, tSfDOtb, tSfQtb, tSfQ2};
+static_assert(sf_cols_ok(kSfCols, tDK + 128), "dK/dV kernel TMEM scale columns overlap");
 }  // namespace kvk
 
 // kNv: tm_ktb and tm_kpt map K's NVFP4 codes (only tm_ktb is read), tm_qpt Q's

@@ -98,6 +98,8 @@ constexpr uint32_t kSfQ2 = 404, kSfK2 = 408, kSfKpt2 = 412;  // mixed path: chan
 // S(j + 1), which reads the other set, has been seen complete, so it must not
 // overwrite that set (it overwrites S(j)'s, which the softmax warps have read)
 constexpr uint32_t kSfK1 = 416, kSfK21 = 420;
+constexpr uint32_t kSfCols[] = {kSfQ, kSfK, kSfKpt, kSfP, kSfV, kSfQ2, kSfK2, kSfKpt2, kSfK1, kSfK21};
+static_assert(sf_cols_ok(kSfCols, kO + 128), "forward TMEM scale columns overlap");
 constexpr int kNvTile = 128 * 64;  // 128 rows x 128 E2M1 codes
 
 struct Params {

@@ -177,6 +177,19 @@ __device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// A scale block copied by tmem_cp_sf takes 4 TMEM columns (128 bits per lane).
+// True when the blocks starting at cols[] are pairwise disjoint, start at or
+// after first_free (the end of the accumulators) and end within 512 columns.
+template <int N>
+constexpr bool sf_cols_ok(const uint32_t (&cols)[N], uint32_t first_free) {
+  for (int i = 0; i < N; ++i) {
+    if (cols[i] < first_free || cols[i] + 4 > 512) return false;
+    for (int j = 0; j < i; ++j)
+      if (cols[i] < cols[j] + 4 && cols[j] < cols[i] + 4) return false;
+  }
+  return true;
+}
+
 // Copy a 512-byte scale-factor block from shared memory into 4 TMEM columns,
 // replicated into all four 32-lane quarters.  The block holds the 4 scale
 // bytes (one per 32-element K block) of 128 rows: row r = r0 + 32 r1 at byte
